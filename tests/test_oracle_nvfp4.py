@@ -1,0 +1,142 @@
+"""Pins of the oracle's NVFP4 quantiser: exhaustive E2M1 codes and ties, E4M3
+against torch's float8_e4m3fn conversion (a library routine), saturation,
+round trips and the per-element error bound."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import nvfp4 as Q
+
+
+def test_format_fixture_matches_oracle(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "nvfp4_format.json")))
+    assert g["micro_block"] == Q.BLOCK == 16
+    assert g["element_format"] == "E2M1" and g["block_scale_format"] == "E4M3"
+    assert g["default_rounding"] == "RTNE"
+
+
+def test_e2m1_all_codes_round_trip():
+    # E2M1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; exponent 0 subnormal
+    expected = []
+    for code in range(16):
+        s, e, m = code >> 3, (code >> 1) & 3, code & 1
+        mag = (m * 0.5) if e == 0 else (1 + m * 0.5) * 2.0 ** (e - 1)
+        expected.append(-mag if s else mag)
+    vals = Q.e2m1_decode(np.arange(16))
+    assert np.array_equal(vals, np.array(expected))
+    assert np.array_equal(np.abs(vals[:8]), [0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    assert np.array_equal(Q.e2m1_rtne(vals), np.arange(16, dtype=np.uint8))
+
+
+def test_e2m1_ties_to_even_and_saturation():
+    ties = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for x, want in ties.items():
+        assert Q.e2m1_decode(Q.e2m1_rtne(np.array([x])))[0] == want
+        assert Q.e2m1_decode(Q.e2m1_rtne(np.array([-x])))[0] == -want
+    off = {0.2: 0.0, 0.3: 0.5, 0.8: 1.0, 1.3: 1.5, 2.6: 3.0, 3.4: 3.0, 4.9: 4.0,
+           5.1: 6.0, 6.0: 6.0, 7.0: 6.0, 1e30: 6.0}
+    for x, want in off.items():
+        assert Q.e2m1_decode(Q.e2m1_rtne(np.array([x])))[0] == want
+
+
+def test_e2m1_is_nearest_grid_point_brute_force():
+    rng = np.random.default_rng(0)
+    x = rng.uniform(-7, 7, 20000)
+    grid = np.concatenate([-Q.E2M1_GRID[::-1], Q.E2M1_GRID])
+    got = Q.e2m1_decode(Q.e2m1_rtne(x))
+    dist = np.abs(np.clip(x, -6, 6)[:, None] - grid[None, :]).min(axis=1)
+    assert np.allclose(np.abs(np.clip(x, -6, 6) - got), dist, atol=0)
+
+
+def test_e4m3_all_codes_match_torch():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    ours = Q.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(ours, ref)
+    assert Q.e4m3_decode(np.array([0x7E]))[0] == 448.0
+    # every finite code encodes back to itself (except -0 -> sign kept)
+    assert np.array_equal(Q.e4m3_rtne(ours), codes)
+
+
+def test_e4m3_rounding_matches_torch_in_range():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.uniform(0, 448, 20000), np.exp(rng.uniform(-14, 6, 20000)),
+        # exact midpoints between neighbouring codes
+        0.5 * (Q.e4m3_decode(np.arange(1, 126)) + Q.e4m3_decode(np.arange(2, 127))),
+    ]).astype(np.float32)
+    ours = Q.e4m3_decode(Q.e4m3_rtne(x))
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_saturates():
+    assert np.array_equal(Q.e4m3_decode(Q.e4m3_rtne(np.array([449.0, 464.0, 500.0, 1e9]))),
+                          [448.0] * 4)
+
+
+def test_quantize_round_trip_of_grid_values():
+    # blocks whose elements are q * s * g with representable s come back exactly
+    rng = np.random.default_rng(2)
+    g = np.float32(0.25)
+    s_codes = rng.integers(0x20, 0x70, size=(4, 8))
+    s = Q.e4m3_decode(s_codes)
+    q = Q.e2m1_decode(rng.integers(0, 16, size=(4, 8, 16)))
+    q[..., 0] = 6.0                       # each block reaches the E2M1 max
+    X = (q * s[..., None] * g).reshape(4, 128)
+    out = Q.fake_quant(X, g)
+    assert np.array_equal(out, X)
+
+
+def test_quantize_error_bound_and_zero_blocks():
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((64, 256)).astype(np.float32) * 3
+    X[5, 16:32] = 0.0
+    g = Q.weight_global_scale(X)
+    codes, sc, sb = Q.quantize(X, g)
+    out = Q.fake_quant(X, g)
+    assert np.all(out[5, 16:32] == 0.0)
+    step = sb.astype(np.float64) * np.float64(g)       # per block
+    err = np.abs(out - X).reshape(64, 16, 16)
+    # nearest-point rounding: |err| <= half the widest E2M1 gap (1.0) * s*g
+    # plus the saturation excess of the block max (scale rounding)
+    amax = np.abs(X).reshape(64, 16, 16).max(axis=2)
+    sat_excess = np.maximum(amax - 6 * step, 0)
+    assert np.all(err <= (1.0 * step + sat_excess)[..., None] + 1e-12)
+    # with g = amax/2688 the largest block scale is 448 (E4M3 max)
+    assert sb.max() <= 448.0
+    assert abs(float(sb.max()) - 448.0) <= 16.0
+
+
+def test_weight_global_scale_closed_form():
+    W = np.array([[0.5, -2688.0], [1.0, 0.0]], dtype=np.float32)
+    assert Q.weight_global_scale(W) == np.float32(1.0)
+    W = np.zeros((3, 16), dtype=np.float32)
+    assert Q.weight_global_scale(W) == 0.0
+    codes, sc, sb = Q.quantize(W, 0.0)
+    assert np.all(codes == 0) and np.all(sb == 0)
+
+
+def test_fake_quant_layer_close_to_bf16_layer():
+    """The NVFP4 layer differs from the unquantised layer by a few percent of
+    the routed output (a sanity bound on the dequantised values)."""
+    from oracle import lmoe as O
+    rng = np.random.default_rng(4)
+    T, d, l, N, K, h, hs = 16, 64, 32, 8, 2, 48, 64
+    x = rng.standard_normal((T, d))
+    W = lambda *s: rng.standard_normal(s) * 0.1
+    W_r, W_dn, W1, W2 = W(N, d), W(l, d), W(N, h, l), W(N, l, h)
+    W_upl, W_s1, W_s2 = W(d, l), W(hs, d), W(d, hs)
+    su = 0.1 * np.sqrt(d)
+    sa = 0.1 * np.sqrt(l) * su
+    quant = {"g_u": 8 * su / 2688, "g_h": (8 * sa) ** 2 / 2688}
+    a = O.layer_forward(x, W_r, None, W_dn, lambda e: W1[e], lambda e: W2[e],
+                        W_upl, W_s1, W_s2, K)
+    b = O.layer_forward(x, W_r, None, W_dn, lambda e: W1[e], lambda e: W2[e],
+                        W_upl, W_s1, W_s2, K, quant=quant)
+    rel = np.sqrt(np.mean((a["r"] - b["r"]) ** 2)) / np.sqrt(np.mean(a["r"] ** 2))
+    assert 0.0 < rel < 0.25
+    assert np.array_equal(a["sh"], b["sh"])
