@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Throughput of the LatentMoE layer forward pass on B200 (tokens/s per layer)
+and its fraction of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl lmoe|reference]
+
+One step = one lmoe_forward of the workload's T tokens with weights resident
+in HBM.  Default workload: the Super-dims decode layer (T=256, d=4096, l=1024,
+N=512, K=22, h=2688, h_s=5376, uniform router).  Under torchrun each rank runs
+its own token batch (seed + rank) against replicated weights: no collective on
+the data path, weak scaling; the timed region is bracketed by barriers and the
+reported time is the max over ranks.
+
+--impl reference times the CPU float64 oracle (the only other implementation
+of the layer) on a bounded token sample of the same workload, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from lmoe_synth import CONFIGS, make_weights, make_x  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "LatentMoE layer tokens/s at 1 B200 (Super dims) and % of roofline"
+
+
+# ---------------------------------------------------------------------------
+# host-side helpers (covered by CPU tests)
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Token-batch seed of a rank: every rank draws its own batch."""
+    return base_seed * 1000 + 17 + rank
+
+
+def load_peaks(path: str = os.path.join(ROOT, "MEASURED_PEAKS.json")):
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_work(cfg, T: int, counts: np.ndarray):
+    """Algorithmic bytes and flops of one forward and of each contraction.
+
+    Bytes count the weights a forward must read (dense weights plus the W1/W2
+    of experts with at least one routed row), x and y, and for each kernel its
+    own operands and results; flops count real rows only (no tile padding).
+    """
+    d, l, N, K, h, hs = cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs
+    touched = int((counts > 0).sum())
+    R = T * K
+    wx = (N + l + hs) * d * 2
+    wy = d * (l + hs) * 2
+    wexp = touched * h * l * 2
+    per_kernel = {
+        "xgemm(router|W_dn|W_s1)": dict(bytes=wx + T * d * 2 + T * (N * 4 + l * 2 + hs * 2),
+                                        flops=2 * T * d * (N + l + hs)),
+        "grouped_gemm1(W1,sqrelu)": dict(bytes=wexp + R * l * 2 + R * h * 2, flops=2 * R * l * h),
+        "grouped_gemm2(W2,*w)": dict(bytes=wexp + R * h * 2 + R * l * 2 + R * 4,
+                                     flops=2 * R * h * l),
+        "ygemm([W_upl|W_s2])": dict(bytes=wy + T * (l + hs) * 2 + T * d * 2,
+                                    flops=2 * T * d * (l + hs)),
+    }
+    layer = dict(bytes=wx + wy + 2 * wexp + 2 * T * d * 2,
+                 flops=sum(v["flops"] for v in per_kernel.values()))
+    return layer, per_kernel
+
+
+def roofline_entry(name, kw, total_ms, launches, peaks, peak_kind, cfg, T):
+    """The roofline object of one kernel from its live CUDA-event times."""
+    avg_s = total_ms / 1e3 / max(launches, 1)
+    intensity = kw["flops"] / kw["bytes"]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity < ridge:
+        achieved = kw["bytes"] / avg_s / 1e9
+        return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "alg_bytes_per_launch": kw["bytes"], "avg_launch_us": round(avg_s * 1e6, 2),
+                "peak_source": peak_kind + " hbm_gbs"}
+    achieved = kw["flops"] / avg_s / 1e12
+    return {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1),
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+            "alg_flops_per_launch": kw["flops"], "avg_launch_us": round(avg_s * 1e6, 2),
+            "peak_source": peak_kind + " bf16_tflops (burst)"}
+
+
+def max_over_ranks(value: float) -> float:
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([value], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+    return value
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+class ClockSampler:
+    """SM clock and throttle reasons sampled through NVML during a region."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, int(rs)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self, t0: float, t1: float):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        reasons = set()
+        for _, _, r in inside:
+            for name, bit in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for _, m, _ in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle leg
+
+
+def oracle_rate(cfg, w, x, seconds: float, seed: int):
+    """Tokens/s of the float64 oracle on a bounded sample of the batch, in
+    batches of 8 tokens (expert weights fetched and up-cast per expert)."""
+    from oracle import lmoe as O
+
+    def to64(t):
+        return t.detach().to("cpu").to(torch.float64).numpy()
+
+    dense = {k: to64(w[k]) for k in ("w_router", "router_bias", "w_dn", "w_upl", "w_s1",
+                                     "w_s2")}
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(x.shape[0])
+    done, t0 = 0, time.perf_counter()
+    while True:
+        toks = np.sort(order[done:done + 8])
+        if len(toks) == 0:
+            break
+        xs = to64(x[torch.as_tensor(toks, device=x.device)])
+        O.layer_forward(xs, dense["w_router"], dense["router_bias"], dense["w_dn"],
+                        lambda e: to64(w["w1"][e]), lambda e: to64(w["w2"][e]), dense["w_upl"],
+                        dense["w_s1"], dense["w_s2"], cfg.K)
+        done += len(toks)
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count()
+    return done / el, done, el, cores
+
+
+# ---------------------------------------------------------------------------
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="super_decode", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="lmoe", choices=["lmoe", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = CONFIGS[args.config]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(args, cfg, world)
+
+    from datetime import timedelta
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    from latent_space_mixture_b200 import LatentMoE
+
+    dev = torch.device("cuda", local_rank)
+    w, _ = make_weights(cfg, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(shard_seed(cfg.seed, rank))
+    x = make_x(cfg, gen, device=dev)
+    T = cfg.T
+    layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w)
+    y = torch.empty_like(x)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        layer.forward(x, out=y)
+    torch.cuda.synchronize()
+    rc = layer.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} after warm-up")
+
+    clocks = ClockSampler(local_rank).start()
+    layer.profile_enable(True)
+    layer.profile_read(reset=True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()                      # L2 flush, outside the step's events
+        starts[i].record(stream)
+        layer.forward(x, out=y)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.perf_counter()
+    clocks.stop()
+    prof = layer.profile_read(reset=True)
+    layer.profile_enable(False)
+    rc = layer.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} after the timed steps")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms))
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    counts = layer.debug("counts").numpy()
+    lay, per_kernel = algorithmic_work(cfg, T, counts)
+    peaks, peak_kind = load_peaks()
+    prof_by = {n: (ms, c) for n, ms, c in prof}
+    dom = max((n for n in per_kernel if n in prof_by), key=lambda n: prof_by[n][0])
+    roof = roofline_entry(dom, per_kernel[dom], prof_by[dom][0], prof_by[dom][1], peaks,
+                          peak_kind, cfg, T)
+    kernels = {n: {"ms_total": round(ms, 3), "launches": c,
+                   "share": round(ms / max(sum(p[1] for p in prof), 1e-9), 4)}
+               for n, ms, c in prof}
+    layer_time_s = ms_per_step / 1e3
+    layer_roof = {"alg_bytes": lay["bytes"], "alg_flops": lay["flops"],
+                  "hbm_frac": round(lay["bytes"] / layer_time_s / 1e9 / peaks["hbm_gbs"], 4),
+                  "tensor_frac": round(lay["flops"] / layer_time_s / 1e12 / peaks["bf16_tflops"],
+                                       4),
+                  "tflops": round(lay["flops"] / layer_time_s / 1e12, 2)}
+
+    # end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        for _ in range(args.warmup):
+            layer.forward_host(xh, yh)
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            es[i].record(stream)
+            layer.forward_host(xh, yh)
+            ee[i].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es, ee)))
+        e2e = {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
+               "ms_per_step": round(e2e_ms / args.steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, el, cores = oracle_rate(cfg, w, x, args.cpu_seconds, 1000 + cfg.seed)
+        cpu = {"value": round(rate, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} of the {T} tokens of this batch, in batches of 8, {el:.1f} s"}
+
+    launches = layer.launches_per_forward() * args.steps
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; weights N(0, std) bf16, x N(0,1) bf16)",
+            "config": {"workload": cfg.name, "T": T, "d": cfg.d, "latent": cfg.l,
+                       "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
+                       "shared_hidden": cfg.hs, "router_bias": cfg.bias,
+                       "tokens_per_rank": T, "parallelism": f"dp{world} (replicated weights)",
+                       "l2": "256 MiB write between steps, outside the per-step events"},
+            "roofline": roof, "layer_roofline": layer_roof, "kernels": kernels,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clocks.summary(t_wall0, t_wall1),
+            "wall_s_timed_region": round(t_wall1 - t_wall0, 4),
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def run_reference(args, cfg, world):
+    """The oracle as the reference arm: each step is the oracle on a bounded
+    sample of the workload's tokens (rank 0 only)."""
+    from oracle import lmoe as O  # noqa: F401  (fail early if missing)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w, gen = make_weights(cfg, device=dev)
+    x = make_x(cfg, gen, device=dev)
+    per_step = max(1.0, 150.0 / max(args.steps + args.warmup, 1))
+    for _ in range(args.warmup):
+        oracle_rate(cfg, w, x, per_step / 4, 7)
+    rates, n_tot, el_tot, cores = [], 0, 0.0, 1
+    for i in range(args.steps):
+        r, n, el, cores = oracle_rate(cfg, w, x, per_step, 1000 + i)
+        rates.append(r)
+        n_tot += n
+        el_tot += el
+    value = n_tot / el_tot
+    line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * el_tot / args.steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "latent": cfg.l,
+                       "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
+                       "shared_hidden": cfg.hs},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{n_tot} tokens over {args.steps} steps, {el_tot:.1f} s"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,174 @@
+/*
+ * lmoe.h -- C ABI of the B200 (sm_100a) LatentMoE layer forward pass.
+ *
+ * The layer ("NVIDIA Nemotron 3: Efficient and Open Intelligence", xllm-io
+ * paper review, section 三 "LatentMoE 架构" with eq.(1); "Nemotron-3 Super
+ * 精读报告", section 3.3 and table 2.2):
+ *   router at hidden width d: z = W_r x, s = sigmoid(z), key = s + b
+ *     ("Nemotron-3 Super 精读报告", table 6.3: Sigmoid + Expert Biasing);
+ *   the top-K experts by key, weights w = s_sel / sum(s_sel);
+ *   u = W_dn x (d -> l, BF16: the latent projections stay BF16 under the
+ *     pages' NVFP4 recipe, "Nemotron-3 Super 精读报告" table 5.2);
+ *   every selected expert in latent space: o_k = W2[e] sqrelu(W1[e] u);
+ *   v = sum_k w_k o_k; r = W_upl v (l -> d);
+ *   shared expert at width d: sh = W_s2 sqrelu(W_s1 x);  y = r + sh.
+ * sqrelu(a) = max(a, 0)^2 is a convention: the pages name no activation.
+ *
+ * Conventions of every entry point:
+ *   - matrices are row-major [out][in] (K-major), bf16 unless stated;
+ *   - "device" pointers are CUDA device memory of the current device;
+ *   - a `stream` argument is a cudaStream_t (NULL = legacy default stream);
+ *   - calls return LMOE_OK (0) or a negative LMOE_ERR_* code and never throw,
+ *     abort or print; lmoe_strerror() names a code;
+ *   - kernels never trap: a bounded device-side wait that runs out records
+ *     LMOE_ERR_TIMEOUT, read back by lmoe_sync_status().
+ */
+#ifndef LMOE_H_
+#define LMOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LMOE_OK 0
+#define LMOE_ERR_INVALID_ARG (-1) /* null pointer, bad size, T > max_tokens */
+#define LMOE_ERR_UNSUPPORTED (-2) /* dims outside what the kernels handle   */
+#define LMOE_ERR_OOM (-3)         /* device allocation failed (create only) */
+#define LMOE_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed      */
+#define LMOE_ERR_TIMEOUT (-5)     /* a bounded device wait ran out          */
+#define LMOE_ERR_DEVICE (-6)      /* a kernel flagged bad data (e.g. index) */
+
+#define LMOE_FMT_BF16 0  /* experts in BF16                                   */
+#define LMOE_FMT_NVFP4 1 /* experts in NVFP4 (reserved: returns UNSUPPORTED)  */
+
+/* Layer shape.  d, latent, expert_hidden, shared_hidden: multiples of 64.
+ * n_experts: multiple of 32, at most 1024.  top_k: 1..min(32, n_experts).
+ * max_tokens: the largest T a forward call accepts (sizes the workspace). */
+typedef struct lmoe_config {
+  int32_t d;             /* hidden width                                  */
+  int32_t latent;        /* latent width l                                */
+  int32_t n_experts;     /* N                                             */
+  int32_t top_k;         /* K                                             */
+  int32_t expert_hidden; /* h: expert FFN hidden width                    */
+  int32_t shared_hidden; /* h_s: shared-expert hidden width               */
+  int32_t expert_format; /* LMOE_FMT_*                                     */
+  int32_t reserved;      /* must be 0                                     */
+  int64_t max_tokens;    /* >= 1                                          */
+} lmoe_config;
+
+/* Layer weights, all device pointers, copied by lmoe_create (the caller may
+ * free them afterwards). */
+typedef struct lmoe_weights {
+  const void* w_router;    /* [N][d]      bf16                              */
+  const float* router_bias;/* [N]         fp32, or NULL for zeros           */
+  const void* w_dn;        /* [l][d]      bf16                              */
+  const void* w1;          /* [N][h][l]   bf16                              */
+  const void* w2;          /* [N][l][h]   bf16                              */
+  const void* w_upl;       /* [d][l]      bf16                              */
+  const void* w_s1;        /* [h_s][d]    bf16                              */
+  const void* w_s2;        /* [d][h_s]    bf16                              */
+  float act_gscale_latent; /* NVFP4 only: static global scale of u          */
+  float act_gscale_hidden; /* NVFP4 only: static global scale of the expert
+                              hidden activation                             */
+} lmoe_weights;
+
+typedef struct lmoe_handle lmoe_handle;
+
+/* Build a layer on the current device: validates cfg, allocates the weights'
+ * copies (re-laid out: [W_r; W_dn; W_s1] as one [N+l+h_s][d] matrix and
+ * [W_upl | W_s2] as one [d][l+h_s] matrix) and a workspace for max_tokens,
+ * and synchronizes the device once.  *out receives the handle, owned by the
+ * caller until lmoe_destroy.  Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA. */
+int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out);
+
+/* y = layer(x) for T tokens.  x: [T][d] bf16 device, y: [T][d] bf16 device,
+ * both caller-owned, y must not overlap x.  Asynchronous on `stream`: no host
+ * synchronisation, no allocation, no host<->device copy.  T == 0 is a no-op.
+ * One forward may be in flight per handle (the workspace is shared); a handle
+ * is not thread-safe.  Errors: INVALID_ARG (null, T < 0, T > max_tokens),
+ * CUDA (a launch failed).  Device-side faults surface in lmoe_sync_status. */
+int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream);
+
+/* Same as lmoe_forward with HOST buffers: copies x [T][d] bf16 to the device,
+ * runs the layer and copies y [T][d] bf16 back on `stream`, then waits for the
+ * stream.  Page-locked host buffers make the copies asynchronous.  Returns the
+ * lmoe_sync_status() of the call. */
+int lmoe_forward_host(lmoe_handle* h, const void* x_host, int64_t T, void* y_host, void* stream);
+
+/* Waits for `stream`, then returns TIMEOUT or DEVICE if a kernel of this
+ * handle raised its error word since the last call (and clears it), CUDA if
+ * the stream reports an error, else OK. */
+int lmoe_sync_status(lmoe_handle* h, void* stream);
+
+/* Debug/test readout of the last forward's intermediates into HOST memory
+ * (synchronizes the device first).  `bytes` must equal the item's size for
+ * the last T:
+ *   LMOE_DBG_TOPK_IDX  int32 [T][K]   selected experts, key-descending
+ *   LMOE_DBG_TOPK_W    fp32  [T][K]   renormalised router weights
+ *   LMOE_DBG_COUNTS    int32 [N]      routed rows per expert
+ *   LMOE_DBG_OFFSETS   int32 [N+1]    exclusive scan of counts
+ *   LMOE_DBG_PERM      int32 [T*K]    row -> t*K + k (expert, then token order)
+ *   LMOE_DBG_INV       int32 [T][K]   slot -> row
+ *   LMOE_DBG_LOGITS    fp32  [T][N]   router logits z
+ *   LMOE_DBG_U         bf16  [T][l]   latent u
+ *   LMOE_DBG_V         bf16  [T][l]   latent combine v
+ *   LMOE_DBG_HS        bf16  [T][h_s] shared hidden sqrelu(W_s1 x)
+ * Errors: INVALID_ARG (unknown item, wrong size), CUDA. */
+#define LMOE_DBG_TOPK_IDX 1
+#define LMOE_DBG_TOPK_W 2
+#define LMOE_DBG_COUNTS 3
+#define LMOE_DBG_OFFSETS 4
+#define LMOE_DBG_PERM 5
+#define LMOE_DBG_INV 6
+#define LMOE_DBG_LOGITS 7
+#define LMOE_DBG_U 8
+#define LMOE_DBG_V 9
+#define LMOE_DBG_HS 10
+int lmoe_get_debug(lmoe_handle* h, int what, void* dst_host, size_t bytes);
+
+/* Kernel launches one forward of T tokens issues (the same count for every
+ * T > 0 of a handle), or a negative error code. */
+int lmoe_launches_per_forward(const lmoe_handle* h);
+
+/* Per-kernel timing: when enabled, every forward records CUDA events around
+ * each of its kernels on the forward's stream and accumulates their elapsed
+ * times (read at lmoe_profile_read, which synchronizes the device).
+ * lmoe_profile_read fills up to `max` entries: name (static string), total
+ * milliseconds and launch count, and returns the number of entries; `reset`
+ * != 0 clears the accumulators.  Errors: INVALID_ARG, CUDA. */
+int lmoe_profile_enable(lmoe_handle* h, int on);
+int lmoe_profile_read(lmoe_handle* h, const char** names, double* total_ms, int64_t* launches,
+                      int max, int reset);
+
+/* Standalone routing and segment build (the router's top-K, weights and the
+ * per-expert row order) from precomputed fp32 logits [T][N] (device):
+ * outputs (device, caller-owned) topk_idx [T][K] int32, topk_w [T][K] fp32,
+ * counts [N] int32, offsets [N+1] int32, perm [T*K] int32, inv [T][K] int32.
+ * bias: [N] fp32 device or NULL.  workspace: device scratch of at least
+ * lmoe_route_workspace_size(T, N) bytes, 256-byte aligned, caller-owned.
+ * Asynchronous on `stream`.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+size_t lmoe_route_workspace_size(int64_t T, int32_t N);
+int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int32_t K,
+               int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+               int32_t* perm, int32_t* inv, void* workspace, size_t workspace_bytes,
+               void* stream);
+
+/* Runs a one-CTA kernel that waits on an mbarrier nothing arrives on, with a
+ * wait limit of limit_ns nanoseconds (1e3..1e10), and returns the status the
+ * host reads afterwards: LMOE_ERR_TIMEOUT when the bounded wait gave up as
+ * designed.  Checks the device-side failure path without a fault. */
+int lmoe_check_bounded_wait(int64_t limit_ns);
+
+/* Frees everything the handle owns (synchronizes the device first). */
+void lmoe_destroy(lmoe_handle* h);
+
+/* Static description of an error code. */
+const char* lmoe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LMOE_H_ */

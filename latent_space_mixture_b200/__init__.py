@@ -1,0 +1,17 @@
+"""B200-native (sm_100a) LatentMoE layer forward pass.
+
+The layer (NVIDIA Nemotron 3): a sigmoid router with expert biasing at hidden
+width d picks the top-K experts and renormalises their weights; a BF16
+down-projection maps tokens to the latent width l, where the experts
+(squared-ReLU FFNs) run; their weighted sum is projected back to d and added
+to a d-wide shared expert.
+
+All of it runs in liblmoe.so (hand-written CUDA for sm_100a behind the C ABI
+of include/lmoe.h).  This package only marshals arguments: every entry point
+loads the library first and raises when it has not been built (there is no
+other implementation to fall back to).
+"""
+from ._lib import LmoeError
+from .layer import LatentMoE, lmoe_check_bounded_wait, lmoe_route
+
+__all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]

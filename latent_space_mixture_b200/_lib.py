@@ -1,0 +1,82 @@
+"""ctypes declarations of the C ABI in include/lmoe.h (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import (POINTER, Structure, c_char_p, c_double, c_float, c_int, c_int32, c_int64,
+                    c_size_t, c_void_p)
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblmoe.so")
+
+LMOE_OK = 0
+ERRORS = {-1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "OOM", -4: "CUDA", -5: "TIMEOUT",
+          -6: "DEVICE"}
+FMT_BF16, FMT_NVFP4 = 0, 1
+DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 6,
+       "logits": 7, "u": 8, "v": 9, "hs": 10}
+
+
+class LmoeConfig(Structure):
+    _fields_ = [("d", c_int32), ("latent", c_int32), ("n_experts", c_int32), ("top_k", c_int32),
+                ("expert_hidden", c_int32), ("shared_hidden", c_int32),
+                ("expert_format", c_int32), ("reserved", c_int32), ("max_tokens", c_int64)]
+
+
+class LmoeWeights(Structure):
+    _fields_ = [("w_router", c_void_p), ("router_bias", c_void_p), ("w_dn", c_void_p),
+                ("w1", c_void_p), ("w2", c_void_p), ("w_upl", c_void_p), ("w_s1", c_void_p),
+                ("w_s2", c_void_p), ("act_gscale_latent", c_float),
+                ("act_gscale_hidden", c_float)]
+
+
+class LmoeError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        name = ERRORS.get(code, str(code))
+        super().__init__(f"lmoe error {name} ({code}){': ' + what if what else ''}")
+
+
+# exported C symbols with (restype, argtypes)
+SIGNATURES = {
+    "lmoe_create": (c_int, [POINTER(LmoeConfig), POINTER(LmoeWeights), POINTER(c_void_p)]),
+    "lmoe_forward": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
+    "lmoe_forward_host": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
+    "lmoe_sync_status": (c_int, [c_void_p, c_void_p]),
+    "lmoe_get_debug": (c_int, [c_void_p, c_int, c_void_p, c_size_t]),
+    "lmoe_launches_per_forward": (c_int, [c_void_p]),
+    "lmoe_profile_enable": (c_int, [c_void_p, c_int]),
+    "lmoe_profile_read": (c_int, [c_void_p, POINTER(c_char_p), POINTER(c_double),
+                                  POINTER(c_int64), c_int, c_int]),
+    "lmoe_route_workspace_size": (c_size_t, [c_int64, c_int32]),
+    "lmoe_route": (c_int, [c_void_p, c_void_p, c_int64, c_int32, c_int32, c_void_p, c_void_p,
+                           c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                           c_void_p]),
+    "lmoe_check_bounded_wait": (c_int, [c_int64]),
+    "lmoe_destroy": (None, [c_void_p]),
+    "lmoe_strerror": (c_char_p, [c_int]),
+}
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """The CUDA library; raises when it has not been built (there is no
+    fallback implementation)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m latent_space_mixture_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def check(rc: int, what: str = "") -> None:
+    if rc != LMOE_OK:
+        raise LmoeError(rc, what)

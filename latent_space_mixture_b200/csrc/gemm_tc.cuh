@@ -1,0 +1,300 @@
+// Persistent, warp-specialised tcgen05 GEMM used for every contraction of the
+// LatentMoE layer forward pass.
+//
+// Orientation ("swap AB"): the weight matrix W [features][K] is the MMA A
+// operand and fills the 128-row M of tcgen05.mma; a block of token rows
+// X [tokens][K] is the B operand and sets N per tile at run time (a multiple
+// of 16, up to BN).  D = W X^T lands in TMEM with one feature per lane and one
+// token per column.  This keeps ragged per-expert token counts cheap: an
+// expert with 11 routed rows costs an N=16 MMA, not a 128-row tile.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over a static tile list):
+//   warp 0      TMA producer: A tile 128x64 and B rows in 16-row boxes per
+//               k-step, 128-byte swizzle, completion on a "full" mbarrier;
+//   warp 1      TMEM allocator and MMA issuer: 4 x (M128 N K16) per k-step,
+//               tcgen05.commit frees the smem stage, a second commit marks the
+//               accumulator full;
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, transpose through a
+//               per-warp smem tile, call the epilogue functor on 8 consecutive
+//               features of one token row, release the accumulator.
+// Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap
+// the main loop of tile i+1.  Every mbarrier wait is bounded (ptx.cuh).
+#pragma once
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace lmoe {
+
+constexpr int GEMM_BM = 128;          // MMA M: features per tile
+constexpr int GEMM_BK = 64;           // K elements per pipeline stage (128 B)
+constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_EPI_WARPS = 4;
+constexpr int GEMM_STG_LD = 36;       // fp32 staging pitch (32 + 4)
+constexpr int GEMM_BROWS = 16;        // rows per B TMA box
+
+// Where the tiles of one GEMM come from.
+struct TileSource {
+  int dense;               // 1: tokens [0, T) in blocks of BN; 0: device block list
+  int T;                   // dense: number of token rows
+  const int4* blocks;      // list: {expert, first row, rows, 0}
+  const int* nblocks;      // list: number of blocks (device scalar)
+  int FB;                  // feature blocks of 128 per expert
+  int a_rows_per_expert;   // rows of A per expert (0 when dense)
+  int m_valid;             // valid features per expert (multiple of 8)
+  int kblocks;             // K / 64
+};
+
+struct TileInfo {
+  int e, fb, row0, nrows, a_row;
+};
+
+__device__ __forceinline__ int gemm_num_tiles(const TileSource& s, int BN) {
+  const int nb = s.dense ? (s.T + BN - 1) / BN : *s.nblocks;
+  return nb * s.FB;
+}
+
+__device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int tile) {
+  TileInfo t;
+  const int tb = tile / s.FB;
+  t.fb = tile - tb * s.FB;
+  if (s.dense) {
+    t.e = 0;
+    t.row0 = tb * BN;
+    t.nrows = min(BN, s.T - t.row0);
+  } else {
+    const int4 b = s.blocks[tb];
+    t.e = b.x;
+    t.row0 = b.y;
+    t.nrows = b.z;
+  }
+  t.a_row = t.e * s.a_rows_per_expert + t.fb * GEMM_BM;
+  return t;
+}
+
+template <int BN, int STAGES>
+struct GemmLayout {
+  static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
+  static constexpr int B_BYTES = BN * GEMM_BK * 2;
+  static constexpr int STG_BYTES = GEMM_EPI_WARPS * 32 * GEMM_STG_LD * 4;
+  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES) +
+                                    STG_BYTES + BAR_BYTES + 16;
+  static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N range for M=128");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of 2");
+};
+
+template <int BN, int STAGES, class Epi>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+          const TileSource src, const Epi epi, int* err, unsigned long long limit_ns) {
+  using L = GemmLayout<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * L::A_BYTES;
+  float* stg = reinterpret_cast<float*>(sB + STAGES * L::B_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stg) + L::STG_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;   // [2]
+  uint64_t* tempty = tfull + 2;       // [2]
+  uint64_t* drain = tempty + 2;       // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], GEMM_EPI_WARPS * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = gemm_num_tiles(src, BN);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_a = policy_evict_first();   // weights: streamed
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const TileInfo t = gemm_tile(src, BN, tile);
+        const int nload = (t.nrows + GEMM_BROWS - 1) / GEMM_BROWS;
+        const uint32_t tx = L::A_BYTES + nload * GEMM_BROWS * GEMM_BK * 2;
+        for (int kb = 0; kb < src.kblocks; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err, limit_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], tx);
+          tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, kb * GEMM_BK, t.a_row, &full[stage],
+                           pol_a);
+          uint8_t* b_dst = sB + stage * L::B_BYTES;
+          for (int j = 0; j < nload; ++j)
+            tma_load_2d(b_dst + j * GEMM_BROWS * GEMM_BK * 2, &tmB, kb * GEMM_BK,
+                        t.row0 + j * GEMM_BROWS, &full[stage]);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA's smem goes away
+        const long first = issued > STAGES ? issued - STAGES : 0;
+        for (long i = first; i < issued; ++i) {
+          uint64_t* b = &full[i % STAGES];
+          const uint32_t par = static_cast<uint32_t>((i / STAGES) & 1);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(b, par) && global_timer_ns() - t0 < limit_ns) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const TileInfo t = gemm_tile(src, BN, tile);
+        const int n_mma = (t.nrows + 15) & ~15;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err, limit_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t idesc = idesc_bf16(GEMM_BM, n_mma);
+        for (int kb = 0; kb < src.kblocks; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + stage * L::A_BYTES));
+          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + stage * L::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / 16; ++k)   // +32 bytes per K=16 step
+            umma_bf16(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0);
+          umma_commit(&empty[stage]);
+          issued_any = true;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok && issued_any) {
+        umma_commit(drain);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit_ns) {
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                  // TMEM lane quarter of this warp
+    float* my = stg + (warp - 2) * 32 * GEMM_STG_LD;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const TileInfo t = gemm_tile(src, BN, tile);
+      // one lane waits, the warp follows: the TMEM loads below are .sync.aligned
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err, limit_ns);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      tc_fence_after();
+      const int feat_base = t.fb * GEMM_BM + q * 32;
+      for (int c0 = 0; c0 < t.nrows; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) my[j * GEMM_STG_LD + lane] = __uint_as_float(r[j]);
+        __syncwarp();
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int item = lane + 32 * it;
+          const int j = item >> 2;
+          const int g = item & 3;
+          const int feat = feat_base + g * 8;
+          if (c0 + j < t.nrows && feat < src.m_valid) {
+            const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
+            const float4 lo = p[0], hi = p[1];
+            const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            epi.store8(t.e, static_cast<long>(t.row0 + c0 + j), feat, v);
+          }
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, L::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// epilogue helpers
+
+__device__ __forceinline__ void store8_bf16(__nv_bfloat16* dst, const float* v) {
+  __nv_bfloat162 p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(p);
+}
+
+__device__ __forceinline__ float sqrelu(float a) {
+  const float r = fmaxf(a, 0.0f);
+  return r * r;
+}
+
+}  // namespace lmoe

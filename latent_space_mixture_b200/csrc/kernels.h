@@ -1,0 +1,42 @@
+// Launchers of the non-GEMM kernels of the LatentMoE forward pass (host side).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace lmoe {
+
+// Sigmoid router with expert biasing, top-K by key (ties to the lower expert
+// id, slots key-descending) and weights renormalised from the unbiased scores.
+// One warp per token.  N <= 1024, N % 32 == 0, 1 <= K <= min(N, 32).
+cudaError_t launch_route(const float* logits, const float* bias, int64_t T, int N, int K,
+                         int32_t* topk_idx, float* topk_w, cudaStream_t st);
+
+// Per-chunk (32 tokens) expert histograms: chunk_cnt[c][e].
+cudaError_t launch_hist(const int32_t* topk_idx, int64_t T, int N, int K, int32_t* chunk_cnt,
+                        int* err, cudaStream_t st);
+
+// Column scan of chunk_cnt over chunks (in place, exclusive) and counts[e].
+cudaError_t launch_scan(int32_t* chunk_cnt, int64_t T, int N, int32_t* counts, cudaStream_t st);
+
+// Offsets (exclusive scan of counts), perm / inv / per-row weights, and the
+// list of token blocks (at most `bn` rows, one expert each) for the grouped
+// GEMMs: blocks[i] = {expert, first row, rows, 0}, *nblocks = count.
+cudaError_t launch_scatter(const int32_t* topk_idx, const float* topk_w, const int32_t* chunk_base,
+                           const int32_t* counts, int64_t T, int N, int K, int bn,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, float* wrow,
+                           int4* blocks, int32_t* nblocks, int* err, cudaStream_t st);
+
+// u_perm[r] = u[perm[r] / K] for r < T*K (rows of width l, bf16).
+cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int K, int l,
+                          void* u_perm, cudaStream_t st);
+
+// v[t] = sum_k O[inv[t][k]] (fp32, slot order), written as bf16 into the first
+// l columns of vh (row pitch ldv).
+cudaError_t launch_combine(const void* O, const int32_t* inv, int64_t T, int K, int l, void* vh,
+                           int ldv, cudaStream_t st);
+
+// A kernel whose mbarrier wait never completes, bounded by limit_ns: sets
+// DEVERR_TIMEOUT in *err and returns.  Used to check the failure path.
+cudaError_t launch_wait_probe(int* err, unsigned long long limit_ns, cudaStream_t st);
+
+}  // namespace lmoe

@@ -1,0 +1,691 @@
+// C ABI of the LatentMoE layer forward pass (declarations and contracts in
+// include/lmoe.h).  Host orchestration only: every step of the layer runs in
+// the kernels of gemm_tc.cuh and routing.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "gemm_tc.cuh"
+#include "kernels.h"
+#include "lmoe.h"
+
+using bf16 = __nv_bfloat16;
+
+namespace lmoe {
+
+// ---------------------------------------------------------------------------
+// epilogues of the four contractions
+
+// x -> [W_r; W_dn; W_s1] x: router logits (fp32), latent u (bf16) and the
+// shared-expert hidden sqrelu(W_s1 x) (bf16, into columns [l, l+h_s) of vh).
+struct EpiX {
+  float* logits;
+  bf16* u;
+  bf16* vh;
+  int N, l, ldvh;
+  __device__ __forceinline__ void store8(int, long row, int feat, const float* v) const {
+    if (feat < N) {
+      float4* p = reinterpret_cast<float4*>(logits + row * N + feat);
+      p[0] = make_float4(v[0], v[1], v[2], v[3]);
+      p[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else if (feat < N + l) {
+      store8_bf16(u + row * l + (feat - N), v);
+    } else {
+      float a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = sqrelu(v[i]);
+      store8_bf16(vh + row * ldvh + l + (feat - N - l), a);
+    }
+  }
+};
+
+// expert FC1: H[row] = sqrelu(W1[e] u[row])
+struct EpiH {
+  bf16* H;
+  int h;
+  __device__ __forceinline__ void store8(int, long row, int feat, const float* v) const {
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = sqrelu(v[i]);
+    store8_bf16(H + row * h + feat, a);
+  }
+};
+
+// expert FC2 times the router weight of the row: O[row] = w[row] W2[e] H[row]
+struct EpiO {
+  bf16* O;
+  const float* wrow;
+  int l;
+  __device__ __forceinline__ void store8(int, long row, int feat, const float* v) const {
+    const float w = wrow[row];
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = v[i] * w;
+    store8_bf16(O + row * l + feat, a);
+  }
+};
+
+// [W_upl | W_s2] [v ; hs]: routed branch plus shared branch in one K loop
+struct EpiY {
+  bf16* y;
+  int d;
+  __device__ __forceinline__ void store8(int, long row, int feat, const float* v) const {
+    store8_bf16(y + row * d + feat, v);
+  }
+};
+
+// GEMM variants: (BN, STAGES)
+template <int BN>
+struct Stages;
+template <>
+struct Stages<256> {
+  static constexpr int value = 4;
+};
+template <>
+struct Stages<128> {
+  static constexpr int value = 6;
+};
+template <>
+struct Stages<32> {
+  static constexpr int value = 10;
+};
+
+template <int BN, class Epi>
+cudaError_t set_gemm_smem() {
+  using L = GemmLayout<BN, Stages<BN>::value>;
+  return cudaFuncSetAttribute(k_gemm_tc<BN, Stages<BN>::value, Epi>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
+}
+
+template <int BN, class Epi>
+cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const TileSource& src,
+                        const Epi& epi, int grid, int* err, unsigned long long limit,
+                        cudaStream_t st) {
+  using L = GemmLayout<BN, Stages<BN>::value>;
+  k_gemm_tc<BN, Stages<BN>::value, Epi><<<grid, GEMM_THREADS, L::SMEM_BYTES, st>>>(A, B, src, epi,
+                                                                                  err, limit);
+  return cudaGetLastError();
+}
+
+template <class Epi>
+cudaError_t launch_gemm_bn(int bn, const CUtensorMap& A, const CUtensorMap& B,
+                           const TileSource& src, const Epi& epi, int grid, int* err,
+                           unsigned long long limit, cudaStream_t st) {
+  switch (bn) {
+    case 256: return launch_gemm<256>(A, B, src, epi, grid, err, limit, st);
+    case 128: return launch_gemm<128>(A, B, src, epi, grid, err, limit, st);
+    default: return launch_gemm<32>(A, B, src, epi, grid, err, limit, st);
+  }
+}
+
+template <class Epi>
+cudaError_t set_smem_all() {
+  cudaError_t e;
+  if ((e = set_gemm_smem<256, Epi>()) != cudaSuccess) return e;
+  if ((e = set_gemm_smem<128, Epi>()) != cudaSuccess) return e;
+  return set_gemm_smem<32, Epi>();
+}
+
+// ---------------------------------------------------------------------------
+// tensor maps (driver entry point fetched through the runtime)
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major [rows][cols] matrix, box of 64 columns x box_rows rows,
+// 128-byte swizzle; out-of-range rows read as zero.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) cudaSetDevice(dev);
+    else prev = -1;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+static size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace lmoe
+
+using namespace lmoe;
+
+// names of the kernels one forward launches, in launch order
+static const char* const kKernelNames[] = {
+    "xgemm(router|W_dn|W_s1)", "route(sigmoid+bias+topK)", "hist", "scan", "scatter",
+    "gather(u->expert order)", "grouped_gemm1(W1,sqrelu)", "grouped_gemm2(W2,*w)",
+    "combine", "ygemm([W_upl|W_s2])"};
+static constexpr int kNumKernels = 10;
+
+struct lmoe_handle {
+  lmoe_config cfg;
+  int dev = 0;
+  int sms = 148;
+  // weights
+  bf16* w_x = nullptr;     // [N+l+h_s][d]
+  float* bias = nullptr;   // [N]
+  bf16* w1 = nullptr;      // [N][h][l]
+  bf16* w2 = nullptr;      // [N][l][h]
+  bf16* w_y = nullptr;     // [d][l+h_s]
+  // workspace
+  float* logits = nullptr;
+  int32_t* topk_idx = nullptr;
+  float* topk_w = nullptr;
+  int32_t* chunk = nullptr;
+  int32_t* counts = nullptr;
+  int32_t* offsets = nullptr;
+  int32_t* perm = nullptr;
+  int32_t* inv = nullptr;
+  float* wrow = nullptr;
+  int4* blocks = nullptr;
+  int32_t* nblocks = nullptr;
+  bf16* u = nullptr;
+  bf16* u_perm = nullptr;
+  bf16* H = nullptr;
+  bf16* O = nullptr;
+  bf16* vh = nullptr;      // [max_tokens][l+h_s]: v | hs
+  bf16* x_dev = nullptr;   // staging for lmoe_forward_host
+  bf16* y_dev = nullptr;
+  int* err = nullptr;
+  std::vector<void*> allocs;
+  CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy, tm_uperm, tm_H, tm_vh;
+  int64_t last_T = 0;
+  unsigned long long wait_limit_ns = 2000000000ull;
+  // profiling
+  bool prof = false;
+  std::vector<cudaEvent_t> ev;      // pairs
+  std::vector<int> ev_kernel;
+  size_t ev_used = 0;
+  double prof_ms[kNumKernels] = {};
+  int64_t prof_n[kNumKernels] = {};
+};
+
+static int alloc_dev(lmoe_handle* h, void** p, size_t bytes) {
+  if (cudaMalloc(p, bytes < 256 ? 256 : bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return LMOE_ERR_OOM;
+  }
+  h->allocs.push_back(*p);
+  return LMOE_OK;
+}
+
+static void free_all(lmoe_handle* h) {
+  for (void* p : h->allocs) cudaFree(p);
+  h->allocs.clear();
+  for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+  h->ev.clear();
+}
+
+static int check_cfg(const lmoe_config* c) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  if (c->d <= 0 || c->latent <= 0 || c->n_experts <= 0 || c->top_k <= 0 ||
+      c->expert_hidden <= 0 || c->shared_hidden <= 0 || c->max_tokens < 1 || c->reserved != 0)
+    return LMOE_ERR_INVALID_ARG;
+  if (c->top_k > c->n_experts) return LMOE_ERR_INVALID_ARG;
+  if (c->expert_format != LMOE_FMT_BF16 && c->expert_format != LMOE_FMT_NVFP4)
+    return LMOE_ERR_INVALID_ARG;
+  if (c->expert_format == LMOE_FMT_NVFP4) return LMOE_ERR_UNSUPPORTED;
+  if (c->d % 64 || c->latent % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
+    return LMOE_ERR_UNSUPPORTED;
+  if (c->n_experts % 32 || c->n_experts > 1024 || c->top_k > 32) return LMOE_ERR_UNSUPPORTED;
+  const int64_t rows = c->max_tokens * c->top_k;
+  if (rows >= (int64_t(1) << 31) - 65536) return LMOE_ERR_UNSUPPORTED;
+  if (int64_t(c->n_experts) * c->expert_hidden >= (int64_t(1) << 31)) return LMOE_ERR_UNSUPPORTED;
+  if (int64_t(c->n_experts) * c->latent >= (int64_t(1) << 31)) return LMOE_ERR_UNSUPPORTED;
+  return LMOE_OK;
+}
+
+// grouped-GEMM token-block width for a forward of T tokens
+static int grouped_bn(const lmoe_config& c, int64_t T) {
+  const double avg = double(T) * c.top_k / c.n_experts;
+  if (avg <= 40.0) return 32;
+  if (avg <= 160.0) return 128;
+  return 256;
+}
+
+// dense-GEMM token-block width: the widest whose tile count fills the GPU
+static int dense_bn(int64_t T, int fb, int sms) {
+  const int cand[3] = {256, 128, 32};
+  for (int i = 0; i < 3; ++i)
+    if (((T + cand[i] - 1) / cand[i]) * fb >= sms) return cand[i];
+  return 32;
+}
+
+extern "C" {
+
+const char* lmoe_strerror(int code) {
+  switch (code) {
+    case LMOE_OK: return "ok";
+    case LMOE_ERR_INVALID_ARG: return "invalid argument";
+    case LMOE_ERR_UNSUPPORTED: return "unsupported layer shape or format";
+    case LMOE_ERR_OOM: return "device allocation failed";
+    case LMOE_ERR_CUDA: return "CUDA call failed";
+    case LMOE_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case LMOE_ERR_DEVICE: return "a kernel flagged invalid data";
+    default: return "unknown error";
+  }
+}
+
+int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out) {
+  if (!out) return LMOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = check_cfg(cfg);
+  if (rc != LMOE_OK) return rc;
+  if (!w || !w->w_router || !w->w_dn || !w->w1 || !w->w2 || !w->w_upl || !w->w_s1 || !w->w_s2)
+    return LMOE_ERR_INVALID_ARG;
+  if (!get_encode()) return LMOE_ERR_CUDA;
+
+  lmoe_handle* h = new (std::nothrow) lmoe_handle();
+  if (!h) return LMOE_ERR_OOM;
+  h->cfg = *cfg;
+  if (cudaGetDevice(&h->dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess) {
+    delete h;
+    return LMOE_ERR_CUDA;
+  }
+  const lmoe_config& c = h->cfg;
+  const int64_t N = c.n_experts, d = c.d, l = c.latent, hh = c.expert_hidden,
+                hs = c.shared_hidden, K = c.top_k, Tm = c.max_tokens;
+  const int64_t rows = Tm * K;
+  const int64_t C = (Tm + 31) / 32;
+  // operand buffers read by TMA hold at least one box of rows
+  const int64_t rows_b = rows < 256 ? 256 : rows;
+  const int64_t Tm_b = Tm < 256 ? 256 : Tm;
+  const int64_t d_a = d < GEMM_BM ? GEMM_BM : d;
+  const int64_t max_blocks = rows / 32 + N + 1;
+  struct Req {
+    void** p;
+    size_t bytes;
+  } reqs[] = {
+      {(void**)&h->w_x, size_t((N + l + hs) * d * 2)},
+      {(void**)&h->bias, size_t(N * 4)},
+      {(void**)&h->w1, size_t(N * hh * l * 2)},
+      {(void**)&h->w2, size_t(N * l * hh * 2)},
+      {(void**)&h->w_y, size_t(d_a * (l + hs) * 2)},
+      {(void**)&h->logits, size_t(Tm * N * 4)},
+      {(void**)&h->topk_idx, size_t(rows * 4)},
+      {(void**)&h->topk_w, size_t(rows * 4)},
+      {(void**)&h->chunk, size_t(C * N * 4)},
+      {(void**)&h->counts, size_t(N * 4)},
+      {(void**)&h->offsets, size_t((N + 1) * 4)},
+      {(void**)&h->perm, size_t(rows * 4)},
+      {(void**)&h->inv, size_t(rows * 4)},
+      {(void**)&h->wrow, size_t(rows * 4)},
+      {(void**)&h->blocks, size_t(max_blocks * 16)},
+      {(void**)&h->nblocks, size_t(4)},
+      {(void**)&h->u, size_t(Tm * l * 2)},
+      {(void**)&h->u_perm, size_t(rows_b * l * 2)},
+      {(void**)&h->H, size_t(rows_b * hh * 2)},
+      {(void**)&h->O, size_t(rows * l * 2)},
+      {(void**)&h->vh, size_t(Tm_b * (l + hs) * 2)},
+      {(void**)&h->x_dev, size_t(Tm_b * d * 2)},
+      {(void**)&h->y_dev, size_t(Tm * d * 2)},
+      {(void**)&h->err, size_t(4)},
+  };
+  for (auto& r : reqs) {
+    if ((rc = alloc_dev(h, r.p, r.bytes)) != LMOE_OK) {
+      free_all(h);
+      delete h;
+      return rc;
+    }
+  }
+  bool ok = true;
+  // weights, re-laid: [W_r; W_dn; W_s1] and [W_upl | W_s2]
+  ok &= cudaMemcpy(h->w_x, w->w_router, N * d * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemcpy(h->w_x + N * d, w->w_dn, l * d * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemcpy(h->w_x + (N + l) * d, w->w_s1, hs * d * 2, cudaMemcpyDeviceToDevice) ==
+        cudaSuccess;
+  ok &= cudaMemcpy(h->w1, w->w1, N * hh * l * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemcpy(h->w2, w->w2, N * l * hh * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemcpy2D(h->w_y, (l + hs) * 2, w->w_upl, l * 2, l * 2, d,
+                     cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemcpy2D(h->w_y + l, (l + hs) * 2, w->w_s2, hs * 2, hs * 2, d,
+                     cudaMemcpyDeviceToDevice) == cudaSuccess;
+  if (w->router_bias)
+    ok &= cudaMemcpy(h->bias, w->router_bias, N * 4, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  else
+    ok &= cudaMemset(h->bias, 0, N * 4) == cudaSuccess;
+  ok &= cudaMemset(h->err, 0, 4) == cudaSuccess;
+  ok &= cudaMemset(h->vh, 0, Tm_b * (l + hs) * 2) == cudaSuccess;
+  ok &= cudaMemset(h->u_perm, 0, rows_b * l * 2) == cudaSuccess;
+  ok &= cudaMemset(h->H, 0, rows_b * hh * 2) == cudaSuccess;
+  ok &= cudaMemset(h->x_dev, 0, Tm_b * d * 2) == cudaSuccess;
+  if (d_a > d)
+    ok &= cudaMemset(h->w_y + d * (l + hs), 0, (d_a - d) * (l + hs) * 2) == cudaSuccess;
+  // tensor maps of the fixed operands
+  ok &= make_map(&h->tm_wx, h->w_x, N + l + hs, d, GEMM_BM);
+  ok &= make_map(&h->tm_w1, h->w1, N * hh, l, GEMM_BM);
+  ok &= make_map(&h->tm_w2, h->w2, N * l, hh, GEMM_BM);
+  ok &= make_map(&h->tm_wy, h->w_y, d_a, l + hs, GEMM_BM);
+  ok &= make_map(&h->tm_uperm, h->u_perm, rows_b, l, GEMM_BROWS);
+  ok &= make_map(&h->tm_H, h->H, rows_b, hh, GEMM_BROWS);
+  ok &= make_map(&h->tm_vh, h->vh, Tm_b, l + hs, GEMM_BROWS);
+  ok &= set_smem_all<EpiX>() == cudaSuccess;
+  ok &= set_smem_all<EpiH>() == cudaSuccess;
+  ok &= set_smem_all<EpiO>() == cudaSuccess;
+  ok &= set_smem_all<EpiY>() == cudaSuccess;
+  ok &= cudaDeviceSynchronize() == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    free_all(h);
+    delete h;
+    return LMOE_ERR_CUDA;
+  }
+  *out = h;
+  return LMOE_OK;
+}
+
+void lmoe_destroy(lmoe_handle* h) {
+  if (!h) return;
+  DeviceGuard g(h->dev);
+  cudaDeviceSynchronize();
+  free_all(h);
+  delete h;
+}
+
+int lmoe_launches_per_forward(const lmoe_handle* h) {
+  return h ? kNumKernels : LMOE_ERR_INVALID_ARG;
+}
+
+static int prof_begin(lmoe_handle* h, int kernel, cudaStream_t st) {
+  if (!h->prof) return -1;
+  if (h->ev_used + 2 > h->ev.size()) return -1;   // pool full: not recorded
+  const size_t i = h->ev_used;
+  h->ev_used += 2;
+  h->ev_kernel[i / 2] = kernel;
+  cudaEventRecord(h->ev[i], st);
+  return static_cast<int>(i);
+}
+
+static void prof_end(lmoe_handle* h, int slot, cudaStream_t st) {
+  if (slot >= 0) cudaEventRecord(h->ev[slot + 1], st);
+}
+
+#define LMOE_STEP(kidx, call)                        \
+  do {                                               \
+    const int _slot = prof_begin(h, (kidx), st);     \
+    const cudaError_t _e = (call);                   \
+    prof_end(h, _slot, st);                          \
+    if (_e != cudaSuccess) return LMOE_ERR_CUDA;     \
+  } while (0)
+
+int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return LMOE_OK;
+  if (!x || !y) return LMOE_ERR_INVALID_ARG;
+  const lmoe_config& c = h->cfg;
+  const int64_t d = c.d;
+  const char* xb = static_cast<const char*>(x);
+  const char* yb = static_cast<const char*>(y);
+  if (xb < yb + T * d * 2 && yb < xb + T * d * 2) return LMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15)
+    return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int N = c.n_experts, l = c.latent, hh = c.expert_hidden, hs = c.shared_hidden,
+            K = c.top_k;
+  const int ldvh = l + hs;
+  const unsigned long long lim = h->wait_limit_ns;
+  CUtensorMap tm_x;
+  if (T < GEMM_BROWS) {
+    // fewer rows than one TMA box: read x from the padded staging buffer
+    if (x != h->x_dev &&
+        cudaMemcpyAsync(h->x_dev, x, T * d * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    if (!make_map(&tm_x, h->x_dev, GEMM_BROWS, d, GEMM_BROWS)) return LMOE_ERR_CUDA;
+  } else if (!make_map(&tm_x, x, T, d, GEMM_BROWS)) {
+    return LMOE_ERR_CUDA;
+  }
+  h->last_T = T;
+
+  // 1. [W_r; W_dn; W_s1] x: logits, u, shared hidden
+  {
+    TileSource s{1, static_cast<int>(T), nullptr, nullptr, (N + l + hs + 127) / 128, 0,
+                 N + l + hs, static_cast<int>(d / 64)};
+    const int bn = dense_bn(T, s.FB, h->sms);
+    const int64_t tiles = ((T + bn - 1) / bn) * s.FB;
+    const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
+    EpiX epi{h->logits, h->u, h->vh, N, l, ldvh};
+    LMOE_STEP(0, launch_gemm_bn(bn, h->tm_wx, tm_x, s, epi, grid, h->err, lim, st));
+  }
+  // 2-5. routing and segments
+  const int gbn = grouped_bn(c, T);
+  LMOE_STEP(1, launch_route(h->logits, h->bias, T, N, K, h->topk_idx, h->topk_w, st));
+  LMOE_STEP(2, launch_hist(h->topk_idx, T, N, K, h->chunk, h->err, st));
+  LMOE_STEP(3, launch_scan(h->chunk, T, N, h->counts, st));
+  LMOE_STEP(4, launch_scatter(h->topk_idx, h->topk_w, h->chunk, h->counts, T, N, K, gbn,
+                              h->offsets, h->perm, h->inv, h->wrow, h->blocks, h->nblocks,
+                              h->err, st));
+  // 6. latent rows into expert order
+  LMOE_STEP(5, launch_gather(h->u, h->perm, T * K, K, l, h->u_perm, st));
+  // 7. H = sqrelu(W1[e] u)
+  {
+    TileSource s{0, 0, h->blocks, h->nblocks, (hh + 127) / 128, hh, hh, l / 64};
+    EpiH epi{h->H, hh};
+    LMOE_STEP(6, launch_gemm_bn(gbn, h->tm_w1, h->tm_uperm, s, epi, h->sms, h->err, lim, st));
+  }
+  // 8. O = w * W2[e] H
+  {
+    TileSource s{0, 0, h->blocks, h->nblocks, (l + 127) / 128, l, l, hh / 64};
+    EpiO epi{h->O, h->wrow, l};
+    LMOE_STEP(7, launch_gemm_bn(gbn, h->tm_w2, h->tm_H, s, epi, h->sms, h->err, lim, st));
+  }
+  // 9. v = sum_k O[inv[t][k]]
+  LMOE_STEP(8, launch_combine(h->O, h->inv, T, K, l, h->vh, ldvh, st));
+  // 10. y = [W_upl | W_s2] [v ; hs]
+  {
+    TileSource s{1, static_cast<int>(T), nullptr, nullptr, static_cast<int>((d + 127) / 128), 0,
+                 static_cast<int>(d), ldvh / 64};
+    const int bn = dense_bn(T, s.FB, h->sms);
+    const int64_t tiles = ((T + bn - 1) / bn) * s.FB;
+    const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
+    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d)};
+    LMOE_STEP(9, launch_gemm_bn(bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
+  }
+  return LMOE_OK;
+}
+
+int lmoe_sync_status(lmoe_handle* h, void* stream) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LMOE_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpy(&flag, h->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (flag) {
+    if (cudaMemset(h->err, 0, 4) != cudaSuccess) return LMOE_ERR_CUDA;
+    return (flag & DEVERR_TIMEOUT) ? LMOE_ERR_TIMEOUT : LMOE_ERR_DEVICE;
+  }
+  return LMOE_OK;
+}
+
+int lmoe_forward_host(lmoe_handle* h, const void* x_host, int64_t T, void* y_host, void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return LMOE_OK;
+  if (!x_host || !y_host) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = size_t(T) * h->cfg.d * 2;
+  if (cudaMemcpyAsync(h->x_dev, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  int rc = lmoe_forward(h, h->x_dev, T, h->y_dev, stream);
+  if (rc != LMOE_OK) return rc;
+  if (cudaMemcpyAsync(y_host, h->y_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  return lmoe_sync_status(h, stream);
+}
+
+int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
+  if (!h || !dst) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  const lmoe_config& c = h->cfg;
+  const int64_t T = h->last_T, K = c.top_k, N = c.n_experts, l = c.latent,
+                hs = c.shared_hidden;
+  const void* src = nullptr;
+  size_t want = 0;
+  bool strided = false;
+  size_t col0 = 0, cols = 0;
+  switch (what) {
+    case LMOE_DBG_TOPK_IDX: src = h->topk_idx; want = T * K * 4; break;
+    case LMOE_DBG_TOPK_W: src = h->topk_w; want = T * K * 4; break;
+    case LMOE_DBG_COUNTS: src = h->counts; want = N * 4; break;
+    case LMOE_DBG_OFFSETS: src = h->offsets; want = (N + 1) * 4; break;
+    case LMOE_DBG_PERM: src = h->perm; want = T * K * 4; break;
+    case LMOE_DBG_INV: src = h->inv; want = T * K * 4; break;
+    case LMOE_DBG_LOGITS: src = h->logits; want = T * N * 4; break;
+    case LMOE_DBG_U: src = h->u; want = T * l * 2; break;
+    case LMOE_DBG_V: strided = true; col0 = 0; cols = l; want = T * l * 2; break;
+    case LMOE_DBG_HS: strided = true; col0 = l; cols = hs; want = T * hs * 2; break;
+    default: return LMOE_ERR_INVALID_ARG;
+  }
+  if (bytes != want) return LMOE_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LMOE_ERR_CUDA;
+  if (want == 0) return LMOE_OK;
+  cudaError_t e;
+  if (strided)
+    e = cudaMemcpy2D(dst, cols * 2, h->vh + col0, (l + hs) * 2, cols * 2, T,
+                     cudaMemcpyDeviceToHost);
+  else
+    e = cudaMemcpy(dst, src, want, cudaMemcpyDeviceToHost);
+  return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+int lmoe_profile_enable(lmoe_handle* h, int on) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  if (on && h->ev.empty()) {
+    const size_t pairs = 4096;
+    h->ev.resize(2 * pairs);
+    h->ev_kernel.assign(pairs, 0);
+    for (auto& e : h->ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return LMOE_ERR_CUDA;
+  }
+  h->prof = on != 0;
+  return LMOE_OK;
+}
+
+int lmoe_profile_read(lmoe_handle* h, const char** names, double* total_ms, int64_t* launches,
+                      int max, int reset) {
+  if (!h || max < 0) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  if (cudaDeviceSynchronize() != cudaSuccess) return LMOE_ERR_CUDA;
+  for (size_t i = 0; i + 1 < h->ev_used; i += 2) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, h->ev[i], h->ev[i + 1]) != cudaSuccess) return LMOE_ERR_CUDA;
+    h->prof_ms[h->ev_kernel[i / 2]] += ms;
+    h->prof_n[h->ev_kernel[i / 2]] += 1;
+  }
+  h->ev_used = 0;
+  const int n = max < kNumKernels ? max : kNumKernels;
+  for (int k = 0; k < n; ++k) {
+    if (names) names[k] = kKernelNames[k];
+    if (total_ms) total_ms[k] = h->prof_ms[k];
+    if (launches) launches[k] = h->prof_n[k];
+  }
+  if (reset)
+    for (int k = 0; k < kNumKernels; ++k) {
+      h->prof_ms[k] = 0;
+      h->prof_n[k] = 0;
+    }
+  return n;
+}
+
+size_t lmoe_route_workspace_size(int64_t T, int32_t N) {
+  if (T < 0 || N <= 0) return 0;
+  const int64_t C = (T + 31) / 32;
+  const int64_t rows = T * 32;   // K <= 32
+  return align256(C * N * 4) + align256(rows * 4) + align256((rows / 32 + N + 1) * 16) +
+         align256(4) + align256(4);
+}
+
+int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int32_t K,
+               int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+               int32_t* perm, int32_t* inv, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  if (T < 0 || N <= 0 || K <= 0 || K > N) return LMOE_ERR_INVALID_ARG;
+  if (N % 32 || N > 1024 || K > 32) return LMOE_ERR_UNSUPPORTED;
+  if (T * K >= (int64_t(1) << 31)) return LMOE_ERR_UNSUPPORTED;
+  if (!counts || !offsets || (T > 0 && (!logits || !topk_idx || !topk_w || !perm || !inv)))
+    return LMOE_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < lmoe_route_workspace_size(T, N) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return LMOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t C = (T + 31) / 32;
+  const int64_t rows = T * 32;
+  char* ws = static_cast<char*>(workspace);
+  int32_t* chunk = reinterpret_cast<int32_t*>(ws);
+  ws += align256(C * N * 4);
+  float* wrow = reinterpret_cast<float*>(ws);
+  ws += align256(rows * 4);
+  int4* blocks = reinterpret_cast<int4*>(ws);
+  ws += align256((rows / 32 + N + 1) * 16);
+  int32_t* nblocks = reinterpret_cast<int32_t*>(ws);
+  ws += align256(4);
+  int* err = reinterpret_cast<int*>(ws);
+  if (cudaMemsetAsync(err, 0, 4, st) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (T == 0) {
+    if (cudaMemsetAsync(counts, 0, N * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, (N + 1) * 4, st) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    return LMOE_OK;
+  }
+  if (launch_route(logits, bias, T, N, K, topk_idx, topk_w, st) != cudaSuccess ||
+      launch_hist(topk_idx, T, N, K, chunk, err, st) != cudaSuccess ||
+      launch_scan(chunk, T, N, counts, st) != cudaSuccess ||
+      launch_scatter(topk_idx, topk_w, chunk, counts, T, N, K, 256, offsets, perm, inv, wrow,
+                     blocks, nblocks, err, st) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  return LMOE_OK;
+}
+
+int lmoe_check_bounded_wait(int64_t limit_ns) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ll) return LMOE_ERR_INVALID_ARG;
+  int* err = nullptr;
+  if (cudaMalloc(&err, 4) != cudaSuccess) return LMOE_ERR_OOM;
+  int flag = 0;
+  bool ok = cudaMemset(err, 0, 4) == cudaSuccess &&
+            launch_wait_probe(err, static_cast<unsigned long long>(limit_ns), 0) == cudaSuccess &&
+            cudaDeviceSynchronize() == cudaSuccess &&
+            cudaMemcpy(&flag, err, 4, cudaMemcpyDeviceToHost) == cudaSuccess;
+  cudaFree(err);
+  if (!ok) return LMOE_ERR_CUDA;
+  return (flag & DEVERR_TIMEOUT) ? LMOE_ERR_TIMEOUT : LMOE_OK;
+}
+
+}  // extern "C"

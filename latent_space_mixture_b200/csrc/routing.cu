@@ -1,0 +1,381 @@
+// Routing, per-expert segments, row gather and latent combine of the LatentMoE
+// forward pass.
+//
+// Router: sigmoid scores with expert biasing ("Nemotron-3 Super 精读报告",
+// table 6.3: 路由机制 Sigmoid + Expert Biasing), top-K per token and weights
+// renormalised to sum 1; the gating stays at width d ("NVIDIA Nemotron 3:
+// Efficient and Open Intelligence", section 五 架构实现要点).  The bias enters
+// the selection only.
+//
+// Segments: rows ordered by expert, then token (a stable counting sort of the
+// routed (token, slot) pairs), built deterministically without atomics on
+// global memory: per 32-token chunk a bitmask per expert gives each token's
+// rank inside the chunk, a column scan over chunks gives the chunk's base.
+#include <cfloat>
+#include <climits>
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace lmoe {
+
+// ---------------------------------------------------------------------------
+// router: one warp per token
+
+__global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
+                                               const float* __restrict__ bias, int64_t T, int N,
+                                               int K, int32_t* __restrict__ topk_idx,
+                                               float* __restrict__ topk_w) {
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const float* z = logits + t * N;
+  const int npl = N >> 5;   // experts per lane: e = lane + 32 i
+  float key[32], s[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (i < npl) {
+      const int e = lane + 32 * i;
+      const float sc = 1.0f / (1.0f + expf(-z[e]));
+      s[i] = sc;
+      key[i] = sc + (bias ? bias[e] : 0.0f);
+    } else {
+      s[i] = 0.0f;
+      key[i] = -INFINITY;
+    }
+  }
+  uint32_t taken = 0;
+  int my_e = 0;
+  float my_s = 0.0f;
+  for (int k = 0; k < K; ++k) {
+    float bk = -INFINITY, bs = 0.0f;
+    int be = INT_MAX;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i < npl && !((taken >> i) & 1u) && (be == INT_MAX || key[i] > bk)) {
+        bk = key[i];
+        be = lane + 32 * i;
+        bs = s[i];
+      }
+    }
+    // warp arg-max: key descending, then expert id ascending
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+        bs = os;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == k) {
+      my_e = be;
+      my_s = bs;
+    }
+  }
+  // sum of the selected scores in slot order (identical on every lane)
+  float sum = 0.0f;
+  for (int k = 0; k < K; ++k) sum += __shfl_sync(0xffffffffu, my_s, k);
+  if (lane < K) {
+    topk_idx[t * K + lane] = my_e;
+    topk_w[t * K + lane] = __fdiv_rn(my_s, sum);
+  }
+}
+
+cudaError_t launch_route(const float* logits, const float* bias, int64_t T, int N, int K,
+                         int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  const int64_t blocks = (T + 7) / 8;
+  k_route<<<static_cast<unsigned>(blocks), 256, 0, st>>>(logits, bias, T, N, K, topk_idx, topk_w);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// per-chunk expert masks and histograms (chunk = 32 tokens = one warp)
+
+__device__ __forceinline__ void build_chunk_masks(uint32_t* m, const int32_t* __restrict__ idx,
+                                                  int64_t c, int64_t T, int N, int K, int lane,
+                                                  int* err) {
+  for (int e = lane; e < N; e += 32) m[e] = 0u;
+  __syncwarp();
+  const int64_t t = c * 32 + lane;
+  if (t < T) {
+    for (int k = 0; k < K; ++k) {
+      const int e = idx[t * K + k];
+      if (e < 0 || e >= N) {
+        atomicOr(err, DEVERR_BAD_INDEX);
+        continue;
+      }
+      atomicOr(&m[e], 1u << lane);
+    }
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, int64_t T, int N,
+                                              int K, int32_t* __restrict__ chunk_cnt, int* err) {
+  extern __shared__ uint32_t hist_masks[];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + w;
+  const int64_t nchunks = (T + 31) / 32;
+  if (c >= nchunks) return;
+  uint32_t* m = hist_masks + w * N;
+  build_chunk_masks(m, idx, c, T, N, K, lane, err);
+  for (int e = lane; e < N; e += 32) chunk_cnt[c * N + e] = __popc(m[e]);
+}
+
+cudaError_t launch_hist(const int32_t* topk_idx, int64_t T, int N, int K, int32_t* chunk_cnt,
+                        int* err, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  const int64_t nchunks = (T + 31) / 32;
+  const unsigned blocks = static_cast<unsigned>((nchunks + 7) / 8);
+  k_hist<<<blocks, 256, 8 * N * sizeof(uint32_t), st>>>(topk_idx, T, N, K, chunk_cnt, err);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// exclusive column scan of chunk_cnt over chunks; 32 experts per block
+
+__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ chunk, int64_t C, int N,
+                                               int32_t* __restrict__ counts) {
+  __shared__ int32_t tile[32][33];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int e0 = blockIdx.x * 32;
+  int carry = 0;   // running total of expert e0 + ty (held by warp ty)
+  for (int64_t g = 0; g < C; g += 32) {
+    const int64_t c = g + ty;
+    tile[ty][tx] = (c < C) ? chunk[c * N + e0 + tx] : 0;
+    __syncthreads();
+    // warp ty scans expert column ty over the 32 chunks of this group
+    const int v = tile[tx][ty];
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (tx >= off) incl += o;
+    }
+    tile[tx][ty] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+    __syncthreads();
+    if (c < C) chunk[c * N + e0 + tx] = tile[ty][tx];
+    __syncthreads();
+  }
+  if (tx == 0) counts[e0 + ty] = carry;
+}
+
+cudaError_t launch_scan(int32_t* chunk_cnt, int64_t T, int N, int32_t* counts, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  const int64_t C = (T + 31) / 32;
+  k_scan<<<N / 32, dim3(32, 32), 0, st>>>(chunk_cnt, C, N, counts);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// offsets, perm / inv / row weights, and the token-block list
+
+// Exclusive prefix of `v` over the 256 threads of the block.
+__device__ __forceinline__ int block_excl_scan_256(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) wsum[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int s = (lane < 8) ? wsum[lane] : 0;
+    int si = s;
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, si, off);
+      if (lane >= off) si += o;
+    }
+    if (lane < 8) wsum[8 + lane] = si - s;
+    if (lane == 7) *total = si;
+  }
+  __syncthreads();
+  const int r = wsum[8 + w] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(256) k_scatter(
+    const int32_t* __restrict__ idx, const float* __restrict__ topk_w,
+    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ counts, int64_t T, int N,
+    int K, int bn, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv, float* __restrict__ wrow, int4* __restrict__ blocks,
+    int32_t* __restrict__ nblocks, int* err) {
+  extern __shared__ int32_t sc_smem[];
+  int32_t* off = sc_smem;                                    // [N + 1]
+  uint32_t* masks = reinterpret_cast<uint32_t*>(off + N + 1);  // [8][N]
+  __shared__ int wsum[16];
+  __shared__ int total;
+
+  // offsets: exclusive scan of counts, 4 experts per thread (N <= 1024)
+  const int e4 = threadIdx.x * 4;
+  int c4[4];
+  int s4 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    c4[i] = (e4 + i < N) ? counts[e4 + i] : 0;
+    s4 += c4[i];
+  }
+  int base = block_excl_scan_256(s4, wsum, &total);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (e4 + i < N) off[e4 + i] = base;
+    base += c4[i];
+  }
+  if (threadIdx.x == 0) off[N] = total;
+  __syncthreads();
+
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e <= N; e += blockDim.x) offsets[e] = off[e];
+    // token blocks of at most bn rows per expert, in expert order
+    int nb4[4];
+    int snb = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      nb4[i] = (c4[i] + bn - 1) / bn;
+      snb += nb4[i];
+    }
+    int bbase = block_excl_scan_256(snb, wsum, &total);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = e4 + i;
+      for (int j = 0; j < nb4[i]; ++j) {
+        const int r0 = j * bn;
+        blocks[bbase + j] = make_int4(e, off[e] + r0, min(bn, c4[i] - r0), 0);
+      }
+      bbase += nb4[i];
+    }
+    if (threadIdx.x == 0) *nblocks = total;
+  }
+
+  // rows of the routed (token, slot) pairs of this warp's chunk
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * 8 + w;
+  const int64_t nchunks = (T + 31) / 32;
+  if (c >= nchunks) return;
+  uint32_t* m = masks + w * N;
+  build_chunk_masks(m, idx, c, T, N, K, lane, err);
+  const int64_t t = c * 32 + lane;
+  if (t < T) {
+    const uint32_t lower = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) {
+      const int e = idx[t * K + k];
+      if (e < 0 || e >= N) continue;
+      const int row = off[e] + chunk_base[c * N + e] + __popc(m[e] & lower);
+      inv[t * K + k] = row;
+      perm[row] = static_cast<int32_t>(t * K + k);
+      wrow[row] = topk_w[t * K + k];
+    }
+  }
+}
+
+cudaError_t launch_scatter(const int32_t* topk_idx, const float* topk_w, const int32_t* chunk_base,
+                           const int32_t* counts, int64_t T, int N, int K, int bn,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, float* wrow,
+                           int4* blocks, int32_t* nblocks, int* err, cudaStream_t st) {
+  const int64_t nchunks = (T + 31) / 32;
+  const unsigned nblk = static_cast<unsigned>(nchunks > 0 ? (nchunks + 7) / 8 : 1);
+  const size_t smem = (N + 1) * sizeof(int32_t) + 8 * N * sizeof(uint32_t);
+  k_scatter<<<nblk, 256, smem, st>>>(topk_idx, topk_w, chunk_base, counts, T, N, K, bn, offsets,
+                                     perm, inv, wrow, blocks, nblocks, err);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// gather of latent rows into expert order: u_perm[r] = u[perm[r] / K]
+
+__global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ u,
+                                                const int32_t* __restrict__ perm, int64_t rows,
+                                                int K, int l8, uint4* __restrict__ u_perm) {
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += nwarps) {
+    const int64_t tok = perm[r] / K;
+    const uint4* src = u + tok * l8;
+    uint4* dst = u_perm + r * l8;
+    for (int i = lane; i < l8; i += 32) dst[i] = src[i];
+  }
+}
+
+cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int K, int l,
+                          void* u_perm, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  int64_t blocks = (rows + 7) / 8;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_gather<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const uint4*>(u), perm, rows, K, l / 8, static_cast<uint4*>(u_perm));
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// latent combine in token order: v[t] = sum_k O[inv[t][k]], fixed slot order
+
+__global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict__ O,
+                                                 const int32_t* __restrict__ inv, int64_t T,
+                                                 int K, int l, __nv_bfloat16* __restrict__ vh,
+                                                 int ldv) {
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const int my_row = (lane < K) ? inv[t * K + lane] : 0;
+  for (int c = lane * 8; c < l; c += 256) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int k = 0; k < K; ++k) {
+      const int64_t row = __shfl_sync(0xffffffffu, my_row, k);
+      const uint4 raw = *reinterpret_cast<const uint4*>(O + row * l + c);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(p[i]);
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    }
+    __nv_bfloat162 outp[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) outp[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4*>(vh + t * ldv + c) = *reinterpret_cast<const uint4*>(outp);
+  }
+}
+
+cudaError_t launch_combine(const void* O, const int32_t* inv, int64_t T, int K, int l, void* vh,
+                           int ldv, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  const int64_t blocks = (T + 7) / 8;
+  k_combine<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(O), inv, T, K, l, static_cast<__nv_bfloat16*>(vh), ldv);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// bounded-wait probe: an mbarrier that nothing arrives on
+
+__global__ void k_wait_probe(int* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &abort_flag, err, limit_ns);
+}
+
+cudaError_t launch_wait_probe(int* err, unsigned long long limit_ns, cudaStream_t st) {
+  k_wait_probe<<<1, 32, 0, st>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace lmoe

@@ -1,0 +1,172 @@
+"""Python binding of the LatentMoE layer: the C ABI's calls with the same names,
+taking torch tensors for device memory and torch streams.  Every step of the
+layer runs in the CUDA library; nothing here computes."""
+from __future__ import annotations
+
+import ctypes
+from ctypes import byref, c_char_p, c_double, c_int64, c_void_p
+from typing import Dict, Optional
+
+import torch
+
+from . import _lib
+from ._lib import DBG, FMT_BF16, FMT_NVFP4, LmoeConfig, LmoeError, LmoeWeights, check
+
+__all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]
+
+_WEIGHT_SHAPES = {
+    "w_router": ("N", "d"), "w_dn": ("l", "d"), "w1": ("N", "h", "l"), "w2": ("N", "l", "h"),
+    "w_upl": ("d", "l"), "w_s1": ("hs", "d"), "w_s2": ("d", "hs"),
+}
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return c_void_p(s.cuda_stream)
+
+
+class LatentMoE:
+    """lmoe_create / lmoe_forward / lmoe_destroy for one layer.
+
+    weights: dict of CUDA bf16 tensors w_router [N][d], w_dn [l][d],
+    w1 [N][h][l], w2 [N][l][h], w_upl [d][l], w_s1 [h_s][d], w_s2 [d][h_s],
+    and optionally router_bias [N] fp32.  The library copies them.
+    """
+
+    def __init__(self, d: int, latent: int, n_experts: int, top_k: int, expert_hidden: int,
+                 shared_hidden: int, max_tokens: int, weights: Dict[str, torch.Tensor],
+                 expert_format: str = "bf16", act_gscales=(0.0, 0.0)):
+        self.lib = _lib.load()
+        dims = {"d": d, "l": latent, "N": n_experts, "h": expert_hidden, "hs": shared_hidden}
+        for k, shape in _WEIGHT_SHAPES.items():
+            t = weights[k]
+            want = tuple(dims[s] for s in shape)
+            if tuple(t.shape) != want or t.dtype != torch.bfloat16 or not t.is_cuda:
+                raise ValueError(f"{k}: need CUDA bf16 {want}, got {t.dtype} {tuple(t.shape)}")
+            if not t.is_contiguous():
+                raise ValueError(f"{k} must be contiguous")
+        bias = weights.get("router_bias")
+        if bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (n_experts,)
+                                 or not bias.is_cuda):
+            raise ValueError("router_bias: need CUDA fp32 [N]")
+        self.cfg = LmoeConfig(d, latent, n_experts, top_k, expert_hidden, shared_hidden,
+                              {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4}[expert_format], 0,
+                              max_tokens)
+        w = LmoeWeights(weights["w_router"].data_ptr(),
+                        bias.data_ptr() if bias is not None else None,
+                        weights["w_dn"].data_ptr(), weights["w1"].data_ptr(),
+                        weights["w2"].data_ptr(), weights["w_upl"].data_ptr(),
+                        weights["w_s1"].data_ptr(), weights["w_s2"].data_ptr(),
+                        float(act_gscales[0]), float(act_gscales[1]))
+        self.device = weights["w1"].device
+        h = c_void_p()
+        with torch.cuda.device(self.device):
+            check(self.lib.lmoe_create(byref(self.cfg), byref(w), byref(h)), "lmoe_create")
+        self.h = h
+        self.last_T = 0
+
+    # -- forward ----------------------------------------------------------
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """lmoe_forward: x [T][d] CUDA bf16 -> y [T][d] CUDA bf16 (async)."""
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != self.cfg.d or not x.is_cuda:
+            raise ValueError("x: need CUDA bf16 [T][d]")
+        x = x.contiguous()
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.cfg.d), dtype=torch.bfloat16, device=x.device)
+        check(self.lib.lmoe_forward(self.h, c_void_p(x.data_ptr()), T, c_void_p(out.data_ptr()),
+                                    _stream_ptr(stream)), "lmoe_forward")
+        self.last_T = T
+        return out
+
+    __call__ = forward
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor,
+                     stream: Optional[torch.cuda.Stream] = None) -> None:
+        """lmoe_forward_host: host (pinned) bf16 buffers in and out, synchronous."""
+        if x_host.is_cuda or y_host.is_cuda or x_host.dtype != torch.bfloat16 \
+                or y_host.dtype != torch.bfloat16 or x_host.shape != y_host.shape:
+            raise ValueError("host bf16 [T][d] buffers required")
+        T = x_host.shape[0]
+        check(self.lib.lmoe_forward_host(self.h, c_void_p(x_host.data_ptr()), T,
+                                         c_void_p(y_host.data_ptr()), _stream_ptr(stream)),
+              "lmoe_forward_host")
+        self.last_T = T
+
+    def sync_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
+        return self.lib.lmoe_sync_status(self.h, _stream_ptr(stream))
+
+    def launches_per_forward(self) -> int:
+        return self.lib.lmoe_launches_per_forward(self.h)
+
+    # -- debug readout ----------------------------------------------------
+    def debug(self, what: str) -> torch.Tensor:
+        """lmoe_get_debug: a host copy of an intermediate of the last forward."""
+        c, T = self.cfg, self.last_T
+        spec = {
+            "topk_idx": (torch.int32, (T, c.top_k)), "topk_w": (torch.float32, (T, c.top_k)),
+            "counts": (torch.int32, (c.n_experts,)), "offsets": (torch.int32, (c.n_experts + 1,)),
+            "perm": (torch.int32, (T * c.top_k,)), "inv": (torch.int32, (T, c.top_k)),
+            "logits": (torch.float32, (T, c.n_experts)), "u": (torch.bfloat16, (T, c.latent)),
+            "v": (torch.bfloat16, (T, c.latent)), "hs": (torch.bfloat16, (T, c.shared_hidden)),
+        }[what]
+        out = torch.empty(spec[1], dtype=spec[0])
+        check(self.lib.lmoe_get_debug(self.h, DBG[what], c_void_p(out.data_ptr()),
+                                      out.numel() * out.element_size()), f"debug {what}")
+        return out
+
+    # -- profiling --------------------------------------------------------
+    def profile_enable(self, on: bool = True) -> None:
+        check(self.lib.lmoe_profile_enable(self.h, int(on)), "profile_enable")
+
+    def profile_read(self, reset: bool = True):
+        n = 16
+        names = (c_char_p * n)()
+        ms = (c_double * n)()
+        cnt = (c_int64 * n)()
+        k = self.lib.lmoe_profile_read(self.h, names, ms, cnt, n, int(reset))
+        if k < 0:
+            raise LmoeError(k, "profile_read")
+        return [(names[i].decode(), ms[i], cnt[i]) for i in range(k)]
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            self.lib.lmoe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def lmoe_route(logits: torch.Tensor, bias: Optional[torch.Tensor], K: int,
+               stream: Optional[torch.cuda.Stream] = None) -> Dict[str, torch.Tensor]:
+    """lmoe_route: routing and per-expert segments from fp32 logits [T][N]."""
+    lib = _lib.load()
+    T, N = logits.shape
+    dev = logits.device
+    logits = logits.contiguous()
+    out = {
+        "topk_idx": torch.empty((T, K), dtype=torch.int32, device=dev),
+        "topk_w": torch.empty((T, K), dtype=torch.float32, device=dev),
+        "counts": torch.empty((N,), dtype=torch.int32, device=dev),
+        "offsets": torch.empty((N + 1,), dtype=torch.int32, device=dev),
+        "perm": torch.empty((T * K,), dtype=torch.int32, device=dev),
+        "inv": torch.empty((T, K), dtype=torch.int32, device=dev),
+    }
+    ws_bytes = lib.lmoe_route_workspace_size(T, N)
+    ws = torch.empty((max(ws_bytes, 256),), dtype=torch.uint8, device=dev)
+    p = lambda t: c_void_p(t.data_ptr()) if t is not None else None  # noqa: E731
+    check(lib.lmoe_route(p(logits), p(bias), T, N, K, p(out["topk_idx"]), p(out["topk_w"]),
+                         p(out["counts"]), p(out["offsets"]), p(out["perm"]), p(out["inv"]),
+                         p(ws), ws.numel(), _stream_ptr(stream)), "lmoe_route")
+    out["_workspace"] = ws
+    return out
+
+
+def lmoe_check_bounded_wait(limit_ns: int) -> int:
+    """lmoe_check_bounded_wait: the status of a wait that nothing completes."""
+    return _lib.load().lmoe_check_bounded_wait(int(limit_ns))

@@ -158,7 +158,8 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     u, W1[e], W2[e] and the expert hidden activation are replaced by their
     NVFP4 quantise-dequantise images (oracle.nvfp4).
 
-    Returns a dict with S, w, gap, s, u, v, r, sh, y (float64).
+    Returns a dict with S, w, gap, s, z, u, v, r, hs, sh, y (float64); hs is
+    the shared expert's hidden activation sqrelu(W_s1 x).
     """
     x = np.atleast_2d(np.asarray(x, dtype=np.float64))
     T = x.shape[0]
@@ -194,9 +195,10 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     # 5: one projection back to width d
     r = v @ W_upl.T
     # 6: shared expert at width d
-    sh = sqrelu(x @ W_s1.T) @ W_s2.T
+    hs = sqrelu(x @ W_s1.T)
+    sh = hs @ W_s2.T
     return {"S": S, "w": w, "gap": gap, "s": s, "z": z, "u": u, "v": v,
-            "r": r, "sh": sh, "y": r + sh}
+            "r": r, "hs": hs, "sh": sh, "y": r + sh}
 
 
 def token_forward(x_t: np.ndarray, S_t: np.ndarray, s_t: np.ndarray,

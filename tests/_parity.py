@@ -1,0 +1,126 @@
+"""Helpers of the GPU parity tests: build a layer from a seeded workload, run
+the oracle on a subset of its tokens, and compare.
+
+Tolerances (the layer's stated bar): routing indices equal for every token
+whose oracle gap between the K-th and (K+1)-th key exceeds 1e-3; outputs
+within max|err| <= 2e-2 * RMS (BF16 experts) of the oracle's, per compared
+tensor (u, hs, v, y), over the compared tokens.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import lmoe as O
+
+GAP = 1e-3
+TOL_BF16 = 2e-2
+W_TOL = 1e-5
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None):
+    """Seeded weights and x on the device, and the layer built from them."""
+    from lmoe_synth import make_weights, make_x
+    from latent_space_mixture_b200 import LatentMoE
+    w, gen = make_weights(cfg, device=device)
+    x = make_x(cfg, gen, T=T, device=device)
+    if overrides:
+        for k, fn in overrides.items():
+            w[k] = fn(w[k])
+    layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs,
+                      max_tokens or x.shape[0], w)
+    return w, x, layer
+
+
+def oracle_tokens(w, x_rows: torch.Tensor, K: int, quant=None):
+    """The oracle on the given token rows, expert weights fetched per expert."""
+    cache = {}
+
+    def fetch(name, e):
+        key = (name, e)
+        if key not in cache:
+            cache[key] = to64(w[name][e])
+        return cache[key]
+
+    out = O.layer_forward(to64(x_rows), to64(w["w_router"]), to64(w["router_bias"]),
+                          to64(w["w_dn"]), lambda e: fetch("w1", e), lambda e: fetch("w2", e),
+                          to64(w["w_upl"]), to64(w["w_s1"]), to64(w["w_s2"]), K, quant=quant)
+    out["_fetch"] = fetch
+    return out
+
+
+def max_rel(a: np.ndarray, b: np.ndarray) -> float:
+    """max|a - b| / RMS(b)."""
+    rms = float(np.sqrt(np.mean(b * b)))
+    return float(np.max(np.abs(a - b))) / (rms if rms > 0 else 1.0)
+
+
+def compare_layer(layer, w, x, y, tokens, K, tol=TOL_BF16, quant=None):
+    """Compare the last forward of `layer` (x -> y) with the oracle on `tokens`.
+
+    Returns a dict of measured errors; asserts the bar.  Near-tie tokens whose
+    GPU set differs from the oracle's must hold a valid top-K set under the
+    oracle's keys (within GAP), and their outputs are compared with the
+    oracle's for that set.
+    """
+    tokens = np.asarray(tokens)
+    o = oracle_tokens(w, x[tokens], K, quant=quant)
+    gi = layer.debug("topk_idx").numpy()[tokens]
+    gw = layer.debug("topk_w").numpy()[tokens]
+    key = o["s"] + to64(w["router_bias"])[None, :]
+    v_ref = o["v"].copy()
+    y_ref = o["y"].copy()
+    n_tie_diff = 0
+    for i in range(len(tokens)):
+        same = sorted(gi[i].tolist()) == sorted(o["S"][i].tolist())
+        if o["gap"][i] > GAP:
+            assert same, f"token {tokens[i]}: routing {sorted(gi[i])} != {sorted(o['S'][i])}"
+        if same:
+            ref_w = dict(zip(o["S"][i].tolist(), o["w"][i].tolist()))
+            for e, wv in zip(gi[i].tolist(), gw[i].tolist()):
+                assert abs(wv - ref_w[e]) <= W_TOL, (tokens[i], e, wv, ref_w[e])
+        else:
+            n_tie_diff += 1
+            assert O.is_valid_topk(key[i], gi[i], GAP), f"token {tokens[i]}: invalid top-K"
+            tf = O.token_forward(to64(x[tokens[i]]), gi[i], o["s"][i], to64(w["w_dn"]),
+                                 lambda e: o["_fetch"]("w1", e), lambda e: o["_fetch"]("w2", e),
+                                 to64(w["w_upl"]), quant=quant)
+            v_ref[i] = tf["v"]
+            y_ref[i] = tf["r"] + o["sh"][i]
+    errs = {
+        "u": max_rel(to64(layer.debug("u"))[tokens], o["u"]),
+        "hs": max_rel(to64(layer.debug("hs"))[tokens], o["hs"]),
+        "v": max_rel(to64(layer.debug("v"))[tokens], v_ref),
+        "y": max_rel(to64(y)[tokens], y_ref),
+        "near_tie_sets_differing": n_tie_diff,
+    }
+    for k in ("u", "hs", "v", "y"):
+        assert errs[k] <= tol, f"{k}: max|err|/RMS = {errs[k]:.3g} > {tol}"
+    return errs
+
+
+def check_segments_valid(layer, T, N, K):
+    """Properties of the per-expert segments that hold at any size."""
+    idx = layer.debug("topk_idx").numpy().astype(np.int64)
+    counts = layer.debug("counts").numpy().astype(np.int64)
+    offsets = layer.debug("offsets").numpy().astype(np.int64)
+    perm = layer.debug("perm").numpy().astype(np.int64)
+    inv = layer.debug("inv").numpy().astype(np.int64)
+    assert idx.min() >= 0 and idx.max() < N
+    assert np.all(np.sort(idx, axis=1)[:, 1:] != np.sort(idx, axis=1)[:, :-1]), "duplicate expert"
+    assert np.array_equal(counts, np.bincount(idx.reshape(-1), minlength=N))
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts)
+    flat = idx.reshape(-1)
+    assert np.array_equal(np.sort(perm), np.arange(T * K))
+    assert np.array_equal(perm[inv.reshape(-1)], np.arange(T * K))
+    # rows of each expert: that expert, ascending tokens
+    seg_e = np.repeat(np.arange(N), counts)
+    assert np.array_equal(flat[perm], seg_e)
+    tok = perm // K
+    same = seg_e[1:] == seg_e[:-1]
+    assert np.all(tok[1:][same] > tok[:-1][same])
+    return counts
