@@ -217,8 +217,8 @@ def oracle_rate(cfg, w, x, seconds: float, seed: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="super_decode", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="lmoe", choices=["lmoe", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -60,6 +60,10 @@ CONFIGS: Dict[str, LayerConfig] = {
     # Ultra dims
     "ultra": LayerConfig("ultra", 4096, 8192, 2048, 512, 22, 5120, 10240,
                          0.015, "zero", 3),
+    # Super dims with 64 experts and 32 tokens (11 rows per expert, as in the
+    # decode batch): a small case of the same kernels for profiler captures
+    "super_decode_n64": LayerConfig("super_decode_n64", 32, 4096, 1024, 64, 22, 2688,
+                                    5376, 0.02, "zero", 5),
     # Super dims prefill with NVFP4 experts, Zipf(1.1) router bias
     "super_prefill_nvfp4": LayerConfig("super_prefill_nvfp4", 8192, 4096, 1024,
                                        512, 22, 2688, 5376, 0.02, "zipf", 4,
