@@ -6,13 +6,17 @@ Tolerances:
     and (K+1)-th key exceeds 1e-3 (the stated bar);
   * the layer output y within max|err| <= 2e-2 * RMS(y) over the compared
     tokens (the stated bar for BF16 experts);
-  * intermediates (u, hs, v) and single-branch outputs elementwise within
-    |err| <= 2^-7 |ref| + 1e-2 RMS(ref).  Each is stored in bf16 (relative
-    rounding <= 2^-9) and is computed from bf16 operands (<= 2^-9 each), so
-    2^-7 covers up to four such roundings of the element itself; 1e-2 RMS
-    absorbs the averaged rounding of upstream bf16 intermediates.  A plain
-    max|err|/RMS bar does not fit heavy-tailed tensors: hs = sqrelu(.) has
-    max/RMS ~ 13, so its bf16 storage alone costs ~ 0.025 RMS.
+  * intermediates (u, hs, v) and single-branch outputs, two derived bars:
+      - RMS(err) <= 1e-2 RMS(ref): each value is stored in bf16 (relative
+        rounding <= 2^-9) and carries the independent roundings of a few bf16
+        upstream operands (x, u, H, O, v), so its relative RMS error is a few
+        times 2^-9 (~0.4% measured for v); 1e-2 is ~5 x 2^-9;
+      - elementwise |err| <= 2^-7 |ref| + 3e-2 RMS(ref): 2^-7 covers the
+        element's own and its operands' roundings, 3e-2 RMS the tail of the
+        accumulated upstream noise (max over ~1e4..1e5 elements of a noise
+        with sigma ~ 2 x 2^-9 RMS is ~ 4.5 sigma ~ 1.8e-2 RMS).
+    A plain max|err|/RMS bar does not fit heavy-tailed tensors: hs = sqrelu(.)
+    has max/RMS ~ 13, so its bf16 storage alone costs ~ 0.025 RMS.
 """
 from __future__ import annotations
 
@@ -24,7 +28,8 @@ from oracle import lmoe as O
 GAP = 1e-3
 TOL_BF16 = 2e-2
 REL_ELEM = 2.0 ** -7
-ABS_RMS = 1e-2
+ABS_RMS = 3e-2
+REL_RMS = 1e-2
 W_TOL = 1e-5
 
 
@@ -66,12 +71,21 @@ def max_rel(a: np.ndarray, b: np.ndarray) -> float:
     return float(np.max(np.abs(a - b))) / (rms if rms > 0 else 1.0)
 
 
-def elem_ok(a: np.ndarray, ref: np.ndarray, rel=REL_ELEM, abs_rms=ABS_RMS):
-    """Elementwise bf16 error model; returns (ok, worst ratio err / bound)."""
+def rms_rel(a: np.ndarray, ref: np.ndarray) -> float:
+    """RMS(a - ref) / RMS(ref)."""
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    return float(np.sqrt(np.mean((a - ref) ** 2))) / (rms if rms > 0 else 1.0)
+
+
+def elem_ok(a: np.ndarray, ref: np.ndarray, rel=REL_ELEM, abs_rms=ABS_RMS, rel_rms=REL_RMS):
+    """The bf16 error model of an intermediate: relative RMS error and the
+    elementwise tail bound.  Returns (ok, worst elementwise err / bound,
+    relative RMS error)."""
     rms = float(np.sqrt(np.mean(ref * ref)))
     bound = rel * np.abs(ref) + abs_rms * rms
     ratio = float(np.max(np.abs(a - ref) / np.maximum(bound, 1e-300)))
-    return ratio <= 1.0, ratio
+    rr = rms_rel(a, ref)
+    return ratio <= 1.0 and rr <= rel_rms, ratio, rr
 
 
 def compare_layer(layer, w, x, y, tokens, K, tol=TOL_BF16, quant=None, elem_rel=REL_ELEM):
@@ -112,10 +126,11 @@ def compare_layer(layer, w, x, y, tokens, K, tol=TOL_BF16, quant=None, elem_rel=
     errs = {"y_maxerr_over_rms": max_rel(to64(y)[tokens], y_ref),
             "near_tie_sets_differing": n_tie_diff}
     for k in ("u", "hs", "v"):
-        ok, ratio = elem_ok(got[k], ref[k], rel=elem_rel)
+        ok, ratio, rr = elem_ok(got[k], ref[k], rel=elem_rel)
         errs[k + "_maxerr_over_rms"] = max_rel(got[k], ref[k])
         errs[k + "_err_over_bound"] = ratio
-        assert ok, f"{k}: elementwise error {ratio:.3g} x the bf16 bound"
+        errs[k + "_rms_rel"] = rr
+        assert ok, f"{k}: elementwise error {ratio:.3g} x bound, RMS rel error {rr:.3g}"
     assert errs["y_maxerr_over_rms"] <= tol, \
         f"y: max|err|/RMS = {errs['y_maxerr_over_rms']:.3g} > {tol}"
     return errs

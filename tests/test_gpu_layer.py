@@ -90,8 +90,8 @@ def test_routed_branch_alone():
     y = layer.forward(x)
     o = oracle_tokens(w, x, cfg.K)
     assert np.all(o["sh"] == 0)
-    ok, ratio = elem_ok(to64(y), o["r"])
-    assert ok, ratio
+    ok, ratio, rr = elem_ok(to64(y), o["r"])
+    assert ok, (ratio, rr)
     layer.close()
 
 
@@ -103,8 +103,8 @@ def test_shared_branch_alone():
     o = oracle_tokens(w, x, cfg.K)
     assert np.all(o["r"] == 0)
     assert np.all(to64(layer.debug("v")) == 0)
-    ok, ratio = elem_ok(to64(y), o["sh"])
-    assert ok, ratio
+    ok, ratio, rr = elem_ok(to64(y), o["sh"])
+    assert ok, (ratio, rr)
     assert max_rel(to64(y), o["sh"]) <= TOL_BF16
     layer.close()
 
