@@ -156,6 +156,27 @@ int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int
                int32_t* perm, int32_t* inv, void* workspace, size_t workspace_bytes,
                void* stream);
 
+/* Allocation-free variant of lmoe_route (no counterpart on the pages: it is a
+ * deployment convenience).  For callers that cannot give this library device
+ * memory -- e.g. a serving engine that reserves all of HBM for its own pool at
+ * start-up, or a host path where cudaMalloc (which may synchronize the device)
+ * is not allowed -- the scratch lives in a static device array of about 2 MiB
+ * that every GPU loading the library holds until the process exits.  Same
+ * arguments and outputs as lmoe_route minus the workspace; it allocates
+ * nothing (no cudaMalloc/cudaFree, no allocating library call).
+ * Limits: T <= LMOE_NOALLOC_MAX_TOKENS, T*K <= LMOE_NOALLOC_MAX_ROUTED,
+ * N <= 1024; larger sizes return LMOE_ERR_UNSUPPORTED.
+ * The first call on a device looks up the array's device address once (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array, so calls whose work overlaps on the GPU
+ * (other streams, other host threads) race: serialize them.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+#define LMOE_NOALLOC_MAX_TOKENS 8192
+#define LMOE_NOALLOC_MAX_ROUTED 262144
+int lmoe_route_noalloc(const float* logits, const float* bias, int64_t T, int32_t N, int32_t K,
+                       int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                       int32_t* perm, int32_t* inv, void* stream);
+
 /* Runs a one-CTA kernel that waits on an mbarrier nothing arrives on, with a
  * wait limit of limit_ns nanoseconds (1e3..1e10), and returns the status the
  * host reads afterwards: LMOE_ERR_TIMEOUT when the bounded wait gave up as

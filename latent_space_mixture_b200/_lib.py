@@ -52,6 +52,8 @@ SIGNATURES = {
     "lmoe_route": (c_int, [c_void_p, c_void_p, c_int64, c_int32, c_int32, c_void_p, c_void_p,
                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                            c_void_p]),
+    "lmoe_route_noalloc": (c_int, [c_void_p, c_void_p, c_int64, c_int32, c_int32, c_void_p,
+                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "lmoe_check_bounded_wait": (c_int, [c_int64]),
     "lmoe_destroy": (None, [c_void_p]),
     "lmoe_strerror": (c_char_p, [c_int]),

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "liblmoe.so")
-SOURCES = ["lmoe_abi.cu", "routing.cu"]
+SOURCES = ["lmoe_abi.cu", "routing.cu", "route_noalloc.cu"]
 HEADERS = ["ptx.cuh", "gemm_tc.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
