@@ -335,7 +335,7 @@ def main():
         cpu = {"value": round(rate, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} of the {T} tokens of this batch, in batches of 8, {el:.1f} s"}
 
-    launches = layer.launches_per_forward() * args.steps
+    launches = layer.launches_per_forward(T) * args.steps
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

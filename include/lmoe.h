@@ -129,9 +129,9 @@ int lmoe_sync_status(lmoe_handle* h, void* stream);
 #define LMOE_DBG_HS 10
 int lmoe_get_debug(lmoe_handle* h, int what, void* dst_host, size_t bytes);
 
-/* Kernel launches one forward of T tokens issues (the same count for every
- * T > 0 of a handle), or a negative error code. */
-int lmoe_launches_per_forward(const lmoe_handle* h);
+/* Kernel launches one lmoe_forward of T tokens issues (10, plus one split-K
+ * reduction per dense GEMM when T is small), or a negative error code. */
+int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T);
 
 /* Per-kernel timing: when enabled, every forward records CUDA events around
  * each of its kernels on the forward's stream and accumulates their elapsed

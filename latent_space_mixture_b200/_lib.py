@@ -44,7 +44,7 @@ SIGNATURES = {
     "lmoe_forward_host": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
     "lmoe_sync_status": (c_int, [c_void_p, c_void_p]),
     "lmoe_get_debug": (c_int, [c_void_p, c_int, c_void_p, c_size_t]),
-    "lmoe_launches_per_forward": (c_int, [c_void_p]),
+    "lmoe_launches_per_forward": (c_int, [c_void_p, c_int64]),
     "lmoe_profile_enable": (c_int, [c_void_p, c_int]),
     "lmoe_profile_read": (c_int, [c_void_p, POINTER(c_char_p), POINTER(c_double),
                                   POINTER(c_int64), c_int, c_int]),

@@ -31,7 +31,8 @@ constexpr int GEMM_BK = 64;           // K elements per pipeline stage (128 B)
 constexpr int GEMM_THREADS = 192;
 constexpr int GEMM_EPI_WARPS = 4;
 constexpr int GEMM_STG_LD = 36;       // fp32 staging pitch (32 + 4)
-constexpr int GEMM_BROWS = 16;        // rows per B TMA box
+constexpr int GEMM_BROWS = 16;        // rows per small B TMA box (ragged tails)
+constexpr int GEMM_BROWS_BIG = 64;    // rows per large B TMA box (full row groups)
 
 // Where the tiles of one GEMM come from.
 struct TileSource {
@@ -43,21 +44,29 @@ struct TileSource {
   int a_rows_per_expert;   // rows of A per expert (0 when dense)
   int m_valid;             // valid features per expert (multiple of 8)
   int kblocks;             // K / 64
+  int ksplit;              // dense only: K slices (1 = none); each slice writes
+  float* part;             //   fp32 partials part[slice][row][feature]
+  int a_stream_once;       // 1: each A tile is read by one tile only (L2 evict-first)
 };
 
 struct TileInfo {
-  int e, fb, row0, nrows, a_row;
+  int e, fb, row0, nrows, a_row, ks, kb0, kb1;
 };
 
 __device__ __forceinline__ int gemm_num_tiles(const TileSource& s, int BN) {
   const int nb = s.dense ? (s.T + BN - 1) / BN : *s.nblocks;
-  return nb * s.FB;
+  return nb * s.FB * s.ksplit;
 }
 
+// tile -> (token block, K slice, feature block), feature block fastest
 __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int tile) {
   TileInfo t;
-  const int tb = tile / s.FB;
-  t.fb = tile - tb * s.FB;
+  const int tk = tile / s.FB;
+  t.fb = tile - tk * s.FB;
+  const int tb = tk / s.ksplit;
+  t.ks = tk - tb * s.ksplit;
+  t.kb0 = t.ks * s.kblocks / s.ksplit;
+  t.kb1 = (t.ks + 1) * s.kblocks / s.ksplit;
   if (s.dense) {
     t.e = 0;
     t.row0 = tb * BN;
@@ -89,7 +98,8 @@ struct GemmLayout {
 template <int BN, int STAGES, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const TileSource src, const Epi epi, int* err, unsigned long long limit_ns) {
+          const __grid_constant__ CUtensorMap tmB64, const TileSource src, const Epi epi, int* err,
+          unsigned long long limit_ns) {
   using L = GemmLayout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -124,6 +134,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB64);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::TMEM_COLS);
@@ -138,16 +149,21 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_a = policy_evict_first();   // weights: streamed
+      // weights read once per launch are streamed past L2; weights that
+      // several token blocks share are left to the default policy
+      const uint64_t pol_a = src.a_stream_once ? policy_evict_first() : policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const TileInfo t = gemm_tile(src, BN, tile);
-        const int nload = (t.nrows + GEMM_BROWS - 1) / GEMM_BROWS;
-        const uint32_t tx = L::A_BYTES + nload * GEMM_BROWS * GEMM_BK * 2;
-        for (int kb = 0; kb < src.kblocks; ++kb) {
+        // B rows: 64-row boxes while 64 rows remain, then 16-row boxes
+        const int nbig = t.nrows / GEMM_BROWS_BIG;
+        const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
+        const uint32_t tx =
+            L::A_BYTES + (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_BK * 2;
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err, limit_ns)) {
             ok = false;
             break;
@@ -156,9 +172,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, kb * GEMM_BK, t.a_row, &full[stage],
                            pol_a);
           uint8_t* b_dst = sB + stage * L::B_BYTES;
-          for (int j = 0; j < nload; ++j)
-            tma_load_2d(b_dst + j * GEMM_BROWS * GEMM_BK * 2, &tmB, kb * GEMM_BK,
-                        t.row0 + j * GEMM_BROWS, &full[stage]);
+          for (int j = 0; j < nbig; ++j)
+            tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_BK * 2, &tmB64, kb * GEMM_BK,
+                        t.row0 + j * GEMM_BROWS_BIG, &full[stage]);
+          for (int j = 0; j < nsmall; ++j) {
+            const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
+            tma_load_2d(b_dst + r * GEMM_BK * 2, &tmB, kb * GEMM_BK, t.row0 + r, &full[stage]);
+          }
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -198,7 +218,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         const uint32_t idesc = idesc_bf16(GEMM_BM, n_mma);
-        for (int kb = 0; kb < src.kblocks; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns)) {
             ok = false;
             break;
@@ -208,7 +228,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + stage * L::B_BYTES));
 #pragma unroll
           for (int k = 0; k < GEMM_BK / 16; ++k)   // +32 bytes per K=16 step
-            umma_bf16(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0);
+            umma_bf16(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
           umma_commit(&empty[stage]);
           issued_any = true;
           if (++stage == STAGES) {
@@ -261,8 +281,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           if (c0 + j < t.nrows && feat < src.m_valid) {
             const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
             const float4 lo = p[0], hi = p[1];
-            const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-            epi.store8(t.e, static_cast<long>(t.row0 + c0 + j), feat, v);
+            const long row = static_cast<long>(t.row0 + c0 + j);
+            if (src.ksplit > 1) {
+              float4* dst = reinterpret_cast<float4*>(
+                  src.part + (static_cast<long>(t.ks) * src.T + row) * src.m_valid + feat);
+              dst[0] = lo;
+              dst[1] = hi;
+            } else {
+              const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+              epi.store8(t.e, row, feat, v);
+            }
           }
         }
         __syncwarp();
@@ -280,6 +308,27 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, L::TMEM_COLS);
+}
+
+// Sum of the K-slice partials in slice order (deterministic), then the real
+// epilogue: thread per 8 consecutive features of one row.
+template <class Epi>
+__global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ part, int ksplit,
+                                                       int T, int F, const Epi epi) {
+  const long g = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int f8 = F / 8;
+  const long row = g / f8;
+  if (row >= T) return;
+  const int feat = static_cast<int>(g - row * f8) * 8;
+  float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int s = 0; s < ksplit; ++s) {
+    const float4* p = reinterpret_cast<const float4*>(part + (static_cast<long>(s) * T + row) * F +
+                                                      feat);
+    const float4 a = p[0], b = p[1];
+    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  }
+  epi.store8(0, row, feat, v);
 }
 
 // ---------------------------------------------------------------------------

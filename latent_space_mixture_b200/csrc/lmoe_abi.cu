@@ -102,25 +102,39 @@ cudaError_t set_gemm_smem() {
                               cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
 }
 
+// B operand: the same matrix under two tensor maps (16-row and 64-row boxes)
+struct BMaps {
+  CUtensorMap b16, b64;
+};
+
 template <int BN, class Epi>
-cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const TileSource& src,
+cudaError_t launch_gemm(const CUtensorMap& A, const BMaps& B, const TileSource& src,
                         const Epi& epi, int grid, int* err, unsigned long long limit,
                         cudaStream_t st) {
   using L = GemmLayout<BN, Stages<BN>::value>;
-  k_gemm_tc<BN, Stages<BN>::value, Epi><<<grid, GEMM_THREADS, L::SMEM_BYTES, st>>>(A, B, src, epi,
-                                                                                  err, limit);
+  k_gemm_tc<BN, Stages<BN>::value, Epi>
+      <<<grid, GEMM_THREADS, L::SMEM_BYTES, st>>>(A, B.b16, B.b64, src, epi, err, limit);
   return cudaGetLastError();
 }
 
 template <class Epi>
-cudaError_t launch_gemm_bn(int bn, const CUtensorMap& A, const CUtensorMap& B,
-                           const TileSource& src, const Epi& epi, int grid, int* err,
-                           unsigned long long limit, cudaStream_t st) {
+cudaError_t launch_gemm_bn(int bn, const CUtensorMap& A, const BMaps& B, const TileSource& src,
+                           const Epi& epi, int grid, int* err, unsigned long long limit,
+                           cudaStream_t st) {
   switch (bn) {
     case 256: return launch_gemm<256>(A, B, src, epi, grid, err, limit, st);
     case 128: return launch_gemm<128>(A, B, src, epi, grid, err, limit, st);
     default: return launch_gemm<32>(A, B, src, epi, grid, err, limit, st);
   }
+}
+
+template <class Epi>
+cudaError_t launch_reduce(const float* part, int ksplit, int T, int F, const Epi& epi,
+                          cudaStream_t st) {
+  const long threads = static_cast<long>(T) * (F / 8);
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  k_splitk_reduce<Epi><<<blocks, 256, 0, st>>>(part, ksplit, T, F, epi);
+  return cudaGetLastError();
 }
 
 template <class Epi>
@@ -185,12 +199,32 @@ static size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255);
 
 using namespace lmoe;
 
-// names of the kernels one forward launches, in launch order
+// names of the kernels one forward launches, in launch order (the two
+// split-K reductions run only for small token counts)
 static const char* const kKernelNames[] = {
     "xgemm(router|W_dn|W_s1)", "route(sigmoid+bias+topK)", "hist", "scan", "scatter",
     "gather(u->expert order)", "grouped_gemm1(W1,sqrelu)", "grouped_gemm2(W2,*w)",
-    "combine", "ygemm([W_upl|W_s2])"};
-static constexpr int kNumKernels = 10;
+    "combine", "ygemm([W_upl|W_s2])", "xgemm split-K reduce", "ygemm split-K reduce"};
+static constexpr int kNumKernels = 12;
+
+// Dense-GEMM plan for T tokens: token-block width and number of K slices.
+// Enough tiles to fill the GPU first by narrower token blocks (while one
+// block still spans 128 rows), else by splitting K, so that every weight byte
+// is read once and no token block is re-read more than necessary.
+struct DensePlan {
+  int bn, ksplit;
+};
+static DensePlan plan_dense(int64_t T, int fb, int kblocks, int sms) {
+  for (int bn : {256, 128})
+    if (((T + bn - 1) / bn) * fb >= sms) return {bn, 1};
+  const int bn = T <= 32 ? 32 : (T <= 128 ? 128 : 256);
+  const int64_t tiles = ((T + bn - 1) / bn) * fb;
+  int64_t ks = sms / tiles;   // one wave: tiles * ks <= sms
+  if (ks > 8) ks = 8;
+  if (ks > kblocks / 4) ks = kblocks / 4;
+  if (ks < 1) ks = 1;
+  return {bn, static_cast<int>(ks)};
+}
 
 struct lmoe_handle {
   lmoe_config cfg;
@@ -221,9 +255,11 @@ struct lmoe_handle {
   bf16* vh = nullptr;      // [max_tokens][l+h_s]: v | hs
   bf16* x_dev = nullptr;   // staging for lmoe_forward_host
   bf16* y_dev = nullptr;
+  float* part = nullptr;   // split-K partials of the dense GEMMs
   int* err = nullptr;
   std::vector<void*> allocs;
-  CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy, tm_uperm, tm_H, tm_vh;
+  CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
+  BMaps tm_uperm, tm_H, tm_vh;
   int64_t last_T = 0;
   unsigned long long wait_limit_ns = 2000000000ull;
   // profiling
@@ -278,14 +314,6 @@ static int grouped_bn(const lmoe_config& c, int64_t T) {
   return 256;
 }
 
-// dense-GEMM token-block width: the widest whose tile count fills the GPU
-static int dense_bn(int64_t T, int fb, int sms) {
-  const int cand[3] = {256, 128, 32};
-  for (int i = 0; i < 3; ++i)
-    if (((T + cand[i] - 1) / cand[i]) * fb >= sms) return cand[i];
-  return 32;
-}
-
 extern "C" {
 
 const char* lmoe_strerror(int code) {
@@ -327,6 +355,20 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   const int64_t rows_b = rows < 256 ? 256 : rows;
   const int64_t Tm_b = Tm < 256 ? 256 : Tm;
   const int64_t d_a = d < GEMM_BM ? GEMM_BM : d;
+  // largest split-K partials buffer over the token counts this handle accepts
+  int64_t part_floats = 0;
+  {
+    const int fbx = static_cast<int>((N + l + hs + 127) / 128);
+    const int fby = static_cast<int>((d + 127) / 128);
+    const int64_t tmax = Tm < 256LL * h->sms ? Tm : 256LL * h->sms;
+    for (int64_t T = 1; T <= tmax; ++T) {
+      const DensePlan px = plan_dense(T, fbx, static_cast<int>(d / 64), h->sms);
+      const DensePlan py = plan_dense(T, fby, static_cast<int>((l + hs) / 64), h->sms);
+      if (px.ksplit > 1 && px.ksplit * T * (N + l + hs) > part_floats)
+        part_floats = px.ksplit * T * (N + l + hs);
+      if (py.ksplit > 1 && py.ksplit * T * d > part_floats) part_floats = py.ksplit * T * d;
+    }
+  }
   const int64_t max_blocks = rows / 32 + N + 1;
   struct Req {
     void** p;
@@ -355,6 +397,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->vh, size_t(Tm_b * (l + hs) * 2)},
       {(void**)&h->x_dev, size_t(Tm_b * d * 2)},
       {(void**)&h->y_dev, size_t(Tm * d * 2)},
+      {(void**)&h->part, size_t(part_floats * 4)},
       {(void**)&h->err, size_t(4)},
   };
   for (auto& r : reqs) {
@@ -392,9 +435,12 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   ok &= make_map(&h->tm_w1, h->w1, N * hh, l, GEMM_BM);
   ok &= make_map(&h->tm_w2, h->w2, N * l, hh, GEMM_BM);
   ok &= make_map(&h->tm_wy, h->w_y, d_a, l + hs, GEMM_BM);
-  ok &= make_map(&h->tm_uperm, h->u_perm, rows_b, l, GEMM_BROWS);
-  ok &= make_map(&h->tm_H, h->H, rows_b, hh, GEMM_BROWS);
-  ok &= make_map(&h->tm_vh, h->vh, Tm_b, l + hs, GEMM_BROWS);
+  ok &= make_map(&h->tm_uperm.b16, h->u_perm, rows_b, l, GEMM_BROWS);
+  ok &= make_map(&h->tm_uperm.b64, h->u_perm, rows_b, l, GEMM_BROWS_BIG);
+  ok &= make_map(&h->tm_H.b16, h->H, rows_b, hh, GEMM_BROWS);
+  ok &= make_map(&h->tm_H.b64, h->H, rows_b, hh, GEMM_BROWS_BIG);
+  ok &= make_map(&h->tm_vh.b16, h->vh, Tm_b, l + hs, GEMM_BROWS);
+  ok &= make_map(&h->tm_vh.b64, h->vh, Tm_b, l + hs, GEMM_BROWS_BIG);
   ok &= set_smem_all<EpiX>() == cudaSuccess;
   ok &= set_smem_all<EpiH>() == cudaSuccess;
   ok &= set_smem_all<EpiO>() == cudaSuccess;
@@ -418,8 +464,15 @@ void lmoe_destroy(lmoe_handle* h) {
   delete h;
 }
 
-int lmoe_launches_per_forward(const lmoe_handle* h) {
-  return h ? kNumKernels : LMOE_ERR_INVALID_ARG;
+int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return 0;
+  const lmoe_config& c = h->cfg;
+  const DensePlan px = plan_dense(T, (c.n_experts + c.latent + c.shared_hidden + 127) / 128,
+                                  c.d / 64, h->sms);
+  const DensePlan py =
+      plan_dense(T, (c.d + 127) / 128, (c.latent + c.shared_hidden) / 64, h->sms);
+  return 10 + (px.ksplit > 1) + (py.ksplit > 1);
 }
 
 static int prof_begin(lmoe_handle* h, int kernel, cudaStream_t st) {
@@ -461,27 +514,33 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
             K = c.top_k;
   const int ldvh = l + hs;
   const unsigned long long lim = h->wait_limit_ns;
-  CUtensorMap tm_x;
-  if (T < GEMM_BROWS) {
-    // fewer rows than one TMA box: read x from the padded staging buffer
+  BMaps tm_x;
+  if (T < GEMM_BROWS_BIG) {
+    // fewer rows than one large TMA box: read x from the padded staging buffer
     if (x != h->x_dev &&
         cudaMemcpyAsync(h->x_dev, x, T * d * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return LMOE_ERR_CUDA;
-    if (!make_map(&tm_x, h->x_dev, GEMM_BROWS, d, GEMM_BROWS)) return LMOE_ERR_CUDA;
-  } else if (!make_map(&tm_x, x, T, d, GEMM_BROWS)) {
+    if (!make_map(&tm_x.b16, h->x_dev, GEMM_BROWS_BIG, d, GEMM_BROWS) ||
+        !make_map(&tm_x.b64, h->x_dev, GEMM_BROWS_BIG, d, GEMM_BROWS_BIG))
+      return LMOE_ERR_CUDA;
+  } else if (!make_map(&tm_x.b16, x, T, d, GEMM_BROWS) ||
+             !make_map(&tm_x.b64, x, T, d, GEMM_BROWS_BIG)) {
     return LMOE_ERR_CUDA;
   }
   h->last_T = T;
 
   // 1. [W_r; W_dn; W_s1] x: logits, u, shared hidden
   {
-    TileSource s{1, static_cast<int>(T), nullptr, nullptr, (N + l + hs + 127) / 128, 0,
-                 N + l + hs, static_cast<int>(d / 64)};
-    const int bn = dense_bn(T, s.FB, h->sms);
-    const int64_t tiles = ((T + bn - 1) / bn) * s.FB;
+    const int fb = (N + l + hs + 127) / 128;
+    const DensePlan p = plan_dense(T, fb, static_cast<int>(d / 64), h->sms);
+    TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, N + l + hs,
+                 static_cast<int>(d / 64), p.ksplit, h->part, T <= p.bn};
+    const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
     const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
     EpiX epi{h->logits, h->u, h->vh, N, l, ldvh};
-    LMOE_STEP(0, launch_gemm_bn(bn, h->tm_wx, tm_x, s, epi, grid, h->err, lim, st));
+    LMOE_STEP(0, launch_gemm_bn(p.bn, h->tm_wx, tm_x, s, epi, grid, h->err, lim, st));
+    if (p.ksplit > 1)
+      LMOE_STEP(10, launch_reduce(h->part, p.ksplit, static_cast<int>(T), N + l + hs, epi, st));
   }
   // 2-5. routing and segments
   const int gbn = grouped_bn(c, T);
@@ -495,13 +554,15 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   LMOE_STEP(5, launch_gather(h->u, h->perm, T * K, K, l, h->u_perm, st));
   // 7. H = sqrelu(W1[e] u)
   {
-    TileSource s{0, 0, h->blocks, h->nblocks, (hh + 127) / 128, hh, hh, l / 64};
+    TileSource s{0, 0, h->blocks, h->nblocks, (hh + 127) / 128, hh, hh, l / 64, 1, nullptr,
+                 gbn == 32};
     EpiH epi{h->H, hh};
     LMOE_STEP(6, launch_gemm_bn(gbn, h->tm_w1, h->tm_uperm, s, epi, h->sms, h->err, lim, st));
   }
   // 8. O = w * W2[e] H
   {
-    TileSource s{0, 0, h->blocks, h->nblocks, (l + 127) / 128, l, l, hh / 64};
+    TileSource s{0, 0, h->blocks, h->nblocks, (l + 127) / 128, l, l, hh / 64, 1, nullptr,
+                 gbn == 32};
     EpiO epi{h->O, h->wrow, l};
     LMOE_STEP(7, launch_gemm_bn(gbn, h->tm_w2, h->tm_H, s, epi, h->sms, h->err, lim, st));
   }
@@ -509,13 +570,17 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   LMOE_STEP(8, launch_combine(h->O, h->inv, T, K, l, h->vh, ldvh, st));
   // 10. y = [W_upl | W_s2] [v ; hs]
   {
-    TileSource s{1, static_cast<int>(T), nullptr, nullptr, static_cast<int>((d + 127) / 128), 0,
-                 static_cast<int>(d), ldvh / 64};
-    const int bn = dense_bn(T, s.FB, h->sms);
-    const int64_t tiles = ((T + bn - 1) / bn) * s.FB;
+    const int fb = static_cast<int>((d + 127) / 128);
+    const DensePlan p = plan_dense(T, fb, ldvh / 64, h->sms);
+    TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, static_cast<int>(d), ldvh / 64,
+                 p.ksplit, h->part, T <= p.bn};
+    const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
     const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
     EpiY epi{static_cast<bf16*>(y), static_cast<int>(d)};
-    LMOE_STEP(9, launch_gemm_bn(bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
+    LMOE_STEP(9, launch_gemm_bn(p.bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
+    if (p.ksplit > 1)
+      LMOE_STEP(11, launch_reduce(h->part, p.ksplit, static_cast<int>(T), static_cast<int>(d), epi,
+                                  st));
   }
   return LMOE_OK;
 }

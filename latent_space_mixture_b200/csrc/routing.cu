@@ -22,7 +22,29 @@ namespace lmoe {
 
 // ---------------------------------------------------------------------------
 // router: one warp per token
+//
+// Each candidate is packed into one 64-bit word: the key's bits mapped to an
+// unsigned order (high half) and 0xFFFFFFFF - expert (low half), so that the
+// largest word is the largest key and, among equal keys, the lowest expert
+// id.  A lane keeps the best word of its experts (e = lane + 32 i); each of
+// the K rounds takes the warp maximum, and only the winning lane rescans.
 
+__device__ __forceinline__ uint64_t pack_key(float key, int e) {
+  uint32_t b = __float_as_uint(key);
+  b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<uint64_t>(b) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = o > v ? o : v;
+  }
+  return v;
+}
+
+template <int NPL>   // upper bound of experts per lane (N <= 32 NPL)
 __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
                                                const float* __restrict__ bias, int64_t T, int N,
                                                int K, int32_t* __restrict__ topk_idx,
@@ -32,52 +54,42 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
   if (t >= T) return;
   const float* z = logits + t * N;
   const int npl = N >> 5;   // experts per lane: e = lane + 32 i
-  float key[32], s[32];
+  float zz[NPL], bb[NPL];
+  // all loads first (independent), then the arithmetic
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NPL; ++i) {
+    zz[i] = (i < npl) ? z[lane + 32 * i] : 0.0f;
+    bb[i] = (i < npl && bias) ? bias[lane + 32 * i] : 0.0f;
+  }
+  uint64_t cand[NPL];
+  uint64_t best = 0;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    cand[i] = 0;
     if (i < npl) {
-      const int e = lane + 32 * i;
-      const float sc = 1.0f / (1.0f + expf(-z[e]));
-      s[i] = sc;
-      key[i] = sc + (bias ? bias[e] : 0.0f);
-    } else {
-      s[i] = 0.0f;
-      key[i] = -INFINITY;
+      const float sc = 1.0f / (1.0f + expf(-zz[i]));
+      cand[i] = pack_key(sc + bb[i], lane + 32 * i);
+      best = cand[i] > best ? cand[i] : best;
     }
   }
-  uint32_t taken = 0;
   int my_e = 0;
-  float my_s = 0.0f;
   for (int k = 0; k < K; ++k) {
-    float bk = -INFINITY, bs = 0.0f;
-    int be = INT_MAX;
+    const uint64_t win = warp_max_u64(best);
+    const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win));
+    if (lane == k) my_e = e;
+    if ((e & 31) == lane) {
+      // the winner's lane drops it and finds its next best
+      best = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (i < npl && !((taken >> i) & 1u) && (be == INT_MAX || key[i] > bk)) {
-        bk = key[i];
-        be = lane + 32 * i;
-        bs = s[i];
+      for (int i = 0; i < NPL; ++i) {
+        if (cand[i] == win) cand[i] = 0;
+        best = cand[i] > best ? cand[i] : best;
       }
-    }
-    // warp arg-max: key descending, then expert id ascending
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-      if (ok > bk || (ok == bk && oe < be)) {
-        bk = ok;
-        be = oe;
-        bs = os;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == k) {
-      my_e = be;
-      my_s = bs;
     }
   }
-  // sum of the selected scores in slot order (identical on every lane)
+  // weights: the unbiased scores of the selected experts, renormalised; the
+  // score is recomputed from the same logit with the same expression
+  const float my_s = (lane < K) ? 1.0f / (1.0f + expf(-z[my_e])) : 0.0f;
   float sum = 0.0f;
   for (int k = 0; k < K; ++k) sum += __shfl_sync(0xffffffffu, my_s, k);
   if (lane < K) {
@@ -89,8 +101,13 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
 cudaError_t launch_route(const float* logits, const float* bias, int64_t T, int N, int K,
                          int32_t* topk_idx, float* topk_w, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
-  const int64_t blocks = (T + 7) / 8;
-  k_route<<<static_cast<unsigned>(blocks), 256, 0, st>>>(logits, bias, T, N, K, topk_idx, topk_w);
+  const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
+  if (N <= 32 * 4)
+    k_route<4><<<blocks, 256, 0, st>>>(logits, bias, T, N, K, topk_idx, topk_w);
+  else if (N <= 32 * 16)
+    k_route<16><<<blocks, 256, 0, st>>>(logits, bias, T, N, K, topk_idx, topk_w);
+  else
+    k_route<32><<<blocks, 256, 0, st>>>(logits, bias, T, N, K, topk_idx, topk_w);
   return cudaGetLastError();
 }
 
@@ -104,13 +121,18 @@ __device__ __forceinline__ void build_chunk_masks(uint32_t* m, const int32_t* __
   __syncwarp();
   const int64_t t = c * 32 + lane;
   if (t < T) {
-    for (int k = 0; k < K; ++k) {
-      const int e = idx[t * K + k];
-      if (e < 0 || e >= N) {
-        atomicOr(err, DEVERR_BAD_INDEX);
-        continue;
+    int ek[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) ek[k] = (k < K) ? idx[t * K + k] : 0;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      if (k < K) {
+        if (ek[k] < 0 || ek[k] >= N) {
+          atomicOr(err, DEVERR_BAD_INDEX);
+        } else {
+          atomicOr(&m[ek[k]], 1u << lane);
+        }
       }
-      atomicOr(&m[e], 1u << lane);
     }
   }
   __syncwarp();
@@ -268,13 +290,25 @@ __global__ void __launch_bounds__(256) k_scatter(
   const int64_t t = c * 32 + lane;
   if (t < T) {
     const uint32_t lower = (1u << lane) - 1u;
-    for (int k = 0; k < K; ++k) {
-      const int e = idx[t * K + k];
-      if (e < 0 || e >= N) continue;
-      const int row = off[e] + chunk_base[c * N + e] + __popc(m[e] & lower);
-      inv[t * K + k] = row;
-      perm[row] = static_cast<int32_t>(t * K + k);
-      wrow[row] = topk_w[t * K + k];
+    int ek[32], base[32];
+    float wk[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      ek[k] = (k < K) ? idx[t * K + k] : -1;
+      wk[k] = (k < K) ? topk_w[t * K + k] : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      base[k] = (ek[k] >= 0 && ek[k] < N) ? chunk_base[c * N + ek[k]] : 0;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const int e = ek[k];
+      if (k < K && e >= 0 && e < N) {
+        const int row = off[e] + base[k] + __popc(m[e] & lower);
+        inv[t * K + k] = row;
+        perm[row] = static_cast<int32_t>(t * K + k);
+        wrow[row] = wk[k];
+      }
     }
   }
 }
@@ -319,40 +353,58 @@ cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int 
 }
 
 // ---------------------------------------------------------------------------
-// latent combine in token order: v[t] = sum_k O[inv[t][k]], fixed slot order
+// latent combine in token order: v[t] = sum_k O[inv[t][k]], fixed slot order.
+// One thread per 8 consecutive latent elements of one token; the K row
+// indices and the K row loads are issued before the (ordered) sum.
 
 __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict__ O,
                                                  const int32_t* __restrict__ inv, int64_t T,
                                                  int K, int l, __nv_bfloat16* __restrict__ vh,
                                                  int ldv) {
-  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+  const int l8 = l >> 3;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t t = g / l8;
   if (t >= T) return;
-  const int my_row = (lane < K) ? inv[t * K + lane] : 0;
-  for (int c = lane * 8; c < l; c += 256) {
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int k = 0; k < K; ++k) {
-      const int64_t row = __shfl_sync(0xffffffffu, my_row, k);
-      const uint4 raw = *reinterpret_cast<const uint4*>(O + row * l + c);
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  const int c = static_cast<int>(g - t * l8) * 8;
+  int rows[32];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(p[i]);
-        acc[2 * i] += f.x;
-        acc[2 * i + 1] += f.y;
+  for (int k = 0; k < 32; ++k) rows[k] = (k < K) ? inv[t * K + k] : 0;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  // eight row loads in flight, then their sums in slot order
+#pragma unroll
+  for (int k0 = 0; k0 < 32; k0 += 8) {
+    if (k0 < K) {
+      uint4 raw[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        raw[j] = (k0 + j < K)
+                     ? __ldg(reinterpret_cast<const uint4*>(
+                           O + static_cast<int64_t>(rows[k0 + j]) * l + c))
+                     : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (k0 + j < K) {
+          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw[j]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p[i]);
+            acc[2 * i] += f.x;
+            acc[2 * i + 1] += f.y;
+          }
+        }
       }
     }
-    __nv_bfloat162 outp[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) outp[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-    *reinterpret_cast<uint4*>(vh + t * ldv + c) = *reinterpret_cast<const uint4*>(outp);
   }
+  __nv_bfloat162 outp[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) outp[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+  *reinterpret_cast<uint4*>(vh + t * ldv + c) = *reinterpret_cast<const uint4*>(outp);
 }
 
 cudaError_t launch_combine(const void* O, const int32_t* inv, int64_t T, int K, int l, void* vh,
                            int ldv, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
-  const int64_t blocks = (T + 7) / 8;
+  const int64_t blocks = (T * (l / 8) + 255) / 256;
   k_combine<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(O), inv, T, K, l, static_cast<__nv_bfloat16*>(vh), ldv);
   return cudaGetLastError();

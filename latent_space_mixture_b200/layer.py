@@ -97,8 +97,8 @@ class LatentMoE:
     def sync_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
         return self.lib.lmoe_sync_status(self.h, _stream_ptr(stream))
 
-    def launches_per_forward(self) -> int:
-        return self.lib.lmoe_launches_per_forward(self.h)
+    def launches_per_forward(self, T: int) -> int:
+        return self.lib.lmoe_launches_per_forward(self.h, int(T))
 
     # -- debug readout ----------------------------------------------------
     def debug(self, what: str) -> torch.Tensor:

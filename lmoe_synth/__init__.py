@@ -64,6 +64,10 @@ CONFIGS: Dict[str, LayerConfig] = {
     # decode batch): a small case of the same kernels for profiler captures
     "super_decode_n64": LayerConfig("super_decode_n64", 32, 4096, 1024, 64, 22, 2688,
                                     5376, 0.02, "zero", 5),
+    # Super dims with 64 experts and 1024 tokens (352 rows per expert, as in
+    # the prefill batch), Zipf bias: a small prefill case for profiler captures
+    "super_prefill_n64": LayerConfig("super_prefill_n64", 1024, 4096, 1024, 64, 22, 2688,
+                                     5376, 0.02, "zipf", 6),
     # Super dims prefill with NVFP4 experts, Zipf(1.1) router bias
     "super_prefill_nvfp4": LayerConfig("super_prefill_nvfp4", 8192, 4096, 1024,
                                        512, 22, 2688, 5376, 0.02, "zipf", 4,

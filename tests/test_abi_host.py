@@ -68,7 +68,7 @@ def test_create_rejects_bad_configs_without_gpu(lib, kw, code):
 def test_null_handle_calls(lib):
     assert lib.lmoe_forward(None, None, 1, None, None) == -1
     assert lib.lmoe_sync_status(None, None) == -1
-    assert lib.lmoe_launches_per_forward(None) == -1
+    assert lib.lmoe_launches_per_forward(None, 1) == -1
     assert lib.lmoe_get_debug(None, 1, None, 0) == -1
     lib.lmoe_destroy(None)
 
