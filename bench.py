@@ -118,6 +118,39 @@ def barrier():
         torch.distributed.barrier()
 
 
+def timed_region(step, steps: int, new_timer, between=None):
+    """Run `steps` steps bracketed by a barrier on both sides; `new_timer()`
+    returns (start, stop, elapsed_ms) callables for one step (CUDA events on
+    the GPU); `between()` runs before each step, outside its timer (the L2
+    flush).  Returns (per-step ms list, max over ranks of their sum)."""
+    timers = [new_timer() for _ in range(steps)]
+    barrier()
+    for i in range(steps):
+        if between is not None:
+            between()
+        timers[i][0]()
+        step()
+        timers[i][1]()
+    per_step = [t[2]() for t in timers]
+    barrier()
+    return per_step, max_over_ranks(sum(per_step))
+
+
+def throughput(world: int, tokens_per_rank: int, steps: int, total_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (total_ms / 1e3)
+
+
+def cuda_timer(stream):
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+
+    def elapsed():
+        e.synchronize()
+        return s.elapsed_time(e)
+    return (lambda: s.record(stream)), (lambda: e.record(stream)), elapsed
+
+
 class ClockSampler:
     """SM clock and throttle reasons sampled through NVML during a region."""
 
@@ -250,7 +283,9 @@ def main():
     gen.manual_seed(shard_seed(cfg.seed, rank))
     x = make_x(cfg, gen, device=dev)
     T = cfg.T
-    layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w)
+    from lmoe_synth import act_global_scales
+    layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, expert_format=cfg.fmt,
+                      act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0))
     y = torch.empty_like(x)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
     stream = torch.cuda.current_stream()
@@ -265,18 +300,11 @@ def main():
     clocks = ClockSampler(local_rank).start()
     layer.profile_enable(True)
     layer.profile_read(reset=True)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier()
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
-    for i in range(args.steps):
-        flush.zero_()                      # L2 flush, outside the step's events
-        starts[i].record(stream)
-        layer.forward(x, out=y)
-        ends[i].record(stream)
+    step_ms, total_ms = timed_region(lambda: layer.forward(x, out=y), args.steps,
+                                     lambda: cuda_timer(stream), between=flush.zero_)
     torch.cuda.synchronize()
-    barrier()
     t_wall1 = time.perf_counter()
     clocks.stop()
     prof = layer.profile_read(reset=True)
@@ -284,10 +312,8 @@ def main():
     rc = layer.sync_status()
     if rc != 0:
         raise RuntimeError(f"device status {rc} after the timed steps")
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1e3)
+    value = throughput(world, T, args.steps, total_ms)
 
     counts = layer.debug("counts").numpy()
     lay, per_kernel = algorithmic_work(cfg, T, counts)
@@ -313,19 +339,10 @@ def main():
         yh = torch.empty_like(xh).pin_memory()
         for _ in range(args.warmup):
             layer.forward_host(xh, yh)
-        es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        barrier()
         torch.cuda.synchronize()
-        for i in range(args.steps):
-            flush.zero_()
-            es[i].record(stream)
-            layer.forward_host(xh, yh)
-            ee[i].record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es, ee)))
-        e2e = {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        _, e2e_ms = timed_region(lambda: layer.forward_host(xh, yh), args.steps,
+                                 lambda: cuda_timer(stream), between=flush.zero_)
+        e2e = {"value": round(throughput(world, T, args.steps, e2e_ms), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
                "ms_per_step": round(e2e_ms / args.steps, 4)}
 

@@ -42,9 +42,15 @@ extern "C" {
 #define LMOE_ERR_DEVICE (-6)      /* a kernel flagged bad data (e.g. index) */
 
 #define LMOE_FMT_BF16 0  /* experts in BF16                                   */
-#define LMOE_FMT_NVFP4 1 /* experts in NVFP4 (reserved: returns UNSUPPORTED)  */
+#define LMOE_FMT_NVFP4 1 /* experts in NVFP4: W1, W2 and the expert inputs u
+                            and H as E2M1 codes with E4M3 scales per 16
+                            elements along the reduction axis and an FP32
+                            global scale; latent projections, router and
+                            shared expert stay BF16 ("Nemotron-3 Super 精读报告",
+                            table 5.2).  Needs l and h multiples of 128.      */
 
-/* Layer shape.  d, latent, expert_hidden, shared_hidden: multiples of 64.
+/* Layer shape.  d, latent, expert_hidden, shared_hidden: multiples of 64
+ * (latent and expert_hidden multiples of 128 for LMOE_FMT_NVFP4).
  * n_experts: multiple of 32, at most 1024.  top_k: 1..min(32, n_experts).
  * max_tokens: the largest T a forward call accepts (sizes the workspace). */
 typedef struct lmoe_config {
@@ -70,17 +76,20 @@ typedef struct lmoe_weights {
   const void* w_upl;       /* [d][l]      bf16                              */
   const void* w_s1;        /* [h_s][d]    bf16                              */
   const void* w_s2;        /* [d][h_s]    bf16                              */
-  float act_gscale_latent; /* NVFP4 only: static global scale of u          */
-  float act_gscale_hidden; /* NVFP4 only: static global scale of the expert
-                              hidden activation                             */
+  float act_gscale_latent; /* NVFP4 only (> 0): static global scale of u;
+                              its block scales are E4M3(amax16/(6 g))       */
+  float act_gscale_hidden; /* NVFP4 only (> 0): static global scale of the
+                              expert hidden activation sqrelu(W1 u)         */
 } lmoe_weights;
 
 typedef struct lmoe_handle lmoe_handle;
 
 /* Build a layer on the current device: validates cfg, allocates the weights'
  * copies (re-laid out: [W_r; W_dn; W_s1] as one [N+l+h_s][d] matrix and
- * [W_upl | W_s2] as one [d][l+h_s] matrix) and a workspace for max_tokens,
- * and synchronizes the device once.  *out receives the handle, owned by the
+ * [W_upl | W_s2] as one [d][l+h_s] matrix; for NVFP4 experts W1 and W2 are
+ * quantised on the device instead, per expert matrix with global scale
+ * amax/(6*448)) and a workspace for max_tokens, and synchronizes the device
+ * once.  *out receives the handle, owned by the
  * caller until lmoe_destroy.  Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA. */
 int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out);
 
@@ -116,6 +125,12 @@ int lmoe_sync_status(lmoe_handle* h, void* stream);
  *   LMOE_DBG_U         bf16  [T][l]   latent u
  *   LMOE_DBG_V         bf16  [T][l]   latent combine v
  *   LMOE_DBG_HS        bf16  [T][h_s] shared hidden sqrelu(W_s1 x)
+ * and, for NVFP4 experts (lp, hp = l, h rounded up to 256):
+ *   LMOE_DBG_W1Q_CODES u8   [N*h][lp/2]  E2M1 codes, lower index in the low nibble
+ *   LMOE_DBG_W1Q_SF    u8   [N*h/128][lp/64][512] E4M3 scales; row m, 16-block
+ *                           k1 of a 64-chunk at byte (m%32)*16+((m/32)%4)*4+k1
+ *   LMOE_DBG_W1Q_G     fp32 [N]          global scales
+ *   LMOE_DBG_W2Q_CODES / _SF / _G   the same for W2 ([N*l][hp/2], ...)
  * Errors: INVALID_ARG (unknown item, wrong size), CUDA. */
 #define LMOE_DBG_TOPK_IDX 1
 #define LMOE_DBG_TOPK_W 2
@@ -127,6 +142,12 @@ int lmoe_sync_status(lmoe_handle* h, void* stream);
 #define LMOE_DBG_U 8
 #define LMOE_DBG_V 9
 #define LMOE_DBG_HS 10
+#define LMOE_DBG_W1Q_CODES 11
+#define LMOE_DBG_W1Q_SF 12
+#define LMOE_DBG_W1Q_G 13
+#define LMOE_DBG_W2Q_CODES 14
+#define LMOE_DBG_W2Q_SF 15
+#define LMOE_DBG_W2Q_G 16
 int lmoe_get_debug(lmoe_handle* h, int what, void* dst_host, size_t bytes);
 
 /* Kernel launches one lmoe_forward of T tokens issues (10, plus one split-K
@@ -176,6 +197,16 @@ int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int
 int lmoe_route_noalloc(const float* logits, const float* bias, int64_t T, int32_t N, int32_t K,
                        int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
                        int32_t* perm, int32_t* inv, void* stream);
+
+/* NVFP4 quantisation of fp32 rows x [rows][cols] (device, 16-byte aligned,
+ * cols a multiple of 16) with global scale g >= 0, exactly as the layer
+ * quantises its activations: per 16 consecutive elements s = E4M3(amax /
+ * (6 g)) and q = E2M1(x * r) with r = 1 / (s g) rounded once per block
+ * (round to nearest even, saturating; all float32).  Outputs (device): codes [rows][cols/2] (lower index in the low
+ * nibble), scales [rows][cols/16] E4M3 codes.  Asynchronous on `stream`.
+ * Errors: INVALID_ARG, CUDA. */
+int lmoe_nvfp4_quantize(const float* x, int64_t rows, int32_t cols, float g, uint8_t* codes,
+                        uint8_t* scales, void* stream);
 
 /* Runs a one-CTA kernel that waits on an mbarrier nothing arrives on, with a
  * wait limit of limit_ns nanoseconds (1e3..1e10), and returns the status the

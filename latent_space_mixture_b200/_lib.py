@@ -14,7 +14,8 @@ ERRORS = {-1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "OOM", -4: "CUDA", -5: "TIME
           -6: "DEVICE"}
 FMT_BF16, FMT_NVFP4 = 0, 1
 DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 6,
-       "logits": 7, "u": 8, "v": 9, "hs": 10}
+       "logits": 7, "u": 8, "v": 9, "hs": 10, "w1q_codes": 11, "w1q_sf": 12, "w1q_g": 13,
+       "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16}
 
 
 class LmoeConfig(Structure):
@@ -54,6 +55,8 @@ SIGNATURES = {
                            c_void_p]),
     "lmoe_route_noalloc": (c_int, [c_void_p, c_void_p, c_int64, c_int32, c_int32, c_void_p,
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "lmoe_nvfp4_quantize": (c_int, [c_void_p, c_int64, c_int32, c_float, c_void_p, c_void_p,
+                                    c_void_p]),
     "lmoe_check_bounded_wait": (c_int, [c_int64]),
     "lmoe_destroy": (None, [c_void_p]),
     "lmoe_strerror": (c_char_p, [c_int]),

@@ -9,30 +9,39 @@
 // expert with 11 routed rows costs an N=16 MMA, not a 128-row tile.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over a static tile list):
-//   warp 0      TMA producer: A tile 128x64 and B rows in 16-row boxes per
+//   warp 0      TMA producer: A tile and B rows (64- and 16-row boxes) per
 //               k-step, 128-byte swizzle, completion on a "full" mbarrier;
-//   warp 1      TMEM allocator and MMA issuer: 4 x (M128 N K16) per k-step,
-//               tcgen05.commit frees the smem stage, a second commit marks the
-//               accumulator full;
+//               in the NVFP4 variant also the two scale-factor tiles (bulk
+//               copies of 2 KB);
+//   warp 1      TMEM allocator and MMA issuer: per k-step 4 MMAs of K=16
+//               (kind::f16, bf16) or K=64 (kind::mxf4nvf4 with 16-element
+//               block scales copied into TMEM by tcgen05.cp first);
+//               tcgen05.commit frees the smem stage, and at the end of a tile
+//               marks the accumulator full;
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, transpose through a
 //               per-warp smem tile, call the epilogue functor on 8 consecutive
-//               features of one token row, release the accumulator.
+//               features of one token row (all lanes call it; `valid` tells
+//               which carry data), release the accumulator.
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap
 // the main loop of tile i+1.  Every mbarrier wait is bounded (ptx.cuh).
 #pragma once
 #include <cuda_bf16.h>
 
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 
 namespace lmoe {
 
 constexpr int GEMM_BM = 128;          // MMA M: features per tile
-constexpr int GEMM_BK = 64;           // K elements per pipeline stage (128 B)
+constexpr int GEMM_BK = 64;           // bf16 K elements per stage (128 B per row)
 constexpr int GEMM_THREADS = 192;
 constexpr int GEMM_EPI_WARPS = 4;
 constexpr int GEMM_STG_LD = 36;       // fp32 staging pitch (32 + 4)
 constexpr int GEMM_BROWS = 16;        // rows per small B TMA box (ragged tails)
 constexpr int GEMM_BROWS_BIG = 64;    // rows per large B TMA box (full row groups)
+constexpr int GEMM_ROW_BYTES = 128;   // bytes of one operand row per stage
+constexpr int FP4_K_PER_STAGE = 256;  // NVFP4 K elements per stage (128 B per row)
+constexpr int FP4_SF_STAGE_BYTES = 4 * SF_ATOM_BYTES;   // 4 chunks of K=64
 
 // Where the tiles of one GEMM come from.
 struct TileSource {
@@ -43,14 +52,17 @@ struct TileSource {
   int FB;                  // feature blocks of 128 per expert
   int a_rows_per_expert;   // rows of A per expert (0 when dense)
   int m_valid;             // valid features per expert (multiple of 8)
-  int kblocks;             // K / 64
+  int kblocks;             // K steps (K/64 bf16, K/256 NVFP4)
   int ksplit;              // dense only: K slices (1 = none); each slice writes
   float* part;             //   fp32 partials part[slice][row][feature]
   int a_stream_once;       // 1: each A tile is read by one tile only (L2 evict-first)
+  const uint8_t* sfa;      // NVFP4: A scale atoms, [A row / 128][kc][512 B]
+  const uint8_t* sfb;      // NVFP4: B scale atoms, [token block][kc][512 B]
+  int kc;                  // NVFP4: 64-element chunks per row (4 x kblocks)
 };
 
 struct TileInfo {
-  int e, fb, row0, nrows, a_row, ks, kb0, kb1;
+  int e, fb, row0, nrows, a_row, ks, kb0, kb1, tb;
 };
 
 __device__ __forceinline__ int gemm_num_tiles(const TileSource& s, int BN) {
@@ -64,6 +76,7 @@ __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int t
   const int tk = tile / s.FB;
   t.fb = tile - tk * s.FB;
   const int tb = tk / s.ksplit;
+  t.tb = tb;
   t.ks = tk - tb * s.ksplit;
   t.kb0 = t.ks * s.kblocks / s.ksplit;
   t.kb1 = (t.ks + 1) * s.kblocks / s.ksplit;
@@ -81,32 +94,40 @@ __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int t
   return t;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool FP4>
 struct GemmLayout {
-  static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
-  static constexpr int B_BYTES = BN * GEMM_BK * 2;
+  static constexpr int A_BYTES = GEMM_BM * GEMM_ROW_BYTES;
+  static constexpr int B_BYTES = BN * GEMM_ROW_BYTES;
+  static constexpr int SF_BYTES = FP4 ? 2 * FP4_SF_STAGE_BYTES : 0;
   static constexpr int STG_BYTES = GEMM_EPI_WARPS * 32 * GEMM_STG_LD * 4;
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES) +
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES + SF_BYTES) +
                                     STG_BYTES + BAR_BYTES + 16;
-  static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
+  // TMEM: two accumulators of BN columns, then (NVFP4) 32 scale columns per stage
+  static constexpr int SF_COL0 = 2 * BN;
+  static constexpr int COLS_USED = 2 * BN + (FP4 ? 32 * STAGES : 0);
+  static constexpr uint32_t TMEM_COLS =
+      COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
+                                                  : COLS_USED <= 256 ? 256 : 512;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N range for M=128");
+  static_assert(!FP4 || BN <= 128, "NVFP4 tiles: one scale atom of B rows");
+  static_assert(COLS_USED <= 512, "TMEM columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of 2");
 };
 
-template <int BN, int STAGES, class Epi>
+template <int BN, int STAGES, class Epi, bool FP4>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmB64, const TileSource src, const Epi epi, int* err,
           unsigned long long limit_ns) {
-  using L = GemmLayout<BN, STAGES>;
+  using L = GemmLayout<BN, STAGES, FP4>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * L::A_BYTES;
-  float* stg = reinterpret_cast<float*>(sB + STAGES * L::B_BYTES);
+  uint8_t* sSF = sB + STAGES * L::B_BYTES;           // NVFP4: [stage][A 2 KB | B 2 KB]
+  float* stg = reinterpret_cast<float*>(sSF + STAGES * L::SF_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stg) + L::STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;   // [2]
@@ -161,23 +182,33 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         // B rows: 64-row boxes while 64 rows remain, then 16-row boxes
         const int nbig = t.nrows / GEMM_BROWS_BIG;
         const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
-        const uint32_t tx =
-            L::A_BYTES + (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_BK * 2;
+        const uint32_t tx = L::A_BYTES + L::SF_BYTES +
+                            (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_ROW_BYTES;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err, limit_ns)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[stage], tx);
-          tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, kb * GEMM_BK, t.a_row, &full[stage],
-                           pol_a);
+          // x coordinate in elements of the map: bf16 elements or bytes (NVFP4)
+          const int bx = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+          tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, bx, t.a_row, &full[stage], pol_a);
           uint8_t* b_dst = sB + stage * L::B_BYTES;
           for (int j = 0; j < nbig; ++j)
-            tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_BK * 2, &tmB64, kb * GEMM_BK,
+            tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
                         t.row0 + j * GEMM_BROWS_BIG, &full[stage]);
           for (int j = 0; j < nsmall; ++j) {
             const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
-            tma_load_2d(b_dst + r * GEMM_BK * 2, &tmB, kb * GEMM_BK, t.row0 + r, &full[stage]);
+            tma_load_2d(b_dst + r * GEMM_ROW_BYTES, &tmB, bx, t.row0 + r, &full[stage]);
+          }
+          if constexpr (FP4) {
+            uint8_t* sf = sSF + stage * L::SF_BYTES;
+            bulk_load(sf, src.sfa + (static_cast<long>(t.a_row / GEMM_BM) * src.kc + kb * 4) *
+                                        SF_ATOM_BYTES,
+                      FP4_SF_STAGE_BYTES, &full[stage]);
+            bulk_load(sf + FP4_SF_STAGE_BYTES,
+                      src.sfb + (static_cast<long>(t.tb) * src.kc + kb * 4) * SF_ATOM_BYTES,
+                      FP4_SF_STAGE_BYTES, &full[stage]);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -217,7 +248,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        const uint32_t idesc = idesc_bf16(GEMM_BM, n_mma);
+        const uint32_t idesc = FP4 ? idesc_nvf4(GEMM_BM, n_mma) : idesc_bf16(GEMM_BM, n_mma);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns)) {
             ok = false;
@@ -226,9 +257,27 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           tc_fence_after();
           const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + stage * L::A_BYTES));
           const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + stage * L::B_BYTES));
+          if constexpr (FP4) {
+            // scale atoms of this stage into its TMEM slot, then 4 MMAs of K=64
+            const uint32_t sf_col = L::SF_COL0 + stage * 32;
+            const uint32_t sf_smem = smem_u32(sSF + stage * L::SF_BYTES);
 #pragma unroll
-          for (int k = 0; k < GEMM_BK / 16; ++k)   // +32 bytes per K=16 step
-            umma_bf16(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
+            for (int k = 0; k < 4; ++k) {
+              tmem_cp_32x128b_warpx4(tmem_base + sf_col + 4 * k,
+                                     sdesc_sf_atom(sf_smem + k * SF_ATOM_BYTES));
+              tmem_cp_32x128b_warpx4(
+                  tmem_base + sf_col + 16 + 4 * k,
+                  sdesc_sf_atom(sf_smem + FP4_SF_STAGE_BYTES + k * SF_ATOM_BYTES));
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)   // +32 bytes per K=64 step
+              umma_nvf4(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, tmem_base + sf_col + 4 * k,
+                        tmem_base + sf_col + 16 + 4 * k, (kb != t.kb0) || (k != 0));
+          } else {
+#pragma unroll
+            for (int k = 0; k < GEMM_BK / 16; ++k)   // +32 bytes per K=16 step
+              umma_bf16(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
+          }
           umma_commit(&empty[stage]);
           issued_any = true;
           if (++stage == STAGES) {
@@ -274,23 +323,25 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         __syncwarp();
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
+          // lanes 4j..4j+3 hold the four 8-feature groups of token row j
           const int item = lane + 32 * it;
           const int j = item >> 2;
           const int g = item & 3;
           const int feat = feat_base + g * 8;
-          if (c0 + j < t.nrows && feat < src.m_valid) {
-            const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
-            const float4 lo = p[0], hi = p[1];
-            const long row = static_cast<long>(t.row0 + c0 + j);
-            if (src.ksplit > 1) {
+          const bool valid = c0 + j < t.nrows && feat < src.m_valid;
+          const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
+          const float4 lo = p[0], hi = p[1];
+          const long row = static_cast<long>(t.row0 + c0 + j);
+          if (src.ksplit > 1) {
+            if (valid) {
               float4* dst = reinterpret_cast<float4*>(
                   src.part + (static_cast<long>(t.ks) * src.T + row) * src.m_valid + feat);
               dst[0] = lo;
               dst[1] = hi;
-            } else {
-              const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-              epi.store8(t.e, row, feat, v);
             }
+          } else {
+            const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            epi.store8(t, row, feat, v, valid);
           }
         }
         __syncwarp();
@@ -311,24 +362,29 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 }
 
 // Sum of the K-slice partials in slice order (deterministic), then the real
-// epilogue: thread per 8 consecutive features of one row.
+// epilogue: thread per 8 consecutive features of one row.  All threads of a
+// warp reach the epilogue call (lanes 2i and 2i+1 hold one 16-feature block).
 template <class Epi>
 __global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ part, int ksplit,
                                                        int T, int F, const Epi epi) {
   const long g = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int f8 = F / 8;
   const long row = g / f8;
-  if (row >= T) return;
-  const int feat = static_cast<int>(g - row * f8) * 8;
+  const bool valid = row < T;
+  const long r = valid ? row : 0;
+  const int feat = valid ? static_cast<int>(g - row * f8) * 8 : 0;
   float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int s = 0; s < ksplit; ++s) {
-    const float4* p = reinterpret_cast<const float4*>(part + (static_cast<long>(s) * T + row) * F +
-                                                      feat);
-    const float4 a = p[0], b = p[1];
-    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  if (valid) {
+    for (int s = 0; s < ksplit; ++s) {
+      const float4* p =
+          reinterpret_cast<const float4*>(part + (static_cast<long>(s) * T + r) * F + feat);
+      const float4 a = p[0], b = p[1];
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
   }
-  epi.store8(0, row, feat, v);
+  TileInfo t{};
+  epi.store8(t, r, feat, v, valid);
 }
 
 // ---------------------------------------------------------------------------
@@ -344,6 +400,28 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* dst, const float* v) 
 __device__ __forceinline__ float sqrelu(float a) {
   const float r = fmaxf(a, 0.0f);
   return r * r;
+}
+
+// NVFP4 quantisation of 8 features whose 16-block partner is lane ^ 1 (lane
+// pairs hold a block's halves; every lane of the warp must call this).
+// Returns this lane's 4 code bytes (lower feature in the lower nibble) and
+// the block's E4M3 scale code.
+__device__ __forceinline__ uint32_t nvfp4_pair(const float* v, float g, uint8_t* sc) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  const float six_g = __fmul_rn(6.0f, g);
+  const float sbf = six_g > 0.0f ? __fdiv_rn(amax, six_g) : 0.0f;
+  const uint8_t code = e4m3_code(sbf);
+  const float denom = __fmul_rn(e4m3_value(code), g);
+  const float rcp = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w |= e2m1x2(__fmul_rn(v[2 * i], rcp), __fmul_rn(v[2 * i + 1], rcp)) << (8 * i);
+  *sc = code;
+  return w;
 }
 
 }  // namespace lmoe

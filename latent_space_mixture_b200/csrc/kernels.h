@@ -21,10 +21,12 @@ cudaError_t launch_scan(int32_t* chunk_cnt, int64_t T, int N, int32_t* counts, c
 // Offsets (exclusive scan of counts), perm / inv / per-row weights, and the
 // list of token blocks (at most `bn` rows, one expert each) for the grouped
 // GEMMs: blocks[i] = {expert, first row, rows, 0}, *nblocks = count.
+// rblock (optional, may be NULL): per row, (token block << 8) | row in block.
 cudaError_t launch_scatter(const int32_t* topk_idx, const float* topk_w, const int32_t* chunk_base,
                            const int32_t* counts, int64_t T, int N, int K, int bn,
                            int32_t* offsets, int32_t* perm, int32_t* inv, float* wrow,
-                           int4* blocks, int32_t* nblocks, int* err, cudaStream_t st);
+                           int4* blocks, int32_t* nblocks, int32_t* rblock, int* err,
+                           cudaStream_t st);
 
 // u_perm[r] = u[perm[r] / K] for r < T*K (rows of width l, bf16).
 cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int K, int l,
@@ -34,6 +36,19 @@ cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int 
 // l columns of vh (row pitch ldv).
 cudaError_t launch_combine(const void* O, const int32_t* inv, int64_t T, int K, int l, void* vh,
                            int ldv, cudaStream_t st);
+
+// NVFP4 (nvfp4.cu).  Expert weights [E][rows_per][K] bf16 -> codes
+// [E*rows_per][Kp/2], scale atoms [E*rows_per/128][Kp/64][512], global scales
+// [E]; amax is [E] scratch.  Kp = K rounded up to 256; padding pre-zeroed.
+cudaError_t launch_quant_weights(const void* w, int E, int rows_per, int K, int Kp, float* amax,
+                                 uint8_t* codes, uint8_t* atoms, float* gscale, cudaStream_t st);
+// fp32 rows -> codes [rows][cols/2], scales [rows][cols/16] (canonical layout).
+cudaError_t launch_quant_rows(const float* x, int64_t rows, int cols, float g, uint8_t* codes,
+                              uint8_t* scales, cudaStream_t st);
+// quantised u rows into expert order plus their scales into block atoms.
+cudaError_t launch_gather_q(const uint8_t* uq, const uint8_t* usf, const int32_t* perm,
+                            const int32_t* rblock, int64_t rows, int K, int l, int lp,
+                            uint8_t* u_perm_q, uint8_t* atoms, cudaStream_t st);
 
 // A kernel whose mbarrier wait never completes, bounded by limit_ns: sets
 // DEVERR_TIMEOUT in *err and returns.  Used to check the failure path.

@@ -28,7 +28,22 @@ struct EpiX {
   bf16* u;
   bf16* vh;
   int N, l, ldvh;
-  __device__ __forceinline__ void store8(int, long row, int feat, const float* v) const {
+  uint8_t* uq;    // NVFP4 experts: u codes [T][l/2] (nullptr for BF16 experts)
+  uint8_t* usf;   //   and its E4M3 block scales [T][l/16]
+  float g_u;      //   static global scale of u
+  __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (uq) {
+      // every lane takes part in the 16-block pair exchange; only u lanes store
+      uint8_t sc;
+      const uint32_t codes = nvfp4_pair(v, g_u, &sc);
+      if (valid && feat >= N && feat < N + l) {
+        const int f = feat - N;
+        *reinterpret_cast<uint32_t*>(uq + row * (l / 2) + f / 2) = codes;
+        if ((f & 15) == 0) usf[row * (l / 16) + f / 16] = sc;
+      }
+    }
+    if (!valid) return;
     if (feat < N) {
       float4* p = reinterpret_cast<float4*>(logits + row * N + feat);
       p[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -48,7 +63,9 @@ struct EpiX {
 struct EpiH {
   bf16* H;
   int h;
-  __device__ __forceinline__ void store8(int, long row, int feat, const float* v) const {
+  __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
     float a[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = sqrelu(v[i]);
@@ -61,7 +78,9 @@ struct EpiO {
   bf16* O;
   const float* wrow;
   int l;
-  __device__ __forceinline__ void store8(int, long row, int feat, const float* v) const {
+  __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
     const float w = wrow[row];
     float a[8];
 #pragma unroll
@@ -74,31 +93,84 @@ struct EpiO {
 struct EpiY {
   bf16* y;
   int d;
-  __device__ __forceinline__ void store8(int, long row, int feat, const float* v) const {
+  __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
     store8_bf16(y + row * d + feat, v);
   }
 };
 
-// GEMM variants: (BN, STAGES)
-template <int BN>
+// NVFP4 expert FC1: H = sqrelu(g_W1[e] g_u * acc), quantised with the static
+// global scale g_h into codes [R][hp/2] and the B-operand scale atoms of the
+// second grouped GEMM ([token block][hp/64][512 B], row = index in the block).
+struct EpiHq {
+  uint8_t* Hq;
+  uint8_t* sfh;
+  const float* gw1;
+  float g_u, g_h;
+  int hp;   // h rounded up to 256 (row pitch hp/2 bytes)
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    const float s = __fmul_rn(gw1[t.e], g_u);
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = sqrelu(v[i] * s);
+    uint8_t sc;
+    const uint32_t codes = nvfp4_pair(a, g_h, &sc);
+    if (!valid) return;
+    *reinterpret_cast<uint32_t*>(Hq + row * (hp / 2) + feat / 2) = codes;
+    if ((feat & 15) == 0)
+      sfh[(static_cast<long>(t.tb) * (hp / 64) + feat / 64) * SF_ATOM_BYTES +
+          sf_atom_offset(static_cast<int>(row - t.row0), (feat & 63) >> 4)] = sc;
+  }
+};
+
+// NVFP4 expert FC2 times the router weight: O = w g_W2[e] g_h * acc (bf16)
+struct EpiOq {
+  bf16* O;
+  const float* wrow;
+  const float* gw2;
+  float g_h;
+  int l;
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(__fmul_rn(gw2[t.e], g_h), wrow[row]);
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = v[i] * s;
+    store8_bf16(O + row * l + feat, a);
+  }
+};
+
+// GEMM variants: (BN, operand format) -> pipeline stages
+template <int BN, bool FP4>
 struct Stages;
 template <>
-struct Stages<256> {
+struct Stages<256, false> {
   static constexpr int value = 4;
 };
 template <>
-struct Stages<128> {
+struct Stages<128, false> {
   static constexpr int value = 6;
 };
 template <>
-struct Stages<32> {
+struct Stages<32, false> {
   static constexpr int value = 10;
 };
+template <>
+struct Stages<128, true> {
+  static constexpr int value = 5;
+};
+template <>
+struct Stages<32, true> {
+  static constexpr int value = 8;
+};
 
-template <int BN, class Epi>
+template <int BN, class Epi, bool FP4 = false>
 cudaError_t set_gemm_smem() {
-  using L = GemmLayout<BN, Stages<BN>::value>;
-  return cudaFuncSetAttribute(k_gemm_tc<BN, Stages<BN>::value, Epi>,
+  using L = GemmLayout<BN, Stages<BN, FP4>::value, FP4>;
+  return cudaFuncSetAttribute(k_gemm_tc<BN, Stages<BN, FP4>::value, Epi, FP4>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
 }
 
@@ -107,14 +179,22 @@ struct BMaps {
   CUtensorMap b16, b64;
 };
 
-template <int BN, class Epi>
+template <int BN, class Epi, bool FP4 = false>
 cudaError_t launch_gemm(const CUtensorMap& A, const BMaps& B, const TileSource& src,
                         const Epi& epi, int grid, int* err, unsigned long long limit,
                         cudaStream_t st) {
-  using L = GemmLayout<BN, Stages<BN>::value>;
-  k_gemm_tc<BN, Stages<BN>::value, Epi>
+  using L = GemmLayout<BN, Stages<BN, FP4>::value, FP4>;
+  k_gemm_tc<BN, Stages<BN, FP4>::value, Epi, FP4>
       <<<grid, GEMM_THREADS, L::SMEM_BYTES, st>>>(A, B.b16, B.b64, src, epi, err, limit);
   return cudaGetLastError();
+}
+
+template <class Epi>
+cudaError_t launch_gemm_fp4(int bn, const CUtensorMap& A, const BMaps& B, const TileSource& src,
+                            const Epi& epi, int grid, int* err, unsigned long long limit,
+                            cudaStream_t st) {
+  if (bn == 128) return launch_gemm<128, Epi, true>(A, B, src, epi, grid, err, limit, st);
+  return launch_gemm<32, Epi, true>(A, B, src, epi, grid, err, limit, st);
 }
 
 template <class Epi>
@@ -178,6 +258,21 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D byte matrix [rows][cols] (packed NVFP4 codes), box of 128 bytes x
+// box_rows rows, 128-byte swizzle.
+static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                        uint32_t box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -257,6 +352,26 @@ struct lmoe_handle {
   bf16* y_dev = nullptr;
   float* part = nullptr;   // split-K partials of the dense GEMMs
   int* err = nullptr;
+  // NVFP4 experts: quantised weights, activations and their scale atoms
+  bool fp4 = false;
+  int lp = 0, hp = 0;          // l, h rounded up to 256 (K of the two grouped GEMMs)
+  float g_u = 0.f, g_h = 0.f;  // static global scales of u and of the expert hidden
+  uint8_t* w1q = nullptr;      // [N*h][lp/2]
+  uint8_t* w1sf = nullptr;     // [N*h/128][lp/64][512]
+  float* gw1 = nullptr;        // [N]
+  uint8_t* w2q = nullptr;      // [N*l][hp/2]
+  uint8_t* w2sf = nullptr;     // [N*l/128][hp/64][512]
+  float* gw2 = nullptr;        // [N]
+  float* amax = nullptr;       // [N] scratch of the weight quantisation
+  uint8_t* uq = nullptr;       // [T][l/2]
+  uint8_t* usf = nullptr;      // [T][l/16]
+  uint8_t* upq = nullptr;      // [T*K][lp/2] expert order
+  uint8_t* sfbu = nullptr;     // [token blocks][lp/64][512]
+  uint8_t* Hq = nullptr;       // [T*K][hp/2]
+  uint8_t* sfbh = nullptr;     // [token blocks][hp/64][512]
+  int32_t* rblock = nullptr;   // [T*K] (token block << 8) | row in block
+  CUtensorMap tm_w1q, tm_w2q;
+  BMaps tm_upq, tm_Hq;
   std::vector<void*> allocs;
   CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
   BMaps tm_uperm, tm_H, tm_vh;
@@ -271,7 +386,13 @@ struct lmoe_handle {
   int64_t prof_n[kNumKernels] = {};
 };
 
+// A zero-byte request leaves the pointer null, so that a buffer of an unused
+// path can never be mistaken for a live one.
 static int alloc_dev(lmoe_handle* h, void** p, size_t bytes) {
+  if (bytes == 0) {
+    *p = nullptr;
+    return LMOE_OK;
+  }
   if (cudaMalloc(p, bytes < 256 ? 256 : bytes) != cudaSuccess) {
     cudaGetLastError();
     return LMOE_ERR_OOM;
@@ -295,7 +416,8 @@ static int check_cfg(const lmoe_config* c) {
   if (c->top_k > c->n_experts) return LMOE_ERR_INVALID_ARG;
   if (c->expert_format != LMOE_FMT_BF16 && c->expert_format != LMOE_FMT_NVFP4)
     return LMOE_ERR_INVALID_ARG;
-  if (c->expert_format == LMOE_FMT_NVFP4) return LMOE_ERR_UNSUPPORTED;
+  if (c->expert_format == LMOE_FMT_NVFP4 && (c->latent % 128 || c->expert_hidden % 128))
+    return LMOE_ERR_UNSUPPORTED;
   if (c->d % 64 || c->latent % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
     return LMOE_ERR_UNSUPPORTED;
   if (c->n_experts % 32 || c->n_experts > 1024 || c->top_k > 32) return LMOE_ERR_UNSUPPORTED;
@@ -306,11 +428,12 @@ static int check_cfg(const lmoe_config* c) {
   return LMOE_OK;
 }
 
-// grouped-GEMM token-block width for a forward of T tokens
+// grouped-GEMM token-block width for a forward of T tokens (NVFP4 tiles have
+// at most 128 token rows: one scale atom)
 static int grouped_bn(const lmoe_config& c, int64_t T) {
   const double avg = double(T) * c.top_k / c.n_experts;
   if (avg <= 40.0) return 32;
-  if (avg <= 160.0) return 128;
+  if (avg <= 160.0 || c.expert_format == LMOE_FMT_NVFP4) return 128;
   return 256;
 }
 
@@ -336,6 +459,10 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   if (rc != LMOE_OK) return rc;
   if (!w || !w->w_router || !w->w_dn || !w->w1 || !w->w2 || !w->w_upl || !w->w_s1 || !w->w_s2)
     return LMOE_ERR_INVALID_ARG;
+  if (cfg->expert_format == LMOE_FMT_NVFP4 &&
+      !(w->act_gscale_latent > 0.0f && w->act_gscale_hidden > 0.0f &&
+        w->act_gscale_latent < 3.0e38f && w->act_gscale_hidden < 3.0e38f))
+    return LMOE_ERR_INVALID_ARG;
   if (!get_encode()) return LMOE_ERR_CUDA;
 
   lmoe_handle* h = new (std::nothrow) lmoe_handle();
@@ -355,6 +482,14 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   const int64_t rows_b = rows < 256 ? 256 : rows;
   const int64_t Tm_b = Tm < 256 ? 256 : Tm;
   const int64_t d_a = d < GEMM_BM ? GEMM_BM : d;
+  const bool fp4 = c.expert_format == LMOE_FMT_NVFP4;
+  h->fp4 = fp4;
+  h->lp = static_cast<int>((l + 255) / 256 * 256);
+  h->hp = static_cast<int>((hh + 255) / 256 * 256);
+  const int64_t lp = h->lp, hp = h->hp;
+  const int64_t nb_max = rows / 32 + N + 1;   // token blocks of >= 32 rows, one partial per expert
+  // bytes of the bf16 expert path buffers that NVFP4 replaces
+  const int64_t bf16_only = fp4 ? 0 : 1;
   // largest split-K partials buffer over the token counts this handle accepts
   int64_t part_floats = 0;
   {
@@ -376,8 +511,8 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   } reqs[] = {
       {(void**)&h->w_x, size_t((N + l + hs) * d * 2)},
       {(void**)&h->bias, size_t(N * 4)},
-      {(void**)&h->w1, size_t(N * hh * l * 2)},
-      {(void**)&h->w2, size_t(N * l * hh * 2)},
+      {(void**)&h->w1, size_t(bf16_only * N * hh * l * 2)},
+      {(void**)&h->w2, size_t(bf16_only * N * l * hh * 2)},
       {(void**)&h->w_y, size_t(d_a * (l + hs) * 2)},
       {(void**)&h->logits, size_t(Tm * N * 4)},
       {(void**)&h->topk_idx, size_t(rows * 4)},
@@ -391,14 +526,28 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->blocks, size_t(max_blocks * 16)},
       {(void**)&h->nblocks, size_t(4)},
       {(void**)&h->u, size_t(Tm * l * 2)},
-      {(void**)&h->u_perm, size_t(rows_b * l * 2)},
-      {(void**)&h->H, size_t(rows_b * hh * 2)},
+      {(void**)&h->u_perm, size_t(bf16_only * rows_b * l * 2)},
+      {(void**)&h->H, size_t(bf16_only * rows_b * hh * 2)},
       {(void**)&h->O, size_t(rows * l * 2)},
       {(void**)&h->vh, size_t(Tm_b * (l + hs) * 2)},
       {(void**)&h->x_dev, size_t(Tm_b * d * 2)},
       {(void**)&h->y_dev, size_t(Tm * d * 2)},
       {(void**)&h->part, size_t(part_floats * 4)},
       {(void**)&h->err, size_t(4)},
+      {(void**)&h->w1q, size_t(fp4 * N * hh * lp / 2)},
+      {(void**)&h->w1sf, size_t(fp4 * (N * hh / 128) * (lp / 64) * 512)},
+      {(void**)&h->gw1, size_t(fp4 * N * 4)},
+      {(void**)&h->w2q, size_t(fp4 * N * l * hp / 2)},
+      {(void**)&h->w2sf, size_t(fp4 * (N * l / 128) * (hp / 64) * 512)},
+      {(void**)&h->gw2, size_t(fp4 * N * 4)},
+      {(void**)&h->amax, size_t(fp4 * N * 4)},
+      {(void**)&h->uq, size_t(fp4 * Tm * l / 2)},
+      {(void**)&h->usf, size_t(fp4 * Tm * l / 16)},
+      {(void**)&h->upq, size_t(fp4 * rows_b * lp / 2)},
+      {(void**)&h->sfbu, size_t(fp4 * nb_max * (lp / 64) * 512)},
+      {(void**)&h->Hq, size_t(fp4 * rows_b * hp / 2)},
+      {(void**)&h->sfbh, size_t(fp4 * nb_max * (hp / 64) * 512)},
+      {(void**)&h->rblock, size_t(fp4 * rows * 4)},
   };
   for (auto& r : reqs) {
     if ((rc = alloc_dev(h, r.p, r.bytes)) != LMOE_OK) {
@@ -413,8 +562,38 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   ok &= cudaMemcpy(h->w_x + N * d, w->w_dn, l * d * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
   ok &= cudaMemcpy(h->w_x + (N + l) * d, w->w_s1, hs * d * 2, cudaMemcpyDeviceToDevice) ==
         cudaSuccess;
-  ok &= cudaMemcpy(h->w1, w->w1, N * hh * l * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
-  ok &= cudaMemcpy(h->w2, w->w2, N * l * hh * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  if (!fp4) {
+    ok &= cudaMemcpy(h->w1, w->w1, N * hh * l * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+    ok &= cudaMemcpy(h->w2, w->w2, N * l * hh * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  } else {
+    // padding (K beyond l or h, unused atoms) must read as zero
+    h->g_u = w->act_gscale_latent;
+    h->g_h = w->act_gscale_hidden;
+    ok &= cudaMemset(h->w1q, 0, N * hh * lp / 2) == cudaSuccess;
+    ok &= cudaMemset(h->w1sf, 0, (N * hh / 128) * (lp / 64) * 512) == cudaSuccess;
+    ok &= cudaMemset(h->w2q, 0, N * l * hp / 2) == cudaSuccess;
+    ok &= cudaMemset(h->w2sf, 0, (N * l / 128) * (hp / 64) * 512) == cudaSuccess;
+    ok &= cudaMemset(h->upq, 0, rows_b * lp / 2) == cudaSuccess;
+    ok &= cudaMemset(h->sfbu, 0, nb_max * (lp / 64) * 512) == cudaSuccess;
+    ok &= cudaMemset(h->Hq, 0, rows_b * hp / 2) == cudaSuccess;
+    ok &= cudaMemset(h->sfbh, 0, nb_max * (hp / 64) * 512) == cudaSuccess;
+    ok &= launch_quant_weights(w->w1, static_cast<int>(N), static_cast<int>(hh), static_cast<int>(l),
+                               static_cast<int>(lp), h->amax, h->w1q, h->w1sf, h->gw1,
+                               0) == cudaSuccess;
+    ok &= launch_quant_weights(w->w2, static_cast<int>(N), static_cast<int>(l), static_cast<int>(hh),
+                               static_cast<int>(hp), h->amax, h->w2q, h->w2sf, h->gw2,
+                               0) == cudaSuccess;
+    ok &= make_map_u8(&h->tm_w1q, h->w1q, N * hh, lp / 2, GEMM_BM);
+    ok &= make_map_u8(&h->tm_w2q, h->w2q, N * l, hp / 2, GEMM_BM);
+    ok &= make_map_u8(&h->tm_upq.b16, h->upq, rows_b, lp / 2, GEMM_BROWS);
+    ok &= make_map_u8(&h->tm_upq.b64, h->upq, rows_b, lp / 2, GEMM_BROWS_BIG);
+    ok &= make_map_u8(&h->tm_Hq.b16, h->Hq, rows_b, hp / 2, GEMM_BROWS);
+    ok &= make_map_u8(&h->tm_Hq.b64, h->Hq, rows_b, hp / 2, GEMM_BROWS_BIG);
+    ok &= set_gemm_smem<128, EpiHq, true>() == cudaSuccess;
+    ok &= set_gemm_smem<32, EpiHq, true>() == cudaSuccess;
+    ok &= set_gemm_smem<128, EpiOq, true>() == cudaSuccess;
+    ok &= set_gemm_smem<32, EpiOq, true>() == cudaSuccess;
+  }
   ok &= cudaMemcpy2D(h->w_y, (l + hs) * 2, w->w_upl, l * 2, l * 2, d,
                      cudaMemcpyDeviceToDevice) == cudaSuccess;
   ok &= cudaMemcpy2D(h->w_y + l, (l + hs) * 2, w->w_s2, hs * 2, hs * 2, d,
@@ -425,20 +604,26 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= cudaMemset(h->bias, 0, N * 4) == cudaSuccess;
   ok &= cudaMemset(h->err, 0, 4) == cudaSuccess;
   ok &= cudaMemset(h->vh, 0, Tm_b * (l + hs) * 2) == cudaSuccess;
-  ok &= cudaMemset(h->u_perm, 0, rows_b * l * 2) == cudaSuccess;
-  ok &= cudaMemset(h->H, 0, rows_b * hh * 2) == cudaSuccess;
+  if (!fp4) {
+    ok &= cudaMemset(h->u_perm, 0, rows_b * l * 2) == cudaSuccess;
+    ok &= cudaMemset(h->H, 0, rows_b * hh * 2) == cudaSuccess;
+  }
   ok &= cudaMemset(h->x_dev, 0, Tm_b * d * 2) == cudaSuccess;
   if (d_a > d)
     ok &= cudaMemset(h->w_y + d * (l + hs), 0, (d_a - d) * (l + hs) * 2) == cudaSuccess;
   // tensor maps of the fixed operands
   ok &= make_map(&h->tm_wx, h->w_x, N + l + hs, d, GEMM_BM);
-  ok &= make_map(&h->tm_w1, h->w1, N * hh, l, GEMM_BM);
-  ok &= make_map(&h->tm_w2, h->w2, N * l, hh, GEMM_BM);
+  if (!fp4) {
+    ok &= make_map(&h->tm_w1, h->w1, N * hh, l, GEMM_BM);
+    ok &= make_map(&h->tm_w2, h->w2, N * l, hh, GEMM_BM);
+  }
   ok &= make_map(&h->tm_wy, h->w_y, d_a, l + hs, GEMM_BM);
-  ok &= make_map(&h->tm_uperm.b16, h->u_perm, rows_b, l, GEMM_BROWS);
-  ok &= make_map(&h->tm_uperm.b64, h->u_perm, rows_b, l, GEMM_BROWS_BIG);
-  ok &= make_map(&h->tm_H.b16, h->H, rows_b, hh, GEMM_BROWS);
-  ok &= make_map(&h->tm_H.b64, h->H, rows_b, hh, GEMM_BROWS_BIG);
+  if (!fp4) {
+    ok &= make_map(&h->tm_uperm.b16, h->u_perm, rows_b, l, GEMM_BROWS);
+    ok &= make_map(&h->tm_uperm.b64, h->u_perm, rows_b, l, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_H.b16, h->H, rows_b, hh, GEMM_BROWS);
+    ok &= make_map(&h->tm_H.b64, h->H, rows_b, hh, GEMM_BROWS_BIG);
+  }
   ok &= make_map(&h->tm_vh.b16, h->vh, Tm_b, l + hs, GEMM_BROWS);
   ok &= make_map(&h->tm_vh.b64, h->vh, Tm_b, l + hs, GEMM_BROWS_BIG);
   ok &= set_smem_all<EpiX>() == cudaSuccess;
@@ -537,7 +722,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
                  static_cast<int>(d / 64), p.ksplit, h->part, T <= p.bn};
     const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
     const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
-    EpiX epi{h->logits, h->u, h->vh, N, l, ldvh};
+    EpiX epi{h->logits, h->u, h->vh, N, l, ldvh, h->uq, h->usf, h->g_u};
     LMOE_STEP(0, launch_gemm_bn(p.bn, h->tm_wx, tm_x, s, epi, grid, h->err, lim, st));
     if (p.ksplit > 1)
       LMOE_STEP(10, launch_reduce(h->part, p.ksplit, static_cast<int>(T), N + l + hs, epi, st));
@@ -549,7 +734,26 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   LMOE_STEP(3, launch_scan(h->chunk, T, N, h->counts, st));
   LMOE_STEP(4, launch_scatter(h->topk_idx, h->topk_w, h->chunk, h->counts, T, N, K, gbn,
                               h->offsets, h->perm, h->inv, h->wrow, h->blocks, h->nblocks,
-                              h->err, st));
+                              h->rblock, h->err, st));
+  if (h->fp4) {
+    // 6. quantised latent rows (and their scales) into expert order
+    LMOE_STEP(5, launch_gather_q(h->uq, h->usf, h->perm, h->rblock, T * K, K, l, h->lp, h->upq,
+                                 h->sfbu, st));
+    // 7. H = NVFP4(sqrelu(W1[e] u)), block-scaled FP4 MMA
+    {
+      TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, h->lp / 256, 1, nullptr,
+                   gbn == 32, h->w1sf, h->sfbu, h->lp / 64};
+      EpiHq epi{h->Hq, h->sfbh, h->gw1, h->g_u, h->g_h, h->hp};
+      LMOE_STEP(6, launch_gemm_fp4(gbn, h->tm_w1q, h->tm_upq, s, epi, h->sms, h->err, lim, st));
+    }
+    // 8. O = w * W2[e] H, block-scaled FP4 MMA
+    {
+      TileSource s{0, 0, h->blocks, h->nblocks, l / 128, l, l, h->hp / 256, 1, nullptr,
+                   gbn == 32, h->w2sf, h->sfbh, h->hp / 64};
+      EpiOq epi{h->O, h->wrow, h->gw2, h->g_h, l};
+      LMOE_STEP(7, launch_gemm_fp4(gbn, h->tm_w2q, h->tm_Hq, s, epi, h->sms, h->err, lim, st));
+    }
+  } else {
   // 6. latent rows into expert order
   LMOE_STEP(5, launch_gather(h->u, h->perm, T * K, K, l, h->u_perm, st));
   // 7. H = sqrelu(W1[e] u)
@@ -565,6 +769,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
                  gbn == 32};
     EpiO epi{h->O, h->wrow, l};
     LMOE_STEP(7, launch_gemm_bn(gbn, h->tm_w2, h->tm_H, s, epi, h->sms, h->err, lim, st));
+  }
   }
   // 9. v = sum_k O[inv[t][k]]
   LMOE_STEP(8, launch_combine(h->O, h->inv, T, K, l, h->vh, ldvh, st));
@@ -636,8 +841,15 @@ int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
     case LMOE_DBG_U: src = h->u; want = T * l * 2; break;
     case LMOE_DBG_V: strided = true; col0 = 0; cols = l; want = T * l * 2; break;
     case LMOE_DBG_HS: strided = true; col0 = l; cols = hs; want = T * hs * 2; break;
+    case LMOE_DBG_W1Q_CODES: src = h->w1q; want = N * c.expert_hidden * h->lp / 2; break;
+    case LMOE_DBG_W1Q_SF: src = h->w1sf; want = (N * c.expert_hidden / 128) * (h->lp / 64) * 512; break;
+    case LMOE_DBG_W1Q_G: src = h->gw1; want = N * 4; break;
+    case LMOE_DBG_W2Q_CODES: src = h->w2q; want = N * l * h->hp / 2; break;
+    case LMOE_DBG_W2Q_SF: src = h->w2sf; want = (N * l / 128) * (h->hp / 64) * 512; break;
+    case LMOE_DBG_W2Q_G: src = h->gw2; want = N * 4; break;
     default: return LMOE_ERR_INVALID_ARG;
   }
+  if (what >= LMOE_DBG_W1Q_CODES && !h->fp4) return LMOE_ERR_INVALID_ARG;
   if (bytes != want) return LMOE_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return LMOE_ERR_CUDA;
   if (want == 0) return LMOE_OK;
@@ -734,9 +946,23 @@ int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int
       launch_hist(topk_idx, T, N, K, chunk, err, st) != cudaSuccess ||
       launch_scan(chunk, T, N, counts, st) != cudaSuccess ||
       launch_scatter(topk_idx, topk_w, chunk, counts, T, N, K, 256, offsets, perm, inv, wrow,
-                     blocks, nblocks, err, st) != cudaSuccess)
+                     blocks, nblocks, nullptr, err, st) != cudaSuccess)
     return LMOE_ERR_CUDA;
   return LMOE_OK;
+}
+
+int lmoe_nvfp4_quantize(const float* x, int64_t rows, int32_t cols, float g, uint8_t* codes,
+                        uint8_t* scales, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 16 || !(g >= 0.0f && g < 3.0e38f))
+    return LMOE_ERR_INVALID_ARG;
+  if (rows == 0) return LMOE_OK;
+  if (!x || !codes || !scales || (reinterpret_cast<uintptr_t>(x) & 15) ||
+      (reinterpret_cast<uintptr_t>(codes) & 7))
+    return LMOE_ERR_INVALID_ARG;
+  return launch_quant_rows(x, rows, cols, g, codes, scales, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? LMOE_OK
+             : LMOE_ERR_CUDA;
 }
 
 int lmoe_check_bounded_wait(int64_t limit_ns) {

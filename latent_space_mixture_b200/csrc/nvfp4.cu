@@ -1,0 +1,162 @@
+// NVFP4 kernels of the LatentMoE expert path: quantisation of the expert
+// weights at layer creation (per-expert FP32 global scale, E4M3 block scales,
+// E2M1 codes), a standalone row quantiser, and the gather of quantised
+// latent rows into expert order.  Format: "NVIDIA Nemotron 3: Efficient and
+// Open Intelligence", section 三 "NVFP4 训练"; "Nemotron-3 Super 精读报告",
+// section 5.3 (blocks along the GEMM reduction axis).
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "nvfp4.cuh"
+
+namespace lmoe {
+
+// amax[e] = max |W[e]| over a [E][rows_per][K] bf16 tensor (amax pre-zeroed;
+// non-negative floats order like their bit patterns, so atomicMax on ints).
+__global__ void __launch_bounds__(256) k_amax_expert(const __nv_bfloat16* __restrict__ w,
+                                                     int64_t per_expert, float* amax) {
+  const int e = blockIdx.y;
+  const __nv_bfloat162* p =
+      reinterpret_cast<const __nv_bfloat162*>(w + static_cast<int64_t>(e) * per_expert);
+  const int64_t n2 = per_expert / 2;
+  float m = 0.0f;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n2;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float2 f = __bfloat1622float2(p[i]);
+    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  __shared__ float wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.0f;
+    for (int i = 0; i < 8; ++i) b = fmaxf(b, wm[i]);
+    atomicMax(reinterpret_cast<int*>(amax + e), __float_as_int(b));
+  }
+}
+
+// One thread per (row, 16-element block) of a [E * rows_per][K] bf16 matrix:
+// codes into [row][Kp/2] bytes, scale into the 512-byte atoms
+// [row / 128][Kp / 64], global scale g[e] = amax[e] / (6 * 448).
+__global__ void __launch_bounds__(256) k_quant_weight(const __nv_bfloat16* __restrict__ w,
+                                                      int64_t rows, int rows_per, int K, int Kp,
+                                                      const float* __restrict__ amax,
+                                                      uint8_t* __restrict__ codes,
+                                                      uint8_t* __restrict__ atoms,
+                                                      float* __restrict__ gscale) {
+  const int kb16 = K / 16;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * kb16) return;
+  const int64_t row = i / kb16;
+  const int blk = static_cast<int>(i - row * kb16);
+  const int e = static_cast<int>(row / rows_per);
+  const float g = __fdiv_rn(amax[e], 6.0f * 448.0f);
+  if (blk == 0 && row % rows_per == 0) gscale[e] = g;
+  float x[16];
+  const __nv_bfloat162* src = reinterpret_cast<const __nv_bfloat162*>(w + row * K + blk * 16);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float2 f = __bfloat1622float2(src[j]);
+    x[2 * j] = f.x;
+    x[2 * j + 1] = f.y;
+  }
+  uint8_t q[8];
+  const uint8_t sc = nvfp4_block(x, g, q);
+  uint8_t* dst = codes + row * (Kp / 2) + blk * 8;
+  *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(q);
+  const int kc = blk / 4, k1 = blk % 4;
+  atoms[((row / 128) * (Kp / 64) + kc) * SF_ATOM_BYTES + sf_atom_offset(static_cast<int>(row % 128), k1)] = sc;
+}
+
+cudaError_t launch_quant_weights(const void* w, int E, int rows_per, int K, int Kp, float* amax,
+                                 uint8_t* codes, uint8_t* atoms, float* gscale, cudaStream_t st) {
+  if (cudaMemsetAsync(amax, 0, E * sizeof(float), st) != cudaSuccess) return cudaGetLastError();
+  const int64_t per = static_cast<int64_t>(rows_per) * K;
+  k_amax_expert<<<dim3(64, E), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), per, amax);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t rows = static_cast<int64_t>(E) * rows_per;
+  const int64_t n = rows * (K / 16);
+  k_quant_weight<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w), rows, rows_per, K, Kp, amax, codes, atoms, gscale);
+  return cudaGetLastError();
+}
+
+// Row quantiser with canonical outputs: codes [rows][cols/2], scales [rows][cols/16].
+__global__ void __launch_bounds__(256) k_quant_rows(const float* __restrict__ x, int64_t rows,
+                                                    int cols, float g, uint8_t* __restrict__ codes,
+                                                    uint8_t* __restrict__ scales) {
+  const int nb = cols / 16;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * nb) return;
+  const int64_t row = i / nb;
+  const int blk = static_cast<int>(i - row * nb);
+  float v[16];
+  const float4* src = reinterpret_cast<const float4*>(x + row * cols + blk * 16);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float4 f = src[j];
+    v[4 * j] = f.x;
+    v[4 * j + 1] = f.y;
+    v[4 * j + 2] = f.z;
+    v[4 * j + 3] = f.w;
+  }
+  uint8_t q[8];
+  scales[row * nb + blk] = nvfp4_block(v, g, q);
+  *reinterpret_cast<uint2*>(codes + row * (cols / 2) + blk * 8) = *reinterpret_cast<const uint2*>(q);
+}
+
+cudaError_t launch_quant_rows(const float* x, int64_t rows, int cols, float g, uint8_t* codes,
+                              uint8_t* scales, cudaStream_t st) {
+  const int64_t n = rows * (cols / 16);
+  if (n <= 0) return cudaSuccess;
+  k_quant_rows<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(x, rows, cols, g, codes,
+                                                                        scales);
+  return cudaGetLastError();
+}
+
+// Quantised latent rows into expert order: codes u_q[tok] -> u_perm_q[r]
+// (row pitch Kp/2 bytes) and the row's scales [tok][l/16] into the B-operand
+// atoms of its token block: atom (block, kc), row j of the block.
+__global__ void __launch_bounds__(256) k_gather_q(const uint8_t* __restrict__ uq,
+                                                  const uint8_t* __restrict__ usf,
+                                                  const int32_t* __restrict__ perm,
+                                                  const int32_t* __restrict__ rblock, int64_t rows,
+                                                  int K, int l, int lp,
+                                                  uint8_t* __restrict__ u_perm_q,
+                                                  uint8_t* __restrict__ atoms) {
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int c16 = l / 32;   // 16-byte chunks of codes per row
+  const int kc = l / 64;    // 64-element chunks (4 scales each)
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += nwarps) {
+    const int64_t tok = perm[r] / K;
+    const uint4* src = reinterpret_cast<const uint4*>(uq + tok * (l / 2));
+    uint4* dst = reinterpret_cast<uint4*>(u_perm_q + r * (lp / 2));
+    for (int i = lane; i < c16; i += 32) dst[i] = src[i];
+    const int rb = rblock[r];
+    const int b = rb >> 8, j = rb & 255;
+    const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(usf + tok * (l / 16));
+    for (int c = lane; c < kc; c += 32) {
+      const int64_t off = (static_cast<int64_t>(b) * (lp / 64) + c) * SF_ATOM_BYTES +
+                          (j & 31) * 16 + ((j >> 5) & 3) * 4;
+      *reinterpret_cast<uint32_t*>(atoms + off) = ssrc[c];
+    }
+  }
+}
+
+cudaError_t launch_gather_q(const uint8_t* uq, const uint8_t* usf, const int32_t* perm,
+                            const int32_t* rblock, int64_t rows, int K, int l, int lp,
+                            uint8_t* u_perm_q, uint8_t* atoms, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  int64_t blocks = (rows + 7) / 8;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_gather_q<<<static_cast<unsigned>(blocks), 256, 0, st>>>(uq, usf, perm, rblock, rows, K, l, lp,
+                                                            u_perm_q, atoms);
+  return cudaGetLastError();
+}
+
+}  // namespace lmoe

@@ -1,0 +1,67 @@
+// NVFP4 on the device: E2M1 elements, 16-element micro-blocks along the GEMM
+// reduction axis, E4M3 block scales, FP32 global scale ("NVIDIA Nemotron 3:
+// Efficient and Open Intelligence", section 三 "NVFP4 训练"; "Nemotron-3 Super
+// 精读报告", section 5.3).  Rounding is round-to-nearest-even with saturation
+// (the cvt instructions below), the scale arithmetic IEEE float32 in a fixed
+// order so that the codes are reproducible:
+//   six_g = 6 g; sbf = amax / six_g; s = E4M3(sbf); denom = s g;
+//   r = 1 / denom (rounded once per block); q = E2M1(x * r), or 0 when
+//   denom == 0.
+//
+// Scale-factor layout consumed by tcgen05.mma ... block_scale (block16): an
+// "atom" of 512 bytes covers 128 rows x 64 reduction elements (4 scales per
+// row); the scale of row m (0..127) and 16-block k1 (0..3) is byte
+// (m % 32) * 16 + (m / 32) * 4 + k1.  A matrix's atoms are stored with the
+// 64-wide reduction chunk fastest.
+#pragma once
+#include <cuda_fp8.h>
+#include <cstdint>
+
+namespace lmoe {
+
+constexpr int NVFP4_BLOCK = 16;
+constexpr int SF_ATOM_BYTES = 512;
+
+__device__ __forceinline__ int sf_atom_offset(int m, int k1) {
+  return (m & 31) * 16 + ((m >> 5) & 3) * 4 + k1;
+}
+
+// Two floats to two E2M1 codes in one byte: `lo` in bits 0-3, `hi` in bits 4-7
+// (the lower reduction index in the lower nibble).
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u16.u8 %0, t;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ uint8_t e4m3_code(float x) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ float e4m3_value(uint8_t code) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// Quantise one 16-element block: returns the E4M3 scale code and writes the 8
+// packed bytes of codes.
+__device__ __forceinline__ uint8_t nvfp4_block(const float (&x)[16], float g, uint8_t (&out)[8]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  const float six_g = __fmul_rn(6.0f, g);
+  const float sbf = six_g > 0.0f ? __fdiv_rn(amax, six_g) : 0.0f;
+  const uint8_t sc = e4m3_code(sbf);
+  const float denom = __fmul_rn(e4m3_value(sc), g);
+  const float r = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    out[i] = static_cast<uint8_t>(e2m1x2(__fmul_rn(x[2 * i], r), __fmul_rn(x[2 * i + 1], r)));
+  return sc;
+}
+
+}  // namespace lmoe

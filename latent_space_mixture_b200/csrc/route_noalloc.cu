@@ -92,7 +92,7 @@ extern "C" int lmoe_route_noalloc(const float* logits, const float* bias, int64_
       lmoe::launch_hist(topk_idx, T, N, K, chunk, err, st) != cudaSuccess ||
       lmoe::launch_scan(chunk, T, N, counts, st) != cudaSuccess ||
       lmoe::launch_scatter(topk_idx, topk_w, chunk, counts, T, N, K, kBlockRows, offsets, perm,
-                           inv, wrow, blocks, nblocks, err, st) != cudaSuccess)
+                           inv, wrow, blocks, nblocks, nullptr, err, st) != cudaSuccess)
     return LMOE_ERR_CUDA;
   return LMOE_OK;
 }

@@ -232,10 +232,11 @@ __global__ void __launch_bounds__(256) k_scatter(
     const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ counts, int64_t T, int N,
     int K, int bn, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
     int32_t* __restrict__ inv, float* __restrict__ wrow, int4* __restrict__ blocks,
-    int32_t* __restrict__ nblocks, int* err) {
+    int32_t* __restrict__ nblocks, int32_t* __restrict__ rblock, int* err) {
   extern __shared__ int32_t sc_smem[];
   int32_t* off = sc_smem;                                    // [N + 1]
-  uint32_t* masks = reinterpret_cast<uint32_t*>(off + N + 1);  // [8][N]
+  int32_t* bbase = off + N + 1;                              // [N]
+  uint32_t* masks = reinterpret_cast<uint32_t*>(bbase + N);  // [8][N]
   __shared__ int wsum[16];
   __shared__ int total;
 
@@ -257,25 +258,30 @@ __global__ void __launch_bounds__(256) k_scatter(
   if (threadIdx.x == 0) off[N] = total;
   __syncthreads();
 
+  // token blocks of at most bn rows per expert, in expert order
+  int nb4[4];
+  int snb = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    nb4[i] = (c4[i] + bn - 1) / bn;
+    snb += nb4[i];
+  }
+  int bb = block_excl_scan_256(snb, wsum, &total);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (e4 + i < N) bbase[e4 + i] = bb;
+    bb += nb4[i];
+  }
+  __syncthreads();
   if (blockIdx.x == 0) {
     for (int e = threadIdx.x; e <= N; e += blockDim.x) offsets[e] = off[e];
-    // token blocks of at most bn rows per expert, in expert order
-    int nb4[4];
-    int snb = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      nb4[i] = (c4[i] + bn - 1) / bn;
-      snb += nb4[i];
-    }
-    int bbase = block_excl_scan_256(snb, wsum, &total);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int e = e4 + i;
       for (int j = 0; j < nb4[i]; ++j) {
         const int r0 = j * bn;
-        blocks[bbase + j] = make_int4(e, off[e] + r0, min(bn, c4[i] - r0), 0);
+        blocks[bbase[e] + j] = make_int4(e, off[e] + r0, min(bn, c4[i] - r0), 0);
       }
-      bbase += nb4[i];
     }
     if (threadIdx.x == 0) *nblocks = total;
   }
@@ -304,10 +310,13 @@ __global__ void __launch_bounds__(256) k_scatter(
     for (int k = 0; k < 32; ++k) {
       const int e = ek[k];
       if (k < K && e >= 0 && e < N) {
-        const int row = off[e] + base[k] + __popc(m[e] & lower);
+        const int rank = base[k] + __popc(m[e] & lower);
+        const int row = off[e] + rank;
         inv[t * K + k] = row;
         perm[row] = static_cast<int32_t>(t * K + k);
         wrow[row] = wk[k];
+        // token block of the row and its index inside the block (bn <= 256)
+        if (rblock) rblock[row] = ((bbase[e] + rank / bn) << 8) | (rank % bn);
       }
     }
   }
@@ -316,12 +325,13 @@ __global__ void __launch_bounds__(256) k_scatter(
 cudaError_t launch_scatter(const int32_t* topk_idx, const float* topk_w, const int32_t* chunk_base,
                            const int32_t* counts, int64_t T, int N, int K, int bn,
                            int32_t* offsets, int32_t* perm, int32_t* inv, float* wrow,
-                           int4* blocks, int32_t* nblocks, int* err, cudaStream_t st) {
+                           int4* blocks, int32_t* nblocks, int32_t* rblock, int* err,
+                           cudaStream_t st) {
   const int64_t nchunks = (T + 31) / 32;
   const unsigned nblk = static_cast<unsigned>(nchunks > 0 ? (nchunks + 7) / 8 : 1);
-  const size_t smem = (N + 1) * sizeof(int32_t) + 8 * N * sizeof(uint32_t);
+  const size_t smem = (2 * N + 1) * sizeof(int32_t) + 8 * N * sizeof(uint32_t);
   k_scatter<<<nblk, 256, smem, st>>>(topk_idx, topk_w, chunk_base, counts, T, N, K, bn, offsets,
-                                     perm, inv, wrow, blocks, nblocks, err);
+                                     perm, inv, wrow, blocks, nblocks, rblock, err);
   return cudaGetLastError();
 }
 

@@ -110,7 +110,19 @@ class LatentMoE:
             "perm": (torch.int32, (T * c.top_k,)), "inv": (torch.int32, (T, c.top_k)),
             "logits": (torch.float32, (T, c.n_experts)), "u": (torch.bfloat16, (T, c.latent)),
             "v": (torch.bfloat16, (T, c.latent)), "hs": (torch.bfloat16, (T, c.shared_hidden)),
-        }[what]
+        }
+        lp = (c.latent + 255) // 256 * 256
+        hp = (c.expert_hidden + 255) // 256 * 256
+        N, h, l = c.n_experts, c.expert_hidden, c.latent
+        spec.update({
+            "w1q_codes": (torch.uint8, (N * h, lp // 2)),
+            "w1q_sf": (torch.uint8, ((N * h // 128) * (lp // 64) * 512,)),
+            "w1q_g": (torch.float32, (N,)),
+            "w2q_codes": (torch.uint8, (N * l, hp // 2)),
+            "w2q_sf": (torch.uint8, ((N * l // 128) * (hp // 64) * 512,)),
+            "w2q_g": (torch.float32, (N,)),
+        })
+        spec = spec[what]
         out = torch.empty(spec[1], dtype=spec[0])
         check(self.lib.lmoe_get_debug(self.h, DBG[what], c_void_p(out.data_ptr()),
                                       out.numel() * out.element_size()), f"debug {what}")

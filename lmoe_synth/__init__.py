@@ -68,6 +68,12 @@ CONFIGS: Dict[str, LayerConfig] = {
     # the prefill batch), Zipf bias: a small prefill case for profiler captures
     "super_prefill_n64": LayerConfig("super_prefill_n64", 1024, 4096, 1024, 64, 22, 2688,
                                      5376, 0.02, "zipf", 6),
+    # tiny layer with NVFP4 experts (latent and expert hidden multiples of 128)
+    "tiny_nvfp4": LayerConfig("tiny_nvfp4", 64, 256, 128, 32, 4, 256, 256, 0.02, "zipf", 7,
+                              "nvfp4"),
+    # the small prefill case with NVFP4 experts, for profiler captures
+    "super_prefill_nvfp4_n64": LayerConfig("super_prefill_nvfp4_n64", 1024, 4096, 1024, 64, 22,
+                                           2688, 5376, 0.02, "zipf", 8, "nvfp4"),
     # Super dims prefill with NVFP4 experts, Zipf(1.1) router bias
     "super_prefill_nvfp4": LayerConfig("super_prefill_nvfp4", 8192, 4096, 1024,
                                        512, 22, 2688, 5376, 0.02, "zipf", 4,

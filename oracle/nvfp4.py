@@ -18,12 +18,15 @@ Readings (the pages fix the format, not the scale arithmetic):
   * blocks are 16 consecutive elements along the last axis, which the caller
     makes the GEMM reduction axis;
   * block scale s_b = E4M3_rtne_satfinite(amax_b / (6 g)), element
-    q = E2M1_rtne_satfinite(x / (s_b g)), value q * s_b * g;
+    q = E2M1_rtne_satfinite(x * r_b) with r_b = 1 / (s_b g) rounded once
+    per block (a reciprocal per block rather than a division per element),
+    value q * s_b * g;
   * a weight matrix's global scale is g_W = amax(W) / (6 * 448);
   * all scale and element arithmetic is IEEE float32 in exactly this order,
     so that two implementations of it produce identical codes:
         six_g = f32(6 * g); sbf = f32(amax / six_g); s_b = e4m3(sbf);
-        denom = f32(s_b * g); q = e2m1(f32(x / denom)), or 0 when denom == 0;
+        denom = f32(s_b * g); r = f32(1 / denom), or 0 when denom == 0;
+        q = e2m1(f32(x * r)) (a zero-scale block gives +-0 codes);
   * weights use the same 1D max-based blocks as activations (the pages'
     training recipe uses 2D weight blocks and their PTQ an MSE search; both
     are left out of this oracle).
@@ -136,10 +139,11 @@ def quantize(X: np.ndarray, g) -> tuple:
     sb = e4m3_decode(sc).astype(np.float32)
     denom = (sb * g32).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
-        ratio = (blocks / denom[..., None]).astype(np.float32)
-    ratio = np.where(denom[..., None] > 0, ratio, np.float32(0.0))
-    codes = e2m1_rtne(ratio)
-    codes = np.where(denom[..., None] > 0, codes, np.uint8(0)).astype(np.uint8)
+        rcp = (np.float32(1.0) / denom).astype(np.float32)
+    rcp = np.where(denom > 0, rcp, np.float32(0.0)).astype(np.float32)
+    ratio = (blocks * rcp[..., None]).astype(np.float32)
+    # a block whose scale is 0 gives x * 0 = +-0: value 0, sign kept (IEEE)
+    codes = e2m1_rtne(ratio).astype(np.uint8)
     return codes.reshape(Xf.shape), sc, sb
 
 

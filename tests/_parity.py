@@ -46,9 +46,20 @@ def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None):
     if overrides:
         for k, fn in overrides.items():
             w[k] = fn(w[k])
+    from lmoe_synth import act_global_scales
     layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs,
-                      max_tokens or x.shape[0], w)
+                      max_tokens or x.shape[0], w, expert_format=cfg.fmt,
+                      act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0))
     return w, x, layer
+
+
+def quant_of(cfg):
+    """The oracle's quantisation settings for a workload (None for BF16)."""
+    from lmoe_synth import act_global_scales
+    if cfg.fmt != "nvfp4":
+        return None
+    g_u, g_h = act_global_scales(cfg)
+    return {"g_u": float(np.float32(g_u)), "g_h": float(np.float32(g_h))}
 
 
 def oracle_tokens(w, x_rows: torch.Tensor, K: int, quant=None):
@@ -88,7 +99,8 @@ def elem_ok(a: np.ndarray, ref: np.ndarray, rel=REL_ELEM, abs_rms=ABS_RMS, rel_r
     return ratio <= 1.0 and rr <= rel_rms, ratio, rr
 
 
-def compare_layer(layer, w, x, y, tokens, K, tol=TOL_BF16, quant=None, elem_rel=REL_ELEM):
+def compare_layer(layer, w, x, y, tokens, K, tol=TOL_BF16, quant=None, elem_rel=REL_ELEM,
+                  check_v=True):
     """Compare the last forward of `layer` (x -> y) with the oracle on `tokens`.
 
     Returns a dict of measured errors; asserts the bar.  Near-tie tokens whose
@@ -130,7 +142,8 @@ def compare_layer(layer, w, x, y, tokens, K, tol=TOL_BF16, quant=None, elem_rel=
         errs[k + "_maxerr_over_rms"] = max_rel(got[k], ref[k])
         errs[k + "_err_over_bound"] = ratio
         errs[k + "_rms_rel"] = rr
-        assert ok, f"{k}: elementwise error {ratio:.3g} x bound, RMS rel error {rr:.3g}"
+        if k != "v" or check_v:
+            assert ok, f"{k}: elementwise error {ratio:.3g} x bound, RMS rel error {rr:.3g}"
     assert errs["y_maxerr_over_rms"] <= tol, \
         f"y: max|err|/RMS = {errs['y_maxerr_over_rms']:.3g} > {tol}"
     return errs

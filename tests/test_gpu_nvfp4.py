@@ -1,0 +1,115 @@
+"""NVFP4 expert path on the GPU against the oracle: the quantiser bit-exact,
+the quantised weights bit-exact, and the layer with identical quantisation
+within the NVFP4 bar (max|err| <= 6e-2 RMS(y))."""
+from ctypes import c_float, c_void_p
+
+import numpy as np
+import pytest
+import torch
+
+from lmoe_synth import CONFIGS
+from oracle import nvfp4 as Q
+
+from _parity import check_segments_valid, compare_layer, make, quant_of, rms_rel, to64
+
+pytestmark = pytest.mark.gpu
+TOL_NVFP4 = 6e-2
+
+
+def _gpu_quantize(x: torch.Tensor, g: float):
+    from latent_space_mixture_b200 import _lib
+    lib = _lib.load()
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
+    rc = lib.lmoe_nvfp4_quantize(c_void_p(x.data_ptr()), rows, cols, c_float(g),
+                                 c_void_p(codes.data_ptr()), c_void_p(scales.data_ptr()),
+                                 c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert rc == 0
+    return codes.cpu().numpy(), scales.cpu().numpy()
+
+
+def _unpack(codes_bytes):
+    lo = codes_bytes & 0x0F
+    hi = codes_bytes >> 4
+    return np.stack([lo, hi], axis=-1).reshape(codes_bytes.shape[0], -1)
+
+
+def test_quantizer_bit_exact_against_oracle():
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal((257, 512)) * np.exp(rng.uniform(-6, 6, (257, 1)))).astype(np.float32)
+    x[3, :16] = 0.0                                   # an all-zero block
+    x[4, :16] = -0.0
+    x[5, 16:32] = rng.choice([0.25, 0.75, 1.25, 2.5, -5.0], 16)   # E2M1 ties at s*g = 1
+    x[6, :] = 1e-30                                   # scale underflow
+    g = float(np.float32(np.abs(x).max() / 2688.0))
+    codes, scales = _gpu_quantize(torch.from_numpy(x).cuda(), g)
+    oc, osc, _ = Q.quantize(x, g)
+    assert np.array_equal(scales, osc)
+    got = _unpack(codes)
+    # +0 and -0 codes are both zero values; compare values and codes
+    assert np.array_equal(Q.e2m1_decode(got), Q.e2m1_decode(oc))
+    assert np.array_equal(got, oc)
+
+
+def _weights_from_atoms(codes, atoms, rows, K, Kp):
+    q = _unpack(codes)[:, :K]
+    sc = np.empty((rows, K // 16), dtype=np.uint8)
+    r = np.arange(rows)[:, None]
+    b = np.arange(K // 16)[None, :]
+    off = ((r // 128) * (Kp // 64) + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4
+    sc[:, :] = atoms[off]
+    return q, sc
+
+
+def test_quantised_weights_bit_exact():
+    cfg = CONFIGS["tiny_nvfp4"]
+    w, x, layer = make(cfg)
+    lp, hp = (cfg.l + 255) // 256 * 256, (cfg.h + 255) // 256 * 256
+    for name, R, K, Kp in (("w1", cfg.h, cfg.l, lp), ("w2", cfg.l, cfg.h, hp)):
+        codes = layer.debug(name + "q_codes").numpy()
+        atoms = layer.debug(name + "q_sf").numpy()
+        g = layer.debug(name + "q_g").numpy()
+        q, sc = _weights_from_atoms(codes, atoms, cfg.N * R, K, Kp)
+        for e in range(cfg.N):
+            We = w[name][e].float().cpu().numpy()
+            ge = Q.weight_global_scale(We)
+            assert g[e] == ge
+            oc, osc, _ = Q.quantize(We, ge)
+            assert np.array_equal(sc[e * R:(e + 1) * R], osc), (name, e)
+            assert np.array_equal(Q.e2m1_decode(q[e * R:(e + 1) * R]), Q.e2m1_decode(oc)), (name, e)
+        # padding beyond K holds zero codes
+        assert np.all(_unpack(codes)[:, K:] == 0)
+    layer.close()
+
+
+@pytest.mark.parametrize("T", [64, 37, 5])
+def test_tiny_nvfp4_layer(T):
+    cfg = CONFIGS["tiny_nvfp4"]
+    w, x, layer = make(cfg, T=T)
+    y = layer.forward(x)
+    torch.cuda.synchronize()
+    assert layer.sync_status() == 0
+    errs = compare_layer(layer, w, x, y, np.arange(T), cfg.K, tol=TOL_NVFP4, quant=quant_of(cfg),
+                         elem_rel=2.0 ** -7, check_v=False)
+    print("tiny_nvfp4", T, errs)
+    assert errs["v_rms_rel"] <= TOL_NVFP4
+    layer.close()
+
+
+def test_super_prefill_nvfp4_sampled_tokens():
+    cfg = CONFIGS["super_prefill_nvfp4"]
+    w, x, layer = make(cfg)
+    y = layer.forward(x)
+    torch.cuda.synchronize()
+    assert layer.sync_status() == 0
+    counts = check_segments_valid(layer, cfg.T, cfg.N, cfg.K)
+    assert (counts == 0).any()
+    rng = np.random.default_rng(1000 + cfg.seed)
+    toks = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 10, replace=False)]))
+    errs = compare_layer(layer, w, x, y, toks, cfg.K, tol=TOL_NVFP4, quant=quant_of(cfg),
+                         check_v=False)
+    print("super_prefill_nvfp4", errs)
+    assert errs["v_rms_rel"] <= TOL_NVFP4
+    layer.close()
