@@ -173,10 +173,31 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       // weights read once per launch are streamed past L2; weights that
       // several token blocks share are left to the default policy
       const uint64_t pol_a = src.a_stream_once ? policy_evict_first() : policy_evict_last();
+      // B operand (and its scales) of one k-step: it depends on the previous
+      // kernel; A (weights, and their scales) does not
+      auto load_b = [&](int st, const TileInfo& t, int kb) {
+        const int nbig = t.nrows / GEMM_BROWS_BIG;
+        const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
+        const int bx = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+        uint8_t* b_dst = sB + st * L::B_BYTES;
+        for (int j = 0; j < nbig; ++j)
+          tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
+                      t.row0 + j * GEMM_BROWS_BIG, &full[st]);
+        for (int j = 0; j < nsmall; ++j) {
+          const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
+          tma_load_2d(b_dst + r * GEMM_ROW_BYTES, &tmB, bx, t.row0 + r, &full[st]);
+        }
+        if constexpr (FP4)
+          bulk_load(sSF + st * L::SF_BYTES + FP4_SF_STAGE_BYTES,
+                    src.sfb + (static_cast<long>(t.tb) * src.kc + kb * 4) * SF_ATOM_BYTES,
+                    FP4_SF_STAGE_BYTES, &full[st]);
+      };
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
+      bool waited = false;   // pdl_wait done; before it only A loads are issued
+      int deferred = 0;      // k-steps of the first tile whose B loads wait for it
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const TileInfo t = gemm_tile(src, BN, tile);
         // B rows: 64-row boxes while 64 rows remain, then 16-row boxes
@@ -191,24 +212,22 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           }
           mbar_arrive_expect_tx(&full[stage], tx);
           // x coordinate in elements of the map: bf16 elements or bytes (NVFP4)
-          const int bx = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
-          tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, bx, t.a_row, &full[stage], pol_a);
-          uint8_t* b_dst = sB + stage * L::B_BYTES;
-          for (int j = 0; j < nbig; ++j)
-            tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
-                        t.row0 + j * GEMM_BROWS_BIG, &full[stage]);
-          for (int j = 0; j < nsmall; ++j) {
-            const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
-            tma_load_2d(b_dst + r * GEMM_ROW_BYTES, &tmB, bx, t.row0 + r, &full[stage]);
-          }
-          if constexpr (FP4) {
-            uint8_t* sf = sSF + stage * L::SF_BYTES;
-            bulk_load(sf, src.sfa + (static_cast<long>(t.a_row / GEMM_BM) * src.kc + kb * 4) *
-                                        SF_ATOM_BYTES,
+          const int ax = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+          tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, ax, t.a_row, &full[stage], pol_a);
+          if constexpr (FP4)
+            bulk_load(sSF + stage * L::SF_BYTES,
+                      src.sfa + (static_cast<long>(t.a_row / GEMM_BM) * src.kc + kb * 4) *
+                                    SF_ATOM_BYTES,
                       FP4_SF_STAGE_BYTES, &full[stage]);
-            bulk_load(sf + FP4_SF_STAGE_BYTES,
-                      src.sfb + (static_cast<long>(t.tb) * src.kc + kb * 4) * SF_ATOM_BYTES,
-                      FP4_SF_STAGE_BYTES, &full[stage]);
+          if (waited) {
+            load_b(stage, t, kb);
+          } else if (++deferred == STAGES || kb + 1 == t.kb1) {
+            // the first tile's first stages: weights are in flight, now the
+            // previous kernel's results
+            pdl_wait();
+            pdl_trigger();
+            waited = true;
+            for (int j = 0; j < deferred; ++j) load_b(j, t, t.kb0 + j);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -216,6 +235,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             phase ^= 1;
           }
         }
+      }
+      if (!waited) {
+        pdl_wait();
+        pdl_trigger();
       }
       if (!ok) {
         // let the copies already issued land before the CTA's smem goes away
@@ -367,6 +390,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 template <class Epi>
 __global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ part, int ksplit,
                                                        int T, int F, const Epi epi) {
+  pdl_wait();
+  pdl_trigger();
   const long g = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int f8 = F / 8;
   const long row = g / f8;

@@ -1,0 +1,28 @@
+// Kernel launch with programmatic stream serialisation (programmatic
+// dependent launch): the kernel may begin while its predecessor on the stream
+// finishes; it synchronises with pdl_wait() (ptx.cuh) before reading the
+// predecessor's results.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <utility>
+
+namespace lmoe {
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+}  // namespace lmoe

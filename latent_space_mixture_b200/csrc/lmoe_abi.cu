@@ -12,6 +12,7 @@
 
 #include "gemm_tc.cuh"
 #include "kernels.h"
+#include "launch.cuh"
 #include "lmoe.h"
 
 using bf16 = __nv_bfloat16;
@@ -184,9 +185,8 @@ cudaError_t launch_gemm(const CUtensorMap& A, const BMaps& B, const TileSource& 
                         const Epi& epi, int grid, int* err, unsigned long long limit,
                         cudaStream_t st) {
   using L = GemmLayout<BN, Stages<BN, FP4>::value, FP4>;
-  k_gemm_tc<BN, Stages<BN, FP4>::value, Epi, FP4>
-      <<<grid, GEMM_THREADS, L::SMEM_BYTES, st>>>(A, B.b16, B.b64, src, epi, err, limit);
-  return cudaGetLastError();
+  return launch_pdl(k_gemm_tc<BN, Stages<BN, FP4>::value, Epi, FP4>, grid, GEMM_THREADS,
+                    L::SMEM_BYTES, st, A, B.b16, B.b64, src, epi, err, limit);
 }
 
 template <class Epi>
@@ -213,8 +213,7 @@ cudaError_t launch_reduce(const float* part, int ksplit, int T, int F, const Epi
                           cudaStream_t st) {
   const long threads = static_cast<long>(T) * (F / 8);
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
-  k_splitk_reduce<Epi><<<blocks, 256, 0, st>>>(part, ksplit, T, F, epi);
-  return cudaGetLastError();
+  return launch_pdl(k_splitk_reduce<Epi>, blocks, 256, 0, st, part, ksplit, T, F, epi);
 }
 
 template <class Epi>

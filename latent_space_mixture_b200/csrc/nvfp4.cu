@@ -7,7 +7,9 @@
 #include <cuda_bf16.h>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "nvfp4.cuh"
+#include "ptx.cuh"
 
 namespace lmoe {
 
@@ -127,6 +129,8 @@ __global__ void __launch_bounds__(256) k_gather_q(const uint8_t* __restrict__ uq
                                                   int K, int l, int lp,
                                                   uint8_t* __restrict__ u_perm_q,
                                                   uint8_t* __restrict__ atoms) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
   const int c16 = l / 32;   // 16-byte chunks of codes per row
@@ -154,9 +158,8 @@ cudaError_t launch_gather_q(const uint8_t* uq, const uint8_t* usf, const int32_t
   if (rows <= 0) return cudaSuccess;
   int64_t blocks = (rows + 7) / 8;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  k_gather_q<<<static_cast<unsigned>(blocks), 256, 0, st>>>(uq, usf, perm, rblock, rows, K, l, lp,
-                                                            u_perm_q, atoms);
-  return cudaGetLastError();
+  return launch_pdl(k_gather_q, static_cast<unsigned>(blocks), 256, 0, st, uq, usf, perm, rblock,
+                    rows, K, l, lp, u_perm_q, atoms);
 }
 
 }  // namespace lmoe

@@ -35,6 +35,22 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start before its predecessor ends; pdl_wait() returns
+// once the predecessor has completed and its writes are visible (a no-op
+// otherwise).  Every kernel here signals its dependents only after its own
+// pdl_wait(), so when a kernel starts, all kernels before its predecessor have
+// completed: it may read their outputs before pdl_wait().
+
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

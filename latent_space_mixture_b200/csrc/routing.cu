@@ -16,6 +16,7 @@
 #include <cuda_bf16.h>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 namespace lmoe {
@@ -49,6 +50,8 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
                                                const float* __restrict__ bias, int64_t T, int N,
                                                int K, int32_t* __restrict__ topk_idx,
                                                float* __restrict__ topk_w) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -103,12 +106,10 @@ cudaError_t launch_route(const float* logits, const float* bias, int64_t T, int 
   if (T <= 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
   if (N <= 32 * 4)
-    k_route<4><<<blocks, 256, 0, st>>>(logits, bias, T, N, K, topk_idx, topk_w);
-  else if (N <= 32 * 16)
-    k_route<16><<<blocks, 256, 0, st>>>(logits, bias, T, N, K, topk_idx, topk_w);
-  else
-    k_route<32><<<blocks, 256, 0, st>>>(logits, bias, T, N, K, topk_idx, topk_w);
-  return cudaGetLastError();
+    return launch_pdl(k_route<4>, blocks, 256, 0, st, logits, bias, T, N, K, topk_idx, topk_w);
+  if (N <= 32 * 16)
+    return launch_pdl(k_route<16>, blocks, 256, 0, st, logits, bias, T, N, K, topk_idx, topk_w);
+  return launch_pdl(k_route<32>, blocks, 256, 0, st, logits, bias, T, N, K, topk_idx, topk_w);
 }
 
 // ---------------------------------------------------------------------------
@@ -141,6 +142,8 @@ __device__ __forceinline__ void build_chunk_masks(uint32_t* m, const int32_t* __
 __global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, int64_t T, int N,
                                               int K, int32_t* __restrict__ chunk_cnt, int* err) {
   extern __shared__ uint32_t hist_masks[];
+  pdl_wait();
+  pdl_trigger();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t c = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + w;
   const int64_t nchunks = (T + 31) / 32;
@@ -155,8 +158,8 @@ cudaError_t launch_hist(const int32_t* topk_idx, int64_t T, int N, int K, int32_
   if (T <= 0) return cudaSuccess;
   const int64_t nchunks = (T + 31) / 32;
   const unsigned blocks = static_cast<unsigned>((nchunks + 7) / 8);
-  k_hist<<<blocks, 256, 8 * N * sizeof(uint32_t), st>>>(topk_idx, T, N, K, chunk_cnt, err);
-  return cudaGetLastError();
+  return launch_pdl(k_hist, blocks, 256, 8 * N * sizeof(uint32_t), st, topk_idx, T, N, K,
+                    chunk_cnt, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -165,6 +168,8 @@ cudaError_t launch_hist(const int32_t* topk_idx, int64_t T, int N, int K, int32_
 __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ chunk, int64_t C, int N,
                                                int32_t* __restrict__ counts) {
   __shared__ int32_t tile[32][33];
+  pdl_wait();
+  pdl_trigger();
   const int tx = threadIdx.x, ty = threadIdx.y;
   const int e0 = blockIdx.x * 32;
   int carry = 0;   // running total of expert e0 + ty (held by warp ty)
@@ -192,8 +197,7 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ chunk, int6
 cudaError_t launch_scan(int32_t* chunk_cnt, int64_t T, int N, int32_t* counts, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   const int64_t C = (T + 31) / 32;
-  k_scan<<<N / 32, dim3(32, 32), 0, st>>>(chunk_cnt, C, N, counts);
-  return cudaGetLastError();
+  return launch_pdl(k_scan, N / 32, dim3(32, 32), 0, st, chunk_cnt, C, N, counts);
 }
 
 // ---------------------------------------------------------------------------
@@ -239,6 +243,8 @@ __global__ void __launch_bounds__(256) k_scatter(
   uint32_t* masks = reinterpret_cast<uint32_t*>(bbase + N);  // [8][N]
   __shared__ int wsum[16];
   __shared__ int total;
+  pdl_wait();
+  pdl_trigger();
 
   // offsets: exclusive scan of counts, 4 experts per thread (N <= 1024)
   const int e4 = threadIdx.x * 4;
@@ -330,9 +336,8 @@ cudaError_t launch_scatter(const int32_t* topk_idx, const float* topk_w, const i
   const int64_t nchunks = (T + 31) / 32;
   const unsigned nblk = static_cast<unsigned>(nchunks > 0 ? (nchunks + 7) / 8 : 1);
   const size_t smem = (2 * N + 1) * sizeof(int32_t) + 8 * N * sizeof(uint32_t);
-  k_scatter<<<nblk, 256, smem, st>>>(topk_idx, topk_w, chunk_base, counts, T, N, K, bn, offsets,
-                                     perm, inv, wrow, blocks, nblocks, rblock, err);
-  return cudaGetLastError();
+  return launch_pdl(k_scatter, nblk, 256, smem, st, topk_idx, topk_w, chunk_base, counts, T, N, K,
+                    bn, offsets, perm, inv, wrow, blocks, nblocks, rblock, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -341,6 +346,8 @@ cudaError_t launch_scatter(const int32_t* topk_idx, const float* topk_w, const i
 __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ u,
                                                 const int32_t* __restrict__ perm, int64_t rows,
                                                 int K, int l8, uint4* __restrict__ u_perm) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
   for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
@@ -357,9 +364,8 @@ cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int 
   if (rows <= 0) return cudaSuccess;
   int64_t blocks = (rows + 7) / 8;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  k_gather<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const uint4*>(u), perm, rows, K, l / 8, static_cast<uint4*>(u_perm));
-  return cudaGetLastError();
+  return launch_pdl(k_gather, static_cast<unsigned>(blocks), 256, 0, st,
+                    static_cast<const uint4*>(u), perm, rows, K, l / 8, static_cast<uint4*>(u_perm));
 }
 
 // ---------------------------------------------------------------------------
@@ -371,6 +377,8 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict
                                                  const int32_t* __restrict__ inv, int64_t T,
                                                  int K, int l, __nv_bfloat16* __restrict__ vh,
                                                  int ldv) {
+  pdl_wait();
+  pdl_trigger();
   const int l8 = l >> 3;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t t = g / l8;
@@ -415,9 +423,9 @@ cudaError_t launch_combine(const void* O, const int32_t* inv, int64_t T, int K, 
                            int ldv, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   const int64_t blocks = (T * (l / 8) + 255) / 256;
-  k_combine<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(O), inv, T, K, l, static_cast<__nv_bfloat16*>(vh), ldv);
-  return cudaGetLastError();
+  return launch_pdl(k_combine, static_cast<unsigned>(blocks), 256, 0, st,
+                    static_cast<const __nv_bfloat16*>(O), inv, T, K, l,
+                    static_cast<__nv_bfloat16*>(vh), ldv);
 }
 
 // ---------------------------------------------------------------------------
