@@ -10,6 +10,7 @@
 #include <new>
 #include <vector>
 
+#include "gemm_pair.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.h"
 #include "launch.cuh"
@@ -187,6 +188,26 @@ cudaError_t launch_gemm(const CUtensorMap& A, const BMaps& B, const TileSource& 
   using L = GemmLayout<BN, Stages<BN, FP4>::value, FP4>;
   return launch_pdl(k_gemm_tc<BN, Stages<BN, FP4>::value, Epi, FP4>, grid, GEMM_THREADS,
                     L::SMEM_BYTES, st, A, B.b16, B.b64, src, epi, err, limit);
+}
+
+// CTA-pair variant: 256 x 256 tiles, 6 stages of 32 KB per CTA
+constexpr int PAIR_BN = 256;
+constexpr int PAIR_STAGES = 6;
+
+template <class Epi>
+cudaError_t set_pair_smem() {
+  return cudaFuncSetAttribute(k_gemm_pair<PAIR_BN, PAIR_STAGES, Epi>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              PairLayout<PAIR_BN, PAIR_STAGES>::SMEM_BYTES);
+}
+
+template <class Epi>
+cudaError_t launch_gemm_pair(const CUtensorMap& A, const BMaps& B, const TileSource& src,
+                             const Epi& epi, int npairs, int* err, unsigned long long limit,
+                             cudaStream_t st) {
+  return launch_pair_pdl(k_gemm_pair<PAIR_BN, PAIR_STAGES, Epi>, 2 * npairs, GEMM_THREADS,
+                         PairLayout<PAIR_BN, PAIR_STAGES>::SMEM_BYTES, st, A, B.b16, B.b64, src,
+                         epi, err, limit);
 }
 
 template <class Epi>
@@ -375,6 +396,7 @@ struct lmoe_handle {
   CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
   BMaps tm_uperm, tm_H, tm_vh;
   int64_t last_T = 0;
+  bool pairs = true;   // CTA-pair GEMMs for large token counts (LMOE_PAIR=0: off)
   unsigned long long wait_limit_ns = 2000000000ull;
   // profiling
   bool prof = false;
@@ -629,6 +651,10 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   ok &= set_smem_all<EpiH>() == cudaSuccess;
   ok &= set_smem_all<EpiO>() == cudaSuccess;
   ok &= set_smem_all<EpiY>() == cudaSuccess;
+  ok &= set_pair_smem<EpiX>() == cudaSuccess;
+  ok &= set_pair_smem<EpiH>() == cudaSuccess;
+  ok &= set_pair_smem<EpiO>() == cudaSuccess;
+  ok &= set_pair_smem<EpiY>() == cudaSuccess;
   ok &= cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -636,6 +662,8 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     delete h;
     return LMOE_ERR_CUDA;
   }
+  const char* pe = getenv("LMOE_PAIR");
+  h->pairs = !(pe && pe[0] == '0');
   *out = h;
   return LMOE_OK;
 }
@@ -717,14 +745,22 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   {
     const int fb = (N + l + hs + 127) / 128;
     const DensePlan p = plan_dense(T, fb, static_cast<int>(d / 64), h->sms);
+    EpiX epi{h->logits, h->u, h->vh, N, l, ldvh, h->uq, h->usf, h->g_u};
+    const int fb2 = (N + l + hs + PAIR_BM - 1) / PAIR_BM;
+    const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
+    if (h->pairs && ptiles >= h->sms / 2) {
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, N + l + hs,
+                   static_cast<int>(d / 64), 1, nullptr, 0};
+      LMOE_STEP(0, launch_gemm_pair(h->tm_wx, tm_x, s, epi, h->sms / 2, h->err, lim, st));
+    } else {
     TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, N + l + hs,
                  static_cast<int>(d / 64), p.ksplit, h->part, T <= p.bn};
     const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
     const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
-    EpiX epi{h->logits, h->u, h->vh, N, l, ldvh, h->uq, h->usf, h->g_u};
     LMOE_STEP(0, launch_gemm_bn(p.bn, h->tm_wx, tm_x, s, epi, grid, h->err, lim, st));
     if (p.ksplit > 1)
       LMOE_STEP(10, launch_reduce(h->part, p.ksplit, static_cast<int>(T), N + l + hs, epi, st));
+    }
   }
   // 2-5. routing and segments
   const int gbn = grouped_bn(c, T);
@@ -757,17 +793,29 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   LMOE_STEP(5, launch_gather(h->u, h->perm, T * K, K, l, h->u_perm, st));
   // 7. H = sqrelu(W1[e] u)
   {
-    TileSource s{0, 0, h->blocks, h->nblocks, (hh + 127) / 128, hh, hh, l / 64, 1, nullptr,
-                 gbn == 32};
     EpiH epi{h->H, hh};
-    LMOE_STEP(6, launch_gemm_bn(gbn, h->tm_w1, h->tm_uperm, s, epi, h->sms, h->err, lim, st));
+    if (h->pairs && gbn == PAIR_BN) {
+      TileSource s{0, 0, h->blocks, h->nblocks, (hh + PAIR_BM - 1) / PAIR_BM, hh, hh, l / 64, 1,
+                   nullptr, 0};
+      LMOE_STEP(6, launch_gemm_pair(h->tm_w1, h->tm_uperm, s, epi, h->sms / 2, h->err, lim, st));
+    } else {
+      TileSource s{0, 0, h->blocks, h->nblocks, (hh + 127) / 128, hh, hh, l / 64, 1, nullptr,
+                   gbn == 32};
+      LMOE_STEP(6, launch_gemm_bn(gbn, h->tm_w1, h->tm_uperm, s, epi, h->sms, h->err, lim, st));
+    }
   }
   // 8. O = w * W2[e] H
   {
-    TileSource s{0, 0, h->blocks, h->nblocks, (l + 127) / 128, l, l, hh / 64, 1, nullptr,
-                 gbn == 32};
     EpiO epi{h->O, h->wrow, l};
-    LMOE_STEP(7, launch_gemm_bn(gbn, h->tm_w2, h->tm_H, s, epi, h->sms, h->err, lim, st));
+    if (h->pairs && gbn == PAIR_BN) {
+      TileSource s{0, 0, h->blocks, h->nblocks, (l + PAIR_BM - 1) / PAIR_BM, l, l, hh / 64, 1,
+                   nullptr, 0};
+      LMOE_STEP(7, launch_gemm_pair(h->tm_w2, h->tm_H, s, epi, h->sms / 2, h->err, lim, st));
+    } else {
+      TileSource s{0, 0, h->blocks, h->nblocks, (l + 127) / 128, l, l, hh / 64, 1, nullptr,
+                   gbn == 32};
+      LMOE_STEP(7, launch_gemm_bn(gbn, h->tm_w2, h->tm_H, s, epi, h->sms, h->err, lim, st));
+    }
   }
   }
   // 9. v = sum_k O[inv[t][k]]
@@ -776,15 +824,23 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   {
     const int fb = static_cast<int>((d + 127) / 128);
     const DensePlan p = plan_dense(T, fb, ldvh / 64, h->sms);
-    TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, static_cast<int>(d), ldvh / 64,
-                 p.ksplit, h->part, T <= p.bn};
-    const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
-    const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
     EpiY epi{static_cast<bf16*>(y), static_cast<int>(d)};
-    LMOE_STEP(9, launch_gemm_bn(p.bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
-    if (p.ksplit > 1)
-      LMOE_STEP(11, launch_reduce(h->part, p.ksplit, static_cast<int>(T), static_cast<int>(d), epi,
-                                  st));
+    const int fb2 = static_cast<int>((d + PAIR_BM - 1) / PAIR_BM);
+    const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
+    if (h->pairs && ptiles >= h->sms / 2) {
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, static_cast<int>(d),
+                   ldvh / 64, 1, nullptr, 0};
+      LMOE_STEP(9, launch_gemm_pair(h->tm_wy, h->tm_vh, s, epi, h->sms / 2, h->err, lim, st));
+    } else {
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, static_cast<int>(d),
+                   ldvh / 64, p.ksplit, h->part, T <= p.bn};
+      const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
+      const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
+      LMOE_STEP(9, launch_gemm_bn(p.bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
+      if (p.ksplit > 1)
+        LMOE_STEP(11, launch_reduce(h->part, p.ksplit, static_cast<int>(T), static_cast<int>(d),
+                                    epi, st));
+    }
   }
   return LMOE_OK;
 }

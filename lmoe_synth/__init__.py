@@ -68,6 +68,9 @@ CONFIGS: Dict[str, LayerConfig] = {
     # the prefill batch), Zipf bias: a small prefill case for profiler captures
     "super_prefill_n64": LayerConfig("super_prefill_n64", 1024, 4096, 1024, 64, 22, 2688,
                                      5376, 0.02, "zipf", 6),
+    # mid-sized layer whose token counts reach the CTA-pair GEMMs (256 rows per
+    # expert, >= 74 dense 256x256 tiles) at sizes the oracle covers quickly
+    "pair_small": LayerConfig("pair_small", 4096, 1024, 512, 64, 4, 512, 1024, 0.03, "zipf", 9),
     # tiny layer with NVFP4 experts (latent and expert hidden multiples of 128)
     "tiny_nvfp4": LayerConfig("tiny_nvfp4", 64, 256, 128, 32, 4, 256, 256, 0.02, "zipf", 7,
                               "nvfp4"),

@@ -181,3 +181,25 @@ def test_large_configs_sampled_tokens(name, n):
     layer.close()
     del w, x, y
     torch.cuda.empty_cache()
+
+
+def test_cta_pair_gemms_match_single_cta_gemms(monkeypatch):
+    """The CTA-pair GEMMs (M=256 over two SMs, used at large token counts) and
+    the single-CTA GEMMs give the same layer, and both match the oracle."""
+    cfg = CONFIGS["pair_small"]
+    monkeypatch.setenv("LMOE_PAIR", "0")
+    w, x, single = make(cfg)
+    y1 = single.forward(x).clone()
+    monkeypatch.setenv("LMOE_PAIR", "1")
+    from lmoe_synth import act_global_scales  # noqa: F401
+    from latent_space_mixture_b200 import LatentMoE
+    pair = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, cfg.T, w)
+    y2 = pair.forward(x)
+    torch.cuda.synchronize()
+    assert pair.sync_status() == 0 and single.sync_status() == 0
+    assert max_rel(to64(y2), to64(y1)) <= 1e-2
+    toks = np.unique(np.concatenate([[0, cfg.T - 1], _sample(cfg.T, 24, 9)]))
+    errs = compare_layer(pair, w, x, y2, toks, cfg.K)
+    print("pair_small errors:", errs)
+    single.close()
+    pair.close()
