@@ -104,6 +104,24 @@ def roofline_entry(name, kw, total_ms, launches, peaks, peak_kind, cfg, T):
             "peak_source": peak_kind + " bf16_tflops (burst)"}
 
 
+def measured_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu record, or None
+    when there is none or the kernel sources changed since it was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        return rec.get(workload, {}).get(kernel)
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def max_over_ranks(value: float) -> float:
     if torch.distributed.is_available() and torch.distributed.is_initialized():
         dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
@@ -327,6 +345,7 @@ def main():
     dom = max((n for n in per_kernel if n in prof_by), key=lambda n: prof_by[n][0])
     roof = roofline_entry(dom, per_kernel[dom], prof_by[dom][0], prof_by[dom][1], peaks,
                           peak_kind, cfg, T)
+    roof["traffic"] = measured_traffic(cfg.name, dom)
     kernels = {n: {"ms_total": round(ms, 3), "launches": c,
                    "share": round(ms / max(sum(p[1] for p in prof), 1e-9), 4)}
                for n, ms, c in prof}
