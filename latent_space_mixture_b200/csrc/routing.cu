@@ -36,16 +36,25 @@ __device__ __forceinline__ uint64_t pack_key(float key, int e) {
   return (static_cast<uint64_t>(b) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
 }
 
+// Warp maximum of 64-bit words with two 32-bit reductions: the high halves,
+// then the low halves among the lanes holding the high maximum.
 __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
-#pragma unroll
-  for (int off = 16; off; off >>= 1) {
-    const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
-    v = o > v ? o : v;
-  }
-  return v;
+  const uint32_t hi = static_cast<uint32_t>(v >> 32);
+  const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+  const uint32_t lo = hi == mhi ? static_cast<uint32_t>(v) : 0u;
+  const uint32_t mlo = __reduce_max_sync(0xffffffffu, lo);
+  return (static_cast<uint64_t>(mhi) << 32) | mlo;
 }
 
-template <int NPL>   // upper bound of experts per lane (N <= 32 NPL)
+// compare-exchange for a descending sort network
+__device__ __forceinline__ void cas_desc(uint64_t& a, uint64_t& b) {
+  const uint64_t hi = a > b ? a : b;
+  const uint64_t lo = a > b ? b : a;
+  a = hi;
+  b = lo;
+}
+
+template <int NPL>   // upper bound of experts per lane (N <= 32 NPL), a power of 2
 __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
                                                const float* __restrict__ bias, int64_t T, int N,
                                                int K, int32_t* __restrict__ topk_idx,
@@ -65,29 +74,38 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
     bb[i] = (i < npl && bias) ? bias[lane + 32 * i] : 0.0f;
   }
   uint64_t cand[NPL];
-  uint64_t best = 0;
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
-    cand[i] = 0;
+    cand[i] = 0;   // below every packed key
     if (i < npl) {
       const float sc = 1.0f / (1.0f + expf(-zz[i]));
       cand[i] = pack_key(sc + bb[i], lane + 32 * i);
-      best = cand[i] > best ? cand[i] : best;
     }
   }
-  int my_e = 0;
-  for (int k = 0; k < K; ++k) {
-    const uint64_t win = warp_max_u64(best);
-    const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win));
-    if (lane == k) my_e = e;
-    if ((e & 31) == lane) {
-      // the winner's lane drops it and finds its next best
-      best = 0;
+  // sort the lane's candidates descending (bitonic network on registers)
+#pragma unroll
+  for (int k = 2; k <= NPL; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
-        if (cand[i] == win) cand[i] = 0;
-        best = cand[i] > best ? cand[i] : best;
+        const int p = i ^ j;
+        if (p > i) {
+          if ((i & k) == 0) cas_desc(cand[i], cand[p]);
+          else cas_desc(cand[p], cand[i]);
+        }
       }
+    }
+  }
+  // K rounds: the warp maximum of the lanes' heads; the winner shifts its list
+  int my_e = 0;
+  for (int k = 0; k < K; ++k) {
+    const uint64_t win = warp_max_u64(cand[0]);
+    if (lane == k) my_e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win));
+    if (cand[0] == win) {
+#pragma unroll
+      for (int i = 0; i + 1 < NPL; ++i) cand[i] = cand[i + 1];
+      cand[NPL - 1] = 0;
     }
   }
   // weights: the unbiased scores of the selected experts, renormalised; the
