@@ -36,6 +36,9 @@ struct PairLayout {
   static_assert(BN % 32 == 0 && BN <= 256, "pair N: two halves of multiples of 16");
   static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of 2");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  // one release per stage: the 256-wide MMAs hide the commit, and a paired
+  // release would hold a stage of the ring back (measured slower here)
+  static constexpr bool PAIRED_RELEASE = false;
 };
 
 // tile -> (token block, 256-row feature block), feature block fastest; the
@@ -120,32 +123,35 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      pdl_wait();
-      pdl_trigger();
-      const uint64_t pol_a = src.a_stream_once ? policy_evict_first() : policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      long issued = 0;
-      bool ok = true;
-      for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
-        const TileInfo t = pair_tile(src, BN, tile, rank);
-        const int n_mma = (t.nrows + 31) & ~31;
-        const int half = n_mma / 2;
-        const int nbig = half / GEMM_BROWS_BIG;
-        const int nsmall = (half - nbig * GEMM_BROWS_BIG) / GEMM_BROWS;
-        const int brow0 = t.row0 + rank * half;
-        const uint32_t tx_pair = 2 * L::A_BYTES + n_mma * GEMM_ROW_BYTES;
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err, limit_ns)) {
-            ok = false;
-            break;
-          }
-          const uint32_t full_leader = mapa_shared(smem_u32(&full[stage]), 0);
+    // whole warp, one elected lane issuing (see k_gemm_tc)
+    pdl_wait();
+    pdl_trigger();
+    const uint64_t pol_a = src.a_stream_once ? policy_evict_first() : policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    long issued = 0;
+    bool ok = true;
+    for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+      const TileInfo t = pair_tile(src, BN, tile, rank);
+      const int n_mma = (t.nrows + 31) & ~31;
+      const int half = n_mma / 2;
+      const int nbig = half / GEMM_BROWS_BIG;
+      const int nsmall = (half - nbig * GEMM_BROWS_BIG) / GEMM_BROWS;
+      const int brow0 = t.row0 + rank * half;
+      const uint32_t tx_pair = 2 * L::A_BYTES + n_mma * GEMM_ROW_BYTES;
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        if (empty_waits_at<L>(stage) &&
+            !__all_sync(0xffffffffu, mbar_wait_bounded(&empty[empty_slot<L>(stage)], phase ^ 1,
+                                                       abort_flag, err, limit_ns))) {
+          ok = false;
+          break;
+        }
+        const uint32_t full_leader = mapa_shared(smem_u32(&full[stage]), 0);
+        const int x = kb * GEMM_BK;
+        uint8_t* b_dst = sB + stage * L::B_BYTES;
+        if (elect_one()) {
           if (leader) mbar_arrive_expect_tx(&full[stage], tx_pair);
-          const int x = kb * GEMM_BK;
           tma_load_2d_pair(sA + stage * L::A_BYTES, &tmA, x, t.a_row, full_leader, pol_a);
-          uint8_t* b_dst = sB + stage * L::B_BYTES;
           for (int j = 0; j < nbig; ++j)
             tma_load_2d_pair(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, x,
                              brow0 + j * GEMM_BROWS_BIG, full_leader, policy_evict_last());
@@ -154,35 +160,37 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             tma_load_2d_pair(b_dst + r * GEMM_ROW_BYTES, &tmB, x, brow0 + r, full_leader,
                              policy_evict_last());
           }
-          ++issued;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
         }
       }
-      if (!ok) {
-        // a stage's copies complete on the even CTA's barrier; wait for this
-        // CTA's in-flight copies there (bounded) before the CTA exits
-        const long first = issued > STAGES ? issued - STAGES : 0;
-        for (long i = first; i < issued && leader; ++i) {
-          uint64_t* b = &full[i % STAGES];
-          const uint32_t par = static_cast<uint32_t>((i / STAGES) & 1);
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(b, par) && global_timer_ns() - t0 < limit_ns) {
-          }
+    }
+    if (!ok && lane == 0) {
+      // a stage's copies complete on the even CTA's barrier; wait for this
+      // CTA's in-flight copies there (bounded) before the CTA exits
+      const long first = issued > STAGES ? issued - STAGES : 0;
+      for (long i = first; i < issued && leader; ++i) {
+        uint64_t* b = &full[i % STAGES];
+        const uint32_t par = static_cast<uint32_t>((i / STAGES) & 1);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(b, par) && global_timer_ns() - t0 < limit_ns) {
         }
-        if (!leader) {
-          const uint64_t t0 = global_timer_ns();
-          while (global_timer_ns() - t0 < limit_ns / 4) {
-          }
+      }
+      if (!leader) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < limit_ns / 4) {
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (lane == 0 && leader) {
+    // whole warp, one elected lane issuing (see k_gemm_tc)
+    if (leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -192,7 +200,8 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
         const TileInfo t = pair_tile(src, BN, tile, 0);
         const int n_mma = (t.nrows + 31) & ~31;
-        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err, limit_ns)) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag,
+                                                        err, limit_ns))) {
           ok = false;
           break;
         }
@@ -200,17 +209,21 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const uint32_t d_tmem = tmem_base + acc * BN;
         const uint32_t idesc = idesc_bf16(PAIR_BM, n_mma);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns)) {
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + stage * L::A_BYTES));
           const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + stage * L::B_BYTES));
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < GEMM_BK / 16; ++k)
-            umma_bf16_pair(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
-          umma_commit_pair(&empty[stage]);
+            for (int k = 0; k < GEMM_BK / 16; ++k)
+              umma_bf16_pair(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
+            if (empty_commits_at<L>(stage)) umma_commit_pair(&empty[empty_slot<L>(stage)]);
+          }
+          __syncwarp();
           issued_any = true;
           if (++stage == STAGES) {
             stage = 0;
@@ -218,14 +231,16 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           }
         }
         if (!ok) break;
-        umma_commit_pair(&tfull[acc]);
+        if (elect_one()) umma_commit_pair(&tfull[acc]);
+        __syncwarp();
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
       if (!ok && issued_any) {
-        umma_commit_pair(drain);
+        if (elect_one()) umma_commit_pair(drain);
+        __syncwarp();
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit_ns) {
         }

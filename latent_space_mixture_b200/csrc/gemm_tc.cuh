@@ -24,6 +24,10 @@
 //               which carry data), release the accumulator.
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap
 // the main loop of tile i+1.  Every mbarrier wait is bounded (ptx.cuh).
+// The producer and MMA warps run their loops converged and issue the TMA and
+// tcgen05 instructions from one elected lane (elect.sync): issued from a lone
+// divergent thread, each of these instructions cost several times as long,
+// which starved the ring and stretched every small-N MMA.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -113,7 +117,18 @@ struct GemmLayout {
   static_assert(!FP4 || BN <= 128, "NVFP4 tiles: one scale atom of B rows");
   static_assert(COLS_USED <= 512, "TMEM columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  // with an even ring, one tcgen05.commit releases two consecutive stages
+  // (every commit costs the tensor pipe a bubble of about 200 clocks)
+  static constexpr bool PAIRED_RELEASE = STAGES % 2 == 0;
 };
+
+// "empty" barrier of ring slot s, and whether the producer waits on it there
+template <class L>
+__device__ __forceinline__ int empty_slot(int s) { return L::PAIRED_RELEASE ? s >> 1 : s; }
+template <class L>
+__device__ __forceinline__ bool empty_waits_at(int s) { return !L::PAIRED_RELEASE || !(s & 1); }
+template <class L>
+__device__ __forceinline__ bool empty_commits_at(int s) { return !L::PAIRED_RELEASE || (s & 1); }
 
 template <int BN, int STAGES, class Epi, bool FP4>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -169,117 +184,131 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      // weights read once per launch are streamed past L2; weights that
-      // several token blocks share are left to the default policy
-      const uint64_t pol_a = src.a_stream_once ? policy_evict_first() : policy_evict_last();
-      // B operand (and its scales) of one k-step: it depends on the previous
-      // kernel; A (weights, and their scales) does not
-      auto load_b = [&](int st, const TileInfo& t, int kb) {
-        const int nbig = t.nrows / GEMM_BROWS_BIG;
-        const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
-        const int bx = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
-        uint8_t* b_dst = sB + st * L::B_BYTES;
-        for (int j = 0; j < nbig; ++j)
-          tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
-                      t.row0 + j * GEMM_BROWS_BIG, &full[st]);
-        for (int j = 0; j < nsmall; ++j) {
-          const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
-          tma_load_2d(b_dst + r * GEMM_ROW_BYTES, &tmB, bx, t.row0 + r, &full[st]);
+    // Like the MMA issuer: the whole warp walks the ring (warp-uniform
+    // coordinates and addresses), one elected lane issues the copies.  (A lone
+    // thread spent about 300 ns issuing one k-step's copies, so the ring ran
+    // about one stage ahead of the MMAs instead of STAGES.)
+    // weights read once per launch are streamed past L2; weights that
+    // several token blocks share are left to the default policy
+    const uint64_t pol_a = src.a_stream_once ? policy_evict_first() : policy_evict_last();
+    // B operand (and its scales) of one k-step: it depends on the previous
+    // kernel; A (weights, and their scales) does not.  Elected lane only.
+    auto load_b = [&](int st, const TileInfo& t, int kb) {
+      const int nbig = t.nrows / GEMM_BROWS_BIG;
+      const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
+      const int bx = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+      uint8_t* b_dst = sB + st * L::B_BYTES;
+      for (int j = 0; j < nbig; ++j)
+        tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
+                    t.row0 + j * GEMM_BROWS_BIG, &full[st]);
+      for (int j = 0; j < nsmall; ++j) {
+        const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
+        tma_load_2d(b_dst + r * GEMM_ROW_BYTES, &tmB, bx, t.row0 + r, &full[st]);
+      }
+      if constexpr (FP4)
+        bulk_load(sSF + st * L::SF_BYTES + FP4_SF_STAGE_BYTES,
+                  src.sfb + (static_cast<long>(t.tb) * src.kc + kb * 4) * SF_ATOM_BYTES,
+                  FP4_SF_STAGE_BYTES, &full[st]);
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    long issued = 0;
+    bool ok = true;
+    bool waited = false;   // pdl_wait done; before it only A loads are issued
+    int deferred = 0;      // k-steps of the first tile whose B loads wait for it
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const TileInfo t = gemm_tile(src, BN, tile);
+      // B rows: 64-row boxes while 64 rows remain, then 16-row boxes
+      const int nbig = t.nrows / GEMM_BROWS_BIG;
+      const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
+      const uint32_t tx = L::A_BYTES + L::SF_BYTES +
+                          (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_ROW_BYTES;
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        if (empty_waits_at<L>(stage) &&
+            !__all_sync(0xffffffffu, mbar_wait_bounded(&empty[empty_slot<L>(stage)], phase ^ 1,
+                                                       abort_flag, err, limit_ns))) {
+          ok = false;
+          break;
         }
-        if constexpr (FP4)
-          bulk_load(sSF + st * L::SF_BYTES + FP4_SF_STAGE_BYTES,
-                    src.sfb + (static_cast<long>(t.tb) * src.kc + kb * 4) * SF_ATOM_BYTES,
-                    FP4_SF_STAGE_BYTES, &full[st]);
-      };
-      int stage = 0;
-      uint32_t phase = 0;
-      long issued = 0;
-      bool ok = true;
-      bool waited = false;   // pdl_wait done; before it only A loads are issued
-      int deferred = 0;      // k-steps of the first tile whose B loads wait for it
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const TileInfo t = gemm_tile(src, BN, tile);
-        // B rows: 64-row boxes while 64 rows remain, then 16-row boxes
-        const int nbig = t.nrows / GEMM_BROWS_BIG;
-        const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
-        const uint32_t tx = L::A_BYTES + L::SF_BYTES +
-                            (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_ROW_BYTES;
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err, limit_ns)) {
-            ok = false;
-            break;
-          }
+        // x coordinate in elements of the map: bf16 elements or bytes (NVFP4)
+        const int ax = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+        if (elect_one()) {
           mbar_arrive_expect_tx(&full[stage], tx);
-          // x coordinate in elements of the map: bf16 elements or bytes (NVFP4)
-          const int ax = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
           tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, ax, t.a_row, &full[stage], pol_a);
           if constexpr (FP4)
             bulk_load(sSF + stage * L::SF_BYTES,
                       src.sfa + (static_cast<long>(t.a_row / GEMM_BM) * src.kc + kb * 4) *
                                     SF_ATOM_BYTES,
                       FP4_SF_STAGE_BYTES, &full[stage]);
-          if (waited) {
-            load_b(stage, t, kb);
-          } else if (++deferred == STAGES || kb + 1 == t.kb1) {
-            // the first tile's first stages: weights are in flight, now the
-            // previous kernel's results
-            pdl_wait();
-            pdl_trigger();
-            waited = true;
+          if (waited) load_b(stage, t, kb);
+        }
+        __syncwarp();
+        if (!waited && (++deferred == STAGES || kb + 1 == t.kb1)) {
+          // the first tile's first stages: weights are in flight, now the
+          // previous kernel's results
+          pdl_wait();
+          pdl_trigger();
+          waited = true;
+          if (elect_one())
             for (int j = 0; j < deferred; ++j) load_b(j, t, t.kb0 + j);
-          }
-          ++issued;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+          __syncwarp();
+        }
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
         }
       }
-      if (!waited) {
-        pdl_wait();
-        pdl_trigger();
-      }
-      if (!ok) {
-        // let the copies already issued land before the CTA's smem goes away
-        const long first = issued > STAGES ? issued - STAGES : 0;
-        for (long i = first; i < issued; ++i) {
-          uint64_t* b = &full[i % STAGES];
-          const uint32_t par = static_cast<uint32_t>((i / STAGES) & 1);
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(b, par) && global_timer_ns() - t0 < limit_ns) {
-          }
+    }
+    if (!waited) {
+      pdl_wait();
+      pdl_trigger();
+    }
+    if (!ok && lane == 0) {
+      // let the copies already issued land before the CTA's smem goes away
+      const long first = issued > STAGES ? issued - STAGES : 0;
+      for (long i = first; i < issued; ++i) {
+        uint64_t* b = &full[i % STAGES];
+        const uint32_t par = static_cast<uint32_t>((i / STAGES) & 1);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(b, par) && global_timer_ns() - t0 < limit_ns) {
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      bool issued_any = false;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const TileInfo t = gemm_tile(src, BN, tile);
-        const int n_mma = (t.nrows + 15) & ~15;
-        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err, limit_ns)) {
+    // The whole warp walks the ring, so that descriptors and TMEM addresses
+    // stay warp-uniform; one elected lane issues the tcgen05 instructions.
+    // (Issued from a lone thread, an MMA whose descriptors change every
+    // k-step costs the tensor pipe about twice the cycles.)
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    bool issued_any = false;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const TileInfo t = gemm_tile(src, BN, tile);
+      const int n_mma = (t.nrows + 15) & ~15;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err, limit_ns))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      const uint32_t idesc = FP4 ? idesc_nvf4(GEMM_BM, n_mma) : idesc_bf16(GEMM_BM, n_mma);
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        const uint32_t idesc = FP4 ? idesc_nvf4(GEMM_BM, n_mma) : idesc_bf16(GEMM_BM, n_mma);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + stage * L::A_BYTES));
-          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + stage * L::B_BYTES));
+        const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + stage * L::A_BYTES));
+        const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + stage * L::B_BYTES));
+        if (elect_one()) {
           if constexpr (FP4) {
             // scale atoms of this stage into its TMEM slot, then 4 MMAs of K=64
             const uint32_t sf_col = L::SF_COL0 + stage * 32;
@@ -301,25 +330,28 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             for (int k = 0; k < GEMM_BK / 16; ++k)   // +32 bytes per K=16 step
               umma_bf16(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
           }
-          umma_commit(&empty[stage]);
-          issued_any = true;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+          if (empty_commits_at<L>(stage)) umma_commit(&empty[empty_slot<L>(stage)]);
         }
-        if (!ok) break;
-        umma_commit(&tfull[acc]);
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1;
+        __syncwarp();
+        issued_any = true;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
         }
       }
-      if (!ok && issued_any) {
-        umma_commit(drain);
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit_ns) {
-        }
+      if (!ok) break;
+      if (elect_one()) umma_commit(&tfull[acc]);
+      __syncwarp();
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+    if (!ok && issued_any) {
+      if (elect_one()) umma_commit(drain);
+      __syncwarp();
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit_ns) {
       }
     }
     __syncwarp();
