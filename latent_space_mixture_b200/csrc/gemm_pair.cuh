@@ -24,10 +24,18 @@ namespace lmoe {
 
 constexpr int PAIR_BM = 256;
 
-template <int BN, int STAGES>
+// A stage holds KSUB consecutive 64-wide K sub-tiles of both operands (each
+// its own 128-byte-swizzled region) and completes on one barrier phase: a
+// CTA's TMA stream is limited by a roughly fixed cost per barrier phase
+// (~450 clocks: one 16 KB box per phase moves ~36 B/clock, two ~68, three or
+// more ~85), so a k-step of 16 KB of weights and a few token rows would be
+// bound by it rather than by the MMAs.
+template <int BN, int STAGES, int KSUB>
 struct PairLayout {
-  static constexpr int A_BYTES = GEMM_BM * GEMM_ROW_BYTES;
-  static constexpr int B_BYTES = (BN / 2) * GEMM_ROW_BYTES;
+  static constexpr int A_SUB = GEMM_BM * GEMM_ROW_BYTES;
+  static constexpr int B_SUB = (BN / 2) * GEMM_ROW_BYTES;
+  static constexpr int A_BYTES = KSUB * A_SUB;
+  static constexpr int B_BYTES = KSUB * B_SUB;
   static constexpr int STG_BYTES = GEMM_EPI_WARPS * 32 * GEMM_STG_LD * 4;
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
   static constexpr int SMEM_BYTES =
@@ -65,12 +73,12 @@ __device__ __forceinline__ TileInfo pair_tile(const TileSource& s, int BN, int t
   return t;
 }
 
-template <int BN, int STAGES, class Epi>
+template <int BN, int STAGES, int KSUB, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmB64, const TileSource src, const Epi epi,
             int* err, unsigned long long limit_ns) {
-  using L = PairLayout<BN, STAGES>;
+  using L = PairLayout<BN, STAGES, KSUB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -138,8 +146,9 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       const int nbig = half / GEMM_BROWS_BIG;
       const int nsmall = (half - nbig * GEMM_BROWS_BIG) / GEMM_BROWS;
       const int brow0 = t.row0 + rank * half;
-      const uint32_t tx_pair = 2 * L::A_BYTES + n_mma * GEMM_ROW_BYTES;
-      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+      // bytes of one K sub-tile, both CTAs (A halves and B halves)
+      const uint32_t tx_sub = 2 * L::A_SUB + n_mma * GEMM_ROW_BYTES;
+      for (int kb = t.kb0; kb < t.kb1; kb += KSUB) {
         if (empty_waits_at<L>(stage) &&
             !__all_sync(0xffffffffu, mbar_wait_bounded(&empty[empty_slot<L>(stage)], phase ^ 1,
                                                        abort_flag, err, limit_ns))) {
@@ -147,18 +156,22 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           break;
         }
         const uint32_t full_leader = mapa_shared(smem_u32(&full[stage]), 0);
-        const int x = kb * GEMM_BK;
-        uint8_t* b_dst = sB + stage * L::B_BYTES;
+        const int nsub = min(KSUB, t.kb1 - kb);
         if (elect_one()) {
-          if (leader) mbar_arrive_expect_tx(&full[stage], tx_pair);
-          tma_load_2d_pair(sA + stage * L::A_BYTES, &tmA, x, t.a_row, full_leader, pol_a);
-          for (int j = 0; j < nbig; ++j)
-            tma_load_2d_pair(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, x,
-                             brow0 + j * GEMM_BROWS_BIG, full_leader, policy_evict_last());
-          for (int j = 0; j < nsmall; ++j) {
-            const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
-            tma_load_2d_pair(b_dst + r * GEMM_ROW_BYTES, &tmB, x, brow0 + r, full_leader,
-                             policy_evict_last());
+          if (leader) mbar_arrive_expect_tx(&full[stage], nsub * tx_sub);
+          for (int q = 0; q < nsub; ++q) {
+            const int x = (kb + q) * GEMM_BK;
+            tma_load_2d_pair(sA + stage * L::A_BYTES + q * L::A_SUB, &tmA, x, t.a_row,
+                             full_leader, pol_a);
+            uint8_t* b_dst = sB + stage * L::B_BYTES + q * L::B_SUB;
+            for (int j = 0; j < nbig; ++j)
+              tma_load_2d_pair(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, x,
+                               brow0 + j * GEMM_BROWS_BIG, full_leader, policy_evict_last());
+            for (int j = 0; j < nsmall; ++j) {
+              const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
+              tma_load_2d_pair(b_dst + r * GEMM_ROW_BYTES, &tmB, x, brow0 + r, full_leader,
+                               policy_evict_last());
+            }
           }
         }
         __syncwarp();
@@ -208,19 +221,23 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         const uint32_t idesc = idesc_bf16(PAIR_BM, n_mma);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; kb += KSUB) {
           if (!__all_sync(0xffffffffu,
                           mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + stage * L::A_BYTES));
-          const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + stage * L::B_BYTES));
+          const int nsub = min(KSUB, t.kb1 - kb);
           if (elect_one()) {
+            for (int q = 0; q < nsub; ++q) {
+              const uint64_t a0 = sdesc_k_sw128(smem_u32(sA + stage * L::A_BYTES + q * L::A_SUB));
+              const uint64_t b0 = sdesc_k_sw128(smem_u32(sB + stage * L::B_BYTES + q * L::B_SUB));
 #pragma unroll
-            for (int k = 0; k < GEMM_BK / 16; ++k)
-              umma_bf16_pair(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
+              for (int k = 0; k < GEMM_BK / 16; ++k)
+                umma_bf16_pair(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc,
+                               (kb != t.kb0) || (q != 0) || (k != 0));
+            }
             if (empty_commits_at<L>(stage)) umma_commit_pair(&empty[empty_slot<L>(stage)]);
           }
           __syncwarp();

@@ -190,24 +190,25 @@ cudaError_t launch_gemm(const CUtensorMap& A, const BMaps& B, const TileSource& 
                     L::SMEM_BYTES, st, A, B.b16, B.b64, src, epi, err, limit);
 }
 
-// CTA-pair variant: 256 x 256 tiles, 6 stages of 32 KB per CTA
+// CTA-pair variant: 256 x 256 tiles, 3 stages of K = 128 (64 KB per CTA)
 constexpr int PAIR_BN = 256;
-constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_STAGES = 3;
+constexpr int PAIR_KSUB = 2;
 
 template <class Epi>
 cudaError_t set_pair_smem() {
-  return cudaFuncSetAttribute(k_gemm_pair<PAIR_BN, PAIR_STAGES, Epi>,
+  return cudaFuncSetAttribute(k_gemm_pair<PAIR_BN, PAIR_STAGES, PAIR_KSUB, Epi>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              PairLayout<PAIR_BN, PAIR_STAGES>::SMEM_BYTES);
+                              PairLayout<PAIR_BN, PAIR_STAGES, PAIR_KSUB>::SMEM_BYTES);
 }
 
 template <class Epi>
 cudaError_t launch_gemm_pair(const CUtensorMap& A, const BMaps& B, const TileSource& src,
                              const Epi& epi, int npairs, int* err, unsigned long long limit,
                              cudaStream_t st) {
-  return launch_pair_pdl(k_gemm_pair<PAIR_BN, PAIR_STAGES, Epi>, 2 * npairs, GEMM_THREADS,
-                         PairLayout<PAIR_BN, PAIR_STAGES>::SMEM_BYTES, st, A, B.b16, B.b64, src,
-                         epi, err, limit);
+  return launch_pair_pdl(k_gemm_pair<PAIR_BN, PAIR_STAGES, PAIR_KSUB, Epi>, 2 * npairs,
+                         GEMM_THREADS, PairLayout<PAIR_BN, PAIR_STAGES, PAIR_KSUB>::SMEM_BYTES, st,
+                         A, B.b16, B.b64, src, epi, err, limit);
 }
 
 template <class Epi>
