@@ -63,21 +63,24 @@ def algorithmic_work(cfg, T: int, counts: np.ndarray):
     Bytes count the weights a forward must read (dense weights plus the W1/W2
     of experts with at least one routed row), x and y, and for each kernel its
     own operands and results; flops count real rows only (no tile padding).
+    Without projections (the standard MoE) the x-GEMM has no W_dn rows, the
+    y-GEMM no W_upl columns, and it reads v once more for the residual add.
     """
     d, l, N, K, h, hs = cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs
+    lx = l if cfg.proj else 0
     touched = int((counts > 0).sum())
     R = T * K
-    wx = (N + l + hs) * d * 2
-    wy = d * (l + hs) * 2
+    wx = (N + lx + hs) * d * 2
+    wy = d * (lx + hs) * 2
     wexp = touched * h * l * 2
     per_kernel = {
-        "xgemm(router|W_dn|W_s1)": dict(bytes=wx + T * d * 2 + T * (N * 4 + l * 2 + hs * 2),
-                                        flops=2 * T * d * (N + l + hs)),
+        "xgemm(router|W_dn|W_s1)": dict(bytes=wx + T * d * 2 + T * (N * 4 + lx * 2 + hs * 2),
+                                        flops=2 * T * d * (N + lx + hs)),
         "grouped_gemm1(W1,sqrelu)": dict(bytes=wexp + R * l * 2 + R * h * 2, flops=2 * R * l * h),
         "grouped_gemm2(W2,*w)": dict(bytes=wexp + R * h * 2 + R * l * 2 + R * 4,
                                      flops=2 * R * h * l),
         "ygemm([W_upl|W_s2])": dict(bytes=wy + T * (l + hs) * 2 + T * d * 2,
-                                    flops=2 * T * d * (l + hs)),
+                                    flops=2 * T * d * (lx + hs)),
     }
     layer = dict(bytes=wx + wy + 2 * wexp + 2 * T * d * 2,
                  flops=sum(v["flops"] for v in per_kernel.values()))
@@ -237,8 +240,8 @@ def oracle_rate(cfg, w, x, seconds: float, seed: int):
     def to64(t):
         return t.detach().to("cpu").to(torch.float64).numpy()
 
-    dense = {k: to64(w[k]) for k in ("w_router", "router_bias", "w_dn", "w_upl", "w_s1",
-                                     "w_s2")}
+    dense = {k: (to64(w[k]) if k in w else None)
+             for k in ("w_router", "router_bias", "w_dn", "w_upl", "w_s1", "w_s2")}
     rng = np.random.default_rng(seed)
     order = rng.permutation(x.shape[0])
     done, t0 = 0, time.perf_counter()
@@ -303,7 +306,8 @@ def main():
     T = cfg.T
     from lmoe_synth import act_global_scales
     layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, expert_format=cfg.fmt,
-                      act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0))
+                      act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0),
+                      projections=cfg.proj)
     y = torch.empty_like(x)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
     stream = torch.cuda.current_stream()
@@ -386,7 +390,7 @@ def main():
             "config": {"workload": cfg.name, "T": T, "d": cfg.d, "latent": cfg.l,
                        "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
                        "shared_hidden": cfg.hs, "router_bias": cfg.bias,
-                       "tokens_per_rank": T, "parallelism": f"dp{world} (replicated weights)",
+                       "latent_projections": cfg.proj, "tokens_per_rank": T, "parallelism": f"dp{world} (replicated weights)",
                        "l2": "256 MiB write between steps, outside the per-step events"},
             "roofline": roof, "layer_roofline": layer_roof, "kernels": kernels,
             "kernels_note": "per-kernel CUDA events from a second pass of the same steps",
@@ -426,7 +430,7 @@ def run_reference(args, cfg, world):
             "impl": "reference",
             "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "latent": cfg.l,
                        "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
-                       "shared_hidden": cfg.hs},
+                       "shared_hidden": cfg.hs, "latent_projections": cfg.proj},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
                              "kind": "oracle",
                              "sample": f"{n_tot} tokens over {args.steps} steps, {el_tot:.1f} s"},

@@ -41,6 +41,15 @@ extern "C" {
 #define LMOE_ERR_TIMEOUT (-5)     /* a bounded device wait ran out          */
 #define LMOE_ERR_DEVICE (-6)      /* a kernel flagged bad data (e.g. index) */
 
+/* Standard MoE (lmoe_config.flags): no latent projections.  The experts
+ * work at the hidden width (latent must equal d) on x itself, u = x and
+ * r = v; w_dn and w_upl are ignored (may be NULL).  This is the layer the
+ * pages compare LatentMoE against at equal active and total parameters
+ * ("NVIDIA Nemotron 3: Efficient and Open Intelligence", section 三 eq.(1):
+ * N = 128, K = 6 at d = 4096 against N' = 512, K' = 22 at l = 1024; section
+ * 六 Table 1).  BF16 experts only. */
+#define LMOE_FLAG_NO_PROJECTION 1
+
 #define LMOE_FMT_BF16 0  /* experts in BF16                                   */
 #define LMOE_FMT_NVFP4 1 /* experts in NVFP4: W1, W2 and the expert inputs u
                             and H as E2M1 codes with E4M3 scales per 16
@@ -61,7 +70,7 @@ typedef struct lmoe_config {
   int32_t expert_hidden; /* h: expert FFN hidden width                    */
   int32_t shared_hidden; /* h_s: shared-expert hidden width               */
   int32_t expert_format; /* LMOE_FMT_*                                     */
-  int32_t reserved;      /* must be 0                                     */
+  int32_t flags;         /* 0, or LMOE_FLAG_NO_PROJECTION                 */
   int64_t max_tokens;    /* >= 1                                          */
 } lmoe_config;
 
@@ -70,10 +79,10 @@ typedef struct lmoe_config {
 typedef struct lmoe_weights {
   const void* w_router;    /* [N][d]      bf16                              */
   const float* router_bias;/* [N]         fp32, or NULL for zeros           */
-  const void* w_dn;        /* [l][d]      bf16                              */
+  const void* w_dn;        /* [l][d]      bf16 (unused without projections) */
   const void* w1;          /* [N][h][l]   bf16                              */
   const void* w2;          /* [N][l][h]   bf16                              */
-  const void* w_upl;       /* [d][l]      bf16                              */
+  const void* w_upl;       /* [d][l]      bf16 (unused without projections) */
   const void* w_s1;        /* [h_s][d]    bf16                              */
   const void* w_s2;        /* [d][h_s]    bf16                              */
   float act_gscale_latent; /* NVFP4 only (> 0): static global scale of u;

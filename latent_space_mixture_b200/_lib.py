@@ -13,6 +13,7 @@ LMOE_OK = 0
 ERRORS = {-1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "OOM", -4: "CUDA", -5: "TIMEOUT",
           -6: "DEVICE"}
 FMT_BF16, FMT_NVFP4 = 0, 1
+FLAG_NO_PROJECTION = 1   # standard MoE: no latent projections (u = x, r = v)
 DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 6,
        "logits": 7, "u": 8, "v": 9, "hs": 10, "w1q_codes": 11, "w1q_sf": 12, "w1q_g": 13,
        "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16}
@@ -21,7 +22,7 @@ DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 
 class LmoeConfig(Structure):
     _fields_ = [("d", c_int32), ("latent", c_int32), ("n_experts", c_int32), ("top_k", c_int32),
                 ("expert_hidden", c_int32), ("shared_hidden", c_int32),
-                ("expert_format", c_int32), ("reserved", c_int32), ("max_tokens", c_int64)]
+                ("expert_format", c_int32), ("flags", c_int32), ("max_tokens", c_int64)]
 
 
 class LmoeWeights(Structure):

@@ -25,11 +25,13 @@ namespace lmoe {
 
 // x -> [W_r; W_dn; W_s1] x: router logits (fp32), latent u (bf16) and the
 // shared-expert hidden sqrelu(W_s1 x) (bf16, into columns [l, l+h_s) of vh).
+// Features [0, N) are logits, [N, N+lu) u and the rest the shared hidden;
+// lu = 0 for the standard MoE (no W_dn rows, u = x).
 struct EpiX {
   float* logits;
   bf16* u;
   bf16* vh;
-  int N, l, ldvh;
+  int N, lu, l, ldvh;
   uint8_t* uq;    // NVFP4 experts: u codes [T][l/2] (nullptr for BF16 experts)
   uint8_t* usf;   //   and its E4M3 block scales [T][l/16]
   float g_u;      //   static global scale of u
@@ -39,10 +41,10 @@ struct EpiX {
       // every lane takes part in the 16-block pair exchange; only u lanes store
       uint8_t sc;
       const uint32_t codes = nvfp4_pair(v, g_u, &sc);
-      if (valid && feat >= N && feat < N + l) {
+      if (valid && feat >= N && feat < N + lu) {
         const int f = feat - N;
-        *reinterpret_cast<uint32_t*>(uq + row * (l / 2) + f / 2) = codes;
-        if ((f & 15) == 0) usf[row * (l / 16) + f / 16] = sc;
+        *reinterpret_cast<uint32_t*>(uq + row * (lu / 2) + f / 2) = codes;
+        if ((f & 15) == 0) usf[row * (lu / 16) + f / 16] = sc;
       }
     }
     if (!valid) return;
@@ -50,13 +52,13 @@ struct EpiX {
       float4* p = reinterpret_cast<float4*>(logits + row * N + feat);
       p[0] = make_float4(v[0], v[1], v[2], v[3]);
       p[1] = make_float4(v[4], v[5], v[6], v[7]);
-    } else if (feat < N + l) {
-      store8_bf16(u + row * l + (feat - N), v);
+    } else if (feat < N + lu) {
+      store8_bf16(u + row * lu + (feat - N), v);
     } else {
       float a[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) a[i] = sqrelu(v[i]);
-      store8_bf16(vh + row * ldvh + l + (feat - N - l), a);
+      store8_bf16(vh + row * ldvh + l + (feat - N - lu), a);
     }
   }
 };
@@ -91,14 +93,31 @@ struct EpiO {
   }
 };
 
-// [W_upl | W_s2] [v ; hs]: routed branch plus shared branch in one K loop
+// [W_upl | W_s2] [v ; hs]: routed branch plus shared branch in one K loop.
+// Standard MoE (no W_upl): the GEMM is W_s2 hs and the epilogue adds v
+// (resid, row pitch ldr) before the store.
 struct EpiY {
   bf16* y;
   int d;
+  const bf16* resid;
+  int ldr;
   __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
                                          bool valid) const {
     if (!valid) return;
-    store8_bf16(y + row * d + feat, v);
+    if (resid) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(resid + row * ldr + feat);
+      const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      float a[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(r2[i]);
+        a[2 * i] = v[2 * i] + f.x;
+        a[2 * i + 1] = v[2 * i + 1] + f.y;
+      }
+      store8_bf16(y + row * d + feat, a);
+    } else {
+      store8_bf16(y + row * d + feat, v);
+    }
   }
 };
 
@@ -283,6 +302,21 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// as make_map, for a [rows][cols] window of a matrix whose rows are `pitch`
+// elements apart
+static bool make_map_strided(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                             uint64_t pitch, uint32_t box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D byte matrix [rows][cols] (packed NVFP4 codes), box of 128 bytes x
 // box_rows rows, 128-byte swizzle.
 static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
@@ -372,6 +406,7 @@ struct lmoe_handle {
   bf16* x_dev = nullptr;   // staging for lmoe_forward_host
   bf16* y_dev = nullptr;
   float* part = nullptr;   // split-K partials of the dense GEMMs
+  int64_t part_floats = 0; // its capacity
   int* err = nullptr;
   // NVFP4 experts: quantised weights, activations and their scale atoms
   bool fp4 = false;
@@ -398,6 +433,8 @@ struct lmoe_handle {
   BMaps tm_uperm, tm_H, tm_vh;
   int64_t last_T = 0;
   bool pairs = true;   // CTA-pair GEMMs for large token counts (LMOE_PAIR=0: off)
+  bool proj = true;    // latent projections (false: standard MoE, u = x, r = v)
+  int lx = 0;          // W_dn rows in w_x and W_upl columns in w_y (l, or 0)
   unsigned long long wait_limit_ns = 2000000000ull;
   // profiling
   bool prof = false;
@@ -433,8 +470,12 @@ static void free_all(lmoe_handle* h) {
 static int check_cfg(const lmoe_config* c) {
   if (!c) return LMOE_ERR_INVALID_ARG;
   if (c->d <= 0 || c->latent <= 0 || c->n_experts <= 0 || c->top_k <= 0 ||
-      c->expert_hidden <= 0 || c->shared_hidden <= 0 || c->max_tokens < 1 || c->reserved != 0)
+      c->expert_hidden <= 0 || c->shared_hidden <= 0 || c->max_tokens < 1 ||
+      (c->flags & ~LMOE_FLAG_NO_PROJECTION) != 0)
     return LMOE_ERR_INVALID_ARG;
+  if ((c->flags & LMOE_FLAG_NO_PROJECTION) &&
+      (c->latent != c->d || c->expert_format != LMOE_FMT_BF16))
+    return LMOE_ERR_UNSUPPORTED;
   if (c->top_k > c->n_experts) return LMOE_ERR_INVALID_ARG;
   if (c->expert_format != LMOE_FMT_BF16 && c->expert_format != LMOE_FMT_NVFP4)
     return LMOE_ERR_INVALID_ARG;
@@ -479,7 +520,9 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   *out = nullptr;
   int rc = check_cfg(cfg);
   if (rc != LMOE_OK) return rc;
-  if (!w || !w->w_router || !w->w_dn || !w->w1 || !w->w2 || !w->w_upl || !w->w_s1 || !w->w_s2)
+  const bool proj = !(cfg->flags & LMOE_FLAG_NO_PROJECTION);
+  if (!w || !w->w_router || !w->w1 || !w->w2 || !w->w_s1 || !w->w_s2 ||
+      (proj && (!w->w_dn || !w->w_upl)))
     return LMOE_ERR_INVALID_ARG;
   if (cfg->expert_format == LMOE_FMT_NVFP4 &&
       !(w->act_gscale_latent > 0.0f && w->act_gscale_hidden > 0.0f &&
@@ -498,6 +541,9 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   const lmoe_config& c = h->cfg;
   const int64_t N = c.n_experts, d = c.d, l = c.latent, hh = c.expert_hidden,
                 hs = c.shared_hidden, K = c.top_k, Tm = c.max_tokens;
+  h->proj = proj;
+  h->lx = proj ? static_cast<int>(l) : 0;
+  const int64_t lx = h->lx;
   const int64_t rows = Tm * K;
   const int64_t C = (Tm + 31) / 32;
   // operand buffers read by TMA hold at least one box of rows
@@ -512,30 +558,34 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   const int64_t nb_max = rows / 32 + N + 1;   // token blocks of >= 32 rows, one partial per expert
   // bytes of the bf16 expert path buffers that NVFP4 replaces
   const int64_t bf16_only = fp4 ? 0 : 1;
-  // largest split-K partials buffer over the token counts this handle accepts
+  // largest split-K partials buffer over the token counts this handle
+  // accepts, for the same feature and K extents the forward pass plans with
+  // (x-GEMM: N + lx + h_s features over K = d; y-GEMM: d features over
+  // K = lx + h_s)
   int64_t part_floats = 0;
   {
-    const int fbx = static_cast<int>((N + l + hs + 127) / 128);
+    const int fbx = static_cast<int>((N + lx + hs + 127) / 128);
     const int fby = static_cast<int>((d + 127) / 128);
     const int64_t tmax = Tm < 256LL * h->sms ? Tm : 256LL * h->sms;
     for (int64_t T = 1; T <= tmax; ++T) {
       const DensePlan px = plan_dense(T, fbx, static_cast<int>(d / 64), h->sms);
-      const DensePlan py = plan_dense(T, fby, static_cast<int>((l + hs) / 64), h->sms);
-      if (px.ksplit > 1 && px.ksplit * T * (N + l + hs) > part_floats)
-        part_floats = px.ksplit * T * (N + l + hs);
+      const DensePlan py = plan_dense(T, fby, static_cast<int>((lx + hs) / 64), h->sms);
+      if (px.ksplit > 1 && px.ksplit * T * (N + lx + hs) > part_floats)
+        part_floats = px.ksplit * T * (N + lx + hs);
       if (py.ksplit > 1 && py.ksplit * T * d > part_floats) part_floats = py.ksplit * T * d;
     }
   }
+  h->part_floats = part_floats;
   const int64_t max_blocks = rows / 32 + N + 1;
   struct Req {
     void** p;
     size_t bytes;
   } reqs[] = {
-      {(void**)&h->w_x, size_t((N + l + hs) * d * 2)},
+      {(void**)&h->w_x, size_t((N + lx + hs) * d * 2)},
       {(void**)&h->bias, size_t(N * 4)},
       {(void**)&h->w1, size_t(bf16_only * N * hh * l * 2)},
       {(void**)&h->w2, size_t(bf16_only * N * l * hh * 2)},
-      {(void**)&h->w_y, size_t(d_a * (l + hs) * 2)},
+      {(void**)&h->w_y, size_t(d_a * (lx + hs) * 2)},
       {(void**)&h->logits, size_t(Tm * N * 4)},
       {(void**)&h->topk_idx, size_t(rows * 4)},
       {(void**)&h->topk_w, size_t(rows * 4)},
@@ -547,7 +597,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->wrow, size_t(rows * 4)},
       {(void**)&h->blocks, size_t(max_blocks * 16)},
       {(void**)&h->nblocks, size_t(4)},
-      {(void**)&h->u, size_t(Tm * l * 2)},
+      {(void**)&h->u, size_t(Tm * lx * 2)},
       {(void**)&h->u_perm, size_t(bf16_only * rows_b * l * 2)},
       {(void**)&h->H, size_t(bf16_only * rows_b * hh * 2)},
       {(void**)&h->O, size_t(rows * l * 2)},
@@ -581,8 +631,9 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   bool ok = true;
   // weights, re-laid: [W_r; W_dn; W_s1] and [W_upl | W_s2]
   ok &= cudaMemcpy(h->w_x, w->w_router, N * d * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
-  ok &= cudaMemcpy(h->w_x + N * d, w->w_dn, l * d * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
-  ok &= cudaMemcpy(h->w_x + (N + l) * d, w->w_s1, hs * d * 2, cudaMemcpyDeviceToDevice) ==
+  if (proj)
+    ok &= cudaMemcpy(h->w_x + N * d, w->w_dn, l * d * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemcpy(h->w_x + (N + lx) * d, w->w_s1, hs * d * 2, cudaMemcpyDeviceToDevice) ==
         cudaSuccess;
   if (!fp4) {
     ok &= cudaMemcpy(h->w1, w->w1, N * hh * l * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
@@ -616,9 +667,10 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= set_gemm_smem<128, EpiOq, true>() == cudaSuccess;
     ok &= set_gemm_smem<32, EpiOq, true>() == cudaSuccess;
   }
-  ok &= cudaMemcpy2D(h->w_y, (l + hs) * 2, w->w_upl, l * 2, l * 2, d,
-                     cudaMemcpyDeviceToDevice) == cudaSuccess;
-  ok &= cudaMemcpy2D(h->w_y + l, (l + hs) * 2, w->w_s2, hs * 2, hs * 2, d,
+  if (proj)
+    ok &= cudaMemcpy2D(h->w_y, (lx + hs) * 2, w->w_upl, l * 2, l * 2, d,
+                       cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemcpy2D(h->w_y + lx, (lx + hs) * 2, w->w_s2, hs * 2, hs * 2, d,
                      cudaMemcpyDeviceToDevice) == cudaSuccess;
   if (w->router_bias)
     ok &= cudaMemcpy(h->bias, w->router_bias, N * 4, cudaMemcpyDeviceToDevice) == cudaSuccess;
@@ -632,22 +684,25 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   }
   ok &= cudaMemset(h->x_dev, 0, Tm_b * d * 2) == cudaSuccess;
   if (d_a > d)
-    ok &= cudaMemset(h->w_y + d * (l + hs), 0, (d_a - d) * (l + hs) * 2) == cudaSuccess;
+    ok &= cudaMemset(h->w_y + d * (lx + hs), 0, (d_a - d) * (lx + hs) * 2) == cudaSuccess;
   // tensor maps of the fixed operands
-  ok &= make_map(&h->tm_wx, h->w_x, N + l + hs, d, GEMM_BM);
+  ok &= make_map(&h->tm_wx, h->w_x, N + lx + hs, d, GEMM_BM);
   if (!fp4) {
     ok &= make_map(&h->tm_w1, h->w1, N * hh, l, GEMM_BM);
     ok &= make_map(&h->tm_w2, h->w2, N * l, hh, GEMM_BM);
   }
-  ok &= make_map(&h->tm_wy, h->w_y, d_a, l + hs, GEMM_BM);
+  ok &= make_map(&h->tm_wy, h->w_y, d_a, lx + hs, GEMM_BM);
   if (!fp4) {
     ok &= make_map(&h->tm_uperm.b16, h->u_perm, rows_b, l, GEMM_BROWS);
     ok &= make_map(&h->tm_uperm.b64, h->u_perm, rows_b, l, GEMM_BROWS_BIG);
     ok &= make_map(&h->tm_H.b16, h->H, rows_b, hh, GEMM_BROWS);
     ok &= make_map(&h->tm_H.b64, h->H, rows_b, hh, GEMM_BROWS_BIG);
   }
-  ok &= make_map(&h->tm_vh.b16, h->vh, Tm_b, l + hs, GEMM_BROWS);
-  ok &= make_map(&h->tm_vh.b64, h->vh, Tm_b, l + hs, GEMM_BROWS_BIG);
+  // B operand of the y-GEMM: [v | hs], or hs alone (columns [l, l+h_s) of
+  // vh, same row pitch) for the standard MoE, whose v is added in the epilogue
+  ok &= make_map_strided(&h->tm_vh.b16, h->vh + (l - lx), Tm_b, lx + hs, l + hs, GEMM_BROWS);
+  ok &= make_map_strided(&h->tm_vh.b64, h->vh + (l - lx), Tm_b, lx + hs, l + hs,
+                         GEMM_BROWS_BIG);
   ok &= set_smem_all<EpiX>() == cudaSuccess;
   ok &= set_smem_all<EpiH>() == cudaSuccess;
   ok &= set_smem_all<EpiO>() == cudaSuccess;
@@ -681,10 +736,9 @@ int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T) {
   if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return 0;
   const lmoe_config& c = h->cfg;
-  const DensePlan px = plan_dense(T, (c.n_experts + c.latent + c.shared_hidden + 127) / 128,
+  const DensePlan px = plan_dense(T, (c.n_experts + h->lx + c.shared_hidden + 127) / 128,
                                   c.d / 64, h->sms);
-  const DensePlan py =
-      plan_dense(T, (c.d + 127) / 128, (c.latent + c.shared_hidden) / 64, h->sms);
+  const DensePlan py = plan_dense(T, (c.d + 127) / 128, (h->lx + c.shared_hidden) / 64, h->sms);
   return 10 + (px.ksplit > 1) + (py.ksplit > 1);
 }
 
@@ -726,6 +780,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   const int N = c.n_experts, l = c.latent, hh = c.expert_hidden, hs = c.shared_hidden,
             K = c.top_k;
   const int ldvh = l + hs;
+  const int lx = h->lx;   // l, or 0 for the standard MoE
   const unsigned long long lim = h->wait_limit_ns;
   BMaps tm_x;
   if (T < GEMM_BROWS_BIG) {
@@ -744,23 +799,25 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
 
   // 1. [W_r; W_dn; W_s1] x: logits, u, shared hidden
   {
-    const int fb = (N + l + hs + 127) / 128;
+    const int fb = (N + lx + hs + 127) / 128;
     const DensePlan p = plan_dense(T, fb, static_cast<int>(d / 64), h->sms);
-    EpiX epi{h->logits, h->u, h->vh, N, l, ldvh, h->uq, h->usf, h->g_u};
-    const int fb2 = (N + l + hs + PAIR_BM - 1) / PAIR_BM;
+    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u};
+    const int fb2 = (N + lx + hs + PAIR_BM - 1) / PAIR_BM;
     const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
     if (h->pairs && ptiles >= h->sms / 2) {
-      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, N + l + hs,
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, N + lx + hs,
                    static_cast<int>(d / 64), 1, nullptr, 0};
       LMOE_STEP(0, launch_gemm_pair(h->tm_wx, tm_x, s, epi, h->sms / 2, h->err, lim, st));
     } else {
-    TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, N + l + hs,
+    if (p.ksplit > 1 && int64_t(p.ksplit) * T * (N + lx + hs) > h->part_floats)
+      return LMOE_ERR_UNSUPPORTED;   // never: the buffer is sized for every T
+    TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, N + lx + hs,
                  static_cast<int>(d / 64), p.ksplit, h->part, T <= p.bn};
     const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
     const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
     LMOE_STEP(0, launch_gemm_bn(p.bn, h->tm_wx, tm_x, s, epi, grid, h->err, lim, st));
     if (p.ksplit > 1)
-      LMOE_STEP(10, launch_reduce(h->part, p.ksplit, static_cast<int>(T), N + l + hs, epi, st));
+      LMOE_STEP(10, launch_reduce(h->part, p.ksplit, static_cast<int>(T), N + lx + hs, epi, st));
     }
   }
   // 2-5. routing and segments
@@ -791,7 +848,8 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
     }
   } else {
   // 6. latent rows into expert order
-  LMOE_STEP(5, launch_gather(h->u, h->perm, T * K, K, l, h->u_perm, st));
+  LMOE_STEP(5, launch_gather(h->proj ? static_cast<const void*>(h->u) : x, h->perm, T * K, K, l,
+                             h->u_perm, st));
   // 7. H = sqrelu(W1[e] u)
   {
     EpiH epi{h->H, hh};
@@ -824,17 +882,20 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   // 10. y = [W_upl | W_s2] [v ; hs]
   {
     const int fb = static_cast<int>((d + 127) / 128);
-    const DensePlan p = plan_dense(T, fb, ldvh / 64, h->sms);
-    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d)};
+    const int ky = lx + hs;   // K of the y-GEMM
+    const DensePlan p = plan_dense(T, fb, ky / 64, h->sms);
+    if (p.ksplit > 1 && int64_t(p.ksplit) * T * d > h->part_floats)
+      return LMOE_ERR_UNSUPPORTED;   // never: the buffer is sized for every T
+    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d), h->proj ? nullptr : h->vh, ldvh};
     const int fb2 = static_cast<int>((d + PAIR_BM - 1) / PAIR_BM);
     const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
     if (h->pairs && ptiles >= h->sms / 2) {
       TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, static_cast<int>(d),
-                   ldvh / 64, 1, nullptr, 0};
+                   ky / 64, 1, nullptr, 0};
       LMOE_STEP(9, launch_gemm_pair(h->tm_wy, h->tm_vh, s, epi, h->sms / 2, h->err, lim, st));
     } else {
       TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, static_cast<int>(d),
-                   ldvh / 64, p.ksplit, h->part, T <= p.bn};
+                   ky / 64, p.ksplit, h->part, T <= p.bn};
       const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
       const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
       LMOE_STEP(9, launch_gemm_bn(p.bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
@@ -894,7 +955,9 @@ int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
     case LMOE_DBG_PERM: src = h->perm; want = T * K * 4; break;
     case LMOE_DBG_INV: src = h->inv; want = T * K * 4; break;
     case LMOE_DBG_LOGITS: src = h->logits; want = T * N * 4; break;
-    case LMOE_DBG_U: src = h->u; want = T * l * 2; break;
+    case LMOE_DBG_U:
+      if (!h->proj) return LMOE_ERR_INVALID_ARG;   // u is x itself
+      src = h->u; want = T * l * 2; break;
     case LMOE_DBG_V: strided = true; col0 = 0; cols = l; want = T * l * 2; break;
     case LMOE_DBG_HS: strided = true; col0 = l; cols = hs; want = T * hs * 2; break;
     case LMOE_DBG_W1Q_CODES: src = h->w1q; want = N * c.expert_hidden * h->lp / 2; break;

@@ -10,7 +10,8 @@ from typing import Dict, Optional
 import torch
 
 from . import _lib
-from ._lib import DBG, FMT_BF16, FMT_NVFP4, LmoeConfig, LmoeError, LmoeWeights, check
+from ._lib import (DBG, FLAG_NO_PROJECTION, FMT_BF16, FMT_NVFP4, LmoeConfig, LmoeError,
+                   LmoeWeights, check)
 
 __all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]
 
@@ -31,14 +32,18 @@ class LatentMoE:
     weights: dict of CUDA bf16 tensors w_router [N][d], w_dn [l][d],
     w1 [N][h][l], w2 [N][l][h], w_upl [d][l], w_s1 [h_s][d], w_s2 [d][h_s],
     and optionally router_bias [N] fp32.  The library copies them.
+    projections=False builds the standard MoE (latent = d, no w_dn / w_upl:
+    the experts work on x and their combined output is added as is).
     """
 
     def __init__(self, d: int, latent: int, n_experts: int, top_k: int, expert_hidden: int,
                  shared_hidden: int, max_tokens: int, weights: Dict[str, torch.Tensor],
-                 expert_format: str = "bf16", act_gscales=(0.0, 0.0)):
+                 expert_format: str = "bf16", act_gscales=(0.0, 0.0), projections: bool = True):
         self.lib = _lib.load()
         dims = {"d": d, "l": latent, "N": n_experts, "h": expert_hidden, "hs": shared_hidden}
         for k, shape in _WEIGHT_SHAPES.items():
+            if not projections and k in ("w_dn", "w_upl"):
+                continue
             t = weights[k]
             want = tuple(dims[s] for s in shape)
             if tuple(t.shape) != want or t.dtype != torch.bfloat16 or not t.is_cuda:
@@ -50,12 +55,13 @@ class LatentMoE:
                                  or not bias.is_cuda):
             raise ValueError("router_bias: need CUDA fp32 [N]")
         self.cfg = LmoeConfig(d, latent, n_experts, top_k, expert_hidden, shared_hidden,
-                              {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4}[expert_format], 0,
-                              max_tokens)
+                              {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4}[expert_format],
+                              0 if projections else FLAG_NO_PROJECTION, max_tokens)
         w = LmoeWeights(weights["w_router"].data_ptr(),
                         bias.data_ptr() if bias is not None else None,
-                        weights["w_dn"].data_ptr(), weights["w1"].data_ptr(),
-                        weights["w2"].data_ptr(), weights["w_upl"].data_ptr(),
+                        weights["w_dn"].data_ptr() if projections else None,
+                        weights["w1"].data_ptr(), weights["w2"].data_ptr(),
+                        weights["w_upl"].data_ptr() if projections else None,
                         weights["w_s1"].data_ptr(), weights["w_s2"].data_ptr(),
                         float(act_gscales[0]), float(act_gscales[1]))
         self.device = weights["w1"].device

@@ -8,11 +8,17 @@ Workloads (dimensions from the pages' layer tables):
   * Super dims: d=4096, l=1024, N=512, K=22, expert hidden 2688, shared hidden
     5376 -- "Nemotron-3 Super 精读报告", table 2.2 (架构配置详表);
   * Ultra dims: d=8192, l=2048, N=512, K=22, expert hidden 5120, shared hidden
-    10240 -- "Nemotron 3 Ultra 解读:NVFP4 训出的 Mamba 混合 MoE", section 架构一览.
+    10240 -- "Nemotron 3 Ultra 解读:NVFP4 训出的 Mamba 混合 MoE", section 架构一览;
+  * the standard MoE that LatentMoE is compared against: no projections,
+    N=128, K=6 at d=4096 with the same expert and shared hidden widths, so
+    that total and active expert parameters match Super's 512 x 22 at l=1024
+    -- "NVIDIA Nemotron 3: Efficient and Open Intelligence", section 三 eq.(1)
+    ("vs 128", "vs 6") and section 六 Table 1.
 
 Draw order per workload (one torch.Generator seeded with the workload's seed,
 on the device the tensors are made on): W_r, router-bias permutation, W_dn,
-W1 (expert by expert), W2 (expert by expert), W_upl, W_s1, W_s2, x.
+W1 (expert by expert), W2 (expert by expert), W_upl, W_s1, W_s2, x (W_dn and
+W_upl are not drawn for a workload without projections).
 Weights ~ N(0, std^2) rounded to bf16, x ~ N(0, 1) rounded to bf16.
 Router bias: "zero" (uniform router) or "zipf": with a seeded permutation pi
 of the experts, rank r_e = 1 + pi(e) and b_e = 0.1 * ln(r_e^-1.1), which makes
@@ -43,6 +49,7 @@ class LayerConfig:
     bias: str         # "zero" or "zipf"
     seed: int
     fmt: str = "bf16"  # expert format: "bf16" or "nvfp4"
+    proj: bool = True  # latent projections W_dn, W_upl (False: standard MoE, l = d)
 
     def with_(self, **kw) -> "LayerConfig":
         return replace(self, **kw)
@@ -81,6 +88,13 @@ CONFIGS: Dict[str, LayerConfig] = {
     "super_prefill_nvfp4": LayerConfig("super_prefill_nvfp4", 8192, 4096, 1024,
                                        512, 22, 2688, 5376, 0.02, "zipf", 4,
                                        "nvfp4"),
+    # the standard-MoE comparator: tiny, decode- and prefill-sized
+    "tiny_std": LayerConfig("tiny_std", 64, 256, 256, 32, 4, 128, 256, 0.02, "zipf", 10,
+                            proj=False),
+    "std_decode": LayerConfig("std_decode", 256, 4096, 4096, 128, 6, 2688, 5376, 0.02,
+                              "zero", 11, proj=False),
+    "std_prefill": LayerConfig("std_prefill", 8192, 4096, 4096, 128, 6, 2688, 5376, 0.02,
+                               "zipf", 12, proj=False),
 }
 
 
@@ -107,7 +121,10 @@ def make_weights(cfg: LayerConfig, device="cpu", seed: Optional[int] = None):
         w["router_bias"] = torch.zeros(N, dtype=torch.float32, device=device)
     else:
         raise ValueError(cfg.bias)
-    w["w_dn"] = _randn((l, d), sd, gen, device)
+    if cfg.proj:
+        w["w_dn"] = _randn((l, d), sd, gen, device)
+    elif l != d:
+        raise ValueError("a workload without projections has l = d")
     w1 = torch.empty((N, h, l), dtype=torch.bfloat16, device=device)
     for e in range(N):
         w1[e] = _randn((h, l), sd, gen, device)
@@ -116,7 +133,8 @@ def make_weights(cfg: LayerConfig, device="cpu", seed: Optional[int] = None):
     for e in range(N):
         w2[e] = _randn((l, h), sd, gen, device)
     w["w2"] = w2
-    w["w_upl"] = _randn((d, l), sd, gen, device)
+    if cfg.proj:
+        w["w_upl"] = _randn((d, l), sd, gen, device)
     w["w_s1"] = _randn((hs, d), sd, gen, device)
     w["w_s2"] = _randn((d, hs), sd, gen, device)
     return w, gen

@@ -144,14 +144,18 @@ def expert_ffn(U: np.ndarray, W1e: np.ndarray, W2e: np.ndarray) -> np.ndarray:
 
 
 def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
-                  W_dn: np.ndarray, get_w1: Callable[[int], np.ndarray],
-                  get_w2: Callable[[int], np.ndarray], W_upl: np.ndarray,
+                  W_dn: Optional[np.ndarray], get_w1: Callable[[int], np.ndarray],
+                  get_w2: Callable[[int], np.ndarray], W_upl: Optional[np.ndarray],
                   W_s1: np.ndarray, W_s2: np.ndarray, K: int,
                   quant: Optional[Dict] = None) -> Dict[str, np.ndarray]:
     """The LatentMoE layer forward pass for the tokens in x ([T][d], float64).
 
     Weights are [out][in] float64: W_r [N][d], W_dn [l][d], W_upl [d][l],
     W_s1 [h_s][d], W_s2 [d][h_s]; get_w1(e) -> [h][l], get_w2(e) -> [l][h].
+    W_dn = W_upl = None is the standard MoE layer that the pages compare
+    LatentMoE against ("NVIDIA Nemotron 3: Efficient and Open Intelligence",
+    section 三 eq.(1) and section 六 Table 1): no projections, the experts
+    work at width l = d on x itself, u = x and r = v.
     Every token is computed independently, so any subset of tokens may be
     passed.  quant: None for the BF16 layer, or a dict with the NVFP4 global
     scales {"g_u": float, "g_h": float} for the NVFP4-expert layer, in which
@@ -162,14 +166,16 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     the shared expert's hidden activation sqrelu(W_s1 x).
     """
     x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    if (W_dn is None) != (W_upl is None):
+        raise ValueError("W_dn and W_upl are both given (LatentMoE) or both None")
     T = x.shape[0]
     N = W_r.shape[0]
-    l = W_dn.shape[0]
+    l = x.shape[1] if W_dn is None else W_dn.shape[0]
     # 1-2: router at width d
     z = x @ W_r.T
     S, w, gap, s = route(z, bias, K)
-    # 3: latent down-projection
-    u = x @ W_dn.T
+    # 3: latent down-projection (none for the standard MoE)
+    u = x.copy() if W_dn is None else x @ W_dn.T
     if quant is not None:
         from . import nvfp4
         u_in = nvfp4.fake_quant(u, quant["g_u"])
@@ -192,8 +198,8 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
             o = expert_ffn(u_in[tok], W1e, W2e)
         # a token selects e at most once, so tok has no repeats here
         v[tok] += w[tok, slot][:, None] * o
-    # 5: one projection back to width d
-    r = v @ W_upl.T
+    # 5: one projection back to width d (none for the standard MoE)
+    r = v.copy() if W_upl is None else v @ W_upl.T
     # 6: shared expert at width d
     hs = sqrelu(x @ W_s1.T)
     sh = hs @ W_s2.T
@@ -209,17 +215,18 @@ def token_forward(x_t: np.ndarray, S_t: np.ndarray, s_t: np.ndarray,
     Used where the top-K set is not unique at the comparison precision (near
     ties): the caller first checks with is_valid_topk that S_t is a top-K set
     under the oracle's own keys.  Weights are renormalised from the oracle's
-    scores s_t.  Returns v [l] and r [d].
+    scores s_t.  Returns v [l] and r [d].  W_dn = W_upl = None: the standard
+    MoE (u = x, r = v), as in layer_forward.
     """
     x_t = np.asarray(x_t, dtype=np.float64).reshape(-1)
     S_t = np.asarray(S_t, dtype=np.int64).reshape(-1)
     sel = np.asarray(s_t, dtype=np.float64)[S_t]
     w = sel / sel.sum()
-    u = W_dn @ x_t
+    u = x_t.copy() if W_dn is None else W_dn @ x_t
     if quant is not None:
         from . import nvfp4
         u = nvfp4.fake_quant(u[None, :], quant["g_u"])[0]
-    v = np.zeros(W_dn.shape[0], dtype=np.float64)
+    v = np.zeros(u.shape[0], dtype=np.float64)
     for k, e in enumerate(S_t):
         W1e = get_w1(int(e))
         W2e = get_w2(int(e))
@@ -232,7 +239,7 @@ def token_forward(x_t: np.ndarray, S_t: np.ndarray, s_t: np.ndarray,
         else:
             o = W2e @ sqrelu(W1e @ u)
         v += w[k] * o
-    return {"v": v, "r": W_upl @ v, "w": w}
+    return {"v": v, "r": v.copy() if W_upl is None else W_upl @ v, "w": w}
 
 
 def scaling_relation(N: int, K: int, d: int, l: int):

@@ -33,7 +33,10 @@ REL_RMS = 1e-2
 W_TOL = 1e-5
 
 
-def to64(t: torch.Tensor) -> np.ndarray:
+def to64(t):
+    """float64 numpy copy of a tensor (None for a missing weight)."""
+    if t is None:
+        return None
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
@@ -49,7 +52,8 @@ def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None):
     from lmoe_synth import act_global_scales
     layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs,
                       max_tokens or x.shape[0], w, expert_format=cfg.fmt,
-                      act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0))
+                      act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0),
+                      projections=cfg.proj)
     return w, x, layer
 
 
@@ -70,8 +74,9 @@ def oracle_tokens(w, x_rows: torch.Tensor, K: int, quant=None):
         return to64(w[name][e])
 
     out = O.layer_forward(to64(x_rows), to64(w["w_router"]), to64(w["router_bias"]),
-                          to64(w["w_dn"]), lambda e: fetch("w1", e), lambda e: fetch("w2", e),
-                          to64(w["w_upl"]), to64(w["w_s1"]), to64(w["w_s2"]), K, quant=quant)
+                          to64(w.get("w_dn")), lambda e: fetch("w1", e),
+                          lambda e: fetch("w2", e), to64(w.get("w_upl")), to64(w["w_s1"]),
+                          to64(w["w_s2"]), K, quant=quant)
     out["_fetch"] = fetch
     return out
 
@@ -127,17 +132,18 @@ def compare_layer(layer, w, x, y, tokens, K, tol=TOL_BF16, quant=None, elem_rel=
         else:
             n_tie_diff += 1
             assert O.is_valid_topk(key[i], gi[i], GAP), f"token {tokens[i]}: invalid top-K"
-            tf = O.token_forward(to64(x[tokens[i]]), gi[i], o["s"][i], to64(w["w_dn"]),
+            tf = O.token_forward(to64(x[tokens[i]]), gi[i], o["s"][i], to64(w.get("w_dn")),
                                  lambda e: o["_fetch"]("w1", e), lambda e: o["_fetch"]("w2", e),
-                                 to64(w["w_upl"]), quant=quant)
+                                 to64(w.get("w_upl")), quant=quant)
             v_ref[i] = tf["v"]
             y_ref[i] = tf["r"] + o["sh"][i]
-    got = {"u": to64(layer.debug("u"))[tokens], "hs": to64(layer.debug("hs"))[tokens],
-           "v": to64(layer.debug("v"))[tokens]}
+    # u is x itself without projections (the library keeps no copy of it)
+    names = ("u", "hs", "v") if "w_dn" in w else ("hs", "v")
+    got = {k: to64(layer.debug(k))[tokens] for k in names}
     ref = {"u": o["u"], "hs": o["hs"], "v": v_ref}
     errs = {"y_maxerr_over_rms": max_rel(to64(y)[tokens], y_ref),
             "near_tie_sets_differing": n_tie_diff}
-    for k in ("u", "hs", "v"):
+    for k in names:
         ok, ratio, rr = elem_ok(got[k], ref[k], rel=elem_rel)
         errs[k + "_maxerr_over_rms"] = max_rel(got[k], ref[k])
         errs[k + "_err_over_bound"] = ratio

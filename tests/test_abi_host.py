@@ -47,13 +47,15 @@ def test_strerror(lib):
 def _cfg(**kw):
     from latent_space_mixture_b200._lib import LmoeConfig
     base = dict(d=256, latent=64, n_experts=32, top_k=4, expert_hidden=128, shared_hidden=256,
-                expert_format=0, reserved=0, max_tokens=64)
+                expert_format=0, flags=0, max_tokens=64)
     base.update(kw)
     return LmoeConfig(**base)
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(top_k=33), -1), (dict(top_k=0), -1), (dict(max_tokens=0), -1), (dict(reserved=1), -1),
+    (dict(top_k=33), -1), (dict(top_k=0), -1), (dict(max_tokens=0), -1), (dict(flags=2), -1),
+    # no projections: latent must equal d, BF16 experts only
+    (dict(flags=1), -2), (dict(flags=1, latent=256, expert_format=1), -2),
     (dict(d=100), -2), (dict(latent=96), -2), (dict(n_experts=48), -2),
     (dict(n_experts=2048, top_k=4), -2), (dict(expert_format=1), -2), (dict(expert_format=7), -1),
 ])

@@ -310,6 +310,44 @@ def test_identity_projections_give_standard_moe():
     assert np.allclose(out["y"], y, atol=1e-12, rtol=0)
 
 
+@pytest.mark.parametrize("seed,bias_scale", [(3, 0.0), (4, 0.4)])
+def test_standard_moe_matches_loop_only_restatement(seed, bias_scale):
+    """No projections (W_dn = W_upl = None): the loop restatement with u = x
+    and r = v, every expert on every token under a brute-force mask."""
+    rng = np.random.default_rng(seed)
+    T, d, N, K, h, hs = 3, 6, 5, 2, 3, 4
+    p = _rand_layer(rng, T, d, d, N, h, hs, bias_scale)
+    eye = np.eye(d).tolist()
+    y_ref = _dense_masked_layer(p["x"].tolist(), p["W_r"].tolist(), p["b"].tolist(), eye,
+                                p["W1"].tolist(), p["W2"].tolist(), eye,
+                                p["W_s1"].tolist(), p["W_s2"].tolist(), K)
+    p["W_dn"] = None
+    p["W_upl"] = None
+    out = _oracle(p, K)
+    assert np.allclose(out["y"], y_ref, atol=1e-12, rtol=0)
+    assert np.array_equal(out["u"], p["x"])
+    assert np.array_equal(out["r"], out["v"])
+
+
+def test_standard_moe_equals_identity_projections_exactly():
+    rng = np.random.default_rng(12)
+    T, d, N, K, h, hs = 7, 8, 6, 3, 5, 4
+    p = _rand_layer(rng, T, d, d, N, h, hs, 0.3)
+    q = dict(p, W_dn=np.eye(d), W_upl=np.eye(d))
+    p["W_dn"] = None
+    p["W_upl"] = None
+    a, b = _oracle(p, K), _oracle(q, K)
+    for k in ("S", "w", "u", "v", "r", "sh", "y"):
+        assert np.array_equal(a[k], b[k]), k
+    t = 2
+    tf = O.token_forward(p["x"][t], a["S"][t], a["s"][t], None, lambda e: p["W1"][e],
+                         lambda e: p["W2"][e], None)
+    assert np.allclose(tf["r"], a["r"][t], atol=1e-14, rtol=0)
+    with pytest.raises(ValueError):
+        O.layer_forward(p["x"], p["W_r"], p["b"], np.eye(d), lambda e: p["W1"][e],
+                        lambda e: p["W2"][e], None, p["W_s1"], p["W_s2"], K)
+
+
 def test_zero_w1_gives_shared_only():
     rng = np.random.default_rng(9)
     p = _rand_layer(rng, 4, 8, 4, 6, 3, 5)
@@ -388,3 +426,12 @@ def test_workload_dims_follow_the_pages_tables(golden_dir):
     # the Super layer is eq.(1) applied to a 128-expert top-6 layer at d/l = 4
     s = g["super"]
     assert O.scaling_relation(128, 6, s["d"], s["latent"])[0] == s["n_experts"]
+    # the standard-MoE comparator: the pages' 128 experts, top 6, at width d,
+    # with Super's expert widths: expert parameters N h l match in total
+    m = g["standard_moe"]
+    for name in ("std_decode", "std_prefill"):
+        c = CONFIGS[name]
+        assert not c.proj and c.l == c.d == m["d"]
+        assert (c.N, c.K) == (m["n_experts"], m["top_k"])
+        assert (c.h, c.hs) == (s["expert_hidden"], s["shared_hidden"])
+        assert c.N * c.h * c.l == s["n_experts"] * s["expert_hidden"] * s["latent"]
