@@ -160,7 +160,9 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     passed.  quant: None for the BF16 layer, or a dict with the NVFP4 global
     scales {"g_u": float, "g_h": float} for the NVFP4-expert layer, in which
     u, W1[e], W2[e] and the expert hidden activation are replaced by their
-    NVFP4 quantise-dequantise images (oracle.nvfp4).
+    NVFP4 quantise-dequantise images (oracle.nvfp4); optional "w2d" and
+    "wmse" (bool) select 2D 16x16 weight blocks and MSE-searched weight
+    block scales.
 
     Returns a dict with S, w, gap, s, z, u, v, r, hs, sh, y (float64); hs is
     the shared expert's hidden activation sqrelu(W_s1 x).
@@ -189,8 +191,9 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
         W2e = get_w2(int(e))
         if quant is not None:
             from . import nvfp4
-            W1e = nvfp4.fake_quant(W1e, nvfp4.weight_global_scale(W1e))
-            W2e = nvfp4.fake_quant(W2e, nvfp4.weight_global_scale(W2e))
+            wq = dict(block2d=quant.get("w2d", False), mse=quant.get("wmse", False))
+            W1e = nvfp4.fake_quant(W1e, nvfp4.weight_global_scale(W1e), **wq)
+            W2e = nvfp4.fake_quant(W2e, nvfp4.weight_global_scale(W2e), **wq)
             a = u_in[tok] @ W1e.T
             g = nvfp4.fake_quant(sqrelu(a), quant["g_h"])
             o = g @ W2e.T
@@ -232,8 +235,9 @@ def token_forward(x_t: np.ndarray, S_t: np.ndarray, s_t: np.ndarray,
         W2e = get_w2(int(e))
         if quant is not None:
             from . import nvfp4
-            W1e = nvfp4.fake_quant(W1e, nvfp4.weight_global_scale(W1e))
-            W2e = nvfp4.fake_quant(W2e, nvfp4.weight_global_scale(W2e))
+            wq = dict(block2d=quant.get("w2d", False), mse=quant.get("wmse", False))
+            W1e = nvfp4.fake_quant(W1e, nvfp4.weight_global_scale(W1e), **wq)
+            W2e = nvfp4.fake_quant(W2e, nvfp4.weight_global_scale(W2e), **wq)
             g = nvfp4.fake_quant(sqrelu(W1e @ u)[None, :], quant["g_h"])[0]
             o = W2e @ g
         else:

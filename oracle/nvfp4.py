@@ -13,6 +13,9 @@ Sources:
        block scales are max-based; table 5.2: latent projections stay BF16.
   [R5] section 9.3 names round-to-nearest, ties to even (RTNE) as the
        standard rounding (stochastic rounding is used only for the SSM cache).
+  [R5] section 5.3: the training recipe quantises weights with 2D blocks;
+       section 9.2 (NVFP4 PTQ): weight block scales chosen by minimising
+       the weight MSE, activation block scales max-based.
 
 Readings (the pages fix the format, not the scale arithmetic):
   * blocks are 16 consecutive elements along the last axis, which the caller
@@ -27,9 +30,22 @@ Readings (the pages fix the format, not the scale arithmetic):
         six_g = f32(6 * g); sbf = f32(amax / six_g); s_b = e4m3(sbf);
         denom = f32(s_b * g); r = f32(1 / denom), or 0 when denom == 0;
         q = e2m1(f32(x * r)) (a zero-scale block gives +-0 codes);
-  * weights use the same 1D max-based blocks as activations (the pages'
-    training recipe uses 2D weight blocks and their PTQ an MSE search; both
-    are left out of this oracle).
+  * weights use the same 1D max-based blocks as activations by default;
+    two weight variants follow the pages' other recipes:
+      - 2D blocks (block2d): one scale per 16 x 16 block of a [rows][n]
+        matrix (16 rows by 16 reduction elements), from the block's amax,
+        shared by the 16 rows; elements as above;
+      - MSE-searched scales (mse): the scale code of a block (1D or 2D) is
+        the candidate with the smallest squared quantisation error, over
+        the E4M3 codes from 8 below to 2 above the max-based code c0
+        (clipped to the positive finite codes 1..126: down to about half
+        and up to about 1.28 x the max-based scale); the error of a
+        candidate is accumulated in float32 over the block's elements in
+        row-major order, err = f32(err + f32(d * d)) with
+        d = f32(x - f32(q_value * denom)); ties go to the higher code; an
+        all-zero block keeps code 0.
+    The search range and the float32 error order are this oracle's reading
+    (the pages name the criterion, not the search).
 """
 from __future__ import annotations
 
@@ -118,39 +134,93 @@ def weight_global_scale(W: np.ndarray) -> np.float32:
     return np.float32(amax / np.float32(6.0 * E4M3_MAX))
 
 
-def quantize(X: np.ndarray, g) -> tuple:
+MSE_CODES_BELOW, MSE_CODES_ABOVE = 8, 2
+
+
+def _codes_for_scale(vals: np.ndarray, sc: np.ndarray, g32: np.float32):
+    """E2M1 codes of the rows of `vals` ([B, m] float32) under the E4M3 scale
+    codes sc [B], with the float32 scale arithmetic of the module docstring.
+    Returns (codes [B, m], denom [B] float32)."""
+    sb = e4m3_decode(sc).astype(np.float32)
+    denom = (sb * g32).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        rcp = (np.float32(1.0) / denom).astype(np.float32)
+    rcp = np.where(denom > 0, rcp, np.float32(0.0)).astype(np.float32)
+    ratio = (vals * rcp[:, None]).astype(np.float32)
+    # a block whose scale is 0 gives x * 0 = +-0: value 0, sign kept (IEEE)
+    return e2m1_rtne(ratio).astype(np.uint8), denom
+
+
+def _block_sq_error(vals: np.ndarray, codes: np.ndarray, denom: np.ndarray) -> np.ndarray:
+    """float32 squared error of each block, summed in element order."""
+    deq = (e2m1_decode(codes).astype(np.float32) * denom[:, None]).astype(np.float32)
+    d = (vals - deq).astype(np.float32)
+    err = np.zeros(vals.shape[0], dtype=np.float32)
+    for j in range(vals.shape[1]):
+        err = (err + (d[:, j] * d[:, j]).astype(np.float32)).astype(np.float32)
+    return err
+
+
+def _block_scales(vals: np.ndarray, g32: np.float32, mse: bool) -> np.ndarray:
+    """E4M3 scale code of every block ([B, m] float32 values)."""
+    amax = np.max(np.abs(vals), axis=-1)
+    six_g = np.float32(np.float32(6.0) * g32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        sbf = (amax / six_g).astype(np.float32) if six_g > 0 else np.zeros_like(amax)
+    sbf = np.where(np.isfinite(sbf), sbf, np.float32(0.0)).astype(np.float32)
+    c0 = e4m3_rtne(sbf)
+    if not mse:
+        return c0
+    best = c0.copy()
+    best_err = np.full(vals.shape[0], np.inf, dtype=np.float32)
+    base = c0.astype(np.int64)
+    for k in range(-MSE_CODES_BELOW, MSE_CODES_ABOVE + 1):
+        cand = np.clip(base + k, 1, 126).astype(np.uint8)
+        codes, denom = _codes_for_scale(vals, cand, g32)
+        err = _block_sq_error(vals, codes, denom)
+        take = err <= best_err          # ascending codes: ties go to the higher
+        best = np.where(take, cand, best)
+        best_err = np.where(take, err, best_err)
+    return np.where(base == 0, c0, best).astype(np.uint8)
+
+
+def quantize(X: np.ndarray, g, block2d: bool = False, mse: bool = False) -> tuple:
     """NVFP4 codes of X along its last axis (a multiple of 16).
 
+    block2d: X is [rows][n] with rows a multiple of 16 and each scale covers
+    16 rows x 16 elements; mse: MSE-searched block scales (module docstring).
     Returns (codes uint8 [..., n] E2M1 codes, scale_codes uint8 [..., n/16]
-    E4M3 codes, scales float32 [..., n/16] decoded block scales).
+    E4M3 codes, scales float32 [..., n/16] decoded block scales); with
+    block2d the scale of a 2D block is repeated for each of its rows.
     """
     Xf = np.asarray(X, dtype=np.float32)
     n = Xf.shape[-1]
     if n % BLOCK:
         raise ValueError("last axis must be a multiple of 16")
     g32 = np.float32(g)
-    blocks = Xf.reshape(Xf.shape[:-1] + (n // BLOCK, BLOCK))
-    amax = np.max(np.abs(blocks), axis=-1)
-    six_g = np.float32(np.float32(6.0) * g32)
-    with np.errstate(divide="ignore", invalid="ignore"):
-        sbf = (amax / six_g).astype(np.float32) if six_g > 0 else np.zeros_like(amax)
-    sbf = np.where(np.isfinite(sbf), sbf, np.float32(0.0)).astype(np.float32)
-    sc = e4m3_rtne(sbf)
+    if block2d:
+        if Xf.ndim != 2 or Xf.shape[0] % BLOCK:
+            raise ValueError("2D blocks need a [rows][n] matrix, rows a multiple of 16")
+        rows = Xf.shape[0]
+        # [row group][k block][16 rows][16 elements] -> one block per row of vals
+        t = Xf.reshape(rows // BLOCK, BLOCK, n // BLOCK, BLOCK).transpose(0, 2, 1, 3)
+        vals = np.ascontiguousarray(t).reshape(-1, BLOCK * BLOCK)
+        sc2 = _block_scales(vals, g32, mse)                       # [groups * kblocks]
+        sc = np.repeat(sc2.reshape(rows // BLOCK, 1, n // BLOCK), BLOCK, axis=1)
+        sc = sc.reshape(rows, n // BLOCK)
+    else:
+        vals = Xf.reshape(-1, BLOCK)
+        sc = _block_scales(vals, g32, mse).reshape(Xf.shape[:-1] + (n // BLOCK,))
+    blocks = Xf.reshape(-1, BLOCK)
+    codes, _ = _codes_for_scale(blocks, sc.reshape(-1), g32)
     sb = e4m3_decode(sc).astype(np.float32)
-    denom = (sb * g32).astype(np.float32)
-    with np.errstate(divide="ignore", invalid="ignore"):
-        rcp = (np.float32(1.0) / denom).astype(np.float32)
-    rcp = np.where(denom > 0, rcp, np.float32(0.0)).astype(np.float32)
-    ratio = (blocks * rcp[..., None]).astype(np.float32)
-    # a block whose scale is 0 gives x * 0 = +-0: value 0, sign kept (IEEE)
-    codes = e2m1_rtne(ratio).astype(np.uint8)
     return codes.reshape(Xf.shape), sc, sb
 
 
-def fake_quant(X: np.ndarray, g) -> np.ndarray:
+def fake_quant(X: np.ndarray, g, block2d: bool = False, mse: bool = False) -> np.ndarray:
     """Quantise-dequantise image of X (float64): q * s_b * g."""
     X = np.asarray(X)
-    codes, _, sb = quantize(X, g)
+    codes, _, sb = quantize(X, g, block2d=block2d, mse=mse)
     n = X.shape[-1]
     q = e2m1_decode(codes).reshape(X.shape[:-1] + (n // BLOCK, BLOCK))
     out = q * sb.astype(np.float64)[..., None] * np.float64(np.float32(g))

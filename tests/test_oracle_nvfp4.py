@@ -140,3 +140,123 @@ def test_fake_quant_layer_close_to_bf16_layer():
     rel = np.sqrt(np.mean((a["r"] - b["r"]) ** 2)) / np.sqrt(np.mean(a["r"] ** 2))
     assert 0.0 < rel < 0.25
     assert np.array_equal(a["sh"], b["sh"])
+
+
+# ----------------------------------------------------------------------------
+# weight-scale variants: 2D 16x16 blocks and MSE-searched block scales
+
+def _f32(v):
+    return np.float32(v)
+
+
+def _e2m1_nearest(r: float) -> float:
+    """Nearest E2M1 value to r by exhaustive search, ties to the even code,
+    saturating at +-6 (independent of the oracle's searchsorted version)."""
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    mag = min(abs(r), 6.0)
+    best = None
+    for code, gv in enumerate(grid):
+        dist = abs(mag - gv)
+        if best is None or dist < best[0] or (dist == best[0] and code % 2 == 0):
+            best = (dist, code, gv)
+    return -best[2] if np.signbit(r) else best[2]
+
+
+def _scalar_block_error(vals, code, g):
+    """Squared error of one block under E4M3 scale `code`, in float32 scalar
+    steps in element order (plain loops, no vector code)."""
+    s = _f32(Q.e4m3_decode(np.array([code]))[0])
+    denom = _f32(s * _f32(g))
+    rcp = _f32(_f32(1.0) / denom) if denom > 0 else _f32(0.0)
+    err = _f32(0.0)
+    for x in vals:
+        q = _e2m1_nearest(float(_f32(_f32(x) * rcp)))
+        deq = _f32(_f32(q) * denom)
+        d = _f32(_f32(x) - deq)
+        err = _f32(err + _f32(d * d))
+    return err
+
+
+def _scalar_mse_code(vals, g):
+    amax = max(abs(float(v)) for v in vals)
+    six_g = _f32(_f32(6.0) * _f32(g))
+    c0 = int(Q.e4m3_rtne(np.array([_f32(_f32(amax) / six_g)]))[0])
+    if c0 == 0:
+        return 0
+    best_code, best_err = None, None
+    for code in range(max(1, c0 - 8), min(126, c0 + 2) + 1):
+        e = _scalar_block_error(vals, code, g)
+        if best_err is None or e <= best_err:
+            best_code, best_err = code, e
+    return best_code
+
+
+def test_2d_block_scale_is_the_16x16_amax():
+    rng = np.random.default_rng(41)
+    W = (rng.standard_normal((48, 64)) * 0.02).astype(np.float32)
+    W[5, 17] = 0.5          # one large value: its 16x16 block's rows share it
+    g = Q.weight_global_scale(W)
+    codes, sc, sb = Q.quantize(W, g, block2d=True)
+    for rg in range(3):
+        for kb in range(4):
+            blk = W[16 * rg:16 * rg + 16, 16 * kb:16 * kb + 16]
+            want = Q.e4m3_rtne(np.array([_f32(_f32(np.abs(blk).max()) / _f32(6 * g))]))[0]
+            assert np.all(sc[16 * rg:16 * rg + 16, kb] == want)
+    # the rows sharing the large value get its scale, not their own
+    assert sc[0, 1] == sc[15, 1] and sc[0, 1] > Q.quantize(W, g)[1][0, 1]
+    # elements: the 1D quantiser's arithmetic under the shared scale
+    for r in (0, 5, 31):
+        for kb in range(4):
+            denom = _f32(_f32(sb[r, kb]) * g)
+            rcp = _f32(_f32(1.0) / denom)
+            for j in range(16):
+                want = _e2m1_nearest(float(_f32(W[r, 16 * kb + j] * rcp)))
+                assert Q.e2m1_decode(codes[r:r + 1, 16 * kb + j])[0] == want
+
+
+def test_2d_blocks_of_identical_rows_equal_1d_blocks():
+    rng = np.random.default_rng(42)
+    row = (rng.standard_normal((1, 64)) * 0.03).astype(np.float32)
+    W = np.repeat(row, 32, axis=0)
+    g = Q.weight_global_scale(W)
+    a, b = Q.quantize(W, g, block2d=True), Q.quantize(W, g)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("block2d", [False, True])
+def test_mse_scale_matches_scalar_brute_force(block2d):
+    rng = np.random.default_rng(43 + block2d)
+    W = (rng.standard_normal((32, 48)) * 0.02).astype(np.float32)
+    W[3, 5] = 0.2            # outliers make smaller scales competitive
+    W[20, 40] = -0.15
+    g = Q.weight_global_scale(W)
+    _, sc, _ = Q.quantize(W, g, block2d=block2d, mse=True)
+    for r0 in range(0, 32, 16):
+        for kb in range(3):
+            if block2d:
+                vals = W[r0:r0 + 16, 16 * kb:16 * kb + 16].reshape(-1)   # row-major
+                assert np.all(sc[r0:r0 + 16, kb] == _scalar_mse_code(vals, g))
+            else:
+                for r in (r0, r0 + 3, r0 + 15):
+                    vals = W[r, 16 * kb:16 * kb + 16]
+                    assert sc[r, kb] == _scalar_mse_code(vals, g)
+
+
+def test_mse_never_worse_than_max_based_and_keeps_grid_blocks():
+    rng = np.random.default_rng(44)
+    W = (rng.standard_normal((64, 128)) * 0.02).astype(np.float32)
+    g = Q.weight_global_scale(W)
+    f_max = Q.fake_quant(W, g)
+    f_mse = Q.fake_quant(W, g, mse=True)
+    e_max = ((W.astype(np.float64) - f_max) ** 2).reshape(-1, 16).sum(1)
+    e_mse = ((W.astype(np.float64) - f_mse) ** 2).reshape(-1, 16).sum(1)
+    assert np.all(e_mse <= e_max * (1 + 1e-5) + 1e-30)
+    assert (e_mse < e_max * (1 - 1e-3)).any()
+    # a block exactly on the E2M1 grid under its max-based scale keeps it
+    s0 = _f32(Q.e4m3_decode(np.array([0x30]))[0])    # 2^(6-7) * 1 = 0.5
+    gg = _f32(1.0 / 8)
+    blk = np.array([6, -4, 3, 1.5, 0.5, 0, -6, 2, 1, -3, 4, 0.5, -1, 6, 2, -0.5],
+                   dtype=np.float32) * _f32(s0 * gg)
+    _, sc, _ = Q.quantize(blk[None, :], gg, mse=True)
+    assert sc[0, 0] == 0x30
+    assert np.array_equal(Q.fake_quant(blk[None, :], gg, mse=True)[0], blk.astype(np.float64))
