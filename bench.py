@@ -307,7 +307,7 @@ def main():
     from lmoe_synth import act_global_scales
     layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, expert_format=cfg.fmt,
                       act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0),
-                      projections=cfg.proj)
+                      projections=cfg.proj, nvfp4_weights=cfg.wq)
     y = torch.empty_like(x)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
     stream = torch.cuda.current_stream()
@@ -380,12 +380,28 @@ def main():
         cpu = {"value": round(rate, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} of the {T} tokens of this batch, in batches of 8, {el:.1f} s"}
 
+    # NVFP4 experts: the quantisation error of the experts' combined output v
+    # against the same layer with BF16 experts (GPU against GPU, outside the
+    # timed regions), to compare the weight recipes
+    quant_err = None
+    if cfg.fmt == "nvfp4" and rank == 0:
+        v_q = layer.debug("v").float()
+        twin = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, projections=cfg.proj)
+        twin.forward(x, out=torch.empty_like(x))
+        torch.cuda.synchronize()
+        v_b = twin.debug("v").float()
+        twin.close()
+        rms = lambda t: float(torch.sqrt(torch.mean(t.double() ** 2)))
+        quant_err = {"v_rms_rel_vs_bf16_experts": round(rms(v_q - v_b) / rms(v_b), 5),
+                     "nvfp4_weights": cfg.wq}
+
     launches = layer.launches_per_forward(T) * args.steps
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if cfg.fmt == "bf16" else "e2m1 experts, bf16 dense",
             "data": "synthetic (seeded; weights N(0, std) bf16, x N(0,1) bf16)",
             "config": {"workload": cfg.name, "T": T, "d": cfg.d, "latent": cfg.l,
                        "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
@@ -396,6 +412,7 @@ def main():
             "kernels_note": "per-kernel CUDA events from a second pass of the same steps",
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clocks.summary(t_wall0, t_wall1),
+            "quantisation_error": quant_err,
             "wall_s_timed_region": round(t_wall1 - t_wall0, 4),
         }
         print(json.dumps(line), flush=True)

@@ -50,6 +50,21 @@ extern "C" {
  * 六 Table 1).  BF16 experts only. */
 #define LMOE_FLAG_NO_PROJECTION 1
 
+/* NVFP4 expert weights (lmoe_config.flags, LMOE_FMT_NVFP4 only), following
+ * the pages' other weight recipes ("Nemotron-3 Super 精读报告", section 5.3:
+ * 2D block scaling of weights in training; section 9.2: weight block scales
+ * chosen by minimum weight MSE in post-training quantisation).  Activations
+ * keep 1D max-based blocks.
+ *   LMOE_FLAG_NVFP4_WEIGHT_2D: one E4M3 scale per 16 x 16 block of W1[e] and
+ *     W2[e] (16 output rows by 16 reduction elements), from the block's amax.
+ *   LMOE_FLAG_NVFP4_WEIGHT_MSE: each block's scale is the E4M3 code, from 8
+ *     below to 2 above the max-based one, with the smallest squared error
+ *     (float32, summed in row-major element order; ties to the higher code).
+ * Both may be set (MSE search over 2D blocks).  Quantisation runs once, in
+ * lmoe_create. */
+#define LMOE_FLAG_NVFP4_WEIGHT_2D 2
+#define LMOE_FLAG_NVFP4_WEIGHT_MSE 4
+
 #define LMOE_FMT_BF16 0  /* experts in BF16                                   */
 #define LMOE_FMT_NVFP4 1 /* experts in NVFP4: W1, W2 and the expert inputs u
                             and H as E2M1 codes with E4M3 scales per 16
@@ -70,7 +85,7 @@ typedef struct lmoe_config {
   int32_t expert_hidden; /* h: expert FFN hidden width                    */
   int32_t shared_hidden; /* h_s: shared-expert hidden width               */
   int32_t expert_format; /* LMOE_FMT_*                                     */
-  int32_t flags;         /* 0, or LMOE_FLAG_NO_PROJECTION                 */
+  int32_t flags;         /* 0, or LMOE_FLAG_* bits (see above)            */
   int64_t max_tokens;    /* >= 1                                          */
 } lmoe_config;
 

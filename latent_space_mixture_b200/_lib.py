@@ -14,6 +14,10 @@ ERRORS = {-1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "OOM", -4: "CUDA", -5: "TIME
           -6: "DEVICE"}
 FMT_BF16, FMT_NVFP4 = 0, 1
 FLAG_NO_PROJECTION = 1   # standard MoE: no latent projections (u = x, r = v)
+FLAG_NVFP4_WEIGHT_2D = 2   # NVFP4 weights: one scale per 16 x 16 block
+FLAG_NVFP4_WEIGHT_MSE = 4  # NVFP4 weights: MSE-searched block scales
+NVFP4_WEIGHT_FLAGS = {"1d": 0, "2d": FLAG_NVFP4_WEIGHT_2D, "mse": FLAG_NVFP4_WEIGHT_MSE,
+                      "2d_mse": FLAG_NVFP4_WEIGHT_2D | FLAG_NVFP4_WEIGHT_MSE}
 DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 6,
        "logits": 7, "u": 8, "v": 9, "hs": 10, "w1q_codes": 11, "w1q_sf": 12, "w1q_g": 13,
        "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16}

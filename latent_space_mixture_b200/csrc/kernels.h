@@ -40,8 +40,12 @@ cudaError_t launch_combine(const void* O, const int32_t* inv, int64_t T, int K, 
 // NVFP4 (nvfp4.cu).  Expert weights [E][rows_per][K] bf16 -> codes
 // [E*rows_per][Kp/2], scale atoms [E*rows_per/128][Kp/64][512], global scales
 // [E]; amax is [E] scratch.  Kp = K rounded up to 256; padding pre-zeroed.
+// weight quantiser variants (bit set): 2D 16x16 blocks, MSE-searched scales
+constexpr int QUANT_W_2D = 1;
+constexpr int QUANT_W_MSE = 2;
 cudaError_t launch_quant_weights(const void* w, int E, int rows_per, int K, int Kp, float* amax,
-                                 uint8_t* codes, uint8_t* atoms, float* gscale, cudaStream_t st);
+                                 uint8_t* codes, uint8_t* atoms, float* gscale, int variant,
+                                 cudaStream_t st);
 // fp32 rows -> codes [rows][cols/2], scales [rows][cols/16] (canonical layout).
 cudaError_t launch_quant_rows(const float* x, int64_t rows, int cols, float g, uint8_t* codes,
                               uint8_t* scales, cudaStream_t st);

@@ -471,7 +471,11 @@ static int check_cfg(const lmoe_config* c) {
   if (!c) return LMOE_ERR_INVALID_ARG;
   if (c->d <= 0 || c->latent <= 0 || c->n_experts <= 0 || c->top_k <= 0 ||
       c->expert_hidden <= 0 || c->shared_hidden <= 0 || c->max_tokens < 1 ||
-      (c->flags & ~LMOE_FLAG_NO_PROJECTION) != 0)
+      (c->flags & ~(LMOE_FLAG_NO_PROJECTION | LMOE_FLAG_NVFP4_WEIGHT_2D |
+                    LMOE_FLAG_NVFP4_WEIGHT_MSE)) != 0)
+    return LMOE_ERR_INVALID_ARG;
+  if ((c->flags & (LMOE_FLAG_NVFP4_WEIGHT_2D | LMOE_FLAG_NVFP4_WEIGHT_MSE)) &&
+      c->expert_format != LMOE_FMT_NVFP4)
     return LMOE_ERR_INVALID_ARG;
   if ((c->flags & LMOE_FLAG_NO_PROJECTION) &&
       (c->latent != c->d || c->expert_format != LMOE_FMT_BF16))
@@ -650,11 +654,13 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= cudaMemset(h->sfbu, 0, nb_max * (lp / 64) * 512) == cudaSuccess;
     ok &= cudaMemset(h->Hq, 0, rows_b * hp / 2) == cudaSuccess;
     ok &= cudaMemset(h->sfbh, 0, nb_max * (hp / 64) * 512) == cudaSuccess;
+    const int wvar = ((c.flags & LMOE_FLAG_NVFP4_WEIGHT_2D) ? QUANT_W_2D : 0) |
+                     ((c.flags & LMOE_FLAG_NVFP4_WEIGHT_MSE) ? QUANT_W_MSE : 0);
     ok &= launch_quant_weights(w->w1, static_cast<int>(N), static_cast<int>(hh), static_cast<int>(l),
-                               static_cast<int>(lp), h->amax, h->w1q, h->w1sf, h->gw1,
+                               static_cast<int>(lp), h->amax, h->w1q, h->w1sf, h->gw1, wvar,
                                0) == cudaSuccess;
     ok &= launch_quant_weights(w->w2, static_cast<int>(N), static_cast<int>(l), static_cast<int>(hh),
-                               static_cast<int>(hp), h->amax, h->w2q, h->w2sf, h->gw2,
+                               static_cast<int>(hp), h->amax, h->w2q, h->w2sf, h->gw2, wvar,
                                0) == cudaSuccess;
     ok &= make_map_u8(&h->tm_w1q, h->w1q, N * hh, lp / 2, GEMM_BM);
     ok &= make_map_u8(&h->tm_w2q, h->w2q, N * l, hp / 2, GEMM_BM);

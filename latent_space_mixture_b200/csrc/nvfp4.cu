@@ -72,17 +72,101 @@ __global__ void __launch_bounds__(256) k_quant_weight(const __nv_bfloat16* __res
   atoms[((row / 128) * (Kp / 64) + kc) * SF_ATOM_BYTES + sf_atom_offset(static_cast<int>(row % 128), k1)] = sc;
 }
 
+// Weight variants ("Nemotron-3 Super 精读报告", section 5.3: 2D block scaling
+// of weights; section 9.2: weight block scales chosen by minimum MSE).  One
+// thread per scale unit: a (row, 16-block) in 1D, a (16-row group, 16-block)
+// in 2D, whose 16 rows share the scale.  MSE: the candidates are the E4M3
+// codes from 8 below to 2 above the max-based code (clipped to 1..126), the
+// error is the float32 sum in row-major element order, ties go to the higher
+// code, an all-zero unit keeps code 0.
+template <bool TWO_D, bool MSE>
+__global__ void __launch_bounds__(128) k_quant_weight_var(const __nv_bfloat16* __restrict__ w,
+                                                          int64_t rows, int rows_per, int K,
+                                                          int Kp, const float* __restrict__ amax,
+                                                          uint8_t* __restrict__ codes,
+                                                          uint8_t* __restrict__ atoms,
+                                                          float* __restrict__ gscale) {
+  constexpr int R = TWO_D ? 16 : 1;   // rows per unit
+  const int kb16 = K / 16;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= (rows / R) * kb16) return;
+  const int64_t row0 = (i / kb16) * R;
+  const int blk = static_cast<int>(i - (i / kb16) * kb16);
+  const int e = static_cast<int>(row0 / rows_per);
+  const float g = __fdiv_rn(amax[e], 6.0f * 448.0f);
+  if (blk == 0 && row0 % rows_per == 0) gscale[e] = g;
+  auto load = [&](int r, float (&x)[16]) {
+    const __nv_bfloat162* src =
+        reinterpret_cast<const __nv_bfloat162*>(w + (row0 + r) * K + blk * 16);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float2 f = __bfloat1622float2(src[j]);
+      x[2 * j] = f.x;
+      x[2 * j + 1] = f.y;
+    }
+  };
+  float x[16];
+  float m = 0.0f;
+  for (int r = 0; r < R; ++r) {
+    load(r, x);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(x[j]));
+  }
+  const float six_g = __fmul_rn(6.0f, g);
+  const uint8_t c0 = e4m3_code(six_g > 0.0f ? __fdiv_rn(m, six_g) : 0.0f);
+  uint8_t sc = c0;
+  if (MSE && c0 != 0) {
+    float best = __int_as_float(0x7f800000);   // +inf
+    const int lo = c0 > 9 ? c0 - 8 : 1, hi = c0 < 124 ? c0 + 2 : 126;
+    for (int c = lo; c <= hi; ++c) {
+      float err = 0.0f;
+      for (int r = 0; r < R; ++r) {
+        load(r, x);
+        err = nvfp4_sq_error(x, g, static_cast<uint8_t>(c), err);
+      }
+      if (err <= best) {
+        best = err;
+        sc = static_cast<uint8_t>(c);
+      }
+    }
+  }
+  const int kc = blk / 4, k1 = blk % 4;
+  for (int r = 0; r < R; ++r) {
+    const int64_t row = row0 + r;
+    load(r, x);
+    uint8_t q[8];
+    nvfp4_codes_with_scale(x, g, sc, q);
+    *reinterpret_cast<uint2*>(codes + row * (Kp / 2) + blk * 8) = *reinterpret_cast<const uint2*>(q);
+    atoms[((row / 128) * (Kp / 64) + kc) * SF_ATOM_BYTES + sf_atom_offset(static_cast<int>(row % 128), k1)] = sc;
+  }
+}
+
 cudaError_t launch_quant_weights(const void* w, int E, int rows_per, int K, int Kp, float* amax,
-                                 uint8_t* codes, uint8_t* atoms, float* gscale, cudaStream_t st) {
+                                 uint8_t* codes, uint8_t* atoms, float* gscale, int variant,
+                                 cudaStream_t st) {
   if (cudaMemsetAsync(amax, 0, E * sizeof(float), st) != cudaSuccess) return cudaGetLastError();
   const int64_t per = static_cast<int64_t>(rows_per) * K;
   k_amax_expert<<<dim3(64, E), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), per, amax);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(E) * rows_per;
-  const int64_t n = rows * (K / 16);
-  k_quant_weight<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(w), rows, rows_per, K, Kp, amax, codes, atoms, gscale);
+  const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(w);
+  const bool two_d = variant & QUANT_W_2D, mse = variant & QUANT_W_MSE;
+  if (!two_d && !mse) {
+    const int64_t n = rows * (K / 16);
+    k_quant_weight<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        wb, rows, rows_per, K, Kp, amax, codes, atoms, gscale);
+    return cudaGetLastError();
+  }
+  if (two_d && rows_per % 16) return cudaErrorInvalidValue;
+  const int64_t n = (two_d ? rows / 16 : rows) * (K / 16);
+  const unsigned blocks = static_cast<unsigned>((n + 127) / 128);
+  if (two_d && mse)
+    k_quant_weight_var<true, true><<<blocks, 128, 0, st>>>(wb, rows, rows_per, K, Kp, amax, codes, atoms, gscale);
+  else if (two_d)
+    k_quant_weight_var<true, false><<<blocks, 128, 0, st>>>(wb, rows, rows_per, K, Kp, amax, codes, atoms, gscale);
+  else
+    k_quant_weight_var<false, true><<<blocks, 128, 0, st>>>(wb, rows, rows_per, K, Kp, amax, codes, atoms, gscale);
   return cudaGetLastError();
 }
 

@@ -47,6 +47,42 @@ __device__ __forceinline__ float e4m3_value(uint8_t code) {
   return __half2float(__half(h));
 }
 
+// E2M1 code (bit 3 = sign) -> value
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+  const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  const float v = mag[code & 7];
+  return (code & 8) ? -v : v;
+}
+
+// Codes of 16 elements under a given E4M3 scale code (the arithmetic of
+// nvfp4_block after its scale choice).
+__device__ __forceinline__ void nvfp4_codes_with_scale(const float (&x)[16], float g, uint8_t sc,
+                                                       uint8_t (&out)[8]) {
+  const float denom = __fmul_rn(e4m3_value(sc), g);
+  const float r = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    out[i] = static_cast<uint8_t>(e2m1x2(__fmul_rn(x[2 * i], r), __fmul_rn(x[2 * i + 1], r)));
+}
+
+// Continue a float32 squared-error sum over 16 elements quantised with scale
+// code sc, in element order: err += (x - q * denom)^2, every step rounded
+// (no fused multiply-add), as the MSE scale search of the weight quantiser.
+__device__ __forceinline__ float nvfp4_sq_error(const float (&x)[16], float g, uint8_t sc,
+                                                float err) {
+  const float denom = __fmul_rn(e4m3_value(sc), g);
+  const float r = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t b = e2m1x2(__fmul_rn(x[2 * i], r), __fmul_rn(x[2 * i + 1], r));
+    const float d0 = __fsub_rn(x[2 * i], __fmul_rn(e2m1_value(b & 15), denom));
+    err = __fadd_rn(err, __fmul_rn(d0, d0));
+    const float d1 = __fsub_rn(x[2 * i + 1], __fmul_rn(e2m1_value(b >> 4), denom));
+    err = __fadd_rn(err, __fmul_rn(d1, d1));
+  }
+  return err;
+}
+
 // Quantise one 16-element block: returns the E4M3 scale code and writes the 8
 // packed bytes of codes.
 __device__ __forceinline__ uint8_t nvfp4_block(const float (&x)[16], float g, uint8_t (&out)[8]) {

@@ -10,8 +10,8 @@ from typing import Dict, Optional
 import torch
 
 from . import _lib
-from ._lib import (DBG, FLAG_NO_PROJECTION, FMT_BF16, FMT_NVFP4, LmoeConfig, LmoeError,
-                   LmoeWeights, check)
+from ._lib import (DBG, FLAG_NO_PROJECTION, FMT_BF16, FMT_NVFP4, NVFP4_WEIGHT_FLAGS,
+                   LmoeConfig, LmoeError, LmoeWeights, check)
 
 __all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]
 
@@ -34,11 +34,14 @@ class LatentMoE:
     and optionally router_bias [N] fp32.  The library copies them.
     projections=False builds the standard MoE (latent = d, no w_dn / w_upl:
     the experts work on x and their combined output is added as is).
+    nvfp4_weights ("1d", "2d", "mse", "2d_mse") picks the NVFP4 weight blocks
+    and scale choice (LMOE_FLAG_NVFP4_WEIGHT_* of the C ABI).
     """
 
     def __init__(self, d: int, latent: int, n_experts: int, top_k: int, expert_hidden: int,
                  shared_hidden: int, max_tokens: int, weights: Dict[str, torch.Tensor],
-                 expert_format: str = "bf16", act_gscales=(0.0, 0.0), projections: bool = True):
+                 expert_format: str = "bf16", act_gscales=(0.0, 0.0), projections: bool = True,
+                 nvfp4_weights: str = "1d"):
         self.lib = _lib.load()
         dims = {"d": d, "l": latent, "N": n_experts, "h": expert_hidden, "hs": shared_hidden}
         for k, shape in _WEIGHT_SHAPES.items():
@@ -56,7 +59,8 @@ class LatentMoE:
             raise ValueError("router_bias: need CUDA fp32 [N]")
         self.cfg = LmoeConfig(d, latent, n_experts, top_k, expert_hidden, shared_hidden,
                               {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4}[expert_format],
-                              0 if projections else FLAG_NO_PROJECTION, max_tokens)
+                              (0 if projections else FLAG_NO_PROJECTION)
+                              | NVFP4_WEIGHT_FLAGS[nvfp4_weights], max_tokens)
         w = LmoeWeights(weights["w_router"].data_ptr(),
                         bias.data_ptr() if bias is not None else None,
                         weights["w_dn"].data_ptr() if projections else None,

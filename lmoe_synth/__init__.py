@@ -50,6 +50,7 @@ class LayerConfig:
     seed: int
     fmt: str = "bf16"  # expert format: "bf16" or "nvfp4"
     proj: bool = True  # latent projections W_dn, W_upl (False: standard MoE, l = d)
+    wq: str = "1d"     # NVFP4 weight blocks/scales: "1d", "2d", "mse" or "2d_mse"
 
     def with_(self, **kw) -> "LayerConfig":
         return replace(self, **kw)
@@ -88,6 +89,12 @@ CONFIGS: Dict[str, LayerConfig] = {
     "super_prefill_nvfp4": LayerConfig("super_prefill_nvfp4", 8192, 4096, 1024,
                                        512, 22, 2688, 5376, 0.02, "zipf", 4,
                                        "nvfp4"),
+    # Super prefill with NVFP4 experts whose weights use the pages' other
+    # recipes: 2D 16x16 blocks (training) and MSE-searched scales (PTQ)
+    "super_prefill_nvfp4_2d": LayerConfig("super_prefill_nvfp4_2d", 8192, 4096, 1024, 512, 22,
+                                          2688, 5376, 0.02, "zipf", 4, "nvfp4", wq="2d"),
+    "super_prefill_nvfp4_mse": LayerConfig("super_prefill_nvfp4_mse", 8192, 4096, 1024, 512, 22,
+                                           2688, 5376, 0.02, "zipf", 4, "nvfp4", wq="mse"),
     # the standard-MoE comparator: tiny, decode- and prefill-sized
     "tiny_std": LayerConfig("tiny_std", 64, 256, 256, 32, 4, 128, 256, 0.02, "zipf", 10,
                             proj=False),

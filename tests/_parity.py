@@ -53,7 +53,7 @@ def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None):
     layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs,
                       max_tokens or x.shape[0], w, expert_format=cfg.fmt,
                       act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0),
-                      projections=cfg.proj)
+                      projections=cfg.proj, nvfp4_weights=cfg.wq)
     return w, x, layer
 
 
@@ -63,7 +63,8 @@ def quant_of(cfg):
     if cfg.fmt != "nvfp4":
         return None
     g_u, g_h = act_global_scales(cfg)
-    return {"g_u": float(np.float32(g_u)), "g_h": float(np.float32(g_h))}
+    return {"g_u": float(np.float32(g_u)), "g_h": float(np.float32(g_h)),
+            "w2d": cfg.wq in ("2d", "2d_mse"), "wmse": cfg.wq in ("mse", "2d_mse")}
 
 
 def oracle_tokens(w, x_rows: torch.Tensor, K: int, quant=None):

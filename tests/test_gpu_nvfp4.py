@@ -63,9 +63,11 @@ def _weights_from_atoms(codes, atoms, rows, K, Kp):
     return q, sc
 
 
-def test_quantised_weights_bit_exact():
-    cfg = CONFIGS["tiny_nvfp4"]
+@pytest.mark.parametrize("wq", ["1d", "2d", "mse", "2d_mse"])
+def test_quantised_weights_bit_exact(wq):
+    cfg = CONFIGS["tiny_nvfp4"].with_(wq=wq)
     w, x, layer = make(cfg)
+    opt = dict(block2d=wq in ("2d", "2d_mse"), mse=wq in ("mse", "2d_mse"))
     lp, hp = (cfg.l + 255) // 256 * 256, (cfg.h + 255) // 256 * 256
     for name, R, K, Kp in (("w1", cfg.h, cfg.l, lp), ("w2", cfg.l, cfg.h, hp)):
         codes = layer.debug(name + "q_codes").numpy()
@@ -76,7 +78,7 @@ def test_quantised_weights_bit_exact():
             We = w[name][e].float().cpu().numpy()
             ge = Q.weight_global_scale(We)
             assert g[e] == ge
-            oc, osc, _ = Q.quantize(We, ge)
+            oc, osc, _ = Q.quantize(We, ge, **opt)
             assert np.array_equal(sc[e * R:(e + 1) * R], osc), (name, e)
             assert np.array_equal(Q.e2m1_decode(q[e * R:(e + 1) * R]), Q.e2m1_decode(oc)), (name, e)
         # padding beyond K holds zero codes
@@ -84,16 +86,17 @@ def test_quantised_weights_bit_exact():
     layer.close()
 
 
-@pytest.mark.parametrize("T", [64, 37, 5])
-def test_tiny_nvfp4_layer(T):
-    cfg = CONFIGS["tiny_nvfp4"]
+@pytest.mark.parametrize("T,wq", [(64, "1d"), (37, "1d"), (5, "1d"), (64, "2d"), (37, "mse"),
+                                  (64, "2d_mse")])
+def test_tiny_nvfp4_layer(T, wq):
+    cfg = CONFIGS["tiny_nvfp4"].with_(wq=wq)
     w, x, layer = make(cfg, T=T)
     y = layer.forward(x)
     torch.cuda.synchronize()
     assert layer.sync_status() == 0
     errs = compare_layer(layer, w, x, y, np.arange(T), cfg.K, tol=TOL_NVFP4, quant=quant_of(cfg),
                          elem_rel=2.0 ** -7, check_v=False)
-    print("tiny_nvfp4", T, errs)
+    print("tiny_nvfp4", T, wq, errs)
     assert errs["v_rms_rel"] <= TOL_NVFP4
     layer.close()
 
@@ -112,4 +115,26 @@ def test_super_prefill_nvfp4_sampled_tokens():
                          check_v=False)
     print("super_prefill_nvfp4", errs)
     assert errs["v_rms_rel"] <= TOL_NVFP4
+    layer.close()
+
+
+def test_quantised_weights_bit_exact_at_super_widths():
+    """The 2D + MSE weight quantiser on Super-width expert matrices (l = 1024,
+    h = 2688: many K blocks, 16-row groups across 128-row scale atoms), first
+    and last expert (the oracle's MSE search costs seconds per matrix)."""
+    cfg = CONFIGS["tiny_nvfp4"].with_(l=1024, h=2688, N=32, wq="2d_mse")
+    w, x, layer = make(cfg)
+    lp, hp = (cfg.l + 255) // 256 * 256, (cfg.h + 255) // 256 * 256
+    for name, R, K, Kp in (("w1", cfg.h, cfg.l, lp), ("w2", cfg.l, cfg.h, hp)):
+        codes = layer.debug(name + "q_codes").numpy()
+        atoms = layer.debug(name + "q_sf").numpy()
+        g = layer.debug(name + "q_g").numpy()
+        q, sc = _weights_from_atoms(codes, atoms, cfg.N * R, K, Kp)
+        for e in (0, cfg.N - 1):
+            We = w[name][e].float().cpu().numpy()
+            ge = Q.weight_global_scale(We)
+            assert g[e] == ge
+            oc, osc, _ = Q.quantize(We, ge, block2d=True, mse=True)
+            assert np.array_equal(sc[e * R:(e + 1) * R], osc), (name, e)
+            assert np.array_equal(Q.e2m1_decode(q[e * R:(e + 1) * R]), Q.e2m1_decode(oc)), (name, e)
     layer.close()
