@@ -143,6 +143,22 @@ def expert_ffn(U: np.ndarray, W1e: np.ndarray, W2e: np.ndarray) -> np.ndarray:
     return sqrelu(U @ W1e.T) @ W2e.T
 
 
+def _expert_quantisers(quant: Dict):
+    """(q_u, q_w, q_h): quantise-dequantise maps of the expert inputs u, an
+    expert weight matrix and the expert hidden activation, for the NVFP4
+    ("fmt" absent or "nvfp4") or the FP8 W8A8 ("fmt": "fp8") expert layer."""
+    if quant.get("fmt", "nvfp4") == "fp8":
+        from . import fp8
+        return (lambda a: fp8.fake_quant(a, quant["s_u"]),
+                lambda W: fp8.fake_quant(W, fp8.weight_scale(W)),
+                lambda a: fp8.fake_quant(a, quant["s_h"]))
+    from . import nvfp4
+    wq = dict(block2d=quant.get("w2d", False), mse=quant.get("wmse", False))
+    return (lambda a: nvfp4.fake_quant(a, quant["g_u"]),
+            lambda W: nvfp4.fake_quant(W, nvfp4.weight_global_scale(W), **wq),
+            lambda a: nvfp4.fake_quant(a, quant["g_h"]))
+
+
 def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
                   W_dn: Optional[np.ndarray], get_w1: Callable[[int], np.ndarray],
                   get_w2: Callable[[int], np.ndarray], W_upl: Optional[np.ndarray],
@@ -162,7 +178,8 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     u, W1[e], W2[e] and the expert hidden activation are replaced by their
     NVFP4 quantise-dequantise images (oracle.nvfp4); optional "w2d" and
     "wmse" (bool) select 2D 16x16 weight blocks and MSE-searched weight
-    block scales.
+    block scales.  quant = {"fmt": "fp8", "s_u": float, "s_h": float} is the
+    FP8 W8A8 expert layer (oracle.fp8: E4M3, per-tensor scales).
 
     Returns a dict with S, w, gap, s, z, u, v, r, hs, sh, y (float64); hs is
     the shared expert's hidden activation sqrelu(W_s1 x).
@@ -179,8 +196,8 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     # 3: latent down-projection (none for the standard MoE)
     u = x.copy() if W_dn is None else x @ W_dn.T
     if quant is not None:
-        from . import nvfp4
-        u_in = nvfp4.fake_quant(u, quant["g_u"])
+        q_u, q_w, q_h = _expert_quantisers(quant)
+        u_in = q_u(u)
     else:
         u_in = u
     # 4-5: experts in latent space, weighted sum in latent space
@@ -190,12 +207,8 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
         W1e = get_w1(int(e))
         W2e = get_w2(int(e))
         if quant is not None:
-            from . import nvfp4
-            wq = dict(block2d=quant.get("w2d", False), mse=quant.get("wmse", False))
-            W1e = nvfp4.fake_quant(W1e, nvfp4.weight_global_scale(W1e), **wq)
-            W2e = nvfp4.fake_quant(W2e, nvfp4.weight_global_scale(W2e), **wq)
-            a = u_in[tok] @ W1e.T
-            g = nvfp4.fake_quant(sqrelu(a), quant["g_h"])
+            W1e, W2e = q_w(W1e), q_w(W2e)
+            g = q_h(sqrelu(u_in[tok] @ W1e.T))
             o = g @ W2e.T
         else:
             o = expert_ffn(u_in[tok], W1e, W2e)
@@ -227,18 +240,15 @@ def token_forward(x_t: np.ndarray, S_t: np.ndarray, s_t: np.ndarray,
     w = sel / sel.sum()
     u = x_t.copy() if W_dn is None else W_dn @ x_t
     if quant is not None:
-        from . import nvfp4
-        u = nvfp4.fake_quant(u[None, :], quant["g_u"])[0]
+        q_u, q_w, q_h = _expert_quantisers(quant)
+        u = q_u(u[None, :])[0]
     v = np.zeros(u.shape[0], dtype=np.float64)
     for k, e in enumerate(S_t):
         W1e = get_w1(int(e))
         W2e = get_w2(int(e))
         if quant is not None:
-            from . import nvfp4
-            wq = dict(block2d=quant.get("w2d", False), mse=quant.get("wmse", False))
-            W1e = nvfp4.fake_quant(W1e, nvfp4.weight_global_scale(W1e), **wq)
-            W2e = nvfp4.fake_quant(W2e, nvfp4.weight_global_scale(W2e), **wq)
-            g = nvfp4.fake_quant(sqrelu(W1e @ u)[None, :], quant["g_h"])[0]
+            W1e, W2e = q_w(W1e), q_w(W2e)
+            g = q_h(sqrelu(W1e @ u)[None, :])[0]
             o = W2e @ g
         else:
             o = W2e @ sqrelu(W1e @ u)
