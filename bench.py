@@ -65,25 +65,35 @@ def algorithmic_work(cfg, T: int, counts: np.ndarray):
     own operands and results; flops count real rows only (no tile padding).
     Without projections (the standard MoE) the x-GEMM has no W_dn rows, the
     y-GEMM no W_upl columns, and it reads v once more for the residual add.
+    Quantised experts: expert weights and expert inputs at their format's
+    bytes per element (NVFP4 0.5 + one E4M3 scale per 16 = 0.5625, FP8 1),
+    and the grouped GEMMs' peak is the BF16 peak times the format's nominal
+    tensor ratio ("mult": FP4 9/2.25 = 4, FP8 4.5/2.25 = 2).
     """
     d, l, N, K, h, hs = cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs
     lx = l if cfg.proj else 0
+    eb = {"bf16": 2.0, "nvfp4": 0.5625, "fp8": 1.0}[cfg.fmt]
+    mult = {"bf16": 1, "nvfp4": 4, "fp8": 2}[cfg.fmt]
     touched = int((counts > 0).sum())
     R = T * K
     wx = (N + lx + hs) * d * 2
     wy = d * (lx + hs) * 2
-    wexp = touched * h * l * 2
+    wexp = int(touched * h * l * eb)
     per_kernel = {
         "xgemm(router|W_dn|W_s1)": dict(bytes=wx + T * d * 2 + T * (N * 4 + lx * 2 + hs * 2),
                                         flops=2 * T * d * (N + lx + hs)),
-        "grouped_gemm1(W1,sqrelu)": dict(bytes=wexp + R * l * 2 + R * h * 2, flops=2 * R * l * h),
-        "grouped_gemm2(W2,*w)": dict(bytes=wexp + R * h * 2 + R * l * 2 + R * 4,
-                                     flops=2 * R * h * l),
+        "grouped_gemm1(W1,sqrelu)": dict(bytes=int(wexp + R * l * eb + R * h * eb),
+                                         flops=2 * R * l * h, mult=mult),
+        "grouped_gemm2(W2,*w)": dict(bytes=int(wexp + R * h * eb + R * l * 2 + R * 4),
+                                     flops=2 * R * h * l, mult=mult),
         "ygemm([W_upl|W_s2])": dict(bytes=wy + T * (l + hs) * 2 + T * d * 2,
                                     flops=2 * T * d * (lx + hs)),
     }
     layer = dict(bytes=wx + wy + 2 * wexp + 2 * T * d * 2,
-                 flops=sum(v["flops"] for v in per_kernel.values()))
+                 flops=sum(v["flops"] for v in per_kernel.values()),
+                 # tensor time at the peaks, in units of BF16 flops
+                 bf16_equiv_flops=sum(v["flops"] / v.get("mult", 1)
+                                      for v in per_kernel.values()))
     return layer, per_kernel
 
 
@@ -91,7 +101,9 @@ def roofline_entry(name, kw, total_ms, launches, peaks, peak_kind, cfg, T):
     """The roofline object of one kernel from its live CUDA-event times."""
     avg_s = total_ms / 1e3 / max(launches, 1)
     intensity = kw["flops"] / kw["bytes"]
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    mult = kw.get("mult", 1)
+    p_t = peaks["bf16_tflops"] * mult
+    ridge = p_t * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if intensity < ridge:
         achieved = kw["bytes"] / avg_s / 1e9
         return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1),
@@ -100,11 +112,14 @@ def roofline_entry(name, kw, total_ms, launches, peaks, peak_kind, cfg, T):
                 "alg_bytes_per_launch": kw["bytes"], "avg_launch_us": round(avg_s * 1e6, 2),
                 "peak_source": peak_kind + " hbm_gbs"}
     achieved = kw["flops"] / avg_s / 1e12
+    src = peak_kind + " bf16_tflops (burst)"
+    if mult != 1:
+        src += f" x {mult} ({'FP4' if mult == 4 else 'FP8'}/BF16 nominal dense ratio)"
     return {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1),
-            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+            "peak": round(p_t, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / p_t, 4), "traffic": None,
             "alg_flops_per_launch": kw["flops"], "avg_launch_us": round(avg_s * 1e6, 2),
-            "peak_source": peak_kind + " bf16_tflops (burst)"}
+            "peak_source": src}
 
 
 def measured_traffic(workload: str, kernel: str):
@@ -306,7 +321,7 @@ def main():
     T = cfg.T
     from lmoe_synth import act_global_scales
     layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, expert_format=cfg.fmt,
-                      act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0),
+                      act_gscales=act_global_scales(cfg) if cfg.fmt != "bf16" else (0.0, 0.0),
                       projections=cfg.proj, nvfp4_weights=cfg.wq)
     y = torch.empty_like(x)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
@@ -356,8 +371,9 @@ def main():
     layer_time_s = ms_per_step / 1e3
     layer_roof = {"alg_bytes": lay["bytes"], "alg_flops": lay["flops"],
                   "hbm_frac": round(lay["bytes"] / layer_time_s / 1e9 / peaks["hbm_gbs"], 4),
-                  "tensor_frac": round(lay["flops"] / layer_time_s / 1e12 / peaks["bf16_tflops"],
-                                       4),
+                  # time roofline: each contraction at its own dtype's peak
+                  "tensor_frac": round(lay["bf16_equiv_flops"] / layer_time_s / 1e12
+                                       / peaks["bf16_tflops"], 4),
                   "tflops": round(lay["flops"] / layer_time_s / 1e12, 2)}
 
     # end to end through host buffers
@@ -380,11 +396,11 @@ def main():
         cpu = {"value": round(rate, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} of the {T} tokens of this batch, in batches of 8, {el:.1f} s"}
 
-    # NVFP4 experts: the quantisation error of the experts' combined output v
-    # against the same layer with BF16 experts (GPU against GPU, outside the
-    # timed regions), to compare the weight recipes
+    # quantised experts (NVFP4, FP8): the quantisation error of the experts'
+    # combined output v against the same layer with BF16 experts (GPU against
+    # GPU, outside the timed regions), to compare formats and weight recipes
     quant_err = None
-    if cfg.fmt == "nvfp4" and rank == 0:
+    if cfg.fmt != "bf16" and rank == 0:
         v_q = layer.debug("v").float()
         twin = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, projections=cfg.proj)
         twin.forward(x, out=torch.empty_like(x))
@@ -393,7 +409,9 @@ def main():
         twin.close()
         rms = lambda t: float(torch.sqrt(torch.mean(t.double() ** 2)))
         quant_err = {"v_rms_rel_vs_bf16_experts": round(rms(v_q - v_b) / rms(v_b), 5),
-                     "nvfp4_weights": cfg.wq}
+                     "format": cfg.fmt}
+        if cfg.fmt == "nvfp4":
+            quant_err["nvfp4_weights"] = cfg.wq
 
     launches = layer.launches_per_forward(T) * args.steps
     if rank == 0:
@@ -401,7 +419,8 @@ def main():
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if cfg.fmt == "bf16" else "e2m1 experts, bf16 dense",
+            "dtype": {"bf16": "bf16", "nvfp4": "e2m1 experts, bf16 dense",
+                      "fp8": "e4m3 experts, bf16 dense"}[cfg.fmt],
             "data": "synthetic (seeded; weights N(0, std) bf16, x N(0,1) bf16)",
             "config": {"workload": cfg.name, "T": T, "d": cfg.d, "latent": cfg.l,
                        "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,

@@ -72,9 +72,16 @@ extern "C" {
                             global scale; latent projections, router and
                             shared expert stay BF16 ("Nemotron-3 Super 精读报告",
                             table 5.2).  Needs l and h multiples of 128.      */
+#define LMOE_FMT_FP8 2   /* experts in FP8 W8A8 ("Nemotron-3 Super 精读报告",
+                            section 9.1): W1, W2, u and H as E4M3 codes with
+                            one FP32 scale per tensor (s_W = amax / 448 per
+                            expert matrix, static scales for u and H from
+                            act_gscale_*), value = code * s; router, latent
+                            projections and shared expert stay BF16.  Needs
+                            l and h multiples of 128.                        */
 
 /* Layer shape.  d, latent, expert_hidden, shared_hidden: multiples of 64
- * (latent and expert_hidden multiples of 128 for LMOE_FMT_NVFP4).
+ * (latent and expert_hidden multiples of 128 for LMOE_FMT_NVFP4 and _FP8).
  * n_experts: multiple of 32, at most 1024.  top_k: 1..min(32, n_experts).
  * max_tokens: the largest T a forward call accepts (sizes the workspace). */
 typedef struct lmoe_config {
@@ -100,9 +107,11 @@ typedef struct lmoe_weights {
   const void* w_upl;       /* [d][l]      bf16 (unused without projections) */
   const void* w_s1;        /* [h_s][d]    bf16                              */
   const void* w_s2;        /* [d][h_s]    bf16                              */
-  float act_gscale_latent; /* NVFP4 only (> 0): static global scale of u;
-                              its block scales are E4M3(amax16/(6 g))       */
-  float act_gscale_hidden; /* NVFP4 only (> 0): static global scale of the
+  float act_gscale_latent; /* NVFP4 and FP8 only (> 0): static scale of u --
+                              NVFP4: global scale under the E4M3 block
+                              scales E4M3(amax16/(6 g)); FP8: the per-tensor
+                              scale, u = code * s                            */
+  float act_gscale_hidden; /* NVFP4 and FP8 only (> 0): the same for the
                               expert hidden activation sqrelu(W1 u)         */
 } lmoe_weights;
 

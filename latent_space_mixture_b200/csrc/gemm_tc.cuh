@@ -14,8 +14,9 @@
 //               in the NVFP4 variant also the two scale-factor tiles (bulk
 //               copies of 2 KB);
 //   warp 1      TMEM allocator and MMA issuer: per k-step 4 MMAs of K=16
-//               (kind::f16, bf16) or K=64 (kind::mxf4nvf4 with 16-element
-//               block scales copied into TMEM by tcgen05.cp first);
+//               (kind::f16, bf16), K=64 (kind::mxf4nvf4 with 16-element
+//               block scales copied into TMEM by tcgen05.cp first) or K=32
+//               (kind::f8f6f4, E4M3);
 //               tcgen05.commit frees the smem stage, and at the end of a tile
 //               marks the accumulator full;
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, transpose through a
@@ -45,6 +46,11 @@ constexpr int GEMM_BROWS = 16;        // rows per small B TMA box (ragged tails)
 constexpr int GEMM_BROWS_BIG = 64;    // rows per large B TMA box (full row groups)
 constexpr int GEMM_ROW_BYTES = 128;   // bytes of one operand row per stage
 constexpr int FP4_K_PER_STAGE = 256;  // NVFP4 K elements per stage (128 B per row)
+constexpr int FP8_K_PER_STAGE = 128;  // FP8 (E4M3) K elements per stage (128 B per row)
+// operand kinds of the GEMM (template parameter KIND)
+constexpr int KIND_BF16 = 0;   // kind::f16, bf16 A and B, K = 16 per MMA
+constexpr int KIND_NVFP4 = 1;  // kind::mxf4nvf4 block16 with E4M3 block scales, K = 64
+constexpr int KIND_FP8 = 2;    // kind::f8f6f4, E4M3 A and B, K = 32
 constexpr int FP4_SF_STAGE_BYTES = 4 * SF_ATOM_BYTES;   // 4 chunks of K=64
 
 // Where the tiles of one GEMM come from.
@@ -56,7 +62,7 @@ struct TileSource {
   int FB;                  // feature blocks of 128 per expert
   int a_rows_per_expert;   // rows of A per expert (0 when dense)
   int m_valid;             // valid features per expert (multiple of 8)
-  int kblocks;             // K steps (K/64 bf16, K/256 NVFP4)
+  int kblocks;             // K steps (K/64 bf16, K/256 NVFP4, K/128 FP8)
   int ksplit;              // dense only: K slices (1 = none); each slice writes
   float* part;             //   fp32 partials part[slice][row][feature]
   int a_stream_once;       // 1: each A tile is read by one tile only (L2 evict-first)
@@ -98,8 +104,9 @@ __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int t
   return t;
 }
 
-template <int BN, int STAGES, bool FP4>
+template <int BN, int STAGES, int KIND>
 struct GemmLayout {
+  static constexpr bool FP4 = KIND == KIND_NVFP4;
   static constexpr int A_BYTES = GEMM_BM * GEMM_ROW_BYTES;
   static constexpr int B_BYTES = BN * GEMM_ROW_BYTES;
   static constexpr int SF_BYTES = FP4 ? 2 * FP4_SF_STAGE_BYTES : 0;
@@ -130,12 +137,14 @@ __device__ __forceinline__ bool empty_waits_at(int s) { return !L::PAIRED_RELEAS
 template <class L>
 __device__ __forceinline__ bool empty_commits_at(int s) { return !L::PAIRED_RELEASE || (s & 1); }
 
-template <int BN, int STAGES, class Epi, bool FP4>
+template <int BN, int STAGES, class Epi, int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmB64, const TileSource src, const Epi epi, int* err,
           unsigned long long limit_ns) {
-  using L = GemmLayout<BN, STAGES, FP4>;
+  using L = GemmLayout<BN, STAGES, KIND>;
+  constexpr bool FP4 = KIND == KIND_NVFP4;
+  constexpr bool F8 = KIND == KIND_FP8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -196,7 +205,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     auto load_b = [&](int st, const TileInfo& t, int kb) {
       const int nbig = t.nrows / GEMM_BROWS_BIG;
       const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
-      const int bx = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+      const int bx = KIND != KIND_BF16 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
       uint8_t* b_dst = sB + st * L::B_BYTES;
       for (int j = 0; j < nbig; ++j)
         tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
@@ -230,8 +239,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           ok = false;
           break;
         }
-        // x coordinate in elements of the map: bf16 elements or bytes (NVFP4)
-        const int ax = FP4 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+        // x coordinate in elements of the map: bf16 elements or bytes (NVFP4, FP8)
+        const int ax = KIND != KIND_BF16 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
         if (elect_one()) {
           mbar_arrive_expect_tx(&full[stage], tx);
           tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, ax, t.a_row, &full[stage], pol_a);
@@ -298,7 +307,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
-      const uint32_t idesc = FP4 ? idesc_nvf4(GEMM_BM, n_mma) : idesc_bf16(GEMM_BM, n_mma);
+      const uint32_t idesc = FP4  ? idesc_nvf4(GEMM_BM, n_mma)
+                             : F8 ? idesc_f8(GEMM_BM, n_mma)
+                                  : idesc_bf16(GEMM_BM, n_mma);
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (!__all_sync(0xffffffffu,
                         mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns))) {
@@ -325,6 +336,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             for (int k = 0; k < 4; ++k)   // +32 bytes per K=64 step
               umma_nvf4(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, tmem_base + sf_col + 4 * k,
                         tmem_base + sf_col + 16 + 4 * k, (kb != t.kb0) || (k != 0));
+          } else if constexpr (F8) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)   // +32 bytes per K=32 step
+              umma_f8(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
           } else {
 #pragma unroll
             for (int k = 0; k < GEMM_BK / 16; ++k)   // +32 bytes per K=16 step

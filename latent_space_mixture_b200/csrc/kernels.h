@@ -46,6 +46,10 @@ constexpr int QUANT_W_MSE = 2;
 cudaError_t launch_quant_weights(const void* w, int E, int rows_per, int K, int Kp, float* amax,
                                  uint8_t* codes, uint8_t* atoms, float* gscale, int variant,
                                  cudaStream_t st);
+// FP8 (E4M3) expert weights [E][rows_per][K] bf16 -> codes [E*rows_per][K]
+// bytes and per-expert scales [E] (amax / 448); amax is [E] scratch.
+cudaError_t launch_quant_w8(const void* w, int E, int rows_per, int K, float* amax, uint8_t* codes,
+                            float* scale, cudaStream_t st);
 // fp32 rows -> codes [rows][cols/2], scales [rows][cols/16] (canonical layout).
 cudaError_t launch_quant_rows(const float* x, int64_t rows, int cols, float g, uint8_t* codes,
                               uint8_t* scales, cudaStream_t st);

@@ -35,6 +35,8 @@ struct EpiX {
   uint8_t* uq;    // NVFP4 experts: u codes [T][l/2] (nullptr for BF16 experts)
   uint8_t* usf;   //   and its E4M3 block scales [T][l/16]
   float g_u;      //   static global scale of u
+  uint8_t* u8;    // FP8 experts: u codes [T][l] (nullptr otherwise)
+  float r_u8;     //   1 / s_u (rounded once)
   __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
                                          bool valid) const {
     if (uq) {
@@ -48,6 +50,12 @@ struct EpiX {
       }
     }
     if (!valid) return;
+    if (u8 && feat >= N && feat < N + lu) {
+      uint8_t q[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = e4m3_code(__fmul_rn(v[i], r_u8));
+      *reinterpret_cast<uint2*>(u8 + row * lu + (feat - N)) = *reinterpret_cast<const uint2*>(q);
+    }
     if (feat < N) {
       float4* p = reinterpret_cast<float4*>(logits + row * N + feat);
       p[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -164,34 +172,60 @@ struct EpiOq {
   }
 };
 
-// GEMM variants: (BN, operand format) -> pipeline stages
-template <int BN, bool FP4>
-struct Stages;
-template <>
-struct Stages<256, false> {
-  static constexpr int value = 4;
+// FP8 expert FC1: H = E4M3(sqrelu(s_W1[e] s_u * acc) / s_h), codes [R][h]
+struct EpiH8 {
+  uint8_t* H8;
+  const float* sw1;
+  float s_u, r_h;
+  int h;
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(sw1[t.e], s_u);
+    uint8_t q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = e4m3_code(__fmul_rn(sqrelu(v[i] * s), r_h));
+    *reinterpret_cast<uint2*>(H8 + row * h + feat) = *reinterpret_cast<const uint2*>(q);
+  }
+};
+
+// FP8 expert FC2: O = w * s_W2[e] s_h * acc
+struct EpiO8 {
+  bf16* O;
+  const float* wrow;
+  const float* sw2;
+  float s_h;
+  int l;
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(__fmul_rn(sw2[t.e], s_h), wrow[row]);
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = v[i] * s;
+    store8_bf16(O + row * l + feat, a);
+  }
+};
+
+// GEMM variants: (BN, operand kind) -> pipeline stages (FP8 stages hold
+// 128-byte rows like bf16 ones)
+template <int BN, int KIND>
+struct Stages {
+  static constexpr int value = BN == 256 ? 4 : BN == 128 ? 6 : 10;
 };
 template <>
-struct Stages<128, false> {
-  static constexpr int value = 6;
-};
-template <>
-struct Stages<32, false> {
-  static constexpr int value = 10;
-};
-template <>
-struct Stages<128, true> {
+struct Stages<128, KIND_NVFP4> {
   static constexpr int value = 5;
 };
 template <>
-struct Stages<32, true> {
+struct Stages<32, KIND_NVFP4> {
   static constexpr int value = 8;
 };
 
-template <int BN, class Epi, bool FP4 = false>
+template <int BN, class Epi, int KIND = KIND_BF16>
 cudaError_t set_gemm_smem() {
-  using L = GemmLayout<BN, Stages<BN, FP4>::value, FP4>;
-  return cudaFuncSetAttribute(k_gemm_tc<BN, Stages<BN, FP4>::value, Epi, FP4>,
+  using L = GemmLayout<BN, Stages<BN, KIND>::value, KIND>;
+  return cudaFuncSetAttribute(k_gemm_tc<BN, Stages<BN, KIND>::value, Epi, KIND>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
 }
 
@@ -200,12 +234,12 @@ struct BMaps {
   CUtensorMap b16, b64;
 };
 
-template <int BN, class Epi, bool FP4 = false>
+template <int BN, class Epi, int KIND = KIND_BF16>
 cudaError_t launch_gemm(const CUtensorMap& A, const BMaps& B, const TileSource& src,
                         const Epi& epi, int grid, int* err, unsigned long long limit,
                         cudaStream_t st) {
-  using L = GemmLayout<BN, Stages<BN, FP4>::value, FP4>;
-  return launch_pdl(k_gemm_tc<BN, Stages<BN, FP4>::value, Epi, FP4>, grid, GEMM_THREADS,
+  using L = GemmLayout<BN, Stages<BN, KIND>::value, KIND>;
+  return launch_pdl(k_gemm_tc<BN, Stages<BN, KIND>::value, Epi, KIND>, grid, GEMM_THREADS,
                     L::SMEM_BYTES, st, A, B.b16, B.b64, src, epi, err, limit);
 }
 
@@ -230,12 +264,12 @@ cudaError_t launch_gemm_pair(const CUtensorMap& A, const BMaps& B, const TileSou
                          A, B.b16, B.b64, src, epi, err, limit);
 }
 
-template <class Epi>
-cudaError_t launch_gemm_fp4(int bn, const CUtensorMap& A, const BMaps& B, const TileSource& src,
-                            const Epi& epi, int grid, int* err, unsigned long long limit,
-                            cudaStream_t st) {
-  if (bn == 128) return launch_gemm<128, Epi, true>(A, B, src, epi, grid, err, limit, st);
-  return launch_gemm<32, Epi, true>(A, B, src, epi, grid, err, limit, st);
+template <int KIND, class Epi>
+cudaError_t launch_gemm_q(int bn, const CUtensorMap& A, const BMaps& B, const TileSource& src,
+                          const Epi& epi, int grid, int* err, unsigned long long limit,
+                          cudaStream_t st) {
+  if (bn == 128) return launch_gemm<128, Epi, KIND>(A, B, src, epi, grid, err, limit, st);
+  return launch_gemm<32, Epi, KIND>(A, B, src, epi, grid, err, limit, st);
 }
 
 template <class Epi>
@@ -428,6 +462,18 @@ struct lmoe_handle {
   int32_t* rblock = nullptr;   // [T*K] (token block << 8) | row in block
   CUtensorMap tm_w1q, tm_w2q;
   BMaps tm_upq, tm_Hq;
+  // FP8 (E4M3) W8A8 experts: codes and per-tensor scales
+  bool fp8 = false;
+  float r_u8 = 0.f, r_h8 = 0.f;  // 1 / s_u, 1 / s_h (rounded once); s in g_u, g_h
+  uint8_t* w1f8 = nullptr;     // [N*h][l]
+  uint8_t* w2f8 = nullptr;     // [N*l][h]
+  float* sw1 = nullptr;        // [N] amax / 448
+  float* sw2 = nullptr;        // [N]
+  uint8_t* uf8 = nullptr;      // [T][l]
+  uint8_t* upf8 = nullptr;     // [T*K][l] expert order
+  uint8_t* Hf8 = nullptr;      // [T*K][h]
+  CUtensorMap tm_w1f8, tm_w2f8;
+  BMaps tm_upf8, tm_Hf8;
   std::vector<void*> allocs;
   CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
   BMaps tm_uperm, tm_H, tm_vh;
@@ -481,9 +527,10 @@ static int check_cfg(const lmoe_config* c) {
       (c->latent != c->d || c->expert_format != LMOE_FMT_BF16))
     return LMOE_ERR_UNSUPPORTED;
   if (c->top_k > c->n_experts) return LMOE_ERR_INVALID_ARG;
-  if (c->expert_format != LMOE_FMT_BF16 && c->expert_format != LMOE_FMT_NVFP4)
+  if (c->expert_format != LMOE_FMT_BF16 && c->expert_format != LMOE_FMT_NVFP4 &&
+      c->expert_format != LMOE_FMT_FP8)
     return LMOE_ERR_INVALID_ARG;
-  if (c->expert_format == LMOE_FMT_NVFP4 && (c->latent % 128 || c->expert_hidden % 128))
+  if (c->expert_format != LMOE_FMT_BF16 && (c->latent % 128 || c->expert_hidden % 128))
     return LMOE_ERR_UNSUPPORTED;
   if (c->d % 64 || c->latent % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
     return LMOE_ERR_UNSUPPORTED;
@@ -500,7 +547,7 @@ static int check_cfg(const lmoe_config* c) {
 static int grouped_bn(const lmoe_config& c, int64_t T) {
   const double avg = double(T) * c.top_k / c.n_experts;
   if (avg <= 40.0) return 32;
-  if (avg <= 160.0 || c.expert_format == LMOE_FMT_NVFP4) return 128;
+  if (avg <= 160.0 || c.expert_format != LMOE_FMT_BF16) return 128;
   return 256;
 }
 
@@ -528,7 +575,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   if (!w || !w->w_router || !w->w1 || !w->w2 || !w->w_s1 || !w->w_s2 ||
       (proj && (!w->w_dn || !w->w_upl)))
     return LMOE_ERR_INVALID_ARG;
-  if (cfg->expert_format == LMOE_FMT_NVFP4 &&
+  if (cfg->expert_format != LMOE_FMT_BF16 &&
       !(w->act_gscale_latent > 0.0f && w->act_gscale_hidden > 0.0f &&
         w->act_gscale_latent < 3.0e38f && w->act_gscale_hidden < 3.0e38f))
     return LMOE_ERR_INVALID_ARG;
@@ -555,13 +602,16 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   const int64_t Tm_b = Tm < 256 ? 256 : Tm;
   const int64_t d_a = d < GEMM_BM ? GEMM_BM : d;
   const bool fp4 = c.expert_format == LMOE_FMT_NVFP4;
+  const bool fp8 = c.expert_format == LMOE_FMT_FP8;
+  const bool bfx = !fp4 && !fp8;   // BF16 experts
   h->fp4 = fp4;
+  h->fp8 = fp8;
   h->lp = static_cast<int>((l + 255) / 256 * 256);
   h->hp = static_cast<int>((hh + 255) / 256 * 256);
   const int64_t lp = h->lp, hp = h->hp;
   const int64_t nb_max = rows / 32 + N + 1;   // token blocks of >= 32 rows, one partial per expert
   // bytes of the bf16 expert path buffers that NVFP4 replaces
-  const int64_t bf16_only = fp4 ? 0 : 1;
+  const int64_t bf16_only = bfx ? 1 : 0;
   // largest split-K partials buffer over the token counts this handle
   // accepts, for the same feature and K extents the forward pass plans with
   // (x-GEMM: N + lx + h_s features over K = d; y-GEMM: d features over
@@ -616,7 +666,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->w2q, size_t(fp4 * N * l * hp / 2)},
       {(void**)&h->w2sf, size_t(fp4 * (N * l / 128) * (hp / 64) * 512)},
       {(void**)&h->gw2, size_t(fp4 * N * 4)},
-      {(void**)&h->amax, size_t(fp4 * N * 4)},
+      {(void**)&h->amax, size_t((fp4 || fp8) * N * 4)},
       {(void**)&h->uq, size_t(fp4 * Tm * l / 2)},
       {(void**)&h->usf, size_t(fp4 * Tm * l / 16)},
       {(void**)&h->upq, size_t(fp4 * rows_b * lp / 2)},
@@ -624,6 +674,13 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->Hq, size_t(fp4 * rows_b * hp / 2)},
       {(void**)&h->sfbh, size_t(fp4 * nb_max * (hp / 64) * 512)},
       {(void**)&h->rblock, size_t(fp4 * rows * 4)},
+      {(void**)&h->w1f8, size_t(fp8 * N * hh * l)},
+      {(void**)&h->w2f8, size_t(fp8 * N * l * hh)},
+      {(void**)&h->sw1, size_t(fp8 * N * 4)},
+      {(void**)&h->sw2, size_t(fp8 * N * 4)},
+      {(void**)&h->uf8, size_t(fp8 * Tm * l)},
+      {(void**)&h->upf8, size_t(fp8 * rows_b * l)},
+      {(void**)&h->Hf8, size_t(fp8 * rows_b * hh)},
   };
   for (auto& r : reqs) {
     if ((rc = alloc_dev(h, r.p, r.bytes)) != LMOE_OK) {
@@ -639,9 +696,31 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= cudaMemcpy(h->w_x + N * d, w->w_dn, l * d * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
   ok &= cudaMemcpy(h->w_x + (N + lx) * d, w->w_s1, hs * d * 2, cudaMemcpyDeviceToDevice) ==
         cudaSuccess;
-  if (!fp4) {
+  if (bfx) {
     ok &= cudaMemcpy(h->w1, w->w1, N * hh * l * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
     ok &= cudaMemcpy(h->w2, w->w2, N * l * hh * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  } else if (fp8) {
+    // per-tensor scales: s = amax / 448 per expert matrix; activations static
+    h->g_u = w->act_gscale_latent;
+    h->g_h = w->act_gscale_hidden;
+    h->r_u8 = 1.0f / h->g_u;
+    h->r_h8 = 1.0f / h->g_h;
+    ok &= cudaMemset(h->upf8, 0, rows_b * l) == cudaSuccess;
+    ok &= cudaMemset(h->Hf8, 0, rows_b * hh) == cudaSuccess;
+    ok &= launch_quant_w8(w->w1, static_cast<int>(N), static_cast<int>(hh), static_cast<int>(l),
+                          h->amax, h->w1f8, h->sw1, 0) == cudaSuccess;
+    ok &= launch_quant_w8(w->w2, static_cast<int>(N), static_cast<int>(l), static_cast<int>(hh),
+                          h->amax, h->w2f8, h->sw2, 0) == cudaSuccess;
+    ok &= make_map_u8(&h->tm_w1f8, h->w1f8, N * hh, l, GEMM_BM);
+    ok &= make_map_u8(&h->tm_w2f8, h->w2f8, N * l, hh, GEMM_BM);
+    ok &= make_map_u8(&h->tm_upf8.b16, h->upf8, rows_b, l, GEMM_BROWS);
+    ok &= make_map_u8(&h->tm_upf8.b64, h->upf8, rows_b, l, GEMM_BROWS_BIG);
+    ok &= make_map_u8(&h->tm_Hf8.b16, h->Hf8, rows_b, hh, GEMM_BROWS);
+    ok &= make_map_u8(&h->tm_Hf8.b64, h->Hf8, rows_b, hh, GEMM_BROWS_BIG);
+    ok &= set_gemm_smem<128, EpiH8, KIND_FP8>() == cudaSuccess;
+    ok &= set_gemm_smem<32, EpiH8, KIND_FP8>() == cudaSuccess;
+    ok &= set_gemm_smem<128, EpiO8, KIND_FP8>() == cudaSuccess;
+    ok &= set_gemm_smem<32, EpiO8, KIND_FP8>() == cudaSuccess;
   } else {
     // padding (K beyond l or h, unused atoms) must read as zero
     h->g_u = w->act_gscale_latent;
@@ -668,10 +747,10 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= make_map_u8(&h->tm_upq.b64, h->upq, rows_b, lp / 2, GEMM_BROWS_BIG);
     ok &= make_map_u8(&h->tm_Hq.b16, h->Hq, rows_b, hp / 2, GEMM_BROWS);
     ok &= make_map_u8(&h->tm_Hq.b64, h->Hq, rows_b, hp / 2, GEMM_BROWS_BIG);
-    ok &= set_gemm_smem<128, EpiHq, true>() == cudaSuccess;
-    ok &= set_gemm_smem<32, EpiHq, true>() == cudaSuccess;
-    ok &= set_gemm_smem<128, EpiOq, true>() == cudaSuccess;
-    ok &= set_gemm_smem<32, EpiOq, true>() == cudaSuccess;
+    ok &= set_gemm_smem<128, EpiHq, KIND_NVFP4>() == cudaSuccess;
+    ok &= set_gemm_smem<32, EpiHq, KIND_NVFP4>() == cudaSuccess;
+    ok &= set_gemm_smem<128, EpiOq, KIND_NVFP4>() == cudaSuccess;
+    ok &= set_gemm_smem<32, EpiOq, KIND_NVFP4>() == cudaSuccess;
   }
   if (proj)
     ok &= cudaMemcpy2D(h->w_y, (lx + hs) * 2, w->w_upl, l * 2, l * 2, d,
@@ -684,7 +763,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= cudaMemset(h->bias, 0, N * 4) == cudaSuccess;
   ok &= cudaMemset(h->err, 0, 4) == cudaSuccess;
   ok &= cudaMemset(h->vh, 0, Tm_b * (l + hs) * 2) == cudaSuccess;
-  if (!fp4) {
+  if (bfx) {
     ok &= cudaMemset(h->u_perm, 0, rows_b * l * 2) == cudaSuccess;
     ok &= cudaMemset(h->H, 0, rows_b * hh * 2) == cudaSuccess;
   }
@@ -693,12 +772,12 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= cudaMemset(h->w_y + d * (lx + hs), 0, (d_a - d) * (lx + hs) * 2) == cudaSuccess;
   // tensor maps of the fixed operands
   ok &= make_map(&h->tm_wx, h->w_x, N + lx + hs, d, GEMM_BM);
-  if (!fp4) {
+  if (bfx) {
     ok &= make_map(&h->tm_w1, h->w1, N * hh, l, GEMM_BM);
     ok &= make_map(&h->tm_w2, h->w2, N * l, hh, GEMM_BM);
   }
   ok &= make_map(&h->tm_wy, h->w_y, d_a, lx + hs, GEMM_BM);
-  if (!fp4) {
+  if (bfx) {
     ok &= make_map(&h->tm_uperm.b16, h->u_perm, rows_b, l, GEMM_BROWS);
     ok &= make_map(&h->tm_uperm.b64, h->u_perm, rows_b, l, GEMM_BROWS_BIG);
     ok &= make_map(&h->tm_H.b16, h->H, rows_b, hh, GEMM_BROWS);
@@ -807,7 +886,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   {
     const int fb = (N + lx + hs + 127) / 128;
     const DensePlan p = plan_dense(T, fb, static_cast<int>(d / 64), h->sms);
-    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u};
+    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->uf8, h->r_u8};
     const int fb2 = (N + lx + hs + PAIR_BM - 1) / PAIR_BM;
     const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
     if (h->pairs && ptiles >= h->sms / 2) {
@@ -834,7 +913,25 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   LMOE_STEP(4, launch_scatter(h->topk_idx, h->topk_w, h->chunk, h->counts, T, N, K, gbn,
                               h->offsets, h->perm, h->inv, h->wrow, h->blocks, h->nblocks,
                               h->rblock, h->err, st));
-  if (h->fp4) {
+  if (h->fp8) {
+    // 6. FP8 latent rows into expert order (rows of l bytes: l/2 bf16 units)
+    LMOE_STEP(5, launch_gather(h->uf8, h->perm, T * K, K, l / 2, h->upf8, st));
+    // 7. H = E4M3(sqrelu(s_W1 s_u W1q[e] uq) / s_h), kind::f8f6f4
+    {
+      TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, l / 128, 1, nullptr,
+                   gbn == 32};
+      EpiH8 epi{h->Hf8, h->sw1, h->g_u, h->r_h8, hh};
+      LMOE_STEP(6, launch_gemm_q<KIND_FP8>(gbn, h->tm_w1f8, h->tm_upf8, s, epi, h->sms, h->err,
+                                           lim, st));
+    }
+    // 8. O = w s_W2 s_h W2q[e] Hq
+    {
+      TileSource s{0, 0, h->blocks, h->nblocks, l / 128, l, l, hh / 128, 1, nullptr, gbn == 32};
+      EpiO8 epi{h->O, h->wrow, h->sw2, h->g_h, l};
+      LMOE_STEP(7, launch_gemm_q<KIND_FP8>(gbn, h->tm_w2f8, h->tm_Hf8, s, epi, h->sms, h->err,
+                                           lim, st));
+    }
+  } else if (h->fp4) {
     // 6. quantised latent rows (and their scales) into expert order
     LMOE_STEP(5, launch_gather_q(h->uq, h->usf, h->perm, h->rblock, T * K, K, l, h->lp, h->upq,
                                  h->sfbu, st));
@@ -843,14 +940,14 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
       TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, h->lp / 256, 1, nullptr,
                    gbn == 32, h->w1sf, h->sfbu, h->lp / 64};
       EpiHq epi{h->Hq, h->sfbh, h->gw1, h->g_u, h->g_h, h->hp};
-      LMOE_STEP(6, launch_gemm_fp4(gbn, h->tm_w1q, h->tm_upq, s, epi, h->sms, h->err, lim, st));
+      LMOE_STEP(6, launch_gemm_q<KIND_NVFP4>(gbn, h->tm_w1q, h->tm_upq, s, epi, h->sms, h->err, lim, st));
     }
     // 8. O = w * W2[e] H, block-scaled FP4 MMA
     {
       TileSource s{0, 0, h->blocks, h->nblocks, l / 128, l, l, h->hp / 256, 1, nullptr,
                    gbn == 32, h->w2sf, h->sfbh, h->hp / 64};
       EpiOq epi{h->O, h->wrow, h->gw2, h->g_h, l};
-      LMOE_STEP(7, launch_gemm_fp4(gbn, h->tm_w2q, h->tm_Hq, s, epi, h->sms, h->err, lim, st));
+      LMOE_STEP(7, launch_gemm_q<KIND_NVFP4>(gbn, h->tm_w2q, h->tm_Hq, s, epi, h->sms, h->err, lim, st));
     }
   } else {
   // 6. latent rows into expert order
@@ -966,15 +1063,22 @@ int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
       src = h->u; want = T * l * 2; break;
     case LMOE_DBG_V: strided = true; col0 = 0; cols = l; want = T * l * 2; break;
     case LMOE_DBG_HS: strided = true; col0 = l; cols = hs; want = T * hs * 2; break;
-    case LMOE_DBG_W1Q_CODES: src = h->w1q; want = N * c.expert_hidden * h->lp / 2; break;
+    // quantised expert weights: NVFP4 codes, scale atoms and global scales,
+    // or FP8 codes and per-tensor scales (no atoms)
+    case LMOE_DBG_W1Q_CODES:
+      if (h->fp8) { src = h->w1f8; want = N * c.expert_hidden * l; break; }
+      src = h->w1q; want = N * c.expert_hidden * h->lp / 2; break;
     case LMOE_DBG_W1Q_SF: src = h->w1sf; want = (N * c.expert_hidden / 128) * (h->lp / 64) * 512; break;
-    case LMOE_DBG_W1Q_G: src = h->gw1; want = N * 4; break;
-    case LMOE_DBG_W2Q_CODES: src = h->w2q; want = N * l * h->hp / 2; break;
+    case LMOE_DBG_W1Q_G: src = h->fp8 ? h->sw1 : h->gw1; want = N * 4; break;
+    case LMOE_DBG_W2Q_CODES:
+      if (h->fp8) { src = h->w2f8; want = N * l * c.expert_hidden; break; }
+      src = h->w2q; want = N * l * h->hp / 2; break;
     case LMOE_DBG_W2Q_SF: src = h->w2sf; want = (N * l / 128) * (h->hp / 64) * 512; break;
-    case LMOE_DBG_W2Q_G: src = h->gw2; want = N * 4; break;
+    case LMOE_DBG_W2Q_G: src = h->fp8 ? h->sw2 : h->gw2; want = N * 4; break;
     default: return LMOE_ERR_INVALID_ARG;
   }
-  if (what >= LMOE_DBG_W1Q_CODES && !h->fp4) return LMOE_ERR_INVALID_ARG;
+  if (what >= LMOE_DBG_W1Q_CODES && !h->fp4 && !h->fp8) return LMOE_ERR_INVALID_ARG;
+  if ((what == LMOE_DBG_W1Q_SF || what == LMOE_DBG_W2Q_SF) && !h->fp4) return LMOE_ERR_INVALID_ARG;
   if (bytes != want) return LMOE_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return LMOE_ERR_CUDA;
   if (want == 0) return LMOE_OK;

@@ -170,6 +170,46 @@ cudaError_t launch_quant_weights(const void* w, int E, int rows_per, int K, int 
   return cudaGetLastError();
 }
 
+// FP8 (E4M3) W8A8 expert weights ("Nemotron-3 Super 精读报告", section 9.1):
+// one float32 scale per expert matrix, s = amax / 448, r = 1 / s (rounded
+// once), code = E4M3(x * r) round-to-nearest-even, saturating.  Thread per 8
+// consecutive elements of a [E * rows_per][K] bf16 matrix.
+__global__ void __launch_bounds__(256) k_quant_w8(const __nv_bfloat16* __restrict__ w,
+                                                  int64_t n8, int64_t per_expert,
+                                                  const float* __restrict__ amax,
+                                                  uint8_t* __restrict__ codes,
+                                                  float* __restrict__ scale) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const int e = static_cast<int>(i * 8 / per_expert);
+  const float s = __fdiv_rn(amax[e], 448.0f);
+  if (i * 8 == static_cast<int64_t>(e) * per_expert) scale[e] = s;
+  const float r = s > 0.0f ? __fdiv_rn(1.0f, s) : 0.0f;
+  const uint4 raw = reinterpret_cast<const uint4*>(w)[i];
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  uint8_t q[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(p[j]);
+    q[2 * j] = e4m3_code(__fmul_rn(f.x, r));
+    q[2 * j + 1] = e4m3_code(__fmul_rn(f.y, r));
+  }
+  reinterpret_cast<uint2*>(codes)[i] = *reinterpret_cast<const uint2*>(q);
+}
+
+cudaError_t launch_quant_w8(const void* w, int E, int rows_per, int K, float* amax, uint8_t* codes,
+                            float* scale, cudaStream_t st) {
+  if (cudaMemsetAsync(amax, 0, E * sizeof(float), st) != cudaSuccess) return cudaGetLastError();
+  const int64_t per = static_cast<int64_t>(rows_per) * K;
+  k_amax_expert<<<dim3(64, E), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), per, amax);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t n8 = static_cast<int64_t>(E) * per / 8;
+  k_quant_w8<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w), n8, per, amax, codes, scale);
+  return cudaGetLastError();
+}
+
 // Row quantiser with canonical outputs: codes [rows][cols/2], scales [rows][cols/16].
 __global__ void __launch_bounds__(256) k_quant_rows(const float* __restrict__ x, int64_t rows,
                                                     int cols, float g, uint8_t* __restrict__ codes,

@@ -190,6 +190,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 with E4M3 A and B (K = 32
+// per instruction: 32 bytes of each operand row), fp32 accumulate.
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= (A * sfA)[smem] * (B * sfB)[smem]^T, kind::mxf4nvf4: packed E2M1
 // A and B, one E4M3 scale per 16 elements along K taken from TMEM, K = 64.
 __device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -352,6 +364,13 @@ __host__ __device__ __forceinline__ uint32_t idesc_nvf4(int M, int N) {
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, both K-major.
 //   bits 4-5 D format (1 = f32); 7-9 A format (1 = bf16); 10-12 B format;
 //   15/16 A/B major (0 = K); 17-22 N >> 3; 24-28 M >> 4.
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0 in
+// bits 7-9 and 10-12), fp32 D (bits 4-5 = 1), K-major operands, N >> 3 in
+// bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ __forceinline__ uint32_t idesc_f8(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 __host__ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);

@@ -10,7 +10,7 @@ from typing import Dict, Optional
 import torch
 
 from . import _lib
-from ._lib import (DBG, FLAG_NO_PROJECTION, FMT_BF16, FMT_NVFP4, NVFP4_WEIGHT_FLAGS,
+from ._lib import (DBG, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8, FMT_NVFP4, NVFP4_WEIGHT_FLAGS,
                    LmoeConfig, LmoeError, LmoeWeights, check)
 
 __all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]
@@ -58,7 +58,7 @@ class LatentMoE:
                                  or not bias.is_cuda):
             raise ValueError("router_bias: need CUDA fp32 [N]")
         self.cfg = LmoeConfig(d, latent, n_experts, top_k, expert_hidden, shared_hidden,
-                              {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4}[expert_format],
+                              {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4, "fp8": FMT_FP8}[expert_format],
                               (0 if projections else FLAG_NO_PROJECTION)
                               | NVFP4_WEIGHT_FLAGS[nvfp4_weights], max_tokens)
         w = LmoeWeights(weights["w_router"].data_ptr(),
@@ -124,7 +124,11 @@ class LatentMoE:
         lp = (c.latent + 255) // 256 * 256
         hp = (c.expert_hidden + 255) // 256 * 256
         N, h, l = c.n_experts, c.expert_hidden, c.latent
-        spec.update({
+        if c.expert_format == FMT_FP8:
+            # E4M3 codes, one byte per element, and per-expert scales
+            spec.update({"w1q_codes": (torch.uint8, (N * h, l)), "w1q_g": (torch.float32, (N,)),
+                         "w2q_codes": (torch.uint8, (N * l, h)), "w2q_g": (torch.float32, (N,))})
+        spec.update({} if c.expert_format == FMT_FP8 else {
             "w1q_codes": (torch.uint8, (N * h, lp // 2)),
             "w1q_sf": (torch.uint8, ((N * h // 128) * (lp // 64) * 512,)),
             "w1q_g": (torch.float32, (N,)),

@@ -48,7 +48,7 @@ class LayerConfig:
     std: float        # weight init std
     bias: str         # "zero" or "zipf"
     seed: int
-    fmt: str = "bf16"  # expert format: "bf16" or "nvfp4"
+    fmt: str = "bf16"  # expert format: "bf16", "nvfp4" or "fp8"
     proj: bool = True  # latent projections W_dn, W_upl (False: standard MoE, l = d)
     wq: str = "1d"     # NVFP4 weight blocks/scales: "1d", "2d", "mse" or "2d_mse"
 
@@ -95,6 +95,12 @@ CONFIGS: Dict[str, LayerConfig] = {
                                           2688, 5376, 0.02, "zipf", 4, "nvfp4", wq="2d"),
     "super_prefill_nvfp4_mse": LayerConfig("super_prefill_nvfp4_mse", 8192, 4096, 1024, 512, 22,
                                            2688, 5376, 0.02, "zipf", 4, "nvfp4", wq="mse"),
+    # FP8 (E4M3) W8A8 experts: tiny, and Super prefill with Zipf bias
+    "tiny_fp8": LayerConfig("tiny_fp8", 64, 256, 128, 32, 4, 256, 256, 0.02, "zipf", 13, "fp8"),
+    "super_prefill_fp8": LayerConfig("super_prefill_fp8", 8192, 4096, 1024, 512, 22, 2688, 5376,
+                                     0.02, "zipf", 4, "fp8"),
+    "super_decode_fp8": LayerConfig("super_decode_fp8", 256, 4096, 1024, 512, 22, 2688, 5376,
+                                    0.02, "zero", 1, "fp8"),
     # the standard-MoE comparator: tiny, decode- and prefill-sized
     "tiny_std": LayerConfig("tiny_std", 64, 256, 256, 32, 4, 128, 256, 0.02, "zipf", 10,
                             proj=False),
@@ -156,11 +162,14 @@ def make_x(cfg: LayerConfig, gen: torch.Generator, T: Optional[int] = None,
 
 
 def act_global_scales(cfg: LayerConfig):
-    """Static NVFP4 global scales (g_u, g_h) of the latent activation u and the
-    expert hidden activation, set from the synthetic distribution: with
-    sigma_u = std*sqrt(d) and sigma_a = std*sqrt(l)*sigma_u, the amax bounds
-    8*sigma_u and (8*sigma_a)^2 map to E2M1 max (6) times E4M3 max (448).
-    Values beyond the bound saturate."""
+    """Static scales (u, hidden) of the latent activation u and the expert
+    hidden activation for quantised experts, set from the synthetic
+    distribution: with sigma_u = std*sqrt(d) and sigma_a = std*sqrt(l)*sigma_u,
+    the amax bounds 8*sigma_u and (8*sigma_a)^2 map to E2M1 max (6) times
+    E4M3 max (448) for NVFP4 (global scales over E4M3 block scales), or to
+    E4M3 max (448) for FP8 (per-tensor scales).  Values beyond the bound
+    saturate."""
     sigma_u = cfg.std * math.sqrt(cfg.d)
     sigma_a = cfg.std * math.sqrt(cfg.l) * sigma_u
-    return (8.0 * sigma_u) / (6.0 * 448.0), (8.0 * sigma_a) ** 2 / (6.0 * 448.0)
+    top = 448.0 if cfg.fmt == "fp8" else 6.0 * 448.0
+    return (8.0 * sigma_u) / top, (8.0 * sigma_a) ** 2 / top

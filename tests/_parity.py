@@ -52,7 +52,7 @@ def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None):
     from lmoe_synth import act_global_scales
     layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs,
                       max_tokens or x.shape[0], w, expert_format=cfg.fmt,
-                      act_gscales=act_global_scales(cfg) if cfg.fmt == "nvfp4" else (0.0, 0.0),
+                      act_gscales=act_global_scales(cfg) if cfg.fmt != "bf16" else (0.0, 0.0),
                       projections=cfg.proj, nvfp4_weights=cfg.wq)
     return w, x, layer
 
@@ -60,9 +60,11 @@ def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None):
 def quant_of(cfg):
     """The oracle's quantisation settings for a workload (None for BF16)."""
     from lmoe_synth import act_global_scales
-    if cfg.fmt != "nvfp4":
+    if cfg.fmt == "bf16":
         return None
     g_u, g_h = act_global_scales(cfg)
+    if cfg.fmt == "fp8":
+        return {"fmt": "fp8", "s_u": float(np.float32(g_u)), "s_h": float(np.float32(g_h))}
     return {"g_u": float(np.float32(g_u)), "g_h": float(np.float32(g_h)),
             "w2d": cfg.wq in ("2d", "2d_mse"), "wmse": cfg.wq in ("mse", "2d_mse")}
 

@@ -58,6 +58,8 @@ def _cfg(**kw):
     (dict(flags=1), -2), (dict(flags=1, latent=256, expert_format=1), -2),
     # NVFP4 weight variants need NVFP4 experts; unknown bits are rejected
     (dict(flags=2), -1), (dict(flags=4), -1), (dict(flags=8), -1),
+    # FP8 experts: latent and expert hidden multiples of 128
+    (dict(expert_format=2), -2), (dict(expert_format=2, flags=2), -1),
     (dict(d=100), -2), (dict(latent=96), -2), (dict(n_experts=48), -2),
     (dict(n_experts=2048, top_k=4), -2), (dict(expert_format=1), -2), (dict(expert_format=7), -1),
 ])
