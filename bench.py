@@ -72,8 +72,9 @@ def algorithmic_work(cfg, T: int, counts: np.ndarray):
     """
     d, l, N, K, h, hs = cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs
     lx = l if cfg.proj else 0
-    eb = {"bf16": 2.0, "nvfp4": 0.5625, "fp8": 1.0}[cfg.fmt]
-    mult = {"bf16": 1, "nvfp4": 4, "fp8": 2}[cfg.fmt]
+    eb = {"bf16": 2.0, "nvfp4": 0.5625, "fp8": 1.0, "w4a16": 0.5625}[cfg.fmt]   # weights
+    ea = {"bf16": 2.0, "nvfp4": 0.5625, "fp8": 1.0, "w4a16": 2.0}[cfg.fmt]     # u, H rows
+    mult = {"bf16": 1, "nvfp4": 4, "fp8": 2, "w4a16": 1}[cfg.fmt]
     touched = int((counts > 0).sum())
     R = T * K
     wx = (N + lx + hs) * d * 2
@@ -82,9 +83,9 @@ def algorithmic_work(cfg, T: int, counts: np.ndarray):
     per_kernel = {
         "xgemm(router|W_dn|W_s1)": dict(bytes=wx + T * d * 2 + T * (N * 4 + lx * 2 + hs * 2),
                                         flops=2 * T * d * (N + lx + hs)),
-        "grouped_gemm1(W1,sqrelu)": dict(bytes=int(wexp + R * l * eb + R * h * eb),
+        "grouped_gemm1(W1,sqrelu)": dict(bytes=int(wexp + R * l * ea + R * h * ea),
                                          flops=2 * R * l * h, mult=mult),
-        "grouped_gemm2(W2,*w)": dict(bytes=int(wexp + R * h * eb + R * l * 2 + R * 4),
+        "grouped_gemm2(W2,*w)": dict(bytes=int(wexp + R * h * ea + R * l * 2 + R * 4),
                                      flops=2 * R * h * l, mult=mult),
         "ygemm([W_upl|W_s2])": dict(bytes=wy + T * (l + hs) * 2 + T * d * 2,
                                     flops=2 * T * d * (lx + hs)),
@@ -410,7 +411,7 @@ def main():
         rms = lambda t: float(torch.sqrt(torch.mean(t.double() ** 2)))
         quant_err = {"v_rms_rel_vs_bf16_experts": round(rms(v_q - v_b) / rms(v_b), 5),
                      "format": cfg.fmt}
-        if cfg.fmt == "nvfp4":
+        if cfg.fmt in ("nvfp4", "w4a16"):
             quant_err["nvfp4_weights"] = cfg.wq
 
     launches = layer.launches_per_forward(T) * args.steps
@@ -420,7 +421,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": {"bf16": "bf16", "nvfp4": "e2m1 experts, bf16 dense",
-                      "fp8": "e4m3 experts, bf16 dense"}[cfg.fmt],
+                      "fp8": "e4m3 experts, bf16 dense",
+                      "w4a16": "e2m1 weights expanded to f16, f16 activations, bf16 dense"}[cfg.fmt],
             "data": "synthetic (seeded; weights N(0, std) bf16, x N(0,1) bf16)",
             "config": {"workload": cfg.name, "T": T, "d": cfg.d, "latent": cfg.l,
                        "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,

@@ -72,6 +72,14 @@ extern "C" {
                             global scale; latent projections, router and
                             shared expert stay BF16 ("Nemotron-3 Super 精读报告",
                             table 5.2).  Needs l and h multiples of 128.      */
+#define LMOE_FMT_W4A16 3 /* experts with NVFP4 weights (as LMOE_FMT_NVFP4,
+                            LMOE_FLAG_NVFP4_WEIGHT_* apply) and 16-bit
+                            activations ("Nemotron 3 Ultra 解读", W4A16):
+                            u and H stay unquantised, in FP16; the GEMMs
+                            expand each weight tile to f16 in shared memory
+                            (code value x block scale, exact) and apply the
+                            global scale in the epilogue.  Needs l and h
+                            multiples of 128; act_gscale_* unused.          */
 #define LMOE_FMT_FP8 2   /* experts in FP8 W8A8 ("Nemotron-3 Super 精读报告",
                             section 9.1): W1, W2, u and H as E4M3 codes with
                             one FP32 scale per tensor (s_W = amax / 448 per

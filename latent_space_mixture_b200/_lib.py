@@ -12,7 +12,7 @@ LIB_PATH = os.path.join(HERE, "liblmoe.so")
 LMOE_OK = 0
 ERRORS = {-1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "OOM", -4: "CUDA", -5: "TIMEOUT",
           -6: "DEVICE"}
-FMT_BF16, FMT_NVFP4, FMT_FP8 = 0, 1, 2
+FMT_BF16, FMT_NVFP4, FMT_FP8, FMT_W4A16 = 0, 1, 2, 3
 FLAG_NO_PROJECTION = 1   # standard MoE: no latent projections (u = x, r = v)
 FLAG_NVFP4_WEIGHT_2D = 2   # NVFP4 weights: one scale per 16 x 16 block
 FLAG_NVFP4_WEIGHT_MSE = 4  # NVFP4 weights: MSE-searched block scales

@@ -31,6 +31,7 @@
 // which starved the ring and stretched every small-N MMA.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "nvfp4.cuh"
 #include "ptx.cuh"
@@ -51,6 +52,10 @@ constexpr int FP8_K_PER_STAGE = 128;  // FP8 (E4M3) K elements per stage (128 B 
 constexpr int KIND_BF16 = 0;   // kind::f16, bf16 A and B, K = 16 per MMA
 constexpr int KIND_NVFP4 = 1;  // kind::mxf4nvf4 block16 with E4M3 block scales, K = 64
 constexpr int KIND_FP8 = 2;    // kind::f8f6f4, E4M3 A and B, K = 32
+constexpr int KIND_W4A16 = 3;  // NVFP4 weights expanded to f16 in shared memory by
+                               // converter warps, f16 B, kind::f16, K = 16
+constexpr int W4_CONV_THREADS = 256;          // converter threads: two per weight row
+constexpr int W4_CODE_BYTES = GEMM_BM * 32;   // one k-step of FP4 weight codes
 constexpr int FP4_SF_STAGE_BYTES = 4 * SF_ATOM_BYTES;   // 4 chunks of K=64
 
 // Where the tiles of one GEMM come from.
@@ -107,13 +112,20 @@ __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int t
 template <int BN, int STAGES, int KIND>
 struct GemmLayout {
   static constexpr bool FP4 = KIND == KIND_NVFP4;
+  static constexpr bool W4 = KIND == KIND_W4A16;
   static constexpr int A_BYTES = GEMM_BM * GEMM_ROW_BYTES;
   static constexpr int B_BYTES = BN * GEMM_ROW_BYTES;
   static constexpr int SF_BYTES = FP4 ? 2 * FP4_SF_STAGE_BYTES : 0;
+  // W4A16: the k-step's FP4 codes (128 rows x 32 B) and its A scale atom
+  static constexpr int RAW_BYTES = W4 ? W4_CODE_BYTES + SF_ATOM_BYTES : 0;
+  static constexpr int THREADS = GEMM_THREADS + (W4 ? W4_CONV_THREADS : 0);   // + converters
   static constexpr int STG_BYTES = GEMM_EPI_WARPS * 32 * GEMM_STG_LD * 4;
-  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES + SF_BYTES) +
+  static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ +
+                                    STAGES * (A_BYTES + B_BYTES + SF_BYTES + RAW_BYTES) +
                                     STG_BYTES + BAR_BYTES + 16;
+  // bytes a stage's TMA and bulk copies bring, besides the B rows
+  static constexpr int TX_A = W4 ? RAW_BYTES : A_BYTES + SF_BYTES;
   // TMEM: two accumulators of BN columns, then (NVFP4) 32 scale columns per stage
   static constexpr int SF_COL0 = 2 * BN;
   static constexpr int COLS_USED = 2 * BN + (FP4 ? 32 * STAGES : 0);
@@ -138,26 +150,30 @@ template <class L>
 __device__ __forceinline__ bool empty_commits_at(int s) { return !L::PAIRED_RELEASE || (s & 1); }
 
 template <int BN, int STAGES, class Epi, int KIND>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(GemmLayout<BN, STAGES, KIND>::THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmB64, const TileSource src, const Epi epi, int* err,
           unsigned long long limit_ns) {
   using L = GemmLayout<BN, STAGES, KIND>;
   constexpr bool FP4 = KIND == KIND_NVFP4;
   constexpr bool F8 = KIND == KIND_FP8;
+  constexpr bool W4 = KIND == KIND_W4A16;
+  constexpr bool BYTE_MAPS = FP4 || F8;   // operand maps in bytes (128 per stage row)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * L::A_BYTES;
   uint8_t* sSF = sB + STAGES * L::B_BYTES;           // NVFP4: [stage][A 2 KB | B 2 KB]
-  float* stg = reinterpret_cast<float*>(sSF + STAGES * L::SF_BYTES);
+  uint8_t* sR = sSF + STAGES * L::SF_BYTES;          // W4A16: [stage][codes | atom]
+  float* stg = reinterpret_cast<float*>(sR + STAGES * L::RAW_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stg) + L::STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;   // [2]
   uint64_t* tempty = tfull + 2;       // [2]
   uint64_t* drain = tempty + 2;       // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* aready = drain + 1;       // [STAGES] W4A16: the stage's f16 A tile is written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aready + STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -173,6 +189,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       mbar_init(&tempty[a], GEMM_EPI_WARPS * 32);
     }
     mbar_init(drain, 1);
+    if constexpr (W4)
+      for (int s = 0; s < STAGES; ++s) mbar_init(&aready[s], W4_CONV_THREADS);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -205,7 +223,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     auto load_b = [&](int st, const TileInfo& t, int kb) {
       const int nbig = t.nrows / GEMM_BROWS_BIG;
       const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
-      const int bx = KIND != KIND_BF16 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+      const int bx = BYTE_MAPS ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
       uint8_t* b_dst = sB + st * L::B_BYTES;
       for (int j = 0; j < nbig; ++j)
         tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
@@ -230,8 +248,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       // B rows: 64-row boxes while 64 rows remain, then 16-row boxes
       const int nbig = t.nrows / GEMM_BROWS_BIG;
       const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
-      const uint32_t tx = L::A_BYTES + L::SF_BYTES +
-                          (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_ROW_BYTES;
+      const uint32_t tx = L::TX_A + (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_ROW_BYTES;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (empty_waits_at<L>(stage) &&
             !__all_sync(0xffffffffu, mbar_wait_bounded(&empty[empty_slot<L>(stage)], phase ^ 1,
@@ -239,11 +256,20 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           ok = false;
           break;
         }
-        // x coordinate in elements of the map: bf16 elements or bytes (NVFP4, FP8)
-        const int ax = KIND != KIND_BF16 ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
+        // x coordinate in elements of the map: bf16 elements or bytes (NVFP4,
+        // FP8); W4A16: bytes of FP4 codes, 32 per k-step
+        const int ax = W4 ? kb * 32 : BYTE_MAPS ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
         if (elect_one()) {
           mbar_arrive_expect_tx(&full[stage], tx);
-          tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, ax, t.a_row, &full[stage], pol_a);
+          if constexpr (W4) {
+            uint8_t* raw = sR + stage * L::RAW_BYTES;
+            tma_load_2d_hint(raw, &tmA, ax, t.a_row, &full[stage], pol_a);
+            bulk_load(raw + W4_CODE_BYTES,
+                      src.sfa + (static_cast<long>(t.a_row / GEMM_BM) * src.kc + kb) * SF_ATOM_BYTES,
+                      SF_ATOM_BYTES, &full[stage]);
+          } else {
+            tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, ax, t.a_row, &full[stage], pol_a);
+          }
           if constexpr (FP4)
             bulk_load(sSF + stage * L::SF_BYTES,
                       src.sfa + (static_cast<long>(t.a_row / GEMM_BM) * src.kc + kb * 4) *
@@ -309,10 +335,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       const uint32_t d_tmem = tmem_base + acc * BN;
       const uint32_t idesc = FP4  ? idesc_nvf4(GEMM_BM, n_mma)
                              : F8 ? idesc_f8(GEMM_BM, n_mma)
+                             : W4 ? idesc_f16(GEMM_BM, n_mma)
                                   : idesc_bf16(GEMM_BM, n_mma);
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (!__all_sync(0xffffffffu,
                         mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns))) {
+          ok = false;
+          break;
+        }
+        // W4A16: and the converter warps have written the stage's f16 A tile
+        if (W4 && !__all_sync(0xffffffffu, mbar_wait_bounded(&aready[stage], phase, abort_flag,
+                                                              err, limit_ns))) {
           ok = false;
           break;
         }
@@ -370,7 +403,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < 2 + GEMM_EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter of this warp
     float* my = stg + (warp - 2) * 32 * GEMM_STG_LD;
@@ -425,6 +458,63 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     }
   }
 
+  if constexpr (W4) {
+    if (warp >= 2 + GEMM_EPI_WARPS) {
+      // ---------------------------------------------------------- converters
+      // Two threads per row of the 128-row weight tile, 32 of its 64 E2M1
+      // codes each, times the E4M3 scales of their 16-blocks, as f16 (the
+      // product of an E2M1 and an E4M3 value is exact in f16), written in
+      // the 128-byte-swizzled K-major layout the MMA reads; the per-expert
+      // global scale is applied in the epilogue.
+      const int ct = threadIdx.x - (2 + GEMM_EPI_WARPS) * 32;
+      const int r = ct >> 1, half = ct & 1;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const TileInfo t = gemm_tile(src, BN, tile);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns))) {
+            ok = false;
+            break;
+          }
+          const uint8_t* raw = sR + stage * L::RAW_BYTES;
+          const uint4 c = *reinterpret_cast<const uint4*>(raw + r * 32 + half * 16);
+          const uint32_t sc4 =
+              *reinterpret_cast<const uint32_t*>(raw + W4_CODE_BYTES + sf_atom_offset(r, 0));
+          const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+          uint8_t* dst = sA + stage * L::A_BYTES + r * GEMM_ROW_BYTES;
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const int blk = 2 * half + b;   // 16-element block of the row
+            const uint32_t sb = (sc4 >> (8 * blk)) & 0xFFu;
+            const uint32_t s2 = f16x2_from_e4m3x2(sb | (sb << 8));
+            uint32_t lo[4], hi[4];
+            f16x2_from_e2m1x8(cw[2 * b], lo);
+            f16x2_from_e2m1x8(cw[2 * b + 1], hi);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              lo[i] = hmul2_f16(lo[i], s2);
+              hi[i] = hmul2_f16(hi[i], s2);
+            }
+            // elements 16 blk .. +15 are 16-byte chunks 2 blk and 2 blk + 1 of the row
+            *reinterpret_cast<uint4*>(dst + (((2 * blk) ^ (r & 7)) * 16)) =
+                make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *reinterpret_cast<uint4*>(dst + (((2 * blk + 1) ^ (r & 7)) * 16)) =
+                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&aready[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -466,6 +556,16 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* dst, const float* v) 
   __nv_bfloat162 p[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(p);
+}
+
+// 8 floats -> 8 f16 (16-byte store), finite: saturating at +-65504
+__device__ __forceinline__ void store8_f16(__half* dst, const float* v) {
+  __half2 p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    p[i] = __floats2half2_rn(fminf(fmaxf(v[2 * i], -65504.0f), 65504.0f),
+                             fminf(fmaxf(v[2 * i + 1], -65504.0f), 65504.0f));
   *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(p);
 }
 

@@ -37,6 +37,7 @@ struct EpiX {
   float g_u;      //   static global scale of u
   uint8_t* u8;    // FP8 experts: u codes [T][l] (nullptr otherwise)
   float r_u8;     //   1 / s_u (rounded once)
+  __half* u16;    // W4A16 experts: u in f16 [T][l] (nullptr otherwise)
   __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
                                          bool valid) const {
     if (uq) {
@@ -56,6 +57,7 @@ struct EpiX {
       for (int i = 0; i < 8; ++i) q[i] = e4m3_code(__fmul_rn(v[i], r_u8));
       *reinterpret_cast<uint2*>(u8 + row * lu + (feat - N)) = *reinterpret_cast<const uint2*>(q);
     }
+    if (u16 && feat >= N && feat < N + lu) store8_f16(u16 + row * lu + (feat - N), v);
     if (feat < N) {
       float4* p = reinterpret_cast<float4*>(logits + row * N + feat);
       p[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -207,6 +209,40 @@ struct EpiO8 {
   }
 };
 
+// W4A16 expert FC1: H = sqrelu(g_W1[e] * acc) in f16 (the MMA summed the
+// FP4 codes times their block scales; the global scale comes here)
+struct EpiH16 {
+  __half* H16;
+  const float* gw1;
+  int h;
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    const float g = gw1[t.e];
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = sqrelu(v[i] * g);
+    store8_f16(H16 + row * h + feat, a);
+  }
+};
+
+// W4A16 expert FC2: O = w * g_W2[e] * acc
+struct EpiO16 {
+  bf16* O;
+  const float* wrow;
+  const float* gw2;
+  int l;
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(gw2[t.e], wrow[row]);
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = v[i] * s;
+    store8_bf16(O + row * l + feat, a);
+  }
+};
+
 // GEMM variants: (BN, operand kind) -> pipeline stages (FP8 stages hold
 // 128-byte rows like bf16 ones)
 template <int BN, int KIND>
@@ -219,6 +255,15 @@ struct Stages<128, KIND_NVFP4> {
 };
 template <>
 struct Stages<32, KIND_NVFP4> {
+  static constexpr int value = 8;
+};
+// W4A16 stages also hold the raw FP4 codes and scale atom (4.5 KB)
+template <>
+struct Stages<128, KIND_W4A16> {
+  static constexpr int value = 5;
+};
+template <>
+struct Stages<32, KIND_W4A16> {
   static constexpr int value = 8;
 };
 
@@ -239,7 +284,7 @@ cudaError_t launch_gemm(const CUtensorMap& A, const BMaps& B, const TileSource& 
                         const Epi& epi, int grid, int* err, unsigned long long limit,
                         cudaStream_t st) {
   using L = GemmLayout<BN, Stages<BN, KIND>::value, KIND>;
-  return launch_pdl(k_gemm_tc<BN, Stages<BN, KIND>::value, Epi, KIND>, grid, GEMM_THREADS,
+  return launch_pdl(k_gemm_tc<BN, Stages<BN, KIND>::value, Epi, KIND>, grid, L::THREADS,
                     L::SMEM_BYTES, st, A, B.b16, B.b64, src, epi, err, limit);
 }
 
@@ -348,6 +393,20 @@ static bool make_map_strided(CUtensorMap* m, const void* base, uint64_t rows, ui
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D byte matrix [rows][cols] of packed FP4 codes read as 32-byte x 128-row
+// tiles without swizzle (the W4A16 converter reads them row by row)
+static bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {32, GEMM_BM};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -474,6 +533,11 @@ struct lmoe_handle {
   uint8_t* Hf8 = nullptr;      // [T*K][h]
   CUtensorMap tm_w1f8, tm_w2f8;
   BMaps tm_upf8, tm_Hf8;
+  // W4A16 experts: the NVFP4 weights above, read as raw code tiles (32 B x
+  // 128 rows, no swizzle) and expanded to f16 in the GEMM; u and H in f16
+  bool w4 = false;
+  __half* u16 = nullptr;       // [T][l]
+  CUtensorMap tm_w1c, tm_w2c;
   std::vector<void*> allocs;
   CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
   BMaps tm_uperm, tm_H, tm_vh;
@@ -521,14 +585,14 @@ static int check_cfg(const lmoe_config* c) {
                     LMOE_FLAG_NVFP4_WEIGHT_MSE)) != 0)
     return LMOE_ERR_INVALID_ARG;
   if ((c->flags & (LMOE_FLAG_NVFP4_WEIGHT_2D | LMOE_FLAG_NVFP4_WEIGHT_MSE)) &&
-      c->expert_format != LMOE_FMT_NVFP4)
+      c->expert_format != LMOE_FMT_NVFP4 && c->expert_format != LMOE_FMT_W4A16)
     return LMOE_ERR_INVALID_ARG;
   if ((c->flags & LMOE_FLAG_NO_PROJECTION) &&
       (c->latent != c->d || c->expert_format != LMOE_FMT_BF16))
     return LMOE_ERR_UNSUPPORTED;
   if (c->top_k > c->n_experts) return LMOE_ERR_INVALID_ARG;
   if (c->expert_format != LMOE_FMT_BF16 && c->expert_format != LMOE_FMT_NVFP4 &&
-      c->expert_format != LMOE_FMT_FP8)
+      c->expert_format != LMOE_FMT_FP8 && c->expert_format != LMOE_FMT_W4A16)
     return LMOE_ERR_INVALID_ARG;
   if (c->expert_format != LMOE_FMT_BF16 && (c->latent % 128 || c->expert_hidden % 128))
     return LMOE_ERR_UNSUPPORTED;
@@ -575,7 +639,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   if (!w || !w->w_router || !w->w1 || !w->w2 || !w->w_s1 || !w->w_s2 ||
       (proj && (!w->w_dn || !w->w_upl)))
     return LMOE_ERR_INVALID_ARG;
-  if (cfg->expert_format != LMOE_FMT_BF16 &&
+  if ((cfg->expert_format == LMOE_FMT_NVFP4 || cfg->expert_format == LMOE_FMT_FP8) &&
       !(w->act_gscale_latent > 0.0f && w->act_gscale_hidden > 0.0f &&
         w->act_gscale_latent < 3.0e38f && w->act_gscale_hidden < 3.0e38f))
     return LMOE_ERR_INVALID_ARG;
@@ -601,17 +665,21 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   const int64_t rows_b = rows < 256 ? 256 : rows;
   const int64_t Tm_b = Tm < 256 ? 256 : Tm;
   const int64_t d_a = d < GEMM_BM ? GEMM_BM : d;
-  const bool fp4 = c.expert_format == LMOE_FMT_NVFP4;
+  const bool w4 = c.expert_format == LMOE_FMT_W4A16;
+  const bool fp4 = c.expert_format == LMOE_FMT_NVFP4;   // NVFP4 activations too
   const bool fp8 = c.expert_format == LMOE_FMT_FP8;
-  const bool bfx = !fp4 && !fp8;   // BF16 experts
+  const bool bfx = !fp4 && !fp8 && !w4;   // BF16 experts
+  const bool qw4 = fp4 || w4;             // NVFP4-quantised expert weights
   h->fp4 = fp4;
   h->fp8 = fp8;
+  h->w4 = w4;
   h->lp = static_cast<int>((l + 255) / 256 * 256);
   h->hp = static_cast<int>((hh + 255) / 256 * 256);
   const int64_t lp = h->lp, hp = h->hp;
   const int64_t nb_max = rows / 32 + N + 1;   // token blocks of >= 32 rows, one partial per expert
   // bytes of the bf16 expert path buffers that NVFP4 replaces
   const int64_t bf16_only = bfx ? 1 : 0;
+  const int64_t act16 = (bfx || w4) ? 1 : 0;   // 16-bit expert activations (u_perm, H)
   // largest split-K partials buffer over the token counts this handle
   // accepts, for the same feature and K extents the forward pass plans with
   // (x-GEMM: N + lx + h_s features over K = d; y-GEMM: d features over
@@ -652,21 +720,22 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->blocks, size_t(max_blocks * 16)},
       {(void**)&h->nblocks, size_t(4)},
       {(void**)&h->u, size_t(Tm * lx * 2)},
-      {(void**)&h->u_perm, size_t(bf16_only * rows_b * l * 2)},
-      {(void**)&h->H, size_t(bf16_only * rows_b * hh * 2)},
+      {(void**)&h->u_perm, size_t(act16 * rows_b * l * 2)},
+      {(void**)&h->H, size_t(act16 * rows_b * hh * 2)},
       {(void**)&h->O, size_t(rows * l * 2)},
       {(void**)&h->vh, size_t(Tm_b * (l + hs) * 2)},
       {(void**)&h->x_dev, size_t(Tm_b * d * 2)},
       {(void**)&h->y_dev, size_t(Tm * d * 2)},
       {(void**)&h->part, size_t(part_floats * 4)},
       {(void**)&h->err, size_t(4)},
-      {(void**)&h->w1q, size_t(fp4 * N * hh * lp / 2)},
-      {(void**)&h->w1sf, size_t(fp4 * (N * hh / 128) * (lp / 64) * 512)},
-      {(void**)&h->gw1, size_t(fp4 * N * 4)},
-      {(void**)&h->w2q, size_t(fp4 * N * l * hp / 2)},
-      {(void**)&h->w2sf, size_t(fp4 * (N * l / 128) * (hp / 64) * 512)},
-      {(void**)&h->gw2, size_t(fp4 * N * 4)},
-      {(void**)&h->amax, size_t((fp4 || fp8) * N * 4)},
+      {(void**)&h->w1q, size_t(qw4 * N * hh * lp / 2)},
+      {(void**)&h->w1sf, size_t(qw4 * (N * hh / 128) * (lp / 64) * 512)},
+      {(void**)&h->gw1, size_t(qw4 * N * 4)},
+      {(void**)&h->w2q, size_t(qw4 * N * l * hp / 2)},
+      {(void**)&h->w2sf, size_t(qw4 * (N * l / 128) * (hp / 64) * 512)},
+      {(void**)&h->gw2, size_t(qw4 * N * 4)},
+      {(void**)&h->amax, size_t((qw4 || fp8) * N * 4)},
+      {(void**)&h->u16, size_t(w4 * Tm * l * 2)},
       {(void**)&h->uq, size_t(fp4 * Tm * l / 2)},
       {(void**)&h->usf, size_t(fp4 * Tm * l / 16)},
       {(void**)&h->upq, size_t(fp4 * rows_b * lp / 2)},
@@ -729,10 +798,12 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= cudaMemset(h->w1sf, 0, (N * hh / 128) * (lp / 64) * 512) == cudaSuccess;
     ok &= cudaMemset(h->w2q, 0, N * l * hp / 2) == cudaSuccess;
     ok &= cudaMemset(h->w2sf, 0, (N * l / 128) * (hp / 64) * 512) == cudaSuccess;
-    ok &= cudaMemset(h->upq, 0, rows_b * lp / 2) == cudaSuccess;
-    ok &= cudaMemset(h->sfbu, 0, nb_max * (lp / 64) * 512) == cudaSuccess;
-    ok &= cudaMemset(h->Hq, 0, rows_b * hp / 2) == cudaSuccess;
-    ok &= cudaMemset(h->sfbh, 0, nb_max * (hp / 64) * 512) == cudaSuccess;
+    if (fp4) {
+      ok &= cudaMemset(h->upq, 0, rows_b * lp / 2) == cudaSuccess;
+      ok &= cudaMemset(h->sfbu, 0, nb_max * (lp / 64) * 512) == cudaSuccess;
+      ok &= cudaMemset(h->Hq, 0, rows_b * hp / 2) == cudaSuccess;
+      ok &= cudaMemset(h->sfbh, 0, nb_max * (hp / 64) * 512) == cudaSuccess;
+    }
     const int wvar = ((c.flags & LMOE_FLAG_NVFP4_WEIGHT_2D) ? QUANT_W_2D : 0) |
                      ((c.flags & LMOE_FLAG_NVFP4_WEIGHT_MSE) ? QUANT_W_MSE : 0);
     ok &= launch_quant_weights(w->w1, static_cast<int>(N), static_cast<int>(hh), static_cast<int>(l),
@@ -741,16 +812,26 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= launch_quant_weights(w->w2, static_cast<int>(N), static_cast<int>(l), static_cast<int>(hh),
                                static_cast<int>(hp), h->amax, h->w2q, h->w2sf, h->gw2, wvar,
                                0) == cudaSuccess;
-    ok &= make_map_u8(&h->tm_w1q, h->w1q, N * hh, lp / 2, GEMM_BM);
-    ok &= make_map_u8(&h->tm_w2q, h->w2q, N * l, hp / 2, GEMM_BM);
-    ok &= make_map_u8(&h->tm_upq.b16, h->upq, rows_b, lp / 2, GEMM_BROWS);
-    ok &= make_map_u8(&h->tm_upq.b64, h->upq, rows_b, lp / 2, GEMM_BROWS_BIG);
-    ok &= make_map_u8(&h->tm_Hq.b16, h->Hq, rows_b, hp / 2, GEMM_BROWS);
-    ok &= make_map_u8(&h->tm_Hq.b64, h->Hq, rows_b, hp / 2, GEMM_BROWS_BIG);
-    ok &= set_gemm_smem<128, EpiHq, KIND_NVFP4>() == cudaSuccess;
-    ok &= set_gemm_smem<32, EpiHq, KIND_NVFP4>() == cudaSuccess;
-    ok &= set_gemm_smem<128, EpiOq, KIND_NVFP4>() == cudaSuccess;
-    ok &= set_gemm_smem<32, EpiOq, KIND_NVFP4>() == cudaSuccess;
+    if (fp4) {
+      ok &= make_map_u8(&h->tm_w1q, h->w1q, N * hh, lp / 2, GEMM_BM);
+      ok &= make_map_u8(&h->tm_w2q, h->w2q, N * l, hp / 2, GEMM_BM);
+      ok &= make_map_u8(&h->tm_upq.b16, h->upq, rows_b, lp / 2, GEMM_BROWS);
+      ok &= make_map_u8(&h->tm_upq.b64, h->upq, rows_b, lp / 2, GEMM_BROWS_BIG);
+      ok &= make_map_u8(&h->tm_Hq.b16, h->Hq, rows_b, hp / 2, GEMM_BROWS);
+      ok &= make_map_u8(&h->tm_Hq.b64, h->Hq, rows_b, hp / 2, GEMM_BROWS_BIG);
+      ok &= set_gemm_smem<128, EpiHq, KIND_NVFP4>() == cudaSuccess;
+      ok &= set_gemm_smem<32, EpiHq, KIND_NVFP4>() == cudaSuccess;
+      ok &= set_gemm_smem<128, EpiOq, KIND_NVFP4>() == cudaSuccess;
+      ok &= set_gemm_smem<32, EpiOq, KIND_NVFP4>() == cudaSuccess;
+    } else {
+      // W4A16: code tiles of one k-step (64 elements = 32 bytes) x 128 rows
+      ok &= make_map_codes(&h->tm_w1c, h->w1q, N * hh, lp / 2);
+      ok &= make_map_codes(&h->tm_w2c, h->w2q, N * l, hp / 2);
+      ok &= set_gemm_smem<128, EpiH16, KIND_W4A16>() == cudaSuccess;
+      ok &= set_gemm_smem<32, EpiH16, KIND_W4A16>() == cudaSuccess;
+      ok &= set_gemm_smem<128, EpiO16, KIND_W4A16>() == cudaSuccess;
+      ok &= set_gemm_smem<32, EpiO16, KIND_W4A16>() == cudaSuccess;
+    }
   }
   if (proj)
     ok &= cudaMemcpy2D(h->w_y, (lx + hs) * 2, w->w_upl, l * 2, l * 2, d,
@@ -763,7 +844,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= cudaMemset(h->bias, 0, N * 4) == cudaSuccess;
   ok &= cudaMemset(h->err, 0, 4) == cudaSuccess;
   ok &= cudaMemset(h->vh, 0, Tm_b * (l + hs) * 2) == cudaSuccess;
-  if (bfx) {
+  if (bfx || w4) {
     ok &= cudaMemset(h->u_perm, 0, rows_b * l * 2) == cudaSuccess;
     ok &= cudaMemset(h->H, 0, rows_b * hh * 2) == cudaSuccess;
   }
@@ -777,7 +858,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= make_map(&h->tm_w2, h->w2, N * l, hh, GEMM_BM);
   }
   ok &= make_map(&h->tm_wy, h->w_y, d_a, lx + hs, GEMM_BM);
-  if (bfx) {
+  if (bfx || w4) {   // 2-byte rows (bf16, or f16 for W4A16)
     ok &= make_map(&h->tm_uperm.b16, h->u_perm, rows_b, l, GEMM_BROWS);
     ok &= make_map(&h->tm_uperm.b64, h->u_perm, rows_b, l, GEMM_BROWS_BIG);
     ok &= make_map(&h->tm_H.b16, h->H, rows_b, hh, GEMM_BROWS);
@@ -886,7 +967,8 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   {
     const int fb = (N + lx + hs + 127) / 128;
     const DensePlan p = plan_dense(T, fb, static_cast<int>(d / 64), h->sms);
-    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->uf8, h->r_u8};
+    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->uf8, h->r_u8,
+             h->u16};
     const int fb2 = (N + lx + hs + PAIR_BM - 1) / PAIR_BM;
     const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
     if (h->pairs && ptiles >= h->sms / 2) {
@@ -913,7 +995,26 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   LMOE_STEP(4, launch_scatter(h->topk_idx, h->topk_w, h->chunk, h->counts, T, N, K, gbn,
                               h->offsets, h->perm, h->inv, h->wrow, h->blocks, h->nblocks,
                               h->rblock, h->err, st));
-  if (h->fp8) {
+  if (h->w4) {
+    // 6. f16 latent rows into expert order
+    LMOE_STEP(5, launch_gather(h->u16, h->perm, T * K, K, l, h->u_perm, st));
+    // 7. H = sqrelu(g_W1 * (W1 codes x block scales) u), weights expanded in the GEMM
+    {
+      TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, l / 64, 1, nullptr,
+                   gbn == 32, h->w1sf, nullptr, h->lp / 64};
+      EpiH16 epi{reinterpret_cast<__half*>(h->H), h->gw1, hh};
+      LMOE_STEP(6, launch_gemm_q<KIND_W4A16>(gbn, h->tm_w1c, h->tm_uperm, s, epi, h->sms,
+                                             h->err, lim, st));
+    }
+    // 8. O = w g_W2 (W2 codes x block scales) H
+    {
+      TileSource s{0, 0, h->blocks, h->nblocks, l / 128, l, l, hh / 64, 1, nullptr, gbn == 32,
+                   h->w2sf, nullptr, h->hp / 64};
+      EpiO16 epi{h->O, h->wrow, h->gw2, l};
+      LMOE_STEP(7, launch_gemm_q<KIND_W4A16>(gbn, h->tm_w2c, h->tm_H, s, epi, h->sms, h->err,
+                                             lim, st));
+    }
+  } else if (h->fp8) {
     // 6. FP8 latent rows into expert order (rows of l bytes: l/2 bf16 units)
     LMOE_STEP(5, launch_gather(h->uf8, h->perm, T * K, K, l / 2, h->upf8, st));
     // 7. H = E4M3(sqrelu(s_W1 s_u W1q[e] uq) / s_h), kind::f8f6f4
@@ -1077,8 +1178,9 @@ int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
     case LMOE_DBG_W2Q_G: src = h->fp8 ? h->sw2 : h->gw2; want = N * 4; break;
     default: return LMOE_ERR_INVALID_ARG;
   }
-  if (what >= LMOE_DBG_W1Q_CODES && !h->fp4 && !h->fp8) return LMOE_ERR_INVALID_ARG;
-  if ((what == LMOE_DBG_W1Q_SF || what == LMOE_DBG_W2Q_SF) && !h->fp4) return LMOE_ERR_INVALID_ARG;
+  if (what >= LMOE_DBG_W1Q_CODES && !h->fp4 && !h->fp8 && !h->w4) return LMOE_ERR_INVALID_ARG;
+  if ((what == LMOE_DBG_W1Q_SF || what == LMOE_DBG_W2Q_SF) && !h->fp4 && !h->w4)
+    return LMOE_ERR_INVALID_ARG;
   if (bytes != want) return LMOE_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return LMOE_ERR_CUDA;
   if (want == 0) return LMOE_OK;

@@ -364,6 +364,53 @@ __host__ __device__ __forceinline__ uint32_t idesc_nvf4(int M, int N) {
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, both K-major.
 //   bits 4-5 D format (1 = f32); 7-9 A format (1 = bf16); 10-12 B format;
 //   15/16 A/B major (0 = K); 17-22 N >> 3; 24-28 M >> 4.
+// Instruction descriptor of kind::f16 with f16 A and B (format code 0), fp32 D.
+__host__ __device__ __forceinline__ uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Two E2M1 codes (one byte, the lower element in bits 0-3) -> f16x2 (lower
+// element in the lower half).
+__device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(r) : "r"(byte));
+  return r;
+}
+
+// Eight E2M1 codes (four bytes, the lowest element in the low nibble of the
+// low byte) -> four f16x2 in element order.
+__device__ __forceinline__ void f16x2_from_e2m1x8(uint32_t w, uint32_t (&o)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+
+// Two E4M3 codes (bits 0-7 and 8-15) -> f16x2.
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t two) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+      : "=r"(r) : "r"(two));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2_f16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// order this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (TMA stores, tcgen05.mma operands)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0 in
 // bits 7-9 and 10-12), fp32 D (bits 4-5 = 1), K-major operands, N >> 3 in
 // bits 17-22, M >> 4 in bits 24-28.

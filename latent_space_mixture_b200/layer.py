@@ -10,7 +10,8 @@ from typing import Dict, Optional
 import torch
 
 from . import _lib
-from ._lib import (DBG, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8, FMT_NVFP4, NVFP4_WEIGHT_FLAGS,
+from ._lib import (DBG, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8, FMT_NVFP4, FMT_W4A16,
+                   NVFP4_WEIGHT_FLAGS,
                    LmoeConfig, LmoeError, LmoeWeights, check)
 
 __all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]
@@ -58,7 +59,8 @@ class LatentMoE:
                                  or not bias.is_cuda):
             raise ValueError("router_bias: need CUDA fp32 [N]")
         self.cfg = LmoeConfig(d, latent, n_experts, top_k, expert_hidden, shared_hidden,
-                              {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4, "fp8": FMT_FP8}[expert_format],
+                              {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4, "fp8": FMT_FP8,
+                               "w4a16": FMT_W4A16}[expert_format],
                               (0 if projections else FLAG_NO_PROJECTION)
                               | NVFP4_WEIGHT_FLAGS[nvfp4_weights], max_tokens)
         w = LmoeWeights(weights["w_router"].data_ptr(),

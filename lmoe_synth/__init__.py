@@ -48,7 +48,7 @@ class LayerConfig:
     std: float        # weight init std
     bias: str         # "zero" or "zipf"
     seed: int
-    fmt: str = "bf16"  # expert format: "bf16", "nvfp4" or "fp8"
+    fmt: str = "bf16"  # expert format: "bf16", "nvfp4", "fp8" or "w4a16"
     proj: bool = True  # latent projections W_dn, W_upl (False: standard MoE, l = d)
     wq: str = "1d"     # NVFP4 weight blocks/scales: "1d", "2d", "mse" or "2d_mse"
 
@@ -101,6 +101,14 @@ CONFIGS: Dict[str, LayerConfig] = {
                                      0.02, "zipf", 4, "fp8"),
     "super_decode_fp8": LayerConfig("super_decode_fp8", 256, 4096, 1024, 512, 22, 2688, 5376,
                                     0.02, "zero", 1, "fp8"),
+    # W4A16 experts (NVFP4 weights, 16-bit activations): tiny, Super decode
+    # and prefill ("Nemotron 3 Ultra 解读": one NVFP4 checkpoint serves W4A16)
+    "tiny_w4a16": LayerConfig("tiny_w4a16", 64, 256, 128, 32, 4, 256, 256, 0.02, "zipf", 14,
+                              "w4a16"),
+    "super_decode_w4a16": LayerConfig("super_decode_w4a16", 256, 4096, 1024, 512, 22, 2688, 5376,
+                                      0.02, "zero", 1, "w4a16"),
+    "super_prefill_w4a16": LayerConfig("super_prefill_w4a16", 8192, 4096, 1024, 512, 22, 2688,
+                                       5376, 0.02, "zipf", 4, "w4a16"),
     # the standard-MoE comparator: tiny, decode- and prefill-sized
     "tiny_std": LayerConfig("tiny_std", 64, 256, 256, 32, 4, 128, 256, 0.02, "zipf", 10,
                             proj=False),

@@ -147,6 +147,13 @@ def _expert_quantisers(quant: Dict):
     """(q_u, q_w, q_h): quantise-dequantise maps of the expert inputs u, an
     expert weight matrix and the expert hidden activation, for the NVFP4
     ("fmt" absent or "nvfp4") or the FP8 W8A8 ("fmt": "fp8") expert layer."""
+    if quant.get("fmt", "nvfp4") == "w4a16":
+        # NVFP4 weights, unquantised (16-bit) activations
+        from . import nvfp4
+        wq = dict(block2d=quant.get("w2d", False), mse=quant.get("wmse", False))
+        return (lambda a: a,
+                lambda W: nvfp4.fake_quant(W, nvfp4.weight_global_scale(W), **wq),
+                lambda a: a)
     if quant.get("fmt", "nvfp4") == "fp8":
         from . import fp8
         return (lambda a: fp8.fake_quant(a, quant["s_u"]),
@@ -179,7 +186,9 @@ def layer_forward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     NVFP4 quantise-dequantise images (oracle.nvfp4); optional "w2d" and
     "wmse" (bool) select 2D 16x16 weight blocks and MSE-searched weight
     block scales.  quant = {"fmt": "fp8", "s_u": float, "s_h": float} is the
-    FP8 W8A8 expert layer (oracle.fp8: E4M3, per-tensor scales).
+    FP8 W8A8 expert layer (oracle.fp8: E4M3, per-tensor scales);
+    {"fmt": "w4a16"} (with optional "w2d", "wmse") has NVFP4 weights and
+    unquantised activations.
 
     Returns a dict with S, w, gap, s, z, u, v, r, hs, sh, y (float64); hs is
     the shared expert's hidden activation sqrelu(W_s1 x).

@@ -65,6 +65,9 @@ def quant_of(cfg):
     g_u, g_h = act_global_scales(cfg)
     if cfg.fmt == "fp8":
         return {"fmt": "fp8", "s_u": float(np.float32(g_u)), "s_h": float(np.float32(g_h))}
+    if cfg.fmt == "w4a16":
+        return {"fmt": "w4a16", "w2d": cfg.wq in ("2d", "2d_mse"),
+                "wmse": cfg.wq in ("mse", "2d_mse")}
     return {"g_u": float(np.float32(g_u)), "g_h": float(np.float32(g_h)),
             "w2d": cfg.wq in ("2d", "2d_mse"), "wmse": cfg.wq in ("mse", "2d_mse")}
 

@@ -109,3 +109,24 @@ def test_fp8_layer_matches_restatement_and_is_close_to_bf16():
                          lambda e: p["W2"][e], p["W_upl"], p["W_s1"], p["W_s2"], K)
     rel = np.sqrt(np.mean((out["r"] - bf["r"]) ** 2) / np.mean(bf["r"] ** 2))
     assert 0 < rel < 0.08
+
+
+def test_w4a16_layer_quantises_weights_only():
+    """W4A16: NVFP4 weights, activations untouched -- equal to the BF16 layer
+    run on the NVFP4 images of W1 and W2."""
+    from oracle import nvfp4 as Q
+    rng = np.random.default_rng(5)
+    T, d, l, N, K, h, hs = 4, 32, 32, 6, 2, 32, 16
+    p = dict(x=rng.standard_normal((T, d)), W_r=rng.standard_normal((N, d)) * 0.3,
+             b=np.zeros(N), W_dn=rng.standard_normal((l, d)) * 0.2,
+             W1=rng.standard_normal((N, h, l)) * 0.2, W2=rng.standard_normal((N, l, h)) * 0.2,
+             W_upl=rng.standard_normal((d, l)) * 0.2, W_s1=rng.standard_normal((hs, d)) * 0.2,
+             W_s2=rng.standard_normal((d, hs)) * 0.2)
+    out = O.layer_forward(p["x"], p["W_r"], p["b"], p["W_dn"], lambda e: p["W1"][e],
+                          lambda e: p["W2"][e], p["W_upl"], p["W_s1"], p["W_s2"], K,
+                          quant={"fmt": "w4a16"})
+    fq = lambda W: Q.fake_quant(W, Q.weight_global_scale(W))
+    ref = O.layer_forward(p["x"], p["W_r"], p["b"], p["W_dn"], lambda e: fq(p["W1"][e]),
+                          lambda e: fq(p["W2"][e]), p["W_upl"], p["W_s1"], p["W_s2"], K)
+    assert np.array_equal(out["y"], ref["y"])
+    assert np.array_equal(out["u"], ref["u"])
