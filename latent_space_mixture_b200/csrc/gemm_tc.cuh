@@ -55,6 +55,7 @@ constexpr int KIND_FP8 = 2;    // kind::f8f6f4, E4M3 A and B, K = 32
 constexpr int KIND_W4A16 = 3;  // NVFP4 weights expanded to f16 in shared memory by
                                // converter warps, f16 B, kind::f16, K = 16
 constexpr int W4_CONV_THREADS = 256;          // converter threads: two per weight row
+constexpr int W4_KSUB = 2;   // W4A16 stages hold two 64-wide K sub-tiles (one barrier phase)
 constexpr int W4_CODE_BYTES = GEMM_BM * 32;   // one k-step of FP4 weight codes
 constexpr int FP4_SF_STAGE_BYTES = 4 * SF_ATOM_BYTES;   // 4 chunks of K=64
 
@@ -113,11 +114,17 @@ template <int BN, int STAGES, int KIND>
 struct GemmLayout {
   static constexpr bool FP4 = KIND == KIND_NVFP4;
   static constexpr bool W4 = KIND == KIND_W4A16;
-  static constexpr int A_BYTES = GEMM_BM * GEMM_ROW_BYTES;
-  static constexpr int B_BYTES = BN * GEMM_ROW_BYTES;
+  // 64-wide K sub-tiles per stage: W4A16 moves only 4.5 KB of weights per
+  // sub-tile, and a CTA's TMA stream pays a roughly fixed cost per barrier
+  // phase, so its stages take two
+  static constexpr int KS = W4 ? W4_KSUB : 1;
+  static constexpr int A_SUB = GEMM_BM * GEMM_ROW_BYTES;
+  static constexpr int B_SUB = BN * GEMM_ROW_BYTES;
+  static constexpr int A_BYTES = KS * A_SUB;
+  static constexpr int B_BYTES = KS * B_SUB;
   static constexpr int SF_BYTES = FP4 ? 2 * FP4_SF_STAGE_BYTES : 0;
-  // W4A16: the k-step's FP4 codes (128 rows x 32 B) and its A scale atom
-  static constexpr int RAW_BYTES = W4 ? W4_CODE_BYTES + SF_ATOM_BYTES : 0;
+  // W4A16: the stage's FP4 codes (128 rows x 32 B per sub-tile) and A scale atoms
+  static constexpr int RAW_BYTES = W4 ? KS * (W4_CODE_BYTES + SF_ATOM_BYTES) : 0;
   static constexpr int THREADS = GEMM_THREADS + (W4 ? W4_CONV_THREADS : 0);   // + converters
   static constexpr int STG_BYTES = GEMM_EPI_WARPS * 32 * GEMM_STG_LD * 4;
   static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8;
@@ -138,7 +145,7 @@ struct GemmLayout {
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   // with an even ring, one tcgen05.commit releases two consecutive stages
   // (every commit costs the tensor pipe a bubble of about 200 clocks)
-  static constexpr bool PAIRED_RELEASE = STAGES % 2 == 0;
+  static constexpr bool PAIRED_RELEASE = STAGES % 2 == 0 && !W4;
 };
 
 // "empty" barrier of ring slot s, and whether the producer waits on it there
@@ -223,14 +230,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     auto load_b = [&](int st, const TileInfo& t, int kb) {
       const int nbig = t.nrows / GEMM_BROWS_BIG;
       const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
-      const int bx = BYTE_MAPS ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
-      uint8_t* b_dst = sB + st * L::B_BYTES;
-      for (int j = 0; j < nbig; ++j)
-        tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
-                    t.row0 + j * GEMM_BROWS_BIG, &full[st]);
-      for (int j = 0; j < nsmall; ++j) {
-        const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
-        tma_load_2d(b_dst + r * GEMM_ROW_BYTES, &tmB, bx, t.row0 + r, &full[st]);
+      for (int q = 0; q < L::KS; ++q) {
+        const int bx = BYTE_MAPS ? (kb + q) * GEMM_ROW_BYTES : (kb + q) * GEMM_BK;
+        uint8_t* b_dst = sB + st * L::B_BYTES + q * L::B_SUB;
+        for (int j = 0; j < nbig; ++j)
+          tma_load_2d(b_dst + j * GEMM_BROWS_BIG * GEMM_ROW_BYTES, &tmB64, bx,
+                      t.row0 + j * GEMM_BROWS_BIG, &full[st]);
+        for (int j = 0; j < nsmall; ++j) {
+          const int r = nbig * GEMM_BROWS_BIG + j * GEMM_BROWS;
+          tma_load_2d(b_dst + r * GEMM_ROW_BYTES, &tmB, bx, t.row0 + r, &full[st]);
+        }
       }
       if constexpr (FP4)
         bulk_load(sSF + st * L::SF_BYTES + FP4_SF_STAGE_BYTES,
@@ -248,8 +257,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       // B rows: 64-row boxes while 64 rows remain, then 16-row boxes
       const int nbig = t.nrows / GEMM_BROWS_BIG;
       const int nsmall = (t.nrows - nbig * GEMM_BROWS_BIG + GEMM_BROWS - 1) / GEMM_BROWS;
-      const uint32_t tx = L::TX_A + (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_ROW_BYTES;
-      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+      const uint32_t tx =
+          L::TX_A + L::KS * (nbig * GEMM_BROWS_BIG + nsmall * GEMM_BROWS) * GEMM_ROW_BYTES;
+      for (int kb = t.kb0; kb < t.kb1; kb += L::KS) {
         if (empty_waits_at<L>(stage) &&
             !__all_sync(0xffffffffu, mbar_wait_bounded(&empty[empty_slot<L>(stage)], phase ^ 1,
                                                        abort_flag, err, limit_ns))) {
@@ -257,16 +267,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           break;
         }
         // x coordinate in elements of the map: bf16 elements or bytes (NVFP4,
-        // FP8); W4A16: bytes of FP4 codes, 32 per k-step
+        // FP8); W4A16: bytes of FP4 codes, 32 per 64-wide sub-tile
         const int ax = W4 ? kb * 32 : BYTE_MAPS ? kb * GEMM_ROW_BYTES : kb * GEMM_BK;
         if (elect_one()) {
           mbar_arrive_expect_tx(&full[stage], tx);
           if constexpr (W4) {
             uint8_t* raw = sR + stage * L::RAW_BYTES;
             tma_load_2d_hint(raw, &tmA, ax, t.a_row, &full[stage], pol_a);
-            bulk_load(raw + W4_CODE_BYTES,
+            // the sub-tiles' scale atoms are consecutive (64-element chunk fastest)
+            bulk_load(raw + L::KS * W4_CODE_BYTES,
                       src.sfa + (static_cast<long>(t.a_row / GEMM_BM) * src.kc + kb) * SF_ATOM_BYTES,
-                      SF_ATOM_BYTES, &full[stage]);
+                      L::KS * SF_ATOM_BYTES, &full[stage]);
           } else {
             tma_load_2d_hint(sA + stage * L::A_BYTES, &tmA, ax, t.a_row, &full[stage], pol_a);
           }
@@ -278,14 +289,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           if (waited) load_b(stage, t, kb);
         }
         __syncwarp();
-        if (!waited && (++deferred == STAGES || kb + 1 == t.kb1)) {
+        if (!waited && (++deferred == STAGES || kb + L::KS >= t.kb1)) {
           // the first tile's first stages: weights are in flight, now the
           // previous kernel's results
           pdl_wait();
           pdl_trigger();
           waited = true;
           if (elect_one())
-            for (int j = 0; j < deferred; ++j) load_b(j, t, t.kb0 + j);
+            for (int j = 0; j < deferred; ++j) load_b(j, t, t.kb0 + j * L::KS);
           __syncwarp();
         }
         ++issued;
@@ -337,7 +348,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                              : F8 ? idesc_f8(GEMM_BM, n_mma)
                              : W4 ? idesc_f16(GEMM_BM, n_mma)
                                   : idesc_bf16(GEMM_BM, n_mma);
-      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+      for (int kb = t.kb0; kb < t.kb1; kb += L::KS) {
         if (!__all_sync(0xffffffffu,
                         mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns))) {
           ok = false;
@@ -375,8 +386,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
               umma_f8(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
           } else {
 #pragma unroll
-            for (int k = 0; k < GEMM_BK / 16; ++k)   // +32 bytes per K=16 step
-              umma_bf16(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, (kb != t.kb0) || (k != 0));
+            for (int q = 0; q < L::KS; ++q) {
+              // sub-tile q: its own 128-byte-swizzled regions (+A_SUB, +B_SUB bytes)
+              const uint64_t aq = a0 + ((q * L::A_SUB) >> 4), bq = b0 + ((q * L::B_SUB) >> 4);
+#pragma unroll
+              for (int k = 0; k < GEMM_BK / 16; ++k)   // +32 bytes per K=16 step
+                umma_bf16(d_tmem, aq + 2 * k, bq + 2 * k, idesc,
+                          (kb != t.kb0) || (q != 0) || (k != 0));
+            }
           }
           if (empty_commits_at<L>(stage)) umma_commit(&empty[empty_slot<L>(stage)]);
         }
@@ -461,38 +478,40 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   if constexpr (W4) {
     if (warp >= 2 + GEMM_EPI_WARPS) {
       // ---------------------------------------------------------- converters
-      // Two threads per row of the 128-row weight tile, 32 of its 64 E2M1
-      // codes each, times the E4M3 scales of their 16-blocks, as f16 (the
+      // One thread per row of the 128-row weight tile and K sub-tile: its 64
+      // E2M1 codes times the E4M3 scales of their 16-blocks, as f16 (the
       // product of an E2M1 and an E4M3 value is exact in f16), written in
       // the 128-byte-swizzled K-major layout the MMA reads; the per-expert
       // global scale is applied in the epilogue.
       const int ct = threadIdx.x - (2 + GEMM_EPI_WARPS) * 32;
-      const int r = ct >> 1, half = ct & 1;
+      const int r = ct >> 1, q = ct & 1;   // row, and K sub-tile of the stage
+      static_assert(W4_CONV_THREADS == 128 * W4_KSUB, "a converter thread per row and sub-tile");
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const TileInfo t = gemm_tile(src, BN, tile);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; kb += L::KS) {
           if (!__all_sync(0xffffffffu,
                           mbar_wait_bounded(&full[stage], phase, abort_flag, err, limit_ns))) {
             ok = false;
             break;
           }
           const uint8_t* raw = sR + stage * L::RAW_BYTES;
-          const uint4 c = *reinterpret_cast<const uint4*>(raw + r * 32 + half * 16);
-          const uint32_t sc4 =
-              *reinterpret_cast<const uint32_t*>(raw + W4_CODE_BYTES + sf_atom_offset(r, 0));
-          const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-          uint8_t* dst = sA + stage * L::A_BYTES + r * GEMM_ROW_BYTES;
+          // codes: [128 rows][KS x 32 B]; scales: KS atoms after them
+          const uint4 c0 = *reinterpret_cast<const uint4*>(raw + r * 32 * L::KS + q * 32);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(raw + r * 32 * L::KS + q * 32 + 16);
+          const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(
+              raw + L::KS * W4_CODE_BYTES + q * SF_ATOM_BYTES + sf_atom_offset(r, 0));
+          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          uint8_t* dst = sA + stage * L::A_BYTES + q * L::A_SUB + r * GEMM_ROW_BYTES;
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            const int blk = 2 * half + b;   // 16-element block of the row
+          for (int blk = 0; blk < 4; ++blk) {   // 16-element blocks of the row
             const uint32_t sb = (sc4 >> (8 * blk)) & 0xFFu;
             const uint32_t s2 = f16x2_from_e4m3x2(sb | (sb << 8));
             uint32_t lo[4], hi[4];
-            f16x2_from_e2m1x8(cw[2 * b], lo);
-            f16x2_from_e2m1x8(cw[2 * b + 1], hi);
+            f16x2_from_e2m1x8(cw[2 * blk], lo);
+            f16x2_from_e2m1x8(cw[2 * blk + 1], hi);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               lo[i] = hmul2_f16(lo[i], s2);

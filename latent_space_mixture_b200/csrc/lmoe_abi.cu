@@ -257,14 +257,14 @@ template <>
 struct Stages<32, KIND_NVFP4> {
   static constexpr int value = 8;
 };
-// W4A16 stages also hold the raw FP4 codes and scale atom (4.5 KB)
+// W4A16 stages hold two K sub-tiles plus the raw FP4 codes and scale atoms
 template <>
 struct Stages<128, KIND_W4A16> {
-  static constexpr int value = 5;
+  static constexpr int value = 2;
 };
 template <>
 struct Stages<32, KIND_W4A16> {
-  static constexpr int value = 8;
+  static constexpr int value = 4;
 };
 
 template <int BN, class Epi, int KIND = KIND_BF16>
@@ -396,14 +396,14 @@ static bool make_map_strided(CUtensorMap* m, const void* base, uint64_t rows, ui
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D byte matrix [rows][cols] of packed FP4 codes read as 32-byte x 128-row
-// tiles without swizzle (the W4A16 converter reads them row by row)
+// 2-D byte matrix [rows][cols] of packed FP4 codes read as (32 x W4_KSUB)-byte
+// x 128-row tiles without swizzle (the W4A16 converter reads them row by row)
 static bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   PFN_encodeTiled enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols};
-  const cuuint32_t box[2] = {32, GEMM_BM};
+  const cuuint32_t box[2] = {32 * W4_KSUB, GEMM_BM};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,

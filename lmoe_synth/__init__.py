@@ -85,6 +85,9 @@ CONFIGS: Dict[str, LayerConfig] = {
     # the small prefill case with NVFP4 experts, for profiler captures
     "super_prefill_nvfp4_n64": LayerConfig("super_prefill_nvfp4_n64", 1024, 4096, 1024, 64, 22,
                                            2688, 5376, 0.02, "zipf", 8, "nvfp4"),
+    # Super dims decode with NVFP4 experts (weights and activations: W4A4)
+    "super_decode_nvfp4": LayerConfig("super_decode_nvfp4", 256, 4096, 1024, 512, 22, 2688, 5376,
+                                      0.02, "zero", 1, "nvfp4"),
     # Super dims prefill with NVFP4 experts, Zipf(1.1) router bias
     "super_prefill_nvfp4": LayerConfig("super_prefill_nvfp4", 8192, 4096, 1024,
                                        512, 22, 2688, 5376, 0.02, "zipf", 4,
