@@ -313,6 +313,8 @@ template <int KIND, class Epi>
 cudaError_t launch_gemm_q(int bn, const CUtensorMap& A, const BMaps& B, const TileSource& src,
                           const Epi& epi, int grid, int* err, unsigned long long limit,
                           cudaStream_t st) {
+  if constexpr (KIND == KIND_FP8)
+    if (bn == 256) return launch_gemm<256, Epi, KIND>(A, B, src, epi, grid, err, limit, st);
   if (bn == 128) return launch_gemm<128, Epi, KIND>(A, B, src, epi, grid, err, limit, st);
   return launch_gemm<32, Epi, KIND>(A, B, src, epi, grid, err, limit, st);
 }
@@ -611,7 +613,10 @@ static int check_cfg(const lmoe_config* c) {
 static int grouped_bn(const lmoe_config& c, int64_t T) {
   const double avg = double(T) * c.top_k / c.n_experts;
   if (avg <= 40.0) return 32;
-  if (avg <= 160.0 || c.expert_format != LMOE_FMT_BF16) return 128;
+  // NVFP4 B tiles carry one scale atom (<= 128 rows); W4A16 stages at 256
+  // rows would leave one stage of shared memory
+  if (avg <= 160.0 || c.expert_format == LMOE_FMT_NVFP4 || c.expert_format == LMOE_FMT_W4A16)
+    return 128;
   return 256;
 }
 
@@ -786,6 +791,8 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= make_map_u8(&h->tm_upf8.b64, h->upf8, rows_b, l, GEMM_BROWS_BIG);
     ok &= make_map_u8(&h->tm_Hf8.b16, h->Hf8, rows_b, hh, GEMM_BROWS);
     ok &= make_map_u8(&h->tm_Hf8.b64, h->Hf8, rows_b, hh, GEMM_BROWS_BIG);
+    ok &= set_gemm_smem<256, EpiH8, KIND_FP8>() == cudaSuccess;
+    ok &= set_gemm_smem<256, EpiO8, KIND_FP8>() == cudaSuccess;
     ok &= set_gemm_smem<128, EpiH8, KIND_FP8>() == cudaSuccess;
     ok &= set_gemm_smem<32, EpiH8, KIND_FP8>() == cudaSuccess;
     ok &= set_gemm_smem<128, EpiO8, KIND_FP8>() == cudaSuccess;
