@@ -64,6 +64,9 @@ extern "C" {
  * lmoe_create. */
 #define LMOE_FLAG_NVFP4_WEIGHT_2D 2
 #define LMOE_FLAG_NVFP4_WEIGHT_MSE 4
+/* LMOE_FLAG_BACKWARD: also reserve the workspace of lmoe_backward (BF16
+ * experts with latent projections only; UNSUPPORTED otherwise). */
+#define LMOE_FLAG_BACKWARD 8
 
 #define LMOE_FMT_BF16 0  /* experts in BF16                                   */
 #define LMOE_FMT_NVFP4 1 /* experts in NVFP4: W1, W2 and the expert inputs u
@@ -153,6 +156,47 @@ int lmoe_forward_host(lmoe_handle* h, const void* x_host, int64_t T, void* y_hos
  * the stream reports an error, else OK. */
 int lmoe_sync_status(lmoe_handle* h, void* stream);
 
+/* Gradients of the weights, fp32 device buffers in the layouts of
+ * lmoe_weights, written (not accumulated) by lmoe_backward. */
+typedef struct lmoe_grads {
+  float* d_router;  /* [N][d]     dL/dW_r                                   */
+  float* d_dn;      /* [l][d]     dL/dW_dn                                  */
+  float* d_w1;      /* [N][h][l]  dL/dW1 (zero for experts no token chose)  */
+  float* d_w2;      /* [N][l][h]  dL/dW2                                    */
+  float* d_upl;     /* [d][l]     dL/dW_upl                                 */
+  float* d_s1;      /* [h_s][d]   dL/dW_s1                                  */
+  float* d_s2;      /* [d][h_s]   dL/dW_s2                                  */
+} lmoe_grads;
+
+/* Backward pass of the last lmoe_forward on this handle: given dy = dL/dy
+ * [T][d] bf16 (device), writes dx = dL/dx [T][d] bf16 (device) and the weight
+ * gradients into *g.  x must be the forward's input (same pointer contents
+ * and the same T); no other forward may run on the handle in between, since
+ * the backward reads the forward's routing and saved activations (expert
+ * inputs u, expert hidden sqrelu(W1 u), v and the shared hidden) from the
+ * workspace.  The derivative is the exact one of the forward: the top-K
+ * selection is piecewise constant, so the router receives gradient through
+ * the renormalised weights w = s_S / sum s_S only, and the expert bias none
+ * (see lmoe_bias_update).  The activation derivative 2 max(a, 0) is taken
+ * as 2 sqrt(sqrelu(a)) from the saved bf16 hidden activations.  Products in
+ * bf16 with fp32 accumulation; dx and the intermediate gradients rounded to
+ * bf16.  Asynchronous on `stream`, no allocation.  dx must not overlap x or
+ * dy; every pointer 16-byte aligned.  T == 0 is a no-op.
+ * Errors: INVALID_ARG (null, T differs from the last forward's, overlap,
+ * misalignment), UNSUPPORTED (handle without LMOE_FLAG_BACKWARD, or not
+ * BF16 experts with projections), CUDA. */
+int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void* dx,
+                  const lmoe_grads* g, void* stream);
+
+/* Aux-loss-free load balancing ("Nemotron-3 Super 精读报告", table 6.3:
+ * update rate 1e-3): after a forward, every expert bias moves by
+ * rate * sign(mean - c_e), c_e the rows routed to expert e by that forward
+ * and mean = T K / N (an expert exactly at the mean keeps its bias); float32
+ * arithmetic on the handle's router bias, which the next forward uses.
+ * Asynchronous on `stream`.  Errors: INVALID_ARG (no forward yet, rate not
+ * finite), CUDA. */
+int lmoe_bias_update(lmoe_handle* h, float rate, void* stream);
+
 /* Debug/test readout of the last forward's intermediates into HOST memory
  * (synchronizes the device first).  `bytes` must equal the item's size for
  * the last T:
@@ -166,6 +210,7 @@ int lmoe_sync_status(lmoe_handle* h, void* stream);
  *   LMOE_DBG_U         bf16  [T][l]   latent u
  *   LMOE_DBG_V         bf16  [T][l]   latent combine v
  *   LMOE_DBG_HS        bf16  [T][h_s] shared hidden sqrelu(W_s1 x)
+ *   LMOE_DBG_BIAS      fp32  [N]      the router bias (after lmoe_bias_update)
  * and, for NVFP4 experts (lp, hp = l, h rounded up to 256):
  *   LMOE_DBG_W1Q_CODES u8   [N*h][lp/2]  E2M1 codes, lower index in the low nibble
  *   LMOE_DBG_W1Q_SF    u8   [N*h/128][lp/64][512] E4M3 scales; row m, 16-block
@@ -189,6 +234,7 @@ int lmoe_sync_status(lmoe_handle* h, void* stream);
 #define LMOE_DBG_W2Q_CODES 14
 #define LMOE_DBG_W2Q_SF 15
 #define LMOE_DBG_W2Q_G 16
+#define LMOE_DBG_BIAS 17
 int lmoe_get_debug(lmoe_handle* h, int what, void* dst_host, size_t bytes);
 
 /* Kernel launches one lmoe_forward of T tokens issues (10, plus one split-K

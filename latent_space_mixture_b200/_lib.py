@@ -16,11 +16,12 @@ FMT_BF16, FMT_NVFP4, FMT_FP8, FMT_W4A16 = 0, 1, 2, 3
 FLAG_NO_PROJECTION = 1   # standard MoE: no latent projections (u = x, r = v)
 FLAG_NVFP4_WEIGHT_2D = 2   # NVFP4 weights: one scale per 16 x 16 block
 FLAG_NVFP4_WEIGHT_MSE = 4  # NVFP4 weights: MSE-searched block scales
+FLAG_BACKWARD = 8   # reserve the workspace of lmoe_backward
 NVFP4_WEIGHT_FLAGS = {"1d": 0, "2d": FLAG_NVFP4_WEIGHT_2D, "mse": FLAG_NVFP4_WEIGHT_MSE,
                       "2d_mse": FLAG_NVFP4_WEIGHT_2D | FLAG_NVFP4_WEIGHT_MSE}
 DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 6,
        "logits": 7, "u": 8, "v": 9, "hs": 10, "w1q_codes": 11, "w1q_sf": 12, "w1q_g": 13,
-       "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16}
+       "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16, "bias": 17}
 
 
 class LmoeConfig(Structure):
@@ -36,6 +37,11 @@ class LmoeWeights(Structure):
                 ("act_gscale_hidden", c_float)]
 
 
+class LmoeGrads(Structure):
+    _fields_ = [("d_router", c_void_p), ("d_dn", c_void_p), ("d_w1", c_void_p),
+                ("d_w2", c_void_p), ("d_upl", c_void_p), ("d_s1", c_void_p), ("d_s2", c_void_p)]
+
+
 class LmoeError(RuntimeError):
     def __init__(self, code: int, what: str = ""):
         self.code = code
@@ -48,6 +54,9 @@ SIGNATURES = {
     "lmoe_create": (c_int, [POINTER(LmoeConfig), POINTER(LmoeWeights), POINTER(c_void_p)]),
     "lmoe_forward": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
     "lmoe_forward_host": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
+    "lmoe_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p,
+                              POINTER(LmoeGrads), c_void_p]),
+    "lmoe_bias_update": (c_int, [c_void_p, c_float, c_void_p]),
     "lmoe_sync_status": (c_int, [c_void_p, c_void_p]),
     "lmoe_get_debug": (c_int, [c_void_p, c_int, c_void_p, c_size_t]),
     "lmoe_launches_per_forward": (c_int, [c_void_p, c_int64]),

@@ -58,6 +58,26 @@ cudaError_t launch_gather_q(const uint8_t* uq, const uint8_t* usf, const int32_t
                             const int32_t* rblock, int64_t rows, int K, int l, int lp,
                             uint8_t* u_perm_q, uint8_t* atoms, cudaStream_t st);
 
+// Backward pass (backward.cu).  dst[r] = wrow[r] * dv[perm[r] / K], rows of
+// width l (bf16, l % 8 == 0).
+cudaError_t launch_gather_scaled(const void* dv, const int32_t* perm, const float* wrow,
+                                 int64_t rows, int K, int l, void* dst, cudaStream_t st);
+
+// Expert activation derivative per routed row: da = dg * 2 sqrt(g) in place
+// (da holds dg on entry; g = H, both [rows][h] bf16), dwacc[r] = g . dg.
+cudaError_t launch_dact(void* da, const void* H, int64_t rows, int h, float* dwacc,
+                        cudaStream_t st);
+
+// Router backward: dz of the selected experts (zero elsewhere) into columns
+// [0, N) of dxh (bf16, row pitch ldx), from dwacc[r] = sum_h g_r[h] dg_r[h].
+cudaError_t launch_route_bw(const float* logits, const int32_t* topk_idx, const int32_t* inv,
+                            const float* wrow, const float* dwacc, int64_t T, int N, int K,
+                            void* dxh, int ldx, cudaStream_t st);
+
+// Aux-loss-free bias update: bias[e] += rate * sign(total - N * counts[e]).
+cudaError_t launch_bias_update(float* bias, const int32_t* counts, int N, int64_t total, float rate,
+                               cudaStream_t st);
+
 // A kernel whose mbarrier wait never completes, bounded by limit_ns: sets
 // DEVERR_TIMEOUT in *err and returns.  Used to check the failure path.
 cudaError_t launch_wait_probe(int* err, unsigned long long limit_ns, cudaStream_t st);

@@ -1,6 +1,7 @@
-// C ABI of the LatentMoE layer forward pass (declarations and contracts in
-// include/lmoe.h).  Host orchestration only: every step of the layer runs in
-// the kernels of gemm_tc.cuh and routing.cu.
+// C ABI of the LatentMoE layer forward and backward passes (declarations and
+// contracts in include/lmoe.h).  Host orchestration only: every step of the
+// layer runs in the kernels of gemm_tc.cuh, gemm_pair.cuh, gemm_bw.cuh,
+// routing.cu, nvfp4.cu and backward.cu.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -10,6 +11,7 @@
 #include <new>
 #include <vector>
 
+#include "gemm_bw.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.h"
@@ -243,6 +245,145 @@ struct EpiO16 {
   }
 };
 
+// ---------------------------------------------------------------------------
+// epilogues of the backward contractions (gemm_bw.cuh; rows are tokens or
+// routed rows for the data gradients, rows of dW for the weight gradients)
+
+// dy -> dy [W_upl | W_s2]: dv (bf16, [T][l]) and the gradient of the shared
+// hidden pre-activation, (dy W_s2) * 2 max(a, 0) with max(a, 0) =
+// sqrt(sqrelu(a)) from the forward's hs (columns [l, l+h_s) of vh), into
+// columns [N+l, N+l+h_s) of dxh.
+struct EpiDVH {
+  static constexpr bool kAux = true;   // reads hs
+  bf16* dv;
+  bf16* dxh;
+  const bf16* vh;
+  int l, ldvh, ldx, N;
+  __device__ __forceinline__ uint4 fetch(long row, int feat, bool valid) const {
+    if (!valid || feat < l) return make_uint4(0u, 0u, 0u, 0u);
+    return *reinterpret_cast<const uint4*>(vh + row * ldvh + feat);
+  }
+  __device__ __forceinline__ void store8(const BwTile&, long row, int feat, const float* v,
+                                         bool valid, const uint4 raw) const {
+    if (!valid) return;
+    if (feat < l) {
+      store8_bf16(dv + row * l + feat, v);
+      return;
+    }
+    const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 g = __bfloat1622float2(hp[i]);
+      a[2 * i] = v[2 * i] * (2.0f * sqrtf(g.x));
+      a[2 * i + 1] = v[2 * i + 1] * (2.0f * sqrtf(g.y));
+    }
+    store8_bf16(dxh + row * ldx + N + feat, a);
+  }
+};
+
+// plain bf16 store of the product (du rows in expert order; dx)
+struct EpiStore {
+  static constexpr bool kAux = false;
+  bf16* out;
+  int ld;
+  __device__ __forceinline__ void store8(const BwTile&, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (valid) store8_bf16(out + row * ld + feat, v);
+  }
+};
+
+__device__ __forceinline__ void store8_f32(float* dst, const float* v) {
+  float4* q = reinterpret_cast<float4*>(dst);
+  q[0] = make_float4(v[0], v[1], v[2], v[3]);
+  q[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// d[W_r; W_dn; W_s1] = dxh^T x: rows [0, r1) to p0, [r1, r2) to p1, the rest
+// to p2 (fp32, row pitch ld)
+struct EpiWRows {
+  static constexpr bool kAux = false;
+  float *p0, *p1, *p2;
+  int r1, r2, ld;
+  __device__ __forceinline__ void store8(const BwTile&, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    float* dst = row < r1 ? p0 + row * ld : row < r2 ? p1 + (row - r1) * ld : p2 + (row - r2) * ld;
+    store8_f32(dst + feat, v);
+  }
+};
+
+// d[W_upl | W_s2] = dy^T [v | hs]: columns [0, c1) to p0 (pitch ld0), the
+// rest to p1 (pitch ld1)
+struct EpiWCols {
+  static constexpr bool kAux = false;
+  float *p0, *p1;
+  int c1, ld0, ld1;
+  __device__ __forceinline__ void store8(const BwTile&, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    if (feat < c1) store8_f32(p0 + row * ld0 + feat, v);
+    else store8_f32(p1 + row * ld1 + (feat - c1), v);
+  }
+};
+
+// per-expert weight gradient dW[e] (fp32, [rows][ld], experts estride apart)
+struct EpiWExp {
+  static constexpr bool kAux = false;
+  float* p;
+  long estride;
+  int ld;
+  __device__ __forceinline__ void store8(const BwTile& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (valid) store8_f32(p + t.e * estride + row * ld + feat, v);
+  }
+};
+
+template <int BN>
+struct BwStages {
+  static constexpr int value = BN == 256 ? 4 : BN == 128 ? 6 : 10;
+};
+
+template <int BN, bool B_MN, class Epi>
+cudaError_t set_bw_smem() {
+  constexpr int S = BwStages<BN>::value;
+  return cudaFuncSetAttribute(k_gemm_bw<BN, S, B_MN, Epi>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              BwLayout<BN, S, B_MN>::SMEM_BYTES);
+}
+
+template <int BN, bool B_MN, class Epi>
+cudaError_t launch_bw(const CUtensorMap& A, const CUtensorMap& B16, const CUtensorMap& B64,
+                      const BwSource& src, const Epi& epi, int grid, int* err,
+                      unsigned long long limit, cudaStream_t st) {
+  constexpr int S = BwStages<BN>::value;
+  return launch_pdl(k_gemm_bw<BN, S, B_MN, Epi>, grid, GEMM_THREADS,
+                    BwLayout<BN, S, B_MN>::SMEM_BYTES, st, A, B16, B64, src, epi, err, limit);
+}
+
+// data-gradient GEMM with a K-major token-row B operand of BN rows per block
+template <class Epi>
+cudaError_t launch_bw_dgrad(int bn, const CUtensorMap& A, const CUtensorMap& B16,
+                            const CUtensorMap& B64, const BwSource& src, const Epi& epi, int grid,
+                            int* err, unsigned long long limit, cudaStream_t st) {
+  switch (bn) {
+    case 256: return launch_bw<256, false>(A, B16, B64, src, epi, grid, err, limit, st);
+    case 128: return launch_bw<128, false>(A, B16, B64, src, epi, grid, err, limit, st);
+    default: return launch_bw<32, false>(A, B16, B64, src, epi, grid, err, limit, st);
+  }
+}
+
+template <class Epi>
+cudaError_t set_bw_dgrad_smem() {
+  cudaError_t e;
+  if ((e = set_bw_smem<256, false, Epi>()) != cudaSuccess) return e;
+  if ((e = set_bw_smem<128, false, Epi>()) != cudaSuccess) return e;
+  return set_bw_smem<32, false, Epi>();
+}
+
+// token-block width of the dense data-gradient GEMMs
+static int bw_dense_bn(int64_t T) { return T >= 2048 ? 256 : T >= 512 ? 128 : 32; }
+
 // GEMM variants: (BN, operand kind) -> pipeline stages (FP8 stages hold
 // 128-byte rows like bf16 ones)
 template <int BN, int KIND>
@@ -449,8 +590,13 @@ using namespace lmoe;
 static const char* const kKernelNames[] = {
     "xgemm(router|W_dn|W_s1)", "route(sigmoid+bias+topK)", "hist", "scan", "scatter",
     "gather(u->expert order)", "grouped_gemm1(W1,sqrelu)", "grouped_gemm2(W2,*w)",
-    "combine", "ygemm([W_upl|W_s2])", "xgemm split-K reduce", "ygemm split-K reduce"};
-static constexpr int kNumKernels = 12;
+    "combine", "ygemm([W_upl|W_s2])", "xgemm split-K reduce", "ygemm split-K reduce",
+    // backward
+    "bw dgrad [W_upl|W_s2]^T (dv, dhs)", "bw gather(w dv -> expert order)",
+    "bw dgrad W2^T (dg)", "bw dgrad W1^T (du rows)", "bw combine(du)", "bw route(dz)",
+    "bw dgrad [W_r;W_dn;W_s1]^T (dx)", "bw wgrad [W_upl|W_s2]", "bw wgrad W2",
+    "bw wgrad W1", "bw wgrad [W_r;W_dn;W_s1]", "bw act'(da = dg 2 sqrt(g), dw)"};
+static constexpr int kNumKernels = 24;
 
 // Dense-GEMM plan for T tokens: token-block width and number of K slices.
 // Enough tiles to fill the GPU first by narrower token blocks (while one
@@ -540,6 +686,17 @@ struct lmoe_handle {
   bool w4 = false;
   __half* u16 = nullptr;       // [T][l]
   CUtensorMap tm_w1c, tm_w2c;
+  // backward workspace (LMOE_FLAG_BACKWARD)
+  bool bw = false;
+  bf16* dv = nullptr;        // [Tm_b][l]   dL/dv
+  bf16* dog = nullptr;       // [rows_b][l] w_r dv rows in expert order
+  bf16* da = nullptr;        // [rows_b][h] gradient of the expert pre-activation
+  bf16* dup = nullptr;       // [rows_b][l] W1[e]^T da rows in expert order
+  float* dwacc = nullptr;    // [rows]      sum_h g dg per routed row
+  bf16* dxh = nullptr;       // [Tm_b][N+l+h_s] dz | du | d(shared pre-activation)
+  bf16* dy_dev = nullptr;    // [64][d]     staging of dy for T < 64
+  CUtensorMap tm_wx64, tm_wy64, tm_w1_64, tm_w2_64;   // weights in 64-row boxes
+  BMaps tm_dog, tm_da, tm_dxh;
   std::vector<void*> allocs;
   CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
   BMaps tm_uperm, tm_H, tm_vh;
@@ -584,13 +741,16 @@ static int check_cfg(const lmoe_config* c) {
   if (c->d <= 0 || c->latent <= 0 || c->n_experts <= 0 || c->top_k <= 0 ||
       c->expert_hidden <= 0 || c->shared_hidden <= 0 || c->max_tokens < 1 ||
       (c->flags & ~(LMOE_FLAG_NO_PROJECTION | LMOE_FLAG_NVFP4_WEIGHT_2D |
-                    LMOE_FLAG_NVFP4_WEIGHT_MSE)) != 0)
+                    LMOE_FLAG_NVFP4_WEIGHT_MSE | LMOE_FLAG_BACKWARD)) != 0)
     return LMOE_ERR_INVALID_ARG;
   if ((c->flags & (LMOE_FLAG_NVFP4_WEIGHT_2D | LMOE_FLAG_NVFP4_WEIGHT_MSE)) &&
       c->expert_format != LMOE_FMT_NVFP4 && c->expert_format != LMOE_FMT_W4A16)
     return LMOE_ERR_INVALID_ARG;
   if ((c->flags & LMOE_FLAG_NO_PROJECTION) &&
       (c->latent != c->d || c->expert_format != LMOE_FMT_BF16))
+    return LMOE_ERR_UNSUPPORTED;
+  if ((c->flags & LMOE_FLAG_BACKWARD) &&
+      ((c->flags & LMOE_FLAG_NO_PROJECTION) || c->expert_format != LMOE_FMT_BF16))
     return LMOE_ERR_UNSUPPORTED;
   if (c->top_k > c->n_experts) return LMOE_ERR_INVALID_ARG;
   if (c->expert_format != LMOE_FMT_BF16 && c->expert_format != LMOE_FMT_NVFP4 &&
@@ -704,6 +864,8 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   }
   h->part_floats = part_floats;
   const int64_t max_blocks = rows / 32 + N + 1;
+  const int64_t bwd = (c.flags & LMOE_FLAG_BACKWARD) ? 1 : 0;
+  h->bw = bwd != 0;
   struct Req {
     void** p;
     size_t bytes;
@@ -755,6 +917,13 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->uf8, size_t(fp8 * Tm * l)},
       {(void**)&h->upf8, size_t(fp8 * rows_b * l)},
       {(void**)&h->Hf8, size_t(fp8 * rows_b * hh)},
+      {(void**)&h->dv, size_t(bwd * Tm_b * l * 2)},
+      {(void**)&h->dog, size_t(bwd * rows_b * l * 2)},
+      {(void**)&h->da, size_t(bwd * rows_b * hh * 2)},
+      {(void**)&h->dup, size_t(bwd * rows_b * l * 2)},
+      {(void**)&h->dwacc, size_t(bwd * rows * 4)},
+      {(void**)&h->dxh, size_t(bwd * Tm_b * (N + l + hs) * 2)},
+      {(void**)&h->dy_dev, size_t(bwd * GEMM_BROWS_BIG * d * 2)},
   };
   for (auto& r : reqs) {
     if ((rc = alloc_dev(h, r.p, r.bytes)) != LMOE_OK) {
@@ -876,6 +1045,29 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   ok &= make_map_strided(&h->tm_vh.b16, h->vh + (l - lx), Tm_b, lx + hs, l + hs, GEMM_BROWS);
   ok &= make_map_strided(&h->tm_vh.b64, h->vh + (l - lx), Tm_b, lx + hs, l + hs,
                          GEMM_BROWS_BIG);
+  if (bwd) {
+    // MN-major operands of the backward GEMMs: 64 x 64 boxes (the same boxes
+    // serve K-major token rows); padding rows read as zero
+    ok &= cudaMemset(h->dog, 0, rows_b * l * 2) == cudaSuccess;
+    ok &= cudaMemset(h->da, 0, rows_b * hh * 2) == cudaSuccess;
+    ok &= cudaMemset(h->dxh, 0, Tm_b * (N + l + hs) * 2) == cudaSuccess;
+    ok &= cudaMemset(h->dy_dev, 0, GEMM_BROWS_BIG * d * 2) == cudaSuccess;
+    ok &= make_map(&h->tm_wx64, h->w_x, N + lx + hs, d, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_wy64, h->w_y, d_a, lx + hs, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_w1_64, h->w1, N * hh, l, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_w2_64, h->w2, N * l, hh, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_dog.b16, h->dog, rows_b, l, GEMM_BROWS);
+    ok &= make_map(&h->tm_dog.b64, h->dog, rows_b, l, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_da.b16, h->da, rows_b, hh, GEMM_BROWS);
+    ok &= make_map(&h->tm_da.b64, h->da, rows_b, hh, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_dxh.b16, h->dxh, Tm_b, N + l + hs, GEMM_BROWS);
+    ok &= make_map(&h->tm_dxh.b64, h->dxh, Tm_b, N + l + hs, GEMM_BROWS_BIG);
+    ok &= set_bw_dgrad_smem<EpiDVH>() == cudaSuccess;
+    ok &= set_bw_dgrad_smem<EpiStore>() == cudaSuccess;
+    ok &= set_bw_smem<256, true, EpiWRows>() == cudaSuccess;
+    ok &= set_bw_smem<256, true, EpiWCols>() == cudaSuccess;
+    ok &= set_bw_smem<256, true, EpiWExp>() == cudaSuccess;
+  }
   ok &= set_smem_all<EpiX>() == cudaSuccess;
   ok &= set_smem_all<EpiH>() == cudaSuccess;
   ok &= set_smem_all<EpiO>() == cudaSuccess;
@@ -1118,6 +1310,162 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   return LMOE_OK;
 }
 
+int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void* dx,
+                  const lmoe_grads* gr, void* stream) {
+  if (!h || T < 0) return LMOE_ERR_INVALID_ARG;
+  if (!h->bw) return LMOE_ERR_UNSUPPORTED;
+  if (T == 0) return LMOE_OK;
+  if (T != h->last_T || !x || !dy || !dx || !gr || !gr->d_router || !gr->d_dn || !gr->d_w1 ||
+      !gr->d_w2 || !gr->d_upl || !gr->d_s1 || !gr->d_s2)
+    return LMOE_ERR_INVALID_ARG;
+  const lmoe_config& c = h->cfg;
+  const int64_t d = c.d;
+  const char* xb = static_cast<const char*>(x);
+  const char* yb = static_cast<const char*>(dy);
+  const char* ob = static_cast<const char*>(dx);
+  const int64_t nb = T * d * 2;
+  if ((ob < xb + nb && xb < ob + nb) || (ob < yb + nb && yb < ob + nb)) return LMOE_ERR_INVALID_ARG;
+  const uintptr_t align = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy) |
+                          reinterpret_cast<uintptr_t>(dx) |
+                          reinterpret_cast<uintptr_t>(gr->d_router) |
+                          reinterpret_cast<uintptr_t>(gr->d_dn) |
+                          reinterpret_cast<uintptr_t>(gr->d_w1) |
+                          reinterpret_cast<uintptr_t>(gr->d_w2) |
+                          reinterpret_cast<uintptr_t>(gr->d_upl) |
+                          reinterpret_cast<uintptr_t>(gr->d_s1) |
+                          reinterpret_cast<uintptr_t>(gr->d_s2);
+  if (align & 15) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int N = c.n_experts, l = c.latent, hh = c.expert_hidden, hs = c.shared_hidden,
+            K = c.top_k;
+  const int ldvh = l + hs, ldx = N + l + hs;
+  const int64_t R = T * K;
+  const unsigned long long lim = h->wait_limit_ns;
+  // dy and x as 64-row boxes (token rows, or MN-major for the weight
+  // gradients); fewer than 64 rows go through the padded staging buffers
+  BMaps tm_dy, tm_x;
+  const void* dy_src = dy;
+  const void* x_src = x;
+  int64_t map_rows = T;
+  if (T < GEMM_BROWS_BIG) {
+    if (cudaMemcpyAsync(h->dy_dev, dy, T * d * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        (x != h->x_dev &&
+         cudaMemcpyAsync(h->x_dev, x, T * d * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess))
+      return LMOE_ERR_CUDA;
+    dy_src = h->dy_dev;
+    x_src = h->x_dev;
+    map_rows = GEMM_BROWS_BIG;
+  }
+  if (!make_map(&tm_dy.b16, dy_src, map_rows, d, GEMM_BROWS) ||
+      !make_map(&tm_dy.b64, dy_src, map_rows, d, GEMM_BROWS_BIG) ||
+      !make_map(&tm_x.b64, x_src, map_rows, d, GEMM_BROWS_BIG))
+    return LMOE_ERR_CUDA;
+  const int dbn = bw_dense_bn(T);
+  const int gbn = grouped_bn(c, T);   // the forward's token blocks
+  auto grid_of = [&](int64_t tiles) { return static_cast<int>(tiles < h->sms ? tiles : h->sms); };
+#define LMOE_BW(kidx, call)                          \
+  do {                                               \
+    const int _slot = prof_begin(h, 12 + (kidx), st); \
+    const cudaError_t _e = (call);                   \
+    prof_end(h, _slot, st);                          \
+    if (_e != cudaSuccess) {                         \
+      cudaGetLastError();                            \
+      return LMOE_ERR_CUDA;                          \
+    }                                                \
+  } while (0)
+  // 1. [dv | dhs] = dy [W_upl | W_s2]; dhs_pre = dhs * 2 sqrt(hs)
+  {
+    const int fb = (l + hs + 127) / 128;
+    BwSource s{0, 1, static_cast<int>(T), nullptr, nullptr, 0, static_cast<int>(d / 64), fb,
+               l + hs, l + hs};
+    EpiDVH epi{h->dv, h->dxh, h->vh, l, ldvh, ldx, N};
+    LMOE_BW(0, launch_bw_dgrad(dbn, h->tm_wy64, tm_dy.b16, tm_dy.b64, s, epi,
+                            grid_of(((T + dbn - 1) / dbn) * fb), h->err, lim, st));
+  }
+  // 2. do[r] = w_r dv[t(r)] in expert order
+  LMOE_BW(1, launch_gather_scaled(h->dv, h->perm, h->wrow, R, K, l, h->dog, st));
+  // 3. dg = W2[e]^T do (bf16, into the da buffer)
+  {
+    BwSource s{0, 0, 0, h->blocks, h->nblocks, l, l / 64, (hh + 127) / 128, hh, hh};
+    EpiStore epi{h->da, hh};
+    LMOE_BW(2, launch_bw_dgrad(gbn, h->tm_w2_64, h->tm_dog.b16, h->tm_dog.b64, s, epi, h->sms,
+                            h->err, lim, st));
+  }
+  // 3b. da = dg * 2 sqrt(g) in place, dwacc[r] = g . dg (g = the saved H row)
+  LMOE_BW(11, launch_dact(h->da, h->H, R, hh, h->dwacc, st));
+  // 4. du rows = W1[e]^T da
+  {
+    BwSource s{0, 0, 0, h->blocks, h->nblocks, hh, hh / 64, (l + 127) / 128, l, l};
+    EpiStore epi{h->dup, l};
+    LMOE_BW(3, launch_bw_dgrad(gbn, h->tm_w1_64, h->tm_da.b16, h->tm_da.b64, s, epi, h->sms, h->err,
+                            lim, st));
+  }
+  // 5. du[t] = sum_k du rows (slot order) into columns [N, N+l) of dxh
+  LMOE_BW(4, launch_combine(h->dup, h->inv, T, K, l, h->dxh + N, ldx, st));
+  // 6. router: dz into columns [0, N) of dxh
+  LMOE_BW(5, launch_route_bw(h->logits, h->topk_idx, h->inv, h->wrow, h->dwacc, T, N, K, h->dxh,
+                             ldx, st));
+  // 7. dx = [dz | du | dhs_pre] [W_r; W_dn; W_s1]
+  {
+    const int fb = static_cast<int>((d + 127) / 128);
+    BwSource s{0, 1, static_cast<int>(T), nullptr, nullptr, 0, (ldx + 63) / 64, fb,
+               static_cast<int>(d), static_cast<int>(d)};
+    EpiStore epi{static_cast<bf16*>(dx), static_cast<int>(d)};
+    LMOE_BW(6, launch_bw_dgrad(dbn, h->tm_wx64, h->tm_dxh.b16, h->tm_dxh.b64, s, epi,
+                            grid_of(((T + dbn - 1) / dbn) * fb), h->err, lim, st));
+  }
+  // 8. d[W_upl | W_s2] = dy^T [v | hs]  (rows d, columns l + h_s)
+  {
+    const int fb = (l + hs + 127) / 128, nbk = static_cast<int>((d + 255) / 256);
+    BwSource s{1, 0, static_cast<int>(T), nullptr, nullptr, 0, 0, fb, l + hs, l + hs,
+               1, nullptr, nbk, static_cast<int>(d), static_cast<int>(d)};
+    EpiWCols epi{gr->d_upl, gr->d_s2, l, l, hs};
+    LMOE_BW(7, (launch_bw<256, true>(h->tm_vh.b64, tm_dy.b64, tm_dy.b64, s, epi,
+                                  grid_of(int64_t(fb) * nbk), h->err, lim, st)));
+  }
+  // 9. dW2[e] = do^T g over the expert's rows  ([l][h])
+  {
+    const int fb = (hh + 127) / 128, nbk = (l + 255) / 256;
+    BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, hh, hh, N, h->offsets, nbk, l, l};
+    EpiWExp epi{gr->d_w2, int64_t(l) * hh, hh};
+    LMOE_BW(8, (launch_bw<256, true>(h->tm_H.b64, h->tm_dog.b64, h->tm_dog.b64, s, epi,
+                                  grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
+  }
+  // 10. dW1[e] = da^T u over the expert's rows  ([h][l])
+  {
+    const int fb = (l + 127) / 128, nbk = (hh + 255) / 256;
+    BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, l, l, N, h->offsets, nbk, hh, hh};
+    EpiWExp epi{gr->d_w1, int64_t(hh) * l, l};
+    LMOE_BW(9, (launch_bw<256, true>(h->tm_uperm.b64, h->tm_da.b64, h->tm_da.b64, s, epi,
+                                  grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
+  }
+  // 11. d[W_r; W_dn; W_s1] = dxh^T x  (rows N + l + h_s, columns d)
+  {
+    const int fb = static_cast<int>((d + 127) / 128), nbk = (ldx + 255) / 256;
+    BwSource s{1, 0, static_cast<int>(T), nullptr, nullptr, 0, 0, fb, static_cast<int>(d),
+               static_cast<int>(d), 1, nullptr, nbk, ldx, ldx};
+    EpiWRows epi{gr->d_router, gr->d_dn, gr->d_s1, N, N + l, static_cast<int>(d)};
+    LMOE_BW(10, (launch_bw<256, true>(tm_x.b64, h->tm_dxh.b64, h->tm_dxh.b64, s, epi,
+                                  grid_of(int64_t(fb) * nbk), h->err, lim, st)));
+  }
+#undef LMOE_BW
+  return LMOE_OK;
+}
+
+int lmoe_bias_update(lmoe_handle* h, float rate, void* stream) {
+  if (!h || h->last_T <= 0 || !(rate == rate) || rate > 3.0e38f || rate < -3.0e38f)
+    return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  const int64_t total = h->last_T * h->cfg.top_k;
+  if (launch_bias_update(h->bias, h->counts, h->cfg.n_experts, total, rate,
+                         static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return LMOE_ERR_CUDA;
+  }
+  return LMOE_OK;
+}
+
 int lmoe_sync_status(lmoe_handle* h, void* stream) {
   if (!h) return LMOE_ERR_INVALID_ARG;
   DeviceGuard g(h->dev);
@@ -1182,10 +1530,12 @@ int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
       if (h->fp8) { src = h->w2f8; want = N * l * c.expert_hidden; break; }
       src = h->w2q; want = N * l * h->hp / 2; break;
     case LMOE_DBG_W2Q_SF: src = h->w2sf; want = (N * l / 128) * (h->hp / 64) * 512; break;
+    case LMOE_DBG_BIAS: src = h->bias; want = N * 4; break;
     case LMOE_DBG_W2Q_G: src = h->fp8 ? h->sw2 : h->gw2; want = N * 4; break;
     default: return LMOE_ERR_INVALID_ARG;
   }
-  if (what >= LMOE_DBG_W1Q_CODES && !h->fp4 && !h->fp8 && !h->w4) return LMOE_ERR_INVALID_ARG;
+  if (what >= LMOE_DBG_W1Q_CODES && what <= LMOE_DBG_W2Q_G && !h->fp4 && !h->fp8 && !h->w4)
+    return LMOE_ERR_INVALID_ARG;
   if ((what == LMOE_DBG_W1Q_SF || what == LMOE_DBG_W2Q_SF) && !h->fp4 && !h->w4)
     return LMOE_ERR_INVALID_ARG;
   if (bytes != want) return LMOE_ERR_INVALID_ARG;

@@ -342,6 +342,21 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile stored as TMA
+// boxes of 64 elements (one 128-byte row) x K rows with 128-byte swizzle:
+// 8-row swizzle atoms of 1024 bytes along K; chunks of 64 MN elements
+// `chunk_bytes` apart (the leading byte offset), 8-row K groups 1024 bytes
+// apart (the stride byte offset).
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t smem_addr, uint32_t chunk_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFF) >> 4);
+  d |= static_cast<uint64_t>((chunk_bytes >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
 // Shared-memory descriptor of one 512-byte scale atom for tcgen05.cp: 32
 // rows of 16 bytes, no swizzle, 8-row core matrices 128 bytes apart.
 __device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t smem_addr) {
@@ -417,6 +432,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __host__ __device__ __forceinline__ uint32_t idesc_f8(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
+
+// instruction-descriptor bits: A (bit 15) or B (bit 16) read MN-major
+constexpr uint32_t IDESC_A_MN = 1u << 15;
+constexpr uint32_t IDESC_B_MN = 1u << 16;
 
 __host__ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |

@@ -10,9 +10,9 @@ from typing import Dict, Optional
 import torch
 
 from . import _lib
-from ._lib import (DBG, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8, FMT_NVFP4, FMT_W4A16,
-                   NVFP4_WEIGHT_FLAGS,
-                   LmoeConfig, LmoeError, LmoeWeights, check)
+from ._lib import (DBG, FLAG_BACKWARD, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8, FMT_NVFP4,
+                   FMT_W4A16, NVFP4_WEIGHT_FLAGS,
+                   LmoeConfig, LmoeError, LmoeGrads, LmoeWeights, check)
 
 __all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]
 
@@ -37,12 +37,13 @@ class LatentMoE:
     the experts work on x and their combined output is added as is).
     nvfp4_weights ("1d", "2d", "mse", "2d_mse") picks the NVFP4 weight blocks
     and scale choice (LMOE_FLAG_NVFP4_WEIGHT_* of the C ABI).
+    backward=True reserves the workspace of lmoe_backward (LMOE_FLAG_BACKWARD).
     """
 
     def __init__(self, d: int, latent: int, n_experts: int, top_k: int, expert_hidden: int,
                  shared_hidden: int, max_tokens: int, weights: Dict[str, torch.Tensor],
                  expert_format: str = "bf16", act_gscales=(0.0, 0.0), projections: bool = True,
-                 nvfp4_weights: str = "1d"):
+                 nvfp4_weights: str = "1d", backward: bool = False):
         self.lib = _lib.load()
         dims = {"d": d, "l": latent, "N": n_experts, "h": expert_hidden, "hs": shared_hidden}
         for k, shape in _WEIGHT_SHAPES.items():
@@ -62,7 +63,8 @@ class LatentMoE:
                               {"bf16": FMT_BF16, "nvfp4": FMT_NVFP4, "fp8": FMT_FP8,
                                "w4a16": FMT_W4A16}[expert_format],
                               (0 if projections else FLAG_NO_PROJECTION)
-                              | NVFP4_WEIGHT_FLAGS[nvfp4_weights], max_tokens)
+                              | NVFP4_WEIGHT_FLAGS[nvfp4_weights]
+                              | (FLAG_BACKWARD if backward else 0), max_tokens)
         w = LmoeWeights(weights["w_router"].data_ptr(),
                         bias.data_ptr() if bias is not None else None,
                         weights["w_dn"].data_ptr() if projections else None,
@@ -106,6 +108,46 @@ class LatentMoE:
               "lmoe_forward_host")
         self.last_T = T
 
+    # -- backward ---------------------------------------------------------
+    GRAD_NAMES = ("d_router", "d_dn", "d_w1", "d_w2", "d_upl", "d_s1", "d_s2")
+
+    def grad_buffers(self) -> Dict[str, torch.Tensor]:
+        """Empty fp32 CUDA tensors for every weight gradient, in weight layout."""
+        c = self.cfg
+        d, l, N, h, hs = c.d, c.latent, c.n_experts, c.expert_hidden, c.shared_hidden
+        shapes = {"d_router": (N, d), "d_dn": (l, d), "d_w1": (N, h, l), "d_w2": (N, l, h),
+                  "d_upl": (d, l), "d_s1": (hs, d), "d_s2": (d, hs)}
+        return {k: torch.empty(v, dtype=torch.float32, device=self.device)
+                for k, v in shapes.items()}
+
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, grads: Dict[str, torch.Tensor],
+                 dx: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """lmoe_backward of the last forward (x its input): dy [T][d] CUDA bf16
+        -> dx [T][d] CUDA bf16; writes the fp32 weight gradients into `grads`
+        (tensors from grad_buffers()).  Asynchronous."""
+        if dy.dtype != torch.bfloat16 or dy.shape != x.shape or not dy.is_cuda:
+            raise ValueError("dy: need CUDA bf16 of x's shape")
+        x = x.contiguous()
+        dy = dy.contiguous()
+        if dx is None:
+            dx = torch.empty_like(dy)
+        for k in self.GRAD_NAMES:
+            t = grads[k]
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{k}: need contiguous CUDA fp32")
+        g = LmoeGrads(*[grads[k].data_ptr() for k in self.GRAD_NAMES])
+        check(self.lib.lmoe_backward(self.h, c_void_p(x.data_ptr()), c_void_p(dy.data_ptr()),
+                                     x.shape[0], c_void_p(dx.data_ptr()), byref(g),
+                                     _stream_ptr(stream)), "lmoe_backward")
+        return dx
+
+    def bias_update(self, rate: float = 1e-3, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """lmoe_bias_update: aux-loss-free step of the router bias from the
+        last forward's expert loads."""
+        check(self.lib.lmoe_bias_update(self.h, ctypes.c_float(rate), _stream_ptr(stream)),
+              "lmoe_bias_update")
+
     def sync_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
         return self.lib.lmoe_sync_status(self.h, _stream_ptr(stream))
 
@@ -122,6 +164,7 @@ class LatentMoE:
             "perm": (torch.int32, (T * c.top_k,)), "inv": (torch.int32, (T, c.top_k)),
             "logits": (torch.float32, (T, c.n_experts)), "u": (torch.bfloat16, (T, c.latent)),
             "v": (torch.bfloat16, (T, c.latent)), "hs": (torch.bfloat16, (T, c.shared_hidden)),
+            "bias": (torch.float32, (c.n_experts,)),
         }
         lp = (c.latent + 255) // 256 * 256
         hp = (c.expert_hidden + 255) // 256 * 256
@@ -149,14 +192,15 @@ class LatentMoE:
         check(self.lib.lmoe_profile_enable(self.h, int(on)), "profile_enable")
 
     def profile_read(self, reset: bool = True):
-        n = 16
+        n = 32
         names = (c_char_p * n)()
         ms = (c_double * n)()
         cnt = (c_int64 * n)()
         k = self.lib.lmoe_profile_read(self.h, names, ms, cnt, n, int(reset))
         if k < 0:
             raise LmoeError(k, "profile_read")
-        return [(names[i].decode(), ms[i], cnt[i]) for i in range(k)]
+        # the forward's kernels always, the backward's when they ran
+        return [(names[i].decode(), ms[i], cnt[i]) for i in range(k) if i < 12 or cnt[i] > 0]
 
     def close(self) -> None:
         if getattr(self, "h", None):

@@ -32,7 +32,7 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["LayerConfig", "CONFIGS", "make_weights", "make_x", "act_global_scales"]
+__all__ = ["LayerConfig", "CONFIGS", "make_weights", "make_x", "make_grad_out", "act_global_scales"]
 
 
 @dataclass(frozen=True)
@@ -168,6 +168,17 @@ def make_x(cfg: LayerConfig, gen: torch.Generator, T: Optional[int] = None,
            device="cpu") -> torch.Tensor:
     """Token batch x [T][d] bf16 ~ N(0, 1), drawn after the weights."""
     T = cfg.T if T is None else T
+    return torch.randn((T, cfg.d), generator=gen, device=device,
+                       dtype=torch.float32).to(torch.bfloat16)
+
+
+def make_grad_out(cfg: LayerConfig, T: Optional[int] = None, device="cpu",
+                  seed: Optional[int] = None) -> torch.Tensor:
+    """Upstream gradient dL/dy [T][d] bf16 ~ N(0, 1) for the backward pass,
+    from its own generator (seed: the workload's seed + 1000)."""
+    T = cfg.T if T is None else T
+    gen = torch.Generator(device=device)
+    gen.manual_seed(cfg.seed + 1000 if seed is None else seed)
     return torch.randn((T, cfg.d), generator=gen, device=device,
                        dtype=torch.float32).to(torch.bfloat16)
 

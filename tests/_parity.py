@@ -40,7 +40,7 @@ def to64(t):
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
-def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None):
+def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None, backward=False):
     """Seeded weights and x on the device, and the layer built from them."""
     from lmoe_synth import make_weights, make_x
     from latent_space_mixture_b200 import LatentMoE
@@ -53,7 +53,7 @@ def make(cfg, T=None, device="cuda", max_tokens=None, overrides=None):
     layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs,
                       max_tokens or x.shape[0], w, expert_format=cfg.fmt,
                       act_gscales=act_global_scales(cfg) if cfg.fmt != "bf16" else (0.0, 0.0),
-                      projections=cfg.proj, nvfp4_weights=cfg.wq)
+                      projections=cfg.proj, nvfp4_weights=cfg.wq, backward=backward)
     return w, x, layer
 
 
