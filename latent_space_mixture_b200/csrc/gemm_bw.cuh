@@ -107,11 +107,15 @@ __device__ __forceinline__ BwTile bw_tile(const BwSource& s, int BN, int tile) {
   return t;
 }
 
-template <int BN, int STAGES, bool B_MN>
+// fp32 epilogue boxes stored by TMA: 32 features x 32 rows, two per warp
+constexpr int BW_TMA_BOX_BYTES = 32 * 32 * 4;
+
+template <int BN, int STAGES, bool B_MN, bool TMA_OUT = false>
 struct BwLayout {
   static constexpr int A_BYTES = 2 * BW_BOX_BYTES;          // 128 x 64 bf16
   static constexpr int B_BYTES = BN * GEMM_ROW_BYTES;       // BN x 64 bf16 (either major)
-  static constexpr int STG_BYTES = GEMM_EPI_WARPS * 32 * GEMM_STG_LD * 4;
+  static constexpr int STG_BYTES = TMA_OUT ? GEMM_EPI_WARPS * 2 * BW_TMA_BOX_BYTES
+                                           : GEMM_EPI_WARPS * 32 * GEMM_STG_LD * 4;
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
   static constexpr int SMEM_BYTES =
       1024 + STAGES * (A_BYTES + B_BYTES) + STG_BYTES + BAR_BYTES + 16;
@@ -125,9 +129,9 @@ struct BwLayout {
 template <int BN, int STAGES, bool B_MN, class Epi>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 k_gemm_bw(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const __grid_constant__ CUtensorMap tmB64, const BwSource src, const Epi epi, int* err,
-          unsigned long long limit_ns) {
-  using L = BwLayout<BN, STAGES, B_MN>;
+          const __grid_constant__ CUtensorMap tmB64, const BwSource src,
+          const __grid_constant__ Epi epi, int* err, unsigned long long limit_ns) {
+  using L = BwLayout<BN, STAGES, B_MN, Epi::kTma>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -328,8 +332,13 @@ k_gemm_bw(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     // gets it through fetch(): the four loads of a 32-row chunk are issued
     // together, one chunk ahead (the first before the accumulator wait), so
     // their latency overlaps the TMEM reads and the stores of the chunk before.
+    // An fp32 epilogue with Epi::kTma writes each 32-row chunk as one 32 x 32
+    // box through a TMA store (two boxes per warp in flight), so the stores
+    // bypass the load/store path.
     const int q = warp & 3;                  // TMEM lane quarter of this warp
-    float* my = stg + (warp - 2) * 32 * GEMM_STG_LD;
+    float* my = Epi::kTma ? stg + (warp - 2) * 2 * (BW_TMA_BOX_BYTES / 4)
+                          : stg + (warp - 2) * 32 * GEMM_STG_LD;
+    int nbox = 0;                            // TMA boxes this warp has issued
     int acc = 0;
     uint32_t acc_phase = 0;
     auto fetch_chunk = [&](const BwTile& t, int c0, uint4 (&aux)[4]) {
@@ -361,6 +370,29 @@ k_gemm_bw(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = 0u;   // no rows: zero gradient
         }
+        if constexpr (Epi::kTma) {
+          // rows and features come in whole chunks of 32 (both extents are
+          // multiples of 32), so a chunk is either stored or skipped whole
+          if (feat_base < src.m_valid) {
+            float* box = my + (nbox & 1) * (BW_TMA_BOX_BYTES / 4);
+            // the box stored two chunks ago has been read out of this buffer
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) box[j * 32 + lane] = __uint_as_float(r[j]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const CUtensorMap* map;
+              int x, y;
+              epi.target(t, static_cast<long>(t.row0 + c0), feat_base, &map, &x, &y);
+              tma_store_2d(map, box, x, y);
+              bulk_commit_group();
+            }
+            ++nbox;
+          }
+          continue;
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) my[j * GEMM_STG_LD + lane] = __uint_as_float(r[j]);
         __syncwarp();
@@ -380,7 +412,7 @@ k_gemm_bw(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
           if constexpr (Epi::kAux)
             epi.store8(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid, aux[it]);
-          else
+          else if constexpr (!Epi::kTma)
             epi.store8(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid);
         }
         __syncwarp();
@@ -394,6 +426,10 @@ k_gemm_bw(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         acc_phase ^= 1;
       }
     }
+    // the shared memory of the last boxes stays until the stores have read it
+    if constexpr (Epi::kTma)
+      if (lane == 0) bulk_wait_group_read<0>();
+    __syncwarp();
   }
 
   tc_fence_before();

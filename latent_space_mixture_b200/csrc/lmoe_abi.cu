@@ -255,6 +255,7 @@ struct EpiO16 {
 // columns [N+l, N+l+h_s) of dxh.
 struct EpiDVH {
   static constexpr bool kAux = true;   // reads hs
+  static constexpr bool kTma = false;
   bf16* dv;
   bf16* dxh;
   const bf16* vh;
@@ -285,6 +286,7 @@ struct EpiDVH {
 // plain bf16 store of the product (du rows in expert order; dx)
 struct EpiStore {
   static constexpr bool kAux = false;
+  static constexpr bool kTma = false;
   bf16* out;
   int ld;
   __device__ __forceinline__ void store8(const BwTile&, long row, int feat, const float* v,
@@ -293,49 +295,64 @@ struct EpiStore {
   }
 };
 
-__device__ __forceinline__ void store8_f32(float* dst, const float* v) {
-  float4* q = reinterpret_cast<float4*>(dst);
-  q[0] = make_float4(v[0], v[1], v[2], v[3]);
-  q[1] = make_float4(v[4], v[5], v[6], v[7]);
-}
+// Weight gradients (fp32) leave through TMA stores of 32 x 32 boxes: target()
+// names the tensor map and the box coordinates of the chunk of 32 dW rows
+// starting at `row` and the 32 features starting at `feat`.
 
-// d[W_r; W_dn; W_s1] = dxh^T x: rows [0, r1) to p0, [r1, r2) to p1, the rest
-// to p2 (fp32, row pitch ld)
+// d[W_r; W_dn; W_s1] = dxh^T x: rows [0, r1) to m0, [r1, r2) to m1, the rest
+// to m2 (maps of [rows][d] fp32; r1, r2 multiples of 32)
 struct EpiWRows {
   static constexpr bool kAux = false;
-  float *p0, *p1, *p2;
-  int r1, r2, ld;
-  __device__ __forceinline__ void store8(const BwTile&, long row, int feat, const float* v,
-                                         bool valid) const {
-    if (!valid) return;
-    float* dst = row < r1 ? p0 + row * ld : row < r2 ? p1 + (row - r1) * ld : p2 + (row - r2) * ld;
-    store8_f32(dst + feat, v);
+  static constexpr bool kTma = true;
+  CUtensorMap m0, m1, m2;
+  int r1, r2;
+  __device__ __forceinline__ void target(const BwTile&, long row, int feat, const CUtensorMap** m,
+                                         int* x, int* y) const {
+    *x = feat;
+    if (row < r1) {
+      *m = &m0;
+      *y = static_cast<int>(row);
+    } else if (row < r2) {
+      *m = &m1;
+      *y = static_cast<int>(row - r1);
+    } else {
+      *m = &m2;
+      *y = static_cast<int>(row - r2);
+    }
   }
 };
 
-// d[W_upl | W_s2] = dy^T [v | hs]: columns [0, c1) to p0 (pitch ld0), the
-// rest to p1 (pitch ld1)
+// d[W_upl | W_s2] = dy^T [v | hs]: features [0, c1) to m0 ([d][l]), the rest
+// to m1 ([d][h_s]); c1 a multiple of 32
 struct EpiWCols {
   static constexpr bool kAux = false;
-  float *p0, *p1;
-  int c1, ld0, ld1;
-  __device__ __forceinline__ void store8(const BwTile&, long row, int feat, const float* v,
-                                         bool valid) const {
-    if (!valid) return;
-    if (feat < c1) store8_f32(p0 + row * ld0 + feat, v);
-    else store8_f32(p1 + row * ld1 + (feat - c1), v);
+  static constexpr bool kTma = true;
+  CUtensorMap m0, m1;
+  int c1;
+  __device__ __forceinline__ void target(const BwTile&, long row, int feat, const CUtensorMap** m,
+                                         int* x, int* y) const {
+    *y = static_cast<int>(row);
+    if (feat < c1) {
+      *m = &m0;
+      *x = feat;
+    } else {
+      *m = &m1;
+      *x = feat - c1;
+    }
   }
 };
 
-// per-expert weight gradient dW[e] (fp32, [rows][ld], experts estride apart)
+// per-expert weight gradient dW[e] ([E * rows_per][cols] fp32)
 struct EpiWExp {
   static constexpr bool kAux = false;
-  float* p;
-  long estride;
-  int ld;
-  __device__ __forceinline__ void store8(const BwTile& t, long row, int feat, const float* v,
-                                         bool valid) const {
-    if (valid) store8_f32(p + t.e * estride + row * ld + feat, v);
+  static constexpr bool kTma = true;
+  CUtensorMap m;
+  int rows_per;
+  __device__ __forceinline__ void target(const BwTile& t, long row, int feat, const CUtensorMap** mp,
+                                         int* x, int* y) const {
+    *mp = &m;
+    *x = feat;
+    *y = t.e * rows_per + static_cast<int>(row);
   }
 };
 
@@ -349,7 +366,7 @@ cudaError_t set_bw_smem() {
   constexpr int S = BwStages<BN>::value;
   return cudaFuncSetAttribute(k_gemm_bw<BN, S, B_MN, Epi>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              BwLayout<BN, S, B_MN>::SMEM_BYTES);
+                              BwLayout<BN, S, B_MN, Epi::kTma>::SMEM_BYTES);
 }
 
 template <int BN, bool B_MN, class Epi>
@@ -358,7 +375,8 @@ cudaError_t launch_bw(const CUtensorMap& A, const CUtensorMap& B16, const CUtens
                       unsigned long long limit, cudaStream_t st) {
   constexpr int S = BwStages<BN>::value;
   return launch_pdl(k_gemm_bw<BN, S, B_MN, Epi>, grid, GEMM_THREADS,
-                    BwLayout<BN, S, B_MN>::SMEM_BYTES, st, A, B16, B64, src, epi, err, limit);
+                    BwLayout<BN, S, B_MN, Epi::kTma>::SMEM_BYTES, st, A, B16, B64, src, epi, err,
+                    limit);
 }
 
 // data-gradient GEMM with a K-major token-row B operand of BN rows per block
@@ -565,6 +583,21 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D fp32 row-major [rows][cols] matrix written by TMA stores of 32 x 32
+// boxes, no swizzle (cols * 4 a multiple of 16 bytes); out-of-range elements
+// of a box are not written.
+static bool make_map_f32_out(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1420,7 +1453,10 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
     const int fb = (l + hs + 127) / 128, nbk = static_cast<int>((d + 255) / 256);
     BwSource s{1, 0, static_cast<int>(T), nullptr, nullptr, 0, 0, fb, l + hs, l + hs,
                1, nullptr, nbk, static_cast<int>(d), static_cast<int>(d)};
-    EpiWCols epi{gr->d_upl, gr->d_s2, l, l, hs};
+    EpiWCols epi{};
+    if (!make_map_f32_out(&epi.m0, gr->d_upl, d, l) || !make_map_f32_out(&epi.m1, gr->d_s2, d, hs))
+      return LMOE_ERR_CUDA;
+    epi.c1 = l;
     LMOE_BW(7, (launch_bw<256, true>(h->tm_vh.b64, tm_dy.b64, tm_dy.b64, s, epi,
                                   grid_of(int64_t(fb) * nbk), h->err, lim, st)));
   }
@@ -1428,7 +1464,9 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
   {
     const int fb = (hh + 127) / 128, nbk = (l + 255) / 256;
     BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, hh, hh, N, h->offsets, nbk, l, l};
-    EpiWExp epi{gr->d_w2, int64_t(l) * hh, hh};
+    EpiWExp epi{};
+    if (!make_map_f32_out(&epi.m, gr->d_w2, int64_t(N) * l, hh)) return LMOE_ERR_CUDA;
+    epi.rows_per = l;
     LMOE_BW(8, (launch_bw<256, true>(h->tm_H.b64, h->tm_dog.b64, h->tm_dog.b64, s, epi,
                                   grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
   }
@@ -1436,7 +1474,9 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
   {
     const int fb = (l + 127) / 128, nbk = (hh + 255) / 256;
     BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, l, l, N, h->offsets, nbk, hh, hh};
-    EpiWExp epi{gr->d_w1, int64_t(hh) * l, l};
+    EpiWExp epi{};
+    if (!make_map_f32_out(&epi.m, gr->d_w1, int64_t(N) * hh, l)) return LMOE_ERR_CUDA;
+    epi.rows_per = hh;
     LMOE_BW(9, (launch_bw<256, true>(h->tm_uperm.b64, h->tm_da.b64, h->tm_da.b64, s, epi,
                                   grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
   }
@@ -1445,7 +1485,12 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
     const int fb = static_cast<int>((d + 127) / 128), nbk = (ldx + 255) / 256;
     BwSource s{1, 0, static_cast<int>(T), nullptr, nullptr, 0, 0, fb, static_cast<int>(d),
                static_cast<int>(d), 1, nullptr, nbk, ldx, ldx};
-    EpiWRows epi{gr->d_router, gr->d_dn, gr->d_s1, N, N + l, static_cast<int>(d)};
+    EpiWRows epi{};
+    if (!make_map_f32_out(&epi.m0, gr->d_router, N, d) ||
+        !make_map_f32_out(&epi.m1, gr->d_dn, l, d) || !make_map_f32_out(&epi.m2, gr->d_s1, hs, d))
+      return LMOE_ERR_CUDA;
+    epi.r1 = N;
+    epi.r2 = N + l;
     LMOE_BW(10, (launch_bw<256, true>(tm_x.b64, h->tm_dxh.b64, h->tm_dxh.b64, s, epi,
                                   grid_of(int64_t(fb) * nbk), h->err, lim, st)));
   }
