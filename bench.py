@@ -294,6 +294,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the training step: forward, backward and the router-bias update")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -306,6 +308,9 @@ def main():
         if rank != 0:
             return 0
         return run_reference(args, cfg, world)
+
+    if args.backward:
+        return run_training(args, cfg, world, rank, local_rank)
 
     from datetime import timedelta
     torch.cuda.set_device(local_rank)
@@ -434,6 +439,194 @@ def main():
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clocks.summary(t_wall0, t_wall1),
             "quantisation_error": quant_err,
+            "wall_s_timed_region": round(t_wall1 - t_wall0, 4),
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+TRAIN_METRIC = "LatentMoE layer training step (forward + backward + bias update) tokens/s at 1 B200"
+
+
+def backward_work(cfg, T: int, counts: np.ndarray):
+    """Algorithmic flops and bytes of each backward contraction.  Data
+    gradients read the weights (dense ones and the touched experts') and the
+    token rows and write the gradient rows; weight gradients read the saved
+    activations and the output gradients and write fp32 gradients of every
+    weight (all N experts' dW1, dW2)."""
+    d, l, N, K, h, hs = cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs
+    R = T * K
+    touched = int((counts > 0).sum())
+    wexp = touched * h * l * 2
+    return {
+        "bw dgrad [W_upl|W_s2]^T (dv, dhs)": dict(flops=2 * T * d * (l + hs),
+                                                  bytes=d * (l + hs) * 2 + T * d * 2 + T * (l + 2 * hs) * 2),
+        "bw dgrad W2^T (dg)": dict(flops=2 * R * l * h, bytes=wexp + R * l * 2 + R * h * 2),
+        "bw dgrad W1^T (du rows)": dict(flops=2 * R * h * l, bytes=wexp + R * h * 2 + R * l * 2),
+        "bw dgrad [W_r;W_dn;W_s1]^T (dx)": dict(flops=2 * T * d * (N + l + hs),
+                                                bytes=(N + l + hs) * d * 2 + T * (N + l + hs) * 2
+                                                + T * d * 2),
+        "bw wgrad [W_upl|W_s2]": dict(flops=2 * T * d * (l + hs),
+                                      bytes=d * (l + hs) * 4 + T * (d + l + hs) * 2),
+        "bw wgrad W2": dict(flops=2 * R * l * h, bytes=N * l * h * 4 + R * (l + h) * 2),
+        "bw wgrad W1": dict(flops=2 * R * h * l, bytes=N * h * l * 4 + R * (l + h) * 2),
+        "bw wgrad [W_r;W_dn;W_s1]": dict(flops=2 * T * d * (N + l + hs),
+                                         bytes=(N + l + hs) * d * 4 + T * (N + l + hs + d) * 2),
+    }
+
+
+def oracle_train_rate(cfg, w, x, dy, seconds: float, seed: int):
+    """Tokens/s of the float64 oracle's forward + backward on a bounded
+    sample of the batch, one token at a time (its expert gradients are
+    22 dense matrices per token)."""
+    from oracle import backward as OB
+
+    def to64(t):
+        return t.detach().to("cpu").to(torch.float64).numpy()
+
+    dense = {k: to64(w[k]) for k in ("w_router", "router_bias", "w_dn", "w_upl", "w_s1", "w_s2")}
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(x.shape[0])
+    done, t0 = 0, time.perf_counter()
+    while done < len(order):
+        t = int(order[done])
+        OB.layer_backward(to64(x[t:t + 1]), dense["w_router"], dense["router_bias"], dense["w_dn"],
+                          lambda e: to64(w["w1"][e]), lambda e: to64(w["w2"][e]), dense["w_upl"],
+                          dense["w_s1"], dense["w_s2"], cfg.K, to64(dy[t:t + 1]))
+        done += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count()
+    return done / el, done, el, cores
+
+
+def run_training(args, cfg, world, rank, local_rank):
+    """--backward: one step is lmoe_forward, lmoe_backward and
+    lmoe_bias_update on a synthetic batch and upstream gradient (BF16 experts
+    with latent projections)."""
+    from datetime import timedelta
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    from latent_space_mixture_b200 import LatentMoE
+    from lmoe_synth import make_grad_out
+    if cfg.fmt != "bf16" or not cfg.proj:
+        raise SystemExit("--backward needs a BF16 workload with latent projections")
+    dev = torch.device("cuda", local_rank)
+    w, _ = make_weights(cfg, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(shard_seed(cfg.seed, rank))
+    x = make_x(cfg, gen, device=dev)
+    T = cfg.T
+    dy = make_grad_out(cfg, T=T, device=dev, seed=shard_seed(cfg.seed + 1000, rank))
+    layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, backward=True)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    grads = layer.grad_buffers()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(x, out=y)
+        layer.backward(x, dy, grads, dx=dx)
+        layer.bias_update(1e-3)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if layer.sync_status() != 0:
+        raise RuntimeError("device status after warm-up")
+    clocks = ClockSampler(local_rank).start()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    _, total_ms = timed_region(step, args.steps, lambda: cuda_timer(stream), between=flush.zero_)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    clocks.stop()
+    layer.profile_enable(True)
+    layer.profile_read(reset=True)
+    timed_region(step, args.steps, lambda: cuda_timer(stream), between=flush.zero_)
+    prof = layer.profile_read(reset=True)
+    layer.profile_enable(False)
+    if layer.sync_status() != 0:
+        raise RuntimeError("device status after the timed steps")
+    ms_per_step = total_ms / args.steps
+    value = throughput(world, T, args.steps, total_ms)
+    counts = layer.debug("counts").numpy()
+    lay, fwd_kernels = algorithmic_work(cfg, T, counts)
+    bwd_kernels = backward_work(cfg, T, counts)
+    peaks, peak_kind = load_peaks()
+    prof_by = {n: (ms, c) for n, ms, c in prof if c > 0}
+    dom = max((n for n in bwd_kernels if n in prof_by), key=lambda n: prof_by[n][0])
+    roof = roofline_entry(dom, bwd_kernels[dom], prof_by[dom][0], prof_by[dom][1], peaks,
+                          peak_kind, cfg, T)
+    roof["traffic"] = None
+    total_prof = max(sum(v[0] for v in prof_by.values()), 1e-9)
+    kernels = {n: {"ms_total": round(ms, 3), "launches": c, "share": round(ms / total_prof, 4)}
+               for n, (ms, c) in prof_by.items()}
+    step_flops = lay["flops"] + sum(v["flops"] for v in bwd_kernels.values())
+    step_roof = {"alg_flops": step_flops,
+                 "tflops": round(step_flops / (ms_per_step / 1e3) / 1e12, 2),
+                 "tensor_frac": round(step_flops / (ms_per_step / 1e3) / 1e12
+                                      / peaks["bf16_tflops"], 4)}
+
+    e2e = None
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory()
+        dyh = dy.cpu().pin_memory()
+        dxh = torch.empty_like(xh).pin_memory()
+        xd = torch.empty_like(x)
+        dyd = torch.empty_like(dy)
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            dyd.copy_(dyh, non_blocking=True)
+            layer.forward(xd, out=y)
+            layer.backward(xd, dyd, grads, dx=dx)
+            layer.bias_update(1e-3)
+            dxh.copy_(dx, non_blocking=True)
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        _, e2e_ms = timed_region(e2e_step, args.steps, lambda: cuda_timer(stream),
+                                 between=flush.zero_)
+        e2e = {"value": round(throughput(world, T, args.steps, e2e_ms), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int((xh.numel() + dyh.numel()) * 2),
+               "d2h_bytes_per_step": int(dxh.numel() * 2),
+               "ms_per_step": round(e2e_ms / args.steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, el, cores = oracle_train_rate(cfg, w, x, dy, args.cpu_seconds, 1000 + cfg.seed)
+        cpu = {"value": round(rate, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} of the {T} tokens (forward + backward, one at a time), {el:.1f} s"}
+    launches = (layer.launches_per_forward(T) + 12 + 1) * args.steps
+    if rank == 0:
+        line = {
+            "metric": TRAIN_METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 (fp32 accumulation, fp32 weight gradients)",
+            "data": "synthetic (seeded; weights N(0, std) bf16, x and dL/dy N(0,1) bf16)",
+            "config": {"workload": cfg.name, "T": T, "d": cfg.d, "latent": cfg.l,
+                       "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
+                       "shared_hidden": cfg.hs, "router_bias": cfg.bias,
+                       "tokens_per_rank": T, "parallelism": f"dp{world} (replicated weights)",
+                       "l2": "256 MiB write between steps, outside the per-step events"},
+            "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
+            "kernels_note": "per-kernel CUDA events from a second pass of the same steps",
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clocks.summary(t_wall0, t_wall1),
             "wall_s_timed_region": round(t_wall1 - t_wall0, 4),
         }
         print(json.dumps(line), flush=True)
