@@ -110,7 +110,7 @@ __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int t
   return t;
 }
 
-template <int BN, int STAGES, int KIND>
+template <int BN, int STAGES, int KIND, int EPIW = GEMM_EPI_WARPS>
 struct GemmLayout {
   static constexpr bool FP4 = KIND == KIND_NVFP4;
   static constexpr bool W4 = KIND == KIND_W4A16;
@@ -125,8 +125,12 @@ struct GemmLayout {
   static constexpr int SF_BYTES = FP4 ? 2 * FP4_SF_STAGE_BYTES : 0;
   // W4A16: the stage's FP4 codes (128 rows x 32 B per sub-tile) and A scale atoms
   static constexpr int RAW_BYTES = W4 ? KS * (W4_CODE_BYTES + SF_ATOM_BYTES) : 0;
-  static constexpr int THREADS = GEMM_THREADS + (W4 ? W4_CONV_THREADS : 0);   // + converters
-  static constexpr int STG_BYTES = GEMM_EPI_WARPS * 32 * GEMM_STG_LD * 4;
+  // epilogue warps: 4, or several per TMEM lane quarter (each takes every
+  // (EPI_WARPS / 4)-th 32-column chunk), chosen per epilogue (GemmEpiWarps)
+  static constexpr int EPI_WARPS = EPIW;
+  static_assert(EPIW % 4 == 0 && EPIW >= 4 && EPIW <= 16, "epilogue warps per lane quarter");
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS + (W4 ? W4_CONV_THREADS : 0);   // + converters
+  static constexpr int STG_BYTES = EPI_WARPS * 32 * GEMM_STG_LD * 4;
   static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8;
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ +
                                     STAGES * (A_BYTES + B_BYTES + SF_BYTES + RAW_BYTES) +
@@ -148,6 +152,30 @@ struct GemmLayout {
   static constexpr bool PAIRED_RELEASE = STAGES % 2 == 0 && !W4;
 };
 
+// Epilogue warps of a GEMM variant: Epi::kWarps for token blocks of 128 rows
+// or more, where the epilogue of a tile can take several times its main loop
+// (quantising H to NVFP4 costs ~9x the tile's FP4 MMAs); 4 for the narrow
+// decode blocks, whose shared memory goes to the ring.
+template <int BN, class Epi>
+struct GemmEpiWarps {
+  static constexpr int value = BN >= 128 ? Epi::kWarps : GEMM_EPI_WARPS;
+};
+
+// Ring depth: `want` stages, or as many as fit in shared memory beside the
+// epilogue staging.
+template <int BN, int KIND, int EPIW>
+constexpr int gemm_fit_stages(int want) {
+  int s = want;
+  while (s > 2 && GemmLayout<BN, 2, KIND, EPIW>::SMEM_BYTES +
+                          (s - 2) * (GemmLayout<BN, 2, KIND, EPIW>::A_BYTES +
+                                     GemmLayout<BN, 2, KIND, EPIW>::B_BYTES +
+                                     GemmLayout<BN, 2, KIND, EPIW>::SF_BYTES +
+                                     GemmLayout<BN, 2, KIND, EPIW>::RAW_BYTES + 24) >
+                      232448)
+    --s;
+  return s;
+}
+
 // "empty" barrier of ring slot s, and whether the producer waits on it there
 template <class L>
 __device__ __forceinline__ int empty_slot(int s) { return L::PAIRED_RELEASE ? s >> 1 : s; }
@@ -157,11 +185,11 @@ template <class L>
 __device__ __forceinline__ bool empty_commits_at(int s) { return !L::PAIRED_RELEASE || (s & 1); }
 
 template <int BN, int STAGES, class Epi, int KIND>
-__global__ void __launch_bounds__(GemmLayout<BN, STAGES, KIND>::THREADS, 1)
+__global__ void __launch_bounds__(GemmLayout<BN, STAGES, KIND, GemmEpiWarps<BN, Epi>::value>::THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmB64, const TileSource src, const Epi epi, int* err,
           unsigned long long limit_ns) {
-  using L = GemmLayout<BN, STAGES, KIND>;
+  using L = GemmLayout<BN, STAGES, KIND, GemmEpiWarps<BN, Epi>::value>;
   constexpr bool FP4 = KIND == KIND_NVFP4;
   constexpr bool F8 = KIND == KIND_FP8;
   constexpr bool W4 = KIND == KIND_W4A16;
@@ -193,7 +221,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], GEMM_EPI_WARPS * 32);
+      mbar_init(&tempty[a], L::EPI_WARPS * 32);
     }
     mbar_init(drain, 1);
     if constexpr (W4)
@@ -420,10 +448,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       }
     }
     __syncwarp();
-  } else if (warp < 2 + GEMM_EPI_WARPS) {
+  } else if (warp < 2 + L::EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter of this warp
-    float* my = stg + (warp - 2) * 32 * GEMM_STG_LD;
+    const int ew = warp - 2;                 // epilogue warp index
+    const int cstep = 32 * (L::EPI_WARPS / 4);   // column chunks: this warp's, then every cstep
+    const int cfirst = 32 * (ew / 4);
+    float* my = stg + ew * 32 * GEMM_STG_LD;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -434,7 +465,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
       const int feat_base = t.fb * GEMM_BM + q * 32;
-      for (int c0 = 0; c0 < t.nrows; c0 += 32) {
+      for (int c0 = cfirst; c0 < t.nrows; c0 += cstep) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c0, r);
         tmem_ld_wait();
@@ -476,14 +507,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   }
 
   if constexpr (W4) {
-    if (warp >= 2 + GEMM_EPI_WARPS) {
+    if (warp >= 2 + L::EPI_WARPS) {
       // ---------------------------------------------------------- converters
       // One thread per row of the 128-row weight tile and K sub-tile: its 64
       // E2M1 codes times the E4M3 scales of their 16-blocks, as f16 (the
       // product of an E2M1 and an E4M3 value is exact in f16), written in
       // the 128-byte-swizzled K-major layout the MMA reads; the per-expert
       // global scale is applied in the epilogue.
-      const int ct = threadIdx.x - (2 + GEMM_EPI_WARPS) * 32;
+      const int ct = threadIdx.x - (2 + L::EPI_WARPS) * 32;
       const int r = ct >> 1, q = ct & 1;   // row, and K sub-tile of the stage
       static_assert(W4_CONV_THREADS == 128 * W4_KSUB, "a converter thread per row and sub-tile");
       int stage = 0;

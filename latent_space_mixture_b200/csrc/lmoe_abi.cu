@@ -30,6 +30,7 @@ namespace lmoe {
 // Features [0, N) are logits, [N, N+lu) u and the rest the shared hidden;
 // lu = 0 for the standard MoE (no W_dn rows, u = x).
 struct EpiX {
+  static constexpr int kWarps = 4;
   float* logits;
   bf16* u;
   bf16* vh;
@@ -77,6 +78,7 @@ struct EpiX {
 
 // expert FC1: H[row] = sqrelu(W1[e] u[row])
 struct EpiH {
+  static constexpr int kWarps = 4;
   bf16* H;
   int h;
   __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
@@ -91,6 +93,7 @@ struct EpiH {
 
 // expert FC2 times the router weight of the row: O[row] = w[row] W2[e] H[row]
 struct EpiO {
+  static constexpr int kWarps = 4;
   bf16* O;
   const float* wrow;
   int l;
@@ -109,6 +112,7 @@ struct EpiO {
 // Standard MoE (no W_upl): the GEMM is W_s2 hs and the epilogue adds v
 // (resid, row pitch ldr) before the store.
 struct EpiY {
+  static constexpr int kWarps = 4;
   bf16* y;
   int d;
   const bf16* resid;
@@ -137,6 +141,8 @@ struct EpiY {
 // global scale g_h into codes [R][hp/2] and the B-operand scale atoms of the
 // second grouped GEMM ([token block][hp/64][512 B], row = index in the block).
 struct EpiHq {
+  // epilogue warps at >= 128-row token blocks: quantising H is ~9x the FP4 MMAs
+  static constexpr int kWarps = 16;
   uint8_t* Hq;
   uint8_t* sfh;
   const float* gw1;
@@ -160,6 +166,8 @@ struct EpiHq {
 
 // NVFP4 expert FC2 times the router weight: O = w g_W2[e] g_h * acc (bf16)
 struct EpiOq {
+  // epilogue warps at >= 128-row token blocks
+  static constexpr int kWarps = 8;
   bf16* O;
   const float* wrow;
   const float* gw2;
@@ -178,6 +186,8 @@ struct EpiOq {
 
 // FP8 expert FC1: H = E4M3(sqrelu(s_W1[e] s_u * acc) / s_h), codes [R][h]
 struct EpiH8 {
+  // epilogue warps at >= 128-row token blocks
+  static constexpr int kWarps = 8;
   uint8_t* H8;
   const float* sw1;
   float s_u, r_h;
@@ -195,6 +205,8 @@ struct EpiH8 {
 
 // FP8 expert FC2: O = w * s_W2[e] s_h * acc
 struct EpiO8 {
+  // epilogue warps at >= 128-row token blocks
+  static constexpr int kWarps = 8;
   bf16* O;
   const float* wrow;
   const float* sw2;
@@ -214,6 +226,7 @@ struct EpiO8 {
 // W4A16 expert FC1: H = sqrelu(g_W1[e] * acc) in f16 (the MMA summed the
 // FP4 codes times their block scales; the global scale comes here)
 struct EpiH16 {
+  static constexpr int kWarps = 4;
   __half* H16;
   const float* gw1;
   int h;
@@ -230,6 +243,7 @@ struct EpiH16 {
 
 // W4A16 expert FC2: O = w * g_W2[e] * acc
 struct EpiO16 {
+  static constexpr int kWarps = 4;
   bf16* O;
   const float* wrow;
   const float* gw2;
@@ -426,11 +440,20 @@ struct Stages<32, KIND_W4A16> {
   static constexpr int value = 4;
 };
 
+// the ring depth of a variant: its default, or what fits beside the staging
+// of a wider epilogue
+template <int BN, class Epi, int KIND>
+struct StagesOf {
+  static constexpr int EPIW = GemmEpiWarps<BN, Epi>::value;
+  static constexpr int value = gemm_fit_stages<BN, KIND, EPIW>(Stages<BN, KIND>::value);
+  using L = GemmLayout<BN, value, KIND, EPIW>;
+};
+
 template <int BN, class Epi, int KIND = KIND_BF16>
 cudaError_t set_gemm_smem() {
-  using L = GemmLayout<BN, Stages<BN, KIND>::value, KIND>;
-  return cudaFuncSetAttribute(k_gemm_tc<BN, Stages<BN, KIND>::value, Epi, KIND>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
+  using S = StagesOf<BN, Epi, KIND>;
+  return cudaFuncSetAttribute(k_gemm_tc<BN, S::value, Epi, KIND>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::L::SMEM_BYTES);
 }
 
 // B operand: the same matrix under two tensor maps (16-row and 64-row boxes)
@@ -442,9 +465,9 @@ template <int BN, class Epi, int KIND = KIND_BF16>
 cudaError_t launch_gemm(const CUtensorMap& A, const BMaps& B, const TileSource& src,
                         const Epi& epi, int grid, int* err, unsigned long long limit,
                         cudaStream_t st) {
-  using L = GemmLayout<BN, Stages<BN, KIND>::value, KIND>;
-  return launch_pdl(k_gemm_tc<BN, Stages<BN, KIND>::value, Epi, KIND>, grid, L::THREADS,
-                    L::SMEM_BYTES, st, A, B.b16, B.b64, src, epi, err, limit);
+  using S = StagesOf<BN, Epi, KIND>;
+  return launch_pdl(k_gemm_tc<BN, S::value, Epi, KIND>, grid, S::L::THREADS, S::L::SMEM_BYTES, st,
+                    A, B.b16, B.b64, src, epi, err, limit);
 }
 
 // CTA-pair variant: 256 x 256 tiles, 3 stages of K = 128 (64 KB per CTA)
