@@ -295,6 +295,29 @@ int lmoe_route_noalloc(const float* logits, const float* bias, int64_t T, int32_
 int lmoe_nvfp4_quantize(const float* x, int64_t rows, int32_t cols, float g, uint8_t* codes,
                         uint8_t* scales, void* stream);
 
+/* Gradient-path pieces of the NVFP4 training recipe ("Nemotron-3 Super
+ * 精读报告", section 5.3: a random Hadamard transform on the weight-gradient
+ * GEMMs' inputs, stochastic rounding of gradients).  Random bits come from
+ * SplitMix64 (Steele, Lea, Flood, OOPSLA 2014) as a counter-based generator:
+ * counter i of `seed` gives mix(seed + (i + 1) * 0x9E3779B97F4A7C15).
+ *
+ * lmoe_rht16: y = (1/4) H16 diag(s) x on every 16 consecutive elements of
+ * the fp32 rows x [rows][cols] (cols a multiple of 16), H16 the 16 x 16
+ * Sylvester Hadamard matrix and s the 16 signs of counters 0..15 (-1 where
+ * bit 63 is set), shared by all blocks; float32 butterflies (stages 1, 2, 4,
+ * 8: (a, b) -> (a + b, a - b)), then x 0.25.  Orthonormal and its own inverse
+ * up to the signs.  x and y device, 16-byte aligned; y may equal x.
+ *
+ * lmoe_nvfp4_quantize_sr: as lmoe_nvfp4_quantize (same block scales), but
+ * each element v = f32(x * r) rounds to the upper of its two E2M1 grid
+ * neighbours with probability (|v| - lo) / (hi - lo), decided by the
+ * uniform (top 24 bits x 2^-24) of counter row * cols + col: unbiased in
+ * expectation.  Asynchronous on `stream`.  Errors: INVALID_ARG, CUDA. */
+int lmoe_rht16(const float* x, int64_t rows, int32_t cols, uint64_t seed, float* y,
+               void* stream);
+int lmoe_nvfp4_quantize_sr(const float* x, int64_t rows, int32_t cols, float g, uint64_t seed,
+                           uint8_t* codes, uint8_t* scales, void* stream);
+
 /* Runs a one-CTA kernel that waits on an mbarrier nothing arrives on, with a
  * wait limit of limit_ns nanoseconds (1e3..1e10), and returns the status the
  * host reads afterwards: LMOE_ERR_TIMEOUT when the bounded wait gave up as

@@ -12,6 +12,8 @@ loads the library first and raises when it has not been built (there is no
 other implementation to fall back to).
 """
 from ._lib import LmoeError
-from .layer import LatentMoE, lmoe_check_bounded_wait, lmoe_route
+from .layer import (LatentMoE, lmoe_check_bounded_wait, lmoe_nvfp4_quantize_sr, lmoe_rht16,
+                    lmoe_route)
 
-__all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]
+__all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError", "lmoe_rht16",
+           "lmoe_nvfp4_quantize_sr"]

@@ -4,6 +4,7 @@ from __future__ import annotations
 import ctypes
 import os
 from ctypes import (POINTER, Structure, c_char_p, c_double, c_float, c_int, c_int32, c_int64,
+                    c_uint64,
                     c_size_t, c_void_p)
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +72,9 @@ SIGNATURES = {
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "lmoe_nvfp4_quantize": (c_int, [c_void_p, c_int64, c_int32, c_float, c_void_p, c_void_p,
                                     c_void_p]),
+    "lmoe_rht16": (c_int, [c_void_p, c_int64, c_int32, c_uint64, c_void_p, c_void_p]),
+    "lmoe_nvfp4_quantize_sr": (c_int, [c_void_p, c_int64, c_int32, c_float, c_uint64, c_void_p,
+                                       c_void_p, c_void_p]),
     "lmoe_check_bounded_wait": (c_int, [c_int64]),
     "lmoe_destroy": (None, [c_void_p]),
     "lmoe_strerror": (c_char_p, [c_int]),

@@ -53,6 +53,13 @@ cudaError_t launch_quant_w8(const void* w, int E, int rows_per, int K, float* am
 // fp32 rows -> codes [rows][cols/2], scales [rows][cols/16] (canonical layout).
 cudaError_t launch_quant_rows(const float* x, int64_t rows, int cols, float g, uint8_t* codes,
                               uint8_t* scales, cudaStream_t st);
+// Gradient-path pieces of the NVFP4 training recipe: the random Hadamard
+// transform (1/4) H16 diag(s) on every 16-element block of fp32 rows, and
+// NVFP4 rows with stochastically rounded elements (SplitMix64 counters).
+cudaError_t launch_rht16(const float* x, int64_t rows, int cols, uint64_t seed, float* y,
+                         cudaStream_t st);
+cudaError_t launch_quant_rows_sr(const float* x, int64_t rows, int cols, float g, uint64_t seed,
+                                 uint8_t* codes, uint8_t* scales, cudaStream_t st);
 // quantised u rows into expert order plus their scales into block atoms.
 cudaError_t launch_gather_q(const uint8_t* uq, const uint8_t* usf, const int32_t* perm,
                             const int32_t* rblock, int64_t rows, int K, int l, int lp,

@@ -1721,6 +1721,31 @@ int lmoe_nvfp4_quantize(const float* x, int64_t rows, int32_t cols, float g, uin
              : LMOE_ERR_CUDA;
 }
 
+int lmoe_rht16(const float* x, int64_t rows, int32_t cols, uint64_t seed, float* y,
+               void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 16) return LMOE_ERR_INVALID_ARG;
+  if (rows == 0) return LMOE_OK;
+  if (!x || !y || ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15))
+    return LMOE_ERR_INVALID_ARG;
+  return launch_rht16(x, rows, cols, seed, y, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LMOE_OK
+             : LMOE_ERR_CUDA;
+}
+
+int lmoe_nvfp4_quantize_sr(const float* x, int64_t rows, int32_t cols, float g, uint64_t seed,
+                           uint8_t* codes, uint8_t* scales, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 16 || !(g >= 0.0f && g < 3.0e38f))
+    return LMOE_ERR_INVALID_ARG;
+  if (rows == 0) return LMOE_OK;
+  if (!x || !codes || !scales || (reinterpret_cast<uintptr_t>(x) & 15) ||
+      (reinterpret_cast<uintptr_t>(codes) & 7))
+    return LMOE_ERR_INVALID_ARG;
+  return launch_quant_rows_sr(x, rows, cols, g, seed, codes, scales,
+                              static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LMOE_OK
+             : LMOE_ERR_CUDA;
+}
+
 int lmoe_check_bounded_wait(int64_t limit_ns) {
   if (limit_ns < 1000 || limit_ns > 10000000000ll) return LMOE_ERR_INVALID_ARG;
   int* err = nullptr;

@@ -243,6 +243,146 @@ cudaError_t launch_quant_rows(const float* x, int64_t rows, int cols, float g, u
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Gradient-path pieces of the NVFP4 training recipe ("Nemotron-3 Super 精读报告",
+// section 5.3: a random Hadamard transform on the inputs of the weight-gradient
+// GEMMs, stochastic rounding of gradient tensors; section 9.3: stochastic
+// rounding is unbiased in expectation).
+//
+// Random bits: SplitMix64 (Steele, Lea, Flood, "Fast splittable pseudorandom
+// number generators", OOPSLA 2014) used as a counter-based generator: counter
+// i gives mix(seed + (i + 1) * 0x9E3779B97F4A7C15).  Element (row, col) of a
+// [rows][cols] tensor takes counter row * cols + col; the transform's signs
+// take counters 0..15 (sign -1 when bit 63 is set); a uniform in [0, 1) is
+// the top 24 bits times 2^-24.
+
+__device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t ctr) {
+  uint64_t z = seed + (ctr + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ float uniform24(uint64_t seed, uint64_t ctr) {
+  return static_cast<float>(static_cast<uint32_t>(splitmix64(seed, ctr) >> 40)) *
+         5.9604644775390625e-8f;   // 2^-24
+}
+
+// Stochastic rounding of v to an E2M1 code (bit 3 = sign): the upper grid
+// neighbour with probability (|v| - lo) / (hi - lo), the lower otherwise;
+// |v| >= 6 saturates.  The probability is exact in float32 (hi - lo is a
+// power of two, |v| - lo is exact).
+__device__ __forceinline__ uint32_t e2m1_sr(float v, float u) {
+  const float mag = fabsf(v);
+  uint32_t code;
+  if (mag >= 6.0f) {
+    code = 7;
+  } else {
+    const int lo = mag < 0.5f ? 0 : mag < 1.0f ? 1 : mag < 1.5f ? 2 : mag < 2.0f ? 3
+                 : mag < 3.0f ? 4 : mag < 4.0f ? 5 : 6;
+    const float lo_v = e2m1_value(static_cast<uint32_t>(lo));
+    const float hi_v = e2m1_value(static_cast<uint32_t>(lo + 1));
+    const float p = __fdiv_rn(__fsub_rn(mag, lo_v), __fsub_rn(hi_v, lo_v));
+    code = static_cast<uint32_t>(u < p ? lo + 1 : lo);
+  }
+  return code | (signbit(v) ? 8u : 0u);
+}
+
+// One thread per 16-element block: y = (1/4) H16 (s * x) as float32
+// butterflies (stages 1, 2, 4, 8: (a, b) -> (a + b, a - b)).
+__global__ void __launch_bounds__(256) k_rht16(const float* __restrict__ x, int64_t nblocks,
+                                               uint64_t seed, float* __restrict__ y) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= nblocks) return;
+  float b[16];
+  const float4* src = reinterpret_cast<const float4*>(x + i * 16);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float4 f = src[j];
+    b[4 * j] = f.x;
+    b[4 * j + 1] = f.y;
+    b[4 * j + 2] = f.z;
+    b[4 * j + 3] = f.w;
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    if (splitmix64(seed, static_cast<uint64_t>(j)) >> 63) b[j] = -b[j];
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j & h) continue;
+      const float a = b[j], c = b[j + h];
+      b[j] = __fadd_rn(a, c);
+      b[j + h] = __fsub_rn(a, c);
+    }
+  }
+  float4* dst = reinterpret_cast<float4*>(y + i * 16);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    dst[j] = make_float4(b[4 * j] * 0.25f, b[4 * j + 1] * 0.25f, b[4 * j + 2] * 0.25f,
+                         b[4 * j + 3] * 0.25f);
+}
+
+cudaError_t launch_rht16(const float* x, int64_t rows, int cols, uint64_t seed, float* y,
+                         cudaStream_t st) {
+  const int64_t n = rows * (cols / 16);
+  if (n <= 0) return cudaSuccess;
+  k_rht16<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(x, n, seed, y);
+  return cudaGetLastError();
+}
+
+// NVFP4 rows with stochastically rounded elements: the block scale of the
+// round-to-nearest quantiser (nvfp4_block's arithmetic), then e2m1_sr of
+// f32(x * r) with the uniform of the element's counter.
+__global__ void __launch_bounds__(256) k_quant_rows_sr(const float* __restrict__ x, int64_t rows,
+                                                       int cols, float g, uint64_t seed,
+                                                       uint8_t* __restrict__ codes,
+                                                       uint8_t* __restrict__ scales) {
+  const int nb = cols / 16;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * nb) return;
+  const int64_t row = i / nb;
+  const int blk = static_cast<int>(i - row * nb);
+  float v[16];
+  const float4* src = reinterpret_cast<const float4*>(x + row * cols + blk * 16);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float4 f = src[j];
+    v[4 * j] = f.x;
+    v[4 * j + 1] = f.y;
+    v[4 * j + 2] = f.z;
+    v[4 * j + 3] = f.w;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  const float six_g = __fmul_rn(6.0f, g);
+  const float sbf = six_g > 0.0f ? __fdiv_rn(amax, six_g) : 0.0f;
+  const uint8_t sc = e4m3_code(sbf);
+  const float denom = __fmul_rn(e4m3_value(sc), g);
+  const float r = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+  const uint64_t c0 = static_cast<uint64_t>(row) * cols + blk * 16;
+  uint8_t q[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t lo = e2m1_sr(__fmul_rn(v[2 * j], r), uniform24(seed, c0 + 2 * j));
+    const uint32_t hi = e2m1_sr(__fmul_rn(v[2 * j + 1], r), uniform24(seed, c0 + 2 * j + 1));
+    q[j] = static_cast<uint8_t>(lo | (hi << 4));
+  }
+  scales[row * nb + blk] = sc;
+  *reinterpret_cast<uint2*>(codes + row * (cols / 2) + blk * 8) = *reinterpret_cast<const uint2*>(q);
+}
+
+cudaError_t launch_quant_rows_sr(const float* x, int64_t rows, int cols, float g, uint64_t seed,
+                                 uint8_t* codes, uint8_t* scales, cudaStream_t st) {
+  const int64_t n = rows * (cols / 16);
+  if (n <= 0) return cudaSuccess;
+  k_quant_rows_sr<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(x, rows, cols, g, seed,
+                                                                           codes, scales);
+  return cudaGetLastError();
+}
+
 // Quantised latent rows into expert order: codes u_q[tok] -> u_perm_q[r]
 // (row pitch Kp/2 bytes) and the row's scales [tok][l/16] into the B-operand
 // atoms of its token block: atom (block, kc), row j of the block.

@@ -14,7 +14,8 @@ from ._lib import (DBG, FLAG_BACKWARD, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8, FM
                    FMT_W4A16, NVFP4_WEIGHT_FLAGS,
                    LmoeConfig, LmoeError, LmoeGrads, LmoeWeights, check)
 
-__all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError"]
+__all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError", "lmoe_rht16",
+           "lmoe_nvfp4_quantize_sr"]
 
 _WEIGHT_SHAPES = {
     "w_router": ("N", "d"), "w_dn": ("l", "d"), "w1": ("N", "h", "l"), "w2": ("N", "l", "h"),
@@ -237,6 +238,39 @@ def lmoe_route(logits: torch.Tensor, bias: Optional[torch.Tensor], K: int,
                          p(ws), ws.numel(), _stream_ptr(stream)), "lmoe_route")
     out["_workspace"] = ws
     return out
+
+
+def lmoe_rht16(x: torch.Tensor, seed: int, out: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """lmoe_rht16: random Hadamard transform of 16-element blocks of fp32
+    CUDA rows [rows][cols] (async)."""
+    if x.dtype != torch.float32 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x: need CUDA fp32 [rows][cols]")
+    x = x.contiguous()
+    if out is None:
+        out = torch.empty_like(x)
+    check(_lib.load().lmoe_rht16(c_void_p(x.data_ptr()), x.shape[0], x.shape[1], int(seed),
+                                 c_void_p(out.data_ptr()), _stream_ptr(stream)), "lmoe_rht16")
+    return out
+
+
+def lmoe_nvfp4_quantize_sr(x: torch.Tensor, g: float, seed: int,
+                           stream: Optional[torch.cuda.Stream] = None):
+    """lmoe_nvfp4_quantize_sr: NVFP4 codes [rows][cols/2] and E4M3 block
+    scales [rows][cols/16] of fp32 CUDA rows, elements stochastically rounded
+    (async)."""
+    if x.dtype != torch.float32 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x: need CUDA fp32 [rows][cols]")
+    x = x.contiguous()
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
+    check(_lib.load().lmoe_nvfp4_quantize_sr(c_void_p(x.data_ptr()), rows, cols,
+                                             ctypes.c_float(g), int(seed),
+                                             c_void_p(codes.data_ptr()),
+                                             c_void_p(scales.data_ptr()), _stream_ptr(stream)),
+          "lmoe_nvfp4_quantize_sr")
+    return codes, scales
 
 
 def lmoe_check_bounded_wait(limit_ns: int) -> int:
