@@ -8,7 +8,8 @@
 // token per column.  This keeps ragged per-expert token counts cheap: an
 // expert with 11 routed rows costs an N=16 MMA, not a 128-row tile.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over a static tile list):
+// Warp roles (64 + 32 x epilogue-warp threads, one CTA per SM, persistent
+// over a static tile list):
 //   warp 0      TMA producer: A tile and B rows (64- and 16-row boxes) per
 //               k-step, 128-byte swizzle, completion on a "full" mbarrier;
 //               in the NVFP4 variant also the two scale-factor tiles (bulk
@@ -19,7 +20,10 @@
 //               (kind::f8f6f4, E4M3);
 //               tcgen05.commit frees the smem stage, and at the end of a tile
 //               marks the accumulator full;
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, transpose through a
+//   warps 2..   epilogue (4 warps, or 8 / 16 where the epilogue outlasts the
+//               main loop: GemmEpiWarps): tcgen05.ld 32 columns at a time
+//               (warp w reads TMEM lanes 32 (w % 4)..; several warps per lane
+//               quarter take alternate 32-column chunks), transpose through a
 //               per-warp smem tile, call the epilogue functor on 8 consecutive
 //               features of one token row (all lanes call it; `valid` tells
 //               which carry data), release the accumulator.
