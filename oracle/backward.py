@@ -64,7 +64,8 @@ def layer_backward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     Returns dx [T][d], dW_r [N][d], dW_dn [l][d], dW_upl [d][l], dW_s1
     [h_s][d], dW_s2 [d][h_s] (dW_dn, dW_upl None for the standard MoE), and
     dW1, dW2: dicts expert -> [h][l], [l][h] over the experts some token
-    selected (the others have zero gradient), plus S, w, dw [T][K] (dL/dw).
+    selected (the others have zero gradient), plus S, w, dw [T][K] (dL/dw),
+    dz [T][N] (dL/dz), and du, dv [T][l] (dL/du, dL/dv).
     """
     x = np.atleast_2d(np.asarray(x, dtype=np.float64))
     G = np.atleast_2d(np.asarray(G, dtype=np.float64))
@@ -125,7 +126,7 @@ def layer_backward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     dx += dz @ W_r
     return {"dx": dx, "dW_r": dW_r, "dW_dn": dW_dn, "dW1": dW1, "dW2": dW2,
             "dW_upl": dW_upl, "dW_s1": dW_s1, "dW_s2": dW_s2, "S": S, "w": w,
-            "dw": dw, "dz": dz}
+            "dw": dw, "dz": dz, "du": du, "dv": dv}
 
 
 def bias_update(bias: np.ndarray, counts: np.ndarray,
