@@ -1,5 +1,7 @@
 /*
- * lmoe.h -- C ABI of the B200 (sm_100a) LatentMoE layer forward pass.
+ * lmoe.h -- C ABI of the B200 (sm_100a) LatentMoE layer: forward pass, its
+ * backward pass (lmoe_backward) with the aux-loss-free router-bias update,
+ * and the NVFP4 gradient-path pieces (lmoe_rht16, lmoe_nvfp4_quantize_sr).
  *
  * The layer ("NVIDIA Nemotron 3: Efficient and Open Intelligence", xllm-io
  * paper review, section 三 "LatentMoE 架构" with eq.(1); "Nemotron-3 Super
