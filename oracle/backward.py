@@ -40,7 +40,7 @@ from typing import Callable, Dict, Optional
 
 import numpy as np
 
-from .lmoe import route, sigmoid, sqrelu
+from .lmoe import route, sqrelu
 
 __all__ = ["layer_backward", "bias_update", "BIAS_UPDATE_RATE"]
 

@@ -33,7 +33,7 @@ import pytest
 import torch
 
 from oracle import backward as B
-from tests._parity import elem_ok, make, max_rel, rms_rel, to64
+from tests._parity import elem_ok, make, max_rel, to64
 
 pytestmark = pytest.mark.gpu
 

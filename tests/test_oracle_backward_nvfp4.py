@@ -8,7 +8,6 @@ import numpy as np
 
 from oracle import backward as B
 from oracle import backward_nvfp4 as BN
-from oracle import lmoe as O
 
 
 def _problem(seed, T=20, d=32, l=32, N=6, K=2, h=48, hs=16):
