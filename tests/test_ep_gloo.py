@@ -69,6 +69,90 @@ def _worker(rank, world, port, q, seed, bias_scale):
         dist.destroy_process_group()
 
 
+def _bw_worker(rank, world, port, q, seed):
+    """Forward and backward with expert parallelism: the output-gradient rows
+    take the forward's plan to the experts' owners (dispatch), the latent
+    input gradients come back by combine; each rank keeps its experts'
+    weight gradients."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from latent_space_mixture_b200 import ep
+        from oracle import lmoe as O
+        p, N, K = _layer(seed)
+        T = p["x"].shape[0]
+        G = np.random.default_rng(seed + 7).standard_normal((T, p["x"].shape[1]))
+        mine = np.arange(T)[rank::world]
+        x = p["x"][mine]
+        S, w, _, _ = O.route(x @ p["W_r"].T, p["b"], K)
+        counts, offsets, perm, inv = O.segments(S, N)
+        tok, slot = perm // K, perm % K
+        u = x @ p["W_dn"].T
+        pl = ep.plan(torch.from_numpy(counts))
+        u_loc = ep.dispatch(torch.from_numpy(u[tok]), pl).numpy()
+        lo, _ = ep.expert_range(N, world, rank)
+        seg = np.concatenate([[0], np.cumsum(pl.local_counts.numpy())])
+        o_loc = np.zeros_like(u_loc)
+        for j in range(N // world):
+            r = slice(seg[j], seg[j + 1])
+            o_loc[r] = O.expert_ffn(u_loc[r], p["W1"][lo + j], p["W2"][lo + j])
+        o = ep.combine(torch.from_numpy(o_loc), pl).numpy()      # sender's expert order
+        # backward: dv at this rank, the expert-side gradients at the owners
+        dv = G[mine] @ p["W_upl"]
+        do = w[tok, slot][:, None] * dv[tok]
+        do_loc = ep.dispatch(torch.from_numpy(do), pl).numpy()
+        du_loc = np.zeros_like(u_loc)
+        dW1, dW2 = {}, {}
+        for j in range(N // world):
+            e, r = lo + j, slice(seg[j], seg[j + 1])
+            a = u_loc[r] @ p["W1"][e].T
+            g = O.sqrelu(a)
+            dW2[e] = do_loc[r].T @ g
+            da = (do_loc[r] @ p["W2"][e]) * 2.0 * np.maximum(a, 0.0)
+            dW1[e] = da.T @ u_loc[r]
+            du_loc[r] = da @ p["W1"][e]
+        du_rows = ep.combine(torch.from_numpy(du_loc), pl).numpy()
+        du = np.zeros_like(u)
+        np.add.at(du, tok, du_rows)
+        dw = np.zeros((len(mine), K))
+        dw[tok, slot] = np.sum(dv[tok] * o, axis=1)
+        q.put((rank, mine, du, dw, dW1, dW2))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ep_backward_matches_single_process():
+    from oracle import backward as B
+    world, seed = 2, 5
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bw_worker, args=(r, world, port, q, seed))
+             for r in range(world)]
+    for pr in procs:
+        pr.start()
+    res = sorted((q.get(timeout=180) for _ in range(world)), key=lambda r: r[0])
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    p, N, K = _layer(seed)
+    G = np.random.default_rng(seed + 7).standard_normal((p["x"].shape[0], p["x"].shape[1]))
+    ref = B.layer_backward(p["x"], p["W_r"], p["b"], p["W_dn"], lambda e: p["W1"][e],
+                           lambda e: p["W2"][e], p["W_upl"], p["W_s1"], p["W_s2"], K, G)
+    seen = set()
+    for rank, mine, du, dw, dW1, dW2 in res:
+        np.testing.assert_allclose(du, ref["du"][mine], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dw, ref["dw"][mine], rtol=0, atol=1e-12)
+        for e in dW1:
+            if e in ref["dW1"]:
+                np.testing.assert_allclose(dW1[e], ref["dW1"][e], rtol=0, atol=1e-12)
+                np.testing.assert_allclose(dW2[e], ref["dW2"][e], rtol=0, atol=1e-12)
+            else:
+                assert not dW1[e].any() and not dW2[e].any()
+            seen.add(e)
+    assert seen == set(range(N))
+
+
 def _run(world, seed, bias_scale=0.0):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
