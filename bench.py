@@ -638,22 +638,31 @@ def run_training(args, cfg, world, rank, local_rank):
 
 def run_reference(args, cfg, world):
     """The oracle as the reference arm: each step is the oracle on a bounded
-    sample of the workload's tokens (rank 0 only)."""
+    sample of the workload's tokens (rank 0 only); with --backward, its
+    forward + backward."""
     from oracle import lmoe as O  # noqa: F401  (fail early if missing)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     w, gen = make_weights(cfg, device=dev)
     x = make_x(cfg, gen, device=dev)
     per_step = max(1.0, 150.0 / max(args.steps + args.warmup, 1))
+    if args.backward:
+        # the training step's reference: the oracle's forward + backward
+        from lmoe_synth import make_grad_out
+        dy = make_grad_out(cfg, device=dev)
+        rate_fn = lambda sec, seed: oracle_train_rate(cfg, w, x, dy, sec, seed)  # noqa: E731
+    else:
+        rate_fn = lambda sec, seed: oracle_rate(cfg, w, x, sec, seed)  # noqa: E731
     for _ in range(args.warmup):
-        oracle_rate(cfg, w, x, per_step / 4, 7)
+        rate_fn(per_step / 4, 7)
     rates, n_tot, el_tot, cores = [], 0, 0.0, 1
     for i in range(args.steps):
-        r, n, el, cores = oracle_rate(cfg, w, x, per_step, 1000 + i)
+        r, n, el, cores = rate_fn(per_step, 1000 + i)
         rates.append(r)
         n_tot += n
         el_tot += el
     value = n_tot / el_tot
-    line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+    line = {"metric": TRAIN_METRIC if args.backward else METRIC, "value": round(value, 3),
+            "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * el_tot / args.steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
