@@ -12,6 +12,11 @@ its own token batch (seed + rank) against replicated weights: no collective on
 the data path, weak scaling; the timed region is bracketed by barriers and the
 reported time is the max over ranks.
 
+At N = 1 the line also carries `workloads`: the Super-dims prefill layer
+(T=8192, Zipf router bias), the same with NVFP4 experts, and the Ultra-dims
+layer (T=4096), each timed the same way (fewer steps) with its own layer
+roofline, dominant-kernel roofline and clock record.
+
 --impl reference times the CPU float64 oracle (the only other implementation
 of the layer) on a bounded token sample of the same workload, on rank 0.
 """
@@ -243,6 +248,16 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(inside)}
 
 
+def workload_config(cfg, world: int) -> dict:
+    """The `config` object of a bench line: the same for both arms."""
+    return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "latent": cfg.l,
+            "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
+            "shared_hidden": cfg.hs, "router_bias": cfg.bias, "expert_format": cfg.fmt,
+            "latent_projections": cfg.proj, "tokens_per_rank": cfg.T,
+            "parallelism": f"dp{world} (replicated weights)",
+            "l2": "256 MiB write between steps, outside the per-step events"}
+
+
 # ---------------------------------------------------------------------------
 # the CPU oracle leg
 
@@ -293,6 +308,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time the headline workload only (no extra workloads)")
+    ap.add_argument("--workload-steps", type=int, default=20,
+                    help="timed steps of each extra workload (at most --steps)")
     ap.add_argument("--backward", action="store_true",
                     help="time the training step: forward, backward and the router-bias update")
     args = ap.parse_args()
@@ -310,40 +329,38 @@ def main():
 
     if args.backward:
         return run_training(args, cfg, world, rank, local_rank)
+    return run_forward(args, cfg, world, rank, local_rank)
 
-    from datetime import timedelta
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local_rank))
+
+# Workloads measured beside the headline in the default run (N = 1): the
+# other layer sizes and formats the throughput targets name.
+EXTRA_WORKLOADS = ("super_prefill", "super_prefill_nvfp4", "ultra")
+
+
+def make_layer(cfg, T, w):
     from latent_space_mixture_b200 import LatentMoE
-
-    dev = torch.device("cuda", local_rank)
-    w, _ = make_weights(cfg, device=dev)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(shard_seed(cfg.seed, rank))
-    x = make_x(cfg, gen, device=dev)
-    T = cfg.T
     from lmoe_synth import act_global_scales
-    layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, expert_format=cfg.fmt,
-                      act_gscales=act_global_scales(cfg) if cfg.fmt != "bf16" else (0.0, 0.0),
-                      projections=cfg.proj, nvfp4_weights=cfg.wq)
-    y = torch.empty_like(x)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
-    stream = torch.cuda.current_stream()
+    return LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, expert_format=cfg.fmt,
+                     act_gscales=act_global_scales(cfg) if cfg.fmt != "bf16" else (0.0, 0.0),
+                     projections=cfg.proj, nvfp4_weights=cfg.wq)
 
-    for _ in range(args.warmup):
+
+def time_forward(layer, x, y, steps, warmup, flush, stream, local_rank):
+    """Warm-up, the timed steps (CUDA events per step, L2 flushed between
+    them outside the events, clocks sampled meanwhile), then a second pass of
+    the same steps with per-kernel events.  Returns (max-over-ranks total ms,
+    clock summary, wall seconds of the timed region, per-kernel profile)."""
+    for _ in range(warmup):
         layer.forward(x, out=y)
     torch.cuda.synchronize()
     rc = layer.sync_status()
     if rc != 0:
         raise RuntimeError(f"device status {rc} after warm-up")
-
     clocks = ClockSampler(local_rank).start()
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
-    step_ms, total_ms = timed_region(lambda: layer.forward(x, out=y), args.steps,
-                                     lambda: cuda_timer(stream), between=flush.zero_)
+    _, total_ms = timed_region(lambda: layer.forward(x, out=y), steps,
+                               lambda: cuda_timer(stream), between=flush.zero_)
     torch.cuda.synchronize()
     t_wall1 = time.perf_counter()
     clocks.stop()
@@ -352,17 +369,19 @@ def main():
     # so this pass is not the headline number)
     layer.profile_enable(True)
     layer.profile_read(reset=True)
-    timed_region(lambda: layer.forward(x, out=y), args.steps, lambda: cuda_timer(stream),
+    timed_region(lambda: layer.forward(x, out=y), steps, lambda: cuda_timer(stream),
                  between=flush.zero_)
     prof = layer.profile_read(reset=True)
     layer.profile_enable(False)
     rc = layer.sync_status()
     if rc != 0:
         raise RuntimeError(f"device status {rc} after the timed steps")
-    ms_per_step = total_ms / args.steps
-    value = throughput(world, T, args.steps, total_ms)
+    return total_ms, clocks.summary(t_wall0, t_wall1), t_wall1 - t_wall0, prof
 
-    counts = layer.debug("counts").numpy()
+
+def forward_rooflines(cfg, T, counts, prof, ms_per_step):
+    """The dominant kernel's roofline object, the layer's roofline fractions
+    and the per-kernel table of one measured workload."""
     lay, per_kernel = algorithmic_work(cfg, T, counts)
     peaks, peak_kind = load_peaks()
     prof_by = {n: (ms, c) for n, ms, c in prof}
@@ -379,7 +398,66 @@ def main():
                   # time roofline: each contraction at its own dtype's peak
                   "tensor_frac": round(lay["bf16_equiv_flops"] / layer_time_s / 1e12
                                        / peaks["bf16_tflops"], 4),
-                  "tflops": round(lay["flops"] / layer_time_s / 1e12, 2)}
+                  "tflops": round(lay["flops"] / layer_time_s / 1e12, 2),
+                  "peaks": f"{peak_kind}: HBM {peaks['hbm_gbs']} GB/s, "
+                           f"BF16 {peaks['bf16_tflops']} TFLOP/s (burst)"}
+    return roof, layer_roof, kernels
+
+
+def measure_workload(name, args, local_rank, rank, flush, stream):
+    """One extra workload on this GPU: its own weights, batch and layer,
+    freed before returning."""
+    cfg = CONFIGS[name]
+    dev = torch.device("cuda", local_rank)
+    w, _ = make_weights(cfg, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(shard_seed(cfg.seed, rank))
+    x = make_x(cfg, gen, device=dev)
+    layer = make_layer(cfg, cfg.T, w)
+    del w
+    y = torch.empty_like(x)
+    steps = max(1, min(args.steps, args.workload_steps))
+    total_ms, clk, wall, prof = time_forward(layer, x, y, steps, args.warmup, flush, stream,
+                                             local_rank)
+    ms = total_ms / steps
+    counts = layer.debug("counts").numpy()
+    roof, layer_roof, _ = forward_rooflines(cfg, cfg.T, counts, prof, ms)
+    out = {"ms_per_step": round(ms, 4), "value": round(throughput(1, cfg.T, steps, total_ms), 1),
+           "unit": "tokens/s", "steps": steps, "warmup": args.warmup,
+           "config": workload_config(cfg, 1), "layer_roofline": layer_roof, "roofline": roof,
+           "clocks": clk, "gpu_launches": layer.launches_per_forward(cfg.T) * steps,
+           "wall_s_timed_region": round(wall, 4)}
+    layer.close()
+    del x, y, layer
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_forward(args, cfg, world, rank, local_rank):
+    from datetime import timedelta
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    from latent_space_mixture_b200 import LatentMoE
+
+    dev = torch.device("cuda", local_rank)
+    w, _ = make_weights(cfg, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(shard_seed(cfg.seed, rank))
+    x = make_x(cfg, gen, device=dev)
+    T = cfg.T
+    layer = make_layer(cfg, T, w)
+    y = torch.empty_like(x)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
+    stream = torch.cuda.current_stream()
+
+    total_ms, clk, wall, prof = time_forward(layer, x, y, args.steps, args.warmup, flush, stream,
+                                             local_rank)
+    ms_per_step = total_ms / args.steps
+    value = throughput(world, T, args.steps, total_ms)
+    counts = layer.debug("counts").numpy()
+    roof, layer_roof, kernels = forward_rooflines(cfg, T, counts, prof, ms_per_step)
 
     # end to end through host buffers
     e2e = None
@@ -419,33 +497,42 @@ def main():
             quant_err["nvfp4_weights"] = cfg.wq
 
     launches = layer.launches_per_forward(T) * args.steps
+    layer.close()
+    del w, x, y, layer
+    torch.cuda.empty_cache()
+
+    # the other workloads of the throughput targets, one after another on
+    # this GPU (N = 1 only: the scaling runs time the headline alone)
+    workloads = None
+    if world == 1 and not args.no_workloads:
+        workloads = {n: measure_workload(n, args, local_rank, rank, flush, stream)
+                     for n in EXTRA_WORKLOADS if n != cfg.name}
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": {"bf16": "bf16", "nvfp4": "e2m1 experts, bf16 dense",
-                      "fp8": "e4m3 experts, bf16 dense",
-                      "w4a16": "e2m1 weights expanded to f16, f16 activations, bf16 dense"}[cfg.fmt],
+            "dtype": DTYPES[cfg.fmt],
             "data": "synthetic (seeded; weights N(0, std) bf16, x N(0,1) bf16)",
-            "config": {"workload": cfg.name, "T": T, "d": cfg.d, "latent": cfg.l,
-                       "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
-                       "shared_hidden": cfg.hs, "router_bias": cfg.bias,
-                       "latent_projections": cfg.proj, "tokens_per_rank": T, "parallelism": f"dp{world} (replicated weights)",
-                       "l2": "256 MiB write between steps, outside the per-step events"},
+            "config": workload_config(cfg, world),
             "roofline": roof, "layer_roofline": layer_roof, "kernels": kernels,
             "kernels_note": "per-kernel CUDA events from a second pass of the same steps",
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clocks.summary(t_wall0, t_wall1),
+            "clocks": clk,
             "quantisation_error": quant_err,
-            "wall_s_timed_region": round(t_wall1 - t_wall0, 4),
+            "wall_s_timed_region": round(wall, 4),
+            "workloads": workloads,
         }
         print(json.dumps(line), flush=True)
-    layer.close()
     if world > 1:
         barrier()
         torch.distributed.destroy_process_group()
     return 0
+
+
+DTYPES = {"bf16": "bf16", "nvfp4": "e2m1 experts, bf16 dense", "fp8": "e4m3 experts, bf16 dense",
+          "w4a16": "e2m1 weights expanded to f16, f16 activations, bf16 dense"}
 
 
 TRAIN_METRIC = "LatentMoE layer training step (forward + backward + bias update) tokens/s at 1 B200"
@@ -641,6 +728,9 @@ def run_reference(args, cfg, world):
     sample of the workload's tokens (rank 0 only); with --backward, its
     forward + backward."""
     from oracle import lmoe as O  # noqa: F401  (fail early if missing)
+    if args.backward and (cfg.fmt != "bf16" or not cfg.proj):
+        # the GPU arm's training step has the same restriction
+        raise SystemExit("--backward needs a BF16 workload with latent projections")
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     w, gen = make_weights(cfg, device=dev)
     x = make_x(cfg, gen, device=dev)
@@ -664,15 +754,18 @@ def run_reference(args, cfg, world):
     line = {"metric": TRAIN_METRIC if args.backward else METRIC, "value": round(value, 3),
             "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(1e3 * el_tot / args.steps, 2), "higher_is_better": True,
+            # a step is the whole workload (T tokens); each timed step ran a
+            # bounded sample of it, so this is the sample rate's time for T
+            "ms_per_step": round(1e3 * cfg.T / value, 2),
+            "sample_ms_per_step": round(1e3 * el_tot / args.steps, 2),
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "latent": cfg.l,
-                       "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,
-                       "shared_hidden": cfg.hs, "latent_projections": cfg.proj},
+            "config": workload_config(cfg, world),
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
                              "kind": "oracle",
-                             "sample": f"{n_tot} tokens over {args.steps} steps, {el_tot:.1f} s"},
+                             "sample": f"{n_tot} of the workload's {cfg.T} tokens over "
+                                       f"{args.steps} steps, {el_tot:.1f} s"},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

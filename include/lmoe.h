@@ -259,12 +259,22 @@ int lmoe_profile_read(lmoe_handle* h, const char** names, double* total_ms, int6
  * counts [N] int32, offsets [N+1] int32, perm [T*K] int32, inv [T][K] int32.
  * bias: [N] fp32 device or NULL.  workspace: device scratch of at least
  * lmoe_route_workspace_size(T, N) bytes, 256-byte aligned, caller-owned.
- * Asynchronous on `stream`.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+ * Asynchronous on `stream`.  Errors: INVALID_ARG, UNSUPPORTED, CUDA; a
+ * selected expert index outside [0, N) found by the segment kernels is
+ * recorded in the workspace (cleared at the start of each call) and read by
+ * lmoe_route_status. */
 size_t lmoe_route_workspace_size(int64_t T, int32_t N);
 int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int32_t K,
                int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
                int32_t* perm, int32_t* inv, void* workspace, size_t workspace_bytes,
                void* stream);
+
+/* Device status of the last lmoe_route call that used `workspace` with the
+ * same T and N: waits for `stream`, then returns DEVICE if that call's
+ * kernels flagged an expert index outside [0, N), else OK.  Reading does not
+ * clear the record (the next lmoe_route call on the workspace does).
+ * Errors: INVALID_ARG (null or misaligned workspace, T < 0, N <= 0), CUDA. */
+int lmoe_route_status(const void* workspace, int64_t T, int32_t N, void* stream);
 
 /* Allocation-free variant of lmoe_route (no counterpart on the pages: it is a
  * deployment convenience).  For callers that cannot give this library device
@@ -280,12 +290,20 @@ int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int
  * that device current); make that first call before any stream capture.
  * All calls share the one array, so calls whose work overlaps on the GPU
  * (other streams, other host threads) race: serialize them.
- * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA; a flagged expert index is recorded
+ * in the shared array and read by lmoe_route_noalloc_status. */
 #define LMOE_NOALLOC_MAX_TOKENS 8192
 #define LMOE_NOALLOC_MAX_ROUTED 262144
 int lmoe_route_noalloc(const float* logits, const float* bias, int64_t T, int32_t N, int32_t K,
                        int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
                        int32_t* perm, int32_t* inv, void* stream);
+
+/* Device status of the last lmoe_route_noalloc call on the current device:
+ * waits for `stream`, then returns DEVICE if that call's kernels flagged an
+ * expert index outside [0, N), else OK.  The next lmoe_route_noalloc call
+ * clears the record, so read it before making another call.  Allocates
+ * nothing.  Errors: UNSUPPORTED (device ordinal >= 256), CUDA. */
+int lmoe_route_noalloc_status(void* stream);
 
 /* NVFP4 quantisation of fp32 rows x [rows][cols] (device, 16-byte aligned,
  * cols a multiple of 16) with global scale g >= 0, exactly as the layer

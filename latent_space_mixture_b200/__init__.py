@@ -16,7 +16,7 @@ plans the expert-parallel exchange and moves rows with torch.distributed.
 from . import ep
 from ._lib import LmoeError
 from .layer import (LatentMoE, lmoe_check_bounded_wait, lmoe_nvfp4_quantize_sr, lmoe_rht16,
-                    lmoe_route)
+                    lmoe_route, lmoe_route_status)
 
-__all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError", "lmoe_rht16",
+__all__ = ["LatentMoE", "lmoe_route", "lmoe_route_status", "lmoe_check_bounded_wait", "LmoeError", "lmoe_rht16",
            "lmoe_nvfp4_quantize_sr", "ep"]

@@ -68,6 +68,8 @@ SIGNATURES = {
     "lmoe_route": (c_int, [c_void_p, c_void_p, c_int64, c_int32, c_int32, c_void_p, c_void_p,
                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                            c_void_p]),
+    "lmoe_route_status": (c_int, [c_void_p, c_int64, c_int32, c_void_p]),
+    "lmoe_route_noalloc_status": (c_int, [c_void_p]),
     "lmoe_route_noalloc": (c_int, [c_void_p, c_void_p, c_int64, c_int32, c_int32, c_void_p,
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "lmoe_nvfp4_quantize": (c_int, [c_void_p, c_int64, c_int32, c_float, c_void_p, c_void_p,

@@ -144,7 +144,9 @@ __global__ void __launch_bounds__(256) k_route_bw(const float* __restrict__ logi
   }
   __syncwarp();
   if (lane < K) {
-    const float dw = acc / w;
+    // w = 0 only when the selected score underflowed (s = 0); then dz = 0
+    // whatever dw is, so 0 stands in for the 0/0 quotient
+    const float dw = w > 0.0f ? acc / w : 0.0f;
     const float ds = (dw - m) / Z;
     row[e] = __float2bfloat16_rn(ds * s * (1.0f - s));
   }

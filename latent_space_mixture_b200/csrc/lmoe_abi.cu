@@ -1707,6 +1707,20 @@ int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int
   return LMOE_OK;
 }
 
+int lmoe_route_status(const void* workspace, int64_t T, int32_t N, void* stream) {
+  if (T < 0 || N <= 0 || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return LMOE_ERR_INVALID_ARG;
+  const int64_t C = (T + 31) / 32;
+  const int64_t rows = T * 32;
+  const char* ws = static_cast<const char*>(workspace) + align256(C * N * 4) +
+                   align256(rows * 4) + align256((rows / 32 + N + 1) * 16) + align256(4);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LMOE_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpy(&flag, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
+  return flag ? LMOE_ERR_DEVICE : LMOE_OK;
+}
+
 int lmoe_nvfp4_quantize(const float* x, int64_t rows, int32_t cols, float g, uint8_t* codes,
                         uint8_t* scales, void* stream) {
   if (rows < 0 || cols <= 0 || cols % 16 || !(g >= 0.0f && g < 3.0e38f))

@@ -61,6 +61,9 @@ static int scratch_on_current_device(void** out) {
   return LMOE_OK;
 }
 
+// the error word's byte offset inside the array
+constexpr size_t kErrOffset = kChunkBytes + kWrowBytes + kBlocksBytes + 256;
+
 extern "C" int lmoe_route_noalloc(const float* logits, const float* bias, int64_t T, int32_t N,
                                   int32_t K, int32_t* topk_idx, float* topk_w, int32_t* counts,
                                   int32_t* offsets, int32_t* perm, int32_t* inv, void* stream) {
@@ -78,7 +81,7 @@ extern "C" int lmoe_route_noalloc(const float* logits, const float* bias, int64_
   float* wrow = reinterpret_cast<float*>(s + kChunkBytes);
   int4* blocks = reinterpret_cast<int4*>(s + kChunkBytes + kWrowBytes);
   int32_t* nblocks = reinterpret_cast<int32_t*>(s + kChunkBytes + kWrowBytes + kBlocksBytes);
-  int* err = reinterpret_cast<int*>(s + kChunkBytes + kWrowBytes + kBlocksBytes + 256);
+  int* err = reinterpret_cast<int*>(s + kErrOffset);
   // the array keeps the previous call's contents: the error word starts at 0
   if (cudaMemsetAsync(err, 0, 4, st) != cudaSuccess) return LMOE_ERR_CUDA;
   if (T == 0) {
@@ -95,4 +98,17 @@ extern "C" int lmoe_route_noalloc(const float* logits, const float* bias, int64_
                            inv, wrow, blocks, nblocks, nullptr, err, st) != cudaSuccess)
     return LMOE_ERR_CUDA;
   return LMOE_OK;
+}
+
+extern "C" int lmoe_route_noalloc_status(void* stream) {
+  void* base = nullptr;
+  int rc = scratch_on_current_device(&base);
+  if (rc != LMOE_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpy(&flag, static_cast<char*>(base) + kErrOffset, 4, cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return LMOE_ERR_CUDA;
+  return flag ? LMOE_ERR_DEVICE : LMOE_OK;
 }

@@ -14,8 +14,8 @@ from ._lib import (DBG, FLAG_BACKWARD, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8, FM
                    FMT_W4A16, NVFP4_WEIGHT_FLAGS,
                    LmoeConfig, LmoeError, LmoeGrads, LmoeWeights, check)
 
-__all__ = ["LatentMoE", "lmoe_route", "lmoe_check_bounded_wait", "LmoeError", "lmoe_rht16",
-           "lmoe_nvfp4_quantize_sr"]
+__all__ = ["LatentMoE", "lmoe_route", "lmoe_route_status", "lmoe_check_bounded_wait",
+           "LmoeError", "lmoe_rht16", "lmoe_nvfp4_quantize_sr"]
 
 _WEIGHT_SHAPES = {
     "w_router": ("N", "d"), "w_dn": ("l", "d"), "w1": ("N", "h", "l"), "w2": ("N", "l", "h"),
@@ -238,6 +238,16 @@ def lmoe_route(logits: torch.Tensor, bias: Optional[torch.Tensor], K: int,
                          p(ws), ws.numel(), _stream_ptr(stream)), "lmoe_route")
     out["_workspace"] = ws
     return out
+
+
+def lmoe_route_status(route_out: Dict[str, torch.Tensor],
+                      stream: Optional[torch.cuda.Stream] = None) -> int:
+    """lmoe_route_status: waits for the stream and returns the device status
+    (0, or the DEVICE code) of the lmoe_route call that produced route_out."""
+    T, K = route_out["topk_idx"].shape
+    N = route_out["counts"].shape[0]
+    ws = route_out["_workspace"]
+    return _lib.load().lmoe_route_status(c_void_p(ws.data_ptr()), T, N, _stream_ptr(stream))
 
 
 def lmoe_rht16(x: torch.Tensor, seed: int, out: Optional[torch.Tensor] = None,

@@ -22,3 +22,33 @@ def test_weight_gradient_bytes_cover_fp32_outputs():
     bwd = bench.backward_work(cfg, cfg.T, np.ones(cfg.N, dtype=np.int64))
     assert bwd["bw wgrad W1"]["bytes"] >= cfg.N * cfg.h * cfg.l * 4
     assert bwd["bw wgrad W2"]["bytes"] >= cfg.N * cfg.h * cfg.l * 4
+
+
+def _reference_line(monkeypatch, capsys, name, backward=False):
+    import argparse
+    import json
+    monkeypatch.setattr(bench, "oracle_rate", lambda cfg, w, x, sec, seed: (4.0, 8, 2.0, 3))
+    monkeypatch.setattr(bench, "oracle_train_rate",
+                        lambda cfg, w, x, dy, sec, seed: (1.0, 2, 2.0, 3))
+    args = argparse.Namespace(steps=2, warmup=3, backward=backward)
+    bench.run_reference(args, CONFIGS[name], 1)
+    return json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+
+
+def test_reference_arm_reports_the_gpu_arms_config_and_a_full_step(monkeypatch, capsys):
+    """The reference line names the same config as the GPU line, and its
+    ms_per_step is the time of one whole step (T tokens) at its rate."""
+    cfg = CONFIGS["tiny"]
+    line = _reference_line(monkeypatch, capsys, "tiny")
+    assert line["config"] == bench.workload_config(cfg, 1)
+    assert line["impl"] == "reference"
+    assert line["value"] == 4.0
+    assert abs(line["ms_per_step"] - 1e3 * cfg.T / 4.0) < 1e-6
+
+
+def test_reference_training_arm_refuses_what_the_gpu_arm_refuses(monkeypatch, capsys):
+    import pytest
+    with pytest.raises(SystemExit):
+        _reference_line(monkeypatch, capsys, "tiny_std", backward=True)
+    with pytest.raises(SystemExit):
+        _reference_line(monkeypatch, capsys, "tiny_fp8", backward=True)

@@ -76,3 +76,18 @@ def test_random_logits_within_gap_window():
     assert clear.mean() > 0.9
     assert np.array_equal(np.sort(res["topk_idx"][clear], 1), np.sort(S[clear], 1))
     assert np.allclose(res["topk_w"].sum(1), 1.0, atol=1e-5)
+
+
+def test_route_status_reads_the_device_record():
+    """lmoe_route_status returns OK after a clean call and DEVICE when the
+    workspace's error record is set.  The record is the first word of the
+    workspace's last 256-byte slot; the test plants a value there on the
+    device, since a valid call cannot produce a bad expert index."""
+    from latent_space_mixture_b200 import lmoe_route, lmoe_route_status
+    T, N, K = 100, 64, 8
+    z = _separated_logits(T, N, 9).cuda()
+    out = lmoe_route(z, None, K)
+    assert lmoe_route_status(out) == 0
+    ws = out["_workspace"]
+    ws[ws.numel() - 256:ws.numel() - 252] = 1
+    assert lmoe_route_status(out) == -6

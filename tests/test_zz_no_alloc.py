@@ -57,6 +57,32 @@ def test_noalloc_route_matches_workspace_route_two_calls_in_a_row():
         for k in ("topk_idx", "counts", "offsets", "perm", "inv"):
             assert torch.equal(got[k], ref[k]), k
         assert torch.max(torch.abs(got["topk_w"] - ref["topk_w"])).item() <= W_TOL
+        assert lib.lmoe_route_noalloc_status(
+            c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+
+
+def test_noalloc_route_without_bias_and_with_no_tokens():
+    from latent_space_mixture_b200 import _lib, lmoe_route
+    lib = _lib.load()
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(12)
+    T, N, K = 777, 256, 16
+    logits = torch.randn((T, N), generator=g, device=dev)
+    ref = lmoe_route(logits, None, K)
+    torch.cuda.synchronize()
+    rc, got = _noalloc(lib, logits, None, K)
+    assert rc == 0
+    for k in ("topk_idx", "counts", "offsets", "perm", "inv"):
+        assert torch.equal(got[k], ref[k]), k
+    assert torch.max(torch.abs(got["topk_w"] - ref["topk_w"])).item() <= W_TOL
+    # T = 0: counts and offsets come back zero (the scratch holds the last call's data)
+    rc, got = _noalloc(lib, torch.zeros((0, N), device=dev), None, K)
+    assert rc == 0
+    assert torch.count_nonzero(got["counts"]).item() == 0
+    assert torch.count_nonzero(got["offsets"]).item() == 0
+    assert lib.lmoe_route_noalloc_status(
+        c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
 
 
 def test_noalloc_route_rejects_sizes_beyond_its_scratch():
