@@ -260,3 +260,145 @@ def test_mse_never_worse_than_max_based_and_keeps_grid_blocks():
     _, sc, _ = Q.quantize(blk[None, :], gg, mse=True)
     assert sc[0, 0] == 0x30
     assert np.array_equal(Q.fake_quant(blk[None, :], gg, mse=True)[0], blk.astype(np.float64))
+
+
+# ----------------------------------------------------------------------------
+# the NVFP4 expert layer: which tensors are quantised, along which axis, with
+# which global scale ("Nemotron-3 Super 精读报告", section 5.3: E2M1 elements in
+# 16-element micro-blocks along the GEMM reduction axis, E4M3 block scales, an
+# FP32 global scale; table 5.2: the latent projections stay BF16)
+
+def _torch_e4m3_value(v: np.float32) -> np.float32:
+    """E4M3 value of a non-negative float32 through torch's float8_e4m3fn cast,
+    saturating at 448 first (the cast itself has no saturation)."""
+    v = min(float(v), 448.0)
+    return _f32(torch.tensor([v], dtype=torch.float32).to(torch.float8_e4m3fn)
+                .to(torch.float32).item())
+
+
+def _restated_block_quant(vec, g) -> np.ndarray:
+    """Quantise-dequantise one vector in 16-element blocks along it, scalar
+    float32 steps: s = E4M3(amax / (6 g)), r = 1 / (s g) once per block,
+    q = nearest E2M1 of x r (ties to even), value q s g."""
+    g32 = _f32(g)
+    six_g = _f32(_f32(6.0) * g32)
+    out = []
+    for b0 in range(0, len(vec), 16):
+        blk = [_f32(v) for v in vec[b0:b0 + 16]]
+        amax = max(abs(float(v)) for v in blk)
+        s = _torch_e4m3_value(_f32(_f32(amax) / six_g)) if six_g > 0 else _f32(0.0)
+        denom = _f32(s * g32)
+        r = _f32(_f32(1.0) / denom) if denom > 0 else _f32(0.0)
+        for v in blk:
+            q = _e2m1_nearest(float(_f32(v * r)))
+            out.append(q * float(s) * float(g32))
+    return np.array(out)
+
+
+def _restated_weight_quant(W) -> np.ndarray:
+    """Each row of an expert matrix [out][in] in blocks along `in` (the GEMM
+    reduction axis), global scale amax(W) / (6 * 448) of that matrix."""
+    W32 = np.asarray(W, dtype=np.float32)
+    amax = max(abs(float(v)) for v in W32.reshape(-1))
+    g = _f32(_f32(amax) / _f32(2688.0))
+    return np.stack([_restated_block_quant(row, g) for row in W32])
+
+
+def _restated_nvfp4_layer(p, K, g_u, g_h):
+    """The NVFP4 expert layer with per-token loops: u quantised with g_u, W1[e]
+    and W2[e] with their own weight scales, sqrelu(W1 u) with g_h; the router,
+    projections and shared expert unquantised.  Uses no oracle quantiser."""
+    x = p["x"]
+    T = x.shape[0]
+    sig = 1.0 / (1.0 + np.exp(-(x @ p["W_r"].T)))
+    key = sig + p["b"]
+    y = np.maximum(x @ p["W_s1"].T, 0) ** 2 @ p["W_s2"].T
+    v_all = np.zeros((T, p["W_dn"].shape[0]))
+    for t in range(T):
+        top = sorted(range(len(key[t])), key=lambda e: (-key[t][e], e))[:K]
+        ws = sig[t, top] / sig[t, top].sum()
+        u = _restated_block_quant(p["W_dn"] @ x[t], g_u)
+        v = np.zeros_like(u)
+        for wk, e in zip(ws, top):
+            a = _restated_weight_quant(p["W1"][e]) @ u
+            hq = _restated_block_quant(np.maximum(a, 0) ** 2, g_h)
+            v += wk * (_restated_weight_quant(p["W2"][e]) @ hq)
+        v_all[t] = v
+        y[t] += p["W_upl"] @ v
+    return y, v_all
+
+
+def _small_nvfp4_layer():
+    rng = np.random.default_rng(45)
+    T, d, l, N, K, h, hs = 6, 32, 32, 6, 2, 48, 16     # l != h: the blocking axis shows
+    p = dict(x=rng.standard_normal((T, d)), W_r=rng.standard_normal((N, d)) * 0.3,
+             b=rng.standard_normal(N) * 0.05, W_dn=rng.standard_normal((l, d)) * 0.2,
+             W1=rng.standard_normal((N, h, l)) * 0.2, W2=rng.standard_normal((N, l, h)) * 0.2,
+             W_upl=rng.standard_normal((d, l)) * 0.2, W_s1=rng.standard_normal((hs, d)) * 0.2,
+             W_s2=rng.standard_normal((d, hs)) * 0.2)
+    for k in p:                      # weights and x as bf16 values, as the GPU sees them
+        p[k] = torch.from_numpy(p[k]).to(torch.bfloat16).to(torch.float64).numpy()
+    su = 0.2 * np.sqrt(d)
+    sa = 0.2 * np.sqrt(l) * su
+    # static scales, deliberately not power-of-two multiples of each other
+    return p, K, 8 * su / 2688 * 1.13, (8 * sa) ** 2 / 2688 * 0.71
+
+
+def _oracle_nvfp4(p, K, g_u, g_h):
+    from oracle import lmoe as O
+    return O.layer_forward(p["x"], p["W_r"], p["b"], p["W_dn"], lambda e: p["W1"][e],
+                           lambda e: p["W2"][e], p["W_upl"], p["W_s1"], p["W_s2"], K,
+                           quant={"g_u": g_u, "g_h": g_h})
+
+
+def test_nvfp4_layer_matches_loop_restatement():
+    p, K, g_u, g_h = _small_nvfp4_layer()
+    y_ref, v_ref = _restated_nvfp4_layer(p, K, g_u, g_h)
+    out = _oracle_nvfp4(p, K, g_u, g_h)
+    assert np.allclose(out["v"], v_ref, atol=1e-12, rtol=0)
+    assert np.allclose(out["y"], y_ref, atol=1e-12, rtol=0)
+    # the single-token path (used for near-tie tokens) quantises the same way
+    from oracle import lmoe as O
+    for t in (0, 5):
+        one = O.token_forward(p["x"][t], out["S"][t], out["s"][t], p["W_dn"],
+                              lambda e: p["W1"][e], lambda e: p["W2"][e], p["W_upl"],
+                              quant={"g_u": g_u, "g_h": g_h})
+        assert np.allclose(one["v"], v_ref[t], atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("mistake", ["none", "hidden_unquantised", "g_u_for_hidden",
+                                     "w2_blocked_along_latent", "one_scale_for_all_experts"])
+def test_nvfp4_restatement_catches_planted_mistakes(monkeypatch, mistake):
+    """Each plausible slip in the oracle's quantised composition, planted in
+    the oracle on the CPU, moves its output off the restatement ("none": the
+    same harness without a slip stays on it)."""
+    from oracle import lmoe as O
+    from oracle import nvfp4 as Qn
+    p, K, g_u, g_h = _small_nvfp4_layer()
+    y_ref, _ = _restated_nvfp4_layer(p, K, g_u, g_h)
+    l, h = p["W2"].shape[1], p["W2"].shape[2]
+    g_all = Qn.weight_global_scale(np.concatenate([p["W1"].reshape(-1), p["W2"].reshape(-1)]))
+
+    def q_w(W):
+        if mistake == "w2_blocked_along_latent" and W.shape == (l, h):
+            return Qn.fake_quant(W.T, Qn.weight_global_scale(W)).T
+        if mistake == "one_scale_for_all_experts":
+            return Qn.fake_quant(W, g_all)
+        return Qn.fake_quant(W, Qn.weight_global_scale(W))
+
+    def quantisers(quant):
+        q_u = lambda a: Qn.fake_quant(a, quant["g_u"])  # noqa: E731
+        if mistake == "hidden_unquantised":
+            q_h = lambda a: a  # noqa: E731
+        elif mistake == "g_u_for_hidden":
+            q_h = lambda a: Qn.fake_quant(a, quant["g_u"])  # noqa: E731
+        else:
+            q_h = lambda a: Qn.fake_quant(a, quant["g_h"])  # noqa: E731
+        return q_u, q_w, q_h
+
+    monkeypatch.setattr(O, "_expert_quantisers", quantisers)
+    out = _oracle_nvfp4(p, K, g_u, g_h)
+    if mistake == "none":
+        assert np.allclose(out["y"], y_ref, atol=1e-12, rtol=0)
+    else:
+        assert np.max(np.abs(out["y"] - y_ref)) > 1e-9
