@@ -69,6 +69,12 @@ extern "C" {
 /* LMOE_FLAG_BACKWARD: also reserve the workspace of lmoe_backward (BF16
  * experts with latent projections only; UNSUPPORTED otherwise). */
 #define LMOE_FLAG_BACKWARD 8
+/* LMOE_FLAG_EP_DENSE: a handle for expert parallelism that holds the router,
+ * the latent projections and the shared expert but no expert weights (w1, w2
+ * may be NULL): lmoe_forward_dispatch and lmoe_forward_combine apply, the
+ * experts run in expert shards (lmoe_experts_create), lmoe_forward returns
+ * UNSUPPORTED.  BF16 experts with latent projections only. */
+#define LMOE_FLAG_EP_DENSE 16
 
 #define LMOE_FMT_BF16 0  /* experts in BF16                                   */
 #define LMOE_FMT_NVFP4 1 /* experts in NVFP4: W1, W2 and the expert inputs u
@@ -343,6 +349,66 @@ int lmoe_nvfp4_quantize_sr(const float* x, int64_t rows, int32_t cols, float g, 
  * host reads afterwards: LMOE_ERR_TIMEOUT when the bounded wait gave up as
  * designed.  Checks the device-side failure path without a fault. */
 int lmoe_check_bounded_wait(int64_t limit_ns);
+
+/* Expert parallelism ("NVIDIA Nemotron 3: Efficient and Open Intelligence",
+ * section 三: the routed experts work on l-wide latent rows, so an expert-
+ * parallel exchange moves l values per routed row instead of d;
+ * "Nemotron-3 Super 精读报告", section 6.5: 64-way expert parallelism).  The
+ * experts are split into contiguous ranges, one per rank; a rank's forward is
+ *   lmoe_forward_dispatch   (router, projections, shared expert, segments and
+ *                            the latent rows of every routed (token, expert)
+ *                            pair in expert order: the send buffer);
+ *   exchange                (the caller: all-to-all of row slices by expert
+ *                            range, re-sort into local expert order with
+ *                            lmoe_permute_rows);
+ *   lmoe_experts_forward    (the grouped expert GEMMs of a shard);
+ *   exchange back           (lmoe_permute_rows, reverse all-to-all);
+ *   lmoe_forward_combine    (weighted sum per token, up-projection + shared).
+ * BF16 experts with latent projections only; asynchronous on `stream`.
+ *
+ * lmoe_forward_dispatch: x [T][d] bf16 (device) -> rows_out [T*K][l] bf16
+ * (device, caller-owned, 16-byte aligned): u = W_dn x of the token of each
+ * routed row, rows in expert order (expert, then token, then slot; the
+ * order of LMOE_DBG_PERM), and counts_out [N] int32 (device): rows per
+ * expert.  A layer handle (with or without LMOE_FLAG_EP_DENSE).  Keeps the
+ * routing for lmoe_forward_combine.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+int lmoe_forward_dispatch(lmoe_handle* h, const void* x, int64_t T, void* rows_out,
+                          int32_t* counts_out, void* stream);
+
+/* lmoe_forward_combine: rows_in [T*K][l] bf16 (device) -- the expert outputs
+ * W2[e] sqrelu(W1[e] u), unweighted, in the order of the last dispatch's
+ * rows_out -- -> y [T][d] bf16 (device): v = sum_k w_k o_k per token (fp32,
+ * slot order), y = W_upl v + W_s2 sqrelu(W_s1 x).  T must be the last
+ * dispatch's.  Errors: INVALID_ARG (T differs, null, misaligned),
+ * UNSUPPORTED, CUDA. */
+int lmoe_forward_combine(lmoe_handle* h, const void* rows_in, int64_t T, void* y, void* stream);
+
+/* An expert shard: experts [first_expert, first_expert + n_local) of the layer
+ * described by cfg (n_experts is the layer's N; BF16 experts; flags 0 or
+ * LMOE_FLAG_EP_DENSE).  w1 [n_local][h][l] and w2 [n_local][l][h] bf16
+ * (device) are the shard's experts, copied.  max_rows: the most rows one
+ * lmoe_experts_forward accepts.  The handle takes lmoe_experts_forward,
+ * lmoe_sync_status and lmoe_destroy; the layer calls return UNSUPPORTED or
+ * INVALID_ARG on it.  Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA. */
+int lmoe_experts_create(const lmoe_config* cfg, int32_t first_expert, int32_t n_local,
+                        const void* w1, const void* w2, int64_t max_rows, lmoe_handle** out);
+
+/* out[r] = W2[e] sqrelu(W1[e] rows[r]) for the R rows [R][l] bf16 (device) in
+ * local expert order, counts [n_local] int32 (device) rows per local expert;
+ * out [R][l] bf16 (device, must not overlap rows).  The counts are checked on
+ * the device: a negative count or a sum other than R computes nothing and
+ * records DEVICE (read by lmoe_sync_status).  Errors: INVALID_ARG (null, R <
+ * 0, R > max_rows, overlap, misalignment), CUDA. */
+int lmoe_experts_forward(lmoe_handle* h, const void* rows, const int32_t* counts, int64_t R,
+                         void* out, void* stream);
+
+/* Row permutation of an exchange: rows of row_bytes (a multiple of 16),
+ * gather (scatter = 0) dst[r] = src[idx[r]] or scatter (scatter = 1)
+ * dst[idx[r]] = src[r], for r < n; idx int32 (device).  An index outside
+ * [0, n_other) -- the row count of the indexed side -- skips its row.
+ * src, dst 16-byte aligned, not overlapping.  Errors: INVALID_ARG, CUDA. */
+int lmoe_permute_rows(const void* src, const int32_t* idx, int64_t n, int64_t n_other,
+                      int32_t row_bytes, void* dst, int scatter, void* stream);
 
 /* Frees everything the handle owns (synchronizes the device first). */
 void lmoe_destroy(lmoe_handle* h);

@@ -15,8 +15,8 @@ plans the expert-parallel exchange and moves rows with torch.distributed.
 """
 from . import ep
 from ._lib import LmoeError
-from .layer import (LatentMoE, lmoe_check_bounded_wait, lmoe_nvfp4_quantize_sr, lmoe_rht16,
-                    lmoe_route, lmoe_route_status)
+from .layer import (ExpertShard, LatentMoE, lmoe_check_bounded_wait, lmoe_nvfp4_quantize_sr,
+                    lmoe_permute_rows, lmoe_rht16, lmoe_route, lmoe_route_status)
 
-__all__ = ["LatentMoE", "lmoe_route", "lmoe_route_status", "lmoe_check_bounded_wait", "LmoeError", "lmoe_rht16",
+__all__ = ["LatentMoE", "ExpertShard", "lmoe_permute_rows", "lmoe_route", "lmoe_route_status", "lmoe_check_bounded_wait", "LmoeError", "lmoe_rht16",
            "lmoe_nvfp4_quantize_sr", "ep"]

@@ -18,6 +18,7 @@ FLAG_NO_PROJECTION = 1   # standard MoE: no latent projections (u = x, r = v)
 FLAG_NVFP4_WEIGHT_2D = 2   # NVFP4 weights: one scale per 16 x 16 block
 FLAG_NVFP4_WEIGHT_MSE = 4  # NVFP4 weights: MSE-searched block scales
 FLAG_BACKWARD = 8   # reserve the workspace of lmoe_backward
+FLAG_EP_DENSE = 16  # expert-parallel layer handle without expert weights
 NVFP4_WEIGHT_FLAGS = {"1d": 0, "2d": FLAG_NVFP4_WEIGHT_2D, "mse": FLAG_NVFP4_WEIGHT_MSE,
                       "2d_mse": FLAG_NVFP4_WEIGHT_2D | FLAG_NVFP4_WEIGHT_MSE}
 DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 6,
@@ -72,6 +73,15 @@ SIGNATURES = {
     "lmoe_route_noalloc_status": (c_int, [c_void_p]),
     "lmoe_route_noalloc": (c_int, [c_void_p, c_void_p, c_int64, c_int32, c_int32, c_void_p,
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "lmoe_forward_dispatch": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
+                                      c_void_p]),
+    "lmoe_forward_combine": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
+    "lmoe_experts_create": (c_int, [POINTER(LmoeConfig), c_int32, c_int32, c_void_p, c_void_p,
+                                    c_int64, POINTER(c_void_p)]),
+    "lmoe_experts_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p,
+                                     c_void_p]),
+    "lmoe_permute_rows": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int32, c_void_p,
+                                  c_int, c_void_p]),
     "lmoe_nvfp4_quantize": (c_int, [c_void_p, c_int64, c_int32, c_float, c_void_p, c_void_p,
                                     c_void_p]),
     "lmoe_rht16": (c_int, [c_void_p, c_int64, c_int32, c_uint64, c_void_p, c_void_p]),

@@ -37,6 +37,22 @@ cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int 
 cudaError_t launch_combine(const void* O, const int32_t* inv, int64_t T, int K, int l, void* vh,
                            int ldv, cudaStream_t st);
 
+// v[t] = sum_k w[t][k] O[inv[t][k]] (fp32, slot order): the combine of rows
+// that come back unweighted from an expert-parallel exchange.
+cudaError_t launch_combine_w(const void* O, const int32_t* inv, const float* topk_w, int64_t T,
+                             int K, int l, void* vh, int ldv, cudaStream_t st);
+
+// Caller-given rows per expert: out = in when every count is >= 0 and they
+// sum to R, else zeros and DEVERR_BAD_INDEX in *err.  n <= 1024.
+cudaError_t launch_sanitize_counts(const int32_t* in, int n, int64_t R, int32_t* out, int* err,
+                                   cudaStream_t st);
+
+// Rows of row_bytes (a multiple of 16): gather dst[r] = src[idx[r]] or
+// scatter dst[idx[r]] = src[r] for r < n; indices outside [0, n_other) skip
+// their row.
+cudaError_t launch_permute_rows(const void* src, const int32_t* idx, int64_t n, int64_t n_other,
+                                int row_bytes, void* dst, bool scatter, cudaStream_t st);
+
 // NVFP4 (nvfp4.cu).  Expert weights [E][rows_per][K] bf16 -> codes
 // [E*rows_per][Kp/2], scale atoms [E*rows_per/128][Kp/64][512], global scales
 // [E]; amax is [E] scratch.  Kp = K rounded up to 256; padding pre-zeroed.

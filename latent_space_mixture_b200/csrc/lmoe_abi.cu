@@ -100,7 +100,8 @@ struct EpiO {
   __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
                                          bool valid) const {
     if (!valid) return;
-    const float w = wrow[row];
+    // no weights: an expert shard returns the unweighted outputs
+    const float w = wrow ? wrow[row] : 1.0f;
     float a[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = v[i] * w;
@@ -757,6 +758,12 @@ struct lmoe_handle {
   CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
   BMaps tm_uperm, tm_H, tm_vh;
   int64_t last_T = 0;
+  // expert parallelism: a layer handle without expert weights (dispatch and
+  // combine only), or an expert shard (experts [first_expert, + n_experts))
+  bool ep_dense = false;
+  bool shard = false;
+  int first_expert = 0;
+  int64_t max_rows = 0;       // shard: rows one lmoe_experts_forward accepts
   bool pairs = true;   // CTA-pair GEMMs for large token counts (LMOE_PAIR=0: off)
   bool proj = true;    // latent projections (false: standard MoE, u = x, r = v)
   int lx = 0;          // W_dn rows in w_x and W_upl columns in w_y (l, or 0)
@@ -797,8 +804,12 @@ static int check_cfg(const lmoe_config* c) {
   if (c->d <= 0 || c->latent <= 0 || c->n_experts <= 0 || c->top_k <= 0 ||
       c->expert_hidden <= 0 || c->shared_hidden <= 0 || c->max_tokens < 1 ||
       (c->flags & ~(LMOE_FLAG_NO_PROJECTION | LMOE_FLAG_NVFP4_WEIGHT_2D |
-                    LMOE_FLAG_NVFP4_WEIGHT_MSE | LMOE_FLAG_BACKWARD)) != 0)
+                    LMOE_FLAG_NVFP4_WEIGHT_MSE | LMOE_FLAG_BACKWARD | LMOE_FLAG_EP_DENSE)) != 0)
     return LMOE_ERR_INVALID_ARG;
+  if ((c->flags & LMOE_FLAG_EP_DENSE) &&
+      ((c->flags & (LMOE_FLAG_NO_PROJECTION | LMOE_FLAG_BACKWARD)) ||
+       c->expert_format != LMOE_FMT_BF16))
+    return LMOE_ERR_UNSUPPORTED;
   if ((c->flags & (LMOE_FLAG_NVFP4_WEIGHT_2D | LMOE_FLAG_NVFP4_WEIGHT_MSE)) &&
       c->expert_format != LMOE_FMT_NVFP4 && c->expert_format != LMOE_FMT_W4A16)
     return LMOE_ERR_INVALID_ARG;
@@ -857,7 +868,8 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   int rc = check_cfg(cfg);
   if (rc != LMOE_OK) return rc;
   const bool proj = !(cfg->flags & LMOE_FLAG_NO_PROJECTION);
-  if (!w || !w->w_router || !w->w1 || !w->w2 || !w->w_s1 || !w->w_s2 ||
+  const bool ep_dense = (cfg->flags & LMOE_FLAG_EP_DENSE) != 0;
+  if (!w || !w->w_router || (!ep_dense && (!w->w1 || !w->w2)) || !w->w_s1 || !w->w_s2 ||
       (proj && (!w->w_dn || !w->w_upl)))
     return LMOE_ERR_INVALID_ARG;
   if ((cfg->expert_format == LMOE_FMT_NVFP4 || cfg->expert_format == LMOE_FMT_FP8) &&
@@ -889,7 +901,8 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   const bool w4 = c.expert_format == LMOE_FMT_W4A16;
   const bool fp4 = c.expert_format == LMOE_FMT_NVFP4;   // NVFP4 activations too
   const bool fp8 = c.expert_format == LMOE_FMT_FP8;
-  const bool bfx = !fp4 && !fp8 && !w4;   // BF16 experts
+  h->ep_dense = ep_dense;
+  const bool bfx = !fp4 && !fp8 && !w4 && !ep_dense;   // BF16 experts held by this handle
   const bool qw4 = fp4 || w4;             // NVFP4-quantised expert weights
   h->fp4 = fp4;
   h->fp8 = fp8;
@@ -998,6 +1011,8 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   if (bfx) {
     ok &= cudaMemcpy(h->w1, w->w1, N * hh * l * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
     ok &= cudaMemcpy(h->w2, w->w2, N * l * hh * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  } else if (ep_dense) {
+    // no expert weights: the experts live in expert shards (lmoe_experts_create)
   } else if (fp8) {
     // per-tensor scales: s = amax / 448 per expert matrix; activations static
     h->g_u = w->act_gscale_latent;
@@ -1185,21 +1200,12 @@ static void prof_end(lmoe_handle* h, int slot, cudaStream_t st) {
     if (_e != cudaSuccess) return LMOE_ERR_CUDA;     \
   } while (0)
 
-int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream) {
-  if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
-  if (T == 0) return LMOE_OK;
-  if (!x || !y) return LMOE_ERR_INVALID_ARG;
+// Steps 1-5 of the forward: [W_r; W_dn; W_s1] x (logits, u, shared hidden),
+// routing and the per-expert segments.
+static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st) {
   const lmoe_config& c = h->cfg;
   const int64_t d = c.d;
-  const char* xb = static_cast<const char*>(x);
-  const char* yb = static_cast<const char*>(y);
-  if (xb < yb + T * d * 2 && yb < xb + T * d * 2) return LMOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15)
-    return LMOE_ERR_INVALID_ARG;
-  DeviceGuard g(h->dev);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int N = c.n_experts, l = c.latent, hh = c.expert_hidden, hs = c.shared_hidden,
-            K = c.top_k;
+  const int N = c.n_experts, l = c.latent, hs = c.shared_hidden, K = c.top_k;
   const int ldvh = l + hs;
   const int lx = h->lx;   // l, or 0 for the standard MoE
   const unsigned long long lim = h->wait_limit_ns;
@@ -1250,6 +1256,64 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   LMOE_STEP(4, launch_scatter(h->topk_idx, h->topk_w, h->chunk, h->counts, T, N, K, gbn,
                               h->offsets, h->perm, h->inv, h->wrow, h->blocks, h->nblocks,
                               h->rblock, h->err, st));
+  return LMOE_OK;
+}
+
+// Step 10 of the forward: y = [W_upl | W_s2] [v ; hs] (v already in vh).
+static int fwd_ygemm(lmoe_handle* h, int64_t T, void* y, cudaStream_t st) {
+  const lmoe_config& c = h->cfg;
+  const int64_t d = c.d;
+  const int l = c.latent, hs = c.shared_hidden;
+  const int ldvh = l + hs;
+  const int lx = h->lx;
+  const unsigned long long lim = h->wait_limit_ns;
+  {
+    const int fb = static_cast<int>((d + 127) / 128);
+    const int ky = lx + hs;   // K of the y-GEMM
+    const DensePlan p = plan_dense(T, fb, ky / 64, h->sms);
+    if (p.ksplit > 1 && int64_t(p.ksplit) * T * d > h->part_floats)
+      return LMOE_ERR_UNSUPPORTED;   // never: the buffer is sized for every T
+    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d), h->proj ? nullptr : h->vh, ldvh};
+    const int fb2 = static_cast<int>((d + PAIR_BM - 1) / PAIR_BM);
+    const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
+    if (h->pairs && ptiles >= h->sms / 2) {
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, static_cast<int>(d),
+                   ky / 64, 1, nullptr, 0};
+      LMOE_STEP(9, launch_gemm_pair(h->tm_wy, h->tm_vh, s, epi, h->sms / 2, h->err, lim, st));
+    } else {
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, static_cast<int>(d),
+                   ky / 64, p.ksplit, h->part, T <= p.bn};
+      const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
+      const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
+      LMOE_STEP(9, launch_gemm_bn(p.bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
+      if (p.ksplit > 1)
+        LMOE_STEP(11, launch_reduce(h->part, p.ksplit, static_cast<int>(T), static_cast<int>(d),
+                                    epi, st));
+    }
+  }
+  return LMOE_OK;
+}
+
+int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return LMOE_OK;
+  if (!x || !y) return LMOE_ERR_INVALID_ARG;
+  if (h->shard || h->ep_dense) return LMOE_ERR_UNSUPPORTED;
+  const lmoe_config& c = h->cfg;
+  const int64_t d = c.d;
+  const char* xb = static_cast<const char*>(x);
+  const char* yb = static_cast<const char*>(y);
+  if (xb < yb + T * d * 2 && yb < xb + T * d * 2) return LMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15)
+    return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int l = c.latent, hh = c.expert_hidden, hs = c.shared_hidden, K = c.top_k;
+  const int ldvh = l + hs;
+  const unsigned long long lim = h->wait_limit_ns;
+  int rc = fwd_front(h, x, T, st);
+  if (rc != LMOE_OK) return rc;
+  const int gbn = grouped_bn(c, T);
   if (h->w4) {
     // 6. f16 latent rows into expert order
     LMOE_STEP(5, launch_gather(h->u16, h->perm, T * K, K, l, h->u_perm, st));
@@ -1339,31 +1403,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   // 9. v = sum_k O[inv[t][k]]
   LMOE_STEP(8, launch_combine(h->O, h->inv, T, K, l, h->vh, ldvh, st));
   // 10. y = [W_upl | W_s2] [v ; hs]
-  {
-    const int fb = static_cast<int>((d + 127) / 128);
-    const int ky = lx + hs;   // K of the y-GEMM
-    const DensePlan p = plan_dense(T, fb, ky / 64, h->sms);
-    if (p.ksplit > 1 && int64_t(p.ksplit) * T * d > h->part_floats)
-      return LMOE_ERR_UNSUPPORTED;   // never: the buffer is sized for every T
-    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d), h->proj ? nullptr : h->vh, ldvh};
-    const int fb2 = static_cast<int>((d + PAIR_BM - 1) / PAIR_BM);
-    const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
-    if (h->pairs && ptiles >= h->sms / 2) {
-      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, static_cast<int>(d),
-                   ky / 64, 1, nullptr, 0};
-      LMOE_STEP(9, launch_gemm_pair(h->tm_wy, h->tm_vh, s, epi, h->sms / 2, h->err, lim, st));
-    } else {
-      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, static_cast<int>(d),
-                   ky / 64, p.ksplit, h->part, T <= p.bn};
-      const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
-      const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
-      LMOE_STEP(9, launch_gemm_bn(p.bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
-      if (p.ksplit > 1)
-        LMOE_STEP(11, launch_reduce(h->part, p.ksplit, static_cast<int>(T), static_cast<int>(d),
-                                    epi, st));
-    }
-  }
-  return LMOE_OK;
+  return fwd_ygemm(h, T, y, st);
 }
 
 int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void* dx,
@@ -1548,6 +1588,203 @@ int lmoe_sync_status(lmoe_handle* h, void* stream) {
   return LMOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// expert parallelism
+
+int lmoe_forward_dispatch(lmoe_handle* h, const void* x, int64_t T, void* rows_out,
+                          int32_t* counts_out, void* stream) {
+  if (!h || h->shard || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+  if (!h->proj || h->cfg.expert_format != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED;
+  if (!counts_out) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const lmoe_config& c = h->cfg;
+  if (T == 0) {
+    h->last_T = 0;
+    return cudaMemsetAsync(counts_out, 0, size_t(c.n_experts) * 4, st) == cudaSuccess
+               ? LMOE_OK
+               : LMOE_ERR_CUDA;
+  }
+  if (!x || !rows_out ||
+      ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(rows_out)) & 15))
+    return LMOE_ERR_INVALID_ARG;
+  int rc = fwd_front(h, x, T, st);
+  if (rc != LMOE_OK) return rc;
+  // the latent rows in expert order: the send buffer of the exchange
+  LMOE_STEP(5, launch_gather(h->u, h->perm, T * c.top_k, c.top_k, c.latent, rows_out, st));
+  if (cudaMemcpyAsync(counts_out, h->counts, size_t(c.n_experts) * 4, cudaMemcpyDeviceToDevice,
+                      st) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  return LMOE_OK;
+}
+
+int lmoe_forward_combine(lmoe_handle* h, const void* rows_in, int64_t T, void* y, void* stream) {
+  if (!h || h->shard || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+  if (!h->proj || h->cfg.expert_format != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED;
+  if (T == 0) return LMOE_OK;
+  if (T != h->last_T || !rows_in || !y ||
+      ((reinterpret_cast<uintptr_t>(rows_in) | reinterpret_cast<uintptr_t>(y)) & 15))
+    return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const lmoe_config& c = h->cfg;
+  // v[t] = sum_k w[t][k] o[inv[t][k]]
+  LMOE_STEP(8, launch_combine_w(rows_in, h->inv, h->topk_w, T, c.top_k, c.latent, h->vh,
+                                c.latent + c.shared_hidden, st));
+  return fwd_ygemm(h, T, y, st);
+}
+
+int lmoe_experts_create(const lmoe_config* cfg, int32_t first_expert, int32_t n_local,
+                        const void* w1, const void* w2, int64_t max_rows, lmoe_handle** out) {
+  if (!out) return LMOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = check_cfg(cfg);
+  if (rc != LMOE_OK) return rc;
+  if (cfg->expert_format != LMOE_FMT_BF16 || (cfg->flags & ~LMOE_FLAG_EP_DENSE))
+    return LMOE_ERR_UNSUPPORTED;
+  if (!w1 || !w2 || n_local <= 0 || first_expert < 0 || first_expert + n_local > cfg->n_experts ||
+      max_rows < 1 || max_rows >= (int64_t(1) << 31) - 65536)
+    return LMOE_ERR_INVALID_ARG;
+  if (!get_encode()) return LMOE_ERR_CUDA;
+  lmoe_handle* h = new (std::nothrow) lmoe_handle();
+  if (!h) return LMOE_ERR_OOM;
+  h->cfg = *cfg;
+  h->cfg.n_experts = n_local;
+  h->shard = true;
+  h->first_expert = first_expert;
+  h->max_rows = max_rows;
+  if (cudaGetDevice(&h->dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess) {
+    delete h;
+    return LMOE_ERR_CUDA;
+  }
+  const int64_t n = n_local, l = cfg->latent, hh = cfg->expert_hidden;
+  const int64_t rows_b = max_rows < 256 ? 256 : max_rows;
+  const int64_t max_blocks = max_rows / 32 + n + 1;
+  struct Req {
+    void** p;
+    size_t bytes;
+  } reqs[] = {
+      {(void**)&h->w1, size_t(n * hh * l * 2)},
+      {(void**)&h->w2, size_t(n * l * hh * 2)},
+      {(void**)&h->counts, size_t(n * 4)},
+      {(void**)&h->offsets, size_t((n + 1) * 4)},
+      {(void**)&h->blocks, size_t(max_blocks * 16)},
+      {(void**)&h->nblocks, size_t(4)},
+      {(void**)&h->u_perm, size_t(rows_b * l * 2)},
+      {(void**)&h->H, size_t(rows_b * hh * 2)},
+      {(void**)&h->err, size_t(4)},
+  };
+  for (auto& r : reqs) {
+    if ((rc = alloc_dev(h, r.p, r.bytes)) != LMOE_OK) {
+      free_all(h);
+      delete h;
+      return rc;
+    }
+  }
+  bool ok = cudaMemcpy(h->w1, w1, n * hh * l * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemcpy(h->w2, w2, n * l * hh * 2, cudaMemcpyDeviceToDevice) == cudaSuccess;
+  ok &= cudaMemset(h->u_perm, 0, rows_b * l * 2) == cudaSuccess;
+  ok &= cudaMemset(h->H, 0, rows_b * hh * 2) == cudaSuccess;
+  ok &= cudaMemset(h->err, 0, 4) == cudaSuccess;
+  ok &= make_map(&h->tm_w1, h->w1, n * hh, l, GEMM_BM);
+  ok &= make_map(&h->tm_w2, h->w2, n * l, hh, GEMM_BM);
+  ok &= make_map(&h->tm_uperm.b16, h->u_perm, rows_b, l, GEMM_BROWS);
+  ok &= make_map(&h->tm_uperm.b64, h->u_perm, rows_b, l, GEMM_BROWS_BIG);
+  ok &= make_map(&h->tm_H.b16, h->H, rows_b, hh, GEMM_BROWS);
+  ok &= make_map(&h->tm_H.b64, h->H, rows_b, hh, GEMM_BROWS_BIG);
+  ok &= set_smem_all<EpiH>() == cudaSuccess;
+  ok &= set_smem_all<EpiO>() == cudaSuccess;
+  ok &= set_pair_smem<EpiH>() == cudaSuccess;
+  ok &= set_pair_smem<EpiO>() == cudaSuccess;
+  ok &= cudaDeviceSynchronize() == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    free_all(h);
+    delete h;
+    return LMOE_ERR_CUDA;
+  }
+  const char* pe = getenv("LMOE_PAIR");
+  h->pairs = !(pe && pe[0] == '0');
+  *out = h;
+  return LMOE_OK;
+}
+
+int lmoe_experts_forward(lmoe_handle* h, const void* rows, const int32_t* counts, int64_t R,
+                         void* out, void* stream) {
+  if (!h || !h->shard || R < 0 || R > h->max_rows || !counts) return LMOE_ERR_INVALID_ARG;
+  if (R > 0 && (!rows || !out ||
+                ((reinterpret_cast<uintptr_t>(rows) | reinterpret_cast<uintptr_t>(out)) & 15)))
+    return LMOE_ERR_INVALID_ARG;
+  const char* rb = static_cast<const char*>(rows);
+  const char* ob = static_cast<const char*>(out);
+  const int64_t bytes = R * h->cfg.latent * 2;
+  if (R > 0 && rb < ob + bytes && ob < rb + bytes) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const lmoe_config& c = h->cfg;
+  const int n = c.n_experts, l = c.latent, hh = c.expert_hidden;
+  const unsigned long long lim = h->wait_limit_ns;
+  // counts checked on the device (>= 0, sum R) before any block is built
+  LMOE_STEP(2, launch_sanitize_counts(counts, n, R, h->counts, h->err, st));
+  if (R == 0) return LMOE_OK;
+  const double avg = double(R) / n;
+  const int gbn = avg <= 40.0 ? 32 : avg <= 160.0 ? 128 : 256;
+  // offsets and token blocks of at most gbn rows per expert from the counts
+  LMOE_STEP(4, launch_scatter(nullptr, nullptr, nullptr, h->counts, 0, n, 1, gbn, h->offsets,
+                              nullptr, nullptr, nullptr, h->blocks, h->nblocks, nullptr, h->err,
+                              st));
+  // the B operand: the caller's rows, or the padded staging copy when fewer
+  // rows than one TMA box of 256 rows fit
+  BMaps tm_rows;
+  if (R < 256) {
+    if (cudaMemcpyAsync(h->u_perm, rows, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    tm_rows = h->tm_uperm;
+  } else if (!make_map(&tm_rows.b16, rows, R, l, GEMM_BROWS) ||
+             !make_map(&tm_rows.b64, rows, R, l, GEMM_BROWS_BIG)) {
+    return LMOE_ERR_CUDA;
+  }
+  {
+    EpiH epi{h->H, hh};
+    if (h->pairs && gbn == PAIR_BN) {
+      TileSource s{0, 0, h->blocks, h->nblocks, (hh + PAIR_BM - 1) / PAIR_BM, hh, hh, l / 64, 1,
+                   nullptr, 0};
+      LMOE_STEP(6, launch_gemm_pair(h->tm_w1, tm_rows, s, epi, h->sms / 2, h->err, lim, st));
+    } else {
+      TileSource s{0, 0, h->blocks, h->nblocks, (hh + 127) / 128, hh, hh, l / 64, 1, nullptr,
+                   gbn == 32};
+      LMOE_STEP(6, launch_gemm_bn(gbn, h->tm_w1, tm_rows, s, epi, h->sms, h->err, lim, st));
+    }
+  }
+  {
+    EpiO epi{static_cast<bf16*>(out), nullptr, l};
+    if (h->pairs && gbn == PAIR_BN) {
+      TileSource s{0, 0, h->blocks, h->nblocks, (l + PAIR_BM - 1) / PAIR_BM, l, l, hh / 64, 1,
+                   nullptr, 0};
+      LMOE_STEP(7, launch_gemm_pair(h->tm_w2, h->tm_H, s, epi, h->sms / 2, h->err, lim, st));
+    } else {
+      TileSource s{0, 0, h->blocks, h->nblocks, (l + 127) / 128, l, l, hh / 64, 1, nullptr,
+                   gbn == 32};
+      LMOE_STEP(7, launch_gemm_bn(gbn, h->tm_w2, h->tm_H, s, epi, h->sms, h->err, lim, st));
+    }
+  }
+  return LMOE_OK;
+}
+
+int lmoe_permute_rows(const void* src, const int32_t* idx, int64_t n, int64_t n_other,
+                      int32_t row_bytes, void* dst, int scatter, void* stream) {
+  if (n < 0 || n_other < 0 || row_bytes <= 0 || row_bytes % 16) return LMOE_ERR_INVALID_ARG;
+  if (n == 0) return LMOE_OK;
+  if (!src || !idx || !dst ||
+      ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15))
+    return LMOE_ERR_INVALID_ARG;
+  return launch_permute_rows(src, idx, n, n_other, row_bytes, dst, scatter != 0,
+                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LMOE_OK
+             : LMOE_ERR_CUDA;
+}
+
 int lmoe_forward_host(lmoe_handle* h, const void* x_host, int64_t T, void* y_host, void* stream) {
   if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return LMOE_OK;
@@ -1566,6 +1803,7 @@ int lmoe_forward_host(lmoe_handle* h, const void* x_host, int64_t T, void* y_hos
 
 int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
   if (!h || !dst) return LMOE_ERR_INVALID_ARG;
+  if (h->shard) return LMOE_ERR_UNSUPPORTED;
   DeviceGuard g(h->dev);
   const lmoe_config& c = h->cfg;
   const int64_t T = h->last_T, K = c.top_k, N = c.n_experts, l = c.latent,

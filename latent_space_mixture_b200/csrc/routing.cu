@@ -18,41 +18,12 @@
 #include "kernels.h"
 #include "launch.cuh"
 #include "ptx.cuh"
+#include "route.cuh"
 
 namespace lmoe {
 
 // ---------------------------------------------------------------------------
-// router: one warp per token
-//
-// Each candidate is packed into one 64-bit word: the key's bits mapped to an
-// unsigned order (high half) and 0xFFFFFFFF - expert (low half), so that the
-// largest word is the largest key and, among equal keys, the lowest expert
-// id.  A lane keeps the best word of its experts (e = lane + 32 i); each of
-// the K rounds takes the warp maximum, and only the winning lane rescans.
-
-__device__ __forceinline__ uint64_t pack_key(float key, int e) {
-  uint32_t b = __float_as_uint(key);
-  b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-  return (static_cast<uint64_t>(b) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
-}
-
-// Warp maximum of 64-bit words with two 32-bit reductions: the high halves,
-// then the low halves among the lanes holding the high maximum.
-__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
-  const uint32_t hi = static_cast<uint32_t>(v >> 32);
-  const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
-  const uint32_t lo = hi == mhi ? static_cast<uint32_t>(v) : 0u;
-  const uint32_t mlo = __reduce_max_sync(0xffffffffu, lo);
-  return (static_cast<uint64_t>(mhi) << 32) | mlo;
-}
-
-// compare-exchange for a descending sort network
-__device__ __forceinline__ void cas_desc(uint64_t& a, uint64_t& b) {
-  const uint64_t hi = a > b ? a : b;
-  const uint64_t lo = a > b ? b : a;
-  a = hi;
-  b = lo;
-}
+// router: one warp per token, logits read from memory (route.cuh selects)
 
 template <int NPL>   // upper bound of experts per lane (N <= 32 NPL), a power of 2
 __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
@@ -73,50 +44,7 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
     zz[i] = (i < npl) ? z[lane + 32 * i] : 0.0f;
     bb[i] = (i < npl && bias) ? bias[lane + 32 * i] : 0.0f;
   }
-  uint64_t cand[NPL];
-#pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    cand[i] = 0;   // below every packed key
-    if (i < npl) {
-      const float sc = 1.0f / (1.0f + expf(-zz[i]));
-      cand[i] = pack_key(sc + bb[i], lane + 32 * i);
-    }
-  }
-  // sort the lane's candidates descending (bitonic network on registers)
-#pragma unroll
-  for (int k = 2; k <= NPL; k <<= 1) {
-#pragma unroll
-    for (int j = k >> 1; j > 0; j >>= 1) {
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        const int p = i ^ j;
-        if (p > i) {
-          if ((i & k) == 0) cas_desc(cand[i], cand[p]);
-          else cas_desc(cand[p], cand[i]);
-        }
-      }
-    }
-  }
-  // K rounds: the warp maximum of the lanes' heads; the winner shifts its list
-  int my_e = 0;
-  for (int k = 0; k < K; ++k) {
-    const uint64_t win = warp_max_u64(cand[0]);
-    if (lane == k) my_e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win));
-    if (cand[0] == win) {
-#pragma unroll
-      for (int i = 0; i + 1 < NPL; ++i) cand[i] = cand[i + 1];
-      cand[NPL - 1] = 0;
-    }
-  }
-  // weights: the unbiased scores of the selected experts, renormalised; the
-  // score is recomputed from the same logit with the same expression
-  const float my_s = (lane < K) ? 1.0f / (1.0f + expf(-z[my_e])) : 0.0f;
-  float sum = 0.0f;
-  for (int k = 0; k < K; ++k) sum += __shfl_sync(0xffffffffu, my_s, k);
-  if (lane < K) {
-    topk_idx[t * K + lane] = my_e;
-    topk_w[t * K + lane] = __fdiv_rn(my_s, sum);
-  }
+  route_select<NPL>(zz, bb, npl, z, K, lane, t, topk_idx, topk_w);
 }
 
 cudaError_t launch_route(const float* logits, const float* bias, int64_t T, int N, int K,
@@ -387,12 +315,16 @@ cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int 
 }
 
 // ---------------------------------------------------------------------------
-// latent combine in token order: v[t] = sum_k O[inv[t][k]], fixed slot order.
-// One thread per 8 consecutive latent elements of one token; the K row
-// indices and the K row loads are issued before the (ordered) sum.
+// latent combine in token order: v[t] = sum_k O[inv[t][k]], fixed slot order
+// (WEIGHTED: sum_k w[t][k] O[inv[t][k]], for rows that come back unweighted
+// from an expert-parallel exchange).  One thread per 8 consecutive latent
+// elements of one token; the K row indices and the K row loads are issued
+// before the (ordered) sum.
 
+template <bool WEIGHTED>
 __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict__ O,
-                                                 const int32_t* __restrict__ inv, int64_t T,
+                                                 const int32_t* __restrict__ inv,
+                                                 const float* __restrict__ wts, int64_t T,
                                                  int K, int l, __nv_bfloat16* __restrict__ vh,
                                                  int ldv) {
   pdl_wait();
@@ -403,8 +335,11 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict
   if (t >= T) return;
   const int c = static_cast<int>(g - t * l8) * 8;
   int rows[32];
+  float wk[32];
 #pragma unroll
   for (int k = 0; k < 32; ++k) rows[k] = (k < K) ? inv[t * K + k] : 0;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) wk[k] = (WEIGHTED && k < K) ? wts[t * K + k] : 1.0f;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   // eight row loads in flight, then their sums in slot order
 #pragma unroll
@@ -424,8 +359,13 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 f = __bfloat1622float2(p[i]);
-            acc[2 * i] += f.x;
-            acc[2 * i + 1] += f.y;
+            if (WEIGHTED) {
+              acc[2 * i] = fmaf(wk[k0 + j], f.x, acc[2 * i]);
+              acc[2 * i + 1] = fmaf(wk[k0 + j], f.y, acc[2 * i + 1]);
+            } else {
+              acc[2 * i] += f.x;
+              acc[2 * i + 1] += f.y;
+            }
           }
         }
       }
@@ -441,9 +381,89 @@ cudaError_t launch_combine(const void* O, const int32_t* inv, int64_t T, int K, 
                            int ldv, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   const int64_t blocks = (T * (l / 8) + 255) / 256;
-  return launch_pdl(k_combine, static_cast<unsigned>(blocks), 256, 0, st,
-                    static_cast<const __nv_bfloat16*>(O), inv, T, K, l,
+  return launch_pdl(k_combine<false>, static_cast<unsigned>(blocks), 256, 0, st,
+                    static_cast<const __nv_bfloat16*>(O), inv, static_cast<const float*>(nullptr),
+                    T, K, l, static_cast<__nv_bfloat16*>(vh), ldv);
+}
+
+cudaError_t launch_combine_w(const void* O, const int32_t* inv, const float* topk_w, int64_t T,
+                             int K, int l, void* vh, int ldv, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  const int64_t blocks = (T * (l / 8) + 255) / 256;
+  return launch_pdl(k_combine<true>, static_cast<unsigned>(blocks), 256, 0, st,
+                    static_cast<const __nv_bfloat16*>(O), inv, topk_w, T, K, l,
                     static_cast<__nv_bfloat16*>(vh), ldv);
+}
+
+// ---------------------------------------------------------------------------
+// counts of rows per expert handed in by a caller (an expert-parallel
+// receiver): copied when every count is >= 0 and they sum to R, else zeros
+// (no rows, no tiles) and DEVERR_BAD_INDEX in *err.  One block of 256 threads.
+
+__global__ void __launch_bounds__(256) k_sanitize_counts(const int32_t* __restrict__ in, int n,
+                                                         int64_t R, int32_t* __restrict__ out,
+                                                         int* err) {
+  __shared__ long long part[256];
+  __shared__ int bad;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  long long sum = 0;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int c = in[e];
+    if (c < 0) bad = 1;
+    sum += c;
+  }
+  part[threadIdx.x] = sum;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) part[threadIdx.x] += part[threadIdx.x + o];
+    __syncthreads();
+  }
+  const bool ok = !bad && part[0] == R;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) out[e] = ok ? in[e] : 0;
+  if (!ok && threadIdx.x == 0) atomicOr(err, DEVERR_BAD_INDEX);
+}
+
+cudaError_t launch_sanitize_counts(const int32_t* in, int n, int64_t R, int32_t* out, int* err,
+                                   cudaStream_t st) {
+  return launch_pdl(k_sanitize_counts, 1, 256, 0, st, in, n, R, out, err);
+}
+
+// ---------------------------------------------------------------------------
+// row permutation of an expert-parallel exchange (one warp per row, 16-byte
+// units): gather dst[r] = src[idx[r]], or scatter dst[idx[r]] = src[r].  An
+// index outside [0, n_other) -- the row count of the indexed side -- skips
+// its row.
+
+template <bool SCATTER>
+__global__ void __launch_bounds__(256) k_permute_rows(const uint4* __restrict__ src,
+                                                      const int32_t* __restrict__ idx, int64_t n,
+                                                      int64_t n_other, int w16,
+                                                      uint4* __restrict__ dst) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < n;
+       r += nwarps) {
+    const int64_t j = idx[r];
+    if (j < 0 || j >= n_other) continue;
+    const uint4* s = src + (SCATTER ? r : j) * w16;
+    uint4* d = dst + (SCATTER ? j : r) * w16;
+    for (int i = lane; i < w16; i += 32) d[i] = s[i];
+  }
+}
+
+cudaError_t launch_permute_rows(const void* src, const int32_t* idx, int64_t n, int64_t n_other,
+                                int row_bytes, void* dst, bool scatter, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  int64_t blocks = (n + 7) / 8;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  return launch_pdl(scatter ? k_permute_rows<true> : k_permute_rows<false>,
+                    static_cast<unsigned>(blocks), 256, 0, st, static_cast<const uint4*>(src), idx,
+                    n, n_other, row_bytes / 16, static_cast<uint4*>(dst));
 }
 
 // ---------------------------------------------------------------------------

@@ -18,7 +18,11 @@ arrive in the sender's expert order, where the weighted sum per token runs.
 
 This module holds no arithmetic of the layer: it computes counts,
 permutations and split sizes, and moves rows with
-torch.distributed.all_to_all_single (NCCL on GPUs, gloo on CPU).
+torch.distributed.all_to_all_single (NCCL on GPUs, gloo on CPU).  On GPUs,
+`forward` runs one rank's layer with the library's expert-parallel calls:
+lmoe_forward_dispatch (the latent rows in expert order), the all-to-all,
+lmoe_permute_rows (into local expert order), lmoe_experts_forward (the
+rank's shard of experts), the way back, and lmoe_forward_combine.
 """
 from __future__ import annotations
 
@@ -28,7 +32,8 @@ from typing import List, Optional
 import torch
 import torch.distributed as dist
 
-__all__ = ["expert_range", "EPPlan", "plan", "dispatch", "combine"]
+__all__ = ["expert_range", "EPPlan", "plan", "plan_from_counts", "dispatch", "combine",
+           "forward"]
 
 
 def expert_range(N: int, P: int, rank: int):
@@ -68,9 +73,17 @@ def plan(counts: torch.Tensor, group: Optional[dist.ProcessGroup] = None) -> EPP
     if N % P:
         raise ValueError("the expert count must be a multiple of the ranks")
     c = counts.to(torch.int64).reshape(P, per)          # [dest][local expert of dest]
-    send_counts = c.sum(dim=1).tolist()
     recv_e = torch.empty_like(c)                         # [source][my local expert]
     dist.all_to_all_single(recv_e.reshape(-1), c.reshape(-1).contiguous(), group=group)
+    return plan_from_counts(c, recv_e)
+
+
+def plan_from_counts(c: torch.Tensor, recv_e: torch.Tensor) -> EPPlan:
+    """The plan of one rank from its own rows per (destination, local expert
+    of the destination), c [P][N/P], and the rows every source sends for
+    this rank's local experts, recv_e [P][N/P] (host int64 tensors)."""
+    P, per = c.shape
+    send_counts = c.sum(dim=1).tolist()
     recv_counts = recv_e.sum(dim=1).tolist()
     # received buffer: source-major, each source's rows by local expert
     src_base = torch.zeros(P + 1, dtype=torch.int64)
@@ -104,3 +117,22 @@ def combine(rows: torch.Tensor, p: EPPlan, group: Optional[dist.ProcessGroup] = 
     out = rows.new_empty((sum(p.send_counts),) + tuple(rows.shape[1:]))
     dist.all_to_all_single(out, back.contiguous(), p.send_counts, p.recv_counts, group=group)
     return out
+
+
+def forward(layer, shard, x: torch.Tensor, group: Optional[dist.ProcessGroup] = None):
+    """One rank's expert-parallel forward on GPUs: `layer` a LatentMoE built
+    with ep_dense=True (router, projections, shared expert), `shard` the
+    ExpertShard of this rank's expert range (expert_range), x [T][d] this
+    rank's tokens.  The exchanged rows are l wide.  Returns y [T][d]."""
+    from .layer import lmoe_permute_rows
+    rows, counts = layer.dispatch(x)
+    p = plan(counts.cpu(), group)
+    recv = rows.new_empty((sum(p.recv_counts), rows.shape[1]))
+    dist.all_to_all_single(recv, rows, p.recv_counts, p.send_counts, group=group)
+    order = p.local_order.to(torch.int32).to(rows.device)
+    local = lmoe_permute_rows(recv, order, scatter=False)
+    out = shard.forward(local, p.local_counts.to(torch.int32).to(rows.device))
+    back = lmoe_permute_rows(out, order, scatter=True, out_rows=recv.shape[0])
+    got = torch.empty_like(rows)
+    dist.all_to_all_single(got, back, p.send_counts, p.recv_counts, group=group)
+    return layer.combine(got)

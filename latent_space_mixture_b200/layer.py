@@ -10,12 +10,14 @@ from typing import Dict, Optional
 import torch
 
 from . import _lib
-from ._lib import (DBG, FLAG_BACKWARD, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8, FMT_NVFP4,
+from ._lib import (DBG, FLAG_BACKWARD, FLAG_EP_DENSE, FLAG_NO_PROJECTION, FMT_BF16, FMT_FP8,
+                   FMT_NVFP4,
                    FMT_W4A16, NVFP4_WEIGHT_FLAGS,
                    LmoeConfig, LmoeError, LmoeGrads, LmoeWeights, check)
 
-__all__ = ["LatentMoE", "lmoe_route", "lmoe_route_status", "lmoe_check_bounded_wait",
-           "LmoeError", "lmoe_rht16", "lmoe_nvfp4_quantize_sr"]
+__all__ = ["LatentMoE", "ExpertShard", "lmoe_route", "lmoe_route_status",
+           "lmoe_check_bounded_wait", "LmoeError", "lmoe_rht16", "lmoe_nvfp4_quantize_sr",
+           "lmoe_permute_rows"]
 
 _WEIGHT_SHAPES = {
     "w_router": ("N", "d"), "w_dn": ("l", "d"), "w1": ("N", "h", "l"), "w2": ("N", "l", "h"),
@@ -39,16 +41,20 @@ class LatentMoE:
     nvfp4_weights ("1d", "2d", "mse", "2d_mse") picks the NVFP4 weight blocks
     and scale choice (LMOE_FLAG_NVFP4_WEIGHT_* of the C ABI).
     backward=True reserves the workspace of lmoe_backward (LMOE_FLAG_BACKWARD).
+    ep_dense=True builds the expert-parallel layer handle (LMOE_FLAG_EP_DENSE):
+    no expert weights (w1, w2 not needed), dispatch() and combine() only.
     """
 
     def __init__(self, d: int, latent: int, n_experts: int, top_k: int, expert_hidden: int,
                  shared_hidden: int, max_tokens: int, weights: Dict[str, torch.Tensor],
                  expert_format: str = "bf16", act_gscales=(0.0, 0.0), projections: bool = True,
-                 nvfp4_weights: str = "1d", backward: bool = False):
+                 nvfp4_weights: str = "1d", backward: bool = False, ep_dense: bool = False):
         self.lib = _lib.load()
         dims = {"d": d, "l": latent, "N": n_experts, "h": expert_hidden, "hs": shared_hidden}
         for k, shape in _WEIGHT_SHAPES.items():
             if not projections and k in ("w_dn", "w_upl"):
+                continue
+            if ep_dense and k in ("w1", "w2"):
                 continue
             t = weights[k]
             want = tuple(dims[s] for s in shape)
@@ -65,15 +71,17 @@ class LatentMoE:
                                "w4a16": FMT_W4A16}[expert_format],
                               (0 if projections else FLAG_NO_PROJECTION)
                               | NVFP4_WEIGHT_FLAGS[nvfp4_weights]
-                              | (FLAG_BACKWARD if backward else 0), max_tokens)
+                              | (FLAG_BACKWARD if backward else 0)
+                              | (FLAG_EP_DENSE if ep_dense else 0), max_tokens)
         w = LmoeWeights(weights["w_router"].data_ptr(),
                         bias.data_ptr() if bias is not None else None,
                         weights["w_dn"].data_ptr() if projections else None,
-                        weights["w1"].data_ptr(), weights["w2"].data_ptr(),
+                        None if ep_dense else weights["w1"].data_ptr(),
+                        None if ep_dense else weights["w2"].data_ptr(),
                         weights["w_upl"].data_ptr() if projections else None,
                         weights["w_s1"].data_ptr(), weights["w_s2"].data_ptr(),
                         float(act_gscales[0]), float(act_gscales[1]))
-        self.device = weights["w1"].device
+        self.device = weights["w_router"].device
         h = c_void_p()
         with torch.cuda.device(self.device):
             check(self.lib.lmoe_create(byref(self.cfg), byref(w), byref(h)), "lmoe_create")
@@ -108,6 +116,44 @@ class LatentMoE:
                                          c_void_p(y_host.data_ptr()), _stream_ptr(stream)),
               "lmoe_forward_host")
         self.last_T = T
+
+    # -- expert parallelism -----------------------------------------------
+    def dispatch(self, x: torch.Tensor, rows_out: Optional[torch.Tensor] = None,
+                 counts_out: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None):
+        """lmoe_forward_dispatch: x [T][d] -> (rows [T*K][l] bf16 in expert
+        order, counts [N] int32), both on the device (async)."""
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != self.cfg.d or not x.is_cuda:
+            raise ValueError("x: need CUDA bf16 [T][d]")
+        x = x.contiguous()
+        T, K = x.shape[0], self.cfg.top_k
+        if rows_out is None:
+            rows_out = torch.empty((T * K, self.cfg.latent), dtype=torch.bfloat16,
+                                   device=x.device)
+        if counts_out is None:
+            counts_out = torch.empty((self.cfg.n_experts,), dtype=torch.int32, device=x.device)
+        check(self.lib.lmoe_forward_dispatch(self.h, c_void_p(x.data_ptr()), T,
+                                             c_void_p(rows_out.data_ptr()),
+                                             c_void_p(counts_out.data_ptr()),
+                                             _stream_ptr(stream)), "lmoe_forward_dispatch")
+        self.last_T = T
+        return rows_out, counts_out
+
+    def combine(self, rows_in: torch.Tensor, out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """lmoe_forward_combine: the unweighted expert outputs [T*K][l] in the
+        last dispatch's row order -> y [T][d] (async)."""
+        T = self.last_T
+        if rows_in.dtype != torch.bfloat16 or tuple(rows_in.shape) != (T * self.cfg.top_k,
+                                                                        self.cfg.latent):
+            raise ValueError("rows_in: need bf16 [T*K][l] of the last dispatch")
+        rows_in = rows_in.contiguous()
+        if out is None:
+            out = torch.empty((T, self.cfg.d), dtype=torch.bfloat16, device=rows_in.device)
+        check(self.lib.lmoe_forward_combine(self.h, c_void_p(rows_in.data_ptr()), T,
+                                            c_void_p(out.data_ptr()), _stream_ptr(stream)),
+              "lmoe_forward_combine")
+        return out
 
     # -- backward ---------------------------------------------------------
     GRAD_NAMES = ("d_router", "d_dn", "d_w1", "d_w2", "d_upl", "d_s1", "d_s2")
@@ -213,6 +259,85 @@ class LatentMoE:
             self.close()
         except Exception:
             pass
+
+
+class ExpertShard:
+    """lmoe_experts_create / lmoe_experts_forward: the experts
+    [first, first + n_local) of a layer, run on rows handed in by an
+    expert-parallel exchange.  w1 [n_local][h][l], w2 [n_local][l][h] CUDA
+    bf16 (copied)."""
+
+    def __init__(self, d: int, latent: int, n_experts: int, top_k: int, expert_hidden: int,
+                 shared_hidden: int, first: int, w1: torch.Tensor, w2: torch.Tensor,
+                 max_rows: int):
+        self.lib = _lib.load()
+        n = w1.shape[0]
+        if w1.dtype != torch.bfloat16 or w2.dtype != torch.bfloat16 or not w1.is_cuda \
+                or tuple(w1.shape) != (n, expert_hidden, latent) \
+                or tuple(w2.shape) != (n, latent, expert_hidden) \
+                or not (w1.is_contiguous() and w2.is_contiguous()):
+            raise ValueError("w1 [n][h][l], w2 [n][l][h]: contiguous CUDA bf16")
+        self.cfg = LmoeConfig(d, latent, n_experts, top_k, expert_hidden, shared_hidden,
+                              FMT_BF16, 0, 1)
+        self.first, self.n_local, self.device = first, n, w1.device
+        h = c_void_p()
+        with torch.cuda.device(self.device):
+            check(self.lib.lmoe_experts_create(byref(self.cfg), first, n,
+                                               c_void_p(w1.data_ptr()), c_void_p(w2.data_ptr()),
+                                               int(max_rows), byref(h)), "lmoe_experts_create")
+        self.h = h
+
+    def forward(self, rows: torch.Tensor, counts: torch.Tensor,
+                out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """rows [R][l] bf16 in local expert order, counts [n_local] int32 (both
+        CUDA) -> out [R][l] bf16, the unweighted expert outputs (async)."""
+        if rows.dtype != torch.bfloat16 or counts.dtype != torch.int32 or not rows.is_cuda:
+            raise ValueError("rows: CUDA bf16 [R][l]; counts: CUDA int32 [n_local]")
+        rows = rows.contiguous()
+        if out is None:
+            out = torch.empty_like(rows)
+        check(self.lib.lmoe_experts_forward(self.h, c_void_p(rows.data_ptr()),
+                                            c_void_p(counts.data_ptr()), rows.shape[0],
+                                            c_void_p(out.data_ptr()), _stream_ptr(stream)),
+              "lmoe_experts_forward")
+        return out
+
+    def sync_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
+        return self.lib.lmoe_sync_status(self.h, _stream_ptr(stream))
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            self.lib.lmoe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def lmoe_permute_rows(src: torch.Tensor, idx: torch.Tensor, scatter: bool,
+                      out: Optional[torch.Tensor] = None, out_rows: Optional[int] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """lmoe_permute_rows on CUDA row tensors: gather out[r] = src[idx[r]]
+    (len(idx) rows out), or scatter out[idx[r]] = src[r] (out_rows rows)."""
+    if idx.dtype != torch.int32 or not idx.is_cuda or not src.is_cuda:
+        raise ValueError("idx: CUDA int32; src: CUDA")
+    src = src.contiguous()
+    n = idx.numel()
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else 0
+    if out is None:
+        rows = (out_rows if out_rows is not None else src.shape[0]) if scatter else n
+        out = src.new_empty((rows,) + tuple(src.shape[1:]))
+    n_other = out.shape[0] if scatter else src.shape[0]
+    if n == 0:
+        return out
+    check(_lib.load().lmoe_permute_rows(c_void_p(src.data_ptr()), c_void_p(idx.data_ptr()), n,
+                                        n_other, row_bytes, c_void_p(out.data_ptr()),
+                                        int(scatter), _stream_ptr(stream)), "lmoe_permute_rows")
+    return out
 
 
 def lmoe_route(logits: torch.Tensor, bias: Optional[torch.Tensor], K: int,

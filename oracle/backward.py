@@ -42,11 +42,34 @@ import numpy as np
 
 from .lmoe import route, sqrelu
 
-__all__ = ["layer_backward", "bias_update", "BIAS_UPDATE_RATE"]
+__all__ = ["layer_backward", "expert_backward", "bias_update", "BIAS_UPDATE_RATE"]
 
 # "Nemotron-3 Super 精读报告", table 6.3: update rate of the aux-loss-free
 # balancing strategy
 BIAS_UPDATE_RATE = 1e-3
+
+
+def expert_backward(U: np.ndarray, dV: np.ndarray, w: np.ndarray, W1e: np.ndarray,
+                    W2e: np.ndarray) -> Dict[str, np.ndarray]:
+    """One expert's part of the backward, over the n routed rows that chose it.
+
+    U [n][l]: the rows' expert inputs u; dV [n][l]: dL/dv of the rows' tokens;
+    w [n]: the rows' router weights; W1e [h][l], W2e [l][h].  Per row (the
+    expert lines of the table above): a = W1e u, g = sqrelu(a), o = W2e g,
+    dw = dv . o, do = w dv, dW2e = sum do g^T, da = (W2e^T do) * 2 max(a, 0),
+    dW1e = sum da u^T, du = W1e^T da.
+    Returns o [n][l], dw [n], dW1 [h][l], dW2 [l][h], du [n][l], and the
+    factors of the weight gradients: do [n][l], g [n][h], da [n][h].
+    """
+    a = U @ W1e.T                                        # [n][h]
+    g = sqrelu(a)
+    o = g @ W2e.T                                        # [n][l]
+    dw = np.sum(dV * o, axis=1)
+    do = w[:, None] * dV                                 # [n][l]
+    dW2 = do.T @ g
+    da = (do @ W2e) * 2.0 * np.maximum(a, 0.0)           # [n][h]
+    return {"o": o, "dw": dw, "dW1": da.T @ U, "dW2": dW2, "du": da @ W1e, "do": do, "g": g,
+            "da": da}
 
 
 def layer_backward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
@@ -99,17 +122,13 @@ def layer_backward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
     for e in np.unique(S):
         e = int(e)
         tok, slot = np.nonzero(S == e)
-        W1e, W2e = get_w1(e), get_w2(e)
-        a = u[tok] @ W1e.T                               # [n][h]
-        g = sqrelu(a)
-        o = g @ W2e.T                                    # [n][l]
-        v[tok] += w[tok, slot][:, None] * o
-        dw[tok, slot] = np.sum(dv[tok] * o, axis=1)
-        do = w[tok, slot][:, None] * dv[tok]             # [n][l]
-        dW2[e] = do.T @ g
-        da = (do @ W2e) * 2.0 * np.maximum(a, 0.0)       # [n][h]
-        dW1[e] = da.T @ u[tok]
-        du[tok] += da @ W1e
+        ex = expert_backward(u[tok], dv[tok], w[tok, slot], get_w1(e), get_w2(e))
+        v[tok] += w[tok, slot][:, None] * ex["o"]
+        dw[tok, slot] = ex["dw"]
+        dW2[e] = ex["dW2"]
+        dW1[e] = ex["dW1"]
+        # a token selects e at most once, so tok has no repeats here
+        du[tok] += ex["du"]
     dW_upl = G.T @ v if latent else None
     if latent:
         dW_dn = du.T @ x

@@ -182,3 +182,96 @@ def check_segments_valid(layer, T, N, K):
     same = seg_e[1:] == seg_e[:-1]
     assert np.all(tok[1:][same] > tok[:-1][same])
     return counts
+
+
+# ---------------------------------------------------------------------------
+# quantised layers at full size: the oracle's expert quantisers cost seconds
+# per Super-width matrix, so each touched expert is quantised once, in a pool
+# of spawned processes (never forked: the parent holds a CUDA context)
+
+def _bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 values given as their 16-bit patterns -> float64 (exact)."""
+    return (bits.astype(np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _quantised_expert_rows(args):
+    """Worker: one expert's quantised FFN on the latent rows U that chose it,
+    as the oracle's own one-expert layer (N = 1, K = 1: every row takes the
+    expert with weight 1; no projections, so its u is U itself; a zero-width
+    shared expert contributes nothing).  Returns (e, o [n][l])."""
+    e, w1_bits, w2_bits, U, quant = args
+    W1e = _bf16_bits_to_f64(w1_bits)
+    W2e = _bf16_bits_to_f64(w2_bits)
+    l = U.shape[1]
+    out = O.layer_forward(U, np.zeros((1, l)), None, None, lambda _: W1e, lambda _: W2e, None,
+                          np.zeros((1, l)), np.zeros((l, 1)), 1, quant=quant)
+    return e, out["v"]
+
+
+def oracle_tokens_pooled(w, x_rows: torch.Tensor, K: int, quant, S_use: np.ndarray,
+                         workers: int = 16):
+    """The oracle layer on the given token rows with the selected experts
+    S_use ([n][K], already checked to be a valid top-K set per token): the
+    router, projections and shared expert as in oracle.lmoe.layer_forward,
+    each expert's quantised FFN from _quantised_expert_rows, and
+    v = sum_k w_k o_k with w renormalised from the oracle's scores."""
+    import multiprocessing as mp
+    x64 = to64(x_rows)
+    z = x64 @ to64(w["w_router"]).T
+    _, _, gap, s = O.route(z, to64(w["router_bias"]), K)
+    S_use = np.asarray(S_use, dtype=np.int64)
+    s_sel = np.take_along_axis(s, S_use, axis=1)
+    wk = s_sel / s_sel.sum(axis=1, keepdims=True)
+    u = x64 @ to64(w["w_dn"]).T
+    jobs = []
+    for e in np.unique(S_use):
+        tok = np.nonzero((S_use == e).any(axis=1))[0]
+        jobs.append((int(e), w["w1"][int(e)].view(torch.int16).cpu().numpy(),
+                     w["w2"][int(e)].view(torch.int16).cpu().numpy(), u[tok], quant))
+    v = np.zeros_like(u)
+    with mp.get_context("spawn").Pool(min(workers, len(jobs))) as pool:
+        for e, o in pool.imap_unordered(_quantised_expert_rows, jobs):
+            tok, slot = np.nonzero(S_use == e)
+            v[tok] += wk[tok, slot][:, None] * o
+    hs = O.sqrelu(x64 @ to64(w["w_s1"]).T)
+    y = v @ to64(w["w_upl"]).T + hs @ to64(w["w_s2"]).T
+    return {"v": v, "y": y, "u": u, "hs": hs, "s": s, "gap": gap, "w": wk}
+
+
+def compare_layer_pooled(layer, w, x, y, tokens, K, tol, quant):
+    """compare_layer for quantised experts at full size, with the pooled
+    oracle: routing checked first (equal outside the gap window, a valid
+    top-K inside it), then y, u and hs against the oracle with the GPU's
+    selected experts.  Returns the measured errors."""
+    tokens = np.asarray(tokens)
+    gi = layer.debug("topk_idx").numpy().astype(np.int64)[tokens]
+    gw = layer.debug("topk_w").numpy()[tokens]
+    z = to64(x[tokens]) @ to64(w["w_router"]).T
+    S_o, w_o, gap, s = O.route(z, to64(w["router_bias"]), K)
+    key = s + to64(w["router_bias"])[None, :]
+    n_tie_diff = 0
+    for i in range(len(tokens)):
+        same = sorted(gi[i].tolist()) == sorted(S_o[i].tolist())
+        if gap[i] > GAP:
+            assert same, f"token {tokens[i]}: routing {sorted(gi[i])} != {sorted(S_o[i])}"
+        if same:
+            ref_w = dict(zip(S_o[i].tolist(), w_o[i].tolist()))
+            for e, wv in zip(gi[i].tolist(), gw[i].tolist()):
+                assert abs(wv - ref_w[e]) <= W_TOL, (tokens[i], e, wv, ref_w[e])
+        else:
+            n_tie_diff += 1
+            assert O.is_valid_topk(key[i], gi[i], GAP), f"token {tokens[i]}: invalid top-K"
+    o = oracle_tokens_pooled(w, x[tokens], K, quant, gi)
+    errs = {"y_maxerr_over_rms": max_rel(to64(y)[tokens], o["y"]),
+            "near_tie_sets_differing": n_tie_diff, "tokens": len(tokens)}
+    for k in ("u", "hs"):
+        got = to64(layer.debug(k))[tokens]
+        ok, ratio, rr = elem_ok(got, o[k])
+        errs[k + "_err_over_bound"] = ratio
+        errs[k + "_rms_rel"] = rr
+        assert ok, f"{k}: elementwise error {ratio:.3g} x bound, RMS rel error {rr:.3g}"
+    got_v = to64(layer.debug("v"))[tokens]
+    errs["v_rms_rel"] = rms_rel(got_v, o["v"])
+    assert errs["y_maxerr_over_rms"] <= tol, \
+        f"y: max|err|/RMS = {errs['y_maxerr_over_rms']:.3g} > {tol}"
+    return errs

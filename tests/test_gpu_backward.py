@@ -150,3 +150,44 @@ def test_bias_update_matches_oracle():
     layer.forward(x)
     counts2 = layer.debug("counts").numpy()
     assert counts2.max() <= counts.max()
+
+
+def test_backward_with_an_underflowing_selected_score():
+    """A selected expert whose sigmoid score underflows to 0 in float32 (its
+    logit near -128, chosen through a large bias): its router weight is 0 and
+    the router backward must stay finite (dz = 0 there, since s (1 - s) = 0)."""
+    from lmoe_synth import CONFIGS, make_grad_out
+    cfg = CONFIGS["tiny"]
+
+    def router(t):
+        t = t.clone()
+        t[3] = -0.5           # z[:, 3] = -0.5 * sum(x): about -128 for x = 1
+        return t
+
+    def bias(t):
+        t = t.clone()
+        t[3] = 10.0           # expert 3 is always selected
+        return t
+
+    w, x, layer = make(cfg, backward=True, overrides={"w_router": router, "router_bias": bias})
+    x = x.clone()
+    x[:4] = 1.0
+    layer.forward(x)
+    dy = make_grad_out(cfg, T=x.shape[0], device="cuda")
+    grads = layer.grad_buffers()
+    dx = layer.backward(x, dy, grads)
+    torch.cuda.synchronize()
+    assert layer.sync_status() == 0
+    S = layer.debug("topk_idx").numpy().astype(np.int64)
+    assert np.all(S[:, 0] == 3)
+    assert np.all(layer.debug("topk_w").numpy()[:4, 0] == 0.0)
+    ref = B.layer_backward(to64(x), to64(w["w_router"]), to64(w["router_bias"]), to64(w["w_dn"]),
+                           lambda e: to64(w["w1"][e]), lambda e: to64(w["w2"][e]),
+                           to64(w["w_upl"]), to64(w["w_s1"]), to64(w["w_s2"]), cfg.K, to64(dy),
+                           S=S)
+    for name, got in (("dx", to64(dx)), ("dW_r", to64(grads["d_router"])),
+                      ("dW_dn", to64(grads["d_dn"]))):
+        assert np.isfinite(got).all(), f"{name}: non-finite"
+        rb, ab = (ROUTER_RMS_BAR, ROUTER_ABS_RMS) if name == "dW_r" else (RMS_BAR, ABS_RMS)
+        ok, ratio, rr = elem_ok(got, ref[name], rel=REL_ELEM, abs_rms=ab, rel_rms=rb)
+        assert ok, f"{name}: RMS rel {rr:.3g}, elementwise {ratio:.3g} x bound"

@@ -164,7 +164,7 @@ def test_super_decode_sampled_tokens(super_decode):
     assert layer.sync_status() == 0
 
 
-@pytest.mark.parametrize("name,n", [("super_prefill", 16), ("ultra", 8)])
+@pytest.mark.parametrize("name,n", [("super_prefill", 16), ("ultra", 16)])
 def test_large_configs_sampled_tokens(name, n):
     cfg = CONFIGS[name]
     w, x, layer = make(cfg)

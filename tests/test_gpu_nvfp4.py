@@ -10,7 +10,8 @@ import torch
 from lmoe_synth import CONFIGS
 from oracle import nvfp4 as Q
 
-from _parity import check_segments_valid, compare_layer, make, quant_of, rms_rel, to64
+from _parity import (check_segments_valid, compare_layer, compare_layer_pooled, make, quant_of,
+                     rms_rel, to64)
 
 pytestmark = pytest.mark.gpu
 TOL_NVFP4 = 6e-2
@@ -110,9 +111,8 @@ def test_super_prefill_nvfp4_sampled_tokens():
     counts = check_segments_valid(layer, cfg.T, cfg.N, cfg.K)
     assert (counts == 0).any()
     rng = np.random.default_rng(1000 + cfg.seed)
-    toks = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 10, replace=False)]))
-    errs = compare_layer(layer, w, x, y, toks, cfg.K, tol=TOL_NVFP4, quant=quant_of(cfg),
-                         check_v=False)
+    toks = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 16, replace=False)]))
+    errs = compare_layer_pooled(layer, w, x, y, toks, cfg.K, tol=TOL_NVFP4, quant=quant_of(cfg))
     print("super_prefill_nvfp4", errs)
     assert errs["v_rms_rel"] <= TOL_NVFP4
     layer.close()
