@@ -39,6 +39,7 @@
 
 #include "nvfp4.cuh"
 #include "ptx.cuh"
+#include "route.cuh"
 
 namespace lmoe {
 
@@ -601,6 +602,64 @@ __global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__
   }
   TileInfo t{};
   epi.store8(t, r, feat, v, valid);
+}
+
+// Split-K reduction of the router GEMM [W_r; W_dn; W_s1] x with the router
+// fused into it.  Blocks [0, rblocks) take one token per warp: its N logits,
+// the K slices summed in slice order (as k_splitk_reduce), written as fp32
+// logits and held in the lanes (expert lane + 32 i) for the warp's top-K,
+// scores and renormalised weights (route_select).  The other blocks reduce
+// features [N, F) and apply the epilogue, a thread per 8 features of a row.
+template <class Epi, int NPL>
+__global__ void __launch_bounds__(256) k_splitk_reduce_route(
+    const float* __restrict__ part, int ksplit, int T, int F, int N, const Epi epi,
+    const float* __restrict__ bias, int K, float* __restrict__ logits,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int rblocks) {
+  pdl_wait();
+  pdl_trigger();
+  if (static_cast<int>(blockIdx.x) < rblocks) {
+    const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const int npl = N >> 5;
+    float zz[NPL], bb[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      zz[i] = 0.0f;
+      bb[i] = (i < npl && bias) ? bias[lane + 32 * i] : 0.0f;
+    }
+    for (int sl = 0; sl < ksplit; ++sl) {
+      const float* p = part + (static_cast<int64_t>(sl) * T + t) * F;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i)
+        if (i < npl) zz[i] += p[lane + 32 * i];
+    }
+    float* zrow = logits + t * N;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (i < npl) zrow[lane + 32 * i] = zz[i];
+    __syncwarp();   // the row's logits, written by all lanes, are read back below
+    route_select<NPL>(zz, bb, npl, zrow, K, lane, t, topk_idx, topk_w);
+    return;
+  }
+  const long g = static_cast<long>(blockIdx.x - rblocks) * blockDim.x + threadIdx.x;
+  const int f8 = (F - N) / 8;
+  const long row = g / f8;
+  const bool valid = row < T;
+  const long r = valid ? row : 0;
+  const int feat = N + (valid ? static_cast<int>(g - row * f8) * 8 : 0);
+  float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (valid) {
+    for (int sl = 0; sl < ksplit; ++sl) {
+      const float4* p =
+          reinterpret_cast<const float4*>(part + (static_cast<long>(sl) * T + r) * F + feat);
+      const float4 a = p[0], b = p[1];
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+  }
+  TileInfo ti{};
+  epi.store8(ti, r, feat, v, valid);
 }
 
 // ---------------------------------------------------------------------------

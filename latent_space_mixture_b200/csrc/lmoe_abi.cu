@@ -521,6 +521,24 @@ cudaError_t launch_reduce(const float* part, int ksplit, int T, int F, const Epi
   return launch_pdl(k_splitk_reduce<Epi>, blocks, 256, 0, st, part, ksplit, T, F, epi);
 }
 
+// the x-GEMM's split-K reduction with the router's top-K fused (N <= 1024)
+template <class Epi>
+cudaError_t launch_reduce_route(const float* part, int ksplit, int T, int F, int N,
+                                const Epi& epi, const float* bias, int K, float* logits,
+                                int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+  const int rblocks = (T + 7) / 8;
+  const long threads = static_cast<long>(T) * ((F - N) / 8);
+  const unsigned blocks = static_cast<unsigned>(rblocks + (threads + 255) / 256);
+  if (N <= 32 * 4)
+    return launch_pdl(k_splitk_reduce_route<Epi, 4>, blocks, 256, 0, st, part, ksplit, T, F, N,
+                      epi, bias, K, logits, topk_idx, topk_w, rblocks);
+  if (N <= 32 * 16)
+    return launch_pdl(k_splitk_reduce_route<Epi, 16>, blocks, 256, 0, st, part, ksplit, T, F, N,
+                      epi, bias, K, logits, topk_idx, topk_w, rblocks);
+  return launch_pdl(k_splitk_reduce_route<Epi, 32>, blocks, 256, 0, st, part, ksplit, T, F, N,
+                    epi, bias, K, logits, topk_idx, topk_w, rblocks);
+}
+
 template <class Epi>
 cudaError_t set_smem_all() {
   cudaError_t e;
@@ -647,7 +665,8 @@ using namespace lmoe;
 static const char* const kKernelNames[] = {
     "xgemm(router|W_dn|W_s1)", "route(sigmoid+bias+topK)", "hist", "scan", "scatter",
     "gather(u->expert order)", "grouped_gemm1(W1,sqrelu)", "grouped_gemm2(W2,*w)",
-    "combine", "ygemm([W_upl|W_s2])", "xgemm split-K reduce", "ygemm split-K reduce",
+    "combine", "ygemm([W_upl|W_s2])", "xgemm split-K reduce + route(sigmoid+bias+topK)",
+    "ygemm split-K reduce",
     // backward
     "bw dgrad [W_upl|W_s2]^T (dv, dhs)", "bw gather(w dv -> expert order)",
     "bw dgrad W2^T (dg)", "bw dgrad W1^T (du rows)", "bw combine(du)", "bw route(dz)",
@@ -1175,7 +1194,8 @@ int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T) {
   const DensePlan px = plan_dense(T, (c.n_experts + h->lx + c.shared_hidden + 127) / 128,
                                   c.d / 64, h->sms);
   const DensePlan py = plan_dense(T, (c.d + 127) / 128, (h->lx + c.shared_hidden) / 64, h->sms);
-  return 10 + (px.ksplit > 1) + (py.ksplit > 1);
+  (void)px;   // a split x-GEMM's reduction replaces the router kernel: same count
+  return 10 + (py.ksplit > 1);
 }
 
 static int prof_begin(lmoe_handle* h, int kernel, cudaStream_t st) {
@@ -1223,6 +1243,7 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st) 
     return LMOE_ERR_CUDA;
   }
   h->last_T = T;
+  bool routed = false;   // the top-K ran inside the x-GEMM's split-K reduction
 
   // 1. [W_r; W_dn; W_s1] x: logits, u, shared hidden
   {
@@ -1244,13 +1265,17 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st) 
     const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
     const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
     LMOE_STEP(0, launch_gemm_bn(p.bn, h->tm_wx, tm_x, s, epi, grid, h->err, lim, st));
+    // at split-K sizes the reduction also routes: logits, top-K, weights
     if (p.ksplit > 1)
-      LMOE_STEP(10, launch_reduce(h->part, p.ksplit, static_cast<int>(T), N + lx + hs, epi, st));
+      LMOE_STEP(10, launch_reduce_route(h->part, p.ksplit, static_cast<int>(T), N + lx + hs, N,
+                                        epi, h->bias, K, h->logits, h->topk_idx, h->topk_w, st));
+    routed = p.ksplit > 1;
     }
   }
   // 2-5. routing and segments
   const int gbn = grouped_bn(c, T);
-  LMOE_STEP(1, launch_route(h->logits, h->bias, T, N, K, h->topk_idx, h->topk_w, st));
+  if (!routed)
+    LMOE_STEP(1, launch_route(h->logits, h->bias, T, N, K, h->topk_idx, h->topk_w, st));
   LMOE_STEP(2, launch_hist(h->topk_idx, T, N, K, h->chunk, h->err, st));
   LMOE_STEP(3, launch_scan(h->chunk, T, N, h->counts, st));
   LMOE_STEP(4, launch_scatter(h->topk_idx, h->topk_w, h->chunk, h->counts, T, N, K, gbn,
