@@ -243,6 +243,30 @@ int lmoe_bias_update(lmoe_handle* h, float rate, void* stream);
 #define LMOE_DBG_W2Q_SF 15
 #define LMOE_DBG_W2Q_G 16
 #define LMOE_DBG_BIAS 17
+/* and of the last lmoe_experts_backward_nvfp4 (R = T K routed rows in expert
+ * order, C = columns of the transposed operands, lmoe_nvfp4_bw_columns):
+ *   LMOE_DBG_BW4_DO_CODES u8  [R][l/2]   NVFP4 codes of w dv (stochastic)
+ *   LMOE_DBG_BW4_DO_SF    u8  [R][l/16]  their E4M3 scales
+ *   LMOE_DBG_BW4_DOT_CODES u8 [l][C/2]   codes of the transformed (w dv)^T
+ *   LMOE_DBG_BW4_DOT_SF   u8  [l][C/16]
+ *   LMOE_DBG_BW4_UT_CODES u8  [l][C/2]   codes of the transformed u^T
+ *   LMOE_DBG_BW4_UT_SF    u8  [l][C/16]
+ *   LMOE_DBG_BW4_SCALES   fp32 [16]      amax of w dv, da, (w dv)^T, g^T,
+ *                                        da^T, u^T, two unused, then their
+ *                                        global scales in the same order
+ *   LMOE_DBG_BW4_SEG      int32 [2][N+1] column offsets of the experts in the
+ *                                        transposed operands, segments
+ *                                        padded to 16, then to 256
+ *   LMOE_DBG_BW4_DA       fp32 [R][h]    da = (W2q^T Q(w dv)) 2 max(a, 0) */
+#define LMOE_DBG_BW4_DO_CODES 18
+#define LMOE_DBG_BW4_DO_SF 19
+#define LMOE_DBG_BW4_DOT_CODES 20
+#define LMOE_DBG_BW4_DOT_SF 21
+#define LMOE_DBG_BW4_UT_CODES 22
+#define LMOE_DBG_BW4_UT_SF 23
+#define LMOE_DBG_BW4_SCALES 24
+#define LMOE_DBG_BW4_SEG 25
+#define LMOE_DBG_BW4_DA 26
 int lmoe_get_debug(lmoe_handle* h, int what, void* dst_host, size_t bytes);
 
 /* Kernel launches one lmoe_forward of T tokens issues, or a negative error
@@ -412,6 +436,39 @@ int lmoe_experts_forward(lmoe_handle* h, const void* rows, const int32_t* counts
  * src, dst 16-byte aligned, not overlapping.  Errors: INVALID_ARG, CUDA. */
 int lmoe_permute_rows(const void* src, const int32_t* idx, int64_t n, int64_t n_other,
                       int32_t row_bytes, void* dst, int scatter, void* stream);
+
+/* The routed experts' forward and backward under the NVFP4 training recipe
+ * ("Nemotron-3 Super 精读报告", section 5.3: fprop, dgrad and wgrad GEMMs in
+ * NVFP4; weights in 2D 16 x 16 blocks, whose one scale serves W and W^T;
+ * activations and gradients in 1D blocks along each GEMM's reduction axis; a
+ * random Hadamard transform on the weight-gradient GEMMs' inputs; stochastic
+ * rounding of the gradients).  A handle with LMOE_FMT_NVFP4,
+ * LMOE_FLAG_NVFP4_WEIGHT_2D and LMOE_FLAG_BACKWARD (else UNSUPPORTED).
+ * Inputs (device): u [T][l] bf16 latent rows, topk_idx [T][K] int32 selected
+ * experts (distinct per token), topk_w [T][K] fp32 router weights, dv [T][l]
+ * bf16 = dL/dv.  The forward: u and sqrelu(W1q u) quantised with the
+ * handle's static scales (act_gscale_*), o = W2q g per routed row.  The
+ * backward, rows in expert order (expert, token, slot):
+ *   dw[t][k] = o . dv[t];  do = w dv, stochastically rounded with global
+ *   scale amax / (6 * 448) and the counters of seed + 0;  da = (W2q^T Q(do))
+ *   2 max(a, 0), a = W1q u, stochastically rounded (seed + 1);
+ *   du[t] = sum over t's rows of W1q^T Q(da);
+ *   dW2[e] = Q_sr(R(do_e^T)) Q(R(g_e^T))^T, dW1[e] = Q_sr(R(da_e^T))
+ *   Q(R(u_e^T))^T over expert e's rows, R the transform on 16-row blocks
+ *   (signs of seed + 2 for dW2, seed + 4 for dW1), stochastic rounding with
+ *   seed + 3 (do^T) and seed + 5 (da^T), element (f, j) of an operand taking
+ *   the counter of its place in the layout whose expert segments are padded
+ *   to 16 rows; every tensor's global scale is its amax / (6 * 448).
+ * Outputs (device): du [T][l] bf16, dw [T][K] fp32, d_w1 [N][h][l] and d_w2
+ * [N][l][h] fp32 (zero for experts without rows).  Asynchronous on `stream`;
+ * 16-byte aligned pointers.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+int lmoe_experts_backward_nvfp4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
+                                const float* topk_w, const void* dv, int64_t T, uint64_t seed,
+                                void* du, float* dw, float* d_w1, float* d_w2, void* stream);
+
+/* Columns C of the transposed weight-gradient operands of an NVFP4 training
+ * handle (the row pitch of LMOE_DBG_BW4_*T_*), or a negative error code. */
+int64_t lmoe_nvfp4_bw_columns(const lmoe_handle* h);
 
 /* Frees everything the handle owns (synchronizes the device first). */
 void lmoe_destroy(lmoe_handle* h);

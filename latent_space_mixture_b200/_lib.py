@@ -23,7 +23,9 @@ NVFP4_WEIGHT_FLAGS = {"1d": 0, "2d": FLAG_NVFP4_WEIGHT_2D, "mse": FLAG_NVFP4_WEI
                       "2d_mse": FLAG_NVFP4_WEIGHT_2D | FLAG_NVFP4_WEIGHT_MSE}
 DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 6,
        "logits": 7, "u": 8, "v": 9, "hs": 10, "w1q_codes": 11, "w1q_sf": 12, "w1q_g": 13,
-       "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16, "bias": 17}
+       "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16, "bias": 17,
+       "bw4_do_codes": 18, "bw4_do_sf": 19, "bw4_dot_codes": 20, "bw4_dot_sf": 21,
+       "bw4_ut_codes": 22, "bw4_ut_sf": 23, "bw4_scales": 24, "bw4_seg": 25, "bw4_da": 26}
 
 
 class LmoeConfig(Structure):
@@ -82,6 +84,10 @@ SIGNATURES = {
                                      c_void_p]),
     "lmoe_permute_rows": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int32, c_void_p,
                                   c_int, c_void_p]),
+    "lmoe_experts_backward_nvfp4": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                            c_int64, c_uint64, c_void_p, c_void_p, c_void_p,
+                                            c_void_p, c_void_p]),
+    "lmoe_nvfp4_bw_columns": (c_int64, [c_void_p]),
     "lmoe_nvfp4_quantize": (c_int, [c_void_p, c_int64, c_int32, c_float, c_void_p, c_void_p,
                                     c_void_p]),
     "lmoe_rht16": (c_int, [c_void_p, c_int64, c_int32, c_uint64, c_void_p, c_void_p]),

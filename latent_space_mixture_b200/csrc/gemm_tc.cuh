@@ -66,7 +66,8 @@ constexpr int FP4_SF_STAGE_BYTES = 4 * SF_ATOM_BYTES;   // 4 chunks of K=64
 
 // Where the tiles of one GEMM come from.
 struct TileSource {
-  int dense;               // 1: tokens [0, T) in blocks of BN; 0: device block list
+  int dense;               // 1: tokens [0, T) in blocks of BN; 0: device block list;
+                           // 2: per-group K ranges (weight gradients, below)
   int T;                   // dense: number of token rows
   const int4* blocks;      // list: {expert, first row, rows, 0}
   const int* nblocks;      // list: number of blocks (device scalar)
@@ -80,6 +81,13 @@ struct TileSource {
   const uint8_t* sfa;      // NVFP4: A scale atoms, [A row / 128][kc][512 B]
   const uint8_t* sfb;      // NVFP4: B scale atoms, [token block][kc][512 B]
   int kc;                  // NVFP4: 64-element chunks per row (4 x kblocks)
+  // dense == 2: `groups` groups (experts) share one A matrix (features) and
+  // one B matrix of b_rows rows; group g reduces over its own K range, k-steps
+  // [kofs[g], kofs[g + 1]) (device array), and writes its own output; a group
+  // with an empty range has no tiles (every role skips them)
+  const int* kofs = nullptr;
+  int groups = 0;
+  int b_rows = 0;
 };
 
 struct TileInfo {
@@ -87,6 +95,7 @@ struct TileInfo {
 };
 
 __device__ __forceinline__ int gemm_num_tiles(const TileSource& s, int BN) {
+  if (s.dense == 2) return s.groups * ((s.b_rows + BN - 1) / BN) * s.FB;
   const int nb = s.dense ? (s.T + BN - 1) / BN : *s.nblocks;
   return nb * s.FB * s.ksplit;
 }
@@ -96,6 +105,21 @@ __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int t
   TileInfo t;
   const int tk = tile / s.FB;
   t.fb = tile - tk * s.FB;
+  if (s.dense == 2) {
+    // (group, B row block, feature block), feature block fastest
+    const int nbb = (s.b_rows + BN - 1) / BN;
+    const int g = tk / nbb;
+    const int tb = tk - g * nbb;
+    t.tb = tb;
+    t.ks = 0;
+    t.kb0 = s.kofs[g];
+    t.kb1 = s.kofs[g + 1];
+    t.e = g;
+    t.row0 = tb * BN;
+    t.nrows = min(BN, s.b_rows - t.row0);
+    t.a_row = t.fb * GEMM_BM;
+    return t;
+  }
   const int tb = tk / s.ksplit;
   t.tb = tb;
   t.ks = tk - tb * s.ksplit;
@@ -369,6 +393,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     bool issued_any = false;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const TileInfo t = gemm_tile(src, BN, tile);
+      if (t.kb0 >= t.kb1) continue;   // an empty K range: no accumulator, no epilogue
       const int n_mma = (t.nrows + 15) & ~15;
       if (!__all_sync(0xffffffffu,
                       mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err, limit_ns))) {
@@ -464,6 +489,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const TileInfo t = gemm_tile(src, BN, tile);
+      if (t.kb0 >= t.kb1) continue;   // skipped by the MMA warp too
       // one lane waits, the warp follows: the TMEM loads below are .sync.aligned
       int ok = 0;
       if (lane == 0) ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err, limit_ns);

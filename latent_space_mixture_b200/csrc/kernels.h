@@ -81,6 +81,45 @@ cudaError_t launch_gather_q(const uint8_t* uq, const uint8_t* usf, const int32_t
                             const int32_t* rblock, int64_t rows, int K, int l, int lp,
                             uint8_t* u_perm_q, uint8_t* atoms, cudaStream_t st);
 
+// NVFP4 training backward (nvfp4_bw.cu): see that file for the layouts.
+cudaError_t launch_quant_rows_bf16(const void* x, int64_t rows, int cols, float g, uint8_t* codes,
+                                   int code_pitch, uint8_t* scales, cudaStream_t st);
+cudaError_t launch_rows_scaled(const void* dv, const int32_t* perm, const float* wrow, int64_t R,
+                               int K, int l, float* out, float* amax, cudaStream_t st);
+cudaError_t launch_quant_rows_dev(const float* x, int64_t rows, int cols, const float* amax,
+                                  bool sr, uint64_t seed, uint8_t* codes, int code_pitch,
+                                  uint8_t* scales, float* g_out, cudaStream_t st);
+cudaError_t launch_atoms_rblock(const uint8_t* scales, const int32_t* rblock, int64_t R, int nkb,
+                                int kp64, uint8_t* atoms, cudaStream_t st);
+cudaError_t launch_atoms_dense(const uint8_t* scales, int64_t rows, int nkb, uint8_t* atoms,
+                               cudaStream_t st);
+cudaError_t launch_dw_rows(const void* O, const int32_t* inv, const void* dv, int64_t T, int K,
+                           int l, float* dw, cudaStream_t st);
+cudaError_t launch_seg_offsets(const int32_t* counts, int N, int32_t* po16, int32_t* po256,
+                               int32_t* kofs, cudaStream_t st);
+struct TSrc {
+  const void* p;           // rows: fp32 [R][F], bf16 token rows [T][F], or NVFP4 codes
+  const int32_t* perm;     // bf16 token rows: routed row -> t * K + k
+  const int32_t* rblock;   // NVFP4 rows: (token block << 8) | row in block
+  const uint8_t* atoms;    // NVFP4 rows: B-operand scale atoms
+  int K;
+  int code_pitch;          // NVFP4 rows: bytes per row of codes
+  int fp64;                // NVFP4 rows: 64-element chunks per row of the atoms
+  float g;                 // NVFP4 rows: global scale
+};
+cudaError_t launch_transpose_rht(int src_kind, const TSrc& s, const int32_t* offsets,
+                                 const int32_t* counts, const int32_t* po256, int N, int F,
+                                 int64_t pitch, uint64_t seed, float* out, float* amax,
+                                 cudaStream_t st);
+cudaError_t launch_quant_t(const float* x, int F, int64_t pitch, const int32_t* po16,
+                           const int32_t* po256, int N, const float* amax, bool sr, uint64_t seed,
+                           uint8_t* codes, uint8_t* scales, float* g_out, cudaStream_t st);
+cudaError_t launch_zero_empty(const int32_t* counts, int N, int64_t per, float* dw,
+                              cudaStream_t st);
+cudaError_t launch_transpose_w2d(const uint8_t* codes, const uint8_t* atoms, int E, int R, int C,
+                                 int Cp, int Rp, uint8_t* tcodes, uint8_t* tatoms,
+                                 cudaStream_t st);
+
 // Backward pass (backward.cu).  dst[r] = wrow[r] * dv[perm[r] / K], rows of
 // width l (bf16, l % 8 == 0).
 cudaError_t launch_gather_scaled(const void* dv, const int32_t* perm, const float* wrow,

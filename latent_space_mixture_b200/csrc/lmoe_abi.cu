@@ -149,6 +149,8 @@ struct EpiHq {
   const float* gw1;
   float g_u, g_h;
   int hp;   // h rounded up to 256 (row pitch hp/2 bytes)
+  bf16* a16 = nullptr;   // NVFP4 training: the pre-activation a = W1[e] u, bf16 [R][ha]
+  int ha = 0;
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
                                          bool valid) const {
     const float s = __fmul_rn(gw1[t.e], g_u);
@@ -158,6 +160,12 @@ struct EpiHq {
     uint8_t sc;
     const uint32_t codes = nvfp4_pair(a, g_h, &sc);
     if (!valid) return;
+    if (a16) {
+      float pre[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pre[i] = v[i] * s;
+      store8_bf16(a16 + row * ha + feat, pre);
+    }
     *reinterpret_cast<uint32_t*>(Hq + row * (hp / 2) + feat / 2) = codes;
     if ((feat & 15) == 0)
       sfh[(static_cast<long>(t.tb) * (hp / 64) + feat / 64) * SF_ATOM_BYTES +
@@ -177,11 +185,87 @@ struct EpiOq {
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
                                          bool valid) const {
     if (!valid) return;
-    const float s = __fmul_rn(__fmul_rn(gw2[t.e], g_h), wrow[row]);
+    // no weights: the experts' unweighted outputs (the NVFP4 backward's o)
+    const float s = __fmul_rn(__fmul_rn(gw2[t.e], g_h), wrow ? wrow[row] : 1.0f);
     float a[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = v[i] * s;
     store8_bf16(O + row * l + feat, a);
+  }
+};
+
+// NVFP4 backward, data gradient of FC2: dg = g_W2[e] g_do * acc (the FP4
+// product W2q^T Q(do)), and the pre-activation gradient da = dg 2 max(a, 0)
+// in fp32 [R][h], with its amax (a warp maximum, then one atomic per warp).
+struct EpiDA {
+  static constexpr int kWarps = 8;
+  float* da;
+  const bf16* a16;
+  const float* gw2;
+  const float* g_do;   // device scalar
+  int h;
+  float* amax;
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    float m = 0.0f;
+    if (valid) {
+      const float s = __fmul_rn(gw2[t.e], *g_do);
+      const uint4 raw = *reinterpret_cast<const uint4*>(a16 + row * h + feat);
+      const __nv_bfloat162* ap = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 a = __bfloat1622float2(ap[i]);
+        o[2 * i] = __fmul_rn(__fmul_rn(v[2 * i] * s, 2.0f), fmaxf(a.x, 0.0f));
+        o[2 * i + 1] = __fmul_rn(__fmul_rn(v[2 * i + 1] * s, 2.0f), fmaxf(a.y, 0.0f));
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(o[i]));
+      float4* p = reinterpret_cast<float4*>(da + row * h + feat);
+      p[0] = make_float4(o[0], o[1], o[2], o[3]);
+      p[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    // the atomic only when it would raise the maximum
+    if ((threadIdx.x & 31) == 0 && __float_as_int(m) > *reinterpret_cast<volatile int*>(amax))
+      atomicMax(reinterpret_cast<int*>(amax), __float_as_int(m));
+  }
+};
+
+// NVFP4 backward, data gradient of FC1: du rows = g_W1[e] g_da * acc (bf16)
+struct EpiDU {
+  static constexpr int kWarps = 8;
+  bf16* du;
+  const float* gw1;
+  const float* g_da;   // device scalar
+  int l;
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(gw1[t.e], *g_da);
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = v[i] * s;
+    store8_bf16(du + row * l + feat, o);
+  }
+};
+
+// NVFP4 weight gradient of one expert (group): out[e][row][feat] =
+// g_a g_b * acc, fp32, row = B row, feat = A row.
+struct EpiWq {
+  static constexpr int kWarps = 8;
+  float* out;
+  int rows, cols;
+  const float* g_a;   // device scalars
+  const float* g_b;
+  __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(*g_a, *g_b);
+    float4* p = reinterpret_cast<float4*>(out + (static_cast<long>(t.e) * rows + row) * cols + feat);
+    p[0] = make_float4(v[0] * s, v[1] * s, v[2] * s, v[3] * s);
+    p[1] = make_float4(v[4] * s, v[5] * s, v[6] * s, v[7] * s);
   }
 };
 
@@ -773,6 +857,37 @@ struct lmoe_handle {
   bf16* dy_dev = nullptr;    // [64][d]     staging of dy for T < 64
   CUtensorMap tm_wx64, tm_wy64, tm_w1_64, tm_w2_64;   // weights in 64-row boxes
   BMaps tm_dog, tm_da, tm_dxh;
+  // NVFP4 training (NVFP4 experts, 2D weight blocks, LMOE_FLAG_BACKWARD):
+  // transposed weights, the backward's rows and transposed operands
+  bool bw4 = false;
+  uint8_t* w1qT = nullptr;     // [N*l][hp/2] codes of W1[e]^T
+  uint8_t* w1qT_sf = nullptr;  // [N*l/128][hp/64][512]
+  uint8_t* w2qT = nullptr;     // [N*h][lp/2] codes of W2[e]^T
+  uint8_t* w2qT_sf = nullptr;  // [N*h/128][lp/64][512]
+  bf16* a16 = nullptr;         // [rows_b][h] pre-activations W1[e] u
+  float* do32 = nullptr;       // [rows][l] w dv rows
+  uint8_t* doq = nullptr;      // [rows_b][lp/2]
+  uint8_t* doS = nullptr;      // [rows][l/16]
+  uint8_t* sfbdo = nullptr;    // [token blocks][lp/64][512]
+  float* da32 = nullptr;       // [rows][h]
+  uint8_t* daq = nullptr;      // [rows_b][hp/2]
+  uint8_t* daS = nullptr;      // [rows][h/16]
+  uint8_t* sfbda = nullptr;    // [token blocks][hp/64][512]
+  int32_t* po16 = nullptr;     // [N+1] columns, segments padded to 16
+  int32_t* po256 = nullptr;    // [N+1] columns, segments padded to 256
+  int32_t* kofs = nullptr;     // [N+1] FP4 k-steps of po256
+  float* scal = nullptr;       // [16]: amax 0..7, global scales 8..15
+  int64_t rp_cap = 0;          // columns of the transposed operands
+  float* X1 = nullptr;         // [max(l,h)][rp_cap] fp32 transposed, transformed
+  float* X2 = nullptr;
+  // transposed operands: 0 do^T (B of dW2), 1 g^T (A of dW2), 2 u^T (A of
+  // dW1), 3 da^T (B of dW1): codes [F][rp_cap/2], scales [F][rp_cap/16], atoms
+  uint8_t* tq[4] = {};
+  uint8_t* ts[4] = {};
+  uint8_t* ta[4] = {};
+  CUtensorMap tm_w1qT, tm_w2qT, tm_tA[4];
+  BMaps tm_doq, tm_daq, tm_tB[4];
+  int64_t bw4_T = -1;          // T of the last lmoe_experts_backward_nvfp4
   std::vector<void*> allocs;
   CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
   BMaps tm_uperm, tm_H, tm_vh;
@@ -836,7 +951,9 @@ static int check_cfg(const lmoe_config* c) {
       (c->latent != c->d || c->expert_format != LMOE_FMT_BF16))
     return LMOE_ERR_UNSUPPORTED;
   if ((c->flags & LMOE_FLAG_BACKWARD) &&
-      ((c->flags & LMOE_FLAG_NO_PROJECTION) || c->expert_format != LMOE_FMT_BF16))
+      ((c->flags & LMOE_FLAG_NO_PROJECTION) ||
+       !(c->expert_format == LMOE_FMT_BF16 ||
+         (c->expert_format == LMOE_FMT_NVFP4 && (c->flags & LMOE_FLAG_NVFP4_WEIGHT_2D)))))
     return LMOE_ERR_UNSUPPORTED;
   if (c->top_k > c->n_experts) return LMOE_ERR_INVALID_ARG;
   if (c->expert_format != LMOE_FMT_BF16 && c->expert_format != LMOE_FMT_NVFP4 &&
@@ -952,8 +1069,22 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   }
   h->part_floats = part_floats;
   const int64_t max_blocks = rows / 32 + N + 1;
-  const int64_t bwd = (c.flags & LMOE_FLAG_BACKWARD) ? 1 : 0;
+  // the BF16 backward's workspace, or the NVFP4 training backward's
+  const int64_t bwd = ((c.flags & LMOE_FLAG_BACKWARD) && bfx) ? 1 : 0;
+  const int64_t bw4 = ((c.flags & LMOE_FLAG_BACKWARD) && fp4) ? 1 : 0;
   h->bw = bwd != 0;
+  h->bw4 = bw4 != 0;
+  // transposed operands of the NVFP4 weight gradients: every expert's rows
+  // padded to 256 columns; the transform kernels take a 16-column block per
+  // grid row (at most 65535)
+  const int64_t rp_cap = bw4 ? (rows + 255 * N + 255) / 256 * 256 : 0;
+  if (rp_cap / 16 > 65535) {
+    delete h;
+    return LMOE_ERR_UNSUPPORTED;
+  }
+  h->rp_cap = rp_cap;
+  const int64_t fmax = l > hh ? l : hh;
+  const int64_t tf[4] = {l, hh, l, hh};   // features of the transposed operands
   struct Req {
     void** p;
     size_t bytes;
@@ -1012,6 +1143,37 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->dwacc, size_t(bwd * rows * 4)},
       {(void**)&h->dxh, size_t(bwd * Tm_b * (N + l + hs) * 2)},
       {(void**)&h->dy_dev, size_t(bwd * GEMM_BROWS_BIG * d * 2)},
+      {(void**)&h->w1qT, size_t(bw4 * N * l * hp / 2)},
+      {(void**)&h->w1qT_sf, size_t(bw4 * (N * l / 128) * (hp / 64) * 512)},
+      {(void**)&h->w2qT, size_t(bw4 * N * hh * lp / 2)},
+      {(void**)&h->w2qT_sf, size_t(bw4 * (N * hh / 128) * (lp / 64) * 512)},
+      {(void**)&h->a16, size_t(bw4 * rows_b * hh * 2)},
+      {(void**)&h->do32, size_t(bw4 * rows * l * 4)},
+      {(void**)&h->doq, size_t(bw4 * rows_b * lp / 2)},
+      {(void**)&h->doS, size_t(bw4 * rows * l / 16)},
+      {(void**)&h->sfbdo, size_t(bw4 * nb_max * (lp / 64) * 512)},
+      {(void**)&h->da32, size_t(bw4 * rows * hh * 4)},
+      {(void**)&h->daq, size_t(bw4 * rows_b * hp / 2)},
+      {(void**)&h->daS, size_t(bw4 * rows * hh / 16)},
+      {(void**)&h->sfbda, size_t(bw4 * nb_max * (hp / 64) * 512)},
+      {(void**)&h->po16, size_t(bw4 * (N + 1) * 4)},
+      {(void**)&h->po256, size_t(bw4 * (N + 1) * 4)},
+      {(void**)&h->kofs, size_t(bw4 * (N + 1) * 4)},
+      {(void**)&h->scal, size_t(bw4 * 64)},
+      {(void**)&h->X1, size_t(bw4 * fmax * rp_cap * 4)},
+      {(void**)&h->X2, size_t(bw4 * fmax * rp_cap * 4)},
+      {(void**)&h->tq[0], size_t(bw4 * tf[0] * rp_cap / 2)},
+      {(void**)&h->tq[1], size_t(bw4 * tf[1] * rp_cap / 2)},
+      {(void**)&h->tq[2], size_t(bw4 * tf[2] * rp_cap / 2)},
+      {(void**)&h->tq[3], size_t(bw4 * tf[3] * rp_cap / 2)},
+      {(void**)&h->ts[0], size_t(bw4 * tf[0] * rp_cap / 16)},
+      {(void**)&h->ts[1], size_t(bw4 * tf[1] * rp_cap / 16)},
+      {(void**)&h->ts[2], size_t(bw4 * tf[2] * rp_cap / 16)},
+      {(void**)&h->ts[3], size_t(bw4 * tf[3] * rp_cap / 16)},
+      {(void**)&h->ta[0], size_t(bw4 * tf[0] * rp_cap / 16)},
+      {(void**)&h->ta[1], size_t(bw4 * tf[1] * rp_cap / 16)},
+      {(void**)&h->ta[2], size_t(bw4 * tf[2] * rp_cap / 16)},
+      {(void**)&h->ta[3], size_t(bw4 * tf[3] * rp_cap / 16)},
   };
   for (auto& r : reqs) {
     if ((rc = alloc_dev(h, r.p, r.bytes)) != LMOE_OK) {
@@ -1089,6 +1251,35 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       ok &= set_gemm_smem<32, EpiHq, KIND_NVFP4>() == cudaSuccess;
       ok &= set_gemm_smem<128, EpiOq, KIND_NVFP4>() == cudaSuccess;
       ok &= set_gemm_smem<32, EpiOq, KIND_NVFP4>() == cudaSuccess;
+      if (bw4) {
+        // the dgrad GEMMs read W^T: a 2D block's scale serves both orientations
+        ok &= cudaMemset(h->doq, 0, rows_b * lp / 2) == cudaSuccess;
+        ok &= cudaMemset(h->daq, 0, rows_b * hp / 2) == cudaSuccess;
+        ok &= cudaMemset(h->sfbdo, 0, nb_max * (lp / 64) * 512) == cudaSuccess;
+        ok &= cudaMemset(h->sfbda, 0, nb_max * (hp / 64) * 512) == cudaSuccess;
+        ok &= launch_transpose_w2d(h->w1q, h->w1sf, static_cast<int>(N), static_cast<int>(hh),
+                                   static_cast<int>(l), static_cast<int>(lp),
+                                   static_cast<int>(hp), h->w1qT, h->w1qT_sf, 0) == cudaSuccess;
+        ok &= launch_transpose_w2d(h->w2q, h->w2sf, static_cast<int>(N), static_cast<int>(l),
+                                   static_cast<int>(hh), static_cast<int>(hp),
+                                   static_cast<int>(lp), h->w2qT, h->w2qT_sf, 0) == cudaSuccess;
+        ok &= make_map_u8(&h->tm_w1qT, h->w1qT, N * l, hp / 2, GEMM_BM);
+        ok &= make_map_u8(&h->tm_w2qT, h->w2qT, N * hh, lp / 2, GEMM_BM);
+        ok &= make_map_u8(&h->tm_doq.b16, h->doq, rows_b, lp / 2, GEMM_BROWS);
+        ok &= make_map_u8(&h->tm_doq.b64, h->doq, rows_b, lp / 2, GEMM_BROWS_BIG);
+        ok &= make_map_u8(&h->tm_daq.b16, h->daq, rows_b, hp / 2, GEMM_BROWS);
+        ok &= make_map_u8(&h->tm_daq.b64, h->daq, rows_b, hp / 2, GEMM_BROWS_BIG);
+        for (int i = 0; i < 4; ++i) {
+          ok &= make_map_u8(&h->tm_tA[i], h->tq[i], tf[i], rp_cap / 2, GEMM_BM);
+          ok &= make_map_u8(&h->tm_tB[i].b16, h->tq[i], tf[i], rp_cap / 2, GEMM_BROWS);
+          ok &= make_map_u8(&h->tm_tB[i].b64, h->tq[i], tf[i], rp_cap / 2, GEMM_BROWS_BIG);
+        }
+        ok &= set_gemm_smem<128, EpiDA, KIND_NVFP4>() == cudaSuccess;
+        ok &= set_gemm_smem<32, EpiDA, KIND_NVFP4>() == cudaSuccess;
+        ok &= set_gemm_smem<128, EpiDU, KIND_NVFP4>() == cudaSuccess;
+        ok &= set_gemm_smem<32, EpiDU, KIND_NVFP4>() == cudaSuccess;
+        ok &= set_gemm_smem<128, EpiWq, KIND_NVFP4>() == cudaSuccess;
+      }
     } else {
       // W4A16: code tiles of one k-step (64 elements = 32 bytes) x 128 rows
       ok &= make_map_codes(&h->tm_w1c, h->w1q, N * hh, lp / 2);
@@ -1810,6 +2001,148 @@ int lmoe_permute_rows(const void* src, const int32_t* idx, int64_t n, int64_t n_
              : LMOE_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// routed experts' forward and backward under the NVFP4 training recipe
+
+int lmoe_experts_backward_nvfp4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
+                                const float* topk_w, const void* dv, int64_t T, uint64_t seed,
+                                void* du, float* dw, float* d_w1, float* d_w2, void* stream) {
+  if (!h || h->shard || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+  if (!h->bw4) return LMOE_ERR_UNSUPPORTED;
+  if (!d_w1 || !d_w2 || (T > 0 && (!u || !topk_idx || !topk_w || !dv || !du || !dw)))
+    return LMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(dv) |
+       reinterpret_cast<uintptr_t>(du) | reinterpret_cast<uintptr_t>(d_w1) |
+       reinterpret_cast<uintptr_t>(d_w2)) & 15)
+    return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const lmoe_config& c = h->cfg;
+  const int N = c.n_experts, l = c.latent, hh = c.expert_hidden, K = c.top_k;
+  const int lp = h->lp, hp = h->hp;
+  const int64_t R = T * K;
+  const int64_t pitch = h->rp_cap;
+  const unsigned long long lim = h->wait_limit_ns;
+  h->bw4_T = T;
+  if (T == 0) {
+    // no rows: every weight gradient is zero
+    if (cudaMemsetAsync(d_w1, 0, size_t(N) * hh * l * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(d_w2, 0, size_t(N) * l * hh * 4, st) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    return LMOE_OK;
+  }
+  if (cudaMemsetAsync(h->scal, 0, 64, st) != cudaSuccess) return LMOE_ERR_CUDA;
+  float* amax = h->scal;        // 0 do, 1 da, 2 do^T, 3 g^T, 4 da^T, 5 u^T
+  float* gsc = h->scal + 8;     // their global scales
+  const int gbn = grouped_bn(c, T);
+  // 1. segments of the given routing
+  LMOE_STEP(2, launch_hist(topk_idx, T, N, K, h->chunk, h->err, st));
+  LMOE_STEP(3, launch_scan(h->chunk, T, N, h->counts, st));
+  LMOE_STEP(4, launch_scatter(topk_idx, topk_w, h->chunk, h->counts, T, N, K, gbn, h->offsets,
+                              h->perm, h->inv, h->wrow, h->blocks, h->nblocks, h->rblock, h->err,
+                              st));
+  // 2. the experts' forward: u -> NVFP4, a = W1q u (kept), g = NVFP4(sqrelu a),
+  //    o = W2q g (unweighted)
+  LMOE_STEP(5, launch_quant_rows_bf16(u, T, l, h->g_u, h->uq, l / 2, h->usf, st));
+  LMOE_STEP(5, launch_gather_q(h->uq, h->usf, h->perm, h->rblock, R, K, l, lp, h->upq, h->sfbu,
+                               st));
+  {
+    TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, lp / 256, 1, nullptr,
+                 gbn == 32, h->w1sf, h->sfbu, lp / 64};
+    EpiHq epi{h->Hq, h->sfbh, h->gw1, h->g_u, h->g_h, hp, h->a16, hh};
+    LMOE_STEP(6, launch_gemm_q<KIND_NVFP4>(gbn, h->tm_w1q, h->tm_upq, s, epi, h->sms, h->err, lim,
+                                           st));
+  }
+  {
+    TileSource s{0, 0, h->blocks, h->nblocks, l / 128, l, l, hp / 256, 1, nullptr, gbn == 32,
+                 h->w2sf, h->sfbh, hp / 64};
+    EpiOq epi{h->O, nullptr, h->gw2, h->g_h, l};
+    LMOE_STEP(7, launch_gemm_q<KIND_NVFP4>(gbn, h->tm_w2q, h->tm_Hq, s, epi, h->sms, h->err, lim,
+                                           st));
+  }
+  // 3. dL/dw = o . dv
+  LMOE_STEP(17, launch_dw_rows(h->O, h->inv, dv, T, K, l, dw, st));
+  // 4. do = w dv rows, stochastically rounded to NVFP4 (1D blocks along l)
+  LMOE_STEP(13, launch_rows_scaled(dv, h->perm, h->wrow, R, K, l, h->do32, amax + 0, st));
+  LMOE_STEP(13, launch_quant_rows_dev(h->do32, R, l, amax + 0, true, seed + 0, h->doq, lp / 2,
+                                      h->doS, gsc + 0, st));
+  LMOE_STEP(13, launch_atoms_rblock(h->doS, h->rblock, R, l / 16, lp / 64, h->sfbdo, st));
+  // 5. dg = W2q^T Q(do); da = dg 2 max(a, 0) (fp32) and its amax
+  {
+    TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, lp / 256, 1, nullptr,
+                 gbn == 32, h->w2qT_sf, h->sfbdo, lp / 64};
+    EpiDA epi{h->da32, h->a16, h->gw2, gsc + 0, hh, amax + 1};
+    LMOE_STEP(14, launch_gemm_q<KIND_NVFP4>(gbn, h->tm_w2qT, h->tm_doq, s, epi, h->sms, h->err,
+                                            lim, st));
+  }
+  // 6. da stochastically rounded (1D blocks along h); du rows = W1q^T Q(da)
+  LMOE_STEP(23, launch_quant_rows_dev(h->da32, R, hh, amax + 1, true, seed + 1, h->daq, hp / 2,
+                                      h->daS, gsc + 1, st));
+  LMOE_STEP(23, launch_atoms_rblock(h->daS, h->rblock, R, hh / 16, hp / 64, h->sfbda, st));
+  {
+    TileSource s{0, 0, h->blocks, h->nblocks, l / 128, l, l, hp / 256, 1, nullptr, gbn == 32,
+                 h->w1qT_sf, h->sfbda, hp / 64};
+    EpiDU epi{h->O, h->gw1, gsc + 1, l};
+    LMOE_STEP(15, launch_gemm_q<KIND_NVFP4>(gbn, h->tm_w1qT, h->tm_daq, s, epi, h->sms, h->err,
+                                            lim, st));
+  }
+  // 7. du = sum of a token's rows
+  LMOE_STEP(16, launch_combine(h->O, h->inv, T, K, l, du, l, st));
+  // 8. weight gradients: per expert, over its rows (the K dimension),
+  //    transformed operands padded to 256-row segments
+  LMOE_STEP(20, launch_seg_offsets(h->counts, N, h->po16, h->po256, h->kofs, st));
+  const int64_t kc = pitch / 64;
+  TSrc src_do{h->do32, nullptr, nullptr, nullptr, K, 0, 0, 0.f};
+  TSrc src_g{h->Hq, nullptr, h->rblock, h->sfbh, K, hp / 2, hp / 64, h->g_h};
+  TSrc src_da{h->da32, nullptr, nullptr, nullptr, K, 0, 0, 0.f};
+  TSrc src_u{u, h->perm, nullptr, nullptr, K, 0, 0, 0.f};
+  // dW2[e] = Q_sr(R(do_e^T)) Q(R(g_e^T))^T: A = g^T (features h), B = do^T (rows l)
+  LMOE_STEP(20, launch_transpose_rht(2, src_g, h->offsets, h->counts, h->po256, N, hh, pitch,
+                                     seed + 2, h->X2, amax + 3, st));
+  LMOE_STEP(20, launch_transpose_rht(0, src_do, h->offsets, h->counts, h->po256, N, l, pitch,
+                                     seed + 2, h->X1, amax + 2, st));
+  LMOE_STEP(20, launch_quant_t(h->X2, hh, pitch, h->po16, h->po256, N, amax + 3, false, 0,
+                               h->tq[1], h->ts[1], gsc + 3, st));
+  LMOE_STEP(20, launch_atoms_dense(h->ts[1], hh, static_cast<int>(pitch / 16), h->ta[1], st));
+  LMOE_STEP(20, launch_quant_t(h->X1, l, pitch, h->po16, h->po256, N, amax + 2, true, seed + 3,
+                               h->tq[0], h->ts[0], gsc + 2, st));
+  LMOE_STEP(20, launch_atoms_dense(h->ts[0], l, static_cast<int>(pitch / 16), h->ta[0], st));
+  {
+    TileSource s{2, 0, nullptr, nullptr, hh / 128, 0, hh, 0, 1, nullptr, 0, h->ta[1], h->ta[0],
+                 static_cast<int>(kc), h->kofs, N, l};
+    EpiWq epi{d_w2, l, hh, gsc + 3, gsc + 2};
+    LMOE_STEP(20, launch_gemm_q<KIND_NVFP4>(128, h->tm_tA[1], h->tm_tB[0], s, epi, h->sms, h->err,
+                                            lim, st));
+  }
+  // dW1[e] = Q_sr(R(da_e^T)) Q(R(u_e^T))^T: A = u^T (features l), B = da^T (rows h)
+  LMOE_STEP(21, launch_transpose_rht(1, src_u, h->offsets, h->counts, h->po256, N, l, pitch,
+                                     seed + 4, h->X1, amax + 5, st));
+  LMOE_STEP(21, launch_transpose_rht(0, src_da, h->offsets, h->counts, h->po256, N, hh, pitch,
+                                     seed + 4, h->X2, amax + 4, st));
+  LMOE_STEP(21, launch_quant_t(h->X1, l, pitch, h->po16, h->po256, N, amax + 5, false, 0,
+                               h->tq[2], h->ts[2], gsc + 5, st));
+  LMOE_STEP(21, launch_atoms_dense(h->ts[2], l, static_cast<int>(pitch / 16), h->ta[2], st));
+  LMOE_STEP(21, launch_quant_t(h->X2, hh, pitch, h->po16, h->po256, N, amax + 4, true, seed + 5,
+                               h->tq[3], h->ts[3], gsc + 4, st));
+  LMOE_STEP(21, launch_atoms_dense(h->ts[3], hh, static_cast<int>(pitch / 16), h->ta[3], st));
+  {
+    TileSource s{2, 0, nullptr, nullptr, l / 128, 0, l, 0, 1, nullptr, 0, h->ta[2], h->ta[3],
+                 static_cast<int>(kc), h->kofs, N, hh};
+    EpiWq epi{d_w1, hh, l, gsc + 5, gsc + 4};
+    LMOE_STEP(21, launch_gemm_q<KIND_NVFP4>(128, h->tm_tA[2], h->tm_tB[3], s, epi, h->sms, h->err,
+                                            lim, st));
+  }
+  // experts without rows: zero gradients
+  LMOE_STEP(20, launch_zero_empty(h->counts, N, int64_t(l) * hh, d_w2, st));
+  LMOE_STEP(21, launch_zero_empty(h->counts, N, int64_t(hh) * l, d_w1, st));
+  return LMOE_OK;
+}
+
+int64_t lmoe_nvfp4_bw_columns(const lmoe_handle* h) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  return h->bw4 ? h->rp_cap : LMOE_ERR_UNSUPPORTED;
+}
+
 int lmoe_forward_host(lmoe_handle* h, const void* x_host, int64_t T, void* y_host, void* stream) {
   if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return LMOE_OK;
@@ -1863,8 +2196,39 @@ int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
     case LMOE_DBG_W2Q_SF: src = h->w2sf; want = (N * l / 128) * (h->hp / 64) * 512; break;
     case LMOE_DBG_BIAS: src = h->bias; want = N * 4; break;
     case LMOE_DBG_W2Q_G: src = h->fp8 ? h->sw2 : h->gw2; want = N * 4; break;
-    default: return LMOE_ERR_INVALID_ARG;
+    default: break;
   }
+  if (what >= LMOE_DBG_BW4_DO_CODES && what <= LMOE_DBG_BW4_DA) {
+    // the last lmoe_experts_backward_nvfp4
+    if (!h->bw4 || h->bw4_T < 0) return LMOE_ERR_INVALID_ARG;
+    const int64_t R = h->bw4_T * K, hh = c.expert_hidden, pc = h->rp_cap;
+    switch (what) {
+      case LMOE_DBG_BW4_DO_CODES: strided = true; want = R * l / 2; break;
+      case LMOE_DBG_BW4_DO_SF: src = h->doS; want = R * l / 16; break;
+      case LMOE_DBG_BW4_DOT_CODES: src = h->tq[0]; want = l * pc / 2; break;
+      case LMOE_DBG_BW4_DOT_SF: src = h->ts[0]; want = l * pc / 16; break;
+      case LMOE_DBG_BW4_UT_CODES: src = h->tq[2]; want = l * pc / 2; break;
+      case LMOE_DBG_BW4_UT_SF: src = h->ts[2]; want = l * pc / 16; break;
+      case LMOE_DBG_BW4_SCALES: src = h->scal; want = 64; break;
+      case LMOE_DBG_BW4_SEG: want = 2 * (N + 1) * 4; break;
+      case LMOE_DBG_BW4_DA: src = h->da32; want = R * hh * 4; break;
+    }
+    if (bytes != want) return LMOE_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LMOE_ERR_CUDA;
+    if (want == 0) return LMOE_OK;
+    cudaError_t e;
+    if (what == LMOE_DBG_BW4_DO_CODES)
+      e = cudaMemcpy2D(dst, l / 2, h->doq, h->lp / 2, l / 2, R, cudaMemcpyDeviceToHost);
+    else if (what == LMOE_DBG_BW4_SEG)
+      e = cudaMemcpy(dst, h->po16, (N + 1) * 4, cudaMemcpyDeviceToHost) == cudaSuccess
+              ? cudaMemcpy(static_cast<char*>(dst) + (N + 1) * 4, h->po256, (N + 1) * 4,
+                           cudaMemcpyDeviceToHost)
+              : cudaErrorUnknown;
+    else
+      e = cudaMemcpy(dst, src, want, cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+  }
+  if (!src && !strided) return LMOE_ERR_INVALID_ARG;
   if (what >= LMOE_DBG_W1Q_CODES && what <= LMOE_DBG_W2Q_G && !h->fp4 && !h->fp8 && !h->w4)
     return LMOE_ERR_INVALID_ARG;
   if ((what == LMOE_DBG_W1Q_SF || what == LMOE_DBG_W2Q_SF) && !h->fp4 && !h->w4)

@@ -256,38 +256,6 @@ cudaError_t launch_quant_rows(const float* x, int64_t rows, int cols, float g, u
 // take counters 0..15 (sign -1 when bit 63 is set); a uniform in [0, 1) is
 // the top 24 bits times 2^-24.
 
-__device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t ctr) {
-  uint64_t z = seed + (ctr + 1ull) * 0x9E3779B97F4A7C15ull;
-  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-  return z ^ (z >> 31);
-}
-
-__device__ __forceinline__ float uniform24(uint64_t seed, uint64_t ctr) {
-  return static_cast<float>(static_cast<uint32_t>(splitmix64(seed, ctr) >> 40)) *
-         5.9604644775390625e-8f;   // 2^-24
-}
-
-// Stochastic rounding of v to an E2M1 code (bit 3 = sign): the upper grid
-// neighbour with probability (|v| - lo) / (hi - lo), the lower otherwise;
-// |v| >= 6 saturates.  The probability is exact in float32 (hi - lo is a
-// power of two, |v| - lo is exact).
-__device__ __forceinline__ uint32_t e2m1_sr(float v, float u) {
-  const float mag = fabsf(v);
-  uint32_t code;
-  if (mag >= 6.0f) {
-    code = 7;
-  } else {
-    const int lo = mag < 0.5f ? 0 : mag < 1.0f ? 1 : mag < 1.5f ? 2 : mag < 2.0f ? 3
-                 : mag < 3.0f ? 4 : mag < 4.0f ? 5 : 6;
-    const float lo_v = e2m1_value(static_cast<uint32_t>(lo));
-    const float hi_v = e2m1_value(static_cast<uint32_t>(lo + 1));
-    const float p = __fdiv_rn(__fsub_rn(mag, lo_v), __fsub_rn(hi_v, lo_v));
-    code = static_cast<uint32_t>(u < p ? lo + 1 : lo);
-  }
-  return code | (signbit(v) ? 8u : 0u);
-}
-
 // One thread per 16-element block: y = (1/4) H16 (s * x) as float32
 // butterflies (stages 1, 2, 4, 8: (a, b) -> (a + b, a - b)).
 __global__ void __launch_bounds__(256) k_rht16(const float* __restrict__ x, int64_t nblocks,
@@ -304,24 +272,10 @@ __global__ void __launch_bounds__(256) k_rht16(const float* __restrict__ x, int6
     b[4 * j + 2] = f.z;
     b[4 * j + 3] = f.w;
   }
-#pragma unroll
-  for (int j = 0; j < 16; ++j)
-    if (splitmix64(seed, static_cast<uint64_t>(j)) >> 63) b[j] = -b[j];
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j & h) continue;
-      const float a = b[j], c = b[j + h];
-      b[j] = __fadd_rn(a, c);
-      b[j + h] = __fsub_rn(a, c);
-    }
-  }
+  rht16_block(b, seed);
   float4* dst = reinterpret_cast<float4*>(y + i * 16);
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    dst[j] = make_float4(b[4 * j] * 0.25f, b[4 * j + 1] * 0.25f, b[4 * j + 2] * 0.25f,
-                         b[4 * j + 3] * 0.25f);
+  for (int j = 0; j < 4; ++j) dst[j] = make_float4(b[4 * j], b[4 * j + 1], b[4 * j + 2], b[4 * j + 3]);
 }
 
 cudaError_t launch_rht16(const float* x, int64_t rows, int cols, uint64_t seed, float* y,

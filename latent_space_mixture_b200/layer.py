@@ -189,6 +189,37 @@ class LatentMoE:
                                      _stream_ptr(stream)), "lmoe_backward")
         return dx
 
+    def experts_backward_nvfp4(self, u: torch.Tensor, topk_idx: torch.Tensor,
+                               topk_w: torch.Tensor, dv: torch.Tensor, seed: int,
+                               stream: Optional[torch.cuda.Stream] = None
+                               ) -> Dict[str, torch.Tensor]:
+        """lmoe_experts_backward_nvfp4: the routed experts' forward and
+        backward under the NVFP4 training recipe, for u [T][l] bf16, topk_idx
+        [T][K] int32, topk_w [T][K] fp32, dv [T][l] bf16 (CUDA).  Returns du
+        [T][l] bf16, dw [T][K] fp32, d_w1 [N][h][l] and d_w2 [N][l][h] fp32
+        (async)."""
+        c = self.cfg
+        T = u.shape[0]
+        if u.dtype != torch.bfloat16 or dv.dtype != torch.bfloat16 or \
+                topk_idx.dtype != torch.int32 or topk_w.dtype != torch.float32:
+            raise ValueError("u, dv: bf16 [T][l]; topk_idx int32, topk_w fp32 [T][K]")
+        u, dv = u.contiguous(), dv.contiguous()
+        topk_idx, topk_w = topk_idx.contiguous(), topk_w.contiguous()
+        dev = u.device
+        out = {"du": torch.empty((T, c.latent), dtype=torch.bfloat16, device=dev),
+               "dw": torch.empty((T, c.top_k), dtype=torch.float32, device=dev),
+               "d_w1": torch.empty((c.n_experts, c.expert_hidden, c.latent),
+                                   dtype=torch.float32, device=dev),
+               "d_w2": torch.empty((c.n_experts, c.latent, c.expert_hidden),
+                                   dtype=torch.float32, device=dev)}
+        p = lambda t: c_void_p(t.data_ptr())  # noqa: E731
+        check(self.lib.lmoe_experts_backward_nvfp4(
+            self.h, p(u), p(topk_idx), p(topk_w), p(dv), T, int(seed), p(out["du"]),
+            p(out["dw"]), p(out["d_w1"]), p(out["d_w2"]), _stream_ptr(stream)),
+            "lmoe_experts_backward_nvfp4")
+        self.bw4_T = T
+        return out
+
     def bias_update(self, rate: float = 1e-3, stream: Optional[torch.cuda.Stream] = None) -> None:
         """lmoe_bias_update: aux-loss-free step of the router bias from the
         last forward's expert loads."""
@@ -228,6 +259,15 @@ class LatentMoE:
             "w2q_sf": (torch.uint8, ((N * l // 128) * (hp // 64) * 512,)),
             "w2q_g": (torch.float32, (N,)),
         })
+        if what.startswith("bw4_"):
+            R = getattr(self, "bw4_T", 0) * c.top_k
+            C = self.lib.lmoe_nvfp4_bw_columns(self.h)
+            spec.update({
+                "bw4_do_codes": (torch.uint8, (R, l // 2)), "bw4_do_sf": (torch.uint8, (R, l // 16)),
+                "bw4_dot_codes": (torch.uint8, (l, C // 2)), "bw4_dot_sf": (torch.uint8, (l, C // 16)),
+                "bw4_ut_codes": (torch.uint8, (l, C // 2)), "bw4_ut_sf": (torch.uint8, (l, C // 16)),
+                "bw4_scales": (torch.float32, (16,)), "bw4_seg": (torch.int32, (2, N + 1)),
+                "bw4_da": (torch.float32, (R, h))})
         spec = spec[what]
         out = torch.empty(spec[1], dtype=spec[0])
         check(self.lib.lmoe_get_debug(self.h, DBG[what], c_void_p(out.data_ptr()),

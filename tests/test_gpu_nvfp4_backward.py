@@ -1,0 +1,151 @@
+"""The routed experts' backward under the NVFP4 training recipe on the GPU
+(lmoe_experts_backward_nvfp4) against the oracle (oracle.backward_nvfp4),
+"Nemotron-3 Super 精读报告", section 5.3.
+
+Both sides get the same seeded inputs: latent rows u, the selected experts
+and their router weights, dL/dv, the layer's bf16 weights (2D 16 x 16 weight
+blocks) and the random-bit seed.
+
+Bit-exact: every quantised tensor whose input both sides compute exactly --
+w dv (its codes, E4M3 scales and global scale; stochastic rounding), the
+transformed and stochastically rounded (w dv)^T of the W2 weight gradient
+and the transformed u^T of the W1 weight gradient (codes in the oracle's
+layout, whose expert segments are padded to 16 rows where the GPU pads them
+to 256), and the experts' column offsets.
+
+Within a bar: the gradients du, dL/dw, dW1 and dW2, whose inputs pass through
+GEMMs (fp32 accumulation against the oracle's float64) before they are
+quantised again, so a quantisation boundary can fall between the two sides'
+values and move one code by a full step: relative RMS error <= 6e-2, the
+NVFP4 layer bar."""
+import numpy as np
+import pytest
+import torch
+
+from lmoe_synth import CONFIGS, act_global_scales, make_weights
+from oracle import backward_nvfp4 as B4
+from oracle import lmoe as O
+from oracle import nvfp4 as Q
+from oracle import nvfp4_train as TR
+
+pytestmark = pytest.mark.gpu
+
+TOL = 6e-2
+SEED = 1234
+
+
+def _gscale(X):
+    return np.float32(np.float32(np.max(np.abs(X))) / np.float32(2688.0))
+
+
+def _unpack(codes):
+    """packed bytes [..][n/2] (lower index in the low nibble) -> codes [..][n]"""
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.stack([c & 15, c >> 4], axis=-1).reshape(c.shape[:-1] + (c.shape[-1] * 2,))
+
+
+def _inputs(cfg, T, seed):
+    g = torch.Generator().manual_seed(seed)
+    sigma_u = cfg.std * np.sqrt(cfg.d)
+    u = (torch.randn((T, cfg.l), generator=g) * sigma_u).to(torch.bfloat16)
+    # Zipf-like expert choice, the last two experts never chosen
+    pr = torch.tensor([(1.0 + e) ** -1.1 for e in range(cfg.N - 2)] + [0.0, 0.0])
+    S = torch.stack([torch.multinomial(pr, cfg.K, replacement=False, generator=g)
+                     for _ in range(T)]).to(torch.int32)
+    s = torch.rand((T, cfg.K), generator=g) * 0.9 + 0.1
+    w = (s / s.sum(dim=1, keepdim=True)).to(torch.float32)
+    dv = (torch.randn((T, cfg.l), generator=g) * 0.05).to(torch.bfloat16)
+    return u, S, w, dv
+
+
+def _layer(cfg, w):
+    from latent_space_mixture_b200 import LatentMoE
+    return LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, 64, w, expert_format="nvfp4",
+                     act_gscales=act_global_scales(cfg), nvfp4_weights="2d", backward=True)
+
+
+def _rms_rel(a, b):
+    return float(np.sqrt(np.mean((a - b) ** 2) / max(np.mean(b ** 2), 1e-300)))
+
+
+@pytest.mark.parametrize("T", [64, 37])
+def test_nvfp4_experts_backward_matches_oracle(T):
+    cfg = CONFIGS["tiny_nvfp4"].with_(wq="2d")
+    w, _ = make_weights(cfg, device="cuda")
+    layer = _layer(cfg, w)
+    u, S, wt, dv = _inputs(cfg, T, 50 + T)
+    out = layer.experts_backward_nvfp4(u.cuda(), S.cuda(), wt.cuda(), dv.cuda(), SEED)
+    torch.cuda.synchronize()
+    assert layer.sync_status() == 0
+    g_u, g_h = (float(np.float32(x)) for x in act_global_scales(cfg))
+    U64, S64 = u.double().numpy(), S.numpy().astype(np.int64)
+    w64, dv64 = wt.double().numpy(), dv.double().numpy()
+    w1 = lambda e: w["w1"][e].double().cpu().numpy()  # noqa: E731
+    w2 = lambda e: w["w2"][e].double().cpu().numpy()  # noqa: E731
+    ref = B4.experts_backward_nvfp4(U64, S64, w64, dv64, w1, w2, cfg.N, g_u, g_h, SEED)
+
+    # ---- bit-exact: the quantised tensors of exactly shared inputs --------
+    counts, offsets, perm, inv = O.segments(S64, cfg.N)
+    tok, slot = perm // cfg.K, perm % cfg.K
+    DO = (w64[tok, slot][:, None] * dv64[tok]).astype(np.float32)
+    g_do = _gscale(DO)
+    codes, sc, _ = TR.quantize_sr(DO, g_do, SEED + B4.SEEDS["do"])
+    assert np.array_equal(_unpack(layer.debug("bw4_do_codes").numpy()), codes)
+    assert np.array_equal(layer.debug("bw4_do_sf").numpy(), sc)
+    scal = layer.debug("bw4_scales").numpy()
+    assert scal[8] == g_do
+
+    seg = layer.debug("bw4_seg").numpy()
+    DOt, po = B4._padded_t(DO.astype(np.float64), offsets, counts)
+    assert np.array_equal(seg[0], po)
+    pc = (counts + 15) // 16 * 16
+    DOt = TR.rht16(DOt.astype(np.float32), seed=SEED + B4.SEEDS["rht_w2"])
+    g_dot = _gscale(DOt)
+    dot_codes, dot_sc, _ = TR.quantize_sr(DOt, g_dot, SEED + B4.SEEDS["do_t"])
+    Ut, _ = B4._padded_t(U64[tok], offsets, counts)
+    Ut = TR.rht16(Ut.astype(np.float32), seed=SEED + B4.SEEDS["rht_w1"])
+    g_ut = _gscale(Ut)
+    ut_codes, ut_sc, _ = Q.quantize(Ut, g_ut)
+    assert scal[10] == g_dot and scal[13] == g_ut
+    got_dot = _unpack(layer.debug("bw4_dot_codes").numpy())
+    got_dot_sc = layer.debug("bw4_dot_sf").numpy()
+    got_ut = _unpack(layer.debug("bw4_ut_codes").numpy())
+    got_ut_sc = layer.debug("bw4_ut_sf").numpy()
+    for e in np.nonzero(counts)[0]:
+        a, b, n = seg[1][e], po[e], pc[e]          # GPU columns, oracle columns, 16-padded rows
+        assert np.array_equal(got_dot[:, a:a + n], dot_codes[:, b:b + n]), e
+        assert np.array_equal(got_dot_sc[:, a // 16:(a + n) // 16], dot_sc[:, b // 16:(b + n) // 16])
+        assert np.array_equal(got_ut[:, a:a + n], ut_codes[:, b:b + n]), e
+        assert np.array_equal(got_ut_sc[:, a // 16:(a + n) // 16], ut_sc[:, b // 16:(b + n) // 16])
+
+    # ---- gradients within the NVFP4 bar ----------------------------------
+    errs = {"dw": _rms_rel(out["dw"].double().cpu().numpy(), ref["dw"]),
+            "du": _rms_rel(out["du"].double().cpu().numpy(), ref["du"])}
+    chosen = sorted(ref["dW1"].keys())
+    gw1, gw2 = out["d_w1"].cpu().double().numpy(), out["d_w2"].cpu().double().numpy()
+    errs["dW1"] = _rms_rel(gw1[chosen], np.stack([ref["dW1"][e] for e in chosen]))
+    errs["dW2"] = _rms_rel(gw2[chosen], np.stack([ref["dW2"][e] for e in chosen]))
+    unused = sorted(set(range(cfg.N)) - set(chosen))
+    assert len(unused) >= 2
+    assert not gw1[unused].any() and not gw2[unused].any()
+    print("nvfp4 backward T", T, errs)
+    for k, v in errs.items():
+        assert v <= TOL, (k, v)
+    layer.close()
+
+
+def test_nvfp4_experts_backward_no_rows_and_requirements():
+    from latent_space_mixture_b200 import LatentMoE, LmoeError
+    cfg = CONFIGS["tiny_nvfp4"].with_(wq="2d")
+    w, _ = make_weights(cfg, device="cuda")
+    layer = _layer(cfg, w)
+    z = torch.zeros((0, cfg.l), dtype=torch.bfloat16, device="cuda")
+    out = layer.experts_backward_nvfp4(z, torch.zeros((0, cfg.K), dtype=torch.int32, device="cuda"),
+                                       torch.zeros((0, cfg.K), device="cuda"), z, SEED)
+    torch.cuda.synchronize()
+    assert not out["d_w1"].any() and not out["d_w2"].any()
+    layer.close()
+    # 1D weight blocks have no transposable scales: no NVFP4 training handle
+    with pytest.raises(LmoeError):
+        LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, 64, w, expert_format="nvfp4",
+                  act_gscales=act_global_scales(cfg), nvfp4_weights="1d", backward=True)
