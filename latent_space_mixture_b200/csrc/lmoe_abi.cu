@@ -76,6 +76,22 @@ struct EpiX {
   }
 };
 
+// shared expert FC1 alone (W_s1 x, on the side stream of an overlapped
+// forward): sqrelu into columns [l, l + h_s) of vh
+struct EpiS1 {
+  static constexpr int kWarps = 4;
+  bf16* vh;
+  int l, ldvh;
+  __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
+                                         bool valid) const {
+    if (!valid) return;
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = sqrelu(v[i]);
+    store8_bf16(vh + row * ldvh + l + feat, a);
+  }
+};
+
 // expert FC1: H[row] = sqrelu(W1[e] u[row])
 struct EpiH {
   static constexpr int kWarps = 4;
@@ -755,8 +771,10 @@ static const char* const kKernelNames[] = {
     "bw dgrad [W_upl|W_s2]^T (dv, dhs)", "bw gather(w dv -> expert order)",
     "bw dgrad W2^T (dg)", "bw dgrad W1^T (du rows)", "bw combine(du)", "bw route(dz)",
     "bw dgrad [W_r;W_dn;W_s1]^T (dx)", "bw wgrad [W_upl|W_s2]", "bw wgrad W2",
-    "bw wgrad W1", "bw wgrad [W_r;W_dn;W_s1]", "bw act'(da = dg 2 sqrt(g), dw)"};
-static constexpr int kNumKernels = 24;
+    "bw wgrad W1", "bw wgrad [W_r;W_dn;W_s1]", "bw act'(da = dg 2 sqrt(g), dw)",
+    // overlapped forward: the shared expert on the side stream
+    "shared W_s1 (side stream)", "shared W_s2 (side stream)"};
+static constexpr int kNumKernels = 26;
 
 // Dense-GEMM plan for T tokens: token-block width and number of K slices.
 // Enough tiles to fill the GPU first by narrower token blocks (while one
@@ -888,6 +906,13 @@ struct lmoe_handle {
   CUtensorMap tm_w1qT, tm_w2qT, tm_tA[4];
   BMaps tm_doq, tm_daq, tm_tB[4];
   int64_t bw4_T = -1;          // T of the last lmoe_experts_backward_nvfp4
+  // overlapped forward (BF16 experts bound by HBM): the shared expert's two
+  // GEMMs on a side stream over a share of the SMs
+  cudaStream_t side_st = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  bf16* ys = nullptr;          // [max_tokens][d] W_s2 hs
+  CUtensorMap tm_ws1, tm_ws2;  // W_s1 rows of w_x; W_s2 columns of w_y
+  BMaps tm_hs;                 // hs columns of vh
   std::vector<void*> allocs;
   CUtensorMap tm_wx, tm_w1, tm_w2, tm_wy;
   BMaps tm_uperm, tm_H, tm_vh;
@@ -929,6 +954,11 @@ static int alloc_dev(lmoe_handle* h, void** p, size_t bytes) {
 static void free_all(lmoe_handle* h) {
   for (void* p : h->allocs) cudaFree(p);
   h->allocs.clear();
+  if (h->side_st) cudaStreamDestroy(h->side_st);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  h->side_st = nullptr;
+  h->ev_fork = h->ev_join = nullptr;
   for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
   h->ev.clear();
 }
@@ -1143,6 +1173,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->dwacc, size_t(bwd * rows * 4)},
       {(void**)&h->dxh, size_t(bwd * Tm_b * (N + l + hs) * 2)},
       {(void**)&h->dy_dev, size_t(bwd * GEMM_BROWS_BIG * d * 2)},
+      {(void**)&h->ys, size_t((bfx && proj) ? Tm * d * 2 : 0)},
       {(void**)&h->w1qT, size_t(bw4 * N * l * hp / 2)},
       {(void**)&h->w1qT_sf, size_t(bw4 * (N * l / 128) * (hp / 64) * 512)},
       {(void**)&h->w2qT, size_t(bw4 * N * hh * lp / 2)},
@@ -1326,6 +1357,17 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   ok &= make_map_strided(&h->tm_vh.b16, h->vh + (l - lx), Tm_b, lx + hs, l + hs, GEMM_BROWS);
   ok &= make_map_strided(&h->tm_vh.b64, h->vh + (l - lx), Tm_b, lx + hs, l + hs,
                          GEMM_BROWS_BIG);
+  if (bfx && proj) {
+    ok &= make_map(&h->tm_ws1, h->w_x + (N + lx) * d, hs, d, GEMM_BM);
+    ok &= make_map_strided(&h->tm_ws2, h->w_y + lx, d_a, hs, lx + hs, GEMM_BM);
+    ok &= make_map_strided(&h->tm_hs.b16, h->vh + l, Tm_b, hs, l + hs, GEMM_BROWS);
+    ok &= make_map_strided(&h->tm_hs.b64, h->vh + l, Tm_b, hs, l + hs, GEMM_BROWS_BIG);
+    ok &= cudaStreamCreateWithFlags(&h->side_st, cudaStreamNonBlocking) == cudaSuccess;
+    ok &= cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess;
+    ok &= cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) == cudaSuccess;
+    ok &= set_smem_all<EpiS1>() == cudaSuccess;
+    ok &= set_pair_smem<EpiS1>() == cudaSuccess;
+  }
   if (bwd) {
     // MN-major operands of the backward GEMMs: 64 x 64 boxes (the same boxes
     // serve K-major token rows); padding rows read as zero
@@ -1378,6 +1420,8 @@ void lmoe_destroy(lmoe_handle* h) {
   delete h;
 }
 
+static int overlap_sms(const lmoe_handle* h, int64_t T);
+
 int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T) {
   if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return 0;
@@ -1386,7 +1430,8 @@ int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T) {
                                   c.d / 64, h->sms);
   const DensePlan py = plan_dense(T, (c.d + 127) / 128, (h->lx + c.shared_hidden) / 64, h->sms);
   (void)px;   // a split x-GEMM's reduction replaces the router kernel: same count
-  return 10 + (py.ksplit > 1);
+  // an overlapped forward runs the shared expert's two GEMMs apart
+  return 10 + (py.ksplit > 1) + (overlap_sms(h, T) > 0 ? 2 : 0);
 }
 
 static int prof_begin(lmoe_handle* h, int kernel, cudaStream_t st) {
@@ -1403,17 +1448,48 @@ static void prof_end(lmoe_handle* h, int slot, cudaStream_t st) {
   if (slot >= 0) cudaEventRecord(h->ev[slot + 1], st);
 }
 
-#define LMOE_STEP(kidx, call)                        \
+#define LMOE_STEP_ON(stream, kidx, call)             \
   do {                                               \
-    const int _slot = prof_begin(h, (kidx), st);     \
+    const int _slot = prof_begin(h, (kidx), stream); \
     const cudaError_t _e = (call);                   \
-    prof_end(h, _slot, st);                          \
+    prof_end(h, _slot, stream);                      \
     if (_e != cudaSuccess) return LMOE_ERR_CUDA;     \
   } while (0)
+#define LMOE_STEP(kidx, call) LMOE_STEP_ON(st, kidx, call)
+
+// SMs for the shared expert on the side stream of an overlapped forward, or
+// 0 for a serial one.  Overlap pays when the grouped GEMMs are bound by HBM:
+// each expert's weights are read once per forward, and below about 256 flops
+// per byte (the ratio of dense BF16 tensor throughput to HBM bandwidth on
+// B200) the tensor pipes wait for them, while the shared expert's dense
+// GEMMs are bound by the tensor pipes.  The side stream gets the share of
+// the SMs that makes the two take about the same time: (shared flops / 256)
+// against the grouped GEMMs' weight bytes.  LMOE_OVERLAP=0 turns it off, a
+// number sets the side stream's SMs.
+static int overlap_sms(const lmoe_handle* h, int64_t T) {
+  const lmoe_config& c = h->cfg;
+  if (!h->proj || h->fp4 || h->fp8 || h->w4 || h->ep_dense || h->shard || !h->pairs ||
+      !h->side_st)
+    return 0;
+  int side = -1;
+  if (const char* e = getenv("LMOE_OVERLAP")) side = atoi(e);
+  if (side == 0) return 0;
+  const double rows_per_expert = double(T) * c.top_k / c.n_experts;
+  if (side < 0) {
+    if (T < 1024 || rows_per_expert > 200.0) return 0;
+    const double shared_flops = 4.0 * double(T) * c.d * c.shared_hidden;
+    const double weight_bytes = 4.0 * double(c.n_experts) * c.expert_hidden * c.latent;
+    side = static_cast<int>(h->sms * (shared_flops / 256.0) / weight_bytes + 0.5);
+  }
+  side &= ~1;   // CTA pairs
+  if (side < 8) side = 8;
+  if (side > h->sms / 2) side = h->sms / 2 & ~1;
+  return side;
+}
 
 // Steps 1-5 of the forward: [W_r; W_dn; W_s1] x (logits, u, shared hidden),
 // routing and the per-expert segments.
-static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st) {
+static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st, int side = 0) {
   const lmoe_config& c = h->cfg;
   const int64_t d = c.d;
   const int N = c.n_experts, l = c.latent, hs = c.shared_hidden, K = c.top_k;
@@ -1437,7 +1513,33 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st) 
   bool routed = false;   // the top-K ran inside the x-GEMM's split-K reduction
 
   // 1. [W_r; W_dn; W_s1] x: logits, u, shared hidden
-  {
+  if (side > 0) {
+    // overlapped: the side stream computes hs = sqrelu(W_s1 x) and then
+    // ys = W_s2 hs on `side` SMs while this stream routes and runs the
+    // experts on the others; [W_r; W_dn] x here
+    cudaStream_t ss = h->side_st;
+    if (cudaEventRecord(h->ev_fork, st) != cudaSuccess ||
+        cudaStreamWaitEvent(ss, h->ev_fork, 0) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    {
+      EpiS1 e1{h->vh, l, ldvh};
+      TileSource s1{1, static_cast<int>(T), nullptr, nullptr, (hs + PAIR_BM - 1) / PAIR_BM, 0, hs,
+                    static_cast<int>(d / 64), 1, nullptr, 0};
+      LMOE_STEP_ON(ss, 24, launch_gemm_pair(h->tm_ws1, tm_x, s1, e1, side / 2, h->err, lim, ss));
+      EpiY e2{h->ys, static_cast<int>(d), nullptr, 0};
+      TileSource s2{1, static_cast<int>(T), nullptr, nullptr,
+                    static_cast<int>((d + PAIR_BM - 1) / PAIR_BM), 0, static_cast<int>(d), hs / 64,
+                    1, nullptr, 0};
+      LMOE_STEP_ON(ss, 25, launch_gemm_pair(h->tm_ws2, h->tm_hs, s2, e2, side / 2, h->err, lim,
+                                            ss));
+      if (cudaEventRecord(h->ev_join, ss) != cudaSuccess) return LMOE_ERR_CUDA;
+    }
+    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->uf8, h->r_u8,
+             h->u16};
+    TileSource s{1, static_cast<int>(T), nullptr, nullptr, (N + lx + PAIR_BM - 1) / PAIR_BM, 0,
+                 N + lx, static_cast<int>(d / 64), 1, nullptr, 0};
+    LMOE_STEP(0, launch_gemm_pair(h->tm_wx, tm_x, s, epi, (h->sms - side) / 2, h->err, lim, st));
+  } else {
     const int fb = (N + lx + hs + 127) / 128;
     const DensePlan p = plan_dense(T, fb, static_cast<int>(d / 64), h->sms);
     EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->uf8, h->r_u8,
@@ -1475,21 +1577,25 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st) 
   return LMOE_OK;
 }
 
-// Step 10 of the forward: y = [W_upl | W_s2] [v ; hs] (v already in vh).
-static int fwd_ygemm(lmoe_handle* h, int64_t T, void* y, cudaStream_t st) {
+// Step 10 of the forward: y = [W_upl | W_s2] [v ; hs] (v already in vh);
+// after an overlapped front half, y = W_upl v + ys (the side stream's W_s2 hs).
+static int fwd_ygemm(lmoe_handle* h, int64_t T, void* y, cudaStream_t st, bool overlapped = false) {
   const lmoe_config& c = h->cfg;
   const int64_t d = c.d;
   const int l = c.latent, hs = c.shared_hidden;
   const int ldvh = l + hs;
   const int lx = h->lx;
   const unsigned long long lim = h->wait_limit_ns;
+  if (overlapped && cudaStreamWaitEvent(st, h->ev_join, 0) != cudaSuccess) return LMOE_ERR_CUDA;
   {
     const int fb = static_cast<int>((d + 127) / 128);
-    const int ky = lx + hs;   // K of the y-GEMM
+    const int ky = overlapped ? lx : lx + hs;   // K of the y-GEMM
     const DensePlan p = plan_dense(T, fb, ky / 64, h->sms);
     if (p.ksplit > 1 && int64_t(p.ksplit) * T * d > h->part_floats)
       return LMOE_ERR_UNSUPPORTED;   // never: the buffer is sized for every T
-    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d), h->proj ? nullptr : h->vh, ldvh};
+    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d),
+             overlapped ? h->ys : h->proj ? nullptr : h->vh,
+             overlapped ? static_cast<int>(d) : ldvh};
     const int fb2 = static_cast<int>((d + PAIR_BM - 1) / PAIR_BM);
     const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
     if (h->pairs && ptiles >= h->sms / 2) {
@@ -1527,7 +1633,9 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   const int l = c.latent, hh = c.expert_hidden, hs = c.shared_hidden, K = c.top_k;
   const int ldvh = l + hs;
   const unsigned long long lim = h->wait_limit_ns;
-  int rc = fwd_front(h, x, T, st);
+  const int side = overlap_sms(h, T);   // SMs of the shared expert's side stream, or 0
+  const int gsms = h->sms - side;       // SMs of the grouped GEMMs
+  int rc = fwd_front(h, x, T, st, side);
   if (rc != LMOE_OK) return rc;
   const int gbn = grouped_bn(c, T);
   if (h->w4) {
@@ -1595,11 +1703,11 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
     if (h->pairs && gbn == PAIR_BN) {
       TileSource s{0, 0, h->blocks, h->nblocks, (hh + PAIR_BM - 1) / PAIR_BM, hh, hh, l / 64, 1,
                    nullptr, 0};
-      LMOE_STEP(6, launch_gemm_pair(h->tm_w1, h->tm_uperm, s, epi, h->sms / 2, h->err, lim, st));
+      LMOE_STEP(6, launch_gemm_pair(h->tm_w1, h->tm_uperm, s, epi, gsms / 2, h->err, lim, st));
     } else {
       TileSource s{0, 0, h->blocks, h->nblocks, (hh + 127) / 128, hh, hh, l / 64, 1, nullptr,
                    gbn == 32};
-      LMOE_STEP(6, launch_gemm_bn(gbn, h->tm_w1, h->tm_uperm, s, epi, h->sms, h->err, lim, st));
+      LMOE_STEP(6, launch_gemm_bn(gbn, h->tm_w1, h->tm_uperm, s, epi, gsms, h->err, lim, st));
     }
   }
   // 8. O = w * W2[e] H
@@ -1608,18 +1716,18 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
     if (h->pairs && gbn == PAIR_BN) {
       TileSource s{0, 0, h->blocks, h->nblocks, (l + PAIR_BM - 1) / PAIR_BM, l, l, hh / 64, 1,
                    nullptr, 0};
-      LMOE_STEP(7, launch_gemm_pair(h->tm_w2, h->tm_H, s, epi, h->sms / 2, h->err, lim, st));
+      LMOE_STEP(7, launch_gemm_pair(h->tm_w2, h->tm_H, s, epi, gsms / 2, h->err, lim, st));
     } else {
       TileSource s{0, 0, h->blocks, h->nblocks, (l + 127) / 128, l, l, hh / 64, 1, nullptr,
                    gbn == 32};
-      LMOE_STEP(7, launch_gemm_bn(gbn, h->tm_w2, h->tm_H, s, epi, h->sms, h->err, lim, st));
+      LMOE_STEP(7, launch_gemm_bn(gbn, h->tm_w2, h->tm_H, s, epi, gsms, h->err, lim, st));
     }
   }
   }
   // 9. v = sum_k O[inv[t][k]]
   LMOE_STEP(8, launch_combine(h->O, h->inv, T, K, l, h->vh, ldvh, st));
-  // 10. y = [W_upl | W_s2] [v ; hs]
-  return fwd_ygemm(h, T, y, st);
+  // 10. y = [W_upl | W_s2] [v ; hs], or W_upl v + ys after the side stream
+  return fwd_ygemm(h, T, y, st, side > 0);
 }
 
 int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void* dx,

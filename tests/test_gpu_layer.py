@@ -203,3 +203,26 @@ def test_cta_pair_gemms_match_single_cta_gemms(monkeypatch):
     print("pair_small errors:", errs)
     single.close()
     pair.close()
+
+
+def test_overlapped_shared_expert_matches_serial_forward(monkeypatch):
+    """The forward that runs the shared expert's GEMMs on a side stream over
+    a share of the SMs (chosen by default when the grouped GEMMs are bound by
+    HBM, as at Ultra dims; forced here with LMOE_OVERLAP) equals the serial
+    forward up to the bf16 rounding of the shared branch before the add, and
+    matches the oracle."""
+    cfg = CONFIGS["pair_small"]
+    monkeypatch.setenv("LMOE_OVERLAP", "0")
+    w, x, layer = make(cfg)
+    y0 = layer.forward(x).clone()
+    assert layer.launches_per_forward(cfg.T) == 10
+    monkeypatch.setenv("LMOE_OVERLAP", "16")
+    assert layer.launches_per_forward(cfg.T) == 12
+    y1 = layer.forward(x)
+    torch.cuda.synchronize()
+    assert layer.sync_status() == 0
+    assert max_rel(to64(y1), to64(y0)) <= 1e-2
+    toks = np.unique(np.concatenate([[0, cfg.T - 1], _sample(cfg.T, 24, 19)]))
+    errs = compare_layer(layer, w, x, y1, toks, cfg.K)
+    print("overlapped pair_small errors:", errs)
+    layer.close()
