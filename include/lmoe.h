@@ -267,6 +267,13 @@ int lmoe_bias_update(lmoe_handle* h, float rate, void* stream);
 #define LMOE_DBG_BW4_SCALES 24
 #define LMOE_DBG_BW4_SEG 25
 #define LMOE_DBG_BW4_DA 26
+/* NVFP4 experts: the scale tables of the static scales g_u then g_h, fp32
+ * [2][256]: [k] for k = 1..126 the smallest block amax whose scale code
+ * E4M3(f32(amax / f32(6 g))) is at least k ([0] = 0, [127] = infinity),
+ * [128 + k] = f32(1 / f32(E4M3value(k) g)) (0 when that product is 0),
+ * [255] = f32(1 / f32(6 g)); the activation quantisers use them instead of
+ * dividing. */
+#define LMOE_DBG_SCALE_TABLES 27
 int lmoe_get_debug(lmoe_handle* h, int what, void* dst_host, size_t bytes);
 
 /* Kernel launches one lmoe_forward of T tokens issues, or a negative error

@@ -25,7 +25,8 @@ DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 
        "logits": 7, "u": 8, "v": 9, "hs": 10, "w1q_codes": 11, "w1q_sf": 12, "w1q_g": 13,
        "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16, "bias": 17,
        "bw4_do_codes": 18, "bw4_do_sf": 19, "bw4_dot_codes": 20, "bw4_dot_sf": 21,
-       "bw4_ut_codes": 22, "bw4_ut_sf": 23, "bw4_scales": 24, "bw4_seg": 25, "bw4_da": 26}
+       "bw4_ut_codes": 22, "bw4_ut_sf": 23, "bw4_scales": 24, "bw4_seg": 25, "bw4_da": 26,
+       "scale_tables": 27}
 
 
 class LmoeConfig(Structure):

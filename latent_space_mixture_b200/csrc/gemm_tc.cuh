@@ -37,6 +37,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "nvfp4.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
@@ -92,6 +94,18 @@ struct TileSource {
 
 struct TileInfo {
   int e, fb, row0, nrows, a_row, ks, kb0, kb1, tb;
+};
+
+// Features an epilogue takes per call: 8 consecutive features of one token row
+// (store8), or 16 for an epilogue that declares kVec = 16 (store16: a whole
+// NVFP4 block per lane).
+template <class E, class = void>
+struct EpiVec {
+  static constexpr int value = 8;
+};
+template <class E>
+struct EpiVec<E, std::void_t<decltype(E::kVec)>> {
+  static constexpr int value = E::kVec;
 };
 
 __device__ __forceinline__ int gemm_num_tiles(const TileSource& s, int BN) {
@@ -503,6 +517,24 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
         for (int j = 0; j < 32; ++j) my[j * GEMM_STG_LD + lane] = __uint_as_float(r[j]);
         __syncwarp();
+        if constexpr (EpiVec<Epi>::value == 16) {
+          // lanes 2j, 2j+1 hold the two 16-feature groups of token row j
+#pragma unroll
+          for (int it = 0; it < 2; ++it) {
+            const int item = lane + 32 * it;
+            const int j = item >> 1;
+            const int g = item & 1;
+            const int feat = feat_base + g * 16;
+            const bool valid = c0 + j < t.nrows && feat < src.m_valid;
+            const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 16);
+            const float4 q0 = p[0], q1 = p[1], q2 = p[2], q3 = p[3];
+            const float v[16] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w,
+                                 q2.x, q2.y, q2.z, q2.w, q3.x, q3.y, q3.z, q3.w};
+            epi.store16(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid);
+          }
+          __syncwarp();
+          continue;
+        }
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
           // lanes 4j..4j+3 hold the four 8-feature groups of token row j
@@ -727,6 +759,24 @@ __device__ __forceinline__ uint32_t nvfp4_pair(const float* v, float g, uint8_t*
   const uint8_t code = e4m3_code(sbf);
   const float denom = __fmul_rn(e4m3_value(code), g);
   const float rcp = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w |= e2m1x2(__fmul_rn(v[2 * i], rcp), __fmul_rn(v[2 * i + 1], rcp)) << (8 * i);
+  *sc = code;
+  return w;
+}
+
+// nvfp4_pair with the block scale and its reciprocal from the scale tables of
+// the global scale (nvfp4_scale_tab): the same codes, no division.
+__device__ __forceinline__ uint32_t nvfp4_pair_tab(const float* v, const float* __restrict__ tab,
+                                                   uint8_t* sc) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  float rcp;
+  const uint8_t code = nvfp4_scale_tab(amax, tab, &rcp);
   uint32_t w = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i)

@@ -66,6 +66,8 @@ cudaError_t launch_quant_weights(const void* w, int E, int rows_per, int K, int 
 // bytes and per-expert scales [E] (amax / 448); amax is [E] scratch.
 cudaError_t launch_quant_w8(const void* w, int E, int rows_per, int K, float* amax, uint8_t* codes,
                             float* scale, cudaStream_t st);
+// Scale tables (nvfp4.cuh, NVFP4_TAB floats) of one static global scale g.
+cudaError_t launch_scale_tables(float g, float* tab, cudaStream_t st);
 // fp32 rows -> codes [rows][cols/2], scales [rows][cols/16] (canonical layout).
 cudaError_t launch_quant_rows(const float* x, int64_t rows, int cols, float g, uint8_t* codes,
                               uint8_t* scales, cudaStream_t st);

@@ -38,6 +38,7 @@ struct EpiX {
   uint8_t* uq;    // NVFP4 experts: u codes [T][l/2] (nullptr for BF16 experts)
   uint8_t* usf;   //   and its E4M3 block scales [T][l/16]
   float g_u;      //   static global scale of u
+  const float* tab_u;   //   its scale tables (nvfp4_scale_tab)
   uint8_t* u8;    // FP8 experts: u codes [T][l] (nullptr otherwise)
   float r_u8;     //   1 / s_u (rounded once)
   __half* u16;    // W4A16 experts: u in f16 [T][l] (nullptr otherwise)
@@ -46,7 +47,7 @@ struct EpiX {
     if (uq) {
       // every lane takes part in the 16-block pair exchange; only u lanes store
       uint8_t sc;
-      const uint32_t codes = nvfp4_pair(v, g_u, &sc);
+      const uint32_t codes = nvfp4_pair_tab(v, tab_u, &sc);
       if (valid && feat >= N && feat < N + lu) {
         const int f = feat - N;
         *reinterpret_cast<uint32_t*>(uq + row * (lu / 2) + f / 2) = codes;
@@ -160,11 +161,13 @@ struct EpiY {
 struct EpiHq {
   // epilogue warps at >= 128-row token blocks: quantising H is ~9x the FP4 MMAs
   static constexpr int kWarps = 16;
+  static constexpr int kVec = 16;   // a whole 16-element NVFP4 block per lane
   uint8_t* Hq;
   uint8_t* sfh;
   const float* gw1;
   float g_u, g_h;
   int hp;   // h rounded up to 256 (row pitch hp/2 bytes)
+  const float* tab_h;    // scale tables of g_h (nvfp4_scale_tab)
   bf16* a16 = nullptr;   // NVFP4 training: the pre-activation a = W1[e] u, bf16 [R][ha]
   int ha = 0;
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
@@ -174,7 +177,7 @@ struct EpiHq {
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = sqrelu(v[i] * s);
     uint8_t sc;
-    const uint32_t codes = nvfp4_pair(a, g_h, &sc);
+    const uint32_t codes = nvfp4_pair_tab(a, tab_h, &sc);
     if (!valid) return;
     if (a16) {
       float pre[8];
@@ -186,6 +189,38 @@ struct EpiHq {
     if ((feat & 15) == 0)
       sfh[(static_cast<long>(t.tb) * (hp / 64) + feat / 64) * SF_ATOM_BYTES +
           sf_atom_offset(static_cast<int>(row - t.row0), (feat & 63) >> 4)] = sc;
+  }
+  // one 16-element block of a row: the block's scale from the tables of g_h,
+  // no lane exchange (the same codes as store8)
+  __device__ __forceinline__ void store16(const TileInfo& t, long row, int feat, const float* v,
+                                          bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(gw1[t.e], g_u);
+    float a[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      a[i] = sqrelu(v[i] * s);
+      amax = fmaxf(amax, fabsf(a[i]));
+    }
+    float r;
+    const uint8_t sc = nvfp4_scale_tab(amax, tab_h, &r);
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      w0 |= e2m1x2(__fmul_rn(a[2 * i], r), __fmul_rn(a[2 * i + 1], r)) << (8 * i);
+      w1 |= e2m1x2(__fmul_rn(a[8 + 2 * i], r), __fmul_rn(a[8 + 2 * i + 1], r)) << (8 * i);
+    }
+    *reinterpret_cast<uint2*>(Hq + row * (hp / 2) + feat / 2) = make_uint2(w0, w1);
+    sfh[(static_cast<long>(t.tb) * (hp / 64) + feat / 64) * SF_ATOM_BYTES +
+        sf_atom_offset(static_cast<int>(row - t.row0), (feat & 63) >> 4)] = sc;
+    if (a16) {
+      float pre[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pre[i] = v[i] * s;
+      store8_bf16(a16 + row * ha + feat, pre);
+      store8_bf16(a16 + row * ha + feat + 8, pre + 8);
+    }
   }
 };
 
@@ -838,6 +873,7 @@ struct lmoe_handle {
   uint8_t* w2sf = nullptr;     // [N*l/128][hp/64][512]
   float* gw2 = nullptr;        // [N]
   float* amax = nullptr;       // [N] scratch of the weight quantisation
+  float* stab = nullptr;       // scale tables of g_u, then of g_h (2 x NVFP4_TAB)
   uint8_t* uq = nullptr;       // [T][l/2]
   uint8_t* usf = nullptr;      // [T][l/16]
   uint8_t* upq = nullptr;      // [T*K][lp/2] expert order
@@ -1152,6 +1188,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->gw2, size_t(qw4 * N * 4)},
       {(void**)&h->amax, size_t((qw4 || fp8) * N * 4)},
       {(void**)&h->u16, size_t(w4 * Tm * l * 2)},
+      {(void**)&h->stab, size_t(fp4 * 2 * NVFP4_TAB * 4)},
       {(void**)&h->uq, size_t(fp4 * Tm * l / 2)},
       {(void**)&h->usf, size_t(fp4 * Tm * l / 16)},
       {(void**)&h->upq, size_t(fp4 * rows_b * lp / 2)},
@@ -1272,6 +1309,8 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
                                static_cast<int>(hp), h->amax, h->w2q, h->w2sf, h->gw2, wvar,
                                0) == cudaSuccess;
     if (fp4) {
+      ok &= launch_scale_tables(h->g_u, h->stab, 0) == cudaSuccess;
+      ok &= launch_scale_tables(h->g_h, h->stab + NVFP4_TAB, 0) == cudaSuccess;
       ok &= make_map_u8(&h->tm_w1q, h->w1q, N * hh, lp / 2, GEMM_BM);
       ok &= make_map_u8(&h->tm_w2q, h->w2q, N * l, hp / 2, GEMM_BM);
       ok &= make_map_u8(&h->tm_upq.b16, h->upq, rows_b, lp / 2, GEMM_BROWS);
@@ -1534,7 +1573,7 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st, 
                                             ss));
       if (cudaEventRecord(h->ev_join, ss) != cudaSuccess) return LMOE_ERR_CUDA;
     }
-    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->uf8, h->r_u8,
+    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->stab, h->uf8, h->r_u8,
              h->u16};
     TileSource s{1, static_cast<int>(T), nullptr, nullptr, (N + lx + PAIR_BM - 1) / PAIR_BM, 0,
                  N + lx, static_cast<int>(d / 64), 1, nullptr, 0};
@@ -1542,7 +1581,7 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st, 
   } else {
     const int fb = (N + lx + hs + 127) / 128;
     const DensePlan p = plan_dense(T, fb, static_cast<int>(d / 64), h->sms);
-    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->uf8, h->r_u8,
+    EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->stab, h->uf8, h->r_u8,
              h->u16};
     const int fb2 = (N + lx + hs + PAIR_BM - 1) / PAIR_BM;
     const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
@@ -1683,7 +1722,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
     {
       TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, h->lp / 256, 1, nullptr,
                    gbn == 32, h->w1sf, h->sfbu, h->lp / 64};
-      EpiHq epi{h->Hq, h->sfbh, h->gw1, h->g_u, h->g_h, h->hp};
+      EpiHq epi{h->Hq, h->sfbh, h->gw1, h->g_u, h->g_h, h->hp, h->stab + NVFP4_TAB};
       LMOE_STEP(6, launch_gemm_q<KIND_NVFP4>(gbn, h->tm_w1q, h->tm_upq, s, epi, h->sms, h->err, lim, st));
     }
     // 8. O = w * W2[e] H, block-scaled FP4 MMA
@@ -2157,7 +2196,7 @@ int lmoe_experts_backward_nvfp4(lmoe_handle* h, const void* u, const int32_t* to
   {
     TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, lp / 256, 1, nullptr,
                  gbn == 32, h->w1sf, h->sfbu, lp / 64};
-    EpiHq epi{h->Hq, h->sfbh, h->gw1, h->g_u, h->g_h, hp, h->a16, hh};
+    EpiHq epi{h->Hq, h->sfbh, h->gw1, h->g_u, h->g_h, hp, h->stab + NVFP4_TAB, h->a16, hh};
     LMOE_STEP(6, launch_gemm_q<KIND_NVFP4>(gbn, h->tm_w1q, h->tm_upq, s, epi, h->sms, h->err, lim,
                                            st));
   }
@@ -2304,6 +2343,9 @@ int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
     case LMOE_DBG_W2Q_SF: src = h->w2sf; want = (N * l / 128) * (h->hp / 64) * 512; break;
     case LMOE_DBG_BIAS: src = h->bias; want = N * 4; break;
     case LMOE_DBG_W2Q_G: src = h->fp8 ? h->sw2 : h->gw2; want = N * 4; break;
+    case LMOE_DBG_SCALE_TABLES:
+      if (!h->fp4) return LMOE_ERR_INVALID_ARG;
+      src = h->stab; want = 2 * NVFP4_TAB * 4; break;
     default: break;
   }
   if (what >= LMOE_DBG_BW4_DO_CODES && what <= LMOE_DBG_BW4_DA) {

@@ -210,6 +210,39 @@ cudaError_t launch_quant_w8(const void* w, int E, int rows_per, int K, float* am
   return cudaGetLastError();
 }
 
+// The scale tables of global scale g (nvfp4.cuh, NVFP4_TAB floats): a thread
+// per entry; a threshold is found by bisection over the bit patterns of the
+// non-negative floats, with the quantiser's own float32 operations.
+__global__ void k_scale_tables(float g, float* __restrict__ tab) {
+  const int k = threadIdx.x;
+  const float six_g = __fmul_rn(6.0f, g);
+  if (k == 0) {
+    tab[0] = 0.0f;
+  } else if (k < 127) {
+    uint32_t lo = 0, hi = 0x7F800000u;   // code(lo) < k <= code(hi)
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + (hi - lo) / 2;
+      const float a = __uint_as_float(mid);
+      const int c = e4m3_code(six_g > 0.0f ? __fdiv_rn(a, six_g) : 0.0f);
+      if (c >= k) hi = mid;
+      else lo = mid;
+    }
+    tab[k] = __uint_as_float(hi);
+  } else if (k == 127) {
+    tab[127] = __uint_as_float(0x7F800000u);
+  } else if (k < 255) {
+    const float denom = __fmul_rn(e4m3_value(static_cast<uint8_t>(k - 128)), g);
+    tab[k] = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+  } else {
+    tab[255] = six_g > 0.0f ? __fdiv_rn(1.0f, six_g) : 0.0f;
+  }
+}
+
+cudaError_t launch_scale_tables(float g, float* tab, cudaStream_t st) {
+  k_scale_tables<<<1, NVFP4_TAB, 0, st>>>(g, tab);
+  return cudaGetLastError();
+}
+
 // Row quantiser with canonical outputs: codes [rows][cols/2], scales [rows][cols/16].
 __global__ void __launch_bounds__(256) k_quant_rows(const float* __restrict__ x, int64_t rows,
                                                     int cols, float g, uint8_t* __restrict__ codes,

@@ -101,6 +101,26 @@ __device__ __forceinline__ uint8_t nvfp4_block(const float (&x)[16], float g, ui
 }
 
 // ---------------------------------------------------------------------------
+// Scale tables of one static global scale g (NVFP4_TAB floats, built once by
+// launch_scale_tables): thr[k] (k = 1..126) is the smallest float amax whose
+// block scale code E4M3(f32(amax / f32(6 g))) is at least k, thr[0] = 0 and
+// thr[127] = infinity; rtab[k] = f32(1 / f32(E4M3value(k) g)), or 0 when that
+// product is 0; inv6g = f32(1 / f32(6 g)).  The code is a monotone step
+// function of amax, so counting thresholds reproduces it exactly; a product
+// with inv6g lands within one code of it, and one comparison corrects it.
+constexpr int NVFP4_TAB = 256;   // thr [0, 128), rtab [128, 255), inv6g [255]
+
+__device__ __forceinline__ uint8_t nvfp4_scale_tab(float amax, const float* __restrict__ tab,
+                                                   float* r) {
+  int code = e4m3_code(__fmul_rn(amax, tab[255]));
+  code = code > 126 ? 126 : code;
+  if (amax >= tab[code + 1]) ++code;
+  else if (amax < tab[code]) --code;
+  *r = tab[128 + code];
+  return static_cast<uint8_t>(code);
+}
+
+// ---------------------------------------------------------------------------
 // Gradient-path pieces of the NVFP4 training recipe ("Nemotron-3 Super 精读报告",
 // section 5.3: a random Hadamard transform on the inputs of the weight-gradient
 // GEMMs, stochastic rounding of gradient tensors; section 9.3: stochastic

@@ -243,6 +243,7 @@ class LatentMoE:
             "logits": (torch.float32, (T, c.n_experts)), "u": (torch.bfloat16, (T, c.latent)),
             "v": (torch.bfloat16, (T, c.latent)), "hs": (torch.bfloat16, (T, c.shared_hidden)),
             "bias": (torch.float32, (c.n_experts,)),
+            "scale_tables": (torch.float32, (2, 256)),
         }
         lp = (c.latent + 255) // 256 * 256
         hp = (c.expert_hidden + 255) // 256 * 256

@@ -93,11 +93,13 @@ def test_expert_parallel_forward_matches_oracle(name, P, T_per):
             np.unique(np.concatenate([[0, T - 1], rng.choice(T, 24, replace=False)]))
         errs = compare_layer(layers[r], w, xs[r], ys[r], toks, cfg.K)
         # the single-GPU layer on the same tokens: same kernels, weighting
-        # after instead of before the bf16 rounding of the expert outputs
+        # after instead of before the bf16 rounding of the expert outputs;
+        # each is within 2e-2 RMS(y) of the oracle, so they are within twice
+        # that of each other
         y1 = single.forward(xs[r])
         torch.cuda.synchronize()
         errs["vs_single_gpu_layer"] = max_rel(to64(ys[r]), to64(y1))
-        assert errs["vs_single_gpu_layer"] <= 2e-2
+        assert errs["vs_single_gpu_layer"] <= 2 * 2e-2
         print(name, P, "rank", r, "rows sent", plans[r].send_counts, errs)
     for o in layers + shards + [single]:
         o.close()

@@ -138,3 +138,31 @@ def test_quantised_weights_bit_exact_at_super_widths():
             assert np.array_equal(sc[e * R:(e + 1) * R], osc), (name, e)
             assert np.array_equal(Q.e2m1_decode(q[e * R:(e + 1) * R]), Q.e2m1_decode(oc)), (name, e)
     layer.close()
+
+
+def test_activation_scale_tables_reproduce_the_division():
+    """The activation quantisers of the NVFP4 layer take a block's scale code
+    and the reciprocal of its denominator from tables instead of dividing.
+    Pinned to the quantiser's definition (float32, oracle.nvfp4): threshold k
+    is the smallest float amax whose code E4M3(f32(amax / f32(6 g))) is at
+    least k (checked at the threshold and at the float just below it), and
+    reciprocal k is f32(1 / f32(E4M3value(k) g))."""
+    from lmoe_synth import act_global_scales
+    cfg = CONFIGS["tiny_nvfp4"]
+    w, x, layer = make(cfg)
+    tab = layer.debug("scale_tables").numpy()
+    for row, g in enumerate(act_global_scales(cfg)):
+        g32 = np.float32(g)
+        six_g = np.float32(np.float32(6.0) * g32)
+        code = lambda a: int(Q.e4m3_rtne(np.array([np.float32(np.float32(a) / six_g)]))[0])  # noqa
+        t = tab[row]
+        assert t[0] == 0.0 and np.isinf(t[127])
+        for k in range(1, 127):
+            thr = np.float32(t[k])
+            assert code(thr) >= k, (row, k)
+            assert code(np.nextafter(thr, np.float32(0.0))) < k, (row, k)
+            s = np.float32(Q.e4m3_decode(np.array([k]))[0])
+            assert t[128 + k] == np.float32(np.float32(1.0) / np.float32(s * g32)), (row, k)
+        assert t[128] == 0.0
+        assert t[255] == np.float32(np.float32(1.0) / six_g)
+    layer.close()
