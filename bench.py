@@ -606,8 +606,9 @@ def run_training(args, cfg, world, rank, local_rank):
                                              device_id=torch.device("cuda", local_rank))
     from latent_space_mixture_b200 import LatentMoE
     from lmoe_synth import make_grad_out
-    if cfg.fmt != "bf16" or not cfg.proj:
-        raise SystemExit("--backward needs a BF16 workload with latent projections")
+    if not cfg.proj or not (cfg.fmt == "bf16" or (cfg.fmt == "nvfp4" and "2d" in cfg.wq)):
+        raise SystemExit("--backward needs BF16 or 2D-block NVFP4 experts with latent "
+                         "projections")
     dev = torch.device("cuda", local_rank)
     w, _ = make_weights(cfg, device=dev)
     gen = torch.Generator(device=dev)
@@ -615,7 +616,10 @@ def run_training(args, cfg, world, rank, local_rank):
     x = make_x(cfg, gen, device=dev)
     T = cfg.T
     dy = make_grad_out(cfg, T=T, device=dev, seed=shard_seed(cfg.seed + 1000, rank))
-    layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, backward=True)
+    from lmoe_synth import act_global_scales
+    layer = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, T, w, expert_format=cfg.fmt,
+                      act_gscales=act_global_scales(cfg) if cfg.fmt != "bf16" else (0.0, 0.0),
+                      nvfp4_weights=cfg.wq, backward=True)
     y = torch.empty_like(x)
     dx = torch.empty_like(x)
     grads = layer.grad_buffers()
@@ -702,7 +706,9 @@ def run_training(args, cfg, world, rank, local_rank):
             "metric": TRAIN_METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16 (fp32 accumulation, fp32 weight gradients)",
+            "dtype": ("bf16 (fp32 accumulation, fp32 weight gradients)" if cfg.fmt == "bf16" else
+                      "e2m1 experts (NVFP4 training recipe: fprop, dgrad, wgrad), bf16 dense, "
+                      "fp32 weight gradients"),
             "data": "synthetic (seeded; weights N(0, std) bf16, x and dL/dy N(0,1) bf16)",
             "config": {"workload": cfg.name, "T": T, "d": cfg.d, "latent": cfg.l,
                        "n_experts": cfg.N, "top_k": cfg.K, "expert_hidden": cfg.h,

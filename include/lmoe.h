@@ -67,7 +67,8 @@ extern "C" {
 #define LMOE_FLAG_NVFP4_WEIGHT_2D 2
 #define LMOE_FLAG_NVFP4_WEIGHT_MSE 4
 /* LMOE_FLAG_BACKWARD: also reserve the workspace of lmoe_backward (BF16
- * experts with latent projections only; UNSUPPORTED otherwise). */
+ * experts, or NVFP4 experts with LMOE_FLAG_NVFP4_WEIGHT_2D, with latent
+ * projections; UNSUPPORTED otherwise). */
 #define LMOE_FLAG_BACKWARD 8
 /* LMOE_FLAG_EP_DENSE: a handle for expert parallelism that holds the router,
  * the latent projections and the shared expert but no expert weights (w1, w2
@@ -190,9 +191,14 @@ typedef struct lmoe_grads {
  * bf16 with fp32 accumulation; dx and the intermediate gradients rounded to
  * bf16.  Asynchronous on `stream`, no allocation.  dx must not overlap x or
  * dy; every pointer 16-byte aligned.  T == 0 is a no-op.
+ * NVFP4 experts (LMOE_FMT_NVFP4 with LMOE_FLAG_NVFP4_WEIGHT_2D): the routed
+ * experts follow the NVFP4 training recipe of lmoe_experts_backward_nvfp4
+ * (their forward recomputed from the saved u), with the random bits of seed
+ * 8 c, c the number of earlier lmoe_backward calls on the handle; the router,
+ * the latent projections and the shared expert stay BF16.
  * Errors: INVALID_ARG (null, T differs from the last forward's, overlap,
  * misalignment), UNSUPPORTED (handle without LMOE_FLAG_BACKWARD, or not
- * BF16 experts with projections), CUDA. */
+ * BF16 or 2D-block NVFP4 experts with projections), CUDA. */
 int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void* dx,
                   const lmoe_grads* g, void* stream);
 

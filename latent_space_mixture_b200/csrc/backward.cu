@@ -118,7 +118,8 @@ __global__ void __launch_bounds__(256) k_route_bw(const float* __restrict__ logi
                                                   const float* __restrict__ wrow,
                                                   const float* __restrict__ dwacc, int64_t T,
                                                   int N, int K,
-                                                  __nv_bfloat16* __restrict__ dxh, int ldx) {
+                                                  __nv_bfloat16* __restrict__ dxh, int ldx,
+                                                  bool direct) {
   pdl_wait();
   pdl_trigger();
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -128,14 +129,21 @@ __global__ void __launch_bounds__(256) k_route_bw(const float* __restrict__ logi
   const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
   for (int e = lane; e < N; e += 32) row[e] = zero;
   int e = 0;
-  float s = 0.0f, acc = 0.0f, w = 1.0f;
+  float s = 0.0f, acc = 0.0f, w = 1.0f, dwd = 0.0f;
   if (lane < K) {
     e = topk_idx[t * K + lane];
     const int r = inv[t * K + lane];
     // the score from the same logit and expression as the forward router
     s = 1.0f / (1.0f + expf(-logits[t * N + e]));
-    acc = dwacc[r];
     w = wrow[r];
+    if (direct) {
+      // dL/dw of the slot itself; the weighted sum below takes w dL/dw
+      const float dwv = dwacc[t * K + lane];
+      acc = w * dwv;
+      dwd = dwv;
+    } else {
+      acc = dwacc[r];
+    }
   }
   float Z = 0.0f, m = 0.0f;
   for (int k = 0; k < K; ++k) {   // slot order, as the forward's sum of scores
@@ -146,7 +154,7 @@ __global__ void __launch_bounds__(256) k_route_bw(const float* __restrict__ logi
   if (lane < K) {
     // w = 0 only when the selected score underflowed (s = 0); then dz = 0
     // whatever dw is, so 0 stands in for the 0/0 quotient
-    const float dw = w > 0.0f ? acc / w : 0.0f;
+    const float dw = direct ? dwd : w > 0.0f ? acc / w : 0.0f;
     const float ds = (dw - m) / Z;
     row[e] = __float2bfloat16_rn(ds * s * (1.0f - s));
   }
@@ -154,11 +162,11 @@ __global__ void __launch_bounds__(256) k_route_bw(const float* __restrict__ logi
 
 cudaError_t launch_route_bw(const float* logits, const int32_t* topk_idx, const int32_t* inv,
                             const float* wrow, const float* dwacc, int64_t T, int N, int K,
-                            void* dxh, int ldx, cudaStream_t st) {
+                            void* dxh, int ldx, bool direct, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
   return launch_pdl(k_route_bw, blocks, 256, 0, st, logits, topk_idx, inv, wrow, dwacc, T, N, K,
-                    static_cast<__nv_bfloat16*>(dxh), ldx);
+                    static_cast<__nv_bfloat16*>(dxh), ldx, direct);
 }
 
 // ---------------------------------------------------------------------------

@@ -133,10 +133,11 @@ cudaError_t launch_dact(void* da, const void* H, int64_t rows, int h, float* dwa
                         cudaStream_t st);
 
 // Router backward: dz of the selected experts (zero elsewhere) into columns
-// [0, N) of dxh (bf16, row pitch ldx), from dwacc[r] = sum_h g_r[h] dg_r[h].
+// [0, N) of dxh (bf16, row pitch ldx), from dwacc[r] = sum_h g_r[h] dg_r[h]
+// (= w_r dL/dw_r) per routed row, or (direct) from dL/dw per (token, slot).
 cudaError_t launch_route_bw(const float* logits, const int32_t* topk_idx, const int32_t* inv,
                             const float* wrow, const float* dwacc, int64_t T, int N, int K,
-                            void* dxh, int ldx, cudaStream_t st);
+                            void* dxh, int ldx, bool direct, cudaStream_t st);
 
 // Aux-loss-free bias update: bias[e] += rate * sign(total - N * counts[e]).
 cudaError_t launch_bias_update(float* bias, const int32_t* counts, int N, int64_t total, float rate,

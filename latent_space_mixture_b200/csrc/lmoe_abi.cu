@@ -942,6 +942,7 @@ struct lmoe_handle {
   CUtensorMap tm_w1qT, tm_w2qT, tm_tA[4];
   BMaps tm_doq, tm_daq, tm_tB[4];
   int64_t bw4_T = -1;          // T of the last lmoe_experts_backward_nvfp4
+  uint64_t bw_seed = 0;        // random bits of the next NVFP4 lmoe_backward
   // overlapped forward (BF16 experts bound by HBM): the shared expert's two
   // GEMMs on a side stream over a share of the SMs
   cudaStream_t side_st = nullptr;
@@ -1138,6 +1139,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
   // the BF16 backward's workspace, or the NVFP4 training backward's
   const int64_t bwd = ((c.flags & LMOE_FLAG_BACKWARD) && bfx) ? 1 : 0;
   const int64_t bw4 = ((c.flags & LMOE_FLAG_BACKWARD) && fp4) ? 1 : 0;
+  const int64_t bwx = (bwd || bw4) ? 1 : 0;   // the dense GEMMs' backward
   h->bw = bwd != 0;
   h->bw4 = bw4 != 0;
   // transposed operands of the NVFP4 weight gradients: every expert's rows
@@ -1203,13 +1205,13 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->uf8, size_t(fp8 * Tm * l)},
       {(void**)&h->upf8, size_t(fp8 * rows_b * l)},
       {(void**)&h->Hf8, size_t(fp8 * rows_b * hh)},
-      {(void**)&h->dv, size_t(bwd * Tm_b * l * 2)},
+      {(void**)&h->dv, size_t(bwx * Tm_b * l * 2)},
       {(void**)&h->dog, size_t(bwd * rows_b * l * 2)},
       {(void**)&h->da, size_t(bwd * rows_b * hh * 2)},
       {(void**)&h->dup, size_t(bwd * rows_b * l * 2)},
-      {(void**)&h->dwacc, size_t(bwd * rows * 4)},
-      {(void**)&h->dxh, size_t(bwd * Tm_b * (N + l + hs) * 2)},
-      {(void**)&h->dy_dev, size_t(bwd * GEMM_BROWS_BIG * d * 2)},
+      {(void**)&h->dwacc, size_t(bwx * rows * 4)},
+      {(void**)&h->dxh, size_t(bwx * Tm_b * (N + l + hs) * 2)},
+      {(void**)&h->dy_dev, size_t(bwx * GEMM_BROWS_BIG * d * 2)},
       {(void**)&h->ys, size_t((bfx && proj) ? Tm * d * 2 : 0)},
       {(void**)&h->w1qT, size_t(bw4 * N * l * hp / 2)},
       {(void**)&h->w1qT_sf, size_t(bw4 * (N * l / 128) * (hp / 64) * 512)},
@@ -1407,27 +1409,30 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= set_smem_all<EpiS1>() == cudaSuccess;
     ok &= set_pair_smem<EpiS1>() == cudaSuccess;
   }
-  if (bwd) {
+  if (bwx) {
     // MN-major operands of the backward GEMMs: 64 x 64 boxes (the same boxes
     // serve K-major token rows); padding rows read as zero
-    ok &= cudaMemset(h->dog, 0, rows_b * l * 2) == cudaSuccess;
-    ok &= cudaMemset(h->da, 0, rows_b * hh * 2) == cudaSuccess;
     ok &= cudaMemset(h->dxh, 0, Tm_b * (N + l + hs) * 2) == cudaSuccess;
     ok &= cudaMemset(h->dy_dev, 0, GEMM_BROWS_BIG * d * 2) == cudaSuccess;
     ok &= make_map(&h->tm_wx64, h->w_x, N + lx + hs, d, GEMM_BROWS_BIG);
     ok &= make_map(&h->tm_wy64, h->w_y, d_a, lx + hs, GEMM_BROWS_BIG);
-    ok &= make_map(&h->tm_w1_64, h->w1, N * hh, l, GEMM_BROWS_BIG);
-    ok &= make_map(&h->tm_w2_64, h->w2, N * l, hh, GEMM_BROWS_BIG);
-    ok &= make_map(&h->tm_dog.b16, h->dog, rows_b, l, GEMM_BROWS);
-    ok &= make_map(&h->tm_dog.b64, h->dog, rows_b, l, GEMM_BROWS_BIG);
-    ok &= make_map(&h->tm_da.b16, h->da, rows_b, hh, GEMM_BROWS);
-    ok &= make_map(&h->tm_da.b64, h->da, rows_b, hh, GEMM_BROWS_BIG);
     ok &= make_map(&h->tm_dxh.b16, h->dxh, Tm_b, N + l + hs, GEMM_BROWS);
     ok &= make_map(&h->tm_dxh.b64, h->dxh, Tm_b, N + l + hs, GEMM_BROWS_BIG);
     ok &= set_bw_dgrad_smem<EpiDVH>() == cudaSuccess;
     ok &= set_bw_dgrad_smem<EpiStore>() == cudaSuccess;
     ok &= set_bw_smem<256, true, EpiWRows>() == cudaSuccess;
     ok &= set_bw_smem<256, true, EpiWCols>() == cudaSuccess;
+  }
+  if (bwd) {
+    // the BF16 experts' backward
+    ok &= cudaMemset(h->dog, 0, rows_b * l * 2) == cudaSuccess;
+    ok &= cudaMemset(h->da, 0, rows_b * hh * 2) == cudaSuccess;
+    ok &= make_map(&h->tm_w1_64, h->w1, N * hh, l, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_w2_64, h->w2, N * l, hh, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_dog.b16, h->dog, rows_b, l, GEMM_BROWS);
+    ok &= make_map(&h->tm_dog.b64, h->dog, rows_b, l, GEMM_BROWS_BIG);
+    ok &= make_map(&h->tm_da.b16, h->da, rows_b, hh, GEMM_BROWS);
+    ok &= make_map(&h->tm_da.b64, h->da, rows_b, hh, GEMM_BROWS_BIG);
     ok &= set_bw_smem<256, true, EpiWExp>() == cudaSuccess;
   }
   ok &= set_smem_all<EpiX>() == cudaSuccess;
@@ -1769,10 +1774,14 @@ int lmoe_forward(lmoe_handle* h, const void* x, int64_t T, void* y, void* stream
   return fwd_ygemm(h, T, y, st, side > 0);
 }
 
+static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
+                       const float* topk_w, const void* dv, int64_t T, uint64_t seed, bf16* du,
+                       int ldu, float* dw, float* d_w1, float* d_w2, cudaStream_t st);
+
 int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void* dx,
                   const lmoe_grads* gr, void* stream) {
   if (!h || T < 0) return LMOE_ERR_INVALID_ARG;
-  if (!h->bw) return LMOE_ERR_UNSUPPORTED;
+  if (!h->bw && !h->bw4) return LMOE_ERR_UNSUPPORTED;
   if (T == 0) return LMOE_OK;
   if (T != h->last_T || !x || !dy || !dx || !gr || !gr->d_router || !gr->d_dn || !gr->d_w1 ||
       !gr->d_w2 || !gr->d_upl || !gr->d_s1 || !gr->d_s2)
@@ -1842,6 +1851,18 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
     LMOE_BW(0, launch_bw_dgrad(dbn, h->tm_wy64, tm_dy.b16, tm_dy.b64, s, epi,
                             grid_of(((T + dbn - 1) / dbn) * fb), h->err, lim, st));
   }
+  if (h->bw4) {
+    // 2-6, NVFP4 training recipe: the routed experts' backward (their forward
+    // recomputed from the saved u), du into columns [N, N+l) of dxh, dL/dw
+    // per (token, slot), dW1 and dW2; then the router through those dL/dw
+    const uint64_t seed = h->bw_seed;
+    h->bw_seed += 8;
+    const int rc = experts_bw4(h, h->u, h->topk_idx, h->topk_w, h->dv, T, seed, h->dxh + N, ldx,
+                               h->dwacc, gr->d_w1, gr->d_w2, st);
+    if (rc != LMOE_OK) return rc;
+    LMOE_BW(5, launch_route_bw(h->logits, h->topk_idx, h->inv, h->wrow, h->dwacc, T, N, K,
+                               h->dxh, ldx, true, st));
+  } else {
   // 2. do[r] = w_r dv[t(r)] in expert order
   LMOE_BW(1, launch_gather_scaled(h->dv, h->perm, h->wrow, R, K, l, h->dog, st));
   // 3. dg = W2[e]^T do (bf16, into the da buffer)
@@ -1864,7 +1885,8 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
   LMOE_BW(4, launch_combine(h->dup, h->inv, T, K, l, h->dxh + N, ldx, st));
   // 6. router: dz into columns [0, N) of dxh
   LMOE_BW(5, launch_route_bw(h->logits, h->topk_idx, h->inv, h->wrow, h->dwacc, T, N, K, h->dxh,
-                             ldx, st));
+                             ldx, false, st));
+  }
   // 7. dx = [dz | du | dhs_pre] [W_r; W_dn; W_s1]
   {
     const int fb = static_cast<int>((d + 127) / 128);
@@ -1887,7 +1909,7 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
                                   grid_of(int64_t(fb) * nbk), h->err, lim, st)));
   }
   // 9. dW2[e] = do^T g over the expert's rows  ([l][h])
-  {
+  if (!h->bw4) {
     const int fb = (hh + 127) / 128, nbk = (l + 255) / 256;
     BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, hh, hh, N, h->offsets, nbk, l, l};
     EpiWExp epi{};
@@ -1897,7 +1919,7 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
                                   grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
   }
   // 10. dW1[e] = da^T u over the expert's rows  ([h][l])
-  {
+  if (!h->bw4) {
     const int fb = (l + 127) / 128, nbk = (hh + 255) / 256;
     BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, l, l, N, h->offsets, nbk, hh, hh};
     EpiWExp epi{};
@@ -2151,19 +2173,11 @@ int lmoe_permute_rows(const void* src, const int32_t* idx, int64_t n, int64_t n_
 // ---------------------------------------------------------------------------
 // routed experts' forward and backward under the NVFP4 training recipe
 
-int lmoe_experts_backward_nvfp4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
-                                const float* topk_w, const void* dv, int64_t T, uint64_t seed,
-                                void* du, float* dw, float* d_w1, float* d_w2, void* stream) {
-  if (!h || h->shard || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
-  if (!h->bw4) return LMOE_ERR_UNSUPPORTED;
-  if (!d_w1 || !d_w2 || (T > 0 && (!u || !topk_idx || !topk_w || !dv || !du || !dw)))
-    return LMOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(dv) |
-       reinterpret_cast<uintptr_t>(du) | reinterpret_cast<uintptr_t>(d_w1) |
-       reinterpret_cast<uintptr_t>(d_w2)) & 15)
-    return LMOE_ERR_INVALID_ARG;
-  DeviceGuard g(h->dev);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+// The routed experts' NVFP4 forward and backward on the handle's workspace
+// (checked arguments; du rows of pitch ldu elements).
+static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
+                       const float* topk_w, const void* dv, int64_t T, uint64_t seed, bf16* du,
+                       int ldu, float* dw, float* d_w1, float* d_w2, cudaStream_t st) {
   const lmoe_config& c = h->cfg;
   const int N = c.n_experts, l = c.latent, hh = c.expert_hidden, K = c.top_k;
   const int lp = h->lp, hp = h->hp;
@@ -2234,7 +2248,7 @@ int lmoe_experts_backward_nvfp4(lmoe_handle* h, const void* u, const int32_t* to
                                             lim, st));
   }
   // 7. du = sum of a token's rows
-  LMOE_STEP(16, launch_combine(h->O, h->inv, T, K, l, du, l, st));
+  LMOE_STEP(16, launch_combine(h->O, h->inv, T, K, l, du, ldu, st));
   // 8. weight gradients: per expert, over its rows (the K dimension),
   //    transformed operands padded to 256-row segments
   LMOE_STEP(20, launch_seg_offsets(h->counts, N, h->po16, h->po256, h->kofs, st));
@@ -2283,6 +2297,22 @@ int lmoe_experts_backward_nvfp4(lmoe_handle* h, const void* u, const int32_t* to
   LMOE_STEP(20, launch_zero_empty(h->counts, N, int64_t(l) * hh, d_w2, st));
   LMOE_STEP(21, launch_zero_empty(h->counts, N, int64_t(hh) * l, d_w1, st));
   return LMOE_OK;
+}
+
+int lmoe_experts_backward_nvfp4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
+                                const float* topk_w, const void* dv, int64_t T, uint64_t seed,
+                                void* du, float* dw, float* d_w1, float* d_w2, void* stream) {
+  if (!h || h->shard || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
+  if (!h->bw4) return LMOE_ERR_UNSUPPORTED;
+  if (!d_w1 || !d_w2 || (T > 0 && (!u || !topk_idx || !topk_w || !dv || !du || !dw)))
+    return LMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(dv) |
+       reinterpret_cast<uintptr_t>(du) | reinterpret_cast<uintptr_t>(d_w1) |
+       reinterpret_cast<uintptr_t>(d_w2)) & 15)
+    return LMOE_ERR_INVALID_ARG;
+  DeviceGuard g(h->dev);
+  return experts_bw4(h, u, topk_idx, topk_w, dv, T, seed, static_cast<bf16*>(du),
+                     h->cfg.latent, dw, d_w1, d_w2, static_cast<cudaStream_t>(stream));
 }
 
 int64_t lmoe_nvfp4_bw_columns(const lmoe_handle* h) {

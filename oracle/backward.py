@@ -42,7 +42,8 @@ import numpy as np
 
 from .lmoe import route, sqrelu
 
-__all__ = ["layer_backward", "expert_backward", "bias_update", "BIAS_UPDATE_RATE"]
+__all__ = ["layer_backward", "expert_backward", "router_backward", "bias_update",
+           "BIAS_UPDATE_RATE"]
 
 # "Nemotron-3 Super 精读报告", table 6.3: update rate of the aux-loss-free
 # balancing strategy
@@ -70,6 +71,18 @@ def expert_backward(U: np.ndarray, dV: np.ndarray, w: np.ndarray, W1e: np.ndarra
     da = (do @ W2e) * 2.0 * np.maximum(a, 0.0)           # [n][h]
     return {"o": o, "dw": dw, "dW1": da.T @ U, "dW2": dW2, "du": da @ W1e, "do": do, "g": g,
             "da": da}
+
+
+def router_backward(s_sel: np.ndarray, dw: np.ndarray, S: np.ndarray, N: int) -> np.ndarray:
+    """dL/dz [T][N] through the renormalised weights (the router lines of the
+    table above): s_sel [T][K] the selected experts' scores, dw [T][K] =
+    dL/dw, S [T][K] the selected experts; zero at the unselected experts."""
+    Z = s_sel.sum(axis=1)
+    w = s_sel / Z[:, None]
+    ds_sel = (dw - np.sum(w * dw, axis=1, keepdims=True)) / Z[:, None]
+    dz = np.zeros((S.shape[0], N), dtype=np.float64)
+    np.put_along_axis(dz, S, ds_sel * s_sel * (1.0 - s_sel), axis=1)
+    return dz
 
 
 def layer_backward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
@@ -138,9 +151,7 @@ def layer_backward(x: np.ndarray, W_r: np.ndarray, bias: Optional[np.ndarray],
         dx += du
 
     # router: through the renormalised weights of the selected experts
-    ds_sel = (dw - np.sum(w * dw, axis=1, keepdims=True)) / Z[:, None]
-    dz = np.zeros((T, N), dtype=np.float64)
-    np.put_along_axis(dz, S, ds_sel * s_sel * (1.0 - s_sel), axis=1)
+    dz = router_backward(s_sel, dw, S, N)
     dW_r = dz.T @ x
     dx += dz @ W_r
     return {"dx": dx, "dW_r": dW_r, "dW_dn": dW_dn, "dW1": dW1, "dW2": dW2,

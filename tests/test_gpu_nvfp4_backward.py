@@ -149,3 +149,55 @@ def test_nvfp4_experts_backward_no_rows_and_requirements():
     with pytest.raises(LmoeError):
         LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, 64, w, expert_format="nvfp4",
                   act_gscales=act_global_scales(cfg), nvfp4_weights="1d", backward=True)
+
+
+def test_layer_backward_with_nvfp4_experts():
+    """lmoe_backward of a layer with 2D-block NVFP4 experts: the routed
+    experts under the NVFP4 recipe (seed 0 on the handle's first backward),
+    the router, projections and shared expert in BF16; against the oracle's
+    composition of the same pieces -- dv = G W_upl, the experts' NVFP4
+    backward (oracle.backward_nvfp4), the router through its dL/dw
+    (oracle.backward.router_backward), and the dense gradients -- at the
+    NVFP4 bar (relative RMS 6e-2)."""
+    from oracle import backward as B
+    from tests._parity import make, to64
+    from lmoe_synth import make_grad_out
+    cfg = CONFIGS["tiny_nvfp4"].with_(wq="2d")
+    w, x, layer = make(cfg, backward=True)
+    layer.forward(x)
+    dy = make_grad_out(cfg, T=x.shape[0], device="cuda")
+    grads = layer.grad_buffers()
+    dx = layer.backward(x, dy, grads)
+    torch.cuda.synchronize()
+    assert layer.sync_status() == 0
+    S = layer.debug("topk_idx").numpy().astype(np.int64)
+    X, G = to64(x), to64(dy)
+    Wr, b, Wdn, Wupl = to64(w["w_router"]), to64(w["router_bias"]), to64(w["w_dn"]), to64(w["w_upl"])
+    Ws1, Ws2 = to64(w["w_s1"]), to64(w["w_s2"])
+    S_o, _, gap, s = O.route(X @ Wr.T, b, cfg.K)
+    clear = gap > 1e-3
+    assert np.array_equal(np.sort(S[clear], 1), np.sort(S_o[clear], 1))
+    s_sel = np.take_along_axis(s, S, axis=1)
+    wk = s_sel / s_sel.sum(axis=1, keepdims=True)
+    U = X @ Wdn.T
+    dv = G @ Wupl
+    g_u, g_h = (float(np.float32(v)) for v in act_global_scales(cfg))
+    ref4 = B4.experts_backward_nvfp4(U, S, wk, dv, lambda e: to64(w["w1"][e]),
+                                     lambda e: to64(w["w2"][e]), cfg.N, g_u, g_h, 0)
+    hs_pre = X @ Ws1.T
+    dhs_pre = (G @ Ws2) * 2.0 * np.maximum(hs_pre, 0.0)
+    dz = B.router_backward(s_sel, ref4["dw"], S, cfg.N)
+    v = np.einsum("tk,tkl->tl", wk, ref4["o"])
+    want = {"dx": dhs_pre @ Ws1 + ref4["du"] @ Wdn + dz @ Wr,
+            "d_router": dz.T @ X, "d_dn": ref4["du"].T @ X, "d_s1": dhs_pre.T @ X,
+            "d_s2": G.T @ O.sqrelu(hs_pre), "d_upl": G.T @ v}
+    got = {"dx": to64(dx)}
+    got.update({k: to64(grads[k]) for k in want if k != "dx"})
+    errs = {k: _rms_rel(got[k], want[k]) for k in want}
+    chosen = sorted(ref4["dW1"].keys())
+    errs["dW1"] = _rms_rel(to64(grads["d_w1"])[chosen], np.stack([ref4["dW1"][e] for e in chosen]))
+    errs["dW2"] = _rms_rel(to64(grads["d_w2"])[chosen], np.stack([ref4["dW2"][e] for e in chosen]))
+    print("nvfp4 layer backward", errs)
+    for k, e in errs.items():
+        assert e <= TOL, (k, e)
+    layer.close()
