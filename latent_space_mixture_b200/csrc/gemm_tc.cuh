@@ -697,11 +697,7 @@ __global__ void __launch_bounds__(256) k_splitk_reduce_route(
     for (int i = 0; i < NPL; ++i)
       if (i < npl) zrow[lane + 32 * i] = zz[i];
     __syncwarp();   // the row's logits, written by all lanes, are read back below
-    // candidate lists in shared memory (8 warps x NPL x 32 words) up to 512 experts
-    constexpr int kLists = NPL <= 16 ? 8 * NPL * 32 : 1;
-    __shared__ uint64_t lists[kLists];
-    route_select<NPL>(zz, bb, npl, zrow, K, lane, t, topk_idx, topk_w,
-                      NPL <= 16 ? lists + (threadIdx.x >> 5) * NPL * 32 : nullptr);
+    route_select<NPL>(zz, bb, npl, zrow, K, lane, t, topk_idx, topk_w);
     return;
   }
   const long g = static_cast<long>(blockIdx.x - rblocks) * blockDim.x + threadIdx.x;

@@ -1502,20 +1502,23 @@ static void prof_end(lmoe_handle* h, int slot, cudaStream_t st) {
 #define LMOE_STEP(kidx, call) LMOE_STEP_ON(st, kidx, call)
 
 // SMs for the shared expert on the side stream of an overlapped forward, or
-// 0 for a serial one.  Overlap pays when the grouped GEMMs are bound by HBM:
-// each expert's weights are read once per forward, and below about 256 flops
-// per byte (the ratio of dense BF16 tensor throughput to HBM bandwidth on
-// B200) the tensor pipes wait for them, while the shared expert's dense
-// GEMMs are bound by the tensor pipes.  The side stream gets the share of
-// the SMs that makes the two take about the same time: (shared flops / 256)
-// against the grouped GEMMs' weight bytes.  LMOE_OVERLAP=0 turns it off, a
-// number sets the side stream's SMs.
+// 0 for a serial one.  The idea: when the grouped GEMMs are bound by HBM
+// (below about 256 flops per byte, the ratio of dense BF16 tensor throughput
+// to HBM bandwidth on B200) the tensor pipes wait for the experts' weights,
+// while the shared expert's dense GEMMs are bound by the tensor pipes, so the
+// side stream would get the share of the SMs that makes the two take about
+// the same time: (shared flops / 256) against the grouped GEMMs' weight
+// bytes.  Measured at Ultra dims it loses (7.1 ms against 5.9 serial): one
+// SM streams only ~43 GB/s from HBM, so the grouped GEMMs slow down on fewer
+// SMs as much as the overlap saves.  So it is opt-in: LMOE_OVERLAP=-1 uses
+// that share, a positive number sets the side stream's SMs, 0 or unset
+// keeps the serial forward.
 static int overlap_sms(const lmoe_handle* h, int64_t T) {
   const lmoe_config& c = h->cfg;
   if (!h->proj || h->fp4 || h->fp8 || h->w4 || h->ep_dense || h->shard || !h->pairs ||
       !h->side_st)
     return 0;
-  int side = -1;
+  int side = 0;
   if (const char* e = getenv("LMOE_OVERLAP")) side = atoi(e);
   if (side == 0) return 0;
   const double rows_per_expert = double(T) * c.top_k / c.n_experts;

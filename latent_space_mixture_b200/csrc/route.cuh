@@ -42,16 +42,11 @@ __device__ __forceinline__ void cas_desc(uint64_t& a, uint64_t& b) {
 // token's logits in memory (already written and visible to the warp), from
 // which the selected experts' scores are recomputed with the same
 // expression.  Lanes k < K write slot k of topk_idx / topk_w (row t).
-// lists: this warp's shared-memory scratch of NPL x 32 words, or nullptr:
-// with it, each lane parks its sorted candidates there and a round's winner
-// reads its next head (one load), instead of every lane shifting its whole
-// list in registers.
 template <int NPL>
 __device__ __forceinline__ void route_select(const float (&zz)[NPL], const float (&bb)[NPL],
                                              int npl, const float* z_row, int K, int lane,
                                              int64_t t, int32_t* __restrict__ topk_idx,
-                                             float* __restrict__ topk_w,
-                                             uint64_t* lists = nullptr) {
+                                             float* __restrict__ topk_w) {
   uint64_t cand[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
@@ -76,32 +71,15 @@ __device__ __forceinline__ void route_select(const float (&zz)[NPL], const float
       }
     }
   }
-  // K rounds: the warp maximum of the lanes' heads; the winner moves to its
-  // next candidate
+  // K rounds: the warp maximum of the lanes' heads; the winner shifts its list
   int my_e = 0;
-  if (lists) {
+  for (int k = 0; k < K; ++k) {
+    const uint64_t win = warp_max_u64(cand[0]);
+    if (lane == k) my_e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win));
+    if (cand[0] == win) {
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) lists[i * 32 + lane] = cand[i];
-    __syncwarp();
-    uint64_t head = cand[0];
-    int hi = 0;
-    for (int k = 0; k < K; ++k) {
-      const uint64_t win = warp_max_u64(head);
-      if (lane == k) my_e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win));
-      if (head == win) {
-        ++hi;
-        head = hi < NPL ? lists[hi * 32 + lane] : 0;
-      }
-    }
-  } else {
-    for (int k = 0; k < K; ++k) {
-      const uint64_t win = warp_max_u64(cand[0]);
-      if (lane == k) my_e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(win));
-      if (cand[0] == win) {
-#pragma unroll
-        for (int i = 0; i + 1 < NPL; ++i) cand[i] = cand[i + 1];
-        cand[NPL - 1] = 0;
-      }
+      for (int i = 0; i + 1 < NPL; ++i) cand[i] = cand[i + 1];
+      cand[NPL - 1] = 0;
     }
   }
   // weights: the unbiased scores of the selected experts, renormalised

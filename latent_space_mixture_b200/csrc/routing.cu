@@ -44,11 +44,7 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
     zz[i] = (i < npl) ? z[lane + 32 * i] : 0.0f;
     bb[i] = (i < npl && bias) ? bias[lane + 32 * i] : 0.0f;
   }
-  // candidate lists in shared memory (8 warps x NPL x 32 words) up to 512 experts
-  constexpr int kLists = NPL <= 16 ? 8 * NPL * 32 : 1;
-  __shared__ uint64_t lists[kLists];
-  route_select<NPL>(zz, bb, npl, z, K, lane, t, topk_idx, topk_w,
-                    NPL <= 16 ? lists + (threadIdx.x >> 5) * NPL * 32 : nullptr);
+  route_select<NPL>(zz, bb, npl, z, K, lane, t, topk_idx, topk_w);
 }
 
 cudaError_t launch_route(const float* logits, const float* bias, int64_t T, int N, int K,
