@@ -280,6 +280,9 @@ int lmoe_bias_update(lmoe_handle* h, float rate, void* stream);
  * [255] = f32(1 / f32(6 g)); the activation quantisers use them instead of
  * dividing. */
 #define LMOE_DBG_SCALE_TABLES 27
+/* Handles with LMOE_FLAG_BACKWARD: dL/dv of the last lmoe_backward, bf16
+ * [T][l] (the experts' output gradient before the router weights). */
+#define LMOE_DBG_DV 28
 int lmoe_get_debug(lmoe_handle* h, int what, void* dst_host, size_t bytes);
 
 /* Kernel launches one lmoe_forward of T tokens issues, or a negative error

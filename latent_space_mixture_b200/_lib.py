@@ -26,7 +26,7 @@ DBG = {"topk_idx": 1, "topk_w": 2, "counts": 3, "offsets": 4, "perm": 5, "inv": 
        "w2q_codes": 14, "w2q_sf": 15, "w2q_g": 16, "bias": 17,
        "bw4_do_codes": 18, "bw4_do_sf": 19, "bw4_dot_codes": 20, "bw4_dot_sf": 21,
        "bw4_ut_codes": 22, "bw4_ut_sf": 23, "bw4_scales": 24, "bw4_seg": 25, "bw4_da": 26,
-       "scale_tables": 27}
+       "scale_tables": 27, "dv": 28}
 
 
 class LmoeConfig(Structure):

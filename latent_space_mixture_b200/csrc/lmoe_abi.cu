@@ -2376,6 +2376,9 @@ int lmoe_get_debug(lmoe_handle* h, int what, void* dst, size_t bytes) {
     case LMOE_DBG_W2Q_SF: src = h->w2sf; want = (N * l / 128) * (h->hp / 64) * 512; break;
     case LMOE_DBG_BIAS: src = h->bias; want = N * 4; break;
     case LMOE_DBG_W2Q_G: src = h->fp8 ? h->sw2 : h->gw2; want = N * 4; break;
+    case LMOE_DBG_DV:
+      if (!h->dv) return LMOE_ERR_INVALID_ARG;
+      src = h->dv; want = T * l * 2; break;
     case LMOE_DBG_SCALE_TABLES:
       if (!h->fp4) return LMOE_ERR_INVALID_ARG;
       src = h->stab; want = 2 * NVFP4_TAB * 4; break;

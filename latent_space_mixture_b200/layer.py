@@ -244,6 +244,7 @@ class LatentMoE:
             "v": (torch.bfloat16, (T, c.latent)), "hs": (torch.bfloat16, (T, c.shared_hidden)),
             "bias": (torch.float32, (c.n_experts,)),
             "scale_tables": (torch.float32, (2, 256)),
+            "dv": (torch.bfloat16, (T, c.latent)),
         }
         lp = (c.latent + 255) // 256 * 256
         hp = (c.expert_hidden + 255) // 256 * 256

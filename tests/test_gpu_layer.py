@@ -221,7 +221,9 @@ def test_overlapped_shared_expert_matches_serial_forward(monkeypatch):
     y1 = layer.forward(x)
     torch.cuda.synchronize()
     assert layer.sync_status() == 0
-    assert max_rel(to64(y1), to64(y0)) <= 1e-2
+    # both bf16 outputs within 2e-2 RMS(y) of the oracle: within twice that
+    # of each other
+    assert max_rel(to64(y1), to64(y0)) <= 2 * 2e-2
     toks = np.unique(np.concatenate([[0, cfg.T - 1], _sample(cfg.T, 24, 19)]))
     errs = compare_layer(layer, w, x, y1, toks, cfg.K)
     print("overlapped pair_small errors:", errs)

@@ -154,11 +154,23 @@ def test_nvfp4_experts_backward_no_rows_and_requirements():
 def test_layer_backward_with_nvfp4_experts():
     """lmoe_backward of a layer with 2D-block NVFP4 experts: the routed
     experts under the NVFP4 recipe (seed 0 on the handle's first backward),
-    the router, projections and shared expert in BF16; against the oracle's
-    composition of the same pieces -- dv = G W_upl, the experts' NVFP4
-    backward (oracle.backward_nvfp4), the router through its dL/dw
-    (oracle.backward.router_backward), and the dense gradients -- at the
-    NVFP4 bar (relative RMS 6e-2)."""
+    the router, projections and shared expert in BF16.
+
+      * the layer's expert gradients equal, bit for bit, those of
+        lmoe_experts_backward_nvfp4 on the layer's own saved u, routing and
+        dL/dv (the same kernels on the same values);
+      * the saved u and dL/dv against the oracle's X W_dn^T and G W_upl at
+        the BF16 bar (relative RMS 1e-2);
+      * the oracle's composition of the rest -- the experts' NVFP4 backward
+        (oracle.backward_nvfp4) and the router through its dL/dw
+        (oracle.backward.router_backward) -- fed the layer's own bf16 u and
+        dL/dv and fp32 router weights: the quantised tensors are
+        discontinuous in their inputs (a float64 u instead of the bf16 one
+        moves a fraction of block scales and stochastic-rounding decisions to
+        the neighbouring code, ~0.1 relative RMS on the expert gradients), so
+        the oracle starts where the recipe starts.  The gradients through the
+        experts within the NVFP4 bar (relative RMS 6e-2), dx, the shared
+        expert's and the up-projection's within the BF16 bar."""
     from oracle import backward as B
     from tests._parity import make, to64
     from lmoe_synth import make_grad_out
@@ -170,7 +182,17 @@ def test_layer_backward_with_nvfp4_experts():
     dx = layer.backward(x, dy, grads)
     torch.cuda.synchronize()
     assert layer.sync_status() == 0
-    S = layer.debug("topk_idx").numpy().astype(np.int64)
+    got = {"dx": to64(dx)}
+    got.update({k: to64(v) for k, v in grads.items()})
+    # the expert part: the entry point on the layer's own inputs
+    u, dvg = layer.debug("u"), layer.debug("dv")
+    Sg, wg = layer.debug("topk_idx"), layer.debug("topk_w")
+    again = layer.experts_backward_nvfp4(u.cuda(), Sg.cuda(), wg.cuda(), dvg.cuda(), 0)
+    torch.cuda.synchronize()
+    assert np.array_equal(to64(again["d_w1"]), got["d_w1"])
+    assert np.array_equal(to64(again["d_w2"]), got["d_w2"])
+    # the oracle
+    S = Sg.numpy().astype(np.int64)
     X, G = to64(x), to64(dy)
     Wr, b, Wdn, Wupl = to64(w["w_router"]), to64(w["router_bias"]), to64(w["w_dn"]), to64(w["w_upl"])
     Ws1, Ws2 = to64(w["w_s1"]), to64(w["w_s2"])
@@ -179,25 +201,27 @@ def test_layer_backward_with_nvfp4_experts():
     assert np.array_equal(np.sort(S[clear], 1), np.sort(S_o[clear], 1))
     s_sel = np.take_along_axis(s, S, axis=1)
     wk = s_sel / s_sel.sum(axis=1, keepdims=True)
-    U = X @ Wdn.T
-    dv = G @ Wupl
+    U, dv, wl = to64(u), to64(dvg), wg.numpy().astype(np.float64)
+    assert _rms_rel(U, X @ Wdn.T) <= 1e-2
+    assert _rms_rel(dv, G @ Wupl) <= 1e-2
+    assert np.abs(wl - wk).max() <= 1e-5
     g_u, g_h = (float(np.float32(v)) for v in act_global_scales(cfg))
-    ref4 = B4.experts_backward_nvfp4(U, S, wk, dv, lambda e: to64(w["w1"][e]),
+    ref4 = B4.experts_backward_nvfp4(U, S, wl, dv, lambda e: to64(w["w1"][e]),
                                      lambda e: to64(w["w2"][e]), cfg.N, g_u, g_h, 0)
     hs_pre = X @ Ws1.T
     dhs_pre = (G @ Ws2) * 2.0 * np.maximum(hs_pre, 0.0)
     dz = B.router_backward(s_sel, ref4["dw"], S, cfg.N)
-    v = np.einsum("tk,tkl->tl", wk, ref4["o"])
+    v = np.einsum("tk,tkl->tl", wl, ref4["o"])
     want = {"dx": dhs_pre @ Ws1 + ref4["du"] @ Wdn + dz @ Wr,
             "d_router": dz.T @ X, "d_dn": ref4["du"].T @ X, "d_s1": dhs_pre.T @ X,
             "d_s2": G.T @ O.sqrelu(hs_pre), "d_upl": G.T @ v}
-    got = {"dx": to64(dx)}
-    got.update({k: to64(grads[k]) for k in want if k != "dx"})
-    errs = {k: _rms_rel(got[k], want[k]) for k in want}
     chosen = sorted(ref4["dW1"].keys())
-    errs["dW1"] = _rms_rel(to64(grads["d_w1"])[chosen], np.stack([ref4["dW1"][e] for e in chosen]))
-    errs["dW2"] = _rms_rel(to64(grads["d_w2"])[chosen], np.stack([ref4["dW2"][e] for e in chosen]))
+    errs = {k: _rms_rel(got[k], want[k]) for k in want}
+    errs["d_w1"] = _rms_rel(got["d_w1"][chosen], np.stack([ref4["dW1"][e] for e in chosen]))
+    errs["d_w2"] = _rms_rel(got["d_w2"][chosen], np.stack([ref4["dW2"][e] for e in chosen]))
     print("nvfp4 layer backward", errs)
-    for k, e in errs.items():
-        assert e <= TOL, (k, e)
+    for k in ("dx", "d_s1", "d_s2", "d_upl"):
+        assert errs[k] <= 1e-2, (k, errs[k])
+    for k in ("d_router", "d_dn", "d_w1", "d_w2"):
+        assert errs[k] <= TOL, (k, errs[k])
     layer.close()
