@@ -108,6 +108,21 @@ struct EpiVec<E, std::void_t<decltype(E::kVec)>> {
   static constexpr int value = E::kVec;
 };
 
+// Token-major accumulators: an NVFP4 GEMM with 128-row token blocks whose
+// epilogue declares kTokMajor swaps the MMA operands (tokens in M, features
+// in N; both tiles are 128 K-major rows, so the descriptors and the scale
+// atoms only trade places), so that TMEM holds one token row per lane and a
+// lane's 32 consecutive features come straight from one tcgen05.ld: the
+// epilogue's store32 gets them without the transposing shared-memory tile.
+template <class E, class = void>
+struct EpiTok {
+  static constexpr bool value = false;
+};
+template <class E>
+struct EpiTok<E, std::void_t<decltype(E::kTokMajor)>> {
+  static constexpr bool value = E::kTokMajor;
+};
+
 __device__ __forceinline__ int gemm_num_tiles(const TileSource& s, int BN) {
   if (s.dense == 2) return s.groups * ((s.b_rows + BN - 1) / BN) * s.FB;
   const int nb = s.dense ? (s.T + BN - 1) / BN : *s.nblocks;
@@ -153,7 +168,7 @@ __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int t
   return t;
 }
 
-template <int BN, int STAGES, int KIND, int EPIW = GEMM_EPI_WARPS>
+template <int BN, int STAGES, int KIND, int EPIW = GEMM_EPI_WARPS, bool STG = true>
 struct GemmLayout {
   static constexpr bool FP4 = KIND == KIND_NVFP4;
   static constexpr bool W4 = KIND == KIND_W4A16;
@@ -173,7 +188,8 @@ struct GemmLayout {
   static constexpr int EPI_WARPS = EPIW;
   static_assert(EPIW % 4 == 0 && EPIW >= 4 && EPIW <= 16, "epilogue warps per lane quarter");
   static constexpr int THREADS = 64 + 32 * EPI_WARPS + (W4 ? W4_CONV_THREADS : 0);   // + converters
-  static constexpr int STG_BYTES = EPI_WARPS * 32 * GEMM_STG_LD * 4;
+  // the transposing staging tile (none with token-major accumulators)
+  static constexpr int STG_BYTES = STG ? EPI_WARPS * 32 * GEMM_STG_LD * 4 : 0;
   static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8;
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ +
                                     STAGES * (A_BYTES + B_BYTES + SF_BYTES + RAW_BYTES) +
@@ -206,18 +222,21 @@ struct GemmEpiWarps {
 
 // Ring depth: `want` stages, or as many as fit in shared memory beside the
 // epilogue staging.
-template <int BN, int KIND, int EPIW>
+template <int BN, int KIND, int EPIW, bool STG = true>
 constexpr int gemm_fit_stages(int want) {
+  using L2 = GemmLayout<BN, 2, KIND, EPIW, STG>;
   int s = want;
-  while (s > 2 && GemmLayout<BN, 2, KIND, EPIW>::SMEM_BYTES +
-                          (s - 2) * (GemmLayout<BN, 2, KIND, EPIW>::A_BYTES +
-                                     GemmLayout<BN, 2, KIND, EPIW>::B_BYTES +
-                                     GemmLayout<BN, 2, KIND, EPIW>::SF_BYTES +
-                                     GemmLayout<BN, 2, KIND, EPIW>::RAW_BYTES + 24) >
-                      232448)
+  while (s > 2 && L2::SMEM_BYTES + (s - 2) * (L2::A_BYTES + L2::B_BYTES + L2::SF_BYTES +
+                                               L2::RAW_BYTES + 24) > 232448)
     --s;
   return s;
 }
+
+// whether variant (BN, Epi, KIND) runs with token-major accumulators
+template <int BN, class Epi, int KIND>
+struct GemmTok {
+  static constexpr bool value = KIND == KIND_NVFP4 && BN == GEMM_BM && EpiTok<Epi>::value;
+};
 
 // "empty" barrier of ring slot s, and whether the producer waits on it there
 template <class L>
@@ -228,15 +247,18 @@ template <class L>
 __device__ __forceinline__ bool empty_commits_at(int s) { return !L::PAIRED_RELEASE || (s & 1); }
 
 template <int BN, int STAGES, class Epi, int KIND>
-__global__ void __launch_bounds__(GemmLayout<BN, STAGES, KIND, GemmEpiWarps<BN, Epi>::value>::THREADS, 1)
+__global__ void __launch_bounds__(GemmLayout<BN, STAGES, KIND, GemmEpiWarps<BN, Epi>::value,
+                                             !GemmTok<BN, Epi, KIND>::value>::THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmB64, const TileSource src, const Epi epi, int* err,
           unsigned long long limit_ns) {
-  using L = GemmLayout<BN, STAGES, KIND, GemmEpiWarps<BN, Epi>::value>;
+  using L = GemmLayout<BN, STAGES, KIND, GemmEpiWarps<BN, Epi>::value,
+                       !GemmTok<BN, Epi, KIND>::value>;
   constexpr bool FP4 = KIND == KIND_NVFP4;
   constexpr bool F8 = KIND == KIND_FP8;
   constexpr bool W4 = KIND == KIND_W4A16;
   constexpr bool BYTE_MAPS = FP4 || F8;   // operand maps in bytes (128 per stage row)
+  constexpr bool TOK = GemmTok<BN, Epi, KIND>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -408,7 +430,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const TileInfo t = gemm_tile(src, BN, tile);
       if (t.kb0 >= t.kb1) continue;   // an empty K range: no accumulator, no epilogue
-      const int n_mma = (t.nrows + 15) & ~15;
+      const int n_mma = TOK ? GEMM_BM : (t.nrows + 15) & ~15;
       if (!__all_sync(0xffffffffu,
                       mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err, limit_ns))) {
         ok = false;
@@ -449,9 +471,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                   sdesc_sf_atom(sf_smem + FP4_SF_STAGE_BYTES + k * SF_ATOM_BYTES));
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k)   // +32 bytes per K=64 step
-              umma_nvf4(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, tmem_base + sf_col + 4 * k,
-                        tmem_base + sf_col + 16 + 4 * k, (kb != t.kb0) || (k != 0));
+            for (int k = 0; k < 4; ++k) {   // +32 bytes per K=64 step
+              if constexpr (TOK)
+                umma_nvf4(d_tmem, b0 + 2 * k, a0 + 2 * k, idesc, tmem_base + sf_col + 16 + 4 * k,
+                          tmem_base + sf_col + 4 * k, (kb != t.kb0) || (k != 0));
+              else
+                umma_nvf4(d_tmem, a0 + 2 * k, b0 + 2 * k, idesc, tmem_base + sf_col + 4 * k,
+                          tmem_base + sf_col + 16 + 4 * k, (kb != t.kb0) || (k != 0));
+            }
           } else if constexpr (F8) {
 #pragma unroll
             for (int k = 0; k < 4; ++k)   // +32 bytes per K=32 step
@@ -509,6 +536,23 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       if (lane == 0) ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err, limit_ns);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
+      if constexpr (TOK) {
+        // lane = token row q*32 + lane of the tile; 32 features per TMEM load
+        const int rbase = q * 32;
+        if (rbase < t.nrows) {
+          for (int c = cfirst; c < GEMM_BM; c += cstep) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c, r);
+            tmem_ld_wait();
+            const int feat = t.fb * GEMM_BM + c;
+            const bool valid = rbase + lane < t.nrows && feat < src.m_valid;
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            epi.store32(t, static_cast<long>(t.row0 + rbase + lane), feat, v, valid);
+          }
+        }
+      } else {
       const int feat_base = t.fb * GEMM_BM + q * 32;
       for (int c0 = cfirst; c0 < t.nrows; c0 += cstep) {
         uint32_t r[32];
@@ -559,6 +603,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           }
         }
         __syncwarp();
+      }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

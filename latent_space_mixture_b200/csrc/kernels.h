@@ -93,8 +93,7 @@ cudaError_t launch_quant_rows_dev(const float* x, int64_t rows, int cols, const 
                                   uint8_t* scales, float* g_out, cudaStream_t st);
 cudaError_t launch_atoms_rblock(const uint8_t* scales, const int32_t* rblock, int64_t R, int nkb,
                                 int kp64, uint8_t* atoms, cudaStream_t st);
-cudaError_t launch_atoms_dense(const uint8_t* scales, int64_t rows, int nkb, uint8_t* atoms,
-                               cudaStream_t st);
+
 cudaError_t launch_dw_rows(const void* O, const int32_t* inv, const void* dv, int64_t T, int K,
                            int l, float* dw, cudaStream_t st);
 cudaError_t launch_seg_offsets(const int32_t* counts, int N, int32_t* po16, int32_t* po256,
@@ -109,13 +108,17 @@ struct TSrc {
   int fp64;                // NVFP4 rows: 64-element chunks per row of the atoms
   float g;                 // NVFP4 rows: global scale
 };
-cudaError_t launch_transpose_rht(int src_kind, const TSrc& s, const int32_t* offsets,
-                                 const int32_t* counts, const int32_t* po256, int N, int F,
-                                 int64_t pitch, uint64_t seed, float* out, float* amax,
-                                 cudaStream_t st);
-cudaError_t launch_quant_t(const float* x, int F, int64_t pitch, const int32_t* po16,
-                           const int32_t* po256, int N, const float* amax, bool sr, uint64_t seed,
-                           uint8_t* codes, uint8_t* scales, float* g_out, cudaStream_t st);
+// transposed, transformed operands of the weight-gradient GEMMs: pass 1 the
+// amax, pass 2 codes, canonical scales and scale atoms (nvfp4_bw.cu)
+cudaError_t launch_tq_amax(int src_kind, const TSrc& s, const int32_t* offsets,
+                           const int32_t* counts, const int32_t* po16, const int32_t* po256,
+                           int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
+                           cudaStream_t st);
+cudaError_t launch_tq_quant(int src_kind, bool sr, const TSrc& s, const int32_t* offsets,
+                            const int32_t* counts, const int32_t* po16, const int32_t* po256,
+                            int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
+                            uint64_t seed_sr, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
+                            float* g_out, cudaStream_t st);
 cudaError_t launch_zero_empty(const int32_t* counts, int N, int64_t per, float* dw,
                               cudaStream_t st);
 cudaError_t launch_transpose_w2d(const uint8_t* codes, const uint8_t* atoms, int E, int R, int C,

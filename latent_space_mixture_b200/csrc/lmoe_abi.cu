@@ -135,9 +135,25 @@ struct EpiY {
   int d;
   const bf16* resid;
   int ldr;
+  float* yf = nullptr;             // fp32 output [T][d] instead of y (the side stream's W_s2 hs)
+  const float* residf = nullptr;   // fp32 residual [T][d], added before y's one rounding
   __device__ __forceinline__ void store8(const TileInfo&, long row, int feat, const float* v,
                                          bool valid) const {
     if (!valid) return;
+    if (yf) {
+      float4* p = reinterpret_cast<float4*>(yf + row * d + feat);
+      p[0] = make_float4(v[0], v[1], v[2], v[3]);
+      p[1] = make_float4(v[4], v[5], v[6], v[7]);
+      return;
+    }
+    if (residf) {
+      const float4* p = reinterpret_cast<const float4*>(residf + row * d + feat);
+      const float4 r0 = p[0], r1 = p[1];
+      const float a[8] = {v[0] + r0.x, v[1] + r0.y, v[2] + r0.z, v[3] + r0.w,
+                          v[4] + r1.x, v[5] + r1.y, v[6] + r1.z, v[7] + r1.w};
+      store8_bf16(y + row * d + feat, a);
+      return;
+    }
     if (resid) {
       const uint4 raw = *reinterpret_cast<const uint4*>(resid + row * ldr + feat);
       const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -170,6 +186,41 @@ struct EpiHq {
   const float* tab_h;    // scale tables of g_h (nvfp4_scale_tab)
   bf16* a16 = nullptr;   // NVFP4 training: the pre-activation a = W1[e] u, bf16 [R][ha]
   int ha = 0;
+  static constexpr bool kTokMajor = true;
+  // 32 consecutive features of one token row (token-major accumulators): two
+  // NVFP4 blocks, 16 bytes of codes and two adjacent scale bytes
+  __device__ __forceinline__ void store32(const TileInfo& t, long row, int feat, const float* v,
+                                          bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(gw1[t.e], g_u);
+    float a[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a[i] = sqrelu(v[i] * s);
+    uint32_t w[4];
+    uint8_t sc[2];
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, a[16 * b + i]);   // a >= 0
+      float r;
+      sc[b] = nvfp4_scale_tab(amax, tab_h, &r);
+      w[2 * b] = e2m1x8(a + 16 * b, r);
+      w[2 * b + 1] = e2m1x8(a + 16 * b + 8, r);
+    }
+    *reinterpret_cast<uint4*>(Hq + row * (hp / 2) + feat / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint16_t*>(
+        sfh + (static_cast<long>(t.tb) * (hp / 64) + feat / 64) * SF_ATOM_BYTES +
+        sf_atom_offset(static_cast<int>(row - t.row0), (feat & 63) >> 4)) =
+        static_cast<uint16_t>(sc[0] | (sc[1] << 8));
+    if (a16) {
+      float pre[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pre[i] = v[i] * s;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) store8_bf16(a16 + row * ha + feat + 8 * i, pre + 8 * i);
+    }
+  }
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
                                          bool valid) const {
     const float s = __fmul_rn(gw1[t.e], g_u);
@@ -233,6 +284,17 @@ struct EpiOq {
   const float* gw2;
   float g_h;
   int l;
+  static constexpr bool kTokMajor = true;
+  __device__ __forceinline__ void store32(const TileInfo& t, long row, int feat, const float* v,
+                                          bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(__fmul_rn(gw2[t.e], g_h), wrow ? wrow[row] : 1.0f);
+    float a[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a[i] = v[i] * s;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) store8_bf16(O + row * l + feat + 8 * i, a + 8 * i);
+  }
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
                                          bool valid) const {
     if (!valid) return;
@@ -256,6 +318,36 @@ struct EpiDA {
   const float* g_do;   // device scalar
   int h;
   float* amax;
+  static constexpr bool kTokMajor = true;
+  __device__ __forceinline__ void store32(const TileInfo& t, long row, int feat, const float* v,
+                                          bool valid) const {
+    float m = 0.0f;
+    if (valid) {
+      const float s = __fmul_rn(gw2[t.e], *g_do);
+      const uint4* ap = reinterpret_cast<const uint4*>(a16 + row * h + feat);
+      float4* p = reinterpret_cast<float4*>(da + row * h + feat);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 raw = ap[c];
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 a = __bfloat1622float2(a2[i]);
+          o[2 * i] = __fmul_rn(__fmul_rn(v[8 * c + 2 * i] * s, 2.0f), fmaxf(a.x, 0.0f));
+          o[2 * i + 1] = __fmul_rn(__fmul_rn(v[8 * c + 2 * i + 1] * s, 2.0f), fmaxf(a.y, 0.0f));
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(o[i]));
+        p[2 * c] = make_float4(o[0], o[1], o[2], o[3]);
+        p[2 * c + 1] = make_float4(o[4], o[5], o[6], o[7]);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0 && __float_as_int(m) > *reinterpret_cast<volatile int*>(amax))
+      atomicMax(reinterpret_cast<int*>(amax), __float_as_int(m));
+  }
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
                                          bool valid) const {
     float m = 0.0f;
@@ -291,6 +383,17 @@ struct EpiDU {
   const float* gw1;
   const float* g_da;   // device scalar
   int l;
+  static constexpr bool kTokMajor = true;
+  __device__ __forceinline__ void store32(const TileInfo& t, long row, int feat, const float* v,
+                                          bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(gw1[t.e], *g_da);
+    float o[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] = v[i] * s;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) store8_bf16(du + row * l + feat + 8 * i, o + 8 * i);
+  }
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
                                          bool valid) const {
     if (!valid) return;
@@ -310,6 +413,16 @@ struct EpiWq {
   int rows, cols;
   const float* g_a;   // device scalars
   const float* g_b;
+  static constexpr bool kTokMajor = true;
+  __device__ __forceinline__ void store32(const TileInfo& t, long row, int feat, const float* v,
+                                          bool valid) const {
+    if (!valid) return;
+    const float s = __fmul_rn(*g_a, *g_b);
+    float4* p = reinterpret_cast<float4*>(out + (static_cast<long>(t.e) * rows + row) * cols + feat);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      p[i] = make_float4(v[4 * i] * s, v[4 * i + 1] * s, v[4 * i + 2] * s, v[4 * i + 3] * s);
+  }
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
                                          bool valid) const {
     if (!valid) return;
@@ -560,7 +673,7 @@ struct Stages {
 };
 template <>
 struct Stages<128, KIND_NVFP4> {
-  static constexpr int value = 5;
+  static constexpr int value = 6;
 };
 template <>
 struct Stages<32, KIND_NVFP4> {
@@ -581,8 +694,9 @@ struct Stages<32, KIND_W4A16> {
 template <int BN, class Epi, int KIND>
 struct StagesOf {
   static constexpr int EPIW = GemmEpiWarps<BN, Epi>::value;
-  static constexpr int value = gemm_fit_stages<BN, KIND, EPIW>(Stages<BN, KIND>::value);
-  using L = GemmLayout<BN, value, KIND, EPIW>;
+  static constexpr bool STG = !GemmTok<BN, Epi, KIND>::value;
+  static constexpr int value = gemm_fit_stages<BN, KIND, EPIW, STG>(Stages<BN, KIND>::value);
+  using L = GemmLayout<BN, value, KIND, EPIW, STG>;
 };
 
 template <int BN, class Epi, int KIND = KIND_BF16>
@@ -932,8 +1046,6 @@ struct lmoe_handle {
   int32_t* kofs = nullptr;     // [N+1] FP4 k-steps of po256
   float* scal = nullptr;       // [16]: amax 0..7, global scales 8..15
   int64_t rp_cap = 0;          // columns of the transposed operands
-  float* X1 = nullptr;         // [max(l,h)][rp_cap] fp32 transposed, transformed
-  float* X2 = nullptr;
   // transposed operands: 0 do^T (B of dW2), 1 g^T (A of dW2), 2 u^T (A of
   // dW1), 3 da^T (B of dW1): codes [F][rp_cap/2], scales [F][rp_cap/16], atoms
   uint8_t* tq[4] = {};
@@ -947,7 +1059,7 @@ struct lmoe_handle {
   // GEMMs on a side stream over a share of the SMs
   cudaStream_t side_st = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-  bf16* ys = nullptr;          // [max_tokens][d] W_s2 hs
+  float* ys = nullptr;         // [max_tokens][d] W_s2 hs (fp32)
   CUtensorMap tm_ws1, tm_ws2;  // W_s1 rows of w_x; W_s2 columns of w_y
   BMaps tm_hs;                 // hs columns of vh
   std::vector<void*> allocs;
@@ -1151,7 +1263,6 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     return LMOE_ERR_UNSUPPORTED;
   }
   h->rp_cap = rp_cap;
-  const int64_t fmax = l > hh ? l : hh;
   const int64_t tf[4] = {l, hh, l, hh};   // features of the transposed operands
   struct Req {
     void** p;
@@ -1212,7 +1323,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->dwacc, size_t(bwx * rows * 4)},
       {(void**)&h->dxh, size_t(bwx * Tm_b * (N + l + hs) * 2)},
       {(void**)&h->dy_dev, size_t(bwx * GEMM_BROWS_BIG * d * 2)},
-      {(void**)&h->ys, size_t((bfx && proj) ? Tm * d * 2 : 0)},
+      {(void**)&h->ys, size_t((bfx && proj) ? Tm * d * 4 : 0)},
       {(void**)&h->w1qT, size_t(bw4 * N * l * hp / 2)},
       {(void**)&h->w1qT_sf, size_t(bw4 * (N * l / 128) * (hp / 64) * 512)},
       {(void**)&h->w2qT, size_t(bw4 * N * hh * lp / 2)},
@@ -1230,8 +1341,6 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->po256, size_t(bw4 * (N + 1) * 4)},
       {(void**)&h->kofs, size_t(bw4 * (N + 1) * 4)},
       {(void**)&h->scal, size_t(bw4 * 64)},
-      {(void**)&h->X1, size_t(bw4 * fmax * rp_cap * 4)},
-      {(void**)&h->X2, size_t(bw4 * fmax * rp_cap * 4)},
       {(void**)&h->tq[0], size_t(bw4 * tf[0] * rp_cap / 2)},
       {(void**)&h->tq[1], size_t(bw4 * tf[1] * rp_cap / 2)},
       {(void**)&h->tq[2], size_t(bw4 * tf[2] * rp_cap / 2)},
@@ -1573,7 +1682,7 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st, 
       TileSource s1{1, static_cast<int>(T), nullptr, nullptr, (hs + PAIR_BM - 1) / PAIR_BM, 0, hs,
                     static_cast<int>(d / 64), 1, nullptr, 0};
       LMOE_STEP_ON(ss, 24, launch_gemm_pair(h->tm_ws1, tm_x, s1, e1, side / 2, h->err, lim, ss));
-      EpiY e2{h->ys, static_cast<int>(d), nullptr, 0};
+      EpiY e2{nullptr, static_cast<int>(d), nullptr, 0, h->ys};
       TileSource s2{1, static_cast<int>(T), nullptr, nullptr,
                     static_cast<int>((d + PAIR_BM - 1) / PAIR_BM), 0, static_cast<int>(d), hs / 64,
                     1, nullptr, 0};
@@ -1640,9 +1749,8 @@ static int fwd_ygemm(lmoe_handle* h, int64_t T, void* y, cudaStream_t st, bool o
     const DensePlan p = plan_dense(T, fb, ky / 64, h->sms);
     if (p.ksplit > 1 && int64_t(p.ksplit) * T * d > h->part_floats)
       return LMOE_ERR_UNSUPPORTED;   // never: the buffer is sized for every T
-    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d),
-             overlapped ? h->ys : h->proj ? nullptr : h->vh,
-             overlapped ? static_cast<int>(d) : ldvh};
+    EpiY epi{static_cast<bf16*>(y), static_cast<int>(d), h->proj ? nullptr : h->vh, ldvh,
+             nullptr, overlapped ? h->ys : nullptr};
     const int fb2 = static_cast<int>((d + PAIR_BM - 1) / PAIR_BM);
     const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
     if (h->pairs && ptiles >= h->sms / 2) {
@@ -2261,16 +2369,16 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
   TSrc src_da{h->da32, nullptr, nullptr, nullptr, K, 0, 0, 0.f};
   TSrc src_u{u, h->perm, nullptr, nullptr, K, 0, 0, 0.f};
   // dW2[e] = Q_sr(R(do_e^T)) Q(R(g_e^T))^T: A = g^T (features h), B = do^T (rows l)
-  LMOE_STEP(20, launch_transpose_rht(2, src_g, h->offsets, h->counts, h->po256, N, hh, pitch,
-                                     seed + 2, h->X2, amax + 3, st));
-  LMOE_STEP(20, launch_transpose_rht(0, src_do, h->offsets, h->counts, h->po256, N, l, pitch,
-                                     seed + 2, h->X1, amax + 2, st));
-  LMOE_STEP(20, launch_quant_t(h->X2, hh, pitch, h->po16, h->po256, N, amax + 3, false, 0,
-                               h->tq[1], h->ts[1], gsc + 3, st));
-  LMOE_STEP(20, launch_atoms_dense(h->ts[1], hh, static_cast<int>(pitch / 16), h->ta[1], st));
-  LMOE_STEP(20, launch_quant_t(h->X1, l, pitch, h->po16, h->po256, N, amax + 2, true, seed + 3,
-                               h->tq[0], h->ts[0], gsc + 2, st));
-  LMOE_STEP(20, launch_atoms_dense(h->ts[0], l, static_cast<int>(pitch / 16), h->ta[0], st));
+  LMOE_STEP(20, launch_tq_amax(2, src_g, h->offsets, h->counts, h->po16, h->po256, N, hh, pitch,
+                               seed + 2, amax + 3, st));
+  LMOE_STEP(20, launch_tq_amax(0, src_do, h->offsets, h->counts, h->po16, h->po256, N, l, pitch,
+                               seed + 2, amax + 2, st));
+  LMOE_STEP(20, launch_tq_quant(2, false, src_g, h->offsets, h->counts, h->po16, h->po256, N, hh,
+                                pitch, seed + 2, amax + 3, 0, h->tq[1], h->ts[1], h->ta[1],
+                                gsc + 3, st));
+  LMOE_STEP(20, launch_tq_quant(0, true, src_do, h->offsets, h->counts, h->po16, h->po256, N, l,
+                                pitch, seed + 2, amax + 2, seed + 3, h->tq[0], h->ts[0], h->ta[0],
+                                gsc + 2, st));
   {
     TileSource s{2, 0, nullptr, nullptr, hh / 128, 0, hh, 0, 1, nullptr, 0, h->ta[1], h->ta[0],
                  static_cast<int>(kc), h->kofs, N, l};
@@ -2279,16 +2387,16 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
                                             lim, st));
   }
   // dW1[e] = Q_sr(R(da_e^T)) Q(R(u_e^T))^T: A = u^T (features l), B = da^T (rows h)
-  LMOE_STEP(21, launch_transpose_rht(1, src_u, h->offsets, h->counts, h->po256, N, l, pitch,
-                                     seed + 4, h->X1, amax + 5, st));
-  LMOE_STEP(21, launch_transpose_rht(0, src_da, h->offsets, h->counts, h->po256, N, hh, pitch,
-                                     seed + 4, h->X2, amax + 4, st));
-  LMOE_STEP(21, launch_quant_t(h->X1, l, pitch, h->po16, h->po256, N, amax + 5, false, 0,
-                               h->tq[2], h->ts[2], gsc + 5, st));
-  LMOE_STEP(21, launch_atoms_dense(h->ts[2], l, static_cast<int>(pitch / 16), h->ta[2], st));
-  LMOE_STEP(21, launch_quant_t(h->X2, hh, pitch, h->po16, h->po256, N, amax + 4, true, seed + 5,
-                               h->tq[3], h->ts[3], gsc + 4, st));
-  LMOE_STEP(21, launch_atoms_dense(h->ts[3], hh, static_cast<int>(pitch / 16), h->ta[3], st));
+  LMOE_STEP(21, launch_tq_amax(1, src_u, h->offsets, h->counts, h->po16, h->po256, N, l, pitch,
+                               seed + 4, amax + 5, st));
+  LMOE_STEP(21, launch_tq_amax(0, src_da, h->offsets, h->counts, h->po16, h->po256, N, hh, pitch,
+                               seed + 4, amax + 4, st));
+  LMOE_STEP(21, launch_tq_quant(1, false, src_u, h->offsets, h->counts, h->po16, h->po256, N, l,
+                                pitch, seed + 4, amax + 5, 0, h->tq[2], h->ts[2], h->ta[2],
+                                gsc + 5, st));
+  LMOE_STEP(21, launch_tq_quant(0, true, src_da, h->offsets, h->counts, h->po16, h->po256, N, hh,
+                                pitch, seed + 4, amax + 4, seed + 5, h->tq[3], h->ts[3], h->ta[3],
+                                gsc + 4, st));
   {
     TileSource s{2, 0, nullptr, nullptr, l / 128, 0, l, 0, 1, nullptr, 0, h->ta[2], h->ta[3],
                  static_cast<int>(kc), h->kofs, N, hh};

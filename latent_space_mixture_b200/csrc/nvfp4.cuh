@@ -38,6 +38,23 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
   return r;
 }
 
+// Eight floats times r to eight E2M1 codes in one word: element i in bits
+// 4i..4i+3 (the byte layout of e2m1x2, four bytes packed lowest first).
+__device__ __forceinline__ uint32_t e2m1x8(const float* x, float r) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(w)
+      : "f"(__fmul_rn(x[0], r)), "f"(__fmul_rn(x[1], r)), "f"(__fmul_rn(x[2], r)),
+        "f"(__fmul_rn(x[3], r)), "f"(__fmul_rn(x[4], r)), "f"(__fmul_rn(x[5], r)),
+        "f"(__fmul_rn(x[6], r)), "f"(__fmul_rn(x[7], r)));
+  return w;
+}
+
 __device__ __forceinline__ uint8_t e4m3_code(float x) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
 }
@@ -47,10 +64,12 @@ __device__ __forceinline__ float e4m3_value(uint8_t code) {
   return __half2float(__half(h));
 }
 
-// E2M1 code (bit 3 = sign) -> value
+// E2M1 code (bit 3 = sign) -> value: magnitudes 0, 0.5, 1, 1.5 (codes 0-3,
+// code / 2), 2, 3 (codes 4-5, code - 2), 4, 6 (codes 6-7, 2 code - 8)
 __device__ __forceinline__ float e2m1_value(uint32_t code) {
-  const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
-  const float v = mag[code & 7];
+  const int m = static_cast<int>(code & 7);
+  const float v = m < 4 ? 0.5f * static_cast<float>(m)
+                        : static_cast<float>(m < 6 ? m - 2 : 2 * m - 8);
   return (code & 8) ? -v : v;
 }
 
@@ -110,14 +129,18 @@ __device__ __forceinline__ uint8_t nvfp4_block(const float (&x)[16], float g, ui
 // with inv6g lands within one code of it, and one comparison corrects it.
 constexpr int NVFP4_TAB = 256;   // thr [0, 128), rtab [128, 255), inv6g [255]
 
+// (The five table entries the correction may need are loaded together, so
+// that the lookup costs one load latency.)
 __device__ __forceinline__ uint8_t nvfp4_scale_tab(float amax, const float* __restrict__ tab,
                                                    float* r) {
   int code = e4m3_code(__fmul_rn(amax, tab[255]));
   code = code > 126 ? 126 : code;
-  if (amax >= tab[code + 1]) ++code;
-  else if (amax < tab[code]) --code;
-  *r = tab[128 + code];
-  return static_cast<uint8_t>(code);
+  const float t0 = tab[code], t1 = tab[code + 1];
+  const float r_dn = tab[128 + (code > 0 ? code - 1 : 0)], r_0 = tab[128 + code],
+              r_up = tab[128 + code + 1];
+  const bool up = amax >= t1, dn = !up && amax < t0;
+  *r = up ? r_up : dn ? r_dn : r_0;
+  return static_cast<uint8_t>(code + (up ? 1 : 0) - (dn ? 1 : 0));
 }
 
 // ---------------------------------------------------------------------------
@@ -149,29 +172,41 @@ __device__ __forceinline__ float uniform24(uint64_t seed, uint64_t ctr) {
 // neighbour with probability (|v| - lo) / (hi - lo), the lower otherwise;
 // |v| >= 6 saturates.  The probability is exact in float32 (hi - lo is a
 // power of two, |v| - lo is exact).
+// The grid step is 0.5 below 2, 1 below 4 and 2 below 6, so lo = floor(|v| /
+// step) step, |v| - lo (exact: lo <= |v| < 2 lo or lo = 0) and its quotient
+// by the step (a power of two) are all exact products, without a division.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, float u) {
   const float mag = fabsf(v);
   uint32_t code;
   if (mag >= 6.0f) {
     code = 7;
   } else {
-    const int lo = mag < 0.5f ? 0 : mag < 1.0f ? 1 : mag < 1.5f ? 2 : mag < 2.0f ? 3
-                 : mag < 3.0f ? 4 : mag < 4.0f ? 5 : 6;
-    const float lo_v = e2m1_value(static_cast<uint32_t>(lo));
-    const float hi_v = e2m1_value(static_cast<uint32_t>(lo + 1));
-    const float p = __fdiv_rn(__fsub_rn(mag, lo_v), __fsub_rn(hi_v, lo_v));
+    const bool b0 = mag < 2.0f, b1 = mag < 4.0f;
+    const float inv = b0 ? 2.0f : b1 ? 1.0f : 0.5f;      // 1 / step
+    const float k = floorf(mag * inv);
+    const float p = __fsub_rn(mag * inv, k);              // (|v| - lo) / step
+    const int lo = b0 ? static_cast<int>(k) : b1 ? static_cast<int>(k) + 2 : 6;
     code = static_cast<uint32_t>(u < p ? lo + 1 : lo);
   }
   return code | (signbit(v) ? 8u : 0u);
 }
 
 // y = (1/4) H16 (s * x) on one 16-element block, in place: signs s from
-// counters 0..15 of `seed`, float32 butterflies (stages 1, 2, 4, 8:
-// (a, b) -> (a + b, a - b)), then the exact product by 0.25.
-__device__ __forceinline__ void rht16_block(float (&b)[16], uint64_t seed) {
+// counters 0..15 of `seed` (rht16_signs: bit j set for sign -1), float32
+// butterflies (stages 1, 2, 4, 8: (a, b) -> (a + b, a - b)), then the exact
+// product by 0.25.
+__device__ __forceinline__ uint32_t rht16_signs(uint64_t seed) {
+  uint32_t m = 0;
 #pragma unroll
   for (int j = 0; j < 16; ++j)
-    if (splitmix64(seed, static_cast<uint64_t>(j)) >> 63) b[j] = -b[j];
+    m |= static_cast<uint32_t>(splitmix64(seed, static_cast<uint64_t>(j)) >> 63) << j;
+  return m;
+}
+
+__device__ __forceinline__ void rht16_masked(float (&b)[16], uint32_t signs) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    if ((signs >> j) & 1u) b[j] = -b[j];
 #pragma unroll
   for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
@@ -184,6 +219,10 @@ __device__ __forceinline__ void rht16_block(float (&b)[16], uint64_t seed) {
   }
 #pragma unroll
   for (int j = 0; j < 16; ++j) b[j] = b[j] * 0.25f;
+}
+
+__device__ __forceinline__ void rht16_block(float (&b)[16], uint64_t seed) {
+  rht16_masked(b, rht16_signs(seed));
 }
 
 }  // namespace lmoe

@@ -235,32 +235,6 @@ cudaError_t launch_atoms_rblock(const uint8_t* scales, const int32_t* rblock, in
                     rblock, R, nkb, kp64, atoms);
 }
 
-// Canonical scales of a dense matrix [rows][nkb] (rows a multiple of 128) ->
-// its scale atoms [rows / 128][nkb / 4][512].
-__global__ void __launch_bounds__(256) k_atoms_dense(const uint8_t* __restrict__ scales,
-                                                     int64_t rows, int nkb,
-                                                     uint8_t* __restrict__ atoms) {
-  pdl_wait();
-  pdl_trigger();
-  const int ng = nkb / 4;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= rows * ng) return;
-  const int64_t r = i / ng;
-  const int c = static_cast<int>(i - r * ng);
-  const int64_t off =
-      ((r >> 7) * ng + c) * SF_ATOM_BYTES + sf_atom_offset(static_cast<int>(r & 127), 0);
-  *reinterpret_cast<uint32_t*>(atoms + off) =
-      *reinterpret_cast<const uint32_t*>(scales + r * nkb + 4 * c);
-}
-
-cudaError_t launch_atoms_dense(const uint8_t* scales, int64_t rows, int nkb, uint8_t* atoms,
-                               cudaStream_t st) {
-  const int64_t n = rows * (nkb / 4);
-  if (n <= 0) return cudaSuccess;
-  return launch_pdl(k_atoms_dense, static_cast<unsigned>((n + 255) / 256), 256, 0, st, scales,
-                    rows, nkb, atoms);
-}
-
 // ---------------------------------------------------------------------------
 // dL/dw of every routed (token, slot): dw[t][k] = o[inv[t][k]] . dv[t], o the
 // experts' unweighted outputs (bf16 rows), fp32 in a fixed order (lane
@@ -342,17 +316,30 @@ __device__ __forceinline__ int seg_of(const int32_t* po256, int N, int col) {
 }
 
 // ---------------------------------------------------------------------------
-// Transposed, transformed operand of a weight-gradient GEMM: out[f][col]
-// (row pitch `pitch` floats) for the 16-column block of every thread's
-// column group: expert e's rows j0 .. j0 + 15 of feature f (zero past its
-// c_e rows), through the random Hadamard transform of `seed`; and its amax.
+// Transposed, transformed, quantised operand of a weight-gradient GEMM, in
+// two passes over its source and no intermediate tensor.  Element
+// (f, po256[e] + j) is expert e's row j of feature f (zero past its c_e
+// rows); each 16-column block goes through the random Hadamard transform of
+// seed_rht.
+//   pass 1 (STORE false): the transformed tensor's amax (atomicMax into
+//          *amax);
+//   pass 2 (STORE true): its NVFP4 codes [F][pitch / 2], canonical scales
+//          [F][pitch / 16] and scale atoms [F / 128][pitch / 64][512] under
+//          the global scale of *amax (also written to *g_out); stochastic
+//          rounding (SR) with the counters of the 16-padded layout: element
+//          (f, po256[e] + j) uses f W16 + po16[e] + j, W16 = po16[N] (the
+//          padding past a segment's 16-row multiple is zero, which rounds to
+//          zero whatever its counter).
 // Sources (rows in expert order unless stated):
 //   SRC 0: fp32 rows [R][F];
 //   SRC 1: bf16 token rows [T][F], routed row r reading token perm[r] / K;
 //   SRC 2: NVFP4 rows, codes [R][code_pitch] and B-operand scale atoms
 //          ([block][Fp/64][512] by rblock), dequantised with global scale g.
-// A thread per (feature, 16-column block); blocks past the layout's width
-// (po256[N], on the device) do nothing.
+// A thread per (feature, 64-column group): consecutive threads read
+// consecutive features of a row, and a thread's 32 bytes of codes and 4
+// scales are contiguous.  A 64-column group lies inside one segment (the
+// segments are 256-aligned); groups past the layout's width (po256[N], on
+// the device) do nothing.
 
 template <int SRC>
 __device__ __forceinline__ float t_load(const TSrc& s, int64_t r, int f, int F) {
@@ -372,108 +359,120 @@ __device__ __forceinline__ float t_load(const TSrc& s, int64_t r, int f, int F) 
   }
 }
 
-template <int SRC>
-__global__ void __launch_bounds__(128) k_transpose_rht(TSrc s, const int32_t* __restrict__ offsets,
-                                                       const int32_t* __restrict__ counts,
-                                                       const int32_t* __restrict__ po256, int N,
-                                                       int F, int64_t pitch, uint64_t seed,
-                                                       float* __restrict__ out, float* amax) {
+template <int SRC, bool SR, bool STORE>
+__global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ offsets,
+                                            const int32_t* __restrict__ counts,
+                                            const int32_t* __restrict__ po16,
+                                            const int32_t* __restrict__ po256, int N, int F,
+                                            int64_t pitch, uint64_t seed_rht, float* amax,
+                                            uint64_t seed_sr, uint8_t* __restrict__ codes,
+                                            uint8_t* __restrict__ scales,
+                                            uint8_t* __restrict__ atoms, float* g_out) {
   pdl_wait();
   pdl_trigger();
-  const int bb = blockIdx.y;                      // 16-column block
-  const int col0 = bb * 16;
+  const int col0 = blockIdx.y * 64;
   if (col0 >= po256[N]) return;
   const int f = blockIdx.x * blockDim.x + threadIdx.x;
   const int e = seg_of(po256, N, col0);
   const int j0 = col0 - po256[e];
   const int ce = counts[e];
   const int64_t r0 = offsets[e];
-  float v[16];
+  const uint32_t signs = rht16_signs(seed_rht);
+  float g = 0.0f;
+  if constexpr (STORE) {
+    g = gscale_of(*amax);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
+  }
   float m = 0.0f;
   if (f < F) {
+    uint32_t cw[8];
+    uint32_t sw = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = (j0 + i < ce) ? t_load<SRC>(s, r0 + j0 + i, f, F) : 0.0f;
-    rht16_block(v, seed);
-    float4* dst = reinterpret_cast<float4*>(out + f * pitch + col0);
+    for (int bk = 0; bk < 4; ++bk) {
+      const int jb = j0 + 16 * bk;
+      float v[16];
+      if (jb < ce) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        for (int i = 0; i < 16; ++i) v[i] = (jb + i < ce) ? t_load<SRC>(s, r0 + jb + i, f, F) : 0.0f;
+        rht16_masked(v, signs);
+      } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+      }
+      if constexpr (!STORE) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+      } else {
+        const uint64_t c0 =
+            SR ? static_cast<uint64_t>(f) * static_cast<uint64_t>(po16[N]) + po16[e] + jb : 0;
+        uint8_t q[8];
+        const uint8_t sc = quant16<SR>(v, g, seed_sr, c0, q);
+        cw[2 * bk] = *reinterpret_cast<const uint32_t*>(q);
+        cw[2 * bk + 1] = *reinterpret_cast<const uint32_t*>(q + 4);
+        sw |= static_cast<uint32_t>(sc) << (8 * bk);
+      }
+    }
+    if constexpr (STORE) {
+      uint4* dst = reinterpret_cast<uint4*>(codes + f * (pitch / 2) + col0 / 2);
+      dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      *reinterpret_cast<uint32_t*>(scales + f * (pitch / 16) + col0 / 16) = sw;
+      *reinterpret_cast<uint32_t*>(
+          atoms + ((static_cast<int64_t>(f) >> 7) * (pitch / 64) + col0 / 64) * SF_ATOM_BYTES +
+          sf_atom_offset(f & 127, 0)) = sw;
+    }
   }
-  m = warp_max_f(m);
-  if ((threadIdx.x & 31) == 0) atomic_max_nonneg(amax, m);
+  if constexpr (!STORE) {
+    m = warp_max_f(m);
+    if ((threadIdx.x & 31) == 0) atomic_max_nonneg(amax, m);
+  }
 }
 
-cudaError_t launch_transpose_rht(int src_kind, const TSrc& s, const int32_t* offsets,
-                                 const int32_t* counts, const int32_t* po256, int N, int F,
-                                 int64_t pitch, uint64_t seed, float* out, float* amax,
-                                 cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>((F + 127) / 128), static_cast<unsigned>(pitch / 16));
-  if (src_kind == 0)
-    return launch_pdl(k_transpose_rht<0>, grid, 128, 0, st, s, offsets, counts, po256, N, F,
-                      pitch, seed, out, amax);
-  if (src_kind == 1)
-    return launch_pdl(k_transpose_rht<1>, grid, 128, 0, st, s, offsets, counts, po256, N, F,
-                      pitch, seed, out, amax);
-  return launch_pdl(k_transpose_rht<2>, grid, 128, 0, st, s, offsets, counts, po256, N, F, pitch,
-                    seed, out, amax);
+template <int SRC, bool SR, bool STORE>
+static cudaError_t launch_tq_v(const TSrc& s, const int32_t* offsets, const int32_t* counts,
+                               const int32_t* po16, const int32_t* po256, int N, int F,
+                               int64_t pitch, uint64_t seed_rht, float* amax, uint64_t seed_sr,
+                               uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* g_out,
+                               cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>((F + 127) / 128), static_cast<unsigned>(pitch / 64));
+  return launch_pdl(k_tq<SRC, SR, STORE>, grid, 128, 0, st, s, offsets, counts, po16, po256, N,
+                    F, pitch, seed_rht, amax, seed_sr, codes, scales, atoms, g_out);
 }
 
-// ---------------------------------------------------------------------------
-// Quantisation of a transposed operand [F][pitch] fp32 (columns < po256[N])
-// into codes [F][pitch / 2] and canonical scales [F][pitch / 16], global
-// scale from the amax (also written to *g_out).  Stochastic rounding takes
-// the counters of the 16-padded layout: element (f, po256[e] + j) uses
-// f W16 + po16[e] + j, W16 = po16[N] (the padding past a segment's 16-row
-// multiple is zero, which rounds to zero whatever its counter).
-
-template <bool SR>
-__global__ void __launch_bounds__(256) k_quant_t(const float* __restrict__ x, int F, int64_t pitch,
-                                                 const int32_t* __restrict__ po16,
-                                                 const int32_t* __restrict__ po256, int N,
-                                                 const float* amax, uint64_t seed,
-                                                 uint8_t* __restrict__ codes,
-                                                 uint8_t* __restrict__ scales, float* g_out) {
-  pdl_wait();
-  pdl_trigger();
-  const int64_t nb = pitch / 16;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const float g = gscale_of(*amax);
-  if (i == 0) *g_out = g;
-  if (i >= static_cast<int64_t>(F) * nb) return;
-  const int64_t f = i / nb;
-  const int bb = static_cast<int>(i - f * nb);
-  const int col0 = bb * 16;
-  if (col0 >= po256[N]) return;
-  const float4* src = reinterpret_cast<const float4*>(x + f * pitch + col0);
-  float v[16];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float4 q4 = src[j];
-    v[4 * j] = q4.x;
-    v[4 * j + 1] = q4.y;
-    v[4 * j + 2] = q4.z;
-    v[4 * j + 3] = q4.w;
+cudaError_t launch_tq_amax(int src_kind, const TSrc& s, const int32_t* offsets,
+                           const int32_t* counts, const int32_t* po16, const int32_t* po256,
+                           int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
+                           cudaStream_t st) {
+  switch (src_kind) {
+    case 0: return launch_tq_v<0, false, false>(s, offsets, counts, po16, po256, N, F, pitch,
+                                                seed_rht, amax, 0, nullptr, nullptr, nullptr,
+                                                nullptr, st);
+    case 1: return launch_tq_v<1, false, false>(s, offsets, counts, po16, po256, N, F, pitch,
+                                                seed_rht, amax, 0, nullptr, nullptr, nullptr,
+                                                nullptr, st);
+    default: return launch_tq_v<2, false, false>(s, offsets, counts, po16, po256, N, F, pitch,
+                                                 seed_rht, amax, 0, nullptr, nullptr, nullptr,
+                                                 nullptr, st);
   }
-  uint64_t c0 = 0;
-  if (SR) {
-    const int e = seg_of(po256, N, col0);
-    c0 = static_cast<uint64_t>(f) * static_cast<uint64_t>(po16[N]) + po16[e] + (col0 - po256[e]);
-  }
-  uint8_t q[8];
-  scales[f * nb + bb] = quant16<SR>(v, g, seed, c0, q);
-  *reinterpret_cast<uint2*>(codes + f * (pitch / 2) + bb * 8) = *reinterpret_cast<const uint2*>(q);
 }
 
-cudaError_t launch_quant_t(const float* x, int F, int64_t pitch, const int32_t* po16,
-                           const int32_t* po256, int N, const float* amax, bool sr, uint64_t seed,
-                           uint8_t* codes, uint8_t* scales, float* g_out, cudaStream_t st) {
-  const int64_t n = static_cast<int64_t>(F) * (pitch / 16);
-  const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
-  return sr ? launch_pdl(k_quant_t<true>, blocks, 256, 0, st, x, F, pitch, po16, po256, N, amax,
-                         seed, codes, scales, g_out)
-            : launch_pdl(k_quant_t<false>, blocks, 256, 0, st, x, F, pitch, po16, po256, N, amax,
-                         seed, codes, scales, g_out);
+cudaError_t launch_tq_quant(int src_kind, bool sr, const TSrc& s, const int32_t* offsets,
+                            const int32_t* counts, const int32_t* po16, const int32_t* po256,
+                            int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
+                            uint64_t seed_sr, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
+                            float* g_out, cudaStream_t st) {
+  // the recipe's four operands: gradients (SRC 0) stochastically rounded,
+  // activations (SRC 1, 2) rounded to nearest
+  if (src_kind == 0 && sr)
+    return launch_tq_v<0, true, true>(s, offsets, counts, po16, po256, N, F, pitch, seed_rht,
+                                      amax, seed_sr, codes, scales, atoms, g_out, st);
+  if (src_kind == 1 && !sr)
+    return launch_tq_v<1, false, true>(s, offsets, counts, po16, po256, N, F, pitch, seed_rht,
+                                       amax, 0, codes, scales, atoms, g_out, st);
+  if (src_kind == 2 && !sr)
+    return launch_tq_v<2, false, true>(s, offsets, counts, po16, po256, N, F, pitch, seed_rht,
+                                       amax, 0, codes, scales, atoms, g_out, st);
+  return cudaErrorInvalidValue;
 }
 
 // ---------------------------------------------------------------------------

@@ -170,7 +170,9 @@ def test_layer_backward_with_nvfp4_experts():
         the neighbouring code, ~0.1 relative RMS on the expert gradients), so
         the oracle starts where the recipe starts.  The gradients through the
         experts within the NVFP4 bar (relative RMS 6e-2), dx, the shared
-        expert's and the up-projection's within the BF16 bar."""
+        expert's and the up-projection's within the BF16 bar (the
+        up-projection's from the forward's v, whose u was quantised from the
+        fp32 accumulator)."""
     from oracle import backward as B
     from tests._parity import make, to64
     from lmoe_synth import make_grad_out
@@ -211,7 +213,11 @@ def test_layer_backward_with_nvfp4_experts():
     hs_pre = X @ Ws1.T
     dhs_pre = (G @ Ws2) * 2.0 * np.maximum(hs_pre, 0.0)
     dz = B.router_backward(s_sel, ref4["dw"], S, cfg.N)
-    v = np.einsum("tk,tkl->tl", wl, ref4["o"])
+    # the forward quantised u from its fp32 accumulator, not from the saved
+    # bf16 u: its v against the oracle's forward on the unrounded u
+    o_fwd = B4.experts_backward_nvfp4(X @ Wdn.T, S, wk, G @ Wupl, lambda e: to64(w["w1"][e]),
+                                      lambda e: to64(w["w2"][e]), cfg.N, g_u, g_h, 0)["o"]
+    v = np.einsum("tk,tkl->tl", wk, o_fwd)
     want = {"dx": dhs_pre @ Ws1 + ref4["du"] @ Wdn + dz @ Wr,
             "d_router": dz.T @ X, "d_dn": ref4["du"].T @ X, "d_s1": dhs_pre.T @ X,
             "d_s2": G.T @ O.sqrelu(hs_pre), "d_upl": G.T @ v}
