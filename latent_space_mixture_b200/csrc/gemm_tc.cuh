@@ -168,7 +168,12 @@ __device__ __forceinline__ TileInfo gemm_tile(const TileSource& s, int BN, int t
   return t;
 }
 
-template <int BN, int STAGES, int KIND, int EPIW = GEMM_EPI_WARPS, bool STG = true>
+// epilogue staging of a variant: none (token-major accumulators), the
+// transposing tile, or two 32 x 32 fp32 boxes per warp for TMA stores
+constexpr int STG_NONE = 0, STG_TRANSPOSE = 1, STG_BOXES = 2;
+constexpr int GEMM_BOX_FLOATS = 32 * 32;
+
+template <int BN, int STAGES, int KIND, int EPIW = GEMM_EPI_WARPS, int STG = STG_TRANSPOSE>
 struct GemmLayout {
   static constexpr bool FP4 = KIND == KIND_NVFP4;
   static constexpr bool W4 = KIND == KIND_W4A16;
@@ -188,8 +193,9 @@ struct GemmLayout {
   static constexpr int EPI_WARPS = EPIW;
   static_assert(EPIW % 4 == 0 && EPIW >= 4 && EPIW <= 16, "epilogue warps per lane quarter");
   static constexpr int THREADS = 64 + 32 * EPI_WARPS + (W4 ? W4_CONV_THREADS : 0);   // + converters
-  // the transposing staging tile (none with token-major accumulators)
-  static constexpr int STG_BYTES = STG ? EPI_WARPS * 32 * GEMM_STG_LD * 4 : 0;
+  static constexpr int STG_BYTES = STG == STG_TRANSPOSE ? EPI_WARPS * 32 * GEMM_STG_LD * 4
+                                   : STG == STG_BOXES   ? EPI_WARPS * 2 * GEMM_BOX_FLOATS * 4
+                                                        : 0;
   static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8;
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ +
                                     STAGES * (A_BYTES + B_BYTES + SF_BYTES + RAW_BYTES) +
@@ -222,7 +228,7 @@ struct GemmEpiWarps {
 
 // Ring depth: `want` stages, or as many as fit in shared memory beside the
 // epilogue staging.
-template <int BN, int KIND, int EPIW, bool STG = true>
+template <int BN, int KIND, int EPIW, int STG = STG_TRANSPOSE>
 constexpr int gemm_fit_stages(int want) {
   using L2 = GemmLayout<BN, 2, KIND, EPIW, STG>;
   int s = want;
@@ -238,6 +244,41 @@ struct GemmTok {
   static constexpr bool value = KIND == KIND_NVFP4 && BN == GEMM_BM && EpiTok<Epi>::value;
 };
 
+// An fp32 token-major epilogue may declare kTmaBoxes: each warp's 32 x 32
+// chunk (rows = TMEM lanes, 32 consecutive features) goes out as one TMA
+// store from a 128-byte-swizzled box (a lane writes its row's eight 16-byte
+// pieces at positions c ^ (row % 8): no bank conflicts), instead of 32
+// lanes each storing to its own row.  The functor gives the chunk's scale
+// (scale(t)) and its place (target(t, row, feat, &map, &x, &y)).
+template <class E, class = void>
+struct EpiBoxes {
+  static constexpr bool value = false;
+};
+template <class E>
+struct EpiBoxes<E, std::void_t<decltype(E::kTmaBoxes)>> {
+  static constexpr bool value = E::kTmaBoxes;
+};
+
+// A token-major epilogue that reads a second operand per element may declare
+// kPre32: pre32(t, row, feat, valid, p) loads the 64 bytes of its chunk into
+// p before the accumulator wait (so the load overlaps the tile's MMAs), and
+// store32 takes them as a sixth argument.
+template <class E, class = void>
+struct EpiPre {
+  static constexpr bool value = false;
+};
+template <class E>
+struct EpiPre<E, std::void_t<decltype(E::kPre32)>> {
+  static constexpr bool value = E::kPre32;
+};
+
+template <int BN, class Epi, int KIND>
+struct GemmStg {
+  static constexpr int value = !GemmTok<BN, Epi, KIND>::value ? STG_TRANSPOSE
+                               : EpiBoxes<Epi>::value        ? STG_BOXES
+                                                             : STG_NONE;
+};
+
 // "empty" barrier of ring slot s, and whether the producer waits on it there
 template <class L>
 __device__ __forceinline__ int empty_slot(int s) { return L::PAIRED_RELEASE ? s >> 1 : s; }
@@ -248,12 +289,12 @@ __device__ __forceinline__ bool empty_commits_at(int s) { return !L::PAIRED_RELE
 
 template <int BN, int STAGES, class Epi, int KIND>
 __global__ void __launch_bounds__(GemmLayout<BN, STAGES, KIND, GemmEpiWarps<BN, Epi>::value,
-                                             !GemmTok<BN, Epi, KIND>::value>::THREADS, 1)
+                                             GemmStg<BN, Epi, KIND>::value>::THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const __grid_constant__ CUtensorMap tmB64, const TileSource src, const Epi epi, int* err,
-          unsigned long long limit_ns) {
+          const __grid_constant__ CUtensorMap tmB64, const TileSource src,
+          const __grid_constant__ Epi epi, int* err, unsigned long long limit_ns) {
   using L = GemmLayout<BN, STAGES, KIND, GemmEpiWarps<BN, Epi>::value,
-                       !GemmTok<BN, Epi, KIND>::value>;
+                       GemmStg<BN, Epi, KIND>::value>;
   constexpr bool FP4 = KIND == KIND_NVFP4;
   constexpr bool F8 = KIND == KIND_FP8;
   constexpr bool W4 = KIND == KIND_W4A16;
@@ -526,11 +567,23 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const int cstep = 32 * (L::EPI_WARPS / 4);   // column chunks: this warp's, then every cstep
     const int cfirst = 32 * (ew / 4);
     float* my = stg + ew * 32 * GEMM_STG_LD;
+    int nbox = 0;   // TMA boxes this warp has stored (kTmaBoxes epilogues)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const TileInfo t = gemm_tile(src, BN, tile);
       if (t.kb0 >= t.kb1) continue;   // skipped by the MMA warp too
+      // token-major: this warp's chunks c = cfirst + i * cstep, i < NCH
+      constexpr int NCH = GEMM_BM / (32 * (L::EPI_WARPS / 4));
+      [[maybe_unused]] uint4 pre[TOK && EpiPre<Epi>::value ? NCH : 1][4];
+      if constexpr (TOK && EpiPre<Epi>::value) {
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          const int feat = t.fb * GEMM_BM + cfirst + i * cstep;
+          const bool valid = q * 32 + lane < t.nrows && feat < src.m_valid;
+          epi.pre32(t, static_cast<long>(t.row0 + q * 32 + lane), feat, valid, pre[i]);
+        }
+      }
       // one lane waits, the warp follows: the TMEM loads below are .sync.aligned
       int ok = 0;
       if (lane == 0) ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err, limit_ns);
@@ -540,16 +593,49 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         // lane = token row q*32 + lane of the tile; 32 features per TMEM load
         const int rbase = q * 32;
         if (rbase < t.nrows) {
-          for (int c = cfirst; c < GEMM_BM; c += cstep) {
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            const int c = cfirst + i * cstep;
             uint32_t r[32];
             tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c, r);
             tmem_ld_wait();
             const int feat = t.fb * GEMM_BM + c;
-            const bool valid = rbase + lane < t.nrows && feat < src.m_valid;
-            float v[32];
+            if constexpr (EpiBoxes<Epi>::value) {
+              // whole chunks only: rows and features come in multiples of 32
+              if (feat < src.m_valid) {
+                float* box = stg + (ew * 2 + (nbox & 1)) * GEMM_BOX_FLOATS;
+                // the box stored two chunks ago has been read out of this buffer
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+                const float sc = epi.scale(t);
+                float4* row = reinterpret_cast<float4*>(box + lane * 32);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-            epi.store32(t, static_cast<long>(t.row0 + rbase + lane), feat, v, valid);
+                for (int k = 0; k < 8; ++k)
+                  row[k ^ (lane & 7)] =
+                      make_float4(__uint_as_float(r[4 * k]) * sc, __uint_as_float(r[4 * k + 1]) * sc,
+                                  __uint_as_float(r[4 * k + 2]) * sc,
+                                  __uint_as_float(r[4 * k + 3]) * sc);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  const CUtensorMap* map;
+                  int x, y;
+                  epi.target(t, static_cast<long>(t.row0 + rbase), feat, &map, &x, &y);
+                  tma_store_2d(map, box, x, y);
+                  bulk_commit_group();
+                }
+                ++nbox;
+              }
+            } else {
+              const bool valid = rbase + lane < t.nrows && feat < src.m_valid;
+              float v[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+              if constexpr (EpiPre<Epi>::value)
+                epi.store32(t, static_cast<long>(t.row0 + rbase + lane), feat, v, valid, pre[i]);
+              else
+                epi.store32(t, static_cast<long>(t.row0 + rbase + lane), feat, v, valid);
+            }
           }
         }
       } else {
@@ -611,6 +697,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         acc = 0;
         acc_phase ^= 1;
       }
+    }
+    if constexpr (TOK && EpiBoxes<Epi>::value) {
+      // the boxes' reads of shared memory end before the CTA does
+      if (lane == 0) bulk_wait_group_read<0>();
+      __syncwarp();
     }
   }
 

@@ -319,16 +319,23 @@ struct EpiDA {
   int h;
   float* amax;
   static constexpr bool kTokMajor = true;
+  static constexpr bool kPre32 = true;
+  // the chunk's 32 saved pre-activations, loaded before the accumulator wait
+  __device__ __forceinline__ void pre32(const TileInfo&, long row, int feat, bool valid,
+                                        uint4 (&p)[4]) const {
+    const uint4* ap = reinterpret_cast<const uint4*>(a16 + row * h + feat);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) p[c] = valid ? ap[c] : make_uint4(0u, 0u, 0u, 0u);
+  }
   __device__ __forceinline__ void store32(const TileInfo& t, long row, int feat, const float* v,
-                                          bool valid) const {
+                                          bool valid, const uint4 (&pa)[4]) const {
     float m = 0.0f;
     if (valid) {
       const float s = __fmul_rn(gw2[t.e], *g_do);
-      const uint4* ap = reinterpret_cast<const uint4*>(a16 + row * h + feat);
       float4* p = reinterpret_cast<float4*>(da + row * h + feat);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const uint4 raw = ap[c];
+        const uint4 raw = pa[c];
         const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
         float o[8];
 #pragma unroll
@@ -406,14 +413,24 @@ struct EpiDU {
 };
 
 // NVFP4 weight gradient of one expert (group): out[e][row][feat] =
-// g_a g_b * acc, fp32, row = B row, feat = A row.
+// g_a g_b * acc, fp32, row = B row, feat = A row; stored by TMA through the
+// map m of out ([E * rows][cols] fp32, 32 x 32 boxes, 128-byte swizzle).
 struct EpiWq {
   static constexpr int kWarps = 8;
   float* out;
   int rows, cols;
   const float* g_a;   // device scalars
   const float* g_b;
+  CUtensorMap m;
   static constexpr bool kTokMajor = true;
+  static constexpr bool kTmaBoxes = true;
+  __device__ __forceinline__ float scale(const TileInfo&) const { return __fmul_rn(*g_a, *g_b); }
+  __device__ __forceinline__ void target(const TileInfo& t, long row, int feat,
+                                         const CUtensorMap** mp, int* x, int* y) const {
+    *mp = &m;
+    *x = feat;
+    *y = t.e * rows + static_cast<int>(row);
+  }
   __device__ __forceinline__ void store32(const TileInfo& t, long row, int feat, const float* v,
                                           bool valid) const {
     if (!valid) return;
@@ -694,7 +711,7 @@ struct Stages<32, KIND_W4A16> {
 template <int BN, class Epi, int KIND>
 struct StagesOf {
   static constexpr int EPIW = GemmEpiWarps<BN, Epi>::value;
-  static constexpr bool STG = !GemmTok<BN, Epi, KIND>::value;
+  static constexpr int STG = GemmStg<BN, Epi, KIND>::value;
   static constexpr int value = gemm_fit_stages<BN, KIND, EPIW, STG>(Stages<BN, KIND>::value);
   using L = GemmLayout<BN, value, KIND, EPIW, STG>;
 };
@@ -880,6 +897,20 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_
 // 2-D fp32 row-major [rows][cols] matrix written by TMA stores of 32 x 32
 // boxes, no swizzle (cols * 4 a multiple of 16 bytes); out-of-range elements
 // of a box are not written.
+// fp32 [rows][cols] output map with 32 x 32 boxes stored from 128-byte-swizzled
+// shared memory (the token-major epilogues' boxes)
+static bool make_map_f32_out_sw(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static bool make_map_f32_out(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   PFN_encodeTiled enc = get_encode();
   if (!enc) return false;
@@ -2382,7 +2413,8 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
   {
     TileSource s{2, 0, nullptr, nullptr, hh / 128, 0, hh, 0, 1, nullptr, 0, h->ta[1], h->ta[0],
                  static_cast<int>(kc), h->kofs, N, l};
-    EpiWq epi{d_w2, l, hh, gsc + 3, gsc + 2};
+    EpiWq epi{d_w2, l, hh, gsc + 3, gsc + 2, {}};
+    if (!make_map_f32_out_sw(&epi.m, d_w2, int64_t(N) * l, hh)) return LMOE_ERR_CUDA;
     LMOE_STEP(20, launch_gemm_q<KIND_NVFP4>(128, h->tm_tA[1], h->tm_tB[0], s, epi, h->sms, h->err,
                                             lim, st));
   }
@@ -2400,7 +2432,8 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
   {
     TileSource s{2, 0, nullptr, nullptr, l / 128, 0, l, 0, 1, nullptr, 0, h->ta[2], h->ta[3],
                  static_cast<int>(kc), h->kofs, N, hh};
-    EpiWq epi{d_w1, hh, l, gsc + 5, gsc + 4};
+    EpiWq epi{d_w1, hh, l, gsc + 5, gsc + 4, {}};
+    if (!make_map_f32_out_sw(&epi.m, d_w1, int64_t(N) * hh, l)) return LMOE_ERR_CUDA;
     LMOE_STEP(21, launch_gemm_q<KIND_NVFP4>(128, h->tm_tA[2], h->tm_tB[3], s, epi, h->sms, h->err,
                                             lim, st));
   }

@@ -54,6 +54,14 @@ __device__ __forceinline__ uint8_t quant16(const float (&v)[16], float g, uint64
     float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    if (amax == 0.0f) {
+      // every element rounds to a zero of its own sign: no random bits needed
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        q[j] = static_cast<uint8_t>((signbit(v[2 * j]) ? 8u : 0u) |
+                                    (signbit(v[2 * j + 1]) ? 128u : 0u));
+      return 0;
+    }
     const float six_g = __fmul_rn(6.0f, g);
     const float sbf = six_g > 0.0f ? __fdiv_rn(amax, six_g) : 0.0f;
     const uint8_t sc = e4m3_code(sbf);
@@ -335,27 +343,73 @@ __device__ __forceinline__ int seg_of(const int32_t* po256, int N, int col) {
 //   SRC 1: bf16 token rows [T][F], routed row r reading token perm[r] / K;
 //   SRC 2: NVFP4 rows, codes [R][code_pitch] and B-operand scale atoms
 //          ([block][Fp/64][512] by rblock), dequantised with global scale g.
-// A thread per (feature, 64-column group): consecutive threads read
-// consecutive features of a row, and a thread's 32 bytes of codes and 4
-// scales are contiguous.  A 64-column group lies inside one segment (the
-// segments are 256-aligned); groups past the layout's width (po256[N], on
-// the device) do nothing.
+// A CTA per (128 features, 64-column group): the group's source rows are
+// staged in shared memory with coalesced loads, then a thread takes one
+// feature (a column of the tile), so its 32 bytes of codes and 4 scales are
+// contiguous.  A 64-column group lies inside one segment (the segments are
+// 256-aligned); groups past the layout's width (po256[N], on the device) do
+// nothing.
+
+// The CTA's source tile, rows [0, nr) x features [f0, f0 + 128) of its
+// 64-row group, as floats in shared memory (rows read with coalesced vector
+// loads; NVFP4 rows dequantised 8 codes at a time).
+constexpr int TQ_PITCH = 129;
 
 template <int SRC>
-__device__ __forceinline__ float t_load(const TSrc& s, int64_t r, int f, int F) {
+__device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, int f0, int F,
+                                         float (*tile)[TQ_PITCH]) {
+  const int t = threadIdx.x;
   if constexpr (SRC == 0) {
-    return static_cast<const float*>(s.p)[r * F + f];
+    // fp32 rows: 32 float4 per row
+    for (int i = t; i < nr * 32; i += 128) {
+      const int row = i >> 5, q = i & 31;
+      const int f = f0 + 4 * q;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (f < F) x = *reinterpret_cast<const float4*>(static_cast<const float*>(s.p) +
+                                                       (rbase + row) * F + f);
+      tile[row][4 * q] = x.x;
+      tile[row][4 * q + 1] = x.y;
+      tile[row][4 * q + 2] = x.z;
+      tile[row][4 * q + 3] = x.w;
+    }
   } else if constexpr (SRC == 1) {
-    const int64_t tok = s.perm[r] / s.K;
-    return __bfloat162float(static_cast<const bf16*>(s.p)[tok * F + f]);
+    // bf16 token rows: 16 x 8 elements per row
+    for (int i = t; i < nr * 16; i += 128) {
+      const int row = i >> 4, q = i & 15;
+      const int f = f0 + 8 * q;
+      const int64_t tok = s.perm[rbase + row] / s.K;
+      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+      if (f < F) raw = *reinterpret_cast<const uint4*>(static_cast<const bf16*>(s.p) + tok * F + f);
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 v = __bfloat1622float2(p2[k]);
+        tile[row][8 * q + 2 * k] = v.x;
+        tile[row][8 * q + 2 * k + 1] = v.y;
+      }
+    }
   } else {
-    const uint8_t byte = static_cast<const uint8_t*>(s.p)[r * s.code_pitch + f / 2];
-    const uint32_t code = (f & 1) ? (byte >> 4) : (byte & 15);
-    const int rb = s.rblock[r];
-    const int b = rb >> 8, j = rb & 255;
-    const uint8_t sc = s.atoms[(static_cast<int64_t>(b) * s.fp64 + f / 64) * SF_ATOM_BYTES +
-                               sf_atom_offset(j, (f & 63) >> 4)];
-    return __fmul_rn(__fmul_rn(e2m1_value(code), e4m3_value(sc)), s.g);
+    // NVFP4 rows: 16 words of 8 codes per row, each with its 16-block's scale
+    for (int i = t; i < nr * 16; i += 128) {
+      const int row = i >> 4, q = i & 15;
+      const int f = f0 + 8 * q;
+      const int64_t r = rbase + row;
+      if (f >= F) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) tile[row][8 * q + k] = 0.0f;
+        continue;
+      }
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(s.p) +
+                                                            r * s.code_pitch + f / 2);
+      const int rb = s.rblock[r];
+      const int b = rb >> 8, j = rb & 255;
+      const uint8_t sc = s.atoms[(static_cast<int64_t>(b) * s.fp64 + f / 64) * SF_ATOM_BYTES +
+                                 sf_atom_offset(j, (f & 63) >> 4)];
+      const float scv = e4m3_value(sc);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)   // (code x scale) x g, the dequantisation order
+        tile[row][8 * q + k] = __fmul_rn(__fmul_rn(e2m1_value((w >> (4 * k)) & 15u), scv), s.g);
+    }
   }
 }
 
@@ -368,15 +422,19 @@ __global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ 
                                             uint64_t seed_sr, uint8_t* __restrict__ codes,
                                             uint8_t* __restrict__ scales,
                                             uint8_t* __restrict__ atoms, float* g_out) {
+  __shared__ float tile[64][TQ_PITCH];
   pdl_wait();
   pdl_trigger();
   const int col0 = blockIdx.y * 64;
   if (col0 >= po256[N]) return;
-  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  const int f0 = blockIdx.x * 128;
+  const int f = f0 + threadIdx.x;
   const int e = seg_of(po256, N, col0);
   const int j0 = col0 - po256[e];
   const int ce = counts[e];
-  const int64_t r0 = offsets[e];
+  const int nr = min(64, ce - j0);   // rows of this group that hold data (may be <= 0)
+  if (nr > 0) tq_stage<SRC>(s, static_cast<int64_t>(offsets[e]) + j0, nr, f0, F, tile);
+  __syncthreads();
   const uint32_t signs = rht16_signs(seed_rht);
   float g = 0.0f;
   if constexpr (STORE) {
@@ -389,22 +447,22 @@ __global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ 
     uint32_t sw = 0;
 #pragma unroll
     for (int bk = 0; bk < 4; ++bk) {
-      const int jb = j0 + 16 * bk;
-      float v[16];
-      if (jb < ce) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = (jb + i < ce) ? t_load<SRC>(s, r0 + jb + i, f, F) : 0.0f;
-        rht16_masked(v, signs);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+      if (16 * bk >= nr) {
+        // past the segment's rows: zeros, scale 0
+        cw[2 * bk] = cw[2 * bk + 1] = 0u;
+        continue;
       }
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = (16 * bk + i < nr) ? tile[16 * bk + i][threadIdx.x] : 0.0f;
+      rht16_masked(v, signs);
       if constexpr (!STORE) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
       } else {
-        const uint64_t c0 =
-            SR ? static_cast<uint64_t>(f) * static_cast<uint64_t>(po16[N]) + po16[e] + jb : 0;
+        const uint64_t c0 = SR ? static_cast<uint64_t>(f) * static_cast<uint64_t>(po16[N]) +
+                                     po16[e] + j0 + 16 * bk
+                               : 0;
         uint8_t q[8];
         const uint8_t sc = quant16<SR>(v, g, seed_sr, c0, q);
         cw[2 * bk] = *reinterpret_cast<const uint32_t*>(q);
