@@ -97,7 +97,7 @@ cudaError_t launch_atoms_rblock(const uint8_t* scales, const int32_t* rblock, in
 cudaError_t launch_dw_rows(const void* O, const int32_t* inv, const void* dv, int64_t T, int K,
                            int l, float* dw, cudaStream_t st);
 cudaError_t launch_seg_offsets(const int32_t* counts, int N, int32_t* po16, int32_t* po256,
-                               int32_t* kofs, cudaStream_t st);
+                               int32_t* kofs, int32_t* grp, cudaStream_t st);
 struct TSrc {
   const void* p;           // rows: fp32 [R][F], bf16 token rows [T][F], or NVFP4 codes
   const int32_t* perm;     // bf16 token rows: routed row -> t * K + k
@@ -112,11 +112,11 @@ struct TSrc {
 // amax, pass 2 codes, canonical scales and scale atoms (nvfp4_bw.cu)
 cudaError_t launch_tq_amax(int src_kind, const TSrc& s, const int32_t* offsets,
                            const int32_t* counts, const int32_t* po16, const int32_t* po256,
-                           int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
+                           const int32_t* grp, int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
                            cudaStream_t st);
 cudaError_t launch_tq_quant(int src_kind, bool sr, const TSrc& s, const int32_t* offsets,
                             const int32_t* counts, const int32_t* po16, const int32_t* po256,
-                            int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
+                            const int32_t* grp, int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
                             uint64_t seed_sr, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
                             float* g_out, cudaStream_t st);
 cudaError_t launch_zero_empty(const int32_t* counts, int N, int64_t per, float* dw,

@@ -1075,6 +1075,7 @@ struct lmoe_handle {
   int32_t* po16 = nullptr;     // [N+1] columns, segments padded to 16
   int32_t* po256 = nullptr;    // [N+1] columns, segments padded to 256
   int32_t* kofs = nullptr;     // [N+1] FP4 k-steps of po256
+  int32_t* grp = nullptr;      // [rp_cap / 64] expert of each 64-column group
   float* scal = nullptr;       // [16]: amax 0..7, global scales 8..15
   int64_t rp_cap = 0;          // columns of the transposed operands
   // transposed operands: 0 do^T (B of dW2), 1 g^T (A of dW2), 2 u^T (A of
@@ -1371,6 +1372,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->po16, size_t(bw4 * (N + 1) * 4)},
       {(void**)&h->po256, size_t(bw4 * (N + 1) * 4)},
       {(void**)&h->kofs, size_t(bw4 * (N + 1) * 4)},
+      {(void**)&h->grp, size_t(bw4 * (rp_cap / 64) * 4)},
       {(void**)&h->scal, size_t(bw4 * 64)},
       {(void**)&h->tq[0], size_t(bw4 * tf[0] * rp_cap / 2)},
       {(void**)&h->tq[1], size_t(bw4 * tf[1] * rp_cap / 2)},
@@ -2393,23 +2395,23 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
   LMOE_STEP(16, launch_combine(h->O, h->inv, T, K, l, du, ldu, st));
   // 8. weight gradients: per expert, over its rows (the K dimension),
   //    transformed operands padded to 256-row segments
-  LMOE_STEP(20, launch_seg_offsets(h->counts, N, h->po16, h->po256, h->kofs, st));
+  LMOE_STEP(20, launch_seg_offsets(h->counts, N, h->po16, h->po256, h->kofs, h->grp, st));
   const int64_t kc = pitch / 64;
   TSrc src_do{h->do32, nullptr, nullptr, nullptr, K, 0, 0, 0.f};
   TSrc src_g{h->Hq, nullptr, h->rblock, h->sfbh, K, hp / 2, hp / 64, h->g_h};
   TSrc src_da{h->da32, nullptr, nullptr, nullptr, K, 0, 0, 0.f};
   TSrc src_u{u, h->perm, nullptr, nullptr, K, 0, 0, 0.f};
   // dW2[e] = Q_sr(R(do_e^T)) Q(R(g_e^T))^T: A = g^T (features h), B = do^T (rows l)
-  LMOE_STEP(20, launch_tq_amax(2, src_g, h->offsets, h->counts, h->po16, h->po256, N, hh, pitch,
-                               seed + 2, amax + 3, st));
-  LMOE_STEP(20, launch_tq_amax(0, src_do, h->offsets, h->counts, h->po16, h->po256, N, l, pitch,
-                               seed + 2, amax + 2, st));
-  LMOE_STEP(20, launch_tq_quant(2, false, src_g, h->offsets, h->counts, h->po16, h->po256, N, hh,
-                                pitch, seed + 2, amax + 3, 0, h->tq[1], h->ts[1], h->ta[1],
-                                gsc + 3, st));
-  LMOE_STEP(20, launch_tq_quant(0, true, src_do, h->offsets, h->counts, h->po16, h->po256, N, l,
-                                pitch, seed + 2, amax + 2, seed + 3, h->tq[0], h->ts[0], h->ta[0],
-                                gsc + 2, st));
+  const int32_t *off = h->offsets, *cnt = h->counts, *p16 = h->po16, *p256 = h->po256,
+                *grp = h->grp;
+  LMOE_STEP(20, launch_tq_amax(2, src_g, off, cnt, p16, p256, grp, N, hh, pitch, seed + 2,
+                               amax + 3, st));
+  LMOE_STEP(20, launch_tq_amax(0, src_do, off, cnt, p16, p256, grp, N, l, pitch, seed + 2,
+                               amax + 2, st));
+  LMOE_STEP(20, launch_tq_quant(2, false, src_g, off, cnt, p16, p256, grp, N, hh, pitch, seed + 2,
+                                amax + 3, 0, h->tq[1], h->ts[1], h->ta[1], gsc + 3, st));
+  LMOE_STEP(20, launch_tq_quant(0, true, src_do, off, cnt, p16, p256, grp, N, l, pitch, seed + 2,
+                                amax + 2, seed + 3, h->tq[0], h->ts[0], h->ta[0], gsc + 2, st));
   {
     TileSource s{2, 0, nullptr, nullptr, hh / 128, 0, hh, 0, 1, nullptr, 0, h->ta[1], h->ta[0],
                  static_cast<int>(kc), h->kofs, N, l};
@@ -2419,16 +2421,14 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
                                             lim, st));
   }
   // dW1[e] = Q_sr(R(da_e^T)) Q(R(u_e^T))^T: A = u^T (features l), B = da^T (rows h)
-  LMOE_STEP(21, launch_tq_amax(1, src_u, h->offsets, h->counts, h->po16, h->po256, N, l, pitch,
-                               seed + 4, amax + 5, st));
-  LMOE_STEP(21, launch_tq_amax(0, src_da, h->offsets, h->counts, h->po16, h->po256, N, hh, pitch,
-                               seed + 4, amax + 4, st));
-  LMOE_STEP(21, launch_tq_quant(1, false, src_u, h->offsets, h->counts, h->po16, h->po256, N, l,
-                                pitch, seed + 4, amax + 5, 0, h->tq[2], h->ts[2], h->ta[2],
-                                gsc + 5, st));
-  LMOE_STEP(21, launch_tq_quant(0, true, src_da, h->offsets, h->counts, h->po16, h->po256, N, hh,
-                                pitch, seed + 4, amax + 4, seed + 5, h->tq[3], h->ts[3], h->ta[3],
-                                gsc + 4, st));
+  LMOE_STEP(21, launch_tq_amax(1, src_u, off, cnt, p16, p256, grp, N, l, pitch, seed + 4,
+                               amax + 5, st));
+  LMOE_STEP(21, launch_tq_amax(0, src_da, off, cnt, p16, p256, grp, N, hh, pitch, seed + 4,
+                               amax + 4, st));
+  LMOE_STEP(21, launch_tq_quant(1, false, src_u, off, cnt, p16, p256, grp, N, l, pitch, seed + 4,
+                                amax + 5, 0, h->tq[2], h->ts[2], h->ta[2], gsc + 5, st));
+  LMOE_STEP(21, launch_tq_quant(0, true, src_da, off, cnt, p16, p256, grp, N, hh, pitch, seed + 4,
+                                amax + 4, seed + 5, h->tq[3], h->ts[3], h->ta[3], gsc + 4, st));
   {
     TileSource s{2, 0, nullptr, nullptr, l / 128, 0, l, 0, 1, nullptr, 0, h->ta[2], h->ta[3],
                  static_cast<int>(kc), h->kofs, N, hh};

@@ -156,15 +156,17 @@ __device__ __forceinline__ uint8_t nvfp4_scale_tab(float amax, const float* __re
 // take counters 0..15 (sign -1 when bit 63 is set); a uniform in [0, 1) is
 // the top 24 bits times 2^-24.
 
-__device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t ctr) {
+// SplitMix64 output for counter ctr, up to its last step z ^ (z >> 31): that
+// step leaves bits 33..63 unchanged, and only the top 24 bits (uniforms) and
+// bit 63 (the transform's signs) are used.
+__device__ __forceinline__ uint64_t splitmix64_high(uint64_t seed, uint64_t ctr) {
   uint64_t z = seed + (ctr + 1ull) * 0x9E3779B97F4A7C15ull;
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-  return z ^ (z >> 31);
+  return (z ^ (z >> 27)) * 0x94D049BB133111EBull;
 }
 
 __device__ __forceinline__ float uniform24(uint64_t seed, uint64_t ctr) {
-  return static_cast<float>(static_cast<uint32_t>(splitmix64(seed, ctr) >> 40)) *
+  return static_cast<float>(static_cast<uint32_t>(splitmix64_high(seed, ctr) >> 40)) *
          5.9604644775390625e-8f;   // 2^-24
 }
 
@@ -199,7 +201,7 @@ __device__ __forceinline__ uint32_t rht16_signs(uint64_t seed) {
   uint32_t m = 0;
 #pragma unroll
   for (int j = 0; j < 16; ++j)
-    m |= static_cast<uint32_t>(splitmix64(seed, static_cast<uint64_t>(j)) >> 63) << j;
+    m |= static_cast<uint32_t>(splitmix64_high(seed, static_cast<uint64_t>(j)) >> 63) << j;
   return m;
 }
 

@@ -286,41 +286,39 @@ cudaError_t launch_dw_rows(const void* O, const int32_t* inv, const void* dv, in
 
 // ---------------------------------------------------------------------------
 // Segment offsets of the transposed operands from the rows per expert:
-// po16 / po256 [N + 1] (columns; each segment padded to 16 / 256) and kofs
-// [N + 1] = po256 / 256 (FP4 k-steps).  One thread (N <= 1024).
+// po16 / po256 [N + 1] (columns; each segment padded to 16 / 256), kofs
+// [N + 1] = po256 / 256 (FP4 k-steps) and grp [po256[N] / 64], the expert of
+// each 64-column group.  One CTA: thread 0 scans (N <= 1024), then thread e
+// fills expert e's groups.
 
-__global__ void k_seg_offsets(const int32_t* __restrict__ counts, int N, int32_t* __restrict__ po16,
-                              int32_t* __restrict__ po256, int32_t* __restrict__ kofs) {
+__global__ void __launch_bounds__(1024) k_seg_offsets(const int32_t* __restrict__ counts, int N,
+                                                      int32_t* __restrict__ po16,
+                                                      int32_t* __restrict__ po256,
+                                                      int32_t* __restrict__ kofs,
+                                                      int32_t* __restrict__ grp) {
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int32_t a = 0, b = 0;
-  for (int e = 0; e < N; ++e) {
-    po16[e] = a;
-    po256[e] = b;
-    kofs[e] = b / 256;
-    a += (counts[e] + 15) / 16 * 16;
-    b += (counts[e] + 255) / 256 * 256;
+  if (threadIdx.x == 0) {
+    int32_t a = 0, b = 0;
+    for (int e = 0; e < N; ++e) {
+      po16[e] = a;
+      po256[e] = b;
+      kofs[e] = b / 256;
+      a += (counts[e] + 15) / 16 * 16;
+      b += (counts[e] + 255) / 256 * 256;
+    }
+    po16[N] = a;
+    po256[N] = b;
+    kofs[N] = b / 256;
   }
-  po16[N] = a;
-  po256[N] = b;
-  kofs[N] = b / 256;
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x)
+    for (int g = po256[e] / 64; g < po256[e + 1] / 64; ++g) grp[g] = e;
 }
 
 cudaError_t launch_seg_offsets(const int32_t* counts, int N, int32_t* po16, int32_t* po256,
-                               int32_t* kofs, cudaStream_t st) {
-  return launch_pdl(k_seg_offsets, 1, 32, 0, st, counts, N, po16, po256, kofs);
-}
-
-// the segment (expert) holding column `col` of the 256-padded layout
-__device__ __forceinline__ int seg_of(const int32_t* po256, int N, int col) {
-  int lo = 0, hi = N;   // po256[lo] <= col < po256[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (po256[mid] <= col) lo = mid;
-    else hi = mid;
-  }
-  return lo;
+                               int32_t* kofs, int32_t* grp, cudaStream_t st) {
+  return launch_pdl(k_seg_offsets, 1, 1024, 0, st, counts, N, po16, po256, kofs, grp);
 }
 
 // ---------------------------------------------------------------------------
@@ -358,57 +356,86 @@ constexpr int TQ_PITCH = 129;
 template <int SRC>
 __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, int f0, int F,
                                          float (*tile)[TQ_PITCH]) {
+  // every load of the thread is issued before the first is used
   const int t = threadIdx.x;
   if constexpr (SRC == 0) {
-    // fp32 rows: 32 float4 per row
-    for (int i = t; i < nr * 32; i += 128) {
-      const int row = i >> 5, q = i & 31;
-      const int f = f0 + 4 * q;
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (f < F) x = *reinterpret_cast<const float4*>(static_cast<const float*>(s.p) +
-                                                       (rbase + row) * F + f);
-      tile[row][4 * q] = x.x;
-      tile[row][4 * q + 1] = x.y;
-      tile[row][4 * q + 2] = x.z;
-      tile[row][4 * q + 3] = x.w;
+    // fp32 rows: 32 float4 per row, 16 per thread
+    float4 x[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = t + 128 * k, row = i >> 5, f = f0 + 4 * (i & 31);
+      x[k] = (row < nr && f < F) ? *reinterpret_cast<const float4*>(
+                                       static_cast<const float*>(s.p) + (rbase + row) * F + f)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = t + 128 * k, row = i >> 5, q = i & 31;
+      if (row < nr) {
+        tile[row][4 * q] = x[k].x;
+        tile[row][4 * q + 1] = x[k].y;
+        tile[row][4 * q + 2] = x[k].z;
+        tile[row][4 * q + 3] = x[k].w;
+      }
     }
   } else if constexpr (SRC == 1) {
-    // bf16 token rows: 16 x 8 elements per row
-    for (int i = t; i < nr * 16; i += 128) {
-      const int row = i >> 4, q = i & 15;
-      const int f = f0 + 8 * q;
-      const int64_t tok = s.perm[rbase + row] / s.K;
-      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (f < F) raw = *reinterpret_cast<const uint4*>(static_cast<const bf16*>(s.p) + tok * F + f);
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    // bf16 token rows: 16 x 8 elements per row, 8 per thread
+    uint4 raw[8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 v = __bfloat1622float2(p2[k]);
-        tile[row][8 * q + 2 * k] = v.x;
-        tile[row][8 * q + 2 * k + 1] = v.y;
+    for (int k = 0; k < 8; ++k) {
+      const int i = t + 128 * k, row = i >> 4, f = f0 + 8 * (i & 15);
+      raw[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < nr && f < F) {
+        const int64_t tok = s.perm[rbase + row] / s.K;
+        raw[k] = *reinterpret_cast<const uint4*>(static_cast<const bf16*>(s.p) + tok * F + f);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = t + 128 * k, row = i >> 4, q = i & 15;
+      if (row < nr) {
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float2 v = __bfloat1622float2(p2[c]);
+          tile[row][8 * q + 2 * c] = v.x;
+          tile[row][8 * q + 2 * c + 1] = v.y;
+        }
       }
     }
   } else {
-    // NVFP4 rows: 16 words of 8 codes per row, each with its 16-block's scale
-    for (int i = t; i < nr * 16; i += 128) {
-      const int row = i >> 4, q = i & 15;
-      const int f = f0 + 8 * q;
-      const int64_t r = rbase + row;
-      if (f >= F) {
+    // NVFP4 rows: per row two words of scales (the row's 4 block scales of each
+    // 64-feature chunk are adjacent in its atom) and 16 words of 8 codes
+    __shared__ uint32_t scw[64][2];
+    uint32_t w[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) tile[row][8 * q + k] = 0.0f;
-        continue;
+    for (int k = 0; k < 8; ++k) {
+      const int i = t + 128 * k, row = i >> 4, f = f0 + 8 * (i & 15);
+      w[k] = (row < nr && f < F) ? *reinterpret_cast<const uint32_t*>(
+                                       static_cast<const uint8_t*>(s.p) + (rbase + row) * s.code_pitch + f / 2)
+                                 : 0u;
+    }
+    {
+      const int row = t >> 1, c = t & 1, f = f0 + 64 * c;
+      if (row < nr && f < F) {
+        const int rb = s.rblock[rbase + row];
+        const int b = rb >> 8, j = rb & 255;
+        scw[row][c] = *reinterpret_cast<const uint32_t*>(
+            s.atoms + (static_cast<int64_t>(b) * s.fp64 + f / 64) * SF_ATOM_BYTES +
+            sf_atom_offset(j, 0));
       }
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(s.p) +
-                                                            r * s.code_pitch + f / 2);
-      const int rb = s.rblock[r];
-      const int b = rb >> 8, j = rb & 255;
-      const uint8_t sc = s.atoms[(static_cast<int64_t>(b) * s.fp64 + f / 64) * SF_ATOM_BYTES +
-                                 sf_atom_offset(j, (f & 63) >> 4)];
-      const float scv = e4m3_value(sc);
+    }
+    __syncthreads();
 #pragma unroll
-      for (int k = 0; k < 8; ++k)   // (code x scale) x g, the dequantisation order
-        tile[row][8 * q + k] = __fmul_rn(__fmul_rn(e2m1_value((w >> (4 * k)) & 15u), scv), s.g);
+    for (int k = 0; k < 8; ++k) {
+      const int i = t + 128 * k, row = i >> 4, q = i & 15;
+      if (row < nr) {
+        const uint32_t sc = (scw[row][q >> 3] >> (8 * ((q & 7) >> 1))) & 255u;
+        const float scv = e4m3_value(static_cast<uint8_t>(sc));
+#pragma unroll
+        for (int c = 0; c < 8; ++c)   // (code x scale) x g, the dequantisation order
+          tile[row][8 * q + c] = __fmul_rn(__fmul_rn(e2m1_value((w[k] >> (4 * c)) & 15u), scv), s.g);
+      }
     }
   }
 }
@@ -417,7 +444,8 @@ template <int SRC, bool SR, bool STORE>
 __global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ offsets,
                                             const int32_t* __restrict__ counts,
                                             const int32_t* __restrict__ po16,
-                                            const int32_t* __restrict__ po256, int N, int F,
+                                            const int32_t* __restrict__ po256,
+                                            const int32_t* __restrict__ grp, int N, int F,
                                             int64_t pitch, uint64_t seed_rht, float* amax,
                                             uint64_t seed_sr, uint8_t* __restrict__ codes,
                                             uint8_t* __restrict__ scales,
@@ -426,10 +454,11 @@ __global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ 
   pdl_wait();
   pdl_trigger();
   const int col0 = blockIdx.y * 64;
-  if (col0 >= po256[N]) return;
+  const int width = po256[N];
+  const int e = grp[blockIdx.y];   // read before the test (stale past the width)
+  if (col0 >= width) return;
   const int f0 = blockIdx.x * 128;
   const int f = f0 + threadIdx.x;
-  const int e = seg_of(po256, N, col0);
   const int j0 = col0 - po256[e];
   const int ce = counts[e];
   const int nr = min(64, ce - j0);   // rows of this group that hold data (may be <= 0)
@@ -488,27 +517,28 @@ __global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ 
 
 template <int SRC, bool SR, bool STORE>
 static cudaError_t launch_tq_v(const TSrc& s, const int32_t* offsets, const int32_t* counts,
-                               const int32_t* po16, const int32_t* po256, int N, int F,
+                               const int32_t* po16, const int32_t* po256, const int32_t* grp,
+                               int N, int F,
                                int64_t pitch, uint64_t seed_rht, float* amax, uint64_t seed_sr,
                                uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* g_out,
                                cudaStream_t st) {
   const dim3 grid(static_cast<unsigned>((F + 127) / 128), static_cast<unsigned>(pitch / 64));
-  return launch_pdl(k_tq<SRC, SR, STORE>, grid, 128, 0, st, s, offsets, counts, po16, po256, N,
-                    F, pitch, seed_rht, amax, seed_sr, codes, scales, atoms, g_out);
+  return launch_pdl(k_tq<SRC, SR, STORE>, grid, 128, 0, st, s, offsets, counts, po16, po256, grp,
+                    N, F, pitch, seed_rht, amax, seed_sr, codes, scales, atoms, g_out);
 }
 
 cudaError_t launch_tq_amax(int src_kind, const TSrc& s, const int32_t* offsets,
                            const int32_t* counts, const int32_t* po16, const int32_t* po256,
-                           int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
+                           const int32_t* grp, int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
                            cudaStream_t st) {
   switch (src_kind) {
-    case 0: return launch_tq_v<0, false, false>(s, offsets, counts, po16, po256, N, F, pitch,
+    case 0: return launch_tq_v<0, false, false>(s, offsets, counts, po16, po256, grp, N, F, pitch,
                                                 seed_rht, amax, 0, nullptr, nullptr, nullptr,
                                                 nullptr, st);
-    case 1: return launch_tq_v<1, false, false>(s, offsets, counts, po16, po256, N, F, pitch,
+    case 1: return launch_tq_v<1, false, false>(s, offsets, counts, po16, po256, grp, N, F, pitch,
                                                 seed_rht, amax, 0, nullptr, nullptr, nullptr,
                                                 nullptr, st);
-    default: return launch_tq_v<2, false, false>(s, offsets, counts, po16, po256, N, F, pitch,
+    default: return launch_tq_v<2, false, false>(s, offsets, counts, po16, po256, grp, N, F, pitch,
                                                  seed_rht, amax, 0, nullptr, nullptr, nullptr,
                                                  nullptr, st);
   }
@@ -516,19 +546,19 @@ cudaError_t launch_tq_amax(int src_kind, const TSrc& s, const int32_t* offsets,
 
 cudaError_t launch_tq_quant(int src_kind, bool sr, const TSrc& s, const int32_t* offsets,
                             const int32_t* counts, const int32_t* po16, const int32_t* po256,
-                            int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
+                            const int32_t* grp, int N, int F, int64_t pitch, uint64_t seed_rht, float* amax,
                             uint64_t seed_sr, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
                             float* g_out, cudaStream_t st) {
   // the recipe's four operands: gradients (SRC 0) stochastically rounded,
   // activations (SRC 1, 2) rounded to nearest
   if (src_kind == 0 && sr)
-    return launch_tq_v<0, true, true>(s, offsets, counts, po16, po256, N, F, pitch, seed_rht,
+    return launch_tq_v<0, true, true>(s, offsets, counts, po16, po256, grp, N, F, pitch, seed_rht,
                                       amax, seed_sr, codes, scales, atoms, g_out, st);
   if (src_kind == 1 && !sr)
-    return launch_tq_v<1, false, true>(s, offsets, counts, po16, po256, N, F, pitch, seed_rht,
+    return launch_tq_v<1, false, true>(s, offsets, counts, po16, po256, grp, N, F, pitch, seed_rht,
                                        amax, 0, codes, scales, atoms, g_out, st);
   if (src_kind == 2 && !sr)
-    return launch_tq_v<2, false, true>(s, offsets, counts, po16, po256, N, F, pitch, seed_rht,
+    return launch_tq_v<2, false, true>(s, offsets, counts, po16, po256, grp, N, F, pitch, seed_rht,
                                        amax, 0, codes, scales, atoms, g_out, st);
   return cudaErrorInvalidValue;
 }
