@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "liblmoe.so")
 SOURCES = ["lmoe_abi.cu", "routing.cu", "route_noalloc.cu", "nvfp4.cu", "nvfp4_bw.cu",
            "backward.cu"]
-HEADERS = ["ptx.cuh", "gemm_tc.cuh", "gemm_pair.cuh", "gemm_bw.cuh", "gemm_bw_pair.cuh", "kernels.h", "nvfp4.cuh", "launch.cuh",
+HEADERS = ["ptx.cuh", "gemm_tc.cuh", "gemm_pair.cuh", "gemm_bw.cuh", "kernels.h", "nvfp4.cuh", "launch.cuh",
            "route.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

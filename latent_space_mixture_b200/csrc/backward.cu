@@ -170,43 +170,6 @@ cudaError_t launch_route_bw(const float* logits, const int32_t* topk_idx, const 
 }
 
 // ---------------------------------------------------------------------------
-// Tail copies of two expert-order operands for the CTA-pair weight-gradient
-// GEMM: for each expert with rows, the last 64-row block of its segment,
-// rows past the segment zero: tail[e * 64 + j] = x[off[e] + 64 (kb - 1) + j]
-// for j < c_e - 64 (kb - 1), kb = ceil(c_e / 64).  grid (N, 64), a thread per
-// 8 elements of a row of either operand.
-
-__global__ void __launch_bounds__(256) k_wgrad_tails(const uint4* __restrict__ xa, int fa,
-                                                     const uint4* __restrict__ xb, int fb,
-                                                     const int32_t* __restrict__ offsets,
-                                                     uint4* __restrict__ ta, uint4* __restrict__ tb) {
-  pdl_wait();
-  pdl_trigger();
-  const int e = blockIdx.x, j = blockIdx.y;
-  const int seg0 = offsets[e], cnt = offsets[e + 1] - seg0;
-  if (cnt == 0) return;
-  const int kb = (cnt + 63) / 64;
-  const bool valid = j < cnt - 64 * (kb - 1);
-  const int64_t src = static_cast<int64_t>(seg0) + 64 * (kb - 1) + j;
-  const int64_t dst = static_cast<int64_t>(e) * 64 + j;
-  const int va = fa / 8, vb = fb / 8;
-  for (int c = threadIdx.x; c < va + vb; c += blockDim.x) {
-    if (c < va)
-      ta[dst * va + c] = valid ? xa[src * va + c] : make_uint4(0u, 0u, 0u, 0u);
-    else
-      tb[dst * vb + c - va] = valid ? xb[src * vb + c - va] : make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-cudaError_t launch_wgrad_tails(const void* xa, int fa, const void* xb, int fb,
-                               const int32_t* offsets, int N, void* ta, void* tb,
-                               cudaStream_t st) {
-  return launch_pdl(k_wgrad_tails, dim3(static_cast<unsigned>(N), 64), 256, 0, st,
-                    static_cast<const uint4*>(xa), fa, static_cast<const uint4*>(xb), fb, offsets,
-                    static_cast<uint4*>(ta), static_cast<uint4*>(tb));
-}
-
-// ---------------------------------------------------------------------------
 // Aux-loss-free balancing: b_e += rate * sign(total - N c_e), i.e. experts
 // above the mean load c = total / N lose `rate`, those below gain it (float32
 // arithmetic as the bias is stored).  total = sum of counts (T K).

@@ -143,10 +143,6 @@ cudaError_t launch_route_bw(const float* logits, const int32_t* topk_idx, const 
                             void* dxh, int ldx, bool direct, cudaStream_t st);
 
 // Aux-loss-free bias update: bias[e] += rate * sign(total - N * counts[e]).
-// tail copies of two expert-order operands for the pair weight-gradient GEMM
-cudaError_t launch_wgrad_tails(const void* xa, int fa, const void* xb, int fb,
-                               const int32_t* offsets, int N, void* ta, void* tb,
-                               cudaStream_t st);
 cudaError_t launch_bias_update(float* bias, const int32_t* counts, int N, int64_t total, float rate,
                                cudaStream_t st);
 

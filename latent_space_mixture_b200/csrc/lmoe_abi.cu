@@ -12,7 +12,6 @@
 #include <vector>
 
 #include "gemm_bw.cuh"
-#include "gemm_bw_pair.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.h"
@@ -1057,11 +1056,6 @@ struct lmoe_handle {
   bf16* dy_dev = nullptr;    // [64][d]     staging of dy for T < 64
   CUtensorMap tm_wx64, tm_wy64, tm_w1_64, tm_w2_64;   // weights in 64-row boxes
   BMaps tm_dog, tm_da, tm_dxh;
-  // CTA-pair expert wgrads: the last 64-row block of every expert's segment
-  // of the l-wide and h-wide operands, rows past the segment zero
-  bf16* tail_l = nullptr;      // [N * 64][l]
-  bf16* tail_h = nullptr;      // [N * 64][h]
-  CUtensorMap tm_tail_l, tm_tail_h;
   // NVFP4 training (NVFP4 experts, 2D weight blocks, LMOE_FLAG_BACKWARD):
   // transposed weights, the backward's rows and transposed operands
   bool bw4 = false;
@@ -1357,8 +1351,6 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
       {(void**)&h->dv, size_t(bwx * Tm_b * l * 2)},
       {(void**)&h->dog, size_t(bwd * rows_b * l * 2)},
       {(void**)&h->da, size_t(bwd * rows_b * hh * 2)},
-      {(void**)&h->tail_l, size_t(bwd * N * 64 * l * 2)},
-      {(void**)&h->tail_h, size_t(bwd * N * 64 * hh * 2)},
       {(void**)&h->dup, size_t(bwd * rows_b * l * 2)},
       {(void**)&h->dwacc, size_t(bwx * rows * 4)},
       {(void**)&h->dxh, size_t(bwx * Tm_b * (N + l + hs) * 2)},
@@ -1584,11 +1576,6 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, lmoe_handle** out
     ok &= make_map(&h->tm_da.b16, h->da, rows_b, hh, GEMM_BROWS);
     ok &= make_map(&h->tm_da.b64, h->da, rows_b, hh, GEMM_BROWS_BIG);
     ok &= set_bw_smem<256, true, EpiWExp>() == cudaSuccess;
-    ok &= make_map(&h->tm_tail_l, h->tail_l, int64_t(N) * 64, l, GEMM_BROWS_BIG);
-    ok &= make_map(&h->tm_tail_h, h->tail_h, int64_t(N) * 64, hh, GEMM_BROWS_BIG);
-    ok &= cudaFuncSetAttribute(k_gemm_wgrad_pair<EpiWExp>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               WPairLayout::SMEM_BYTES) == cudaSuccess;
   }
   ok &= set_smem_all<EpiX>() == cudaSuccess;
   ok &= set_smem_all<EpiH>() == cudaSuccess;
@@ -2065,49 +2052,25 @@ int lmoe_backward(lmoe_handle* h, const void* x, const void* dy, int64_t T, void
     LMOE_BW(7, (launch_bw<256, true>(h->tm_vh.b64, tm_dy.b64, tm_dy.b64, s, epi,
                                   grid_of(int64_t(fb) * nbk), h->err, lim, st)));
   }
-  // 9-10: the expert weight gradients, on CTA pairs (256 x 256 tiles) when
-  // the experts' segments hold a 64-row block on average, else single CTAs
-  const char* wpe = getenv("LMOE_WGRAD_PAIR");
-  const bool wpair = h->pairs && R >= int64_t(64) * N && !(wpe && wpe[0] == '0');
-  auto wgrad_pair = [&](const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tat,
-                        const CUtensorMap& tbt, int fa, int fbr, const EpiWExp& epi) {
-    BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, (fa + 255) / 256, fa, fa, N, h->offsets,
-               (fbr + 255) / 256, fbr, fbr};
-    const int64_t tiles = int64_t(N) * s.FB * s.NB;
-    const int npairs = static_cast<int>(tiles < h->sms / 2 ? tiles : h->sms / 2);
-    return launch_pair_pdl(k_gemm_wgrad_pair<EpiWExp>, 2 * npairs, GEMM_THREADS,
-                           WPairLayout::SMEM_BYTES, st, ta, tb, tat, tbt, s, epi, h->err, lim);
-  };
   // 9. dW2[e] = do^T g over the expert's rows  ([l][h])
   if (!h->bw4) {
+    const int fb = (hh + 127) / 128, nbk = (l + 255) / 256;
+    BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, hh, hh, N, h->offsets, nbk, l, l};
     EpiWExp epi{};
     if (!make_map_f32_out(&epi.m, gr->d_w2, int64_t(N) * l, hh)) return LMOE_ERR_CUDA;
     epi.rows_per = l;
-    if (wpair) {
-      LMOE_BW(8, launch_wgrad_tails(h->H, hh, h->dog, l, h->offsets, N, h->tail_h, h->tail_l, st));
-      LMOE_BW(8, wgrad_pair(h->tm_H.b64, h->tm_dog.b64, h->tm_tail_h, h->tm_tail_l, hh, l, epi));
-    } else {
-      const int fb = (hh + 127) / 128, nbk = (l + 255) / 256;
-      BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, hh, hh, N, h->offsets, nbk, l, l};
-      LMOE_BW(8, (launch_bw<256, true>(h->tm_H.b64, h->tm_dog.b64, h->tm_dog.b64, s, epi,
-                                    grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
-    }
+    LMOE_BW(8, (launch_bw<256, true>(h->tm_H.b64, h->tm_dog.b64, h->tm_dog.b64, s, epi,
+                                  grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
   }
   // 10. dW1[e] = da^T u over the expert's rows  ([h][l])
   if (!h->bw4) {
+    const int fb = (l + 127) / 128, nbk = (hh + 255) / 256;
+    BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, l, l, N, h->offsets, nbk, hh, hh};
     EpiWExp epi{};
     if (!make_map_f32_out(&epi.m, gr->d_w1, int64_t(N) * hh, l)) return LMOE_ERR_CUDA;
     epi.rows_per = hh;
-    if (wpair) {
-      LMOE_BW(9, launch_wgrad_tails(h->u_perm, l, h->da, hh, h->offsets, N, h->tail_l, h->tail_h,
-                                    st));
-      LMOE_BW(9, wgrad_pair(h->tm_uperm.b64, h->tm_da.b64, h->tm_tail_l, h->tm_tail_h, l, hh, epi));
-    } else {
-      const int fb = (l + 127) / 128, nbk = (hh + 255) / 256;
-      BwSource s{1, 0, 0, nullptr, nullptr, 0, 0, fb, l, l, N, h->offsets, nbk, hh, hh};
-      LMOE_BW(9, (launch_bw<256, true>(h->tm_uperm.b64, h->tm_da.b64, h->tm_da.b64, s, epi,
-                                    grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
-    }
+    LMOE_BW(9, (launch_bw<256, true>(h->tm_uperm.b64, h->tm_da.b64, h->tm_da.b64, s, epi,
+                                  grid_of(int64_t(N) * fb * nbk), h->err, lim, st)));
   }
   // 11. d[W_r; W_dn; W_s1] = dxh^T x  (rows N + l + h_s, columns d)
   {
