@@ -207,10 +207,8 @@ def test_cta_pair_gemms_match_single_cta_gemms(monkeypatch):
 
 def test_overlapped_shared_expert_matches_serial_forward(monkeypatch):
     """The forward that runs the shared expert's GEMMs on a side stream over
-    a share of the SMs (chosen by default when the grouped GEMMs are bound by
-    HBM, as at Ultra dims; forced here with LMOE_OVERLAP) equals the serial
-    forward up to the bf16 rounding of the shared branch before the add, and
-    matches the oracle."""
+    a share of the SMs (opt-in, LMOE_OVERLAP; forced here) equals the serial
+    forward within the oracle bar, and matches the oracle."""
     cfg = CONFIGS["pair_small"]
     monkeypatch.setenv("LMOE_OVERLAP", "0")
     w, x, layer = make(cfg)
