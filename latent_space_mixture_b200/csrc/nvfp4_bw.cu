@@ -342,9 +342,9 @@ cudaError_t launch_seg_offsets(const int32_t* counts, int N, int32_t* po16, int3
 //   SRC 2: NVFP4 rows, codes [R][code_pitch] and B-operand scale atoms
 //          ([block][Fp/64][512] by rblock), dequantised with global scale g.
 // A CTA per (128 features, 64-column group): the group's source rows are
-// staged in shared memory with coalesced loads, then a thread takes one
-// feature (a column of the tile), so its 32 bytes of codes and 4 scales are
-// contiguous.  A 64-column group lies inside one segment (the segments are
+// staged in shared memory with coalesced loads, then two threads take one
+// feature (a column of the tile), 32 columns each, so a thread's 16 bytes of
+// codes and 2 scales are contiguous.  A 64-column group lies inside one segment (the segments are
 // 256-aligned); groups past the layout's width (po256[N], on the device) do
 // nothing.
 
@@ -352,6 +352,7 @@ cudaError_t launch_seg_offsets(const int32_t* counts, int N, int32_t* po16, int3
 // 64-row group, as floats in shared memory (rows read with coalesced vector
 // loads; NVFP4 rows dequantised 8 codes at a time).
 constexpr int TQ_PITCH = 129;
+constexpr int TQ_THREADS = 256;   // two threads per feature, 32 columns each
 
 template <int SRC>
 __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, int f0, int F,
@@ -359,18 +360,18 @@ __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, i
   // every load of the thread is issued before the first is used
   const int t = threadIdx.x;
   if constexpr (SRC == 0) {
-    // fp32 rows: 32 float4 per row, 16 per thread
-    float4 x[16];
+    // fp32 rows: 32 float4 per row, 8 per thread
+    float4 x[8];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int i = t + 128 * k, row = i >> 5, f = f0 + 4 * (i & 31);
+    for (int k = 0; k < 8; ++k) {
+      const int i = t + TQ_THREADS * k, row = i >> 5, f = f0 + 4 * (i & 31);
       x[k] = (row < nr && f < F) ? *reinterpret_cast<const float4*>(
                                        static_cast<const float*>(s.p) + (rbase + row) * F + f)
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int i = t + 128 * k, row = i >> 5, q = i & 31;
+    for (int k = 0; k < 8; ++k) {
+      const int i = t + TQ_THREADS * k, row = i >> 5, q = i & 31;
       if (row < nr) {
         tile[row][4 * q] = x[k].x;
         tile[row][4 * q + 1] = x[k].y;
@@ -379,11 +380,11 @@ __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, i
       }
     }
   } else if constexpr (SRC == 1) {
-    // bf16 token rows: 16 x 8 elements per row, 8 per thread
-    uint4 raw[8];
+    // bf16 token rows: 16 x 8 elements per row, 4 per thread
+    uint4 raw[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = t + 128 * k, row = i >> 4, f = f0 + 8 * (i & 15);
+    for (int k = 0; k < 4; ++k) {
+      const int i = t + TQ_THREADS * k, row = i >> 4, f = f0 + 8 * (i & 15);
       raw[k] = make_uint4(0u, 0u, 0u, 0u);
       if (row < nr && f < F) {
         const int64_t tok = s.perm[rbase + row] / s.K;
@@ -391,8 +392,8 @@ __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, i
       }
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = t + 128 * k, row = i >> 4, q = i & 15;
+    for (int k = 0; k < 4; ++k) {
+      const int i = t + TQ_THREADS * k, row = i >> 4, q = i & 15;
       if (row < nr) {
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k]);
 #pragma unroll
@@ -407,15 +408,15 @@ __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, i
     // NVFP4 rows: per row two words of scales (the row's 4 block scales of each
     // 64-feature chunk are adjacent in its atom) and 16 words of 8 codes
     __shared__ uint32_t scw[64][2];
-    uint32_t w[8];
+    uint32_t w[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = t + 128 * k, row = i >> 4, f = f0 + 8 * (i & 15);
+    for (int k = 0; k < 4; ++k) {
+      const int i = t + TQ_THREADS * k, row = i >> 4, f = f0 + 8 * (i & 15);
       w[k] = (row < nr && f < F) ? *reinterpret_cast<const uint32_t*>(
                                        static_cast<const uint8_t*>(s.p) + (rbase + row) * s.code_pitch + f / 2)
                                  : 0u;
     }
-    {
+    if (t < 128) {
       const int row = t >> 1, c = t & 1, f = f0 + 64 * c;
       if (row < nr && f < F) {
         const int rb = s.rblock[rbase + row];
@@ -427,8 +428,8 @@ __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, i
     }
     __syncthreads();
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = t + 128 * k, row = i >> 4, q = i & 15;
+    for (int k = 0; k < 4; ++k) {
+      const int i = t + TQ_THREADS * k, row = i >> 4, q = i & 15;
       if (row < nr) {
         const uint32_t sc = (scw[row][q >> 3] >> (8 * ((q & 7) >> 1))) & 255u;
         const float scv = e4m3_value(static_cast<uint8_t>(sc));
@@ -441,7 +442,7 @@ __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, i
 }
 
 template <int SRC, bool SR, bool STORE>
-__global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ offsets,
+__global__ void __launch_bounds__(TQ_THREADS) k_tq(TSrc s, const int32_t* __restrict__ offsets,
                                             const int32_t* __restrict__ counts,
                                             const int32_t* __restrict__ po16,
                                             const int32_t* __restrict__ po256,
@@ -458,7 +459,8 @@ __global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ 
   const int e = grp[blockIdx.y];   // read before the test (stale past the width)
   if (col0 >= width) return;
   const int f0 = blockIdx.x * 128;
-  const int f = f0 + threadIdx.x;
+  const int f = f0 + (threadIdx.x & 127);
+  const int hv = threadIdx.x >> 7;   // this thread's 32 of the group's 64 columns
   const int j0 = col0 - po256[e];
   const int ce = counts[e];
   const int nr = min(64, ce - j0);   // rows of this group that hold data (may be <= 0)
@@ -472,18 +474,20 @@ __global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ 
   }
   float m = 0.0f;
   if (f < F) {
-    uint32_t cw[8];
+    uint32_t cw[4];
     uint32_t sw = 0;
 #pragma unroll
-    for (int bk = 0; bk < 4; ++bk) {
+    for (int b2 = 0; b2 < 2; ++b2) {
+      const int bk = 2 * hv + b2;   // 16-column block of the group
       if (16 * bk >= nr) {
         // past the segment's rows: zeros, scale 0
-        cw[2 * bk] = cw[2 * bk + 1] = 0u;
+        cw[2 * b2] = cw[2 * b2 + 1] = 0u;
         continue;
       }
       float v[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = (16 * bk + i < nr) ? tile[16 * bk + i][threadIdx.x] : 0.0f;
+      for (int i = 0; i < 16; ++i)
+        v[i] = (16 * bk + i < nr) ? tile[16 * bk + i][threadIdx.x & 127] : 0.0f;
       rht16_masked(v, signs);
       if constexpr (!STORE) {
 #pragma unroll
@@ -494,19 +498,20 @@ __global__ void __launch_bounds__(128) k_tq(TSrc s, const int32_t* __restrict__ 
                                : 0;
         uint8_t q[8];
         const uint8_t sc = quant16<SR>(v, g, seed_sr, c0, q);
-        cw[2 * bk] = *reinterpret_cast<const uint32_t*>(q);
-        cw[2 * bk + 1] = *reinterpret_cast<const uint32_t*>(q + 4);
-        sw |= static_cast<uint32_t>(sc) << (8 * bk);
+        cw[2 * b2] = *reinterpret_cast<const uint32_t*>(q);
+        cw[2 * b2 + 1] = *reinterpret_cast<const uint32_t*>(q + 4);
+        sw |= static_cast<uint32_t>(sc) << (8 * b2);
       }
     }
     if constexpr (STORE) {
-      uint4* dst = reinterpret_cast<uint4*>(codes + f * (pitch / 2) + col0 / 2);
-      dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-      *reinterpret_cast<uint32_t*>(scales + f * (pitch / 16) + col0 / 16) = sw;
-      *reinterpret_cast<uint32_t*>(
+      const int c32 = col0 + 32 * hv;
+      *reinterpret_cast<uint4*>(codes + f * (pitch / 2) + c32 / 2) =
+          make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      *reinterpret_cast<uint16_t*>(scales + f * (pitch / 16) + c32 / 16) =
+          static_cast<uint16_t>(sw);
+      *reinterpret_cast<uint16_t*>(
           atoms + ((static_cast<int64_t>(f) >> 7) * (pitch / 64) + col0 / 64) * SF_ATOM_BYTES +
-          sf_atom_offset(f & 127, 0)) = sw;
+          sf_atom_offset(f & 127, 2 * hv)) = static_cast<uint16_t>(sw);
     }
   }
   if constexpr (!STORE) {
@@ -523,8 +528,8 @@ static cudaError_t launch_tq_v(const TSrc& s, const int32_t* offsets, const int3
                                uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* g_out,
                                cudaStream_t st) {
   const dim3 grid(static_cast<unsigned>((F + 127) / 128), static_cast<unsigned>(pitch / 64));
-  return launch_pdl(k_tq<SRC, SR, STORE>, grid, 128, 0, st, s, offsets, counts, po16, po256, grp,
-                    N, F, pitch, seed_rht, amax, seed_sr, codes, scales, atoms, g_out);
+  return launch_pdl(k_tq<SRC, SR, STORE>, grid, TQ_THREADS, 0, st, s, offsets, counts, po16,
+                    po256, grp, N, F, pitch, seed_rht, amax, seed_sr, codes, scales, atoms, g_out);
 }
 
 cudaError_t launch_tq_amax(int src_kind, const TSrc& s, const int32_t* offsets,
