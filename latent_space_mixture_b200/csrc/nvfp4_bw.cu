@@ -354,48 +354,111 @@ cudaError_t launch_seg_offsets(const int32_t* counts, int N, int32_t* po16, int3
 constexpr int TQ_PITCH = 129;
 constexpr int TQ_THREADS = 256;   // two threads per feature, 32 columns each
 
+// One 64-column group of the CTA: its expert, first row of the segment in
+// the group, rows with data (nr, may be <= 0).
+struct TqGroup {
+  int col0, e, j0, nr;
+  int64_t rbase;
+};
+
+__device__ __forceinline__ TqGroup tq_group(int g, const int32_t* __restrict__ grp,
+                                            const int32_t* __restrict__ offsets,
+                                            const int32_t* __restrict__ counts,
+                                            const int32_t* __restrict__ po256) {
+  TqGroup q;
+  q.col0 = g * 64;
+  q.e = grp[g];
+  q.j0 = q.col0 - po256[q.e];
+  q.nr = min(64, counts[q.e] - q.j0);
+  q.rbase = static_cast<int64_t>(offsets[q.e]) + q.j0;
+  return q;
+}
+
+// The group's source rows x features [f0, f0 + 128) in flight in registers
+// (issued a group ahead), then written to the shared tile as floats.
 template <int SRC>
-__device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, int f0, int F,
-                                         float (*tile)[TQ_PITCH]) {
-  // every load of the thread is issued before the first is used
+struct TqRegs;
+template <>
+struct TqRegs<0> {   // fp32 rows: 32 float4 per row, 8 per thread
+  float4 x[8];
+};
+template <>
+struct TqRegs<1> {   // bf16 token rows: 16 x 8 elements per row, 4 per thread
+  uint4 raw[4];
+};
+template <>
+struct TqRegs<2> {   // NVFP4 rows: 16 words of 8 codes per row, 4 per thread, and
+  uint32_t w[4];     // (threads < 128) one word of 4 block scales (row t/2,
+  uint32_t sc;       // 64-feature chunk t%2: adjacent in the row's atom)
+};
+
+template <int SRC>
+__device__ __forceinline__ void tq_issue(TqRegs<SRC>& r, const TSrc& s, int64_t rbase, int nr,
+                                         int f0, int F) {
   const int t = threadIdx.x;
   if constexpr (SRC == 0) {
-    // fp32 rows: 32 float4 per row, 8 per thread
-    float4 x[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int i = t + TQ_THREADS * k, row = i >> 5, f = f0 + 4 * (i & 31);
-      x[k] = (row < nr && f < F) ? *reinterpret_cast<const float4*>(
-                                       static_cast<const float*>(s.p) + (rbase + row) * F + f)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      r.x[k] = (row < nr && f < F) ? *reinterpret_cast<const float4*>(
+                                         static_cast<const float*>(s.p) + (rbase + row) * F + f)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+  } else if constexpr (SRC == 1) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = t + TQ_THREADS * k, row = i >> 4, f = f0 + 8 * (i & 15);
+      r.raw[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < nr && f < F) {
+        const int64_t tok = s.perm[rbase + row] / s.K;
+        r.raw[k] = *reinterpret_cast<const uint4*>(static_cast<const bf16*>(s.p) + tok * F + f);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = t + TQ_THREADS * k, row = i >> 4, f = f0 + 8 * (i & 15);
+      r.w[k] = (row < nr && f < F)
+                   ? *reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(s.p) +
+                                                        (rbase + row) * s.code_pitch + f / 2)
+                   : 0u;
+    }
+    r.sc = 0u;
+    if (t < 128) {
+      const int row = t >> 1, f = f0 + 64 * (t & 1);
+      if (row < nr && f < F) {
+        const int rb = s.rblock[rbase + row];
+        const int b = rb >> 8, j = rb & 255;
+        r.sc = *reinterpret_cast<const uint32_t*>(
+            s.atoms + (static_cast<int64_t>(b) * s.fp64 + f / 64) * SF_ATOM_BYTES +
+            sf_atom_offset(j, 0));
+      }
+    }
+  }
+}
+
+// nr is uniform over the CTA (the NVFP4 branch has a barrier inside)
+template <int SRC>
+__device__ __forceinline__ void tq_commit(const TqRegs<SRC>& r, const TSrc& s, int nr,
+                                          float (*tile)[TQ_PITCH], uint32_t (*scw)[2]) {
+  const int t = threadIdx.x;
+  if constexpr (SRC == 0) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int i = t + TQ_THREADS * k, row = i >> 5, q = i & 31;
       if (row < nr) {
-        tile[row][4 * q] = x[k].x;
-        tile[row][4 * q + 1] = x[k].y;
-        tile[row][4 * q + 2] = x[k].z;
-        tile[row][4 * q + 3] = x[k].w;
+        tile[row][4 * q] = r.x[k].x;
+        tile[row][4 * q + 1] = r.x[k].y;
+        tile[row][4 * q + 2] = r.x[k].z;
+        tile[row][4 * q + 3] = r.x[k].w;
       }
     }
   } else if constexpr (SRC == 1) {
-    // bf16 token rows: 16 x 8 elements per row, 4 per thread
-    uint4 raw[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int i = t + TQ_THREADS * k, row = i >> 4, f = f0 + 8 * (i & 15);
-      raw[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (row < nr && f < F) {
-        const int64_t tok = s.perm[rbase + row] / s.K;
-        raw[k] = *reinterpret_cast<const uint4*>(static_cast<const bf16*>(s.p) + tok * F + f);
-      }
-    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int i = t + TQ_THREADS * k, row = i >> 4, q = i & 15;
       if (row < nr) {
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k]);
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&r.raw[k]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float2 v = __bfloat1622float2(p2[c]);
@@ -405,27 +468,7 @@ __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, i
       }
     }
   } else {
-    // NVFP4 rows: per row two words of scales (the row's 4 block scales of each
-    // 64-feature chunk are adjacent in its atom) and 16 words of 8 codes
-    __shared__ uint32_t scw[64][2];
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int i = t + TQ_THREADS * k, row = i >> 4, f = f0 + 8 * (i & 15);
-      w[k] = (row < nr && f < F) ? *reinterpret_cast<const uint32_t*>(
-                                       static_cast<const uint8_t*>(s.p) + (rbase + row) * s.code_pitch + f / 2)
-                                 : 0u;
-    }
-    if (t < 128) {
-      const int row = t >> 1, c = t & 1, f = f0 + 64 * c;
-      if (row < nr && f < F) {
-        const int rb = s.rblock[rbase + row];
-        const int b = rb >> 8, j = rb & 255;
-        scw[row][c] = *reinterpret_cast<const uint32_t*>(
-            s.atoms + (static_cast<int64_t>(b) * s.fp64 + f / 64) * SF_ATOM_BYTES +
-            sf_atom_offset(j, 0));
-      }
-    }
+    if (t < 128 && (t >> 1) < nr) scw[t >> 1][t & 1] = r.sc;
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -435,84 +478,100 @@ __device__ __forceinline__ void tq_stage(const TSrc& s, int64_t rbase, int nr, i
         const float scv = e4m3_value(static_cast<uint8_t>(sc));
 #pragma unroll
         for (int c = 0; c < 8; ++c)   // (code x scale) x g, the dequantisation order
-          tile[row][8 * q + c] = __fmul_rn(__fmul_rn(e2m1_value((w[k] >> (4 * c)) & 15u), scv), s.g);
+          tile[row][8 * q + c] =
+              __fmul_rn(__fmul_rn(e2m1_value((r.w[k] >> (4 * c)) & 15u), scv), s.g);
       }
     }
   }
 }
 
+// 64-column groups per CTA: the next group's loads are in flight while this
+// one is transformed and quantised
+constexpr int TQ_GROUPS = 4;
+
 template <int SRC, bool SR, bool STORE>
 __global__ void __launch_bounds__(TQ_THREADS) k_tq(TSrc s, const int32_t* __restrict__ offsets,
-                                            const int32_t* __restrict__ counts,
-                                            const int32_t* __restrict__ po16,
-                                            const int32_t* __restrict__ po256,
-                                            const int32_t* __restrict__ grp, int N, int F,
-                                            int64_t pitch, uint64_t seed_rht, float* amax,
-                                            uint64_t seed_sr, uint8_t* __restrict__ codes,
-                                            uint8_t* __restrict__ scales,
-                                            uint8_t* __restrict__ atoms, float* g_out) {
+                                                   const int32_t* __restrict__ counts,
+                                                   const int32_t* __restrict__ po16,
+                                                   const int32_t* __restrict__ po256,
+                                                   const int32_t* __restrict__ grp, int N, int F,
+                                                   int64_t pitch, uint64_t seed_rht, float* amax,
+                                                   uint64_t seed_sr, uint8_t* __restrict__ codes,
+                                                   uint8_t* __restrict__ scales,
+                                                   uint8_t* __restrict__ atoms, float* g_out) {
   __shared__ float tile[64][TQ_PITCH];
+  __shared__ uint32_t scw[64][2];
   pdl_wait();
   pdl_trigger();
-  const int col0 = blockIdx.y * 64;
   const int width = po256[N];
-  const int e = grp[blockIdx.y];   // read before the test (stale past the width)
-  if (col0 >= width) return;
+  const int g0 = blockIdx.y * TQ_GROUPS;
+  if (g0 * 64 >= width) return;
   const int f0 = blockIdx.x * 128;
   const int f = f0 + (threadIdx.x & 127);
-  const int hv = threadIdx.x >> 7;   // this thread's 32 of the group's 64 columns
-  const int j0 = col0 - po256[e];
-  const int ce = counts[e];
-  const int nr = min(64, ce - j0);   // rows of this group that hold data (may be <= 0)
-  if (nr > 0) tq_stage<SRC>(s, static_cast<int64_t>(offsets[e]) + j0, nr, f0, F, tile);
-  __syncthreads();
+  const int hv = threadIdx.x >> 7;   // this thread's 32 of a group's 64 columns
   const uint32_t signs = rht16_signs(seed_rht);
   float g = 0.0f;
   if constexpr (STORE) {
     g = gscale_of(*amax);
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
   }
+  const uint64_t w16 = SR ? static_cast<uint64_t>(po16[N]) : 0;
   float m = 0.0f;
-  if (f < F) {
-    uint32_t cw[4];
-    uint32_t sw = 0;
+  TqGroup cur = tq_group(g0, grp, offsets, counts, po256);
+  TqRegs<SRC> regs;
+  if (cur.nr > 0) tq_issue<SRC>(regs, s, cur.rbase, cur.nr, f0, F);
+  for (int gi = 0; gi < TQ_GROUPS; ++gi) {
+    __syncthreads();   // the previous group's transform has read the tile
+    if (cur.nr > 0) tq_commit<SRC>(regs, s, cur.nr, tile, scw);
+    __syncthreads();
+    const bool more = gi + 1 < TQ_GROUPS && (g0 + gi + 1) * 64 < width;
+    TqGroup nxt = cur;
+    if (more) {
+      nxt = tq_group(g0 + gi + 1, grp, offsets, counts, po256);
+      if (nxt.nr > 0) tq_issue<SRC>(regs, s, nxt.rbase, nxt.nr, f0, F);
+    }
+    if (f < F) {
+      uint32_t cw[4];
+      uint32_t sw = 0;
 #pragma unroll
-    for (int b2 = 0; b2 < 2; ++b2) {
-      const int bk = 2 * hv + b2;   // 16-column block of the group
-      if (16 * bk >= nr) {
-        // past the segment's rows: zeros, scale 0
-        cw[2 * b2] = cw[2 * b2 + 1] = 0u;
-        continue;
+      for (int b2 = 0; b2 < 2; ++b2) {
+        const int bk = 2 * hv + b2;   // 16-column block of the group
+        if (16 * bk >= cur.nr) {
+          // past the segment's rows: zeros, scale 0
+          cw[2 * b2] = cw[2 * b2 + 1] = 0u;
+          continue;
+        }
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[i] = (16 * bk + i < cur.nr) ? tile[16 * bk + i][threadIdx.x & 127] : 0.0f;
+        rht16_masked(v, signs);
+        if constexpr (!STORE) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+        } else {
+          const uint64_t c0 =
+              SR ? static_cast<uint64_t>(f) * w16 + po16[cur.e] + cur.j0 + 16 * bk : 0;
+          uint8_t q[8];
+          const uint8_t sc = quant16<SR>(v, g, seed_sr, c0, q);
+          cw[2 * b2] = *reinterpret_cast<const uint32_t*>(q);
+          cw[2 * b2 + 1] = *reinterpret_cast<const uint32_t*>(q + 4);
+          sw |= static_cast<uint32_t>(sc) << (8 * b2);
+        }
       }
-      float v[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        v[i] = (16 * bk + i < nr) ? tile[16 * bk + i][threadIdx.x & 127] : 0.0f;
-      rht16_masked(v, signs);
-      if constexpr (!STORE) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-      } else {
-        const uint64_t c0 = SR ? static_cast<uint64_t>(f) * static_cast<uint64_t>(po16[N]) +
-                                     po16[e] + j0 + 16 * bk
-                               : 0;
-        uint8_t q[8];
-        const uint8_t sc = quant16<SR>(v, g, seed_sr, c0, q);
-        cw[2 * b2] = *reinterpret_cast<const uint32_t*>(q);
-        cw[2 * b2 + 1] = *reinterpret_cast<const uint32_t*>(q + 4);
-        sw |= static_cast<uint32_t>(sc) << (8 * b2);
+      if constexpr (STORE) {
+        const int c32 = cur.col0 + 32 * hv;
+        *reinterpret_cast<uint4*>(codes + f * (pitch / 2) + c32 / 2) =
+            make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint16_t*>(scales + f * (pitch / 16) + c32 / 16) =
+            static_cast<uint16_t>(sw);
+        *reinterpret_cast<uint16_t*>(
+            atoms + ((static_cast<int64_t>(f) >> 7) * (pitch / 64) + cur.col0 / 64) * SF_ATOM_BYTES +
+            sf_atom_offset(f & 127, 2 * hv)) = static_cast<uint16_t>(sw);
       }
     }
-    if constexpr (STORE) {
-      const int c32 = col0 + 32 * hv;
-      *reinterpret_cast<uint4*>(codes + f * (pitch / 2) + c32 / 2) =
-          make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      *reinterpret_cast<uint16_t*>(scales + f * (pitch / 16) + c32 / 16) =
-          static_cast<uint16_t>(sw);
-      *reinterpret_cast<uint16_t*>(
-          atoms + ((static_cast<int64_t>(f) >> 7) * (pitch / 64) + col0 / 64) * SF_ATOM_BYTES +
-          sf_atom_offset(f & 127, 2 * hv)) = static_cast<uint16_t>(sw);
-    }
+    if (!more) break;
+    cur = nxt;
   }
   if constexpr (!STORE) {
     m = warp_max_f(m);
@@ -527,7 +586,9 @@ static cudaError_t launch_tq_v(const TSrc& s, const int32_t* offsets, const int3
                                int64_t pitch, uint64_t seed_rht, float* amax, uint64_t seed_sr,
                                uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* g_out,
                                cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>((F + 127) / 128), static_cast<unsigned>(pitch / 64));
+  const int64_t groups = pitch / 64;
+  const dim3 grid(static_cast<unsigned>((F + 127) / 128),
+                  static_cast<unsigned>((groups + TQ_GROUPS - 1) / TQ_GROUPS));
   return launch_pdl(k_tq<SRC, SR, STORE>, grid, TQ_THREADS, 0, st, s, offsets, counts, po16,
                     po256, grp, N, F, pitch, seed_rht, amax, seed_sr, codes, scales, atoms, g_out);
 }
