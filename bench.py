@@ -543,11 +543,27 @@ def backward_work(cfg, T: int, counts: np.ndarray):
     gradients read the weights (dense ones and the touched experts') and the
     token rows and write the gradient rows; weight gradients read the saved
     activations and the output gradients and write fp32 gradients of every
-    weight (all N experts' dW1, dW2)."""
+    weight (all N experts' dW1, dW2).  With NVFP4 experts (the training
+    recipe) the experts' GEMMs read 4-bit operands (0.5625 bytes per element
+    with their E4M3 block scales), the FC2 data gradient reads the saved bf16
+    pre-activation and writes fp32 da."""
     d, l, N, K, h, hs = cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs
     R = T * K
     touched = int((counts > 0).sum())
     wexp = touched * h * l * 2
+    if cfg.fmt == "nvfp4":
+        q = 0.5625
+        wq = int(touched * h * l * q)
+        fp4 = {
+            "bw dgrad W2^T (dg)": dict(flops=2 * R * l * h,
+                                       bytes=wq + int(R * l * q) + R * h * 2 + R * h * 4),
+            "bw dgrad W1^T (du rows)": dict(flops=2 * R * h * l,
+                                            bytes=wq + int(R * h * q) + R * l * 2),
+            "bw wgrad W2": dict(flops=2 * R * l * h, bytes=N * l * h * 4 + int(R * (l + h) * q)),
+            "bw wgrad W1": dict(flops=2 * R * h * l, bytes=N * h * l * 4 + int(R * (l + h) * q)),
+        }
+    else:
+        fp4 = {}
     return {
         "bw dgrad [W_upl|W_s2]^T (dv, dhs)": dict(flops=2 * T * d * (l + hs),
                                                   bytes=d * (l + hs) * 2 + T * d * 2 + T * (l + 2 * hs) * 2),
@@ -562,6 +578,7 @@ def backward_work(cfg, T: int, counts: np.ndarray):
         "bw wgrad W1": dict(flops=2 * R * h * l, bytes=N * h * l * 4 + R * (l + h) * 2),
         "bw wgrad [W_r;W_dn;W_s1]": dict(flops=2 * T * d * (N + l + hs),
                                          bytes=(N + l + hs) * d * 4 + T * (N + l + hs + d) * 2),
+        **fp4,
     }
 
 
@@ -700,7 +717,10 @@ def run_training(args, cfg, world, rank, local_rank):
         rate, n, el, cores = oracle_train_rate(cfg, w, x, dy, args.cpu_seconds, 1000 + cfg.seed)
         cpu = {"value": round(rate, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} of the {T} tokens (forward + backward, one at a time), {el:.1f} s"}
-    launches = (layer.launches_per_forward(T) + 12 + 1) * args.steps
+    # the profiled pass counts every kernel of the library's forward and
+    # backward; the bias update adds one
+    launches = int(round(sum(c for _, _, c in prof) / args.steps)) + 1
+    launches *= args.steps
     if rank == 0:
         line = {
             "metric": TRAIN_METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

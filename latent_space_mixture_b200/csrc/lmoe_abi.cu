@@ -953,8 +953,12 @@ static const char* const kKernelNames[] = {
     "bw dgrad [W_r;W_dn;W_s1]^T (dx)", "bw wgrad [W_upl|W_s2]", "bw wgrad W2",
     "bw wgrad W1", "bw wgrad [W_r;W_dn;W_s1]", "bw act'(da = dg 2 sqrt(g), dw)",
     // overlapped forward: the shared expert on the side stream
-    "shared W_s1 (side stream)", "shared W_s2 (side stream)"};
-static constexpr int kNumKernels = 26;
+    "shared W_s1 (side stream)", "shared W_s2 (side stream)",
+    // the routed experts' NVFP4 backward (its GEMMs keep the labels above)
+    "bw4 dL/dw = o . dv", "bw4 w dv rows -> NVFP4 (SR)", "bw4 da rows -> NVFP4 (SR)",
+    "bw4 wgrad W2 operands (g^T, do^T)", "bw4 wgrad W1 operands (u^T, da^T)",
+    "bw4 zero gradients of experts without rows"};
+static constexpr int kNumKernels = 32;
 
 // Dense-GEMM plan for T tokens: token-block width and number of K slices.
 // Enough tiles to fill the GPU first by narrower token blocks (while one
@@ -2366,12 +2370,12 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
                                            st));
   }
   // 3. dL/dw = o . dv
-  LMOE_STEP(17, launch_dw_rows(h->O, h->inv, dv, T, K, l, dw, st));
+  LMOE_STEP(26, launch_dw_rows(h->O, h->inv, dv, T, K, l, dw, st));
   // 4. do = w dv rows, stochastically rounded to NVFP4 (1D blocks along l)
-  LMOE_STEP(13, launch_rows_scaled(dv, h->perm, h->wrow, R, K, l, h->do32, amax + 0, st));
-  LMOE_STEP(13, launch_quant_rows_dev(h->do32, R, l, amax + 0, true, seed + 0, h->doq, lp / 2,
+  LMOE_STEP(27, launch_rows_scaled(dv, h->perm, h->wrow, R, K, l, h->do32, amax + 0, st));
+  LMOE_STEP(27, launch_quant_rows_dev(h->do32, R, l, amax + 0, true, seed + 0, h->doq, lp / 2,
                                       h->doS, gsc + 0, st));
-  LMOE_STEP(13, launch_atoms_rblock(h->doS, h->rblock, R, l / 16, lp / 64, h->sfbdo, st));
+  LMOE_STEP(27, launch_atoms_rblock(h->doS, h->rblock, R, l / 16, lp / 64, h->sfbdo, st));
   // 5. dg = W2q^T Q(do); da = dg 2 max(a, 0) (fp32) and its amax
   {
     TileSource s{0, 0, h->blocks, h->nblocks, hh / 128, hh, hh, lp / 256, 1, nullptr,
@@ -2381,9 +2385,9 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
                                             lim, st));
   }
   // 6. da stochastically rounded (1D blocks along h); du rows = W1q^T Q(da)
-  LMOE_STEP(23, launch_quant_rows_dev(h->da32, R, hh, amax + 1, true, seed + 1, h->daq, hp / 2,
+  LMOE_STEP(28, launch_quant_rows_dev(h->da32, R, hh, amax + 1, true, seed + 1, h->daq, hp / 2,
                                       h->daS, gsc + 1, st));
-  LMOE_STEP(23, launch_atoms_rblock(h->daS, h->rblock, R, hh / 16, hp / 64, h->sfbda, st));
+  LMOE_STEP(28, launch_atoms_rblock(h->daS, h->rblock, R, hh / 16, hp / 64, h->sfbda, st));
   {
     TileSource s{0, 0, h->blocks, h->nblocks, l / 128, l, l, hp / 256, 1, nullptr, gbn == 32,
                  h->w1qT_sf, h->sfbda, hp / 64};
@@ -2395,7 +2399,7 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
   LMOE_STEP(16, launch_combine(h->O, h->inv, T, K, l, du, ldu, st));
   // 8. weight gradients: per expert, over its rows (the K dimension),
   //    transformed operands padded to 256-row segments
-  LMOE_STEP(20, launch_seg_offsets(h->counts, N, h->po16, h->po256, h->kofs, h->grp, st));
+  LMOE_STEP(29, launch_seg_offsets(h->counts, N, h->po16, h->po256, h->kofs, h->grp, st));
   const int64_t kc = pitch / 64;
   TSrc src_do{h->do32, nullptr, nullptr, nullptr, K, 0, 0, 0.f};
   TSrc src_g{h->Hq, nullptr, h->rblock, h->sfbh, K, hp / 2, hp / 64, h->g_h};
@@ -2404,13 +2408,13 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
   // dW2[e] = Q_sr(R(do_e^T)) Q(R(g_e^T))^T: A = g^T (features h), B = do^T (rows l)
   const int32_t *off = h->offsets, *cnt = h->counts, *p16 = h->po16, *p256 = h->po256,
                 *grp = h->grp;
-  LMOE_STEP(20, launch_tq_amax(2, src_g, off, cnt, p16, p256, grp, N, hh, pitch, seed + 2,
+  LMOE_STEP(29, launch_tq_amax(2, src_g, off, cnt, p16, p256, grp, N, hh, pitch, seed + 2,
                                amax + 3, st));
-  LMOE_STEP(20, launch_tq_amax(0, src_do, off, cnt, p16, p256, grp, N, l, pitch, seed + 2,
+  LMOE_STEP(29, launch_tq_amax(0, src_do, off, cnt, p16, p256, grp, N, l, pitch, seed + 2,
                                amax + 2, st));
-  LMOE_STEP(20, launch_tq_quant(2, false, src_g, off, cnt, p16, p256, grp, N, hh, pitch, seed + 2,
+  LMOE_STEP(29, launch_tq_quant(2, false, src_g, off, cnt, p16, p256, grp, N, hh, pitch, seed + 2,
                                 amax + 3, 0, h->tq[1], h->ts[1], h->ta[1], gsc + 3, st));
-  LMOE_STEP(20, launch_tq_quant(0, true, src_do, off, cnt, p16, p256, grp, N, l, pitch, seed + 2,
+  LMOE_STEP(29, launch_tq_quant(0, true, src_do, off, cnt, p16, p256, grp, N, l, pitch, seed + 2,
                                 amax + 2, seed + 3, h->tq[0], h->ts[0], h->ta[0], gsc + 2, st));
   {
     TileSource s{2, 0, nullptr, nullptr, hh / 128, 0, hh, 0, 1, nullptr, 0, h->ta[1], h->ta[0],
@@ -2421,13 +2425,13 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
                                             lim, st));
   }
   // dW1[e] = Q_sr(R(da_e^T)) Q(R(u_e^T))^T: A = u^T (features l), B = da^T (rows h)
-  LMOE_STEP(21, launch_tq_amax(1, src_u, off, cnt, p16, p256, grp, N, l, pitch, seed + 4,
+  LMOE_STEP(30, launch_tq_amax(1, src_u, off, cnt, p16, p256, grp, N, l, pitch, seed + 4,
                                amax + 5, st));
-  LMOE_STEP(21, launch_tq_amax(0, src_da, off, cnt, p16, p256, grp, N, hh, pitch, seed + 4,
+  LMOE_STEP(30, launch_tq_amax(0, src_da, off, cnt, p16, p256, grp, N, hh, pitch, seed + 4,
                                amax + 4, st));
-  LMOE_STEP(21, launch_tq_quant(1, false, src_u, off, cnt, p16, p256, grp, N, l, pitch, seed + 4,
+  LMOE_STEP(30, launch_tq_quant(1, false, src_u, off, cnt, p16, p256, grp, N, l, pitch, seed + 4,
                                 amax + 5, 0, h->tq[2], h->ts[2], h->ta[2], gsc + 5, st));
-  LMOE_STEP(21, launch_tq_quant(0, true, src_da, off, cnt, p16, p256, grp, N, hh, pitch, seed + 4,
+  LMOE_STEP(30, launch_tq_quant(0, true, src_da, off, cnt, p16, p256, grp, N, hh, pitch, seed + 4,
                                 amax + 4, seed + 5, h->tq[3], h->ts[3], h->ta[3], gsc + 4, st));
   {
     TileSource s{2, 0, nullptr, nullptr, l / 128, 0, l, 0, 1, nullptr, 0, h->ta[2], h->ta[3],
@@ -2438,8 +2442,8 @@ static int experts_bw4(lmoe_handle* h, const void* u, const int32_t* topk_idx,
                                             lim, st));
   }
   // experts without rows: zero gradients
-  LMOE_STEP(20, launch_zero_empty(h->counts, N, int64_t(l) * hh, d_w2, st));
-  LMOE_STEP(21, launch_zero_empty(h->counts, N, int64_t(hh) * l, d_w1, st));
+  LMOE_STEP(31, launch_zero_empty(h->counts, N, int64_t(l) * hh, d_w2, st));
+  LMOE_STEP(31, launch_zero_empty(h->counts, N, int64_t(hh) * l, d_w1, st));
   return LMOE_OK;
 }
 
