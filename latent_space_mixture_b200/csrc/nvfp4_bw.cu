@@ -486,8 +486,13 @@ __device__ __forceinline__ void tq_commit(const TqRegs<SRC>& r, const TSrc& s, i
 }
 
 // 64-column groups per CTA: the next group's loads are in flight while this
-// one is transformed and quantised
-constexpr int TQ_GROUPS = 4;
+// one is transformed and quantised.  The stochastically rounding pass keeps
+// one group per CTA: it is bound by its arithmetic (the random bits), and
+// the registers that hold a group in flight would cost it occupancy.
+template <bool SR>
+struct TqGroups {
+  static constexpr int value = SR ? 1 : 4;
+};
 
 template <int SRC, bool SR, bool STORE>
 __global__ void __launch_bounds__(TQ_THREADS) k_tq(TSrc s, const int32_t* __restrict__ offsets,
@@ -504,6 +509,7 @@ __global__ void __launch_bounds__(TQ_THREADS) k_tq(TSrc s, const int32_t* __rest
   pdl_wait();
   pdl_trigger();
   const int width = po256[N];
+  constexpr int TQ_GROUPS = TqGroups<SR>::value;
   const int g0 = blockIdx.y * TQ_GROUPS;
   if (g0 * 64 >= width) return;
   const int f0 = blockIdx.x * 128;
@@ -587,8 +593,9 @@ static cudaError_t launch_tq_v(const TSrc& s, const int32_t* offsets, const int3
                                uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* g_out,
                                cudaStream_t st) {
   const int64_t groups = pitch / 64;
+  constexpr int per = TqGroups<SR>::value;
   const dim3 grid(static_cast<unsigned>((F + 127) / 128),
-                  static_cast<unsigned>((groups + TQ_GROUPS - 1) / TQ_GROUPS));
+                  static_cast<unsigned>((groups + per - 1) / per));
   return launch_pdl(k_tq<SRC, SR, STORE>, grid, TQ_THREADS, 0, st, s, offsets, counts, po16,
                     po256, grp, N, F, pitch, seed_rht, amax, seed_sr, codes, scales, atoms, g_out);
 }
