@@ -49,16 +49,19 @@ struct PairLayout {
   static constexpr bool PAIRED_RELEASE = false;
 };
 
-// tile -> (token block, 256-row feature block), feature block fastest; the
-// CTA of rank r owns weight rows [a_row, a_row + 128)
+// tile -> (token block, K slice, 256-row feature block), feature block
+// fastest; the CTA of rank r owns weight rows [a_row, a_row + 128).  With
+// ksplit > 1 (dense GEMMs of few tokens) each slice writes fp32 partials
+// part[slice][row][feature], summed by the split-K reduction kernels.
 __device__ __forceinline__ TileInfo pair_tile(const TileSource& s, int BN, int tile, int rank) {
   TileInfo t;
-  const int tb = tile / s.FB;
-  t.fb = tile - tb * s.FB;
+  const int tk = tile / s.FB;
+  t.fb = tile - tk * s.FB;
+  const int tb = tk / s.ksplit;
   t.tb = tb;
-  t.ks = 0;
-  t.kb0 = 0;
-  t.kb1 = s.kblocks;
+  t.ks = tk - tb * s.ksplit;
+  t.kb0 = t.ks * s.kblocks / s.ksplit;
+  t.kb1 = (t.ks + 1) * s.kblocks / s.ksplit;
   if (s.dense) {
     t.e = 0;
     t.row0 = tb * BN;
@@ -293,8 +296,18 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           const bool valid = c0 + j < t.nrows && feat < src.m_valid;
           const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
           const float4 lo = p[0], hi = p[1];
-          const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-          epi.store8(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid);
+          const long row = static_cast<long>(t.row0 + c0 + j);
+          if (src.ksplit > 1) {
+            if (valid) {
+              float4* dst = reinterpret_cast<float4*>(
+                  src.part + (static_cast<long>(t.ks) * src.T + row) * src.m_valid + feat);
+              dst[0] = lo;
+              dst[1] = hi;
+            }
+          } else {
+            const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            epi.store8(t, row, feat, v, valid);
+          }
         }
         __syncwarp();
       }

@@ -1612,16 +1612,42 @@ void lmoe_destroy(lmoe_handle* h) {
 
 static int overlap_sms(const lmoe_handle* h, int64_t T);
 
+// A dense GEMM of T tokens over F output features and kblocks 64-wide K
+// steps: on CTA pairs (256 x 256 tiles) when their tiles fill the GPU; for a
+// single token block (decode-sized batches) on pairs with K split into enough
+// slices to fill it (each pair loads half the token block that a single CTA
+// would, per weight byte), when the partials fit the split-K buffer; else on
+// single CTAs (plan_dense).  `ctas` counts pairs for the pair kernel.
+struct DenseChoice {
+  bool pair;
+  int bn, ksplit;
+  int ctas;
+};
+static DenseChoice choose_dense(const lmoe_handle* h, int64_t T, int F, int kblocks) {
+  const int fb2 = (F + PAIR_BM - 1) / PAIR_BM;
+  const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
+  if (h->pairs && ptiles >= h->sms / 2) return {true, PAIR_BN, 1, h->sms / 2};
+  if (h->pairs && T <= PAIR_BN) {
+    int64_t ks = (h->sms / 2) / ptiles;
+    if (ks > 8) ks = 8;
+    if (ks > kblocks / 4) ks = kblocks / 4;
+    if (ks >= 2 && ks * T * F <= h->part_floats)
+      return {true, PAIR_BN, static_cast<int>(ks), static_cast<int>(ptiles * ks)};
+  }
+  const int fb = (F + 127) / 128;
+  const DensePlan p = plan_dense(T, fb, kblocks, h->sms);
+  const int64_t tiles = ((T + p.bn - 1) / p.bn) * fb * p.ksplit;
+  return {false, p.bn, p.ksplit, static_cast<int>(tiles < h->sms ? tiles : h->sms)};
+}
+
 int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T) {
   if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return 0;
   const lmoe_config& c = h->cfg;
-  const DensePlan px = plan_dense(T, (c.n_experts + h->lx + c.shared_hidden + 127) / 128,
-                                  c.d / 64, h->sms);
-  const DensePlan py = plan_dense(T, (c.d + 127) / 128, (h->lx + c.shared_hidden) / 64, h->sms);
-  (void)px;   // a split x-GEMM's reduction replaces the router kernel: same count
+  // a split x-GEMM's reduction replaces the router kernel: same count
+  const DenseChoice cy = choose_dense(h, T, c.d, (h->lx + c.shared_hidden) / 64);
   // an overlapped forward runs the shared expert's two GEMMs apart
-  return 10 + (py.ksplit > 1) + (overlap_sms(h, T) > 0 ? 2 : 0);
+  return 10 + (cy.ksplit > 1) + (overlap_sms(h, T) > 0 ? 2 : 0);
 }
 
 static int prof_begin(lmoe_handle* h, int kernel, cudaStream_t st) {
@@ -1733,30 +1759,26 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st, 
                  N + lx, static_cast<int>(d / 64), 1, nullptr, 0};
     LMOE_STEP(0, launch_gemm_pair(h->tm_wx, tm_x, s, epi, (h->sms - side) / 2, h->err, lim, st));
   } else {
-    const int fb = (N + lx + hs + 127) / 128;
-    const DensePlan p = plan_dense(T, fb, static_cast<int>(d / 64), h->sms);
+    const int F = N + lx + hs;
+    const DenseChoice dc = choose_dense(h, T, F, static_cast<int>(d / 64));
     EpiX epi{h->logits, h->u, h->vh, N, lx, l, ldvh, h->uq, h->usf, h->g_u, h->stab, h->uf8, h->r_u8,
              h->u16};
-    const int fb2 = (N + lx + hs + PAIR_BM - 1) / PAIR_BM;
-    const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
-    if (h->pairs && ptiles >= h->sms / 2) {
-      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, N + lx + hs,
-                   static_cast<int>(d / 64), 1, nullptr, 0};
-      LMOE_STEP(0, launch_gemm_pair(h->tm_wx, tm_x, s, epi, h->sms / 2, h->err, lim, st));
-    } else {
-    if (p.ksplit > 1 && int64_t(p.ksplit) * T * (N + lx + hs) > h->part_floats)
+    if (dc.ksplit > 1 && int64_t(dc.ksplit) * T * F > h->part_floats)
       return LMOE_ERR_UNSUPPORTED;   // never: the buffer is sized for every T
-    TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, N + lx + hs,
-                 static_cast<int>(d / 64), p.ksplit, h->part, T <= p.bn};
-    const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
-    const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
-    LMOE_STEP(0, launch_gemm_bn(p.bn, h->tm_wx, tm_x, s, epi, grid, h->err, lim, st));
-    // at split-K sizes the reduction also routes: logits, top-K, weights
-    if (p.ksplit > 1)
-      LMOE_STEP(10, launch_reduce_route(h->part, p.ksplit, static_cast<int>(T), N + lx + hs, N,
-                                        epi, h->bias, K, h->logits, h->topk_idx, h->topk_w, st));
-    routed = p.ksplit > 1;
+    if (dc.pair) {
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, (F + PAIR_BM - 1) / PAIR_BM, 0, F,
+                   static_cast<int>(d / 64), dc.ksplit, h->part, dc.ksplit > 1};
+      LMOE_STEP(0, launch_gemm_pair(h->tm_wx, tm_x, s, epi, dc.ctas, h->err, lim, st));
+    } else {
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, (F + 127) / 128, 0, F,
+                   static_cast<int>(d / 64), dc.ksplit, h->part, T <= dc.bn};
+      LMOE_STEP(0, launch_gemm_bn(dc.bn, h->tm_wx, tm_x, s, epi, dc.ctas, h->err, lim, st));
     }
+    // at split-K sizes the reduction also routes: logits, top-K, weights
+    if (dc.ksplit > 1)
+      LMOE_STEP(10, launch_reduce_route(h->part, dc.ksplit, static_cast<int>(T), F, N, epi,
+                                        h->bias, K, h->logits, h->topk_idx, h->topk_w, st));
+    routed = dc.ksplit > 1;
   }
   // 2-5. routing and segments
   const int gbn = grouped_bn(c, T);
@@ -1781,29 +1803,24 @@ static int fwd_ygemm(lmoe_handle* h, int64_t T, void* y, cudaStream_t st, bool o
   const unsigned long long lim = h->wait_limit_ns;
   if (overlapped && cudaStreamWaitEvent(st, h->ev_join, 0) != cudaSuccess) return LMOE_ERR_CUDA;
   {
-    const int fb = static_cast<int>((d + 127) / 128);
+    const int F = static_cast<int>(d);
     const int ky = overlapped ? lx : lx + hs;   // K of the y-GEMM
-    const DensePlan p = plan_dense(T, fb, ky / 64, h->sms);
-    if (p.ksplit > 1 && int64_t(p.ksplit) * T * d > h->part_floats)
+    const DenseChoice dc = choose_dense(h, T, F, ky / 64);
+    if (dc.ksplit > 1 && int64_t(dc.ksplit) * T * d > h->part_floats)
       return LMOE_ERR_UNSUPPORTED;   // never: the buffer is sized for every T
     EpiY epi{static_cast<bf16*>(y), static_cast<int>(d), h->proj ? nullptr : h->vh, ldvh,
              nullptr, overlapped ? h->ys : nullptr};
-    const int fb2 = static_cast<int>((d + PAIR_BM - 1) / PAIR_BM);
-    const int64_t ptiles = ((T + PAIR_BN - 1) / PAIR_BN) * fb2;
-    if (h->pairs && ptiles >= h->sms / 2) {
-      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb2, 0, static_cast<int>(d),
-                   ky / 64, 1, nullptr, 0};
-      LMOE_STEP(9, launch_gemm_pair(h->tm_wy, h->tm_vh, s, epi, h->sms / 2, h->err, lim, st));
+    if (dc.pair) {
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, (F + PAIR_BM - 1) / PAIR_BM, 0, F,
+                   ky / 64, dc.ksplit, h->part, dc.ksplit > 1};
+      LMOE_STEP(9, launch_gemm_pair(h->tm_wy, h->tm_vh, s, epi, dc.ctas, h->err, lim, st));
     } else {
-      TileSource s{1, static_cast<int>(T), nullptr, nullptr, fb, 0, static_cast<int>(d),
-                   ky / 64, p.ksplit, h->part, T <= p.bn};
-      const int64_t tiles = ((T + p.bn - 1) / p.bn) * s.FB * p.ksplit;
-      const int grid = static_cast<int>(tiles < h->sms ? tiles : h->sms);
-      LMOE_STEP(9, launch_gemm_bn(p.bn, h->tm_wy, h->tm_vh, s, epi, grid, h->err, lim, st));
-      if (p.ksplit > 1)
-        LMOE_STEP(11, launch_reduce(h->part, p.ksplit, static_cast<int>(T), static_cast<int>(d),
-                                    epi, st));
+      TileSource s{1, static_cast<int>(T), nullptr, nullptr, (F + 127) / 128, 0, F, ky / 64,
+                   dc.ksplit, h->part, T <= dc.bn};
+      LMOE_STEP(9, launch_gemm_bn(dc.bn, h->tm_wy, h->tm_vh, s, epi, dc.ctas, h->err, lim, st));
     }
+    if (dc.ksplit > 1)
+      LMOE_STEP(11, launch_reduce(h->part, dc.ksplit, static_cast<int>(T), F, epi, st));
   }
   return LMOE_OK;
 }
