@@ -391,33 +391,33 @@ k_gemm_bw(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             }
             ++nbox;
           }
-          continue;
-        }
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) my[j * GEMM_STG_LD + lane] = __uint_as_float(r[j]);
-        __syncwarp();
-        uint4 nxt[4] = {};
-        if constexpr (Epi::kAux)
-          if (c0 + 32 < t.nrows) fetch_chunk(t, c0 + 32, nxt);
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          // lanes 4j..4j+3 hold the four 8-feature groups of output row j
-          const int item = lane + 32 * it;
-          const int j = item >> 2;
-          const int g = item & 3;
-          const int feat = feat_base + g * 8;
-          const bool valid = c0 + j < t.nrows && feat < src.m_valid;
-          const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
-          const float4 lo = p[0], hi = p[1];
-          const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          for (int j = 0; j < 32; ++j) my[j * GEMM_STG_LD + lane] = __uint_as_float(r[j]);
+          __syncwarp();
+          uint4 nxt[4] = {};
           if constexpr (Epi::kAux)
-            epi.store8(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid, aux[it]);
-          else if constexpr (!Epi::kTma)
-            epi.store8(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid);
-        }
-        __syncwarp();
+            if (c0 + 32 < t.nrows) fetch_chunk(t, c0 + 32, nxt);
 #pragma unroll
-        for (int it = 0; it < 4; ++it) aux[it] = nxt[it];
+          for (int it = 0; it < 4; ++it) {
+            // lanes 4j..4j+3 hold the four 8-feature groups of output row j
+            const int item = lane + 32 * it;
+            const int j = item >> 2;
+            const int g = item & 3;
+            const int feat = feat_base + g * 8;
+            const bool valid = c0 + j < t.nrows && feat < src.m_valid;
+            const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
+            const float4 lo = p[0], hi = p[1];
+            const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            if constexpr (Epi::kAux)
+              epi.store8(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid, aux[it]);
+            else
+              epi.store8(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 4; ++it) aux[it] = nxt[it];
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

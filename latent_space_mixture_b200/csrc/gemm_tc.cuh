@@ -663,32 +663,32 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             epi.store16(t, static_cast<long>(t.row0 + c0 + j), feat, v, valid);
           }
           __syncwarp();
-          continue;
-        }
+        } else {
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          // lanes 4j..4j+3 hold the four 8-feature groups of token row j
-          const int item = lane + 32 * it;
-          const int j = item >> 2;
-          const int g = item & 3;
-          const int feat = feat_base + g * 8;
-          const bool valid = c0 + j < t.nrows && feat < src.m_valid;
-          const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
-          const float4 lo = p[0], hi = p[1];
-          const long row = static_cast<long>(t.row0 + c0 + j);
-          if (src.ksplit > 1) {
-            if (valid) {
-              float4* dst = reinterpret_cast<float4*>(
-                  src.part + (static_cast<long>(t.ks) * src.T + row) * src.m_valid + feat);
-              dst[0] = lo;
-              dst[1] = hi;
+          for (int it = 0; it < 4; ++it) {
+            // lanes 4j..4j+3 hold the four 8-feature groups of token row j
+            const int item = lane + 32 * it;
+            const int j = item >> 2;
+            const int g = item & 3;
+            const int feat = feat_base + g * 8;
+            const bool valid = c0 + j < t.nrows && feat < src.m_valid;
+            const float4* p = reinterpret_cast<const float4*>(my + j * GEMM_STG_LD + g * 8);
+            const float4 lo = p[0], hi = p[1];
+            const long row = static_cast<long>(t.row0 + c0 + j);
+            if (src.ksplit > 1) {
+              if (valid) {
+                float4* dst = reinterpret_cast<float4*>(
+                    src.part + (static_cast<long>(t.ks) * src.T + row) * src.m_valid + feat);
+                dst[0] = lo;
+                dst[1] = hi;
+              }
+            } else {
+              const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+              epi.store8(t, row, feat, v, valid);
             }
-          } else {
-            const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-            epi.store8(t, row, feat, v, valid);
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
       }
       tc_fence_before();

@@ -24,6 +24,23 @@ def test_weight_gradient_bytes_cover_fp32_outputs():
     assert bwd["bw wgrad W2"]["bytes"] >= cfg.N * cfg.h * cfg.l * 4
 
 
+def test_nvfp4_backward_bytes_count_four_bit_operands():
+    """With NVFP4 experts the experts' backward GEMMs read 4-bit operands
+    (0.5625 bytes per element with their block scales) and still write fp32
+    weight gradients; their flops are those of the BF16 layer."""
+    bf, fp = CONFIGS["super_prefill"], CONFIGS["super_prefill_nvfp4_2d"]
+    counts = np.ones(bf.N, dtype=np.int64)
+    b16 = bench.backward_work(bf, bf.T, counts)
+    b4 = bench.backward_work(fp, fp.T, counts)
+    R = fp.T * fp.K
+    for k in ("bw wgrad W1", "bw wgrad W2"):
+        assert b4[k]["flops"] == b16[k]["flops"]
+        assert b4[k]["bytes"] == fp.N * fp.h * fp.l * 4 + int(R * (fp.l + fp.h) * 0.5625)
+        assert b4[k]["bytes"] < b16[k]["bytes"]
+    for k in ("bw dgrad W2^T (dg)", "bw dgrad W1^T (du rows)"):
+        assert b4[k]["flops"] == b16[k]["flops"]
+
+
 def _reference_line(monkeypatch, capsys, name, backward=False):
     import argparse
     import json
