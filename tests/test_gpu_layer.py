@@ -205,6 +205,30 @@ def test_cta_pair_gemms_match_single_cta_gemms(monkeypatch):
     pair.close()
 
 
+def test_split_k_pair_dense_gemms_match_single_cta(monkeypatch):
+    """At decode-sized batches (one block of <= 256 tokens) the x- and
+    y-GEMMs run on CTA pairs with K split into slices (fp32 partials summed
+    by the split-K reductions); the layer matches the single-CTA split-K one
+    (within 1e-2 of RMS(y): near-tie tokens may route apart) and the
+    oracle."""
+    cfg = CONFIGS["pair_small"]
+    monkeypatch.setenv("LMOE_PAIR", "0")
+    w, x, single = make(cfg, T=256)
+    y1 = single.forward(x).clone()
+    monkeypatch.setenv("LMOE_PAIR", "1")
+    from latent_space_mixture_b200 import LatentMoE
+    pair = LatentMoE(cfg.d, cfg.l, cfg.N, cfg.K, cfg.h, cfg.hs, 256, w)
+    y2 = pair.forward(x)
+    torch.cuda.synchronize()
+    assert pair.sync_status() == 0 and single.sync_status() == 0
+    assert max_rel(to64(y2), to64(y1)) <= 1e-2
+    toks = np.unique(np.concatenate([[0, 255], _sample(256, 24, 11)]))
+    errs = compare_layer(pair, w, x, y2, toks, cfg.K)
+    print("split-K pair errors:", errs)
+    single.close()
+    pair.close()
+
+
 def test_overlapped_shared_expert_matches_serial_forward(monkeypatch):
     """The forward that runs the shared expert's GEMMs on a side stream over
     a share of the SMs (opt-in, LMOE_OVERLAP; forced here) equals the serial
