@@ -159,15 +159,27 @@ __device__ __forceinline__ uint8_t nvfp4_scale_tab(float amax, const float* __re
 // SplitMix64 output for counter ctr, up to its last step z ^ (z >> 31): that
 // step leaves bits 33..63 unchanged, and only the top 24 bits (uniforms) and
 // bit 63 (the transform's signs) are used.
-__device__ __forceinline__ uint64_t splitmix64_high(uint64_t seed, uint64_t ctr) {
-  uint64_t z = seed + (ctr + 1ull) * 0x9E3779B97F4A7C15ull;
+constexpr uint64_t SPLITMIX_GAMMA = 0x9E3779B97F4A7C15ull;
+
+// the mixing steps from the state z = seed + (ctr + 1) gamma
+__device__ __forceinline__ uint64_t splitmix64_mix_high(uint64_t z) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
   return (z ^ (z >> 27)) * 0x94D049BB133111EBull;
 }
 
-__device__ __forceinline__ float uniform24(uint64_t seed, uint64_t ctr) {
-  return static_cast<float>(static_cast<uint32_t>(splitmix64_high(seed, ctr) >> 40)) *
+__device__ __forceinline__ uint64_t splitmix64_high(uint64_t seed, uint64_t ctr) {
+  return splitmix64_mix_high(seed + (ctr + 1ull) * SPLITMIX_GAMMA);
+}
+
+// a uniform in [0, 1) from the state of a counter (consecutive counters'
+// states differ by gamma, so a run of them costs one multiply less each)
+__device__ __forceinline__ float uniform24_z(uint64_t z) {
+  return static_cast<float>(static_cast<uint32_t>(splitmix64_mix_high(z) >> 40)) *
          5.9604644775390625e-8f;   // 2^-24
+}
+
+__device__ __forceinline__ float uniform24(uint64_t seed, uint64_t ctr) {
+  return uniform24_z(seed + (ctr + 1ull) * SPLITMIX_GAMMA);
 }
 
 // Stochastic rounding of v to an E2M1 code (bit 3 = sign): the upper grid

@@ -67,10 +67,14 @@ __device__ __forceinline__ uint8_t quant16(const float (&v)[16], float g, uint64
     const uint8_t sc = e4m3_code(sbf);
     const float denom = __fmul_rn(e4m3_value(sc), g);
     const float r = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+    // counters c0 .. c0 + 15: their states step by gamma
+    uint64_t z = seed + (c0 + 1ull) * SPLITMIX_GAMMA;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const uint32_t lo = e2m1_sr(__fmul_rn(v[2 * j], r), uniform24(seed, c0 + 2 * j));
-      const uint32_t hi = e2m1_sr(__fmul_rn(v[2 * j + 1], r), uniform24(seed, c0 + 2 * j + 1));
+      const uint32_t lo = e2m1_sr(__fmul_rn(v[2 * j], r), uniform24_z(z));
+      z += SPLITMIX_GAMMA;
+      const uint32_t hi = e2m1_sr(__fmul_rn(v[2 * j + 1], r), uniform24_z(z));
+      z += SPLITMIX_GAMMA;
       q[j] = static_cast<uint8_t>(lo | (hi << 4));
     }
     return sc;
