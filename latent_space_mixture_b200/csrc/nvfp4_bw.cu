@@ -358,6 +358,14 @@ cudaError_t launch_seg_offsets(const int32_t* counts, int N, int32_t* po16, int3
 constexpr int TQ_PITCH = 129;
 constexpr int TQ_THREADS = 256;   // two threads per feature, 32 columns each
 
+// E2M1 code -> value with the eight magnitudes x 2 (0, 1, 2, 3, 4, 6, 8, 12)
+// as the nibbles of one word: a shift, a mask and a conversion (the same
+// values as e2m1_value, -0 for code 8 included)
+__device__ __forceinline__ float e2m1_value_nib(uint32_t code) {
+  const float m = static_cast<float>((0xC8643210u >> (4u * (code & 7u))) & 15u) * 0.5f;
+  return (code & 8u) ? -m : m;
+}
+
 // One 64-column group of the CTA: its expert, first row of the segment in
 // the group, rows with data (nr, may be <= 0).
 struct TqGroup {
@@ -483,7 +491,7 @@ __device__ __forceinline__ void tq_commit(const TqRegs<SRC>& r, const TSrc& s, i
 #pragma unroll
         for (int c = 0; c < 8; ++c)   // (code x scale) x g, the dequantisation order
           tile[row][8 * q + c] =
-              __fmul_rn(__fmul_rn(e2m1_value((r.w[k] >> (4 * c)) & 15u), scv), s.g);
+              __fmul_rn(__fmul_rn(e2m1_value_nib((r.w[k] >> (4 * c)) & 15u), scv), s.g);
       }
     }
   }
