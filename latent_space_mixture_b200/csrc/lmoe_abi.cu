@@ -431,15 +431,6 @@ struct EpiWq {
     *x = feat;
     *y = t.e * rows + static_cast<int>(row);
   }
-  __device__ __forceinline__ void store32(const TileInfo& t, long row, int feat, const float* v,
-                                          bool valid) const {
-    if (!valid) return;
-    const float s = __fmul_rn(*g_a, *g_b);
-    float4* p = reinterpret_cast<float4*>(out + (static_cast<long>(t.e) * rows + row) * cols + feat);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      p[i] = make_float4(v[4 * i] * s, v[4 * i + 1] * s, v[4 * i + 2] * s, v[4 * i + 3] * s);
-  }
   __device__ __forceinline__ void store8(const TileInfo& t, long row, int feat, const float* v,
                                          bool valid) const {
     if (!valid) return;
