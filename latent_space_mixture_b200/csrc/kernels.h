@@ -28,6 +28,15 @@ cudaError_t launch_scatter(const int32_t* topk_idx, const float* topk_w, const i
                            int4* blocks, int32_t* nblocks, int32_t* rblock, int* err,
                            cudaStream_t st);
 
+// The three steps above in one block for at most SEG_SMALL_T tokens (N <=
+// 1024): counts[e], offsets, perm / inv / row weights, the token-block list
+// and rblock, the same values as launch_hist + launch_scan + launch_scatter.
+constexpr int SEG_SMALL_T = 256;
+cudaError_t launch_segments_small(const int32_t* topk_idx, const float* topk_w, int64_t T, int N,
+                                  int K, int bn, int32_t* counts, int32_t* offsets, int32_t* perm,
+                                  int32_t* inv, float* wrow, int4* blocks, int32_t* nblocks,
+                                  int32_t* rblock, int* err, cudaStream_t st);
+
 // u_perm[r] = u[perm[r] / K] for r < T*K (rows of width l, bf16).
 cudaError_t launch_gather(const void* u, const int32_t* perm, int64_t rows, int K, int l,
                           void* u_perm, cudaStream_t st);

@@ -948,8 +948,11 @@ static const char* const kKernelNames[] = {
     // the routed experts' NVFP4 backward (its GEMMs keep the labels above)
     "bw4 dL/dw = o . dv", "bw4 w dv rows -> NVFP4 (SR)", "bw4 da rows -> NVFP4 (SR)",
     "bw4 wgrad W2 operands (g^T, do^T)", "bw4 wgrad W1 operands (u^T, da^T)",
-    "bw4 zero gradients of experts without rows"};
-static constexpr int kNumKernels = 32;
+    "bw4 zero gradients of experts without rows",
+    // forward, at most 256 tokens
+    "segments (hist+scan+scatter, one block)"};
+static constexpr int kNumKernels = 33;
+static_assert(sizeof(kKernelNames) / sizeof(kKernelNames[0]) == kNumKernels, "kernel labels");
 
 // Dense-GEMM plan for T tokens: token-block width and number of K slices.
 // Enough tiles to fill the GPU first by narrower token blocks (while one
@@ -1635,10 +1638,12 @@ int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T) {
   if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return 0;
   const lmoe_config& c = h->cfg;
-  // a split x-GEMM's reduction replaces the router kernel: same count
+  // a split x-GEMM's reduction replaces the router kernel: same count; the
+  // segments take one kernel up to SEG_SMALL_T tokens, else three
   const DenseChoice cy = choose_dense(h, T, c.d, (h->lx + c.shared_hidden) / 64);
+  const int seg = (T <= SEG_SMALL_T && c.n_experts <= 1024) ? 1 : 3;
   // an overlapped forward runs the shared expert's two GEMMs apart
-  return 10 + (cy.ksplit > 1) + (overlap_sms(h, T) > 0 ? 2 : 0);
+  return 7 + seg + (cy.ksplit > 1) + (overlap_sms(h, T) > 0 ? 2 : 0);
 }
 
 static int prof_begin(lmoe_handle* h, int kernel, cudaStream_t st) {
@@ -1775,6 +1780,12 @@ static int fwd_front(lmoe_handle* h, const void* x, int64_t T, cudaStream_t st, 
   const int gbn = grouped_bn(c, T);
   if (!routed)
     LMOE_STEP(1, launch_route(h->logits, h->bias, T, N, K, h->topk_idx, h->topk_w, st));
+  if (T <= SEG_SMALL_T && N <= 1024) {
+    LMOE_STEP(32, launch_segments_small(h->topk_idx, h->topk_w, T, N, K, gbn, h->counts,
+                                        h->offsets, h->perm, h->inv, h->wrow, h->blocks,
+                                        h->nblocks, h->rblock, h->err, st));
+    return LMOE_OK;
+  }
   LMOE_STEP(2, launch_hist(h->topk_idx, T, N, K, h->chunk, h->err, st));
   LMOE_STEP(3, launch_scan(h->chunk, T, N, h->counts, st));
   LMOE_STEP(4, launch_scatter(h->topk_idx, h->topk_w, h->chunk, h->counts, T, N, K, gbn,
@@ -2664,8 +2675,13 @@ int lmoe_route(const float* logits, const float* bias, int64_t T, int32_t N, int
       return LMOE_ERR_CUDA;
     return LMOE_OK;
   }
-  if (launch_route(logits, bias, T, N, K, topk_idx, topk_w, st) != cudaSuccess ||
-      launch_hist(topk_idx, T, N, K, chunk, err, st) != cudaSuccess ||
+  if (launch_route(logits, bias, T, N, K, topk_idx, topk_w, st) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (T <= SEG_SMALL_T)
+    return launch_segments_small(topk_idx, topk_w, T, N, K, 256, counts, offsets, perm, inv, wrow,
+                                 blocks, nblocks, nullptr, err, st) == cudaSuccess
+               ? LMOE_OK
+               : LMOE_ERR_CUDA;
+  if (launch_hist(topk_idx, T, N, K, chunk, err, st) != cudaSuccess ||
       launch_scan(chunk, T, N, counts, st) != cudaSuccess ||
       launch_scatter(topk_idx, topk_w, chunk, counts, T, N, K, 256, offsets, perm, inv, wrow,
                      blocks, nblocks, nullptr, err, st) != cudaSuccess)

@@ -11,6 +11,7 @@
 // routed (token, slot) pairs), built deterministically without atomics on
 // global memory: per 32-token chunk a bitmask per expert gives each token's
 // rank inside the chunk, a column scan over chunks gives the chunk's base.
+#include <atomic>
 #include <cfloat>
 #include <climits>
 #include <cuda_bf16.h>
@@ -149,8 +150,10 @@ cudaError_t launch_scan(int32_t* chunk_cnt, int64_t T, int N, int32_t* counts, c
 // ---------------------------------------------------------------------------
 // offsets, perm / inv / row weights, and the token-block list
 
-// Exclusive prefix of `v` over the 256 threads of the block.
-__device__ __forceinline__ int block_excl_scan_256(int v, int* wsum, int* total) {
+// Exclusive prefix of `v` over the NW x 32 threads of the block (wsum: 2 NW
+// ints of shared memory).
+template <int NW>
+__device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int incl = v;
 #pragma unroll
@@ -161,20 +164,107 @@ __device__ __forceinline__ int block_excl_scan_256(int v, int* wsum, int* total)
   if (lane == 31) wsum[w] = incl;
   __syncthreads();
   if (w == 0) {
-    int s = (lane < 8) ? wsum[lane] : 0;
+    int s = (lane < NW) ? wsum[lane] : 0;
     int si = s;
 #pragma unroll
-    for (int off = 1; off < 8; off <<= 1) {
+    for (int off = 1; off < NW; off <<= 1) {
       const int o = __shfl_up_sync(0xffffffffu, si, off);
       if (lane >= off) si += o;
     }
-    if (lane < 8) wsum[8 + lane] = si - s;
-    if (lane == 7) *total = si;
+    if (lane < NW) wsum[NW + lane] = si - s;
+    if (lane == NW - 1) *total = si;
   }
   __syncthreads();
-  const int r = wsum[8 + w] + incl - v;
+  const int r = wsum[NW + w] + incl - v;
   __syncthreads();
   return r;
+}
+
+// Expert offsets (exclusive scan of the counts, EPT experts per thread of an
+// NW-warp block: N <= 32 NW EPT) and each expert's first token block, into
+// shared memory; with `write`, also the offsets, the list of token blocks of
+// at most bn rows per expert (in expert order) and its length.
+template <int EPT, int NW>
+__device__ __forceinline__ void seg_offsets(const int (&cnt)[EPT], int N, int bn, int32_t* off,
+                                            int32_t* bbase, bool write, int32_t* offsets,
+                                            int4* blocks, int32_t* nblocks, int* wsum,
+                                            int* total) {
+  const int e0 = threadIdx.x * EPT;
+  int sc = 0;
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) sc += cnt[i];
+  int base = block_excl_scan<NW>(sc, wsum, total);
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) {
+    if (e0 + i < N) off[e0 + i] = base;
+    base += cnt[i];
+  }
+  if (threadIdx.x == 0) off[N] = *total;
+  __syncthreads();
+  int nb[EPT];
+  int snb = 0;
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) {
+    nb[i] = (cnt[i] + bn - 1) / bn;
+    snb += nb[i];
+  }
+  int bb = block_excl_scan<NW>(snb, wsum, total);
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) {
+    if (e0 + i < N) bbase[e0 + i] = bb;
+    bb += nb[i];
+  }
+  __syncthreads();
+  if (write) {
+    for (int e = threadIdx.x; e <= N; e += blockDim.x) offsets[e] = off[e];
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+      const int e = e0 + i;
+      for (int j = 0; j < nb[i]; ++j) {
+        const int r0 = j * bn;
+        blocks[bbase[e] + j] = make_int4(e, off[e] + r0, min(bn, cnt[i] - r0), 0);
+      }
+    }
+    if (threadIdx.x == 0) *nblocks = *total;
+  }
+}
+
+// Rows of the routed (token, slot) pairs of chunk c (this lane's token): the
+// chunk's masks `m` give the rank inside the chunk, base_of(e) the rows of
+// expert e in earlier chunks.
+template <class BaseOf>
+__device__ __forceinline__ void seg_rows(const uint32_t* m, const int32_t* __restrict__ idx,
+                                         const float* __restrict__ topk_w, int64_t c, int64_t T,
+                                         int N, int K, int bn, const int32_t* off,
+                                         const int32_t* bbase, BaseOf base_of,
+                                         int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                         float* __restrict__ wrow, int32_t* __restrict__ rblock,
+                                         int lane) {
+  const int64_t t = c * 32 + lane;
+  if (t >= T) return;
+  const uint32_t lower = (1u << lane) - 1u;
+  int ek[32], base[32];
+  float wk[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    ek[k] = (k < K) ? idx[t * K + k] : -1;
+    wk[k] = (k < K) ? topk_w[t * K + k] : 0.0f;
+  }
+#pragma unroll
+  for (int k = 0; k < 32; ++k) base[k] = (ek[k] >= 0 && ek[k] < N) ? base_of(ek[k]) : 0;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const int e = ek[k];
+    if (k < K && e >= 0 && e < N) {
+      const int rank = base[k] + __popc(m[e] & lower);
+      const int row = off[e] + rank;
+      inv[t * K + k] = row;
+      perm[row] = static_cast<int32_t>(t * K + k);
+      wrow[row] = wk[k];
+      // token block of the row and its index inside the block (bn <= 256)
+      if (rblock) rblock[row] = ((bbase[e] + rank / bn) << 8) | (rank % bn);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(256) k_scatter(
@@ -192,51 +282,10 @@ __global__ void __launch_bounds__(256) k_scatter(
   pdl_wait();
   pdl_trigger();
 
-  // offsets: exclusive scan of counts, 4 experts per thread (N <= 1024)
-  const int e4 = threadIdx.x * 4;
   int c4[4];
-  int s4 = 0;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    c4[i] = (e4 + i < N) ? counts[e4 + i] : 0;
-    s4 += c4[i];
-  }
-  int base = block_excl_scan_256(s4, wsum, &total);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (e4 + i < N) off[e4 + i] = base;
-    base += c4[i];
-  }
-  if (threadIdx.x == 0) off[N] = total;
-  __syncthreads();
-
-  // token blocks of at most bn rows per expert, in expert order
-  int nb4[4];
-  int snb = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    nb4[i] = (c4[i] + bn - 1) / bn;
-    snb += nb4[i];
-  }
-  int bb = block_excl_scan_256(snb, wsum, &total);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (e4 + i < N) bbase[e4 + i] = bb;
-    bb += nb4[i];
-  }
-  __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int e = threadIdx.x; e <= N; e += blockDim.x) offsets[e] = off[e];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = e4 + i;
-      for (int j = 0; j < nb4[i]; ++j) {
-        const int r0 = j * bn;
-        blocks[bbase[e] + j] = make_int4(e, off[e] + r0, min(bn, c4[i] - r0), 0);
-      }
-    }
-    if (threadIdx.x == 0) *nblocks = total;
-  }
+  for (int i = 0; i < 4; ++i) c4[i] = (threadIdx.x * 4 + i < N) ? counts[threadIdx.x * 4 + i] : 0;
+  seg_offsets<4, 8>(c4, N, bn, off, bbase, blockIdx.x == 0, offsets, blocks, nblocks, wsum, &total);
 
   // rows of the routed (token, slot) pairs of this warp's chunk
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -245,32 +294,96 @@ __global__ void __launch_bounds__(256) k_scatter(
   if (c >= nchunks) return;
   uint32_t* m = masks + w * N;
   build_chunk_masks(m, idx, c, T, N, K, lane, err);
-  const int64_t t = c * 32 + lane;
-  if (t < T) {
-    const uint32_t lower = (1u << lane) - 1u;
-    int ek[32], base[32];
-    float wk[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      ek[k] = (k < K) ? idx[t * K + k] : -1;
-      wk[k] = (k < K) ? topk_w[t * K + k] : 0.0f;
+  seg_rows(m, idx, topk_w, c, T, N, K, bn, off, bbase,
+           [&](int e) { return chunk_base[c * N + e]; }, perm, inv, wrow, rblock, lane);
+}
+
+// The whole segment build of at most 256 tokens (8 chunks) in one block of
+// 1024 threads, with every global access coalesced: thread i takes the routed
+// pairs p = t K + k = i + 1024 j (idx, topk_w and inv in their own order) and
+// expert e = i; the pairs, the chunks' expert masks and chunk bases, and the
+// row-ordered outputs (perm, rblock) are staged in shared memory and written
+// out row by row at the end.  The same rows as k_hist, k_scan and k_scatter in
+// turn.  One SM does it all, so the work goes to as many warps as it holds
+// (their latencies overlap), and the loops stay rolled: the kernel runs once
+// per forward, after the grouped GEMMs of the last one have streamed
+// gigabytes through L2, so its code comes from HBM every time.  Shared
+// memory: masks and chunk bases [8][N] each, off [N + 1], bbase [N], and four
+// [T K] pair / row arrays.
+__global__ void __launch_bounds__(1024) k_segments_small(
+    const int32_t* __restrict__ idx, const float* __restrict__ topk_w, int64_t T, int N, int K,
+    int bn, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, float* __restrict__ wrow,
+    int4* __restrict__ blocks, int32_t* __restrict__ nblocks, int32_t* __restrict__ rblock,
+    int* err) {
+  extern __shared__ int32_t sc_smem[];
+  const int P = static_cast<int>(T) * K;   // routed pairs (<= 256 x 32)
+  uint32_t* masks = reinterpret_cast<uint32_t*>(sc_smem);   // [8][N]
+  int32_t* cbase = sc_smem + 8 * N;                           // [8][N]
+  int32_t* off = cbase + 8 * N;                               // [N + 1]
+  int32_t* bbase = off + N + 1;                               // [N]
+  int32_t* idx_s = bbase + N;                                 // [P] pairs' experts
+  float* w_s = reinterpret_cast<float*>(idx_s + P);           // [P] pairs' weights
+  int32_t* perm_s = idx_s + 2 * P;                            // [P] row -> pair
+  int32_t* rb_s = idx_s + 3 * P;                              // [P] row -> token block
+  __shared__ int wsum[64];
+  __shared__ int total;
+  pdl_wait();
+  pdl_trigger();
+  const int nchunks = static_cast<int>((T + 31) / 32);
+  // token of pair p: (p + 1/2) / K lies at least 1/(2K) >= 1/64 from an
+  // integer, and for p < 2^13 the two roundings below are off by < 1e-3
+  const float rK = 1.0f / static_cast<float>(K);
+  auto token_of = [rK](int p) { return static_cast<int>((static_cast<float>(p) + 0.5f) * rK); };
+#pragma unroll 4
+  for (int p = threadIdx.x; p < P; p += 1024) {
+    idx_s[p] = idx[p];
+    w_s[p] = topk_w[p];
+  }
+  for (int i = threadIdx.x; i < nchunks * N; i += 1024) masks[i] = 0u;
+  __syncthreads();
+  // each token's bit in its chunk's mask of every expert it selected
+#pragma unroll 1
+  for (int p = threadIdx.x; p < P; p += 1024) {
+    const int e = idx_s[p], t = token_of(p);
+    if (e < 0 || e >= N)
+      atomicOr(err, DEVERR_BAD_INDEX);
+    else
+      atomicOr(&masks[(t >> 5) * N + e], 1u << (t & 31));
+  }
+  __syncthreads();
+  // expert e = threadIdx.x: the rows of earlier chunks (chunk bases), its count
+  const int e = threadIdx.x;
+  int cnt[1] = {0};
+  if (e < N) {
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+      cbase[c * N + e] = cnt[0];
+      cnt[0] += __popc(masks[c * N + e]);
     }
-#pragma unroll
-    for (int k = 0; k < 32; ++k)
-      base[k] = (ek[k] >= 0 && ek[k] < N) ? chunk_base[c * N + ek[k]] : 0;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int e = ek[k];
-      if (k < K && e >= 0 && e < N) {
-        const int rank = base[k] + __popc(m[e] & lower);
-        const int row = off[e] + rank;
-        inv[t * K + k] = row;
-        perm[row] = static_cast<int32_t>(t * K + k);
-        wrow[row] = wk[k];
-        // token block of the row and its index inside the block (bn <= 256)
-        if (rblock) rblock[row] = ((bbase[e] + rank / bn) << 8) | (rank % bn);
-      }
-    }
+    counts[e] = cnt[0];
+  }
+  seg_offsets<1, 32>(cnt, N, bn, off, bbase, true, offsets, blocks, nblocks, wsum, &total);
+  // each pair's row: expert offset + chunk base + rank inside the chunk
+#pragma unroll 1
+  for (int p = threadIdx.x; p < P; p += 1024) {
+    const int ep = idx_s[p], t = token_of(p);
+    if (ep < 0 || ep >= N) continue;
+    const int c = t >> 5;
+    const int rank = cbase[c * N + ep] + __popc(masks[c * N + ep] & ((1u << (t & 31)) - 1u));
+    const int row = off[ep] + rank;
+    inv[p] = row;
+    perm_s[row] = p;
+    rb_s[row] = ((bbase[ep] + rank / bn) << 8) | (rank % bn);
+  }
+  __syncthreads();
+  const int rows = off[N];
+#pragma unroll 1
+  for (int r = threadIdx.x; r < rows; r += 1024) {
+    const int p = perm_s[r];
+    perm[r] = p;
+    wrow[r] = w_s[p];
+    if (rblock) rblock[r] = rb_s[r];
   }
 }
 
@@ -284,6 +397,30 @@ cudaError_t launch_scatter(const int32_t* topk_idx, const float* topk_w, const i
   const size_t smem = (2 * N + 1) * sizeof(int32_t) + 8 * N * sizeof(uint32_t);
   return launch_pdl(k_scatter, nblk, 256, smem, st, topk_idx, topk_w, chunk_base, counts, T, N, K,
                     bn, offsets, perm, inv, wrow, blocks, nblocks, rblock, err);
+}
+
+cudaError_t launch_segments_small(const int32_t* topk_idx, const float* topk_w, int64_t T, int N,
+                                  int K, int bn, int32_t* counts, int32_t* offsets, int32_t* perm,
+                                  int32_t* inv, float* wrow, int4* blocks, int32_t* nblocks,
+                                  int32_t* rblock, int* err, cudaStream_t st) {
+  if (T <= 0 || T > SEG_SMALL_T || N > 1024 || K > 32) return cudaErrorInvalidValue;
+  const size_t smem = (18 * N + 1 + 4 * T * K) * sizeof(int32_t);
+  // the largest shared memory any call asks for (N = 1024, 256 x 32 pairs:
+  // 205 KB), allowed once per device
+  constexpr int kMaxSmem = (18 * 1024 + 1 + 4 * SEG_SMALL_T * 32) * sizeof(int32_t);
+  static std::atomic<uint64_t> allowed{0};   // bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? uint64_t(1) << dev : 0;
+  if (!bit || !(allowed.load() & bit)) {
+    e = cudaFuncSetAttribute(k_segments_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxSmem);
+    if (e != cudaSuccess) return e;
+    allowed.fetch_or(bit);
+  }
+  return launch_pdl(k_segments_small, 1u, 1024, smem, st, topk_idx, topk_w, T, N, K, bn, counts,
+                    offsets, perm, inv, wrow, blocks, nblocks, rblock, err);
 }
 
 // ---------------------------------------------------------------------------

@@ -281,7 +281,7 @@ class LatentMoE:
         check(self.lib.lmoe_profile_enable(self.h, int(on)), "profile_enable")
 
     def profile_read(self, reset: bool = True):
-        n = 32
+        n = 64
         names = (c_char_p * n)()
         ms = (c_double * n)()
         cnt = (c_int64 * n)()

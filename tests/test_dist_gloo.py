@@ -30,8 +30,9 @@ def _worker(rank, world, port, q):
                     lambda: t.__setitem__("b", time.perf_counter()),
                     lambda: (t["b"] - t["a"]) * 1e3)
 
-        # rank 1 is slower: the reported time must be its total
-        delay = 0.002 * (rank + 1)
+        # rank 1 is ten times slower (a margin no scheduler jitter on a busy
+        # host closes): the reported time must be its total
+        delay = 0.002 if rank == 0 else 0.02
         per_step, total = bench.timed_region(lambda: time.sleep(delay), 5, host_timer)
         own = sum(per_step)
         value = bench.throughput(world, 256, 5, total)

@@ -61,6 +61,29 @@ def test_noalloc_route_matches_workspace_route_two_calls_in_a_row():
             c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
 
 
+@pytest.mark.parametrize("T,N,K", [(1, 96, 3), (200, 512, 22), (256, 512, 22), (256, 1024, 32),
+                                   (33, 32, 32)])
+def test_one_block_segments_match_three_kernel_segments(T, N, K):
+    """Up to 256 tokens lmoe_route builds the segments in one block (counts
+    and chunk bases as popcounts of the chunks' masks in shared memory);
+    lmoe_route_noalloc always takes the histogram, scan and scatter kernels.
+    Both give the same top-K and bit-identical counts, offsets, perm and inv."""
+    from latent_space_mixture_b200 import _lib, lmoe_route
+    lib = _lib.load()
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(13 + T)
+    logits = torch.randn((T, N), generator=g, device=dev)
+    bias = torch.randn((N,), generator=g, device=dev) * 0.1
+    ref = lmoe_route(logits, bias, K)
+    torch.cuda.synchronize()
+    rc, got = _noalloc(lib, logits, bias, K)
+    assert rc == 0
+    for k in ("topk_idx", "counts", "offsets", "perm", "inv"):
+        assert torch.equal(got[k], ref[k]), k
+    assert torch.max(torch.abs(got["topk_w"] - ref["topk_w"])).item() <= W_TOL
+
+
 def test_noalloc_route_without_bias_and_with_no_tokens():
     from latent_space_mixture_b200 import _lib, lmoe_route
     lib = _lib.load()
