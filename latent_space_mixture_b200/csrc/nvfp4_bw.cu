@@ -499,8 +499,8 @@ __device__ __forceinline__ void tq_commit(const TqRegs<SRC>& r, const TSrc& s, i
 
 // 64-column groups per CTA: the next group's loads are in flight while this
 // one is transformed and quantised.  The stochastically rounding pass keeps
-// one group per CTA: it is bound by its arithmetic (the random bits), and
-// the registers that hold a group in flight would cost it occupancy.
+// one group per CTA: its random bits need registers, and those that would
+// hold a group in flight would cost it occupancy.
 template <bool SR>
 struct TqGroups {
   static constexpr int value = SR ? 1 : 4;
