@@ -94,6 +94,10 @@ CONFIGS: Dict[str, LayerConfig] = {
                                        "nvfp4"),
     # Super prefill with NVFP4 experts whose weights use the pages' other
     # recipes: 2D 16x16 blocks (training) and MSE-searched scales (PTQ)
+    # the small prefill case with 2D-block NVFP4 experts: the NVFP4 training
+    # backward's kernels at prefill-sized segments, for profiler captures
+    "super_prefill_nvfp4_2d_n64": LayerConfig("super_prefill_nvfp4_2d_n64", 1024, 4096, 1024, 64,
+                                              22, 2688, 5376, 0.02, "zipf", 8, "nvfp4", wq="2d"),
     "super_prefill_nvfp4_2d": LayerConfig("super_prefill_nvfp4_2d", 8192, 4096, 1024, 512, 22,
                                           2688, 5376, 0.02, "zipf", 4, "nvfp4", wq="2d"),
     "super_prefill_nvfp4_mse": LayerConfig("super_prefill_nvfp4_mse", 8192, 4096, 1024, 512, 22,
