@@ -286,10 +286,13 @@ int lmoe_bias_update(lmoe_handle* h, float rate, void* stream);
 int lmoe_get_debug(lmoe_handle* h, int what, void* dst_host, size_t bytes);
 
 /* Kernel launches one lmoe_forward of T tokens issues, or a negative error
- * code: 10, plus the y-GEMM's split-K reduction when T is small.  When the
- * x-GEMM ([W_r; W_dn; W_s1] x) splits K, its reduction also runs the router
- * (sigmoid, bias, top-K, renormalised weights) and replaces the router
- * kernel, so the count stays the same. */
+ * code: 10, plus the y-GEMM's split-K reduction when T is small, minus 2
+ * up to 256 tokens (the per-expert segments from one kernel instead of
+ * histogram, scan and scatter), plus 2 for the opt-in overlapped forward
+ * (the shared expert's GEMMs apart).  When the x-GEMM ([W_r; W_dn; W_s1] x)
+ * splits K, its reduction also runs the router (sigmoid, bias, top-K,
+ * renormalised weights) and replaces the router kernel, so the count stays
+ * the same. */
 int lmoe_launches_per_forward(const lmoe_handle* h, int64_t T);
 
 /* Per-kernel timing: when enabled, every forward records CUDA events around
